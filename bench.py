@@ -1,0 +1,576 @@
+"""Benchmark of the KLA hot path on B200 (one JSON line on stdout, rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl kla|reference]
+    torchrun --nproc-per-node N bench.py --gpus N ...      (N > 1: independent replicas)
+
+Headline (`value`): prefill tokens/s of kla_chunk_fwd on the 0.4B-layer-shaped workload
+(B=8, T=2048, H=8, Dk=Dv=128, bf16 inputs, fp32 state), inputs resident in HBM, L2 flushed
+between timed steps.  One step = one kla_chunk_fwd call over the whole batch.  The same line
+carries the decode workload (B=64, H=16, 1024 sequential kla_decode_step calls), the
+training workload (B=4, T=4096, H=16: kla_chunk_fwd + kla_chunk_bwd) and the long-context
+prefill (B=1, T=65536, H=16) as sub-objects, each with its own roofline.
+
+Multi-GPU: the (batch, head) pairs are independent problems, so every rank runs its own
+replica of the workload (different seed), with no collective on the data path; the timed
+region is bracketed by barriers and the time taken is the max over ranks ("weak" scaling).
+
+`--impl reference` times the fp64 CPU oracle (the slow, obviously correct reference) on a
+bounded sample of the same workload, on the host cores; only rank 0 runs it.
+"""
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "prefill tokens/s & decode tokens/s at 1 B200; % of tensor-core/HBM roofline"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20  # > 2x the 126 MB L2
+
+
+# ---------------------------------------------------------------------------------------
+# algorithmic work (fixed at chunk C = 64, whatever the kernel does internally)
+# ---------------------------------------------------------------------------------------
+def fwd_flops_per_token_head(d, C=64):
+    # 10 C d (KK^T, QK^T, the two UT-transform products, (A o QK^T) U) + 6 d^2 (W S, Q S,
+    # K^T U) + (2/3) C^2 (forward substitution)
+    return 10 * C * d + 6 * d * d + (2.0 / 3.0) * C * C
+
+
+def fwd_bytes(B, T, H, Dk, Dv, elt, s0, s_out=True):
+    per_tok = (2 * Dk + Dv) * elt + Dv * elt + 8  # q, k, v in; o out; eta, g
+    state = B * H * Dk * Dv * 4 * ((1 if s0 else 0) + (1 if s_out else 0))
+    return B * T * H * per_tok + state
+
+
+def decode_bytes(B, H, Dk, Dv, elt):
+    return B * H * (2 * Dk * Dv * 4 + (2 * Dk + 2 * Dv) * elt + 8)
+
+
+def bwd_bytes(B, T, H, Dk, Dv, elt):
+    # reads q, k, v, dO, eta, g; writes dq, dk, dv, deta, dg; plus the dS0 write
+    per_tok = (2 * Dk + Dv) * elt + Dv * elt + 8 + (2 * Dk + Dv) * elt + 8
+    return B * T * H * per_tok + B * H * Dk * Dv * 4
+
+
+# ---------------------------------------------------------------------------------------
+# helpers
+# ---------------------------------------------------------------------------------------
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(PEAKS_FALLBACK), "fallback"
+
+
+def kernel_source_hash():
+    """Hash of the CUDA sources; recorded ncu traffic is only valid for the same sources."""
+    h = hashlib.sha256()
+    cdir = os.path.join(ROOT, "gated_delta_rule_kla_b200", "csrc")
+    for f in sorted(os.listdir(cdir)):
+        with open(os.path.join(cdir, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel_key):
+    """DRAM bytes per launch from the committed ncu summary, or None if stale/absent."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(kernel_key)
+    if not e or e.get("source_hash") != kernel_source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """Samples SM clock, power and throttle reasons through NVML while the GPU is busy."""
+
+    def __init__(self, device_index, period=0.05):
+        self.samples = []
+        self.period = period
+        self._stop = threading.Event()
+        self._thr = None
+        self.max_mhz = None
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+            idx = device_index
+            if vis:
+                ids = [x for x in vis.split(",") if x.strip()]
+                if device_index < len(ids) and ids[device_index].strip().isdigit():
+                    idx = int(ids[device_index])
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(idx)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.ok = False
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                clk = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                util = nv.nvmlDeviceGetUtilizationRates(self.h).gpu
+                reasons = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((clk, util, reasons))
+            except Exception:
+                pass
+            self._stop.wait(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self._thr = threading.Thread(target=self._run, daemon=True)
+            self._thr.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thr:
+            self._thr.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"], "samples": 0}
+        nv = self.nv
+        names = {
+            "gpu_idle": getattr(nv, "nvmlClocksEventReasonGpuIdle", 0x1),
+            "applications_clocks_setting": getattr(nv, "nvmlClocksEventReasonApplicationsClocksSetting", 0x2),
+            "sw_power_cap": getattr(nv, "nvmlClocksEventReasonSwPowerCap", 0x4),
+            "hw_slowdown": getattr(nv, "nvmlClocksEventReasonHwSlowdown", 0x8),
+            "sync_boost": getattr(nv, "nvmlClocksEventReasonSyncBoost", 0x10),
+            "sw_thermal_slowdown": getattr(nv, "nvmlClocksEventReasonSwThermalSlowdown", 0x20),
+            "hw_thermal_slowdown": getattr(nv, "nvmlClocksEventReasonHwThermalSlowdown", 0x40),
+            "hw_power_brake_slowdown": getattr(nv, "nvmlClocksEventReasonHwPowerBrakeSlowdown", 0x80),
+        }
+        loaded = [s for s in self.samples if s[1] > 0] or self.samples
+        reasons = set()
+        for _, _, r in loaded:
+            for n, bit in names.items():
+                if n != "gpu_idle" and r & bit:
+                    reasons.add(n)
+        med = statistics.median([s[0] for s in loaded]) if loaded else None
+        return {"sm_mhz": med, "sm_max_mhz": self.max_mhz, "reasons": sorted(reasons),
+                "samples": len(loaded)}
+
+
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def max_over_ranks(value, world):
+    """Max of a float over all ranks (device-timed numbers are combined this way)."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    dev = torch.device("cuda", torch.cuda.current_device()) if dist.get_backend() == "nccl" else torch.device("cpu")
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(value, world):
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    dev = torch.device("cuda", torch.cuda.current_device()) if dist.get_backend() == "nccl" else torch.device("cpu")
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ---------------------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------------------
+class Flusher:
+    """Evicts L2 between timed steps: writes one buffer larger than L2, then reads another,
+    so the next timed kernel starts with a cold, clean L2 (no dirty lines to write back)."""
+
+    def __init__(self, dev):
+        import torch
+        n = L2_FLUSH_BYTES // 4
+        self.a = torch.empty(n, dtype=torch.float32, device=dev)
+        self.b = torch.ones(n, dtype=torch.float32, device=dev)
+        self.sink = torch.empty(1, dtype=torch.float32, device=dev)
+
+    def __call__(self):
+        import torch
+        self.a.fill_(1.0)
+        torch.sum(self.b, dim=0, keepdim=True, out=self.sink)
+
+
+def time_steps(fn, steps, flush, stream):
+    """Run fn `steps` times, L2 flushed before each; returns per-step device ms (events on
+    the launching stream, recorded around the kernel launches only)."""
+    import torch
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for i in range(steps):
+        flush()
+        evs[i][0].record(stream)
+        fn()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in evs]
+
+
+def gpu_arm(args, rank, world, local_rank):
+    import torch
+    import gated_delta_rule_kla_b200 as kla
+    from gated_delta_rule_kla_b200.workloads import WORKLOADS, make_inputs
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    kla.lib()
+    stream = torch.cuda.current_stream(dev)
+    peaks, peaks_kind = load_peaks()
+    hbm_peak = peaks["hbm_gbs"]
+    tc_peak = peaks["bf16_tflops"]
+    flush = Flusher(dev)
+
+    # ---------------- prefill (headline) ----------------
+    w = WORKLOADS[args.workload]
+    w = w.with_(seed=w.seed + 1000 * rank)
+    inp = make_inputs(w)
+    d = {k: (v.to(dev) if v is not None else None) for k, v in inp.items()}
+    o = torch.empty(w.B, w.T, w.H, w.Dv, device=dev, dtype=d["q"].dtype)
+    ST = torch.empty(w.B, w.H, w.Dk, w.Dv, device=dev, dtype=torch.float32)
+
+    def prefill():
+        kla.chunk_fwd(d["q"], d["k"], d["v"], d["eta"], d["g"], w.eps, d["S0"], o=o, S_T=ST)
+
+    sampler = ClockSampler(local_rank)
+    for _ in range(args.warmup):
+        flush()
+        prefill()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    with sampler:
+        ms = time_steps(prefill, args.steps, flush, stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        torch.cuda.synchronize()
+        total_ms = max_over_ranks(sum(ms), world)
+        tokens = sum_over_ranks(float(w.B * w.T), world) * args.steps
+        elt = d["q"].element_size()
+        alg_bytes = fwd_bytes(w.B, w.T, w.H, w.Dk, w.Dv, elt, d["S0"] is not None)
+        alg_flops = fwd_flops_per_token_head(w.Dk) * w.B * w.T * w.H
+        mean_s = statistics.mean(ms) / 1e3
+        achieved_gbs = alg_bytes / mean_s / 1e9
+        achieved_tf = alg_flops / mean_s / 1e12
+
+        extra = {}
+        if not args.skip_extra:
+            extra["decode"] = bench_decode(kla, WORKLOADS, make_inputs, dev, stream, flush, rank, world,
+                                           hbm_peak, args)
+            extra["train"] = bench_train(kla, WORKLOADS, make_inputs, dev, stream, flush, rank, world,
+                                         hbm_peak, tc_peak, args)
+            extra["long_context"] = bench_long(kla, WORKLOADS, make_inputs, dev, stream, rank, world,
+                                               hbm_peak, tc_peak, args)
+
+    # ---------------- end-to-end through the public API with host buffers ----------------
+    e2e = bench_e2e(kla, w, inp, dev, stream, rank, world, args)
+    clocks = sampler.summary()
+
+    line = {
+        "metric": METRIC,
+        "value": tokens / (total_ms / 1e3),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": total_ms / args.steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16" if w.dtype == "bf16" else "f32",
+        "data": "synthetic (seeded; shapes of the paper's 0.4B model, App. C)",
+        "config": {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "Dk": w.Dk, "Dv": w.Dv,
+                   "chunk": w.chunk, "state": "fp32", "l2": "flushed between timed steps",
+                   "parallelism": f"{world} independent replica(s), no collective"},
+        "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": achieved_gbs / hbm_peak, "peak_kind": peaks_kind,
+                     "traffic": recorded_traffic("chunk_fwd_prefill_b8_t2048_h8_d128"),
+                     "alg_bytes_per_launch": alg_bytes, "kernel_us": mean_s * 1e6,
+                     "tensor": {"achieved": achieved_tf, "peak": tc_peak, "unit": "TFLOP/s",
+                                "frac": achieved_tf / tc_peak, "alg_flops_per_launch": alg_flops}},
+        "e2e": e2e,
+        "gpu_launches": args.steps,
+        "clocks": clocks,
+    }
+    line.update(extra)
+    return line
+
+
+def bench_decode(kla, WORKLOADS, make_inputs, dev, stream, flush, rank, world, hbm_peak, args):
+    import torch
+    w = WORKLOADS["decode_b64_h16_d128_x1024"]
+    w = w.with_(seed=w.seed + 1000 * rank)
+    inp = make_inputs(w)
+    q, k, v = inp["q"].to(dev), inp["k"].to(dev), inp["v"].to(dev)
+    eta, g = inp["eta"].to(dev), inp["g"].to(dev)
+    S = inp["S0"].to(dev).clone()
+    o = torch.empty(w.B, w.H, w.Dv, device=dev, dtype=q.dtype)
+    steps = w.T if not args.quick else 64
+    for t in range(8):
+        kla.decode_step(q[t], k[t], v[t], eta[t], g[t], S, w.eps, o=o)
+    S.copy_(inp["S0"].to(dev))
+    torch.cuda.synchronize()
+    barrier(world)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for t in range(steps):
+        flush()
+        evs[t][0].record(stream)
+        kla.decode_step(q[t], k[t], v[t], eta[t], g[t], S, w.eps, o=o)
+        evs[t][1].record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = [a.elapsed_time(b) for a, b in evs]
+    total_ms = max_over_ranks(sum(ms), world)
+    tokens = sum_over_ranks(float(w.B), world) * steps
+    mean_s = statistics.mean(ms) / 1e3
+    alg = decode_bytes(w.B, w.H, w.Dk, w.Dv, q.element_size())
+    gbs = alg / mean_s / 1e9
+    return {"workload": w.name, "value": tokens / (total_ms / 1e3), "unit": "tokens/s",
+            "steps": steps, "us_per_step": total_ms * 1e3 / steps, "gpu_launches": steps,
+            "l2": "flushed between timed steps",
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s",
+                         "frac": gbs / hbm_peak, "alg_bytes_per_launch": alg,
+                         "traffic": recorded_traffic("decode_b64_h16_d128")}}
+
+
+def bench_train(kla, WORKLOADS, make_inputs, dev, stream, flush, rank, world, hbm_peak, tc_peak, args):
+    import torch
+    w = WORKLOADS["train_b4_t4096_h16_d128"]
+    w = w.with_(seed=w.seed + 1000 * rank)
+    inp = make_inputs(w)
+    d = {k: (v.to(dev) if v is not None else None) for k, v in inp.items()}
+    dO = d["dO"].to(d["q"].dtype)
+    ws = torch.empty(kla.lib().kla_chunk_bwd_workspace(w.B, w.T, w.H, w.Dk, w.Dv, 64, 1, 1),
+                     dtype=torch.uint8, device=dev)
+
+    def step():
+        _, _, Sc = kla.chunk_fwd(d["q"], d["k"], d["v"], d["eta"], d["g"], w.eps, d["S0"],
+                                 save_chunk_states=True)
+        kla.chunk_bwd(d["q"], d["k"], d["v"], d["eta"], d["g"], dO, w.eps, d["S0"], None, Sc, workspace=ws)
+
+    nsteps = 2 if args.quick else 5
+    step()
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = time_steps(step, nsteps, flush, stream)
+    barrier(world)
+    total_ms = max_over_ranks(sum(ms), world)
+    tokens = sum_over_ranks(float(w.B * w.T), world) * nsteps
+    mean_s = statistics.mean(ms) / 1e3
+    flops = 3 * fwd_flops_per_token_head(w.Dk) * w.B * w.T * w.H
+    elt = d["q"].element_size()
+    alg = fwd_bytes(w.B, w.T, w.H, w.Dk, w.Dv, elt, False) + bwd_bytes(w.B, w.T, w.H, w.Dk, w.Dv, elt)
+    return {"workload": w.name, "value": tokens / (total_ms / 1e3), "unit": "tokens/s",
+            "steps": nsteps, "ms_per_step": total_ms / nsteps, "gpu_launches_per_step": 4,
+            "roofline": {"bound": "tensor", "achieved": flops / mean_s / 1e12, "peak": tc_peak,
+                         "unit": "TFLOP/s", "frac": flops / mean_s / 1e12 / tc_peak,
+                         "hbm_frac": alg / mean_s / 1e9 / hbm_peak, "alg_flops_per_step": flops,
+                         "alg_bytes_per_step": alg}}
+
+
+def bench_long(kla, WORKLOADS, make_inputs, dev, stream, rank, world, hbm_peak, tc_peak, args):
+    import torch
+    w = WORKLOADS["prefill_b1_t65536_h16_d128"]
+    w = w.with_(seed=w.seed + 1000 * rank)
+    inp = make_inputs(w)
+    d = {k: (v.to(dev) if v is not None else None) for k, v in inp.items()}
+    o = torch.empty(w.B, w.T, w.H, w.Dv, device=dev, dtype=d["q"].dtype)
+    ST = torch.empty(w.B, w.H, w.Dk, w.Dv, device=dev, dtype=torch.float32)
+
+    def run():
+        kla.chunk_fwd(d["q"], d["k"], d["v"], d["eta"], d["g"], w.eps, d["S0"], o=o, S_T=ST)
+
+    run()
+    torch.cuda.synchronize()
+    barrier(world)
+    nsteps = 2 if args.quick else 3
+    ms = time_steps(run, nsteps, lambda: None, stream)  # inputs (403 MB) exceed L2
+    barrier(world)
+    total_ms = max_over_ranks(sum(ms), world)
+    tokens = sum_over_ranks(float(w.B * w.T), world) * nsteps
+    mean_s = statistics.mean(ms) / 1e3
+    alg = fwd_bytes(w.B, w.T, w.H, w.Dk, w.Dv, d["q"].element_size(), True)
+    flops = fwd_flops_per_token_head(w.Dk) * w.B * w.T * w.H
+    return {"workload": w.name, "value": tokens / (total_ms / 1e3), "unit": "tokens/s",
+            "steps": nsteps, "ms_per_step": total_ms / nsteps, "l2": "inputs larger than L2",
+            "roofline": {"bound": "hbm", "achieved": alg / mean_s / 1e9, "peak": hbm_peak, "unit": "GB/s",
+                         "frac": alg / mean_s / 1e9 / hbm_peak,
+                         "tensor_frac": flops / mean_s / 1e12 / tc_peak}}
+
+
+def bench_e2e(kla, w, inp, dev, stream, rank, world, args):
+    """Same metric through the public API from pinned host buffers: H2D of the step's
+    inputs, kla_chunk_fwd, D2H of the result, all inside the timed region."""
+    import torch
+    names = ["q", "k", "v", "eta", "g"]
+    host = {n: inp[n].pin_memory() for n in names}
+    devb = {n: torch.empty_like(host[n], device=dev) for n in names}
+    o_h = torch.empty(w.B, w.T, w.H, w.Dv, dtype=inp["q"].dtype).pin_memory()
+    ST_h = torch.empty(w.B, w.H, w.Dk, w.Dv, dtype=torch.float32).pin_memory()
+
+    def step():
+        for n in names:
+            devb[n].copy_(host[n], non_blocking=True)
+        o, ST = kla.chunk_fwd(devb["q"], devb["k"], devb["v"], devb["eta"], devb["g"], w.eps, None)
+        o_h.copy_(o, non_blocking=True)
+        ST_h.copy_(ST, non_blocking=True)
+
+    step()
+    torch.cuda.synchronize()
+    barrier(world)
+    nsteps = 3 if args.quick else 10
+    st, en = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    st.record(stream)
+    for _ in range(nsteps):
+        step()
+    en.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(st.elapsed_time(en), world)
+    tokens = sum_over_ranks(float(w.B * w.T), world) * nsteps
+    h2d = sum(host[n].numel() * host[n].element_size() for n in names)
+    d2h = o_h.numel() * o_h.element_size() + ST_h.numel() * 4
+    return {"value": tokens / (ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "steps": nsteps}
+
+
+# ---------------------------------------------------------------------------------------
+# CPU oracle arm and CPU baseline
+# ---------------------------------------------------------------------------------------
+def oracle_sample(workload_name, npairs, seed_offset=0):
+    """Inputs of `npairs` (b, h) pairs of the workload, as fp64 arrays [npairs, T, 1, D]."""
+    import numpy as np
+    from gated_delta_rule_kla_b200.workloads import WORKLOADS, make_inputs
+    w = WORKLOADS[workload_name]
+    w = w.with_(seed=w.seed + seed_offset)
+    inp = make_inputs(w)
+    pairs = [(i % w.B, (i * 5) % w.H) for i in range(npairs)]
+
+    def sel(x, state=False):
+        if x is None:
+            return None
+        x = x.double().numpy()
+        if state:
+            return np.ascontiguousarray(np.stack([x[b, h] for b, h in pairs])[:, None])
+        return np.ascontiguousarray(np.stack([x[b, :, h] for b, h in pairs])[:, :, None])
+
+    return w, [sel(inp[n]) for n in ("q", "k", "v", "eta", "g")], sel(inp["S0"], True)
+
+
+def cpu_baseline(workload_name, npairs):
+    import oracle
+    w, args, S0 = oracle_sample(workload_name, npairs)
+    oracle.forward(*[a[:1, :64] for a in args], w.eps, None if S0 is None else S0[:1])  # load
+    t0 = time.perf_counter()
+    oracle.forward(*args, w.eps, S0)
+    dt = time.perf_counter() - t0
+    tokens = npairs * w.T / w.H  # (b, h) pairs -> whole-token equivalents
+    return {"value": tokens / dt, "unit": "tokens/s", "cores": oracle.threads(), "kind": "oracle",
+            "sample": f"{npairs} of {w.B * w.H} (batch, head) pairs of {w.name}, full T={w.T}, "
+                      f"fp64 token recurrence; {dt:.2f} s"}
+
+
+def reference_arm(args, world):
+    import oracle
+    w, inputs, S0 = oracle_sample(args.workload, args.ref_pairs)
+    oracle.forward(*[a[:1, :64] for a in inputs], w.eps, None)
+    for _ in range(args.warmup if args.warmup <= 1 else 1):
+        oracle.forward(*[a[:1] for a in inputs], w.eps, None)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        oracle.forward(*inputs, w.eps, S0)
+        times.append(time.perf_counter() - t0)
+    tokens = args.ref_pairs * w.T / w.H * args.steps
+    value = tokens / sum(times)
+    sample = (f"{args.ref_pairs} of {w.B * w.H} (batch, head) pairs of {w.name} per step, "
+              f"full T={w.T}, fp64 token recurrence")
+    return {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * sum(times) / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded; shapes of the paper's 0.4B model, App. C)",
+            "config": {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "Dk": w.Dk, "Dv": w.Dv},
+            "impl": "reference",
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+# ---------------------------------------------------------------------------------------
+def parse(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["kla", "reference"], default="kla")
+    ap.add_argument("--workload", default="prefill_b8_t2048_h8_d128")
+    ap.add_argument("--ref-pairs", type=int, default=8, help="(b,h) pairs per reference step")
+    ap.add_argument("--cpu-pairs", type=int, default=16, help="(b,h) pairs in the CPU baseline sample")
+    ap.add_argument("--skip-extra", action="store_true", help="headline prefill only")
+    ap.add_argument("--skip-cpu", action="store_true", help="omit the CPU baseline")
+    ap.add_argument("--quick", action="store_true", help="fewer decode/train steps (smoke runs)")
+    return ap.parse_args(argv)
+
+
+def main(argv=None):
+    args = parse(argv)
+    rank, world, local_rank = dist_env()
+    if args.warmup < 3 and args.impl == "kla":
+        args.warmup = 3  # timing rule: at least 3 warm-up steps
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        print(json.dumps(reference_arm(args, world)), flush=True)
+        return 0
+    import torch
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        line = gpu_arm(args, rank, world, local_rank)
+        if rank == 0:
+            if not args.skip_cpu:
+                line["cpu_baseline"] = cpu_baseline(args.workload, args.cpu_pairs)
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,187 @@
+"""Python binding of libkla.so -- Kaczmarz Linear Attention on NVIDIA B200 (sm_100a).
+
+Thin argument marshalling over the C ABI declared in ``include/kla.h``: every step of the
+computation runs in the library's CUDA kernels.  PyTorch is used only to allocate device
+memory and to name the current CUDA stream.  There is no CPU fallback: if the library is
+missing, or a tensor is not on a CUDA device, the call raises.
+
+    chunk_fwd(q, k, v, eta, g, eps, S0)          -> (o, S_T[, S_chunks])   prefill
+    chunk_bwd(q, k, v, eta, g, dO, eps, S0, ...) -> dict of gradients      training
+    decode_step(q, k, v, eta, g, S, eps)         -> o  (S updated in place)
+
+The method ("Kaczmarz Linear Attention", section 3.1 Eq. (3); section 3.3 Algorithm 1):
+beta_t = eta_t/(||k_t||^2+eps), alpha_t = exp(g_t), Sbar = alpha_t S_{t-1},
+S_t = Sbar + beta_t k_t (v_t - Sbar^T k_t)^T, o_t = S_t^T q_t.
+"""
+import ctypes
+import os
+
+import torch
+
+__all__ = ["lib", "chunk_fwd", "chunk_bwd", "decode_step", "KLAError", "CHUNK", "library_path"]
+
+CHUNK = 64
+KLA_F32, KLA_BF16 = 0, 1
+_PKG = os.path.dirname(os.path.abspath(__file__))
+library_path = os.path.join(_PKG, "libkla.so")
+_lib = None
+
+
+class KLAError(RuntimeError):
+    """A non-OK status returned by libkla."""
+
+    def __init__(self, status, name, detail):
+        super().__init__(f"{name}: {detail}")
+        self.status = status
+
+
+def lib():
+    """The loaded libkla.so (ctypes).  Raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(library_path):
+            raise RuntimeError(f"libkla.so not found at {library_path}; build it with "
+                               "`python -m gated_delta_rule_kla_b200.build`")
+        L = ctypes.CDLL(library_path)
+        vp, fp, i, f, sz = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+        L.kla_status_string.argtypes = [i]
+        L.kla_status_string.restype = ctypes.c_char_p
+        L.kla_last_error.argtypes = []
+        L.kla_last_error.restype = ctypes.c_char_p
+        L.kla_version.argtypes = []
+        L.kla_version.restype = i
+        L.kla_chunk_fwd_workspace.argtypes = [i, i, i, i, i, i, i]
+        L.kla_chunk_fwd_workspace.restype = sz
+        L.kla_chunk_fwd.argtypes = [vp, vp, vp, fp, fp, f, fp, vp, fp, fp, i, i, i, i, i, i, i, vp, sz, vp]
+        L.kla_chunk_fwd.restype = i
+        L.kla_chunk_bwd_workspace.argtypes = [i, i, i, i, i, i, i, i]
+        L.kla_chunk_bwd_workspace.restype = sz
+        L.kla_chunk_bwd.argtypes = [vp, vp, vp, fp, fp, f, fp, vp, fp, fp, vp, vp, vp, fp, fp, fp,
+                                    i, i, i, i, i, i, i, vp, sz, vp]
+        L.kla_chunk_bwd.restype = i
+        L.kla_decode_step.argtypes = [vp, vp, vp, fp, fp, f, fp, vp, i, i, i, i, i, vp]
+        L.kla_decode_step.restype = i
+        _lib = L
+    return _lib
+
+
+def _check(status, name):
+    if status != 0:
+        L = lib()
+        raise KLAError(status, name, f"{L.kla_status_string(status).decode()}: "
+                                     f"{L.kla_last_error().decode()}")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _dtype_code(t):
+    if t.dtype == torch.bfloat16:
+        return KLA_BF16
+    if t.dtype == torch.float32:
+        return KLA_F32
+    raise TypeError(f"q/k/v must be bfloat16 or float32, got {t.dtype}")
+
+
+def _need(t, name, device, dtype=None, shape=None):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor) or t.device.type != "cuda":
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    return t
+
+
+def _stream(device, stream):
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def chunk_fwd(q, k, v, eta, g, eps=1e-6, S0=None, *, o=None, S_T=None, save_chunk_states=False,
+              output_final_state=True, stream=None):
+    """Chunkwise prefill (section 4, Propositions 3-4).
+
+    q, k: [B,T,H,Dk]; v: [B,T,H,Dv] (bf16 or fp32, same dtype); eta, g: [B,T,H] fp32;
+    S0: [B,H,Dk,Dv] fp32 or None.  Returns (o, S_T) or (o, S_T, S_chunks) when
+    save_chunk_states (S_chunks: [B,H,ceil(T/64),Dk,Dv], the state at each chunk start).
+    """
+    dev = k.device
+    B, T, H, Dk = k.shape
+    Dv = v.shape[-1]
+    dt = k.dtype
+    _need(q, "q", dev, dt, (B, T, H, Dk)); _need(k, "k", dev, dt); _need(v, "v", dev, dt, (B, T, H, Dv))
+    _need(eta, "eta", dev, torch.float32, (B, T, H)); _need(g, "g", dev, torch.float32, (B, T, H))
+    _need(S0, "S0", dev, torch.float32, (B, H, Dk, Dv))
+    if o is None:
+        o = torch.empty(B, T, H, Dv, device=dev, dtype=dt)
+    _need(o, "o", dev, dt, (B, T, H, Dv))
+    if S_T is None and output_final_state:
+        S_T = torch.empty(B, H, Dk, Dv, device=dev, dtype=torch.float32)
+    _need(S_T, "S_T", dev, torch.float32, (B, H, Dk, Dv))
+    Sc = None
+    if save_chunk_states:
+        Sc = torch.empty(B, H, (T + CHUNK - 1) // CHUNK, Dk, Dv, device=dev, dtype=torch.float32)
+    st = lib().kla_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(eta), _ptr(g), float(eps), _ptr(S0),
+                             _ptr(o), _ptr(S_T), _ptr(Sc), B, T, H, Dk, Dv, CHUNK, _dtype_code(k),
+                             None, 0, _stream(dev, stream))
+    _check(st, "kla_chunk_fwd")
+    return (o, S_T, Sc) if save_chunk_states else (o, S_T)
+
+
+def chunk_bwd(q, k, v, eta, g, dO, eps=1e-6, S0=None, dS_T=None, S_chunks=None, *, stream=None,
+              workspace=None):
+    """Gradients of the chunkwise forward w.r.t. q, k, v, eta, g and S0.
+
+    dO: [B,T,H,Dv] (same dtype as q); dS_T: [B,H,Dk,Dv] fp32 or None; S_chunks: the
+    array chunk_fwd(save_chunk_states=True) returned for the same inputs, or None.
+    Returns dict(dq, dk, dv, deta, dg, dS0).
+    """
+    dev = k.device
+    B, T, H, Dk = k.shape
+    Dv = v.shape[-1]
+    dt = k.dtype
+    _need(q, "q", dev, dt, (B, T, H, Dk)); _need(k, "k", dev, dt); _need(v, "v", dev, dt, (B, T, H, Dv))
+    _need(eta, "eta", dev, torch.float32, (B, T, H)); _need(g, "g", dev, torch.float32, (B, T, H))
+    _need(S0, "S0", dev, torch.float32, (B, H, Dk, Dv)); _need(dO, "dO", dev, dt, (B, T, H, Dv))
+    _need(dS_T, "dS_T", dev, torch.float32, (B, H, Dk, Dv))
+    NC = (T + CHUNK - 1) // CHUNK
+    _need(S_chunks, "S_chunks", dev, torch.float32, (B, H, NC, Dk, Dv))
+    out = dict(dq=torch.empty_like(q), dk=torch.empty_like(k), dv=torch.empty_like(v),
+               deta=torch.empty_like(eta), dg=torch.empty_like(g),
+               dS0=torch.empty(B, H, Dk, Dv, device=dev, dtype=torch.float32))
+    L = lib()
+    need = L.kla_chunk_bwd_workspace(B, T, H, Dk, Dv, CHUNK, _dtype_code(k), int(S_chunks is not None))
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(max(need, 16), device=dev, dtype=torch.uint8)
+    st = L.kla_chunk_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(eta), _ptr(g), float(eps), _ptr(S0), _ptr(dO),
+                         _ptr(dS_T), _ptr(S_chunks), _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]),
+                         _ptr(out["deta"]), _ptr(out["dg"]), _ptr(out["dS0"]), B, T, H, Dk, Dv, CHUNK,
+                         _dtype_code(k), _ptr(workspace), workspace.numel(), _stream(dev, stream))
+    _check(st, "kla_chunk_bwd")
+    return out
+
+
+def decode_step(q, k, v, eta, g, S, eps=1e-6, *, o=None, stream=None):
+    """One decode token for every (b, h): q, k [B,H,Dk]; v [B,H,Dv]; eta, g [B,H] fp32;
+    S [B,H,Dk,Dv] fp32 updated in place.  Returns o [B,H,Dv]."""
+    dev = S.device
+    B, H, Dk, Dv = S.shape
+    dt = k.dtype
+    _need(q, "q", dev, dt, (B, H, Dk)); _need(k, "k", dev, dt, (B, H, Dk)); _need(v, "v", dev, dt, (B, H, Dv))
+    _need(eta, "eta", dev, torch.float32, (B, H)); _need(g, "g", dev, torch.float32, (B, H))
+    _need(S, "S", dev, torch.float32, (B, H, Dk, Dv))
+    if o is None:
+        o = torch.empty(B, H, Dv, device=dev, dtype=dt)
+    _need(o, "o", dev, dt, (B, H, Dv))
+    st = lib().kla_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(eta), _ptr(g), float(eps), _ptr(S), _ptr(o),
+                               B, H, Dk, Dv, _dtype_code(k), _stream(dev, stream))
+    _check(st, "kla_decode_step")
+    return o

@@ -1,0 +1,201 @@
+// kla_abi.cu -- the extern "C" boundary of libkla.so (declared in include/kla.h).
+// Host-side validation, workspace layout and kernel dispatch; no device arithmetic here.
+#include <stdarg.h>
+#include <stdint.h>
+#include <stdio.h>
+
+#include <string>
+
+#include "kla.h"
+#include "kla_launch.h"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+kla_status fail(kla_status st, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+kla_status fail(kla_status st, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return st;
+}
+
+kla_status cuda_fail(cudaError_t e, const char* where) {
+    return fail(KLA_ERR_CUDA, "%s: %s (%s)", where, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return p == nullptr || (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+kla_status check_common(int B, int T, int H, int Dk, int Dv, int chunk, int dtype, float eps) {
+    if (B < 1 || H < 1 || T < 0)
+        return fail(KLA_ERR_INVALID_ARG, "sizes must satisfy B>=1, H>=1, T>=0 (got B=%d T=%d H=%d)",
+                    B, T, H);
+    if (!(eps >= 0.f)) return fail(KLA_ERR_INVALID_ARG, "eps must be >= 0 (got %g)", (double)eps);
+    if ((Dk != 64 && Dk != 128) || (Dv != 64 && Dv != 128))
+        return fail(KLA_ERR_UNSUPPORTED, "Dk, Dv must be 64 or 128 (got Dk=%d Dv=%d)", Dk, Dv);
+    if (chunk != kla::kChunkLen)
+        return fail(KLA_ERR_UNSUPPORTED, "chunk must be %d (got %d)", kla::kChunkLen, chunk);
+    if (dtype != KLA_F32 && dtype != KLA_BF16)
+        return fail(KLA_ERR_UNSUPPORTED, "dtype must be KLA_F32 or KLA_BF16 (got %d)", dtype);
+    // 32-bit index headroom for per-token offsets inside kernels is not assumed: kernels
+    // index with size_t; but B*H and grid sizes must fit the launch limits.
+    if ((long long)B * H > (1LL << 30)) return fail(KLA_ERR_UNSUPPORTED, "B*H too large");
+    return KLA_OK;
+}
+
+#define REQUIRE_PTR(p)                                                                    \
+    do {                                                                                  \
+        if ((p) == nullptr) return fail(KLA_ERR_INVALID_ARG, "%s must not be NULL", #p); \
+        if (!aligned16(p)) return fail(KLA_ERR_INVALID_ARG, "%s must be 16-byte aligned", #p); \
+    } while (0)
+#define OPTIONAL_PTR(p)                                                                        \
+    do {                                                                                       \
+        if (!aligned16(p)) return fail(KLA_ERR_INVALID_ARG, "%s must be 16-byte aligned", #p); \
+    } while (0)
+
+size_t bwd_ws_layout(int B, int T, int H, int Dk, int Dv, bool have_S_chunks, size_t* off) {
+    const size_t NC = (size_t)(T + kla::kChunkLen - 1) / kla::kChunkLen;
+    const size_t ntok = (size_t)B * T * H;
+    size_t o = 0;
+    off[0] = o;  // S_chunks
+    if (!have_S_chunks) o += align256((size_t)B * H * NC * Dk * Dv * sizeof(float));
+    off[1] = o;  // acc_dq
+    o += align256(ntok * Dk * sizeof(float));
+    off[2] = o;  // acc_dkh
+    o += align256(ntok * Dk * sizeof(float));
+    off[3] = o;  // acc_db, acc_dc, acc_dG (contiguous, zeroed together with the above)
+    o += align256(3 * ntok * sizeof(float));
+    off[4] = o;
+    return o;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* kla_status_string(int status) {
+    switch (status) {
+        case KLA_OK: return "KLA_OK";
+        case KLA_ERR_INVALID_ARG: return "KLA_ERR_INVALID_ARG";
+        case KLA_ERR_UNSUPPORTED: return "KLA_ERR_UNSUPPORTED";
+        case KLA_ERR_WORKSPACE: return "KLA_ERR_WORKSPACE";
+        case KLA_ERR_CUDA: return "KLA_ERR_CUDA";
+        case KLA_ERR_TIMEOUT: return "KLA_ERR_TIMEOUT";
+        default: return "KLA_ERR_UNKNOWN";
+    }
+}
+
+const char* kla_last_error(void) { return g_last_error.c_str(); }
+
+int kla_version(void) { return 100; }
+
+size_t kla_chunk_fwd_workspace(int B, int T, int H, int Dk, int Dv, int chunk, int dtype) {
+    (void)B; (void)T; (void)H; (void)Dk; (void)Dv; (void)chunk; (void)dtype;
+    return 0;
+}
+
+kla_status kla_chunk_fwd(const void* q, const void* k, const void* v, const float* eta,
+                         const float* g, float eps, const float* S0, void* o, float* S_T,
+                         float* S_chunks, int B, int T, int H, int Dk, int Dv, int chunk,
+                         int dtype, void* ws, size_t ws_bytes, void* stream) {
+    (void)ws; (void)ws_bytes;
+    kla_status st = check_common(B, T, H, Dk, Dv, chunk, dtype, eps);
+    if (st != KLA_OK) return st;
+    if (T > 0) {
+        REQUIRE_PTR(q); REQUIRE_PTR(k); REQUIRE_PTR(v); REQUIRE_PTR(eta); REQUIRE_PTR(g);
+    }
+    OPTIONAL_PTR(S0); OPTIONAL_PTR(o); OPTIONAL_PTR(S_T); OPTIONAL_PTR(S_chunks);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (T == 0) {
+        if (S_T != nullptr && S_T != S0) {
+            const size_t bytes = (size_t)B * H * Dk * Dv * sizeof(float);
+            cudaError_t e = S0 ? cudaMemcpyAsync(S_T, S0, bytes, cudaMemcpyDeviceToDevice, s)
+                               : cudaMemsetAsync(S_T, 0, bytes, s);
+            if (e != cudaSuccess) return cuda_fail(e, "kla_chunk_fwd(T=0)");
+        }
+        return KLA_OK;
+    }
+    kla::FwdArgs a{q, k, v, eta, g, eps, S0, o, S_T, S_chunks, B, T, H, Dk, Dv, dtype == KLA_BF16};
+    cudaError_t e = kla::chunk_fwd_tc_supported(a) ? kla::launch_chunk_fwd_tc(a, s)
+                                                   : kla::launch_chunk_fwd_simt(a, s);
+    if (e != cudaSuccess) return cuda_fail(e, "kla_chunk_fwd launch");
+    return KLA_OK;
+}
+
+size_t kla_chunk_bwd_workspace(int B, int T, int H, int Dk, int Dv, int chunk, int dtype,
+                               int have_S_chunks) {
+    (void)chunk; (void)dtype;
+    if (B < 1 || H < 1 || T < 0) return 0;
+    size_t off[5];
+    return bwd_ws_layout(B, T, H, Dk, Dv, have_S_chunks != 0, off);
+}
+
+kla_status kla_chunk_bwd(const void* q, const void* k, const void* v, const float* eta,
+                         const float* g, float eps, const float* S0, const void* dO,
+                         const float* dS_T, const float* S_chunks, void* dq, void* dk, void* dv,
+                         float* deta, float* dg, float* dS0, int B, int T, int H, int Dk, int Dv,
+                         int chunk, int dtype, void* ws, size_t ws_bytes, void* stream) {
+    kla_status st = check_common(B, T, H, Dk, Dv, chunk, dtype, eps);
+    if (st != KLA_OK) return st;
+    REQUIRE_PTR(dS0);
+    OPTIONAL_PTR(S0); OPTIONAL_PTR(dS_T); OPTIONAL_PTR(S_chunks);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t sbytes = (size_t)B * H * Dk * Dv * sizeof(float);
+    if (T == 0) {
+        cudaError_t e = dS_T ? cudaMemcpyAsync(dS0, dS_T, sbytes, cudaMemcpyDeviceToDevice, s)
+                             : cudaMemsetAsync(dS0, 0, sbytes, s);
+        if (e != cudaSuccess) return cuda_fail(e, "kla_chunk_bwd(T=0)");
+        return KLA_OK;
+    }
+    REQUIRE_PTR(q); REQUIRE_PTR(k); REQUIRE_PTR(v); REQUIRE_PTR(eta); REQUIRE_PTR(g);
+    REQUIRE_PTR(dO); REQUIRE_PTR(dq); REQUIRE_PTR(dk); REQUIRE_PTR(dv); REQUIRE_PTR(deta);
+    REQUIRE_PTR(dg);
+    size_t off[5];
+    const size_t need = bwd_ws_layout(B, T, H, Dk, Dv, S_chunks != nullptr, off);
+    if (ws == nullptr || ws_bytes < need)
+        return fail(KLA_ERR_WORKSPACE, "kla_chunk_bwd needs %zu workspace bytes (got %zu)", need,
+                    ws == nullptr ? (size_t)0 : ws_bytes);
+    if (!aligned16(ws)) return fail(KLA_ERR_INVALID_ARG, "ws must be 16-byte aligned");
+    char* w = static_cast<char*>(ws);
+    cudaError_t e = cudaMemsetAsync(w + off[1], 0, off[4] - off[1], s);
+    if (e != cudaSuccess) return cuda_fail(e, "kla_chunk_bwd workspace clear");
+    const float* Sc = S_chunks;
+    if (Sc == nullptr) {
+        float* Sc_ws = reinterpret_cast<float*>(w + off[0]);
+        kla::FwdArgs fa{q, k, v, eta, g, eps, S0, nullptr, nullptr, Sc_ws, B, T, H, Dk, Dv,
+                        dtype == KLA_BF16};
+        e = kla::launch_chunk_fwd_simt(fa, s);
+        if (e != cudaSuccess) return cuda_fail(e, "kla_chunk_bwd state recompute");
+        Sc = Sc_ws;
+    }
+    const size_t ntok = (size_t)B * T * H;
+    float* acc3 = reinterpret_cast<float*>(w + off[3]);
+    kla::BwdArgs a{q, k, v, eta, g, eps, Sc, dO, dS_T, dq, dk, dv, deta, dg, dS0,
+                   reinterpret_cast<float*>(w + off[1]), reinterpret_cast<float*>(w + off[2]),
+                   acc3, acc3 + ntok, acc3 + 2 * ntok, B, T, H, Dk, Dv, dtype == KLA_BF16};
+    e = kla::launch_chunk_bwd_simt(a, s);
+    if (e != cudaSuccess) return cuda_fail(e, "kla_chunk_bwd launch");
+    return KLA_OK;
+}
+
+kla_status kla_decode_step(const void* q, const void* k, const void* v, const float* eta,
+                           const float* g, float eps, float* S, void* o, int B, int H, int Dk,
+                           int Dv, int dtype, void* stream) {
+    kla_status st = check_common(B, 0, H, Dk, Dv, kla::kChunkLen, dtype, eps);
+    if (st != KLA_OK) return st;
+    REQUIRE_PTR(q); REQUIRE_PTR(k); REQUIRE_PTR(v); REQUIRE_PTR(eta); REQUIRE_PTR(g);
+    REQUIRE_PTR(S);
+    OPTIONAL_PTR(o);
+    kla::DecodeArgs a{q, k, v, eta, g, eps, S, o, B, H, Dk, Dv, dtype == KLA_BF16};
+    cudaError_t e = kla::launch_decode(a, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "kla_decode_step launch");
+    return KLA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,55 @@
+// kla_launch.h -- internal launch interface between the C ABI layer and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+namespace kla {
+
+constexpr int kChunkLen = 64;  // the only chunk length the library accepts
+
+struct DecodeArgs {
+    const void *q, *k, *v;
+    const float *eta, *g;
+    float eps;
+    float* S;
+    void* o;
+    int B, H, Dk, Dv;
+    bool bf16;
+};
+
+struct FwdArgs {
+    const void *q, *k, *v;
+    const float *eta, *g;
+    float eps;
+    const float* S0;  // may be null (zero state)
+    void* o;          // may be null
+    float* S_T;       // may be null; may alias S0
+    float* S_chunks;  // may be null
+    int B, T, H, Dk, Dv;
+    bool bf16;
+};
+
+struct BwdArgs {
+    const void *q, *k, *v;
+    const float *eta, *g;
+    float eps;
+    const float* S_chunks;  // [B,H,NC,Dk,Dv], required here
+    const void* dO;
+    const float* dS_T;  // may be null
+    void *dq, *dk, *dv;
+    float *deta, *dg, *dS0;
+    // fp32 accumulators (zeroed by the launcher): [B,T,H,Dk] x2, [B,T,H] x3
+    float *acc_dq, *acc_dkh, *acc_db, *acc_dc, *acc_dG;
+    int B, T, H, Dk, Dv;
+    bool bf16;
+};
+
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st);
+cudaError_t launch_chunk_fwd_simt(const FwdArgs& a, cudaStream_t st);
+cudaError_t launch_chunk_bwd_simt(const BwdArgs& a, cudaStream_t st);
+// Tensor-core (tcgen05) forward for bf16 inputs with Dk == Dv == 128.
+bool chunk_fwd_tc_supported(const FwdArgs& a);
+cudaError_t launch_chunk_fwd_tc(const FwdArgs& a, cudaStream_t st);
+
+}  // namespace kla

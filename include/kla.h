@@ -1,0 +1,131 @@
+/*
+ * kla.h -- C ABI of libkla.so: Kaczmarz Linear Attention (KLA) on NVIDIA B200 (sm_100a).
+ *
+ * KLA ("Kaczmarz Linear Attention", arXiv 2605.08587) is a gated delta rule whose write
+ * is normalised by the key energy.  Per head, with state S in R^{Dk x Dv}:
+ *
+ *     beta_t = eta_t / (||k_t||^2 + eps)          section 3.1, Eq. (3)
+ *     alpha_t = exp(g_t)                           (g is the log-decay)
+ *     Sbar = alpha_t S_{t-1};  e_t = v_t - Sbar^T k_t
+ *     S_t  = Sbar + beta_t k_t e_t^T               Algorithm 1 (left panel), lines 2-5
+ *     o_t  = S_t^T q_t                             section 2 readout
+ *
+ * The readout uses q exactly as passed.  Algorithm 1, line 6 divides by ||q_t||; because o
+ * is linear in q, a caller who wants that form passes q_t / ||q_t||.  No 1/sqrt(Dk) scale
+ * and no key normalisation is applied (normalising k would turn KLA into GDN).
+ * When ||k_t||^2 + eps == 0 the write is skipped (beta_t = 0); the paper is silent there.
+ *
+ * Conventions shared by every entry point
+ *   - All pointers are DEVICE pointers owned by the caller; the library allocates nothing
+ *     and keeps no pointer after the call returns.  Buffers must be contiguous in the
+ *     layouts given below and 16-byte aligned.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t passed as void*; NULL = legacy
+ *     default stream) and never synchronise the host.
+ *   - Arguments are validated on the host before any launch; an invalid call returns an
+ *     error status and launches nothing.  A failed launch returns KLA_ERR_CUDA.
+ *     kla_last_error() gives a one-line description of the last failure on this thread.
+ *   - Supported shapes: Dk, Dv in {64, 128}; chunk == 64; B, H >= 1; T >= 0 (T == 0 copies
+ *     S0 to S_T).  The last chunk may be partial.  eps >= 0.  g <= 0 is the intended range
+ *     (the decay factors exp(G_i - G_j) are then <= 1); g > 0 is accepted without an
+ *     accuracy guarantee.
+ *   - dtype selects the element type of q, k, v, o, dO, dq, dk, dv: KLA_F32 or KLA_BF16.
+ *     eta, g, S0, S_T, S, dS_T and every other gradient are fp32.  The state is always fp32.
+ *   - NaN or Inf inputs propagate; they are not checked.
+ *
+ * Layouts (row-major):
+ *   q, k, dq, dk : [B, T, H, Dk]          v, o, dO, dv : [B, T, H, Dv]
+ *   eta, g, deta, dg : [B, T, H]          S0, S_T, dS_T, dS0 : [B, H, Dk, Dv]
+ *   decode: q, k : [B, H, Dk]; v, o : [B, H, Dv]; eta, g : [B, H]; S : [B, H, Dk, Dv]
+ */
+#ifndef KLA_H_
+#define KLA_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    KLA_OK = 0,
+    KLA_ERR_INVALID_ARG = 1, /* null pointer where one is required, negative size, bad eps */
+    KLA_ERR_UNSUPPORTED = 2, /* shape or dtype outside the supported set */
+    KLA_ERR_WORKSPACE = 3,   /* workspace missing or smaller than the *_workspace() size */
+    KLA_ERR_CUDA = 4,        /* a CUDA launch or runtime call failed */
+    KLA_ERR_TIMEOUT = 5      /* reserved: a bounded device-side wait expired */
+} kla_status;
+
+typedef enum { KLA_F32 = 0, KLA_BF16 = 1 } kla_dtype;
+
+/* Static string naming a status code (never NULL). */
+const char *kla_status_string(int status);
+
+/* One-line description of the last non-OK status returned on the calling thread. */
+const char *kla_last_error(void);
+
+/* Library version as major*10000 + minor*100 + patch. */
+int kla_version(void);
+
+/*
+ * kla_chunk_fwd -- chunkwise-parallel prefill.
+ * "Kaczmarz Linear Attention", section 4, Propositions 3 and 4 (Eqs. 7-9), Algorithm 1
+ * (right panel); the result equals the tokenwise recurrence above for every token.
+ *
+ *   q, k, v      in   [B,T,H,Dk|Dv] of `dtype`
+ *   eta, g       in   [B,T,H] fp32: write gate (0..1 intended) and log-decay
+ *   eps          in   stabiliser of Eq. (3), >= 0
+ *   S0           in   [B,H,Dk,Dv] fp32 initial state, or NULL for a zero state
+ *   o            out  [B,T,H,Dv] of `dtype`, or NULL to skip the readout
+ *   S_T          out  [B,H,Dk,Dv] fp32 final state, or NULL.  May alias S0.
+ *   S_chunks     out  [B,H,ceil(T/chunk),Dk,Dv] fp32 state at the start of every chunk, or
+ *                     NULL.  Passing it to kla_chunk_bwd saves the backward's recompute.
+ *   ws, ws_bytes      caller workspace of at least kla_chunk_fwd_workspace() bytes (the
+ *                     forward currently needs none; ws may then be NULL).
+ * Returns KLA_OK or an error status; on error nothing is launched.
+ */
+size_t kla_chunk_fwd_workspace(int B, int T, int H, int Dk, int Dv, int chunk, int dtype);
+kla_status kla_chunk_fwd(const void *q, const void *k, const void *v, const float *eta,
+                         const float *g, float eps, const float *S0, void *o, float *S_T,
+                         float *S_chunks, int B, int T, int H, int Dk, int Dv, int chunk,
+                         int dtype, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * kla_chunk_bwd -- gradients of the chunkwise forward.
+ * The paper gives no backward; this one differentiates the forward above exactly (same
+ * result as reverse-mode differentiation of the tokenwise recurrence).  Given the upstream
+ * gradients dO (of o) and dS_T (of S_T, NULL = zero), it returns the gradients of every
+ * input: dq, dk, dv (of `dtype`), deta, dg ([B,T,H] fp32) and dS0 ([B,H,Dk,Dv] fp32;
+ * written even when S0 is NULL).  S_chunks may be the array kla_chunk_fwd wrote for the
+ * same inputs, or NULL to recompute it inside the workspace.
+ * Gradient of k at a key of exactly zero norm: the normalised-key form used on the GPU has
+ * no finite limit there; dk is returned as zero for such tokens (all other gradients exact).
+ * ws, ws_bytes: caller workspace of at least kla_chunk_bwd_workspace() bytes (required).
+ * Every output is fully overwritten.
+ */
+size_t kla_chunk_bwd_workspace(int B, int T, int H, int Dk, int Dv, int chunk, int dtype,
+                               int have_S_chunks);
+kla_status kla_chunk_bwd(const void *q, const void *k, const void *v, const float *eta,
+                         const float *g, float eps, const float *S0, const void *dO,
+                         const float *dS_T, const float *S_chunks, void *dq, void *dk, void *dv,
+                         float *deta, float *dg, float *dS0, int B, int T, int H, int Dk,
+                         int Dv, int chunk, int dtype, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * kla_decode_step -- one generated token: Algorithm 1 (left panel), lines 2-6 (readout
+ * without the 1/||q|| factor, as above), for every (b, h) at once.
+ *
+ *   q, k    in     [B,H,Dk] of `dtype`      v   in  [B,H,Dv] of `dtype`
+ *   eta, g  in     [B,H] fp32               eps in  >= 0
+ *   S       in/out [B,H,Dk,Dv] fp32, updated in place to S_t
+ *   o       out    [B,H,Dv] of `dtype` (o_t = S_t^T q_t), or NULL
+ * Each state element is read once and written once.
+ */
+kla_status kla_decode_step(const void *q, const void *k, const void *v, const float *eta,
+                           const float *g, float eps, float *S, void *o, int B, int H, int Dk,
+                           int Dv, int dtype, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KLA_H_ */

@@ -1,0 +1,116 @@
+"""Host-only checks of the C ABI (no GPU): the library loads, exports every entry point
+include/kla.h declares, and rejects invalid calls before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "kla.h")
+
+OK, INVALID, UNSUPPORTED, WORKSPACE = 0, 1, 2, 3
+FAKE = ctypes.c_void_p(0x10000)  # aligned, never dereferenced: validation fails first
+MISALIGNED = ctypes.c_void_p(0x10004)
+
+
+@pytest.fixture(scope="module")
+def L():
+    from gated_delta_rule_kla_b200 import build
+    build.build()
+    import gated_delta_rule_kla_b200 as kla
+    return kla.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(kla_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = declared_functions()
+    assert {"kla_chunk_fwd", "kla_chunk_bwd", "kla_decode_step"} <= set(names)
+    for n in names:
+        assert hasattr(L, n), f"libkla.so does not export {n}"
+
+
+def test_status_strings(L):
+    for code, name in [(0, b"KLA_OK"), (1, b"KLA_ERR_INVALID_ARG"), (2, b"KLA_ERR_UNSUPPORTED"),
+                       (3, b"KLA_ERR_WORKSPACE"), (4, b"KLA_ERR_CUDA"), (5, b"KLA_ERR_TIMEOUT")]:
+        assert L.kla_status_string(code) == name
+    assert L.kla_status_string(99) == b"KLA_ERR_UNKNOWN"
+    assert L.kla_version() >= 100
+
+
+def _fwd(L, B=1, T=64, H=1, Dk=128, Dv=128, chunk=64, dtype=1, eps=1e-6, q=FAKE, ws=None):
+    return L.kla_chunk_fwd(q, FAKE, FAKE, FAKE, FAKE, eps, None, FAKE, FAKE, None, B, T, H, Dk, Dv,
+                           chunk, dtype, ws, 0, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(Dk=96), UNSUPPORTED), (dict(Dv=32), UNSUPPORTED), (dict(chunk=32), UNSUPPORTED),
+    (dict(dtype=7), UNSUPPORTED), (dict(eps=-1.0), INVALID), (dict(eps=float("nan")), INVALID),
+    (dict(B=0), INVALID), (dict(H=0), INVALID), (dict(T=-1), INVALID),
+    (dict(q=None), INVALID), (dict(q=MISALIGNED), INVALID),
+])
+def test_fwd_rejects_before_launch(L, kw, code):
+    assert _fwd(L, **kw) == code
+    assert len(L.kla_last_error()) > 0
+
+
+def test_bwd_workspace_checked(L):
+    need = L.kla_chunk_bwd_workspace(2, 100, 3, 64, 128, 64, 1, 0)
+    ntok = 2 * 100 * 3
+    r256 = lambda x: (x + 255) // 256 * 256
+    assert need == r256(2 * 3 * 2 * 64 * 128 * 4) + 2 * r256(ntok * 64 * 4) + r256(3 * ntok * 4)
+    assert L.kla_chunk_bwd_workspace(2, 100, 3, 64, 128, 64, 1, 1) == need - r256(2 * 3 * 2 * 64 * 128 * 4)
+    st = L.kla_chunk_bwd(FAKE, FAKE, FAKE, FAKE, FAKE, 1e-6, None, FAKE, None, None, FAKE, FAKE, FAKE,
+                         FAKE, FAKE, FAKE, 2, 100, 3, 64, 128, 64, 1, None, 0, None)
+    assert st == WORKSPACE
+    assert b"workspace" in L.kla_last_error()
+    st = L.kla_chunk_bwd(FAKE, FAKE, FAKE, FAKE, FAKE, 1e-6, None, FAKE, None, None, FAKE, FAKE, FAKE,
+                         FAKE, FAKE, FAKE, 2, 100, 3, 64, 128, 64, 1, FAKE, need - 1, None)
+    assert st == WORKSPACE
+
+
+def test_bwd_requires_outputs(L):
+    st = L.kla_chunk_bwd(FAKE, FAKE, FAKE, FAKE, FAKE, 1e-6, None, FAKE, None, None, None, FAKE, FAKE,
+                         FAKE, FAKE, FAKE, 1, 64, 1, 64, 64, 64, 1, FAKE, 1 << 30, None)
+    assert st == INVALID
+
+
+def test_decode_rejects_before_launch(L):
+    st = L.kla_decode_step(FAKE, FAKE, FAKE, FAKE, FAKE, 1e-6, FAKE, None, 4, 2, 128, 96, 1, None)
+    assert st == UNSUPPORTED
+    st = L.kla_decode_step(FAKE, FAKE, FAKE, FAKE, FAKE, 1e-6, None, None, 4, 2, 128, 128, 1, None)
+    assert st == INVALID
+    st = L.kla_decode_step(FAKE, FAKE, FAKE, FAKE, FAKE, -0.5, FAKE, None, 4, 2, 128, 128, 1, None)
+    assert st == INVALID
+
+
+def test_binding_has_no_cpu_fallback(L):
+    import gated_delta_rule_kla_b200 as kla
+    x = torch.zeros(1, 64, 1, 64)
+    gates = torch.zeros(1, 64, 1)
+    with pytest.raises(TypeError):
+        kla.chunk_fwd(x, x, x, gates, gates)
+    with pytest.raises(TypeError):
+        kla.decode_step(x[:, 0], x[:, 0], x[:, 0], gates[:, 0], gates[:, 0], torch.zeros(1, 1, 64, 64))
+
+
+def test_product_and_oracle_share_no_code():
+    pkg = os.path.join(ROOT, "gated_delta_rule_kla_b200")
+    imp = re.compile(r"^\s*(from\s+oracle\b|import\s+oracle\b|#\s*include\s*[<\"].*oracle)", re.M)
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                text = open(os.path.join(dirpath, f)).read()
+                assert not imp.search(text), f"{f} imports the oracle"
+                assert "kla_oracle" not in text, f"{f} names the oracle library"
+    for f in os.listdir(os.path.join(ROOT, "oracle")):
+        if f.endswith((".py", ".c", ".h")):
+            text = open(os.path.join(ROOT, "oracle", f)).read()
+            assert "gated_delta_rule_kla_b200" not in text
+            assert "kla.h" not in text

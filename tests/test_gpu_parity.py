@@ -1,0 +1,303 @@
+"""GPU parity: the CUDA path (through the C ABI, via the thin binding) against the fp64
+oracle on identical seeded inputs.
+
+Metric per output tensor: max|gpu - oracle| / rms(oracle).  Bars: 1e-4 for fp32 inputs,
+2e-2 for bf16 inputs (state always fp32).  The oracle sees the exact dtype-rounded values
+the GPU sees, upcast to fp64.  At full workload sizes the oracle runs on a sample of the
+independent (batch, head) pairs; every output of those pairs is compared.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from gated_delta_rule_kla_b200.workloads import WORKLOADS, Workload, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+TOL = {"f32": 1e-4, "bf16": 2e-2}
+
+
+@pytest.fixture(scope="module")
+def kla():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import gated_delta_rule_kla_b200 as kla
+    kla.lib()
+    return kla
+
+
+def rel_err(got, ref):
+    got = got.detach().double().cpu().numpy() if isinstance(got, torch.Tensor) else np.asarray(got)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert got.shape == ref.shape, (got.shape, ref.shape)
+    assert np.all(np.isfinite(got)), "non-finite GPU output"
+    rms = math.sqrt(float(np.mean(ref * ref))) if ref.size else 0.0
+    if rms == 0.0:
+        return float(np.abs(got - ref).max()) if ref.size else 0.0
+    return float(np.abs(got - ref).max()) / rms
+
+
+def np64(t):
+    return None if t is None else t.detach().double().cpu().numpy()
+
+
+def heads_slice(x, pairs, state=False):
+    """Select (b, h) pairs of a [B,T,H,...] (or state [B,H,...]) array into [n,T,1,...]."""
+    if x is None:
+        return None
+    if state:
+        return np.ascontiguousarray(np.stack([x[b, h] for b, h in pairs])[:, None])
+    return np.ascontiguousarray(np.stack([x[b, :, h] for b, h in pairs])[:, :, None])
+
+
+def run_fwd(kla, inp, eps, dev="cuda"):
+    d = {k: (v.to(dev) if v is not None else None) for k, v in inp.items()}
+    o, ST = kla.chunk_fwd(d["q"], d["k"], d["v"], d["eta"], d["g"], eps, d["S0"])
+    torch.cuda.synchronize()
+    return o, ST
+
+
+def small_inputs(B, T, H, Dk, Dv, dtype, seed, s0=True, g_lo=-0.5, key_mode="scaled"):
+    w = Workload("small", "train", B=B, T=T, H=H, Dk=Dk, Dv=Dv, dtype=dtype, key_mode=key_mode,
+                 gate_mode="uniform", s0="normal" if s0 else "zero", seed=seed)
+    inp = make_inputs(w)
+    if g_lo != -0.5:
+        gen = torch.Generator().manual_seed(seed + 1000)
+        inp["g"] = (torch.rand(B, T, H, generator=gen, dtype=torch.float64) * g_lo).float()
+    return inp
+
+
+# ---------------------------------------------------------------------------------------
+# forward
+# ---------------------------------------------------------------------------------------
+FWD_CASES = [
+    # B, T, H, Dk, Dv, dtype, s0, g_lo
+    (1, 1, 1, 64, 64, "f32", True, -0.5),
+    (1, 63, 2, 64, 64, "f32", True, -0.5),
+    (2, 64, 1, 128, 128, "f32", False, -0.5),
+    (1, 65, 3, 128, 64, "f32", True, -0.5),
+    (2, 200, 2, 64, 128, "f32", True, -0.01),   # long memory: S0 matters to the end
+    (1, 333, 2, 128, 128, "bf16", True, -0.5),
+    (2, 130, 3, 128, 128, "bf16", True, -0.01),
+    (1, 129, 2, 64, 64, "bf16", False, -0.5),
+    (1, 100, 1, 128, 64, "bf16", True, -0.5),
+]
+
+
+@pytest.mark.parametrize("B,T,H,Dk,Dv,dtype,s0,g_lo", FWD_CASES)
+def test_fwd_small(kla, oracle_mod, B, T, H, Dk, Dv, dtype, s0, g_lo):
+    inp = small_inputs(B, T, H, Dk, Dv, dtype, seed=T * 7 + H, s0=s0, g_lo=g_lo)
+    eps = 1e-6
+    o, ST = run_fwd(kla, inp, eps)
+    ro, rST = oracle_mod.forward(*(np64(inp[k]) for k in ("q", "k", "v", "eta", "g")), eps, np64(inp["S0"]))
+    assert rel_err(o, ro) <= TOL[dtype]
+    assert rel_err(ST, rST) <= TOL[dtype]
+
+
+def test_fwd_tiny_f32_workload(kla, oracle_mod):
+    w = WORKLOADS["tiny_fwd_f32"]
+    inp = make_inputs(w)
+    o, ST = run_fwd(kla, inp, w.eps)
+    ro, rST = oracle_mod.forward(*(np64(inp[k]) for k in ("q", "k", "v", "eta", "g")), w.eps, None)
+    assert rel_err(o, ro) <= 1e-4
+    assert rel_err(ST, rST) <= 1e-4
+
+
+def test_fwd_prefill_b8_t2048_workload(kla, oracle_mod):
+    w = WORKLOADS["prefill_b8_t2048_h8_d128"]
+    inp = make_inputs(w)
+    o, ST = run_fwd(kla, inp, w.eps)
+    ro, rST = oracle_mod.forward(*(np64(inp[k]) for k in ("q", "k", "v", "eta", "g")), w.eps, None)
+    assert rel_err(o, ro) <= 2e-2
+    assert rel_err(ST, rST) <= 2e-2
+
+
+def test_fwd_long_context_workload_sampled_heads(kla, oracle_mod):
+    w = WORKLOADS["prefill_b1_t65536_h16_d128"]
+    inp = make_inputs(w)
+    o, ST = run_fwd(kla, inp, w.eps)
+    pairs = [(0, 3), (0, 12)]
+    args = [heads_slice(np64(inp[k]), pairs) for k in ("q", "k", "v", "eta", "g")]
+    ro, rST = oracle_mod.forward(*args, w.eps, heads_slice(np64(inp["S0"]), pairs, state=True))
+    go = heads_slice(np64(o), pairs)
+    gST = heads_slice(np64(ST), pairs, state=True)
+    assert rel_err(go, ro) <= 2e-2
+    assert rel_err(gST, rST) <= 2e-2
+
+
+def test_fwd_state_passing_equals_one_call(kla):
+    """Checkpoint/resume: forward(T1) then forward(T2, S0=S_T1) == forward(T1+T2)."""
+    inp = small_inputs(2, 320, 2, 128, 128, "f32", seed=5, g_lo=-0.05)
+    eps = 1e-6
+    o, ST = run_fwd(kla, inp, eps)
+    cut = 192
+    a = {k: (v[:, :cut].contiguous() if v is not None and k != "S0" else v) for k, v in inp.items()}
+    b_ = {k: (v[:, cut:].contiguous() if v is not None and k != "S0" else v) for k, v in inp.items()}
+    o1, S1 = run_fwd(kla, a, eps)
+    b_["S0"] = S1.cpu()
+    o2, S2 = run_fwd(kla, b_, eps)
+    torch.testing.assert_close(torch.cat([o1, o2], 1), o, rtol=1e-4, atol=1e-4 * o.float().pow(2).mean().sqrt().item())
+    torch.testing.assert_close(S2, ST, rtol=1e-4, atol=1e-5)
+
+
+def test_fwd_zero_key_and_zero_eta(kla, oracle_mod):
+    """Edge cases: a key of zero norm with eps=0 skips the write; eta=0 only decays."""
+    inp = small_inputs(1, 70, 2, 64, 64, "f32", seed=11)
+    inp["k"][0, 5] = 0.0
+    inp["k"][0, 66, 1] = 0.0
+    inp["eta"][0, 10:20] = 0.0
+    o, ST = run_fwd(kla, inp, 0.0)
+    ro, rST = oracle_mod.forward(*(np64(inp[k]) for k in ("q", "k", "v", "eta", "g")), 0.0, np64(inp["S0"]))
+    assert rel_err(o, ro) <= 1e-4
+    assert rel_err(ST, rST) <= 1e-4
+
+
+def test_fwd_empty_sequence(kla):
+    S0 = torch.randn(2, 3, 64, 64, device="cuda")
+    z = torch.zeros(2, 0, 3, 64, device="cuda")
+    gz = torch.zeros(2, 0, 3, device="cuda")
+    o, ST = kla.chunk_fwd(z, z, z, gz, gz, 1e-6, S0)
+    torch.cuda.synchronize()
+    assert o.shape == (2, 0, 3, 64)
+    torch.testing.assert_close(ST, S0, rtol=0, atol=0)
+    _, ST0 = kla.chunk_fwd(z, z, z, gz, gz, 1e-6, None)
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(ST0) == 0
+
+
+def test_fwd_state_out_may_alias_initial_state(kla):
+    inp = small_inputs(1, 100, 2, 64, 64, "f32", seed=3)
+    d = {k: v.cuda() for k, v in inp.items()}
+    o_ref, S_ref = kla.chunk_fwd(d["q"], d["k"], d["v"], d["eta"], d["g"], 1e-6, d["S0"])
+    S = d["S0"].clone()
+    o, _ = kla.chunk_fwd(d["q"], d["k"], d["v"], d["eta"], d["g"], 1e-6, S, S_T=S)
+    torch.cuda.synchronize()
+    torch.testing.assert_close(o, o_ref, rtol=0, atol=0)
+    torch.testing.assert_close(S, S_ref, rtol=0, atol=0)
+
+
+# ---------------------------------------------------------------------------------------
+# decode
+# ---------------------------------------------------------------------------------------
+@pytest.mark.parametrize("Dk,Dv,dtype", [(128, 128, "bf16"), (64, 128, "f32"), (128, 64, "f32"), (64, 64, "bf16")])
+def test_decode_small(kla, oracle_mod, Dk, Dv, dtype):
+    w = Workload("dec", "decode", B=3, T=20, H=5, Dk=Dk, Dv=Dv, dtype=dtype, key_mode="scaled",
+                 gate_mode="uniform", s0="normal", seed=Dk + Dv)
+    inp = make_inputs(w)
+    S = inp["S0"].cuda().clone()
+    Sref = np64(inp["S0"])
+    for t in range(w.T):
+        o = kla.decode_step(inp["q"][t].cuda(), inp["k"][t].cuda(), inp["v"][t].cuda(),
+                            inp["eta"][t].cuda(), inp["g"][t].cuda(), S, w.eps)
+        ro, Sref = oracle_mod.decode_step(np64(inp["q"][t]), np64(inp["k"][t]), np64(inp["v"][t]),
+                                          np64(inp["eta"][t]), np64(inp["g"][t]), w.eps, Sref)
+        assert rel_err(o, ro) <= TOL[dtype]
+    assert rel_err(S, Sref) <= TOL[dtype]
+
+
+def test_decode_workload_1024_steps_sampled_heads(kla, oracle_mod):
+    w = WORKLOADS["decode_b64_h16_d128_x1024"]
+    inp = make_inputs(w)
+    pairs = [(0, 0), (17, 5), (63, 15)]
+    S = inp["S0"].cuda().clone()
+    qd, kd, vd = inp["q"].cuda(), inp["k"].cuda(), inp["v"].cuda()
+    ed, gd = inp["eta"].cuda(), inp["g"].cuda()
+    outs = torch.empty(w.T, w.B, w.H, w.Dv, dtype=qd.dtype, device="cuda")
+    for t in range(w.T):
+        kla.decode_step(qd[t], kd[t], vd[t], ed[t], gd[t], S, w.eps, o=outs[t])
+    torch.cuda.synchronize()
+    sel = lambda x: np.ascontiguousarray(np.stack([x[:, b, h] for b, h in pairs], axis=1)[:, :, None])
+    q, k, v, eta, g = (sel(np64(inp[n])) for n in ("q", "k", "v", "eta", "g"))
+    Sref = np.stack([np64(inp["S0"])[b, h] for b, h in pairs])[:, None]
+    got = sel(np64(outs))
+    ref = np.empty_like(got)
+    for t in range(w.T):
+        ref[t], Sref = oracle_mod.decode_step(q[t], k[t], v[t], eta[t], g[t], w.eps, Sref)
+    assert rel_err(got, ref) <= 2e-2
+    gS = np.stack([np64(S)[b, h] for b, h in pairs])[:, None]
+    assert rel_err(gS, Sref) <= 2e-2
+
+
+def test_decode_equals_forward_T1(kla):
+    inp = small_inputs(2, 1, 3, 128, 128, "bf16", seed=21)
+    d = {k: v.cuda() for k, v in inp.items()}
+    o, ST = kla.chunk_fwd(d["q"], d["k"], d["v"], d["eta"], d["g"], 1e-6, d["S0"])
+    S = d["S0"].clone()
+    od = kla.decode_step(d["q"][:, 0], d["k"][:, 0], d["v"][:, 0], d["eta"][:, 0], d["g"][:, 0], S, 1e-6)
+    torch.cuda.synchronize()
+    assert rel_err(od, np64(o[:, 0])) <= 1e-2
+    assert rel_err(S, np64(ST)) <= 1e-5
+
+
+# ---------------------------------------------------------------------------------------
+# backward
+# ---------------------------------------------------------------------------------------
+GRADS = ("dq", "dk", "dv", "deta", "dg", "dS0")
+
+BWD_CASES = [
+    # B, T, H, Dk, Dv, dtype, s0, with dS_T
+    (1, 64, 1, 64, 64, "f32", True, True),
+    (1, 150, 2, 64, 64, "f32", True, False),
+    (2, 97, 2, 128, 128, "f32", True, True),
+    (1, 70, 1, 128, 64, "f32", False, True),
+    (1, 130, 2, 64, 128, "f32", True, True),
+    (2, 200, 2, 128, 128, "bf16", True, True),
+    (1, 65, 3, 128, 128, "bf16", False, False),
+]
+
+
+@pytest.mark.parametrize("B,T,H,Dk,Dv,dtype,s0,with_dST", BWD_CASES)
+def test_bwd_small(kla, oracle_mod, B, T, H, Dk, Dv, dtype, s0, with_dST):
+    inp = small_inputs(B, T, H, Dk, Dv, dtype, seed=T + 3 * H, s0=s0, g_lo=-0.2)
+    gen = torch.Generator().manual_seed(T)
+    dO = torch.randn(B, T, H, Dv, generator=gen).to(inp["q"].dtype)
+    dST = torch.randn(B, H, Dk, Dv, generator=gen) if with_dST else None
+    eps = 1e-6
+    d = {k: (v.cuda() if v is not None else None) for k, v in inp.items()}
+    gr = kla.chunk_bwd(d["q"], d["k"], d["v"], d["eta"], d["g"], dO.cuda(), eps, d["S0"],
+                       dST.cuda() if dST is not None else None)
+    torch.cuda.synchronize()
+    ref = oracle_mod.backward(*(np64(inp[k]) for k in ("q", "k", "v", "eta", "g")), eps, np64(inp["S0"]),
+                              np64(dO), np64(dST))
+    for name in GRADS:
+        assert rel_err(gr[name], ref[name]) <= TOL[dtype], name
+
+
+def test_bwd_with_saved_chunk_states_matches_recompute(kla):
+    inp = small_inputs(1, 190, 2, 128, 128, "bf16", seed=8)
+    d = {k: v.cuda() for k, v in inp.items()}
+    dO = torch.randn(1, 190, 2, 128, device="cuda").to(torch.bfloat16)
+    _, _, Sc = kla.chunk_fwd(d["q"], d["k"], d["v"], d["eta"], d["g"], 1e-6, d["S0"], save_chunk_states=True)
+    g1 = kla.chunk_bwd(d["q"], d["k"], d["v"], d["eta"], d["g"], dO, 1e-6, d["S0"], None, Sc)
+    g2 = kla.chunk_bwd(d["q"], d["k"], d["v"], d["eta"], d["g"], dO, 1e-6, d["S0"], None, None)
+    torch.cuda.synchronize()
+    for name in GRADS:
+        a, b = g1[name].float(), g2[name].float()
+        scale = b.pow(2).mean().sqrt().item() + 1e-30
+        assert (a - b).abs().max().item() / scale <= 2e-2, name
+
+
+def test_bwd_training_workload_sampled_heads(kla, oracle_mod):
+    w = WORKLOADS["train_b4_t4096_h16_d128"]
+    inp = make_inputs(w)
+    d = {k: (v.cuda() if v is not None else None) for k, v in inp.items()}
+    dO = d["dO"].to(d["q"].dtype)
+    gr = kla.chunk_bwd(d["q"], d["k"], d["v"], d["eta"], d["g"], dO, w.eps, d["S0"])
+    torch.cuda.synchronize()
+    pairs = [(0, 0), (3, 9)]
+    args = [heads_slice(np64(inp[k]), pairs) for k in ("q", "k", "v", "eta", "g")]
+    ref = oracle_mod.backward(*args, w.eps, None, heads_slice(np64(dO), pairs), None)
+    for name in GRADS:
+        got = heads_slice(np64(gr[name]), pairs, state=(name == "dS0"))
+        assert rel_err(got, ref[name]) <= 2e-2, name
+
+
+def test_bwd_empty_sequence(kla):
+    dST = torch.randn(1, 2, 64, 64, device="cuda")
+    z = torch.zeros(1, 0, 2, 64, device="cuda")
+    gz = torch.zeros(1, 0, 2, device="cuda")
+    gr = kla.chunk_bwd(z, z, z, gz, gz, z, 1e-6, None, dST)
+    torch.cuda.synchronize()
+    torch.testing.assert_close(gr["dS0"], dST, rtol=0, atol=0)
