@@ -18,7 +18,8 @@ import os
 
 import torch
 
-__all__ = ["lib", "chunk_fwd", "chunk_bwd", "decode_step", "KLAError", "CHUNK", "library_path"]
+__all__ = ["lib", "chunk_fwd", "chunk_bwd", "decode_step", "check_device_error", "KLAError", "CHUNK",
+           "library_path"]
 
 CHUNK = 64
 KLA_F32, KLA_BF16 = 0, 1
@@ -52,15 +53,17 @@ def lib():
         L.kla_version.restype = i
         L.kla_chunk_fwd_workspace.argtypes = [i, i, i, i, i, i, i]
         L.kla_chunk_fwd_workspace.restype = sz
-        L.kla_chunk_fwd.argtypes = [vp, vp, vp, fp, fp, f, fp, vp, fp, fp, i, i, i, i, i, i, i, vp, sz, vp]
+        L.kla_chunk_fwd.argtypes = [vp, vp, vp, fp, fp, f, fp, vp, fp, fp, i, i, i, i, i, i, i, i, vp, sz, vp]
         L.kla_chunk_fwd.restype = i
         L.kla_chunk_bwd_workspace.argtypes = [i, i, i, i, i, i, i, i]
         L.kla_chunk_bwd_workspace.restype = sz
         L.kla_chunk_bwd.argtypes = [vp, vp, vp, fp, fp, f, fp, vp, fp, fp, vp, vp, vp, fp, fp, fp,
-                                    i, i, i, i, i, i, i, vp, sz, vp]
+                                    i, i, i, i, i, i, i, i, vp, sz, vp]
         L.kla_chunk_bwd.restype = i
-        L.kla_decode_step.argtypes = [vp, vp, vp, fp, fp, f, fp, vp, i, i, i, i, i, vp]
+        L.kla_decode_step.argtypes = [vp, vp, vp, fp, fp, f, fp, vp, i, i, i, i, i, i, vp]
         L.kla_decode_step.restype = i
+        L.kla_check_device_error.argtypes = [vp]
+        L.kla_check_device_error.restype = i
         _lib = L
     return _lib
 
@@ -77,11 +80,12 @@ def _ptr(t):
 
 
 def _dtype_code(t):
-    if t.dtype == torch.bfloat16:
+    dt = t if isinstance(t, torch.dtype) else t.dtype
+    if dt == torch.bfloat16:
         return KLA_BF16
-    if t.dtype == torch.float32:
+    if dt == torch.float32:
         return KLA_F32
-    raise TypeError(f"q/k/v must be bfloat16 or float32, got {t.dtype}")
+    raise TypeError(f"expected bfloat16 or float32, got {dt}")
 
 
 def _need(t, name, device, dtype=None, shape=None):
@@ -106,11 +110,12 @@ def _stream(device, stream):
 
 
 def chunk_fwd(q, k, v, eta, g, eps=1e-6, S0=None, *, o=None, S_T=None, save_chunk_states=False,
-              output_final_state=True, stream=None):
+              output_final_state=True, out_dtype=torch.float32, stream=None):
     """Chunkwise prefill (section 4, Propositions 3-4).
 
     q, k: [B,T,H,Dk]; v: [B,T,H,Dv] (bf16 or fp32, same dtype); eta, g: [B,T,H] fp32;
-    S0: [B,H,Dk,Dv] fp32 or None.  Returns (o, S_T) or (o, S_T, S_chunks) when
+    S0: [B,H,Dk,Dv] fp32 or None.  o is written in `out_dtype` (fp32 by default; a bf16
+    store rounds each output once).  Returns (o, S_T) or (o, S_T, S_chunks) when
     save_chunk_states (S_chunks: [B,H,ceil(T/64),Dk,Dv], the state at each chunk start).
     """
     dev = k.device
@@ -121,8 +126,8 @@ def chunk_fwd(q, k, v, eta, g, eps=1e-6, S0=None, *, o=None, S_T=None, save_chun
     _need(eta, "eta", dev, torch.float32, (B, T, H)); _need(g, "g", dev, torch.float32, (B, T, H))
     _need(S0, "S0", dev, torch.float32, (B, H, Dk, Dv))
     if o is None:
-        o = torch.empty(B, T, H, Dv, device=dev, dtype=dt)
-    _need(o, "o", dev, dt, (B, T, H, Dv))
+        o = torch.empty(B, T, H, Dv, device=dev, dtype=out_dtype)
+    _need(o, "o", dev, None, (B, T, H, Dv))
     if S_T is None and output_final_state:
         S_T = torch.empty(B, H, Dk, Dv, device=dev, dtype=torch.float32)
     _need(S_T, "S_T", dev, torch.float32, (B, H, Dk, Dv))
@@ -131,17 +136,18 @@ def chunk_fwd(q, k, v, eta, g, eps=1e-6, S0=None, *, o=None, S_T=None, save_chun
         Sc = torch.empty(B, H, (T + CHUNK - 1) // CHUNK, Dk, Dv, device=dev, dtype=torch.float32)
     st = lib().kla_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(eta), _ptr(g), float(eps), _ptr(S0),
                              _ptr(o), _ptr(S_T), _ptr(Sc), B, T, H, Dk, Dv, CHUNK, _dtype_code(k),
-                             None, 0, _stream(dev, stream))
+                             _dtype_code(o), None, 0, _stream(dev, stream))
     _check(st, "kla_chunk_fwd")
     return (o, S_T, Sc) if save_chunk_states else (o, S_T)
 
 
 def chunk_bwd(q, k, v, eta, g, dO, eps=1e-6, S0=None, dS_T=None, S_chunks=None, *, stream=None,
-              workspace=None):
+              workspace=None, out_dtype=torch.float32):
     """Gradients of the chunkwise forward w.r.t. q, k, v, eta, g and S0.
 
     dO: [B,T,H,Dv] (same dtype as q); dS_T: [B,H,Dk,Dv] fp32 or None; S_chunks: the
     array chunk_fwd(save_chunk_states=True) returned for the same inputs, or None.
+    dq, dk, dv are written in `out_dtype` (fp32 by default).
     Returns dict(dq, dk, dv, deta, dg, dS0).
     """
     dev = k.device
@@ -154,7 +160,9 @@ def chunk_bwd(q, k, v, eta, g, dO, eps=1e-6, S0=None, dS_T=None, S_chunks=None, 
     _need(dS_T, "dS_T", dev, torch.float32, (B, H, Dk, Dv))
     NC = (T + CHUNK - 1) // CHUNK
     _need(S_chunks, "S_chunks", dev, torch.float32, (B, H, NC, Dk, Dv))
-    out = dict(dq=torch.empty_like(q), dk=torch.empty_like(k), dv=torch.empty_like(v),
+    out = dict(dq=torch.empty(q.shape, device=dev, dtype=out_dtype),
+               dk=torch.empty(k.shape, device=dev, dtype=out_dtype),
+               dv=torch.empty(v.shape, device=dev, dtype=out_dtype),
                deta=torch.empty_like(eta), dg=torch.empty_like(g),
                dS0=torch.empty(B, H, Dk, Dv, device=dev, dtype=torch.float32))
     L = lib()
@@ -164,12 +172,13 @@ def chunk_bwd(q, k, v, eta, g, dO, eps=1e-6, S0=None, dS_T=None, S_chunks=None, 
     st = L.kla_chunk_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(eta), _ptr(g), float(eps), _ptr(S0), _ptr(dO),
                          _ptr(dS_T), _ptr(S_chunks), _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]),
                          _ptr(out["deta"]), _ptr(out["dg"]), _ptr(out["dS0"]), B, T, H, Dk, Dv, CHUNK,
-                         _dtype_code(k), _ptr(workspace), workspace.numel(), _stream(dev, stream))
+                         _dtype_code(k), _dtype_code(out_dtype), _ptr(workspace), workspace.numel(),
+                         _stream(dev, stream))
     _check(st, "kla_chunk_bwd")
     return out
 
 
-def decode_step(q, k, v, eta, g, S, eps=1e-6, *, o=None, stream=None):
+def decode_step(q, k, v, eta, g, S, eps=1e-6, *, o=None, out_dtype=torch.float32, stream=None):
     """One decode token for every (b, h): q, k [B,H,Dk]; v [B,H,Dv]; eta, g [B,H] fp32;
     S [B,H,Dk,Dv] fp32 updated in place.  Returns o [B,H,Dv]."""
     dev = S.device
@@ -179,9 +188,15 @@ def decode_step(q, k, v, eta, g, S, eps=1e-6, *, o=None, stream=None):
     _need(eta, "eta", dev, torch.float32, (B, H)); _need(g, "g", dev, torch.float32, (B, H))
     _need(S, "S", dev, torch.float32, (B, H, Dk, Dv))
     if o is None:
-        o = torch.empty(B, H, Dv, device=dev, dtype=dt)
-    _need(o, "o", dev, dt, (B, H, Dv))
+        o = torch.empty(B, H, Dv, device=dev, dtype=out_dtype)
+    _need(o, "o", dev, None, (B, H, Dv))
     st = lib().kla_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(eta), _ptr(g), float(eps), _ptr(S), _ptr(o),
-                               B, H, Dk, Dv, _dtype_code(k), _stream(dev, stream))
+                               B, H, Dk, Dv, _dtype_code(k), _dtype_code(o), _stream(dev, stream))
     _check(st, "kla_decode_step")
     return o
+
+
+def check_device_error(stream=None, device=None):
+    """Synchronise the stream and raise KLAError if a kernel gave up on a bounded wait."""
+    dev = device if device is not None else torch.device("cuda", torch.cuda.current_device())
+    _check(lib().kla_check_device_error(_stream(dev, stream)), "kla_check_device_error")

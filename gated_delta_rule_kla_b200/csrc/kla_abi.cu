@@ -32,7 +32,8 @@ bool aligned16(const void* p) { return p == nullptr || (reinterpret_cast<uintptr
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-kla_status check_common(int B, int T, int H, int Dk, int Dv, int chunk, int dtype, float eps) {
+kla_status check_common(int B, int T, int H, int Dk, int Dv, int chunk, int dtype, int out_dtype,
+                        float eps) {
     if (B < 1 || H < 1 || T < 0)
         return fail(KLA_ERR_INVALID_ARG, "sizes must satisfy B>=1, H>=1, T>=0 (got B=%d T=%d H=%d)",
                     B, T, H);
@@ -43,6 +44,8 @@ kla_status check_common(int B, int T, int H, int Dk, int Dv, int chunk, int dtyp
         return fail(KLA_ERR_UNSUPPORTED, "chunk must be %d (got %d)", kla::kChunkLen, chunk);
     if (dtype != KLA_F32 && dtype != KLA_BF16)
         return fail(KLA_ERR_UNSUPPORTED, "dtype must be KLA_F32 or KLA_BF16 (got %d)", dtype);
+    if (out_dtype != KLA_F32 && out_dtype != KLA_BF16)
+        return fail(KLA_ERR_UNSUPPORTED, "out_dtype must be KLA_F32 or KLA_BF16 (got %d)", out_dtype);
     // 32-bit index headroom for per-token offsets inside kernels is not assumed: kernels
     // index with size_t; but B*H and grid sizes must fit the launch limits.
     if ((long long)B * H > (1LL << 30)) return fail(KLA_ERR_UNSUPPORTED, "B*H too large");
@@ -103,9 +106,9 @@ size_t kla_chunk_fwd_workspace(int B, int T, int H, int Dk, int Dv, int chunk, i
 kla_status kla_chunk_fwd(const void* q, const void* k, const void* v, const float* eta,
                          const float* g, float eps, const float* S0, void* o, float* S_T,
                          float* S_chunks, int B, int T, int H, int Dk, int Dv, int chunk,
-                         int dtype, void* ws, size_t ws_bytes, void* stream) {
+                         int dtype, int out_dtype, void* ws, size_t ws_bytes, void* stream) {
     (void)ws; (void)ws_bytes;
-    kla_status st = check_common(B, T, H, Dk, Dv, chunk, dtype, eps);
+    kla_status st = check_common(B, T, H, Dk, Dv, chunk, dtype, out_dtype, eps);
     if (st != KLA_OK) return st;
     if (T > 0) {
         REQUIRE_PTR(q); REQUIRE_PTR(k); REQUIRE_PTR(v); REQUIRE_PTR(eta); REQUIRE_PTR(g);
@@ -121,7 +124,8 @@ kla_status kla_chunk_fwd(const void* q, const void* k, const void* v, const floa
         }
         return KLA_OK;
     }
-    kla::FwdArgs a{q, k, v, eta, g, eps, S0, o, S_T, S_chunks, B, T, H, Dk, Dv, dtype == KLA_BF16};
+    kla::FwdArgs a{q, k, v, eta, g, eps, S0, o, S_T, S_chunks, B, T, H, Dk, Dv, dtype == KLA_BF16,
+                   out_dtype == KLA_BF16};
     cudaError_t e = kla::chunk_fwd_tc_supported(a) ? kla::launch_chunk_fwd_tc(a, s)
                                                    : kla::launch_chunk_fwd_simt(a, s);
     if (e != cudaSuccess) return cuda_fail(e, "kla_chunk_fwd launch");
@@ -140,8 +144,8 @@ kla_status kla_chunk_bwd(const void* q, const void* k, const void* v, const floa
                          const float* g, float eps, const float* S0, const void* dO,
                          const float* dS_T, const float* S_chunks, void* dq, void* dk, void* dv,
                          float* deta, float* dg, float* dS0, int B, int T, int H, int Dk, int Dv,
-                         int chunk, int dtype, void* ws, size_t ws_bytes, void* stream) {
-    kla_status st = check_common(B, T, H, Dk, Dv, chunk, dtype, eps);
+                         int chunk, int dtype, int out_dtype, void* ws, size_t ws_bytes, void* stream) {
+    kla_status st = check_common(B, T, H, Dk, Dv, chunk, dtype, out_dtype, eps);
     if (st != KLA_OK) return st;
     REQUIRE_PTR(dS0);
     OPTIONAL_PTR(S0); OPTIONAL_PTR(dS_T); OPTIONAL_PTR(S_chunks);
@@ -169,7 +173,7 @@ kla_status kla_chunk_bwd(const void* q, const void* k, const void* v, const floa
     if (Sc == nullptr) {
         float* Sc_ws = reinterpret_cast<float*>(w + off[0]);
         kla::FwdArgs fa{q, k, v, eta, g, eps, S0, nullptr, nullptr, Sc_ws, B, T, H, Dk, Dv,
-                        dtype == KLA_BF16};
+                        dtype == KLA_BF16, false};
         e = kla::launch_chunk_fwd_simt(fa, s);
         if (e != cudaSuccess) return cuda_fail(e, "kla_chunk_bwd state recompute");
         Sc = Sc_ws;
@@ -178,7 +182,8 @@ kla_status kla_chunk_bwd(const void* q, const void* k, const void* v, const floa
     float* acc3 = reinterpret_cast<float*>(w + off[3]);
     kla::BwdArgs a{q, k, v, eta, g, eps, Sc, dO, dS_T, dq, dk, dv, deta, dg, dS0,
                    reinterpret_cast<float*>(w + off[1]), reinterpret_cast<float*>(w + off[2]),
-                   acc3, acc3 + ntok, acc3 + 2 * ntok, B, T, H, Dk, Dv, dtype == KLA_BF16};
+                   acc3, acc3 + ntok, acc3 + 2 * ntok, B, T, H, Dk, Dv, dtype == KLA_BF16,
+                   out_dtype == KLA_BF16};
     e = kla::launch_chunk_bwd_simt(a, s);
     if (e != cudaSuccess) return cuda_fail(e, "kla_chunk_bwd launch");
     return KLA_OK;
@@ -186,15 +191,24 @@ kla_status kla_chunk_bwd(const void* q, const void* k, const void* v, const floa
 
 kla_status kla_decode_step(const void* q, const void* k, const void* v, const float* eta,
                            const float* g, float eps, float* S, void* o, int B, int H, int Dk,
-                           int Dv, int dtype, void* stream) {
-    kla_status st = check_common(B, 0, H, Dk, Dv, kla::kChunkLen, dtype, eps);
+                           int Dv, int dtype, int out_dtype, void* stream) {
+    kla_status st = check_common(B, 0, H, Dk, Dv, kla::kChunkLen, dtype, out_dtype, eps);
     if (st != KLA_OK) return st;
     REQUIRE_PTR(q); REQUIRE_PTR(k); REQUIRE_PTR(v); REQUIRE_PTR(eta); REQUIRE_PTR(g);
     REQUIRE_PTR(S);
     OPTIONAL_PTR(o);
-    kla::DecodeArgs a{q, k, v, eta, g, eps, S, o, B, H, Dk, Dv, dtype == KLA_BF16};
+    kla::DecodeArgs a{q, k, v, eta, g, eps, S, o, B, H, Dk, Dv, dtype == KLA_BF16,
+                      out_dtype == KLA_BF16};
     cudaError_t e = kla::launch_decode(a, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "kla_decode_step launch");
+    return KLA_OK;
+}
+
+kla_status kla_check_device_error(void* stream) {
+    unsigned int flag = 0;
+    cudaError_t e = kla::tc_take_error(static_cast<cudaStream_t>(stream), &flag);
+    if (e != cudaSuccess) return cuda_fail(e, "kla_check_device_error");
+    if (flag) return fail(KLA_ERR_TIMEOUT, "a kernel gave up on a bounded wait (flag %u)", flag);
     return KLA_OK;
 }
 

@@ -124,7 +124,7 @@ __device__ __forceinline__ void chunk_decay(const float* graw, float* Gs, float*
 // ------------------------------------------------------------------------------------
 // Forward
 // ------------------------------------------------------------------------------------
-template <int DK, typename Tin>
+template <int DK, typename Tin, typename TOut>
 __global__ void __launch_bounds__(NT, 1) chunk_fwd_simt_kernel(FwdArgs a) {
     constexpr int NV = 64;
     constexpr int LDK = DK + 1, LDV = NV + 1, LDC = C + 1;
@@ -151,7 +151,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_simt_kernel(FwdArgs a) {
     const Tin* q = static_cast<const Tin*>(a.q);
     const Tin* k = static_cast<const Tin*>(a.k);
     const Tin* v = static_cast<const Tin*>(a.v);
-    Tin* o = static_cast<Tin*>(a.o);
+    TOut* o = static_cast<TOut*>(a.o);
     const size_t sbase = ((size_t)b * H + h) * DK * Dv;
     const int NC = (T + C - 1) / C;
 
@@ -245,10 +245,10 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_simt_kernel(FwdArgs a) {
             for (int m = 0; m < 4; ++m) {
                 const int i = ty + 16 * m;
                 if (i < n) {
-                    Tin* orow = o + tok_index(b, t0 + i, h, T, H) * Dv + v0;
+                    TOut* orow = o + tok_index(b, t0 + i, h, T, H) * Dv + v0;
 #pragma unroll
                     for (int nn = 0; nn < 4; ++nn)
-                        orow[tx + 16 * nn] = from_f32<Tin>(fmaf(gams[i], ao[m][nn], ap[m][nn]));
+                        orow[tx + 16 * nn] = from_f32<TOut>(fmaf(gams[i], ao[m][nn], ap[m][nn]));
                 }
             }
         }
@@ -302,7 +302,7 @@ constexpr size_t fwd_smem_bytes() {
 // A CTA owns NV = 32 value columns; the column-coupled gradients (dq, dkhat, db, dc, dG)
 // are partial sums over its columns and are added atomically into fp32 accumulators.
 // ------------------------------------------------------------------------------------
-template <int DK, typename Tin>
+template <int DK, typename Tin, typename TOut>
 __global__ void __launch_bounds__(NT, 1) chunk_bwd_simt_kernel(BwdArgs a) {
     constexpr int NV = 32;
     constexpr int LDK = DK + 1, LDV = NV + 1, LDC = C + 1;
@@ -340,7 +340,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_bwd_simt_kernel(BwdArgs a) {
     const Tin* k = static_cast<const Tin*>(a.k);
     const Tin* v = static_cast<const Tin*>(a.v);
     const Tin* dO = static_cast<const Tin*>(a.dO);
-    Tin* dv = static_cast<Tin*>(a.dv);
+    TOut* dv = static_cast<TOut*>(a.dv);
     const size_t sbase = ((size_t)b * H + h) * DK * Dv;
     const int NC = (T + C - 1) / C;
 
@@ -474,7 +474,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_bwd_simt_kernel(BwdArgs a) {
             const size_t ti = tok_index(b, t0 + i, h, T, H);
             const float dr = dRs[i * LDV + lane];
             const float vv = to_f32(v[ti * Dv + v0 + lane]);
-            dv[ti * Dv + v0 + lane] = from_f32<Tin>(cs[i] * dr);
+            dv[ti * Dv + v0 + lane] = from_f32<TOut>(cs[i] * dr);
             const float s_rv = warp_sum(dr * vv);
             const float s_rx = warp_sum(dr * Xs[i * LDV + lane]);
             const float s_oq = warp_sum(dOs[i * LDV + lane] * QSs[i * LDV + lane]);
@@ -658,15 +658,15 @@ constexpr size_t bwd_smem_bytes() {
 //   b = eta r^2/(r^2+eps), c = eta r/(r^2+eps), khat = k/r
 //   deta = db r^2/den + dc r/den,  dr = db eta 2 r eps/den^2 + dc eta (eps - r^2)/den^2
 //   dk   = (dkhat - khat (khat . dkhat)) / r + khat dr
-template <int DK, typename Tin>
+template <int DK, typename Tin, typename TOut>
 __global__ void __launch_bounds__(256) bwd_finalize_kernel(BwdArgs a, size_t ntok) {
     const size_t w = (size_t)blockIdx.x * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (w >= ntok) return;
     constexpr int PER = DK / 32;
     const Tin* k = static_cast<const Tin*>(a.k);
-    Tin* dq = static_cast<Tin*>(a.dq);
-    Tin* dk = static_cast<Tin*>(a.dk);
+    TOut* dq = static_cast<TOut*>(a.dq);
+    TOut* dk = static_cast<TOut*>(a.dk);
     float kv[PER], dkh[PER];
     float r2 = 0.f;
 #pragma unroll
@@ -674,7 +674,7 @@ __global__ void __launch_bounds__(256) bwd_finalize_kernel(BwdArgs a, size_t nto
         kv[u] = to_f32(k[w * DK + lane + 32 * u]);
         dkh[u] = a.acc_dkh[w * DK + lane + 32 * u];
         r2 = fmaf(kv[u], kv[u], r2);
-        dq[w * DK + lane + 32 * u] = from_f32<Tin>(a.acc_dq[w * DK + lane + 32 * u]);
+        dq[w * DK + lane + 32 * u] = from_f32<TOut>(a.acc_dq[w * DK + lane + 32 * u]);
     }
     r2 = warp_sum(r2);
     const float r = sqrtf(r2);
@@ -695,7 +695,7 @@ __global__ void __launch_bounds__(256) bwd_finalize_kernel(BwdArgs a, size_t nto
     for (int u = 0; u < PER; ++u) {
         const float kh = kv[u] * inv_r;
         const float val = live ? (dkh[u] - kh * kd) * inv_r + kh * dr : 0.f;
-        dk[w * DK + lane + 32 * u] = from_f32<Tin>(val);
+        dk[w * DK + lane + 32 * u] = from_f32<TOut>(val);
     }
     if (lane == 0) a.deta[w] = deta;
 }
@@ -719,29 +719,29 @@ __global__ void bwd_dg_kernel(BwdArgs a) {
     }
 }
 
-template <int DK, typename Tin>
+template <int DK, typename Tin, typename TOut>
 cudaError_t fwd_launch_t(const FwdArgs& a, cudaStream_t st) {
     const size_t smem = fwd_smem_bytes<DK>();
-    cudaError_t e = cudaFuncSetAttribute(chunk_fwd_simt_kernel<DK, Tin>,
+    cudaError_t e = cudaFuncSetAttribute(chunk_fwd_simt_kernel<DK, Tin, TOut>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid(a.Dv / 64, a.H, a.B);
-    chunk_fwd_simt_kernel<DK, Tin><<<grid, NT, smem, st>>>(a);
+    chunk_fwd_simt_kernel<DK, Tin, TOut><<<grid, NT, smem, st>>>(a);
     return cudaGetLastError();
 }
 
-template <int DK, typename Tin>
+template <int DK, typename Tin, typename TOut>
 cudaError_t bwd_launch_t(const BwdArgs& a, cudaStream_t st) {
     const size_t smem = bwd_smem_bytes<DK>();
-    cudaError_t e = cudaFuncSetAttribute(chunk_bwd_simt_kernel<DK, Tin>,
+    cudaError_t e = cudaFuncSetAttribute(chunk_bwd_simt_kernel<DK, Tin, TOut>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid(a.Dv / 32, a.H, a.B);
-    chunk_bwd_simt_kernel<DK, Tin><<<grid, NT, smem, st>>>(a);
+    chunk_bwd_simt_kernel<DK, Tin, TOut><<<grid, NT, smem, st>>>(a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     const size_t ntok = (size_t)a.B * a.T * a.H;
     if (ntok > 0) {
-        bwd_finalize_kernel<DK, Tin><<<(unsigned)((ntok + 7) / 8), 256, 0, st>>>(a, ntok);
+        bwd_finalize_kernel<DK, Tin, TOut><<<(unsigned)((ntok + 7) / 8), 256, 0, st>>>(a, ntok);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         const size_t nch = (size_t)a.B * a.H * ((a.T + C - 1) / C);
         bwd_dg_kernel<<<(unsigned)((nch + 127) / 128), 128, 0, st>>>(a);
@@ -750,18 +750,28 @@ cudaError_t bwd_launch_t(const BwdArgs& a, cudaStream_t st) {
     return e;
 }
 
+template <int DK, typename Tin>
+cudaError_t fwd_launch_o(const FwdArgs& a, cudaStream_t st) {
+    return a.out_bf16 ? fwd_launch_t<DK, Tin, __nv_bfloat16>(a, st) : fwd_launch_t<DK, Tin, float>(a, st);
+}
+
+template <int DK, typename Tin>
+cudaError_t bwd_launch_o(const BwdArgs& a, cudaStream_t st) {
+    return a.out_bf16 ? bwd_launch_t<DK, Tin, __nv_bfloat16>(a, st) : bwd_launch_t<DK, Tin, float>(a, st);
+}
+
 }  // namespace
 
 cudaError_t launch_chunk_fwd_simt(const FwdArgs& a, cudaStream_t st) {
-    if (a.bf16) return a.Dk == 128 ? fwd_launch_t<128, __nv_bfloat16>(a, st)
-                                   : fwd_launch_t<64, __nv_bfloat16>(a, st);
-    return a.Dk == 128 ? fwd_launch_t<128, float>(a, st) : fwd_launch_t<64, float>(a, st);
+    if (a.bf16) return a.Dk == 128 ? fwd_launch_o<128, __nv_bfloat16>(a, st)
+                                   : fwd_launch_o<64, __nv_bfloat16>(a, st);
+    return a.Dk == 128 ? fwd_launch_o<128, float>(a, st) : fwd_launch_o<64, float>(a, st);
 }
 
 cudaError_t launch_chunk_bwd_simt(const BwdArgs& a, cudaStream_t st) {
-    if (a.bf16) return a.Dk == 128 ? bwd_launch_t<128, __nv_bfloat16>(a, st)
-                                   : bwd_launch_t<64, __nv_bfloat16>(a, st);
-    return a.Dk == 128 ? bwd_launch_t<128, float>(a, st) : bwd_launch_t<64, float>(a, st);
+    if (a.bf16) return a.Dk == 128 ? bwd_launch_o<128, __nv_bfloat16>(a, st)
+                                   : bwd_launch_o<64, __nv_bfloat16>(a, st);
+    return a.Dk == 128 ? bwd_launch_o<128, float>(a, st) : bwd_launch_o<64, float>(a, st);
 }
 
 }  // namespace kla

@@ -1,10 +1,653 @@
-// kla_chunk_tc.cu -- tensor-core (tcgen05) chunk forward; placeholder until written.
+// kla_chunk_tc.cu -- chunkwise KLA forward on the 5th-generation tensor cores (sm_100a):
+// TMA tile loads, tcgen05.mma with fp32 accumulators in TMEM, fp32 state.
+//
+// Math ("Kaczmarz Linear Attention", section 4, Propositions 3-4, written on unit keys
+// khat = k/r with b = eta r^2/(r^2+eps), c = eta r/(r^2+eps); Appendix B.4 coefficient
+// substitution): per chunk of C = 64 tokens with incoming state S (Dk x Dv),
+//   P   = Gam o (Q Khat^T)                      (lower incl. diagonal)
+//   L   = Diag(b) (Gam^- o Khat Khat^T),  T = (I + L)^{-1}   (forward substitution, B.2)
+//   W   = T Diag(b gamma) Khat,  U' = T Diag(c) V,  U = U' - W S          (Eq. 7)
+//   O   = Diag(gamma) Q S + P U                                             (Eq. 8)
+//   S'  = gamma_last S + (Diag(delta) Khat)^T U,  delta_j = e^{G_last - G_j} (Eq. 9)
+//
+// Every product is an M = 128 tcgen05 MMA in a transposed form, so one CTA owns a whole
+// (b, h) head and TMEM lane = matrix row throughout:
+//   Gram   [Q; K] K^T        lane = token (Q rows 0-63, K rows 64-127), col = token
+//   SQ     S^T Q^T           lane = dv, col = token
+//   W^T    K^T T'^T          lane = dk, col = token        (T' = T Diag(b gamma / r))
+//   U^T    V^T T''^T - S^T W^T  lane = dv, col = token     (T'' = T Diag(c))
+//   S     += Ktil^T U        lane = dk, col = dv           (Ktil = Diag(delta / r) K)
+//   PU     U^T P^T           lane = dv, col = token
+// Operands that are computed on chip (P, T', T'', S, U, Ktil) are rounded to bf16 as a
+// hi + lo pair and multiplied term by term (the lo x lo term is dropped), which keeps ~16
+// significant bits; W enters as a single bf16.  q, k, v are bf16 inputs and exact.
+//
+// The fp32 master state lives in TMEM (lane = dk, 128 columns): each chunk scales it by
+// gamma_last and the Ktil^T U MMA accumulates onto it; a bf16 hi/lo copy in shared memory
+// is the MMA operand.  One CTA of 128 threads (thread t <-> TMEM lane t) per (b, h); the
+// chunk loop is sequential, with the next chunk's tiles prefetched by TMA into the other
+// stage.  Every
+// wait is bounded: on timeout the kernel records an error word and returns after freeing
+// TMEM.
+#include <cuda.h>
+
+#include "kla_device.cuh"
 #include "kla_launch.h"
+#include "kla_sm100.cuh"
 
 namespace kla {
 
-bool chunk_fwd_tc_supported(const FwdArgs&) { return false; }
+__device__ unsigned int g_tc_error = 0;
 
-cudaError_t launch_chunk_fwd_tc(const FwdArgs&, cudaStream_t) { return cudaErrorNotSupported; }
+namespace {
+
+using namespace sm100;
+
+constexpr int DK = 128, DV = 128, CH = 64;
+constexpr int NTHREADS = 128;
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
+
+// shared-memory map (offsets from a 1024-aligned base)
+constexpr uint32_t OFF_QK = 0;          // 2 stages x 32 KB: [Q;K] rows, two dk blocks
+constexpr uint32_t QK_STAGE = 32768;
+constexpr uint32_t OFF_V = 65536;       // 2 stages x 16 KB: V, two dv blocks of [64 x 64]
+constexpr uint32_t V_STAGE = 16384;
+constexpr uint32_t OFF_SHI = 98304;     // 32 KB: S hi, two dv blocks of [128 dk x 64]
+constexpr uint32_t OFF_SLO = 131072;    // 32 KB: S lo
+constexpr uint32_t OFF_P = 163840;      // 16 KB: P hi [64 x 64], P lo
+constexpr uint32_t OFF_Z = 180224;      // 32 KB: L/T fp32 -> T' T'' hi/lo -> Ktil hi/lo
+constexpr uint32_t OFF_MISC = 212992;   // barriers, TMEM slot, per-token scalars
+constexpr uint32_t SMEM_BYTES = OFF_MISC + 4096 + 1024;  // + alignment slack
+constexpr int LDL = 65;                 // row stride of the fp32 solve buffer
+
+// TMEM columns
+constexpr uint32_t TM_G = 0, TM_SQ = 64, TM_W = 128, TM_U = 192, TM_S = 256, TM_PU = 384;
+
+struct Misc {
+    uint64_t full[2];
+    uint64_t mma;
+    uint32_t tmem_base;
+    uint32_t pad;
+    float G[CH], gam[CH], del[CH], bco[CH], cco[CH], invr[CH], graw[CH], eta[CH];
+};
+
+__device__ __forceinline__ size_t tok_index(int b, int t, int h, int T, int H) {
+    return ((size_t)b * T + t) * H + h;
+}
+
+// In-place inverse of the unit lower-triangular 64x64 matrix I + L (L strictly lower,
+// fp32, row stride LDL).  Diagonal 16x16 blocks by forward substitution (one warp per
+// block, one lane per column), then block rows I = 1..3:
+//   T_IJ = -T_II sum_{K=J}^{I-1} L_IK T_KJ.
+// X is scratch for 3 * 256 floats.  Must be called by all 128 threads.
+__device__ __forceinline__ void invert_unit_lower64(float* Lf, float* X, int tid) {
+    const int warp = tid >> 5, lane = tid & 31;
+    {
+        const int base = 16 * warp;
+        float x[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            float acc = 0.f;
+#pragma unroll
+            for (int j = 0; j < i; ++j) acc = fmaf(Lf[(base + i) * LDL + base + j], x[j], acc);
+            x[i] = (i < lane) ? 0.f : ((i == lane) ? 1.f : -acc);
+        }
+        __syncwarp();
+        if (lane < 16) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) Lf[(base + i) * LDL + base + lane] = x[i];
+        }
+    }
+    __syncthreads();
+    for (int I = 1; I < 4; ++I) {
+        for (int e = tid; e < I * 256; e += NTHREADS) {
+            const int J = e >> 8, r = (e >> 4) & 15, cc = e & 15;
+            float acc = 0.f;
+            for (int K = J; K < I; ++K) {
+#pragma unroll
+                for (int m = 0; m < 16; ++m)
+                    acc = fmaf(Lf[(16 * I + r) * LDL + 16 * K + m], Lf[(16 * K + m) * LDL + 16 * J + cc], acc);
+            }
+            X[e] = acc;
+        }
+        __syncthreads();
+        for (int e = tid; e < I * 256; e += NTHREADS) {
+            const int J = e >> 8, r = (e >> 4) & 15, cc = e & 15;
+            float acc = 0.f;
+#pragma unroll
+            for (int m = 0; m < 16; ++m)
+                acc = fmaf(Lf[(16 * I + r) * LDL + 16 * I + m], X[(J << 8) + (m << 4) + cc], acc);
+            Lf[(16 * I + r) * LDL + 16 * J + cc] = -acc;
+        }
+        __syncthreads();
+    }
+}
+
+// Write chunks [c0, c0 + n) of row r of a swizzled bf16 block from 8*n fp32 values.
+__device__ __forceinline__ void st_chunks_bf16(uint8_t* block, int r, int c0, int n, const float* v) {
+    for (int c = 0; c < n; ++c) {
+        uint4 u;
+        u.x = pack_bf16x2(v[8 * c + 0], v[8 * c + 1]);
+        u.y = pack_bf16x2(v[8 * c + 2], v[8 * c + 3]);
+        u.z = pack_bf16x2(v[8 * c + 4], v[8 * c + 5]);
+        u.w = pack_bf16x2(v[8 * c + 6], v[8 * c + 7]);
+        *reinterpret_cast<uint4*>(block + sw128_off(r, c0 + c)) = u;
+    }
+}
+
+// Split 8*n fp32 values into hi/lo bf16 and write chunks [c0, c0 + n) of row r of two blocks.
+__device__ __forceinline__ void st_chunks_split(uint8_t* hi_block, uint8_t* lo_block, int r, int c0, int n,
+                                                const float* v) {
+    for (int c = 0; c < n; ++c) {
+        float h[8], l[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) split_bf16(v[8 * c + e], h[e], l[e]);
+        uint4 uh, ul;
+        uh.x = pack_bf16x2(h[0], h[1]); uh.y = pack_bf16x2(h[2], h[3]);
+        uh.z = pack_bf16x2(h[4], h[5]); uh.w = pack_bf16x2(h[6], h[7]);
+        ul.x = pack_bf16x2(l[0], l[1]); ul.y = pack_bf16x2(l[2], l[3]);
+        ul.z = pack_bf16x2(l[4], l[5]); ul.w = pack_bf16x2(l[6], l[7]);
+        *reinterpret_cast<uint4*>(hi_block + sw128_off(r, c0 + c)) = uh;
+        *reinterpret_cast<uint4*>(lo_block + sw128_off(r, c0 + c)) = ul;
+    }
+}
+
+template <typename TOut>
+__global__ void __launch_bounds__(NTHREADS, 1)
+    chunk_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                        const __grid_constant__ CUtensorMap tm_v, FwdArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    Misc* ms = reinterpret_cast<Misc*>(sm + OFF_MISC);
+    float* Lf = reinterpret_cast<float*>(sm + OFF_Z);
+    float* Xs = Lf + 64 * LDL;
+
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int H = a.H, T = a.T;
+    const int b = blockIdx.x / H, h = blockIdx.x % H;
+    const int NC = (T + CH - 1) / CH;
+    const uint32_t sbase = smem_u32(sm);
+    const uint32_t bar_full0 = smem_u32(&ms->full[0]);
+    const uint32_t bar_mma = smem_u32(&ms->mma);
+    const size_t state_off = ((size_t)b * H + h) * DK * DV;
+
+    if (tid == 0) {
+        mbar_init(bar_full0, 1);
+        mbar_init(bar_full0 + 8, 1);
+        mbar_init(bar_mma, 1);
+        fence_mbar_init();
+        prefetch_tmap(&tm_q);
+        prefetch_tmap(&tm_k);
+        prefetch_tmap(&tm_v);
+    }
+    if (warp == 0) {
+        tmem_alloc(smem_u32(&ms->tmem_base), 512);
+        tmem_relinquish();
+    }
+
+    // fp32 master state: thread t owns row dk = t, kept in TMEM columns [TM_S, TM_S + 128)
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = ms->tmem_base;
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+#pragma unroll 1
+    for (int q4 = 0; q4 < 4; ++q4) {
+        float x[32];
+        if (a.S0) {
+            const float4* src = reinterpret_cast<const float4*>(a.S0 + state_off + (size_t)tid * DV + 32 * q4);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float4 v4 = src[i];
+                x[4 * i] = v4.x; x[4 * i + 1] = v4.y; x[4 * i + 2] = v4.z; x[4 * i + 3] = v4.w;
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) x[i] = 0.f;
+        }
+        tmem_st32(tmem + lane_base + TM_S + 32 * q4, x);
+        st_chunks_split(sm + OFF_SHI + (q4 >> 1) * 16384, sm + OFF_SLO + (q4 >> 1) * 16384, tid, 4 * (q4 & 1), 4, x);
+    }
+    tmem_st_wait();
+    fence_proxy_async();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    auto issue_loads = [&](int c, int st) {
+        const uint32_t bar = bar_full0 + 8 * st;
+        const uint32_t qk = sbase + OFF_QK + st * QK_STAGE;
+        const uint32_t vv = sbase + OFF_V + st * V_STAGE;
+        const int t0 = c * CH;
+        mbar_expect_tx(bar, 6 * 8192);
+        tma_load_4d(qk, &tm_q, bar, 0, h, t0, b);
+        tma_load_4d(qk + 16384, &tm_q, bar, 64, h, t0, b);
+        tma_load_4d(qk + 8192, &tm_k, bar, 0, h, t0, b);
+        tma_load_4d(qk + 16384 + 8192, &tm_k, bar, 64, h, t0, b);
+        tma_load_4d(vv, &tm_v, bar, 0, h, t0, b);
+        tma_load_4d(vv + 8192, &tm_v, bar, 64, h, t0, b);
+    };
+
+    if (tid == 0 && NC > 0) issue_loads(0, 0);
+    float g_next = 0.f, eta_next = 0.f;
+    if (tid < CH && tid < T) {
+        const size_t ti = tok_index(b, tid, h, T, H);
+        g_next = a.g[ti];
+        eta_next = a.eta[ti];
+    }
+
+    uint32_t mma_phase = 0;
+    bool aborted = false;
+    int issued = (NC > 0) ? 0 : -1;  // last chunk whose tiles were requested
+    int landed = -1;                 // last chunk whose tiles were waited for
+
+    for (int c = 0; c < NC; ++c) {
+        const int st = c & 1;
+        const int t0 = c * CH;
+        const int n = min(CH, T - t0);
+        uint8_t* qk = sm + OFF_QK + st * QK_STAGE;
+        uint8_t* vt = sm + OFF_V + st * V_STAGE;
+        const uint32_t qk_a = sbase + OFF_QK + st * QK_STAGE;
+        const uint32_t v_a = sbase + OFF_V + st * V_STAGE;
+
+        if (tid < CH) {
+            ms->graw[tid] = (tid < n) ? g_next : 0.f;
+            ms->eta[tid] = (tid < n) ? eta_next : 0.f;
+            if (c + 1 < NC && (c + 1) * CH + tid < T) {
+                const size_t ti = tok_index(b, (c + 1) * CH + tid, h, T, H);
+                g_next = a.g[ti];
+                eta_next = a.eta[ti];
+            }
+        }
+        if (tid == 0 && c + 1 < NC) issue_loads(c + 1, st ^ 1);
+        if (c + 1 < NC) issued = c + 1;
+        const bool ok_tma = mbar_wait_bounded(bar_full0 + 8 * st, (c >> 1) & 1, kWaitLimitNs);
+        if (__syncthreads_or(!ok_tma)) { aborted = true; break; }
+        landed = c;
+
+        // key norms and Kaczmarz coefficients (thread 64 + j reads key row j)
+        if (tid >= CH) {
+            const int j = tid - CH;
+            float r2 = 0.f;
+#pragma unroll
+            for (int blk = 0; blk < 2; ++blk)
+#pragma unroll
+                for (int cc = 0; cc < 8; ++cc) {
+                    float f[8];
+                    unpack_bf16x8(*reinterpret_cast<const uint4*>(qk + blk * 16384 + 8192 + j * 128 + cc * 16), f);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) r2 = fmaf(f[e], f[e], r2);
+                }
+            const KaczCoef cf = kacz_coef(ms->eta[j], r2, a.eps);
+            ms->bco[j] = cf.b;
+            ms->cco[j] = cf.c;
+            ms->invr[j] = cf.inv_r;
+        }
+        if (warp == 0) {  // inclusive prefix sum of g inside the chunk (2 tokens per lane)
+            const int l = tid;
+            const float x0 = ms->graw[2 * l], x1 = ms->graw[2 * l + 1];
+            float s = x0 + x1;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float y = __shfl_up_sync(0xffffffffu, s, o);
+                if (l >= o) s += y;
+            }
+            const float excl = s - (x0 + x1);
+            ms->G[2 * l] = excl + x0;
+            ms->G[2 * l + 1] = excl + x0 + x1;
+        }
+        __syncthreads();
+        if (tid < CH) {
+            ms->gam[tid] = __expf(ms->G[tid]);
+            ms->del[tid] = __expf(ms->G[n - 1] - ms->G[tid]);
+        }
+
+        // ---- MMA: Gram = [Q; K] K^T and SQ = S^T Q^T
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t ig = idesc_bf16(128, 64, false, false);
+#pragma unroll
+            for (int s = 0; s < 8; ++s) {
+                const uint32_t off = (s >> 2) * 16384 + (s & 3) * 32;
+                mma_bf16(tmem + TM_G, smem_desc(qk_a + off, 16, 1024), smem_desc(qk_a + off + 8192, 16, 1024),
+                         ig, s > 0);
+            }
+            const uint32_t isq = idesc_bf16(128, 64, true, false);
+#pragma unroll
+            for (int part = 0; part < 2; ++part) {
+                const uint32_t sa = sbase + (part ? OFF_SLO : OFF_SHI);
+#pragma unroll
+                for (int s = 0; s < 8; ++s)
+                    mma_bf16(tmem + TM_SQ, smem_desc(sa + s * 2048, 16384, 1024),
+                             smem_desc(qk_a + (s >> 2) * 16384 + (s & 3) * 32, 16, 1024), isq, (part | s) > 0);
+            }
+            mma_commit(bar_mma);
+        }
+        if (a.S_chunks) {
+            float4* dst = reinterpret_cast<float4*>(a.S_chunks + ((size_t)blockIdx.x * NC + c) * DK * DV +
+                                                    (size_t)tid * DV);
+#pragma unroll 1
+            for (int q4 = 0; q4 < 4; ++q4) {
+                float x[32];
+                tmem_ld32(tmem + lane_base + TM_S + 32 * q4, x);
+                tmem_ld_wait();
+#pragma unroll
+                for (int i = 0; i < 8; ++i) dst[8 * q4 + i] = make_float4(x[4 * i], x[4 * i + 1], x[4 * i + 2], x[4 * i + 3]);
+            }
+        }
+        {
+            const bool ok = mbar_wait_bounded(bar_mma, mma_phase, kWaitLimitNs);
+            mma_phase ^= 1;
+            if (__syncthreads_or(!ok)) { aborted = true; break; }
+        }
+        tc_fence_after();
+
+        // ---- Gram epilogue: P (rows 0-63, hi/lo bf16) and L (rows 64-127, fp32), 32 columns at a time
+#pragma unroll 1
+        for (int half = 0; half < 2; ++half) {
+            float x[32];
+            tmem_ld32(tmem + lane_base + TM_G + 32 * half, x);
+            tmem_ld_wait();
+            if (tid < CH) {
+                const int i = tid;
+                const float Gi = ms->G[i];
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const int j = 32 * half + e;
+                    x[e] = (j <= i) ? __expf(Gi - ms->G[j]) * x[e] * ms->invr[j] : 0.f;
+                }
+                st_chunks_split(sm + OFF_P, sm + OFF_P + 8192, i, 4 * half, 4, x);
+            } else {
+                const int i = tid - CH;
+                const float Gi = ms->G[i];
+                const float bi = ms->bco[i] * ms->invr[i];
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const int j = 32 * half + e;
+                    Lf[i * LDL + j] = (j < i) ? bi * __expf(Gi - ms->G[j]) * x[e] * ms->invr[j] : 0.f;
+                }
+            }
+        }
+        tc_fence_before();
+        __syncthreads();
+        invert_unit_lower64(Lf, Xs, tid);
+        // T' = T Diag(b gamma / r), T'' = T Diag(c): thread -> row tid/2, 32 columns
+        {
+            const int i = tid >> 1, half = tid & 1;
+            float tv[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) tv[e] = Lf[i * LDL + 32 * half + e];
+            __syncthreads();
+            float hi[32], lo[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+                const int j = 32 * half + e;
+                split_bf16(tv[e] * (ms->bco[j] * ms->gam[j] * ms->invr[j]), hi[e], lo[e]);
+            }
+            st_chunks_bf16(sm + OFF_Z, i, 4 * half, 4, hi);
+            st_chunks_bf16(sm + OFF_Z + 8192, i, 4 * half, 4, lo);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) split_bf16(tv[e] * ms->cco[32 * half + e], hi[e], lo[e]);
+            st_chunks_bf16(sm + OFF_Z + 16384, i, 4 * half, 4, hi);
+            st_chunks_bf16(sm + OFF_Z + 24576, i, 4 * half, 4, lo);
+        }
+        fence_proxy_async();
+        __syncthreads();
+
+        // ---- MMA: W^T = K^T T'^T and U'^T = V^T T''^T
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t iw = idesc_bf16(128, 64, true, false);
+#pragma unroll
+            for (int part = 0; part < 2; ++part)
+#pragma unroll
+                for (int s = 0; s < 4; ++s)
+                    mma_bf16(tmem + TM_W, smem_desc(qk_a + 8192 + s * 2048, 16384, 1024),
+                             smem_desc(sbase + OFF_Z + part * 8192 + s * 32, 16, 1024), iw, (part | s) > 0);
+#pragma unroll
+            for (int part = 0; part < 2; ++part)
+#pragma unroll
+                for (int s = 0; s < 4; ++s)
+                    mma_bf16(tmem + TM_U, smem_desc(v_a + s * 2048, 8192, 1024),
+                             smem_desc(sbase + OFF_Z + 16384 + part * 8192 + s * 32, 16, 1024), iw,
+                             (part | s) > 0);
+            mma_commit(bar_mma);
+        }
+        {
+            const bool ok = mbar_wait_bounded(bar_mma, mma_phase, kWaitLimitNs);
+            mma_phase ^= 1;
+            if (__syncthreads_or(!ok)) { aborted = true; break; }
+        }
+        tc_fence_after();
+        // ---- W^T to bf16 (over the consumed V stage); Ktil = Diag(delta / r) K hi/lo (over T tiles)
+        {
+#pragma unroll 1
+            for (int half = 0; half < 2; ++half) {
+                float x[32];
+                tmem_ld32(tmem + lane_base + TM_W + 32 * half, x);
+                tmem_ld_wait();
+                st_chunks_bf16(vt, tid, 4 * half, 4, x);
+            }
+            {  // S <- gamma_last S, ahead of the MMA that accumulates Ktil^T U onto it
+                const float gC = ms->gam[n - 1];
+#pragma unroll 1
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    float x[32];
+                    tmem_ld32(tmem + lane_base + TM_S + 32 * q4, x);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) x[e] *= gC;
+                    tmem_st32(tmem + lane_base + TM_S + 32 * q4, x);
+                }
+                tmem_st_wait();
+            }
+            const int j = tid >> 1, blk = tid & 1;
+            const float sc = ms->del[j] * ms->invr[j];
+#pragma unroll
+            for (int cc = 0; cc < 8; ++cc) {
+                float f[8], hi[8], lo[8];
+                const uint32_t off = (uint32_t)(j * 128 + cc * 16);  // same swizzle phase: (64 + j) & 7 == j & 7
+                unpack_bf16x8(*reinterpret_cast<const uint4*>(qk + blk * 16384 + 8192 + off), f);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) split_bf16(f[e] * sc, hi[e], lo[e]);
+                uint4 uh, ul;
+                uh.x = pack_bf16x2(hi[0], hi[1]); uh.y = pack_bf16x2(hi[2], hi[3]);
+                uh.z = pack_bf16x2(hi[4], hi[5]); uh.w = pack_bf16x2(hi[6], hi[7]);
+                ul.x = pack_bf16x2(lo[0], lo[1]); ul.y = pack_bf16x2(lo[2], lo[3]);
+                ul.z = pack_bf16x2(lo[4], lo[5]); ul.w = pack_bf16x2(lo[6], lo[7]);
+                *reinterpret_cast<uint4*>(sm + OFF_Z + blk * 8192 + off) = uh;
+                *reinterpret_cast<uint4*>(sm + OFF_Z + 16384 + blk * 8192 + off) = ul;
+            }
+        }
+        tc_fence_before();
+        fence_proxy_async();
+        __syncthreads();
+
+        // ---- MMA: U^T -= S^T W^T
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t isw = idesc_bf16(128, 64, true, true, true);
+#pragma unroll
+            for (int part = 0; part < 2; ++part) {
+                const uint32_t sa = sbase + (part ? OFF_SLO : OFF_SHI);
+#pragma unroll
+                for (int s = 0; s < 8; ++s)
+                    mma_bf16(tmem + TM_U, smem_desc(sa + s * 2048, 16384, 1024),
+                             smem_desc(v_a + s * 2048, 8192, 1024), isw, 1);
+            }
+            mma_commit(bar_mma);
+        }
+        {
+            const bool ok = mbar_wait_bounded(bar_mma, mma_phase, kWaitLimitNs);
+            mma_phase ^= 1;
+            if (__syncthreads_or(!ok)) { aborted = true; break; }
+        }
+        tc_fence_after();
+        // ---- U^T hi/lo to bf16 over the consumed [Q; K] stage (thread = dv row)
+#pragma unroll 1
+        for (int half = 0; half < 2; ++half) {
+            float x[32];
+            tmem_ld32(tmem + lane_base + TM_U + 32 * half, x);
+            tmem_ld_wait();
+            st_chunks_split(qk, qk + 16384, tid, 4 * half, 4, x);
+        }
+        tc_fence_before();
+        fence_proxy_async();
+        __syncthreads();
+
+        // ---- MMA: S += Ktil^T U (N = 128) and PU = U^T P^T
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t ids = idesc_bf16(128, 128, true, false);
+            const uint32_t ipu = idesc_bf16(128, 64, false, false);
+            const uint32_t kt_hi = sbase + OFF_Z, kt_lo = sbase + OFF_Z + 16384;
+            const uint32_t u_hi = qk_a, u_lo = qk_a + 16384;
+            const uint32_t p_hi = sbase + OFF_P, p_lo = sbase + OFF_P + 8192;
+            const uint32_t ka[3] = {kt_hi, kt_hi, kt_lo}, ub[3] = {u_hi, u_lo, u_hi};
+#pragma unroll
+            for (int p = 0; p < 3; ++p)
+#pragma unroll
+                for (int s = 0; s < 4; ++s)
+                    mma_bf16(tmem + TM_S, smem_desc(ka[p] + s * 2048, 8192, 1024),
+                             smem_desc(ub[p] + s * 32, 16, 1024), ids, 1);
+            const uint32_t ua[3] = {u_hi, u_hi, u_lo}, pb[3] = {p_hi, p_lo, p_hi};
+#pragma unroll
+            for (int p = 0; p < 3; ++p)
+#pragma unroll
+                for (int s = 0; s < 4; ++s)
+                    mma_bf16(tmem + TM_PU, smem_desc(ua[p] + s * 32, 16, 1024),
+                             smem_desc(pb[p] + s * 32, 16, 1024), ipu, (p | s) > 0);
+            mma_commit(bar_mma);
+        }
+        {
+            const bool ok = mbar_wait_bounded(bar_mma, mma_phase, kWaitLimitNs);
+            mma_phase ^= 1;
+            if (__syncthreads_or(!ok)) { aborted = true; break; }
+        }
+        tc_fence_after();
+        // ---- new state to bf16 hi/lo (thread = dk row) and outputs (thread = dv)
+        {
+#pragma unroll 1
+            for (int q4 = 0; q4 < 4; ++q4) {
+                float x[32];
+                tmem_ld32(tmem + lane_base + TM_S + 32 * q4, x);
+                tmem_ld_wait();
+                st_chunks_split(sm + OFF_SHI + (q4 >> 1) * 16384, sm + OFF_SLO + (q4 >> 1) * 16384, tid,
+                                4 * (q4 & 1), 4, x);
+            }
+            if (a.o != nullptr) {
+                TOut* o = static_cast<TOut*>(a.o);
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    float sq[32], pu[32];
+                    tmem_ld32(tmem + lane_base + TM_SQ + 32 * half, sq);
+                    tmem_ld32(tmem + lane_base + TM_PU + 32 * half, pu);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const int i = 32 * half + e;
+                        if (i < n)
+                            o[tok_index(b, t0 + i, h, T, H) * DV + tid] =
+                                from_f32<TOut>(fmaf(ms->gam[i], sq[e], pu[e]));
+                    }
+                }
+            }
+        }
+        tc_fence_before();
+        fence_proxy_async();
+        __syncthreads();
+    }
+
+    if (aborted) {
+        if (tid == 0) atomicOr(&g_tc_error, 1u);
+        // let TMA loads that may still be landing in shared memory finish first
+        for (int cc = landed + 1; cc <= issued; ++cc)
+            (void)mbar_wait_bounded(bar_full0 + 8 * (cc & 1), (cc >> 1) & 1, kWaitLimitNs);
+    } else if (a.S_T) {
+        float4* dst = reinterpret_cast<float4*>(a.S_T + state_off + (size_t)tid * DV);
+#pragma unroll 1
+        for (int q4 = 0; q4 < 4; ++q4) {
+            float x[32];
+            tmem_ld32(tmem + lane_base + TM_S + 32 * q4, x);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 8; ++i) dst[8 * q4 + i] = make_float4(x[4 * i], x[4 * i + 1], x[4 * i + 2], x[4 * i + 3]);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// ---------------------------------------------------------------- host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static bool tried = false;
+    if (!tried) {
+        tried = true;
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+// 4-D map over a [B, T, H, 128] bf16 tensor; box = 64 tokens x 64 features of one (b, h).
+bool make_map(CUtensorMap* m, const void* base, int B, int T, int H) {
+    EncodeTiledFn enc = get_encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[4] = {(cuuint64_t)128, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
+    cuuint64_t strides[3] = {(cuuint64_t)128 * 2, (cuuint64_t)H * 128 * 2, (cuuint64_t)T * H * 128 * 2};
+    cuuint32_t box[4] = {64, 1, 64, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bool chunk_fwd_tc_supported(const FwdArgs& a) {
+    return a.bf16 && a.Dk == 128 && a.Dv == 128 && a.T > 0 && get_encode_fn() != nullptr;
+}
+
+cudaError_t launch_chunk_fwd_tc(const FwdArgs& a, cudaStream_t st) {
+    CUtensorMap mq, mk, mv;
+    if (!make_map(&mq, a.q, a.B, a.T, a.H) || !make_map(&mk, a.k, a.B, a.T, a.H) ||
+        !make_map(&mv, a.v, a.B, a.T, a.H))
+        return cudaErrorInvalidValue;
+    cudaError_t e;
+    if (a.out_bf16) {
+        e = cudaFuncSetAttribute(chunk_fwd_tc_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        chunk_fwd_tc_kernel<__nv_bfloat16><<<a.B * a.H, NTHREADS, SMEM_BYTES, st>>>(mq, mk, mv, a);
+    } else {
+        e = cudaFuncSetAttribute(chunk_fwd_tc_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        chunk_fwd_tc_kernel<float><<<a.B * a.H, NTHREADS, SMEM_BYTES, st>>>(mq, mk, mv, a);
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t tc_take_error(cudaStream_t st, unsigned int* flag) {
+    cudaError_t e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return e;
+    e = cudaMemcpyFromSymbol(flag, g_tc_error, sizeof(unsigned int));
+    if (e != cudaSuccess) return e;
+    const unsigned int zero = 0;
+    return cudaMemcpyToSymbol(g_tc_error, &zero, sizeof(unsigned int));
+}
 
 }  // namespace kla

@@ -17,14 +17,14 @@
 
 namespace kla {
 
-template <int DK, int DV, typename Tin>
+template <int DK, int DV, typename Tin, typename TOut>
 __global__ void __launch_bounds__(256) decode_step_kernel(const Tin* __restrict__ q,
                                                           const Tin* __restrict__ k,
                                                           const Tin* __restrict__ v,
                                                           const float* __restrict__ eta,
                                                           const float* __restrict__ g, float eps,
                                                           float* __restrict__ S,
-                                                          Tin* __restrict__ o) {
+                                                          TOut* __restrict__ o) {
     constexpr int NT = 256;
     constexpr int COLG = DV / 4;       // float4 column groups
     constexpr int ROWG = NT / COLG;    // row groups
@@ -69,7 +69,7 @@ __global__ void __launch_bounds__(256) decode_step_kernel(const Tin* __restrict_
         n2 += scal[0][w];
         kdq += scal[1][w];
     }
-    const float alpha = __expf(g[head]);
+    const float alpha = expf(g[head]);
     const float den = n2 + eps;
     const float beta = den > 0.f ? eta[head] / den : 0.f;
 
@@ -116,28 +116,34 @@ __global__ void __launch_bounds__(256) decode_step_kernel(const Tin* __restrict_
     }
     // o = alpha S^T q + (k.q) beta e
     if (o != nullptr && rg == 0) {
-        Tin* oh = o + (size_t)head * DV + cg * 4;
-        oh[0] = from_f32<Tin>(fmaf(alpha, sq.x, kdq * be.x));
-        oh[1] = from_f32<Tin>(fmaf(alpha, sq.y, kdq * be.y));
-        oh[2] = from_f32<Tin>(fmaf(alpha, sq.z, kdq * be.z));
-        oh[3] = from_f32<Tin>(fmaf(alpha, sq.w, kdq * be.w));
+        TOut* oh = o + (size_t)head * DV + cg * 4;
+        oh[0] = from_f32<TOut>(fmaf(alpha, sq.x, kdq * be.x));
+        oh[1] = from_f32<TOut>(fmaf(alpha, sq.y, kdq * be.y));
+        oh[2] = from_f32<TOut>(fmaf(alpha, sq.z, kdq * be.z));
+        oh[3] = from_f32<TOut>(fmaf(alpha, sq.w, kdq * be.w));
     }
 }
 
-template <int DK, int DV, typename Tin>
+template <int DK, int DV, typename Tin, typename TOut>
 static cudaError_t launch_decode_t(const DecodeArgs& a, cudaStream_t st) {
-    decode_step_kernel<DK, DV, Tin><<<a.B * a.H, 256, 0, st>>>(
+    decode_step_kernel<DK, DV, Tin, TOut><<<a.B * a.H, 256, 0, st>>>(
         static_cast<const Tin*>(a.q), static_cast<const Tin*>(a.k), static_cast<const Tin*>(a.v),
-        a.eta, a.g, a.eps, a.S, static_cast<Tin*>(a.o));
+        a.eta, a.g, a.eps, a.S, static_cast<TOut*>(a.o));
     return cudaGetLastError();
+}
+
+template <int DK, int DV, typename Tin>
+static cudaError_t launch_decode_o(const DecodeArgs& a, cudaStream_t st) {
+    return a.out_bf16 ? launch_decode_t<DK, DV, Tin, __nv_bfloat16>(a, st)
+                      : launch_decode_t<DK, DV, Tin, float>(a, st);
 }
 
 template <typename Tin>
 static cudaError_t launch_decode_d(const DecodeArgs& a, cudaStream_t st) {
-    if (a.Dk == 128 && a.Dv == 128) return launch_decode_t<128, 128, Tin>(a, st);
-    if (a.Dk == 128 && a.Dv == 64) return launch_decode_t<128, 64, Tin>(a, st);
-    if (a.Dk == 64 && a.Dv == 128) return launch_decode_t<64, 128, Tin>(a, st);
-    return launch_decode_t<64, 64, Tin>(a, st);
+    if (a.Dk == 128 && a.Dv == 128) return launch_decode_o<128, 128, Tin>(a, st);
+    if (a.Dk == 128 && a.Dv == 64) return launch_decode_o<128, 64, Tin>(a, st);
+    if (a.Dk == 64 && a.Dv == 128) return launch_decode_o<64, 128, Tin>(a, st);
+    return launch_decode_o<64, 64, Tin>(a, st);
 }
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st) {

@@ -15,7 +15,8 @@ struct DecodeArgs {
     float* S;
     void* o;
     int B, H, Dk, Dv;
-    bool bf16;
+    bool bf16;      // q, k, v are bf16 (else fp32)
+    bool out_bf16;  // o is bf16 (else fp32)
 };
 
 struct FwdArgs {
@@ -27,7 +28,8 @@ struct FwdArgs {
     float* S_T;       // may be null; may alias S0
     float* S_chunks;  // may be null
     int B, T, H, Dk, Dv;
-    bool bf16;
+    bool bf16;      // q, k, v are bf16 (else fp32)
+    bool out_bf16;  // o is bf16 (else fp32)
 };
 
 struct BwdArgs {
@@ -42,7 +44,8 @@ struct BwdArgs {
     // fp32 accumulators (zeroed by the launcher): [B,T,H,Dk] x2, [B,T,H] x3
     float *acc_dq, *acc_dkh, *acc_db, *acc_dc, *acc_dG;
     int B, T, H, Dk, Dv;
-    bool bf16;
+    bool bf16;      // q, k, v, dO are bf16 (else fp32)
+    bool out_bf16;  // dq, dk, dv are bf16 (else fp32)
 };
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st);
@@ -51,5 +54,8 @@ cudaError_t launch_chunk_bwd_simt(const BwdArgs& a, cudaStream_t st);
 // Tensor-core (tcgen05) forward for bf16 inputs with Dk == Dv == 128.
 bool chunk_fwd_tc_supported(const FwdArgs& a);
 cudaError_t launch_chunk_fwd_tc(const FwdArgs& a, cudaStream_t st);
+// Synchronise `st`, then read and clear the device error word of the tensor-core kernels
+// (non-zero when a bounded wait expired).
+cudaError_t tc_take_error(cudaStream_t st, unsigned int* flag);
 
 }  // namespace kla

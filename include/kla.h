@@ -24,12 +24,17 @@
  *   - Arguments are validated on the host before any launch; an invalid call returns an
  *     error status and launches nothing.  A failed launch returns KLA_ERR_CUDA.
  *     kla_last_error() gives a one-line description of the last failure on this thread.
+ *   - Kernels never wait without a bound: if an internal wait expires the kernel stops,
+ *     records it, and kla_check_device_error() reports KLA_ERR_TIMEOUT.
  *   - Supported shapes: Dk, Dv in {64, 128}; chunk == 64; B, H >= 1; T >= 0 (T == 0 copies
  *     S0 to S_T).  The last chunk may be partial.  eps >= 0.  g <= 0 is the intended range
  *     (the decay factors exp(G_i - G_j) are then <= 1); g > 0 is accepted without an
  *     accuracy guarantee.
- *   - dtype selects the element type of q, k, v, o, dO, dq, dk, dv: KLA_F32 or KLA_BF16.
- *     eta, g, S0, S_T, S, dS_T and every other gradient are fp32.  The state is always fp32.
+ *   - dtype selects the element type of the inputs q, k, v (and dO): KLA_F32 or KLA_BF16.
+ *     out_dtype selects the element type of the outputs o (and dq, dk, dv): KLA_F32 or
+ *     KLA_BF16.  eta, g, S0, S_T, S, dS_T, deta, dg, dS0 are always fp32, as is the state.
+ *     Outputs are computed in fp32 and rounded once on store; with heavy-tailed outputs a
+ *     bf16 store alone moves the largest elements by 2^-9 of their magnitude.
  *   - NaN or Inf inputs propagate; they are not checked.
  *
  * Layouts (row-major):
@@ -52,7 +57,7 @@ typedef enum {
     KLA_ERR_UNSUPPORTED = 2, /* shape or dtype outside the supported set */
     KLA_ERR_WORKSPACE = 3,   /* workspace missing or smaller than the *_workspace() size */
     KLA_ERR_CUDA = 4,        /* a CUDA launch or runtime call failed */
-    KLA_ERR_TIMEOUT = 5      /* reserved: a bounded device-side wait expired */
+    KLA_ERR_TIMEOUT = 5      /* a bounded device-side wait expired (kla_check_device_error) */
 } kla_status;
 
 typedef enum { KLA_F32 = 0, KLA_BF16 = 1 } kla_dtype;
@@ -75,7 +80,7 @@ int kla_version(void);
  *   eta, g       in   [B,T,H] fp32: write gate (0..1 intended) and log-decay
  *   eps          in   stabiliser of Eq. (3), >= 0
  *   S0           in   [B,H,Dk,Dv] fp32 initial state, or NULL for a zero state
- *   o            out  [B,T,H,Dv] of `dtype`, or NULL to skip the readout
+ *   o            out  [B,T,H,Dv] of `out_dtype`, or NULL to skip the readout
  *   S_T          out  [B,H,Dk,Dv] fp32 final state, or NULL.  May alias S0.
  *   S_chunks     out  [B,H,ceil(T/chunk),Dk,Dv] fp32 state at the start of every chunk, or
  *                     NULL.  Passing it to kla_chunk_bwd saves the backward's recompute.
@@ -87,14 +92,14 @@ size_t kla_chunk_fwd_workspace(int B, int T, int H, int Dk, int Dv, int chunk, i
 kla_status kla_chunk_fwd(const void *q, const void *k, const void *v, const float *eta,
                          const float *g, float eps, const float *S0, void *o, float *S_T,
                          float *S_chunks, int B, int T, int H, int Dk, int Dv, int chunk,
-                         int dtype, void *ws, size_t ws_bytes, void *stream);
+                         int dtype, int out_dtype, void *ws, size_t ws_bytes, void *stream);
 
 /*
  * kla_chunk_bwd -- gradients of the chunkwise forward.
  * The paper gives no backward; this one differentiates the forward above exactly (same
  * result as reverse-mode differentiation of the tokenwise recurrence).  Given the upstream
  * gradients dO (of o) and dS_T (of S_T, NULL = zero), it returns the gradients of every
- * input: dq, dk, dv (of `dtype`), deta, dg ([B,T,H] fp32) and dS0 ([B,H,Dk,Dv] fp32;
+ * input: dq, dk, dv (of `out_dtype`), deta, dg ([B,T,H] fp32) and dS0 ([B,H,Dk,Dv] fp32;
  * written even when S0 is NULL).  S_chunks may be the array kla_chunk_fwd wrote for the
  * same inputs, or NULL to recompute it inside the workspace.
  * Gradient of k at a key of exactly zero norm: the normalised-key form used on the GPU has
@@ -108,7 +113,8 @@ kla_status kla_chunk_bwd(const void *q, const void *k, const void *v, const floa
                          const float *g, float eps, const float *S0, const void *dO,
                          const float *dS_T, const float *S_chunks, void *dq, void *dk, void *dv,
                          float *deta, float *dg, float *dS0, int B, int T, int H, int Dk,
-                         int Dv, int chunk, int dtype, void *ws, size_t ws_bytes, void *stream);
+                         int Dv, int chunk, int dtype, int out_dtype, void *ws, size_t ws_bytes,
+                         void *stream);
 
 /*
  * kla_decode_step -- one generated token: Algorithm 1 (left panel), lines 2-6 (readout
@@ -117,12 +123,20 @@ kla_status kla_chunk_bwd(const void *q, const void *k, const void *v, const floa
  *   q, k    in     [B,H,Dk] of `dtype`      v   in  [B,H,Dv] of `dtype`
  *   eta, g  in     [B,H] fp32               eps in  >= 0
  *   S       in/out [B,H,Dk,Dv] fp32, updated in place to S_t
- *   o       out    [B,H,Dv] of `dtype` (o_t = S_t^T q_t), or NULL
+ *   o       out    [B,H,Dv] of `out_dtype` (o_t = S_t^T q_t), or NULL
  * Each state element is read once and written once.
  */
 kla_status kla_decode_step(const void *q, const void *k, const void *v, const float *eta,
                            const float *g, float eps, float *S, void *o, int B, int H, int Dk,
-                           int Dv, int dtype, void *stream);
+                           int Dv, int dtype, int out_dtype, void *stream);
+
+/*
+ * kla_check_device_error -- synchronises `stream`, then reads and clears the library's
+ * device error word.  Returns KLA_ERR_TIMEOUT if a kernel gave up on a bounded internal
+ * wait since the last check (its outputs are then invalid), KLA_ERR_CUDA if the stream
+ * reports an error, KLA_OK otherwise.  Not part of the paper: a failure-detection hook.
+ */
+kla_status kla_check_device_error(void *stream);
 
 #ifdef __cplusplus
 }

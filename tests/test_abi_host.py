@@ -44,14 +44,14 @@ def test_status_strings(L):
     assert L.kla_version() >= 100
 
 
-def _fwd(L, B=1, T=64, H=1, Dk=128, Dv=128, chunk=64, dtype=1, eps=1e-6, q=FAKE, ws=None):
+def _fwd(L, B=1, T=64, H=1, Dk=128, Dv=128, chunk=64, dtype=1, out_dtype=0, eps=1e-6, q=FAKE, ws=None):
     return L.kla_chunk_fwd(q, FAKE, FAKE, FAKE, FAKE, eps, None, FAKE, FAKE, None, B, T, H, Dk, Dv,
-                           chunk, dtype, ws, 0, None)
+                           chunk, dtype, out_dtype, ws, 0, None)
 
 
 @pytest.mark.parametrize("kw,code", [
     (dict(Dk=96), UNSUPPORTED), (dict(Dv=32), UNSUPPORTED), (dict(chunk=32), UNSUPPORTED),
-    (dict(dtype=7), UNSUPPORTED), (dict(eps=-1.0), INVALID), (dict(eps=float("nan")), INVALID),
+    (dict(dtype=7), UNSUPPORTED), (dict(out_dtype=3), UNSUPPORTED), (dict(eps=-1.0), INVALID), (dict(eps=float("nan")), INVALID),
     (dict(B=0), INVALID), (dict(H=0), INVALID), (dict(T=-1), INVALID),
     (dict(q=None), INVALID), (dict(q=MISALIGNED), INVALID),
 ])
@@ -67,26 +67,26 @@ def test_bwd_workspace_checked(L):
     assert need == r256(2 * 3 * 2 * 64 * 128 * 4) + 2 * r256(ntok * 64 * 4) + r256(3 * ntok * 4)
     assert L.kla_chunk_bwd_workspace(2, 100, 3, 64, 128, 64, 1, 1) == need - r256(2 * 3 * 2 * 64 * 128 * 4)
     st = L.kla_chunk_bwd(FAKE, FAKE, FAKE, FAKE, FAKE, 1e-6, None, FAKE, None, None, FAKE, FAKE, FAKE,
-                         FAKE, FAKE, FAKE, 2, 100, 3, 64, 128, 64, 1, None, 0, None)
+                         FAKE, FAKE, FAKE, 2, 100, 3, 64, 128, 64, 1, 0, None, 0, None)
     assert st == WORKSPACE
     assert b"workspace" in L.kla_last_error()
     st = L.kla_chunk_bwd(FAKE, FAKE, FAKE, FAKE, FAKE, 1e-6, None, FAKE, None, None, FAKE, FAKE, FAKE,
-                         FAKE, FAKE, FAKE, 2, 100, 3, 64, 128, 64, 1, FAKE, need - 1, None)
+                         FAKE, FAKE, FAKE, 2, 100, 3, 64, 128, 64, 1, 0, FAKE, need - 1, None)
     assert st == WORKSPACE
 
 
 def test_bwd_requires_outputs(L):
     st = L.kla_chunk_bwd(FAKE, FAKE, FAKE, FAKE, FAKE, 1e-6, None, FAKE, None, None, None, FAKE, FAKE,
-                         FAKE, FAKE, FAKE, 1, 64, 1, 64, 64, 64, 1, FAKE, 1 << 30, None)
+                         FAKE, FAKE, FAKE, 1, 64, 1, 64, 64, 64, 1, 0, FAKE, 1 << 30, None)
     assert st == INVALID
 
 
 def test_decode_rejects_before_launch(L):
-    st = L.kla_decode_step(FAKE, FAKE, FAKE, FAKE, FAKE, 1e-6, FAKE, None, 4, 2, 128, 96, 1, None)
+    st = L.kla_decode_step(FAKE, FAKE, FAKE, FAKE, FAKE, 1e-6, FAKE, None, 4, 2, 128, 96, 1, 0, None)
     assert st == UNSUPPORTED
-    st = L.kla_decode_step(FAKE, FAKE, FAKE, FAKE, FAKE, 1e-6, None, None, 4, 2, 128, 128, 1, None)
+    st = L.kla_decode_step(FAKE, FAKE, FAKE, FAKE, FAKE, 1e-6, None, None, 4, 2, 128, 128, 1, 0, None)
     assert st == INVALID
-    st = L.kla_decode_step(FAKE, FAKE, FAKE, FAKE, FAKE, -0.5, FAKE, None, 4, 2, 128, 128, 1, None)
+    st = L.kla_decode_step(FAKE, FAKE, FAKE, FAKE, FAKE, -0.5, FAKE, None, 4, 2, 128, 128, 1, 0, None)
     assert st == INVALID
 
 

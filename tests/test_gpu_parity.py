@@ -294,6 +294,39 @@ def test_bwd_training_workload_sampled_heads(kla, oracle_mod):
         assert rel_err(got, ref[name]) <= 2e-2, name
 
 
+def test_bf16_outputs_are_rounded_fp32_outputs(kla):
+    """out_dtype=bf16 stores round the same fp32 results once (forward, decode, backward)."""
+    for Dk in (128, 64):
+        inp = small_inputs(2, 150, 2, Dk, Dk, "bf16", seed=Dk)
+        d = {k: v.cuda() for k, v in inp.items()}
+        o32, _ = kla.chunk_fwd(d["q"], d["k"], d["v"], d["eta"], d["g"], 1e-6, d["S0"])
+        o16, _ = kla.chunk_fwd(d["q"], d["k"], d["v"], d["eta"], d["g"], 1e-6, d["S0"], out_dtype=torch.bfloat16)
+        torch.cuda.synchronize()
+        assert o16.dtype == torch.bfloat16
+        assert torch.equal(o16, o32.to(torch.bfloat16))
+        S1, S2 = d["S0"].clone(), d["S0"].clone()
+        a32 = kla.decode_step(d["q"][:, 0], d["k"][:, 0], d["v"][:, 0], d["eta"][:, 0], d["g"][:, 0], S1, 1e-6)
+        a16 = kla.decode_step(d["q"][:, 0], d["k"][:, 0], d["v"][:, 0], d["eta"][:, 0], d["g"][:, 0], S2, 1e-6,
+                              out_dtype=torch.bfloat16)
+        torch.cuda.synchronize()
+        assert torch.equal(a16, a32.to(torch.bfloat16))
+        dO = torch.randn(2, 150, 2, Dk, device="cuda").to(torch.bfloat16)
+        g32 = kla.chunk_bwd(d["q"], d["k"], d["v"], d["eta"], d["g"], dO, 1e-6, d["S0"])
+        g16 = kla.chunk_bwd(d["q"], d["k"], d["v"], d["eta"], d["g"], dO, 1e-6, d["S0"], out_dtype=torch.bfloat16)
+        torch.cuda.synchronize()
+        for n in ("dq", "dk", "dv"):
+            # fp32 atomics may sum in a different order between the two calls: allow one bf16 ulp
+            ref = g32[n].to(torch.bfloat16).float()
+            assert torch.all((g16[n].float() - ref).abs() <= ref.abs() * 2.0 ** -7 + 1e-30), n
+
+
+def test_no_device_timeouts_recorded(kla):
+    inp = small_inputs(1, 300, 2, 128, 128, "bf16", seed=99)
+    d = {k: v.cuda() for k, v in inp.items()}
+    kla.chunk_fwd(d["q"], d["k"], d["v"], d["eta"], d["g"], 1e-6, d["S0"])
+    kla.check_device_error()
+
+
 def test_bwd_empty_sequence(kla):
     dST = torch.randn(1, 2, 64, 64, device="cuda")
     z = torch.zeros(1, 0, 2, 64, device="cuda")
