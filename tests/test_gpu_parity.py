@@ -204,7 +204,7 @@ def test_decode_workload_1024_steps_sampled_heads(kla, oracle_mod):
     S = inp["S0"].cuda().clone()
     qd, kd, vd = inp["q"].cuda(), inp["k"].cuda(), inp["v"].cuda()
     ed, gd = inp["eta"].cuda(), inp["g"].cuda()
-    outs = torch.empty(w.T, w.B, w.H, w.Dv, dtype=qd.dtype, device="cuda")
+    outs = torch.empty(w.T, w.B, w.H, w.Dv, dtype=torch.float32, device="cuda")
     for t in range(w.T):
         kla.decode_step(qd[t], kd[t], vd[t], ed[t], gd[t], S, w.eps, o=outs[t])
     torch.cuda.synchronize()
@@ -220,15 +220,17 @@ def test_decode_workload_1024_steps_sampled_heads(kla, oracle_mod):
     assert rel_err(gS, Sref) <= 2e-2
 
 
-def test_decode_equals_forward_T1(kla):
-    inp = small_inputs(2, 1, 3, 128, 128, "bf16", seed=21)
+@pytest.mark.parametrize("dtype,tol", [("f32", 1e-5), ("bf16", 2e-2)])
+def test_decode_equals_forward_T1(kla, dtype, tol):
+    inp = small_inputs(2, 1, 3, 128, 128, dtype, seed=21)
     d = {k: v.cuda() for k, v in inp.items()}
     o, ST = kla.chunk_fwd(d["q"], d["k"], d["v"], d["eta"], d["g"], 1e-6, d["S0"])
     S = d["S0"].clone()
-    od = kla.decode_step(d["q"][:, 0], d["k"][:, 0], d["v"][:, 0], d["eta"][:, 0], d["g"][:, 0], S, 1e-6)
+    c = lambda x: x[:, 0].contiguous()
+    od = kla.decode_step(c(d["q"]), c(d["k"]), c(d["v"]), c(d["eta"]), c(d["g"]), S, 1e-6)
     torch.cuda.synchronize()
-    assert rel_err(od, np64(o[:, 0])) <= 1e-2
-    assert rel_err(S, np64(ST)) <= 1e-5
+    assert rel_err(od, np64(o[:, 0])) <= tol
+    assert rel_err(S, np64(ST)) <= tol
 
 
 # ---------------------------------------------------------------------------------------
@@ -305,8 +307,9 @@ def test_bf16_outputs_are_rounded_fp32_outputs(kla):
         assert o16.dtype == torch.bfloat16
         assert torch.equal(o16, o32.to(torch.bfloat16))
         S1, S2 = d["S0"].clone(), d["S0"].clone()
-        a32 = kla.decode_step(d["q"][:, 0], d["k"][:, 0], d["v"][:, 0], d["eta"][:, 0], d["g"][:, 0], S1, 1e-6)
-        a16 = kla.decode_step(d["q"][:, 0], d["k"][:, 0], d["v"][:, 0], d["eta"][:, 0], d["g"][:, 0], S2, 1e-6,
+        c = lambda x: x[:, 0].contiguous()
+        a32 = kla.decode_step(c(d["q"]), c(d["k"]), c(d["v"]), c(d["eta"]), c(d["g"]), S1, 1e-6)
+        a16 = kla.decode_step(c(d["q"]), c(d["k"]), c(d["v"]), c(d["eta"]), c(d["g"]), S2, 1e-6,
                               out_dtype=torch.bfloat16)
         torch.cuda.synchronize()
         assert torch.equal(a16, a32.to(torch.bfloat16))
