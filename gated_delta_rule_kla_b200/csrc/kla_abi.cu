@@ -80,6 +80,13 @@ size_t bwd_ws_layout(int B, int T, int H, int Dk, int Dv, bool have_S_chunks, si
 
 }  // namespace
 
+namespace kla {
+int set_last_error(int status, const char* msg) {
+    g_last_error = msg;
+    return status;
+}
+}  // namespace kla
+
 extern "C" {
 
 const char* kla_status_string(int status) {

@@ -138,6 +138,35 @@ kla_status kla_decode_step(const void *q, const void *k, const void *v, const fl
  */
 kla_status kla_check_device_error(void *stream);
 
+/*
+ * kla_chunk_bwd_noalloc -- kla_chunk_bwd for callers that cannot allocate device memory.
+ * The paper has no counterpart; this entry point exists for deployment reasons only.
+ *
+ * kla_chunk_bwd needs a scratch workspace from the caller.  Some callers cannot allocate
+ * one: code recorded into a CUDA graph that must not allocate, plugins whose host framework
+ * owns all device memory, or latency-critical paths where cudaMalloc may block or
+ * synchronise.  This variant takes no workspace argument and uses a scratch array of
+ * KLA_NOALLOC_SCRATCH_BYTES compiled into libkla.so (every GPU that loads the library holds
+ * it until the process exits).  It calls no cudaMalloc, cudaFree or allocating routine;
+ * inputs and outputs are still the caller's, exactly as for kla_chunk_bwd, and the result is
+ * the same.
+ *   - Limit: calls whose kla_chunk_bwd_workspace() size exceeds KLA_NOALLOC_SCRATCH_BYTES are
+ *     rejected with KLA_ERR_WORKSPACE before anything is launched (about 16K token-heads at
+ *     Dk = Dv = 128 without S_chunks; passing S_chunks roughly doubles that).
+ *   - The first call on each device looks up the scratch array's device address (with that
+ *     device current); make that first call before any stream capture begins.
+ *   - All calls on a device share the one array and the library clears what must start at
+ *     zero on every call.  Calls that may overlap on the GPU (different streams, or host
+ *     threads without ordering) race on the shared scratch: serialise them.
+ */
+#define KLA_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+size_t kla_chunk_bwd_noalloc_scratch_bytes(void);
+kla_status kla_chunk_bwd_noalloc(const void *q, const void *k, const void *v, const float *eta,
+                                 const float *g, float eps, const float *S0, const void *dO,
+                                 const float *dS_T, const float *S_chunks, void *dq, void *dk,
+                                 void *dv, float *deta, float *dg, float *dS0, int B, int T, int H,
+                                 int Dk, int Dv, int chunk, int dtype, int out_dtype, void *stream);
+
 #ifdef __cplusplus
 }
 #endif
