@@ -284,16 +284,19 @@ def gpu_arm(args, rank, world, local_rank):
         achieved_tf = alg_flops / mean_s / 1e12
 
         extra = {}
-        if not args.skip_extra:
+        parts = set(args.parts.split(",")) if not args.skip_extra else set()
+        if "decode" in parts:
             extra["decode"] = bench_decode(kla, WORKLOADS, make_inputs, dev, stream, flush, rank, world,
                                            hbm_peak, args)
+        if "train" in parts:
             extra["train"] = bench_train(kla, WORKLOADS, make_inputs, dev, stream, flush, rank, world,
                                          hbm_peak, tc_peak, args)
+        if "long" in parts:
             extra["long_context"] = bench_long(kla, WORKLOADS, make_inputs, dev, stream, rank, world,
                                                hbm_peak, tc_peak, args)
 
     # ---------------- end-to-end through the public API with host buffers ----------------
-    e2e = bench_e2e(kla, w, inp, dev, stream, rank, world, args)
+    e2e = None if args.skip_e2e else bench_e2e(kla, w, inp, dev, stream, rank, world, args)
     clocks = sampler.summary()
 
     line = {
@@ -535,8 +538,11 @@ def parse(argv=None):
     ap.add_argument("--impl", choices=["kla", "reference"], default="kla")
     ap.add_argument("--workload", default="prefill_b8_t2048_h8_d128")
     ap.add_argument("--ref-pairs", type=int, default=8, help="(b,h) pairs per reference step")
-    ap.add_argument("--cpu-pairs", type=int, default=16, help="(b,h) pairs in the CPU baseline sample")
+    ap.add_argument("--cpu-pairs", type=int, default=64, help="(b,h) pairs in the CPU baseline sample")
     ap.add_argument("--skip-extra", action="store_true", help="headline prefill only")
+    ap.add_argument("--parts", default="decode,train,long",
+                    help="sub-measurements after the headline prefill (comma list of decode,train,long)")
+    ap.add_argument("--skip-e2e", action="store_true", help="omit the host-buffer end-to-end leg")
     ap.add_argument("--skip-cpu", action="store_true", help="omit the CPU baseline")
     ap.add_argument("--quick", action="store_true", help="fewer decode/train steps (smoke runs)")
     return ap.parse_args(argv)

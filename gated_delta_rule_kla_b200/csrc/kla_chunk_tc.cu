@@ -18,15 +18,16 @@
 //   U^T    V^T T''^T - S^T W^T  lane = dv, col = token     (T'' = T Diag(c))
 //   S     += Ktil^T U        lane = dk, col = dv           (Ktil = Diag(delta / r) K)
 //   PU     U^T P^T           lane = dv, col = token
+// T = (I + L)^{-1} itself is a 64x64 triangular inverse done on CUDA cores (blocked).
 // Operands that are computed on chip (P, T', T'', S, U, Ktil) are rounded to bf16 as a
 // hi + lo pair and multiplied term by term (the lo x lo term is dropped), which keeps ~16
 // significant bits; W enters as a single bf16.  q, k, v are bf16 inputs and exact.
 //
-// The fp32 master state lives in TMEM (lane = dk, 128 columns): each chunk scales it by
-// gamma_last and the Ktil^T U MMA accumulates onto it; a bf16 hi/lo copy in shared memory
-// is the MMA operand.  One CTA of 128 threads (thread t <-> TMEM lane t) per (b, h); the
-// chunk loop is sequential, with the next chunk's tiles prefetched by TMA into the other
-// stage.  Every
+// The fp32 master state lives in TMEM (lane = dk, 128 columns): it is kept pre-scaled by the
+// coming chunk's gamma_last, and the Ktil^T U MMA accumulates onto it; a bf16 hi/lo copy in
+// shared memory is the MMA operand.  One CTA of 256 threads per (b, h): warps w and w + 4
+// share TMEM lanes 32 (w % 4) .. + 31 and split the columns of every epilogue.  The chunk loop
+// is sequential, with the next chunk's tiles prefetched by TMA into the other stage.  Every
 // wait is bounded: on timeout the kernel records an error word and returns after freeing
 // TMEM.
 #include <cuda.h>
@@ -44,7 +45,8 @@ namespace {
 using namespace sm100;
 
 constexpr int DK = 128, DV = 128, CH = 64;
-constexpr int NTHREADS = 128;
+constexpr int NTHREADS = 256;
+constexpr int kIssuer = 128;  // thread that issues the MMAs (warp 4: idle during the scalar prep)
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 
 // shared-memory map (offsets from a 1024-aligned base)
@@ -58,7 +60,7 @@ constexpr uint32_t OFF_P = 163840;      // 16 KB: P hi [64 x 64], P lo
 constexpr uint32_t OFF_Z = 180224;      // 32 KB: L/T fp32 -> T' T'' hi/lo -> Ktil hi/lo
 constexpr uint32_t OFF_MISC = 212992;   // barriers, TMEM slot, per-token scalars
 constexpr uint32_t SMEM_BYTES = OFF_MISC + 4096 + 1024;  // + alignment slack
-constexpr int LDL = 65;                 // row stride of the fp32 solve buffer
+constexpr int LDL = 68;                 // row stride (floats) of the fp32 L/T buffer, 16-B rows
 
 // TMEM columns
 constexpr uint32_t TM_G = 0, TM_SQ = 64, TM_W = 128, TM_U = 192, TM_S = 256, TM_PU = 384;
@@ -69,55 +71,83 @@ struct Misc {
     uint32_t tmem_base;
     uint32_t pad;
     float G[CH], gam[CH], del[CH], bco[CH], cco[CH], invr[CH], graw[CH], eta[CH];
+    float gsum[2];  // per-warp sums of the next chunk's log-decays
 };
 
 __device__ __forceinline__ size_t tok_index(int b, int t, int h, int T, int H) {
     return ((size_t)b * T + t) * H + h;
 }
 
-// In-place inverse of the unit lower-triangular 64x64 matrix I + L (L strictly lower,
-// fp32, row stride LDL).  Diagonal 16x16 blocks by forward substitution (one warp per
-// block, one lane per column), then block rows I = 1..3:
-//   T_IJ = -T_II sum_{K=J}^{I-1} L_IK T_KJ.
-// X is scratch for 3 * 256 floats.  Must be called by all 128 threads.
-__device__ __forceinline__ void invert_unit_lower64(float* Lf, float* X, int tid) {
-    const int warp = tid >> 5, lane = tid & 31;
-    {
-        const int base = 16 * warp;
+// Off-diagonal 16x16 block (I, J), I > J, of T in the Toff buffer: blocks ordered by
+// distance d = I - J, then by J: (1,0) (2,1) (3,2) (2,0) (3,1) (3,0).
+__device__ __forceinline__ int toff_block(int I, int J) {
+    const int d = I - J;
+    return (d == 1 ? 0 : (d == 2 ? 3 : 5)) + J;
+}
+
+// T = (I + L)^{-1} of the unit lower-triangular 64x64 matrix of Eq. (7), by blockwise
+// forward substitution (Appendix B.2) on 16x16 blocks.  L: fp32, rows of LDL floats,
+// strictly lower (upper part zero).
+//   diagonal blocks  D_I = (I + L_II)^{-1}: column by column (64 threads), written over L_II
+//   off-diagonal     T_IJ = -D_I sum_{K=J}^{I-1} L_IK T_KJ (T_JJ = D_J), by distance
+//                    d = I - J = 1, 2, 3, into Toff (6 blocks of 16x16); L stays intact.
+// X is scratch for 3 x 256 floats.  All NTHREADS threads must call it.
+__device__ __forceinline__ void invert_unit_lower64(float* Lf, float* Toff, float* X, int tid) {
+    if (tid < 64) {
+        const int base = 16 * (tid >> 4), l = tid & 15;
         float x[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-            float acc = 0.f;
+            float a0 = 0.f, a1 = 0.f;
 #pragma unroll
-            for (int j = 0; j < i; ++j) acc = fmaf(Lf[(base + i) * LDL + base + j], x[j], acc);
-            x[i] = (i < lane) ? 0.f : ((i == lane) ? 1.f : -acc);
+            for (int j = 0; j + 1 < i; j += 2) {
+                a0 = fmaf(Lf[(base + i) * LDL + base + j], x[j], a0);
+                a1 = fmaf(Lf[(base + i) * LDL + base + j + 1], x[j + 1], a1);
+            }
+            if (i & 1) a0 = fmaf(Lf[(base + i) * LDL + base + i - 1], x[i - 1], a0);
+            x[i] = (i < l) ? 0.f : ((i == l) ? 1.f : -(a0 + a1));
         }
         __syncwarp();
-        if (lane < 16) {
 #pragma unroll
-            for (int i = 0; i < 16; ++i) Lf[(base + i) * LDL + base + lane] = x[i];
-        }
+        for (int i = 0; i < 16; ++i) Lf[(base + i) * LDL + base + l] = x[i];
     }
     __syncthreads();
-    for (int I = 1; I < 4; ++I) {
-        for (int e = tid; e < I * 256; e += NTHREADS) {
-            const int J = e >> 8, r = (e >> 4) & 15, cc = e & 15;
-            float acc = 0.f;
+#pragma unroll 1
+    for (int d = 1; d < 4; ++d) {
+        const int njobs = 64 * (4 - d);  // (block, row, column quad)
+        for (int job = tid; job < njobs; job += NTHREADS) {
+            const int J = job >> 6, I = J + d, r = (job >> 2) & 15, cq = job & 3;
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
             for (int K = J; K < I; ++K) {
+                const float* tk = (K == J) ? (Lf + 16 * J * LDL + 16 * J) : (Toff + toff_block(K, J) * 256);
+                const int ldt = (K == J) ? LDL : 16;
 #pragma unroll
-                for (int m = 0; m < 16; ++m)
-                    acc = fmaf(Lf[(16 * I + r) * LDL + 16 * K + m], Lf[(16 * K + m) * LDL + 16 * J + cc], acc);
+                for (int m = 0; m < 16; ++m) {
+                    const float l = Lf[(16 * I + r) * LDL + 16 * K + m];
+                    const float4 t = *reinterpret_cast<const float4*>(tk + m * ldt + 4 * cq);
+                    acc.x = fmaf(l, t.x, acc.x);
+                    acc.y = fmaf(l, t.y, acc.y);
+                    acc.z = fmaf(l, t.z, acc.z);
+                    acc.w = fmaf(l, t.w, acc.w);
+                }
             }
-            X[e] = acc;
+            *reinterpret_cast<float4*>(X + job * 4) = acc;
         }
         __syncthreads();
-        for (int e = tid; e < I * 256; e += NTHREADS) {
-            const int J = e >> 8, r = (e >> 4) & 15, cc = e & 15;
-            float acc = 0.f;
+        for (int job = tid; job < njobs; job += NTHREADS) {
+            const int J = job >> 6, I = J + d, r = (job >> 2) & 15, cq = job & 3;
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-            for (int m = 0; m < 16; ++m)
-                acc = fmaf(Lf[(16 * I + r) * LDL + 16 * I + m], X[(J << 8) + (m << 4) + cc], acc);
-            Lf[(16 * I + r) * LDL + 16 * J + cc] = -acc;
+            for (int m = 0; m < 16; ++m) {
+                const float l = Lf[(16 * I + r) * LDL + 16 * I + m];  // D_I
+                const float4 x = *reinterpret_cast<const float4*>(X + ((J << 6) + (m << 2) + cq) * 4);
+                acc.x = fmaf(l, x.x, acc.x);
+                acc.y = fmaf(l, x.y, acc.y);
+                acc.z = fmaf(l, x.z, acc.z);
+                acc.w = fmaf(l, x.w, acc.w);
+            }
+            *reinterpret_cast<float4*>(Toff + toff_block(I, J) * 256 + r * 16 + 4 * cq) =
+                make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
         }
         __syncthreads();
     }
@@ -125,6 +155,7 @@ __device__ __forceinline__ void invert_unit_lower64(float* Lf, float* X, int tid
 
 // Write chunks [c0, c0 + n) of row r of a swizzled bf16 block from 8*n fp32 values.
 __device__ __forceinline__ void st_chunks_bf16(uint8_t* block, int r, int c0, int n, const float* v) {
+#pragma unroll
     for (int c = 0; c < n; ++c) {
         uint4 u;
         u.x = pack_bf16x2(v[8 * c + 0], v[8 * c + 1]);
@@ -138,6 +169,7 @@ __device__ __forceinline__ void st_chunks_bf16(uint8_t* block, int r, int c0, in
 // Split 8*n fp32 values into hi/lo bf16 and write chunks [c0, c0 + n) of row r of two blocks.
 __device__ __forceinline__ void st_chunks_split(uint8_t* hi_block, uint8_t* lo_block, int r, int c0, int n,
                                                 const float* v) {
+#pragma unroll
     for (int c = 0; c < n; ++c) {
         float h[8], l[8];
 #pragma unroll
@@ -159,10 +191,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     Misc* ms = reinterpret_cast<Misc*>(sm + OFF_MISC);
-    float* Lf = reinterpret_cast<float*>(sm + OFF_Z);
-    float* Xs = Lf + 64 * LDL;
+    float* Lf = reinterpret_cast<float*>(sm + OFF_Z);  // 64 x LDL fp32
+    float* Toff = Lf + 64 * LDL;                          // 6 x 256 fp32
+    float* Xs = Toff + 6 * 256;                           // 3 x 256 fp32
 
     const int tid = threadIdx.x, warp = tid >> 5;
+    const int row = tid & 127;  // TMEM lane owned with the other thread of the pair
+    const int ch = tid >> 7;    // which half of an epilogue's columns this thread takes
     const int H = a.H, T = a.T;
     const int b = blockIdx.x / H, h = blockIdx.x % H;
     const int NC = (T + CH - 1) / CH;
@@ -184,31 +219,56 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         tmem_alloc(smem_u32(&ms->tmem_base), 512);
         tmem_relinquish();
     }
-
-    // fp32 master state: thread t owns row dk = t, kept in TMEM columns [TM_S, TM_S + 128)
+    // log-decays of chunk 0 (threads 0-63); their sum gives gamma_last of chunk 0
+    float g_next = 0.f, eta_next = 0.f;
+    if (tid < CH && tid < T) {
+        const size_t ti = tok_index(b, tid, h, T, H);
+        g_next = a.g[ti];
+        eta_next = a.eta[ti];
+    }
+    if (warp < 2) {
+        const float sg = warp_sum((tid < T) ? g_next : 0.f);
+        if ((tid & 31) == 0) ms->gsum[warp] = sg;
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = ms->tmem_base;
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+
+    // Initial state: this thread holds row dk = `row`, columns [64 ch, 64 ch + 64).
+    {
+        const float g0 = (NC > 0) ? __expf(ms->gsum[0] + ms->gsum[1]) : 1.f;
+        float4* sc0 = (a.S_chunks && NC > 0)
+                          ? reinterpret_cast<float4*>(a.S_chunks + (size_t)blockIdx.x * NC * DK * DV +
+                                                      (size_t)row * DV + 64 * ch)
+                          : nullptr;
 #pragma unroll 1
-    for (int q4 = 0; q4 < 4; ++q4) {
-        float x[32];
-        if (a.S0) {
-            const float4* src = reinterpret_cast<const float4*>(a.S0 + state_off + (size_t)tid * DV + 32 * q4);
+        for (int q2 = 0; q2 < 2; ++q2) {
+            float x[32];
+            if (a.S0) {
+                const float4* src =
+                    reinterpret_cast<const float4*>(a.S0 + state_off + (size_t)row * DV + 64 * ch + 32 * q2);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const float4 v4 = src[i];
-                x[4 * i] = v4.x; x[4 * i + 1] = v4.y; x[4 * i + 2] = v4.z; x[4 * i + 3] = v4.w;
+                for (int i = 0; i < 8; ++i) {
+                    const float4 v4 = src[i];
+                    x[4 * i] = v4.x; x[4 * i + 1] = v4.y; x[4 * i + 2] = v4.z; x[4 * i + 3] = v4.w;
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) x[i] = 0.f;
             }
-        } else {
+            if (sc0) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) x[i] = 0.f;
+                for (int i = 0; i < 8; ++i) sc0[8 * q2 + i] = make_float4(x[4 * i], x[4 * i + 1], x[4 * i + 2], x[4 * i + 3]);
+            }
+            st_chunks_split(sm + OFF_SHI + ch * 16384, sm + OFF_SLO + ch * 16384, row, 4 * q2, 4, x);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) x[i] *= g0;
+            tmem_st32(tmem + lane_base + TM_S + 64 * ch + 32 * q2, x);
         }
-        tmem_st32(tmem + lane_base + TM_S + 32 * q4, x);
-        st_chunks_split(sm + OFF_SHI + (q4 >> 1) * 16384, sm + OFF_SLO + (q4 >> 1) * 16384, tid, 4 * (q4 & 1), 4, x);
+        tmem_st_wait();
     }
-    tmem_st_wait();
     fence_proxy_async();
     tc_fence_before();
     __syncthreads();
@@ -227,19 +287,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         tma_load_4d(vv, &tm_v, bar, 0, h, t0, b);
         tma_load_4d(vv + 8192, &tm_v, bar, 64, h, t0, b);
     };
-
     if (tid == 0 && NC > 0) issue_loads(0, 0);
-    float g_next = 0.f, eta_next = 0.f;
-    if (tid < CH && tid < T) {
-        const size_t ti = tok_index(b, tid, h, T, H);
-        g_next = a.g[ti];
-        eta_next = a.eta[ti];
-    }
 
     uint32_t mma_phase = 0;
     bool aborted = false;
     int issued = (NC > 0) ? 0 : -1;  // last chunk whose tiles were requested
     int landed = -1;                 // last chunk whose tiles were waited for
+
+    // Bounded wait on the MMA barrier shared by the whole CTA; false = give up.
+    auto wait_mma = [&]() -> bool {
+        const bool ok = mbar_wait_bounded(bar_mma, mma_phase, kWaitLimitNs);
+        mma_phase ^= 1;
+        return !__syncthreads_or(!ok);
+    };
 
     for (int c = 0; c < NC; ++c) {
         const int st = c & 1;
@@ -265,8 +325,30 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (__syncthreads_or(!ok_tma)) { aborted = true; break; }
         landed = c;
 
+        // ---- MMA: Gram = [Q; K] K^T and SQ = S^T Q^T (the scalar prep below overlaps them)
+        if (tid == kIssuer) {
+            tc_fence_after();
+            const uint32_t ig = idesc_bf16(128, 64, false, false);
+#pragma unroll
+            for (int s = 0; s < 8; ++s) {
+                const uint32_t off = (s >> 2) * 16384 + (s & 3) * 32;
+                mma_bf16(tmem + TM_G, smem_desc(qk_a + off, 16, 1024), smem_desc(qk_a + off + 8192, 16, 1024),
+                         ig, s > 0);
+            }
+            const uint32_t isq = idesc_bf16(128, 64, true, false);
+#pragma unroll
+            for (int part = 0; part < 2; ++part) {
+                const uint32_t sa = sbase + (part ? OFF_SLO : OFF_SHI);
+#pragma unroll
+                for (int s = 0; s < 8; ++s)
+                    mma_bf16(tmem + TM_SQ, smem_desc(sa + s * 2048, 16384, 1024),
+                             smem_desc(qk_a + (s >> 2) * 16384 + (s & 3) * 32, 16, 1024), isq, (part | s) > 0);
+            }
+            mma_commit(bar_mma);
+        }
+
         // key norms and Kaczmarz coefficients (thread 64 + j reads key row j)
-        if (tid >= CH) {
+        if (tid >= CH && tid < 2 * CH) {
             const int j = tid - CH;
             float r2 = 0.f;
 #pragma unroll
@@ -301,101 +383,72 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             ms->gam[tid] = __expf(ms->G[tid]);
             ms->del[tid] = __expf(ms->G[n - 1] - ms->G[tid]);
         }
-
-        // ---- MMA: Gram = [Q; K] K^T and SQ = S^T Q^T
-        if (tid == 0) {
-            tc_fence_after();
-            const uint32_t ig = idesc_bf16(128, 64, false, false);
-#pragma unroll
-            for (int s = 0; s < 8; ++s) {
-                const uint32_t off = (s >> 2) * 16384 + (s & 3) * 32;
-                mma_bf16(tmem + TM_G, smem_desc(qk_a + off, 16, 1024), smem_desc(qk_a + off + 8192, 16, 1024),
-                         ig, s > 0);
-            }
-            const uint32_t isq = idesc_bf16(128, 64, true, false);
-#pragma unroll
-            for (int part = 0; part < 2; ++part) {
-                const uint32_t sa = sbase + (part ? OFF_SLO : OFF_SHI);
-#pragma unroll
-                for (int s = 0; s < 8; ++s)
-                    mma_bf16(tmem + TM_SQ, smem_desc(sa + s * 2048, 16384, 1024),
-                             smem_desc(qk_a + (s >> 2) * 16384 + (s & 3) * 32, 16, 1024), isq, (part | s) > 0);
-            }
-            mma_commit(bar_mma);
-        }
-        if (a.S_chunks) {
-            float4* dst = reinterpret_cast<float4*>(a.S_chunks + ((size_t)blockIdx.x * NC + c) * DK * DV +
-                                                    (size_t)tid * DV);
-#pragma unroll 1
-            for (int q4 = 0; q4 < 4; ++q4) {
-                float x[32];
-                tmem_ld32(tmem + lane_base + TM_S + 32 * q4, x);
-                tmem_ld_wait();
-#pragma unroll
-                for (int i = 0; i < 8; ++i) dst[8 * q4 + i] = make_float4(x[4 * i], x[4 * i + 1], x[4 * i + 2], x[4 * i + 3]);
-            }
-        }
-        {
-            const bool ok = mbar_wait_bounded(bar_mma, mma_phase, kWaitLimitNs);
-            mma_phase ^= 1;
-            if (__syncthreads_or(!ok)) { aborted = true; break; }
-        }
+        if (!wait_mma()) { aborted = true; break; }
         tc_fence_after();
 
-        // ---- Gram epilogue: P (rows 0-63, hi/lo bf16) and L (rows 64-127, fp32), 32 columns at a time
-#pragma unroll 1
-        for (int half = 0; half < 2; ++half) {
+        // ---- Gram epilogue: P (rows 0-63, hi/lo bf16) and L (rows 64-127, fp32); 32 columns each
+        {
             float x[32];
-            tmem_ld32(tmem + lane_base + TM_G + 32 * half, x);
+            tmem_ld32(tmem + lane_base + TM_G + 32 * ch, x);
             tmem_ld_wait();
-            if (tid < CH) {
-                const int i = tid;
+            if (row < CH) {
+                const int i = row;
                 const float Gi = ms->G[i];
 #pragma unroll
                 for (int e = 0; e < 32; ++e) {
-                    const int j = 32 * half + e;
+                    const int j = 32 * ch + e;
                     x[e] = (j <= i) ? __expf(Gi - ms->G[j]) * x[e] * ms->invr[j] : 0.f;
                 }
-                st_chunks_split(sm + OFF_P, sm + OFF_P + 8192, i, 4 * half, 4, x);
+                st_chunks_split(sm + OFF_P, sm + OFF_P + 8192, i, 4 * ch, 4, x);
             } else {
-                const int i = tid - CH;
+                const int i = row - CH;
                 const float Gi = ms->G[i];
                 const float bi = ms->bco[i] * ms->invr[i];
 #pragma unroll
                 for (int e = 0; e < 32; ++e) {
-                    const int j = 32 * half + e;
-                    Lf[i * LDL + j] = (j < i) ? bi * __expf(Gi - ms->G[j]) * x[e] * ms->invr[j] : 0.f;
+                    const int j = 32 * ch + e;
+                    x[e] = (j < i) ? bi * __expf(Gi - ms->G[j]) * x[e] * ms->invr[j] : 0.f;
                 }
+                float4* lrow = reinterpret_cast<float4*>(Lf + i * LDL + 32 * ch);
+#pragma unroll
+                for (int q = 0; q < 8; ++q) lrow[q] = make_float4(x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]);
             }
         }
         tc_fence_before();
         __syncthreads();
-        invert_unit_lower64(Lf, Xs, tid);
-        // T' = T Diag(b gamma / r), T'' = T Diag(c): thread -> row tid/2, 32 columns
+        invert_unit_lower64(Lf, Toff, Xs, tid);
+        // ---- T' = T Diag(b gamma / r), T'' = T Diag(c): thread -> row tid/4, 16 columns
         {
-            const int i = tid >> 1, half = tid & 1;
-            float tv[32];
+            const int i = tid >> 2, qq = tid & 3, I = i >> 4;
+            float tv[16];
+            if (qq <= I) {  // block (I, qq): D_I on the diagonal, Toff below, zero above
+                const float* src = (qq == I) ? (Lf + i * LDL + 16 * qq) : (Toff + toff_block(I, qq) * 256 + (i & 15) * 16);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) tv[e] = Lf[i * LDL + 32 * half + e];
-            __syncthreads();
-            float hi[32], lo[32];
+                for (int q = 0; q < 4; ++q) {
+                    const float4 t4 = *reinterpret_cast<const float4*>(src + 4 * q);
+                    tv[4 * q] = t4.x; tv[4 * q + 1] = t4.y; tv[4 * q + 2] = t4.z; tv[4 * q + 3] = t4.w;
+                }
+            } else {
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-                const int j = 32 * half + e;
-                split_bf16(tv[e] * (ms->bco[j] * ms->gam[j] * ms->invr[j]), hi[e], lo[e]);
+                for (int e = 0; e < 16; ++e) tv[e] = 0.f;
             }
-            st_chunks_bf16(sm + OFF_Z, i, 4 * half, 4, hi);
-            st_chunks_bf16(sm + OFF_Z + 8192, i, 4 * half, 4, lo);
+            __syncthreads();  // T is read; the tiles below overwrite it
+            float v[16];
 #pragma unroll
-            for (int e = 0; e < 32; ++e) split_bf16(tv[e] * ms->cco[32 * half + e], hi[e], lo[e]);
-            st_chunks_bf16(sm + OFF_Z + 16384, i, 4 * half, 4, hi);
-            st_chunks_bf16(sm + OFF_Z + 24576, i, 4 * half, 4, lo);
+            for (int e = 0; e < 16; ++e) {
+                const int j = 16 * qq + e;
+                v[e] = tv[e] * (ms->bco[j] * ms->gam[j] * ms->invr[j]);
+            }
+            st_chunks_split(sm + OFF_Z, sm + OFF_Z + 8192, i, 2 * qq, 2, v);
+#pragma unroll
+            for (int e = 0; e < 16; ++e) v[e] = tv[e] * ms->cco[16 * qq + e];
+            st_chunks_split(sm + OFF_Z + 16384, sm + OFF_Z + 24576, i, 2 * qq, 2, v);
         }
         fence_proxy_async();
         __syncthreads();
 
         // ---- MMA: W^T = K^T T'^T and U'^T = V^T T''^T
-        if (tid == 0) {
+        if (tid == kIssuer) {
             tc_fence_after();
             const uint32_t iw = idesc_bf16(128, 64, true, false);
 #pragma unroll
@@ -413,38 +466,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                              (part | s) > 0);
             mma_commit(bar_mma);
         }
-        {
-            const bool ok = mbar_wait_bounded(bar_mma, mma_phase, kWaitLimitNs);
-            mma_phase ^= 1;
-            if (__syncthreads_or(!ok)) { aborted = true; break; }
-        }
+        if (!wait_mma()) { aborted = true; break; }
         tc_fence_after();
         // ---- W^T to bf16 (over the consumed V stage); Ktil = Diag(delta / r) K hi/lo (over T tiles)
         {
-#pragma unroll 1
-            for (int half = 0; half < 2; ++half) {
-                float x[32];
-                tmem_ld32(tmem + lane_base + TM_W + 32 * half, x);
-                tmem_ld_wait();
-                st_chunks_bf16(vt, tid, 4 * half, 4, x);
-            }
-            {  // S <- gamma_last S, ahead of the MMA that accumulates Ktil^T U onto it
-                const float gC = ms->gam[n - 1];
-#pragma unroll 1
-                for (int q4 = 0; q4 < 4; ++q4) {
-                    float x[32];
-                    tmem_ld32(tmem + lane_base + TM_S + 32 * q4, x);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) x[e] *= gC;
-                    tmem_st32(tmem + lane_base + TM_S + 32 * q4, x);
-                }
-                tmem_st_wait();
-            }
-            const int j = tid >> 1, blk = tid & 1;
+            float x[32];
+            tmem_ld32(tmem + lane_base + TM_W + 32 * ch, x);
+            tmem_ld_wait();
+            st_chunks_bf16(vt, row, 4 * ch, 4, x);
+            const int j = tid >> 2, blk = (tid >> 1) & 1, c0 = 4 * (tid & 1);
             const float sc = ms->del[j] * ms->invr[j];
 #pragma unroll
-            for (int cc = 0; cc < 8; ++cc) {
+            for (int cc = c0; cc < c0 + 4; ++cc) {
                 float f[8], hi[8], lo[8];
                 const uint32_t off = (uint32_t)(j * 128 + cc * 16);  // same swizzle phase: (64 + j) & 7 == j & 7
                 unpack_bf16x8(*reinterpret_cast<const uint4*>(qk + blk * 16384 + 8192 + off), f);
@@ -464,7 +497,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         __syncthreads();
 
         // ---- MMA: U^T -= S^T W^T
-        if (tid == 0) {
+        if (tid == kIssuer) {
             tc_fence_after();
             const uint32_t isw = idesc_bf16(128, 64, true, true, true);
 #pragma unroll
@@ -477,26 +510,26 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             }
             mma_commit(bar_mma);
         }
-        {
-            const bool ok = mbar_wait_bounded(bar_mma, mma_phase, kWaitLimitNs);
-            mma_phase ^= 1;
-            if (__syncthreads_or(!ok)) { aborted = true; break; }
-        }
+        if (!wait_mma()) { aborted = true; break; }
         tc_fence_after();
-        // ---- U^T hi/lo to bf16 over the consumed [Q; K] stage (thread = dv row)
-#pragma unroll 1
-        for (int half = 0; half < 2; ++half) {
+        // ---- U^T hi/lo to bf16 over the consumed [Q; K] stage (thread pair = dv row)
+        {
             float x[32];
-            tmem_ld32(tmem + lane_base + TM_U + 32 * half, x);
+            tmem_ld32(tmem + lane_base + TM_U + 32 * ch, x);
             tmem_ld_wait();
-            st_chunks_split(qk, qk + 16384, tid, 4 * half, 4, x);
+            st_chunks_split(qk, qk + 16384, row, 4 * ch, 4, x);
+        }
+        if (warp < 2) {  // sum of the next chunk's log-decays (loaded at the top of this chunk)
+            const bool valid = (c + 1 < NC) && ((c + 1) * CH + tid < T);
+            const float sg = warp_sum(valid ? g_next : 0.f);
+            if ((tid & 31) == 0) ms->gsum[warp] = sg;
         }
         tc_fence_before();
         fence_proxy_async();
         __syncthreads();
 
         // ---- MMA: S += Ktil^T U (N = 128) and PU = U^T P^T
-        if (tid == 0) {
+        if (tid == kIssuer) {
             tc_fence_after();
             const uint32_t ids = idesc_bf16(128, 128, true, false);
             const uint32_t ipu = idesc_bf16(128, 64, false, false);
@@ -519,37 +552,46 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                              smem_desc(pb[p] + s * 32, 16, 1024), ipu, (p | s) > 0);
             mma_commit(bar_mma);
         }
-        {
-            const bool ok = mbar_wait_bounded(bar_mma, mma_phase, kWaitLimitNs);
-            mma_phase ^= 1;
-            if (__syncthreads_or(!ok)) { aborted = true; break; }
-        }
+        if (!wait_mma()) { aborted = true; break; }
         tc_fence_after();
-        // ---- new state to bf16 hi/lo (thread = dk row) and outputs (thread = dv)
+        // ---- new state to bf16 hi/lo (thread pair = dk row) and outputs (thread pair = dv);
+        // TMEM keeps gamma_last(next chunk) * S for the next chunk's accumulation
         {
+            const bool has_next = c + 1 < NC;
+            const float gN = has_next ? __expf(ms->gsum[0] + ms->gsum[1]) : 1.f;
+            float4* scn = (a.S_chunks && has_next)
+                              ? reinterpret_cast<float4*>(a.S_chunks + ((size_t)blockIdx.x * NC + c + 1) * DK * DV +
+                                                          (size_t)row * DV + 64 * ch)
+                              : nullptr;
 #pragma unroll 1
-            for (int q4 = 0; q4 < 4; ++q4) {
+            for (int q2 = 0; q2 < 2; ++q2) {
                 float x[32];
-                tmem_ld32(tmem + lane_base + TM_S + 32 * q4, x);
+                tmem_ld32(tmem + lane_base + TM_S + 64 * ch + 32 * q2, x);
                 tmem_ld_wait();
-                st_chunks_split(sm + OFF_SHI + (q4 >> 1) * 16384, sm + OFF_SLO + (q4 >> 1) * 16384, tid,
-                                4 * (q4 & 1), 4, x);
+                st_chunks_split(sm + OFF_SHI + ch * 16384, sm + OFF_SLO + ch * 16384, row, 4 * q2, 4, x);
+                if (scn) {
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        scn[8 * q2 + i] = make_float4(x[4 * i], x[4 * i + 1], x[4 * i + 2], x[4 * i + 3]);
+                }
+                if (has_next) {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) x[e] *= gN;
+                    tmem_st32(tmem + lane_base + TM_S + 64 * ch + 32 * q2, x);
+                }
             }
+            if (has_next) tmem_st_wait();
             if (a.o != nullptr) {
                 TOut* o = static_cast<TOut*>(a.o);
+                float sq[32], pu[32];
+                tmem_ld32(tmem + lane_base + TM_SQ + 32 * ch, sq);
+                tmem_ld32(tmem + lane_base + TM_PU + 32 * ch, pu);
+                tmem_ld_wait();
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    float sq[32], pu[32];
-                    tmem_ld32(tmem + lane_base + TM_SQ + 32 * half, sq);
-                    tmem_ld32(tmem + lane_base + TM_PU + 32 * half, pu);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const int i = 32 * half + e;
-                        if (i < n)
-                            o[tok_index(b, t0 + i, h, T, H) * DV + tid] =
-                                from_f32<TOut>(fmaf(ms->gam[i], sq[e], pu[e]));
-                    }
+                for (int e = 0; e < 32; ++e) {
+                    const int i = 32 * ch + e;
+                    if (i < n)
+                        o[tok_index(b, t0 + i, h, T, H) * DV + row] = from_f32<TOut>(fmaf(ms->gam[i], sq[e], pu[e]));
                 }
             }
         }
@@ -564,14 +606,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         for (int cc = landed + 1; cc <= issued; ++cc)
             (void)mbar_wait_bounded(bar_full0 + 8 * (cc & 1), (cc >> 1) & 1, kWaitLimitNs);
     } else if (a.S_T) {
-        float4* dst = reinterpret_cast<float4*>(a.S_T + state_off + (size_t)tid * DV);
+        float4* dst = reinterpret_cast<float4*>(a.S_T + state_off + (size_t)row * DV + 64 * ch);
 #pragma unroll 1
-        for (int q4 = 0; q4 < 4; ++q4) {
+        for (int q2 = 0; q2 < 2; ++q2) {
             float x[32];
-            tmem_ld32(tmem + lane_base + TM_S + 32 * q4, x);
+            tmem_ld32(tmem + lane_base + TM_S + 64 * ch + 32 * q2, x);
             tmem_ld_wait();
 #pragma unroll
-            for (int i = 0; i < 8; ++i) dst[8 * q4 + i] = make_float4(x[4 * i], x[4 * i + 1], x[4 * i + 2], x[4 * i + 3]);
+            for (int i = 0; i < 8; ++i) dst[8 * q2 + i] = make_float4(x[4 * i], x[4 * i + 1], x[4 * i + 2], x[4 * i + 3]);
         }
     }
     tc_fence_before();
