@@ -44,19 +44,19 @@ def fwd_flops_per_token_head(d, C=64):
     return 10 * C * d + 6 * d * d + (2.0 / 3.0) * C * C
 
 
-def fwd_bytes(B, T, H, Dk, Dv, elt, s0, s_out=True):
-    per_tok = (2 * Dk + Dv) * elt + Dv * elt + 8  # q, k, v in; o out; eta, g
+def fwd_bytes(B, T, H, Dk, Dv, elt, s0, s_out=True, out_elt=4):
+    per_tok = (2 * Dk + Dv) * elt + Dv * out_elt + 8  # q, k, v in; o out (fp32); eta, g
     state = B * H * Dk * Dv * 4 * ((1 if s0 else 0) + (1 if s_out else 0))
     return B * T * H * per_tok + state
 
 
-def decode_bytes(B, H, Dk, Dv, elt):
-    return B * H * (2 * Dk * Dv * 4 + (2 * Dk + 2 * Dv) * elt + 8)
+def decode_bytes(B, H, Dk, Dv, elt, out_elt=4):
+    return B * H * (2 * Dk * Dv * 4 + (2 * Dk + Dv) * elt + Dv * out_elt + 8)
 
 
-def bwd_bytes(B, T, H, Dk, Dv, elt):
-    # reads q, k, v, dO, eta, g; writes dq, dk, dv, deta, dg; plus the dS0 write
-    per_tok = (2 * Dk + Dv) * elt + Dv * elt + 8 + (2 * Dk + Dv) * elt + 8
+def bwd_bytes(B, T, H, Dk, Dv, elt, out_elt=4):
+    # reads q, k, v, dO, eta, g; writes dq, dk, dv (fp32), deta, dg; plus the dS0 write
+    per_tok = (2 * Dk + Dv) * elt + Dv * elt + 8 + (2 * Dk + Dv) * out_elt + 8
     return B * T * H * per_tok + B * H * Dk * Dv * 4
 
 
@@ -207,20 +207,18 @@ def barrier(world):
 # GPU arm
 # ---------------------------------------------------------------------------------------
 class Flusher:
-    """Evicts L2 between timed steps: writes one buffer larger than L2, then reads another,
-    so the next timed kernel starts with a cold, clean L2 (no dirty lines to write back)."""
+    """Evicts L2 between timed steps by writing a buffer larger than L2.  The timed kernel then
+    starts with no useful line in L2 and an L2 full of dirty lines, so the write-backs its own
+    traffic forces are paid inside its timing (as in a loop over many layers' states)."""
 
     def __init__(self, dev):
         import torch
-        n = L2_FLUSH_BYTES // 4
-        self.a = torch.empty(n, dtype=torch.float32, device=dev)
-        self.b = torch.ones(n, dtype=torch.float32, device=dev)
-        self.sink = torch.empty(1, dtype=torch.float32, device=dev)
+        self.a = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+        self.k = 0
 
     def __call__(self):
-        import torch
-        self.a.fill_(1.0)
-        torch.sum(self.b, dim=0, keepdim=True, out=self.sink)
+        self.k += 1
+        self.a.fill_(float(self.k))
 
 
 def time_steps(fn, steps, flush, stream):
@@ -256,7 +254,7 @@ def gpu_arm(args, rank, world, local_rank):
     w = w.with_(seed=w.seed + 1000 * rank)
     inp = make_inputs(w)
     d = {k: (v.to(dev) if v is not None else None) for k, v in inp.items()}
-    o = torch.empty(w.B, w.T, w.H, w.Dv, device=dev, dtype=d["q"].dtype)
+    o = torch.empty(w.B, w.T, w.H, w.Dv, device=dev, dtype=torch.float32)
     ST = torch.empty(w.B, w.H, w.Dk, w.Dv, device=dev, dtype=torch.float32)
 
     def prefill():
@@ -337,7 +335,7 @@ def bench_decode(kla, WORKLOADS, make_inputs, dev, stream, flush, rank, world, h
     q, k, v = inp["q"].to(dev), inp["k"].to(dev), inp["v"].to(dev)
     eta, g = inp["eta"].to(dev), inp["g"].to(dev)
     S = inp["S0"].to(dev).clone()
-    o = torch.empty(w.B, w.H, w.Dv, device=dev, dtype=q.dtype)
+    o = torch.empty(w.B, w.H, w.Dv, device=dev, dtype=torch.float32)
     steps = w.T if not args.quick else 64
     for t in range(8):
         kla.decode_step(q[t], k[t], v[t], eta[t], g[t], S, w.eps, o=o)
@@ -407,7 +405,7 @@ def bench_long(kla, WORKLOADS, make_inputs, dev, stream, rank, world, hbm_peak, 
     w = w.with_(seed=w.seed + 1000 * rank)
     inp = make_inputs(w)
     d = {k: (v.to(dev) if v is not None else None) for k, v in inp.items()}
-    o = torch.empty(w.B, w.T, w.H, w.Dv, device=dev, dtype=d["q"].dtype)
+    o = torch.empty(w.B, w.T, w.H, w.Dv, device=dev, dtype=torch.float32)
     ST = torch.empty(w.B, w.H, w.Dk, w.Dv, device=dev, dtype=torch.float32)
 
     def run():
@@ -438,7 +436,7 @@ def bench_e2e(kla, w, inp, dev, stream, rank, world, args):
     names = ["q", "k", "v", "eta", "g"]
     host = {n: inp[n].pin_memory() for n in names}
     devb = {n: torch.empty_like(host[n], device=dev) for n in names}
-    o_h = torch.empty(w.B, w.T, w.H, w.Dv, dtype=inp["q"].dtype).pin_memory()
+    o_h = torch.empty(w.B, w.T, w.H, w.Dv, dtype=torch.float32).pin_memory()
     ST_h = torch.empty(w.B, w.H, w.Dk, w.Dv, dtype=torch.float32).pin_memory()
 
     def step():

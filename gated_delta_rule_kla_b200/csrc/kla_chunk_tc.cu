@@ -71,7 +71,9 @@ struct Misc {
     uint32_t tmem_base;
     uint32_t pad;
     float G[CH], gam[CH], del[CH], bco[CH], cco[CH], invr[CH], graw[CH], eta[CH];
+    float pk[CH];   // e^{-G_j} / r_j, when the chunk's decay range allows the factorised form
     float gsum[2];  // per-warp sums of the next chunk's log-decays
+    float grange;   // max |G_j| over the current chunk
 };
 
 __device__ __forceinline__ size_t tok_index(int b, int t, int h, int T, int H) {
@@ -354,7 +356,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
             for (int blk = 0; blk < 2; ++blk)
 #pragma unroll
-                for (int cc = 0; cc < 8; ++cc) {
+                for (int c8 = 0; c8 < 8; ++c8) {  // chunk order rotated by row: no bank conflicts
+                    const int cc = (c8 + j) & 7;
                     float f[8];
                     unpack_bf16x8(*reinterpret_cast<const uint4*>(qk + blk * 16384 + 8192 + j * 128 + cc * 16), f);
 #pragma unroll
@@ -375,13 +378,22 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 if (l >= o) s += y;
             }
             const float excl = s - (x0 + x1);
-            ms->G[2 * l] = excl + x0;
-            ms->G[2 * l + 1] = excl + x0 + x1;
+            const float G0 = excl + x0, G1 = excl + x0 + x1;
+            ms->G[2 * l] = G0;
+            ms->G[2 * l + 1] = G1;
+            float gr = fmaxf(fabsf(G0), fabsf(G1));
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) gr = fmaxf(gr, __shfl_xor_sync(0xffffffffu, gr, o));
+            if (l == 0) ms->grange = gr;
         }
         __syncthreads();
+        // e^{G_i - G_j} = gamma_i * e^{-G_j} while every |G_j| < 80 (both factors then stay
+        // finite in fp32); otherwise the exact exp of the difference.  Uniform over the CTA.
+        const bool factored = ms->grange < 80.f;
         if (tid < CH) {
             ms->gam[tid] = __expf(ms->G[tid]);
             ms->del[tid] = __expf(ms->G[n - 1] - ms->G[tid]);
+            ms->pk[tid] = factored ? __expf(-ms->G[tid]) * ms->invr[tid] : 0.f;
         }
         if (!wait_mma()) { aborted = true; break; }
         tc_fence_after();
@@ -393,21 +405,39 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             tmem_ld_wait();
             if (row < CH) {
                 const int i = row;
-                const float Gi = ms->G[i];
+                if (factored) {
+                    const float gi = ms->gam[i];
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const int j = 32 * ch + e;
-                    x[e] = (j <= i) ? __expf(Gi - ms->G[j]) * x[e] * ms->invr[j] : 0.f;
+                    for (int e = 0; e < 32; ++e) {
+                        const int j = 32 * ch + e;
+                        x[e] = (j <= i) ? gi * x[e] * ms->pk[j] : 0.f;
+                    }
+                } else {
+                    const float Gi = ms->G[i];
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const int j = 32 * ch + e;
+                        x[e] = (j <= i) ? __expf(Gi - ms->G[j]) * x[e] * ms->invr[j] : 0.f;
+                    }
                 }
                 st_chunks_split(sm + OFF_P, sm + OFF_P + 8192, i, 4 * ch, 4, x);
             } else {
                 const int i = row - CH;
-                const float Gi = ms->G[i];
                 const float bi = ms->bco[i] * ms->invr[i];
+                if (factored) {
+                    const float bgi = bi * ms->gam[i];
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const int j = 32 * ch + e;
-                    x[e] = (j < i) ? bi * __expf(Gi - ms->G[j]) * x[e] * ms->invr[j] : 0.f;
+                    for (int e = 0; e < 32; ++e) {
+                        const int j = 32 * ch + e;
+                        x[e] = (j < i) ? bgi * x[e] * ms->pk[j] : 0.f;
+                    }
+                } else {
+                    const float Gi = ms->G[i];
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const int j = 32 * ch + e;
+                        x[e] = (j < i) ? bi * __expf(Gi - ms->G[j]) * x[e] * ms->invr[j] : 0.f;
+                    }
                 }
                 float4* lrow = reinterpret_cast<float4*>(Lf + i * LDL + 32 * ch);
 #pragma unroll
@@ -477,7 +507,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             const int j = tid >> 2, blk = (tid >> 1) & 1, c0 = 4 * (tid & 1);
             const float sc = ms->del[j] * ms->invr[j];
 #pragma unroll
-            for (int cc = c0; cc < c0 + 4; ++cc) {
+            for (int c4 = 0; c4 < 4; ++c4) {
+                const int cc = c0 + ((c4 + j) & 3);  // rotated by row: no bank conflicts
                 float f[8], hi[8], lo[8];
                 const uint32_t off = (uint32_t)(j * 128 + cc * 16);  // same swizzle phase: (64 + j) & 7 == j & 7
                 unpack_bf16x8(*reinterpret_cast<const uint4*>(qk + blk * 16384 + 8192 + off), f);

@@ -83,6 +83,8 @@ FWD_CASES = [
     (2, 130, 3, 128, 128, "bf16", True, -0.01),
     (1, 129, 2, 64, 64, "bf16", False, -0.5),
     (1, 100, 1, 128, 64, "bf16", True, -0.5),
+    (1, 150, 2, 128, 128, "bf16", True, -2.0),   # in-chunk decay down to ~e^-64
+    (1, 200, 2, 128, 128, "bf16", True, -4.0),   # beyond e^-80 inside a chunk
 ]
 
 
