@@ -212,9 +212,11 @@ kla_status kla_decode_step(const void* q, const void* k, const void* v, const fl
 }
 
 kla_status kla_check_device_error(void* stream) {
-    unsigned int flag = 0;
+    unsigned int flag = 0, flag2 = 0;
     cudaError_t e = kla::tc_take_error(static_cast<cudaStream_t>(stream), &flag);
+    if (e == cudaSuccess) e = kla::decode_take_error(static_cast<cudaStream_t>(stream), &flag2);
     if (e != cudaSuccess) return cuda_fail(e, "kla_check_device_error");
+    flag |= flag2 << 8;
     if (flag) return fail(KLA_ERR_TIMEOUT, "a kernel gave up on a bounded wait (flag %u)", flag);
     return KLA_OK;
 }

@@ -5,150 +5,289 @@
 //   e_j  = v_j - alpha (S^T k)_j
 //   S'_ij = alpha S_ij + beta k_i e_j
 //   o_j  = (S'^T q)_j = alpha (S^T q)_j + beta (k.q) e_j
-// so one pass that reads S once yields both reductions; the update is then applied to
-// the registers already holding S and written back once.  The kernel is HBM bound:
-// 2 * Dk * Dv * 4 bytes of state traffic per head against ~7 Dk Dv FLOPs.
+// so one pass that reads S once yields both reductions; the update is applied to values
+// already on chip and written back once.  The kernel is HBM bound: 2 * Dk * Dv * 4 bytes of
+// state traffic per head against ~7 Dk Dv FLOPs.
 //
-// Mapping: one CTA per (b, h), 256 threads.  A thread owns 4 adjacent columns (one
-// 16-byte vector) of DK/ROWG rows; a warp reads 32 consecutive float4 = one 512-byte
-// contiguous row segment, so every load and store is fully coalesced.
+// Work unit = one head's state restricted to NV = 64 value columns (the columns are
+// independent): Dk x 64 fp32.  A persistent grid with two CTAs per SM walks the units; a
+// single thread keeps up to STAGES - 1 units ahead in flight with 2-D TMA loads (plus 1-D
+// bulk copies of k, q and the unit's slice of v) into a ring of shared-memory stages, while
+// all threads reduce, update and store the current unit.  Waits are bounded; on expiry the
+// kernel records an error word (reported by kla_check_device_error) and stops.
+#include <cuda.h>
+
 #include "kla_device.cuh"
 #include "kla_launch.h"
+#include "kla_sm100.cuh"
 
 namespace kla {
 
+__device__ unsigned int g_decode_error = 0;
+
+namespace {
+
+using namespace sm100;
+
+constexpr int NT = 256;
+constexpr int NV = 64;            // value columns per unit
+constexpr int CG = NV / 4;        // float4 column groups per unit (16)
+constexpr int RG = NT / CG;       // row groups (32)
+constexpr int STAGES = 3;
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+constexpr int NW = NT / 32;       // warps
+constexpr int MAX_UNITS_PER_CTA = 64;
+
+template <int DK, typename Tin>
+struct DecodeSmem {
+    float s[STAGES][DK][NV];                    // state tiles
+    Tin kv[STAGES][DK], qv[STAGES][DK], vv[STAGES][NV];
+    float4 red_k[NW][CG], red_q[NW][CG];        // per-warp partial S^T k, S^T q
+    float4 be[CG];                              // beta * e for the unit's columns
+    float scal[2][NW];                          // per-warp partial ||k||^2, k.q
+    float alpha[MAX_UNITS_PER_CTA], eta[MAX_UNITS_PER_CTA];
+    uint64_t full[STAGES];
+};
+
 template <int DK, int DV, typename Tin, typename TOut>
-__global__ void __launch_bounds__(256) decode_step_kernel(const Tin* __restrict__ q,
-                                                          const Tin* __restrict__ k,
-                                                          const Tin* __restrict__ v,
-                                                          const float* __restrict__ eta,
-                                                          const float* __restrict__ g, float eps,
-                                                          float* __restrict__ S,
-                                                          TOut* __restrict__ o) {
-    constexpr int NT = 256;
-    constexpr int COLG = DV / 4;       // float4 column groups
-    constexpr int ROWG = NT / COLG;    // row groups
-    constexpr int RPT = DK / ROWG;     // rows per thread
-    static_assert(NT % COLG == 0 && DK % ROWG == 0, "tile mapping");
+__global__ void __launch_bounds__(NT, 2)
+    decode_step_kernel(const __grid_constant__ CUtensorMap tm_s, const Tin* __restrict__ q,
+                       const Tin* __restrict__ k, const Tin* __restrict__ v, const float* __restrict__ eta,
+                       const float* __restrict__ g, float eps, float* __restrict__ S, TOut* __restrict__ o,
+                       int units) {
+    constexpr int RPT = DK / RG;   // rows per thread
+    constexpr int UPH = DV / NV;   // units per head
+    constexpr uint32_t kTileBytes = DK * NV * 4;
+    constexpr uint32_t kVecBytes = DK * sizeof(Tin);
+    constexpr uint32_t kVBytes = NV * sizeof(Tin);
+    extern __shared__ uint8_t smem_raw[];
+    auto& sm = *reinterpret_cast<DecodeSmem<DK, Tin>*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
 
-    __shared__ float ks[DK], qs[DK];
-    __shared__ float4 red_k[ROWG][COLG], red_q[ROWG][COLG];
-    __shared__ float scal[2][8];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int cg = tid % CG;
+    const int rg = tid / CG;
+    const int stride = gridDim.x;
+    const int nmine = (blockIdx.x < units) ? (units - 1 - blockIdx.x) / stride + 1 : 0;
 
-    const int head = blockIdx.x;  // b * H + h
-    const int tid = threadIdx.x;
-    const int cg = tid % COLG;
-    const int rg = tid / COLG;
-
-    // Issue the state loads first: they are the only large traffic.
-    float4* Sh = reinterpret_cast<float4*>(S + (size_t)head * DK * DV);
-    float4 s[RPT];
-#pragma unroll
-    for (int r = 0; r < RPT; ++r) s[r] = Sh[(size_t)(rg + r * ROWG) * COLG + cg];
-
-    // k, q into shared memory; ||k||^2 and k.q reduced over the block.
-    float kk = 0.f, kq = 0.f;
-    for (int i = tid; i < DK; i += NT) {
-        float kv = to_f32(k[(size_t)head * DK + i]);
-        float qv = to_f32(q[(size_t)head * DK + i]);
-        ks[i] = kv;
-        qs[i] = qv;
-        kk += kv * kv;
-        kq += kv * qv;
+    if (tid == 0) {
+        for (int s = 0; s < STAGES; ++s) mbar_init(smem_u32(&sm.full[s]), 1);
+        fence_mbar_init();
+        prefetch_tmap(&tm_s);
     }
-    kk = warp_sum(kk);
-    kq = warp_sum(kq);
-    if ((tid & 31) == 0) {
-        scal[0][tid >> 5] = kk;
-        scal[1][tid >> 5] = kq;
+    // the decay and gate of every unit this CTA will process, loaded once
+    if (tid < nmine) {
+        const int head = (blockIdx.x + tid * stride) / UPH;
+        sm.alpha[tid] = expf(g[head]);
+        sm.eta[tid] = eta[head];
     }
     __syncthreads();
-    float n2 = 0.f, kdq = 0.f;
-#pragma unroll
-    for (int w = 0; w < NT / 32; ++w) {
-        n2 += scal[0][w];
-        kdq += scal[1][w];
-    }
-    const float alpha = expf(g[head]);
-    const float den = n2 + eps;
-    const float beta = den > 0.f ? eta[head] / den : 0.f;
 
-    // Partial S^T k and S^T q over this thread's rows.
-    float4 pk = make_float4(0.f, 0.f, 0.f, 0.f), pq = pk;
-#pragma unroll
-    for (int r = 0; r < RPT; ++r) {
-        const float ki = ks[rg + r * ROWG];
-        const float qi = qs[rg + r * ROWG];
-        pk.x = fmaf(s[r].x, ki, pk.x); pk.y = fmaf(s[r].y, ki, pk.y);
-        pk.z = fmaf(s[r].z, ki, pk.z); pk.w = fmaf(s[r].w, ki, pk.w);
-        pq.x = fmaf(s[r].x, qi, pq.x); pq.y = fmaf(s[r].y, qi, pq.y);
-        pq.z = fmaf(s[r].z, qi, pq.z); pq.w = fmaf(s[r].w, qi, pq.w);
+    // one thread requests unit number i of this CTA into stage i % STAGES
+    auto request = [&](int i) {
+        const int u = blockIdx.x + i * stride;
+        const int head = u / UPH, v0 = (u % UPH) * NV;
+        const int st = i % STAGES;
+        const uint32_t bar = smem_u32(&sm.full[st]);
+        mbar_expect_tx(bar, kTileBytes + 2 * kVecBytes + kVBytes);
+        tma_load_2d(smem_u32(&sm.s[st][0][0]), &tm_s, bar, v0, head * DK);
+        bulk_load(smem_u32(&sm.kv[st][0]), k + (size_t)head * DK, kVecBytes, bar);
+        bulk_load(smem_u32(&sm.qv[st][0]), q + (size_t)head * DK, kVecBytes, bar);
+        bulk_load(smem_u32(&sm.vv[st][0]), v + (size_t)head * DV + v0, kVBytes, bar);
+    };
+    if (tid == 0) {
+        for (int i = 0; i < STAGES - 1 && i < nmine; ++i) request(i);
     }
-    red_k[rg][cg] = pk;
-    red_q[rg][cg] = pq;
-    __syncthreads();
-    float4 sk = make_float4(0.f, 0.f, 0.f, 0.f), sq = sk;
-#pragma unroll
-    for (int w = 0; w < ROWG; ++w) {
-        float4 a = red_k[w][cg], b = red_q[w][cg];
-        sk.x += a.x; sk.y += a.y; sk.z += a.z; sk.w += a.w;
-        sq.x += b.x; sq.y += b.y; sq.z += b.z; sq.w += b.w;
-    }
-    // e = v - alpha S^T k  (four columns of this thread)
-    const Tin* vh = v + (size_t)head * DV + cg * 4;
-    float4 e;
-    e.x = to_f32(vh[0]) - alpha * sk.x;
-    e.y = to_f32(vh[1]) - alpha * sk.y;
-    e.z = to_f32(vh[2]) - alpha * sk.z;
-    e.w = to_f32(vh[3]) - alpha * sk.w;
-    float4 be = make_float4(beta * e.x, beta * e.y, beta * e.z, beta * e.w);
 
-    // S <- alpha S + beta k e^T, written back in place.
+    for (int i = 0; i < nmine; ++i) {
+        const int u = blockIdx.x + i * stride;
+        const int head = u / UPH, v0 = (u % UPH) * NV;
+        const int st = i % STAGES;
+        // keep STAGES - 1 units in flight; every thread finished reading stage (i - 1) % STAGES
+        // before the previous iteration's second barrier (the update uses registers only)
+        if (tid == 0 && i + STAGES - 1 < nmine) {
+            fence_proxy_async();
+            request(i + STAGES - 1);
+        }
+        const bool ok = mbar_wait_bounded(smem_u32(&sm.full[st]), (i / STAGES) & 1, kWaitLimitNs);
+        if (__syncthreads_or(!ok)) {
+            if (tid == 0) {
+                atomicOr(&g_decode_error, 1u);
+                // let the loads already requested land before the CTA exits
+                const int last = min(i + STAGES - 1, nmine - 1);
+                for (int j = i; j <= last; ++j)
+                    (void)mbar_wait_bounded(smem_u32(&sm.full[j % STAGES]), (j / STAGES) & 1, kWaitLimitNs);
+            }
+            break;
+        }
+        // partial ||k||^2, k.q, S^T k, S^T q; the state slice stays in registers
+        float kk = 0.f, kq = 0.f;
+        if (tid < DK) {
+            const float kx = to_f32(sm.kv[st][tid]), qx = to_f32(sm.qv[st][tid]);
+            kk = kx * kx;
+            kq = kx * qx;
+        }
+        float4 cur[RPT];
+        float kir[RPT];  // k rows of this thread, kept for the update (the stage is refilled early)
+        float4 pk = make_float4(0.f, 0.f, 0.f, 0.f), pq = pk;
 #pragma unroll
-    for (int r = 0; r < RPT; ++r) {
-        const float ki = ks[rg + r * ROWG];
-        float4 x = s[r];
-        x.x = fmaf(alpha, x.x, ki * be.x);
-        x.y = fmaf(alpha, x.y, ki * be.y);
-        x.z = fmaf(alpha, x.z, ki * be.z);
-        x.w = fmaf(alpha, x.w, ki * be.w);
-        Sh[(size_t)(rg + r * ROWG) * COLG + cg] = x;
-    }
-    // o = alpha S^T q + (k.q) beta e
-    if (o != nullptr && rg == 0) {
-        TOut* oh = o + (size_t)head * DV + cg * 4;
-        oh[0] = from_f32<TOut>(fmaf(alpha, sq.x, kdq * be.x));
-        oh[1] = from_f32<TOut>(fmaf(alpha, sq.y, kdq * be.y));
-        oh[2] = from_f32<TOut>(fmaf(alpha, sq.z, kdq * be.z));
-        oh[3] = from_f32<TOut>(fmaf(alpha, sq.w, kdq * be.w));
+        for (int r = 0; r < RPT; ++r) {
+            const int row = rg + r * RG;
+            cur[r] = *reinterpret_cast<const float4*>(&sm.s[st][row][4 * cg]);
+            const float ki = to_f32(sm.kv[st][row]);
+            kir[r] = ki;
+            const float qi = to_f32(sm.qv[st][row]);
+            pk.x = fmaf(cur[r].x, ki, pk.x); pk.y = fmaf(cur[r].y, ki, pk.y);
+            pk.z = fmaf(cur[r].z, ki, pk.z); pk.w = fmaf(cur[r].w, ki, pk.w);
+            pq.x = fmaf(cur[r].x, qi, pq.x); pq.y = fmaf(cur[r].y, qi, pq.y);
+            pq.z = fmaf(cur[r].z, qi, pq.z); pq.w = fmaf(cur[r].w, qi, pq.w);
+        }
+        // lanes c and c + 16 hold the same columns (two rows of the warp): fold them
+        pk.x += __shfl_xor_sync(0xffffffffu, pk.x, 16); pk.y += __shfl_xor_sync(0xffffffffu, pk.y, 16);
+        pk.z += __shfl_xor_sync(0xffffffffu, pk.z, 16); pk.w += __shfl_xor_sync(0xffffffffu, pk.w, 16);
+        pq.x += __shfl_xor_sync(0xffffffffu, pq.x, 16); pq.y += __shfl_xor_sync(0xffffffffu, pq.y, 16);
+        pq.z += __shfl_xor_sync(0xffffffffu, pq.z, 16); pq.w += __shfl_xor_sync(0xffffffffu, pq.w, 16);
+        kk = warp_sum(kk);
+        kq = warp_sum(kq);
+        if (lane < CG) {
+            sm.red_k[warp][lane] = pk;
+            sm.red_q[warp][lane] = pq;
+        }
+        if (lane == 0) {
+            sm.scal[0][warp] = kk;
+            sm.scal[1][warp] = kq;
+        }
+        __syncthreads();
+        const float alpha = sm.alpha[i];
+        if (tid < CG) {  // final sums, residual and output for column group cg = tid
+            float n2 = 0.f, kdq = 0.f;
+            float4 sk = make_float4(0.f, 0.f, 0.f, 0.f), sq = sk;
+#pragma unroll
+            for (int w = 0; w < NW; ++w) {
+                n2 += sm.scal[0][w];
+                kdq += sm.scal[1][w];
+                const float4 a = sm.red_k[w][tid], b = sm.red_q[w][tid];
+                sk.x += a.x; sk.y += a.y; sk.z += a.z; sk.w += a.w;
+                sq.x += b.x; sq.y += b.y; sq.z += b.z; sq.w += b.w;
+            }
+            const float den = n2 + eps;
+            const float beta = den > 0.f ? sm.eta[i] / den : 0.f;
+            float4 be;
+            be.x = beta * (to_f32(sm.vv[st][4 * tid + 0]) - alpha * sk.x);
+            be.y = beta * (to_f32(sm.vv[st][4 * tid + 1]) - alpha * sk.y);
+            be.z = beta * (to_f32(sm.vv[st][4 * tid + 2]) - alpha * sk.z);
+            be.w = beta * (to_f32(sm.vv[st][4 * tid + 3]) - alpha * sk.w);
+            sm.be[tid] = be;
+            if (o != nullptr) {  // o = alpha S^T q + (k.q) beta e
+                TOut* oh = o + (size_t)head * DV + v0 + tid * 4;
+                oh[0] = from_f32<TOut>(fmaf(alpha, sq.x, kdq * be.x));
+                oh[1] = from_f32<TOut>(fmaf(alpha, sq.y, kdq * be.y));
+                oh[2] = from_f32<TOut>(fmaf(alpha, sq.z, kdq * be.z));
+                oh[3] = from_f32<TOut>(fmaf(alpha, sq.w, kdq * be.w));
+            }
+        }
+        __syncthreads();
+        // S <- alpha S + beta k e^T, written back in place from registers
+        const float4 be = sm.be[cg];
+        float4* Sh = reinterpret_cast<float4*>(S + (size_t)head * DK * DV + v0) + cg;
+#pragma unroll
+        for (int r = 0; r < RPT; ++r) {
+            const int row = rg + r * RG;
+            const float ki = kir[r];
+            float4 x = cur[r];
+            x.x = fmaf(alpha, x.x, ki * be.x);
+            x.y = fmaf(alpha, x.y, ki * be.y);
+            x.z = fmaf(alpha, x.z, ki * be.z);
+            x.w = fmaf(alpha, x.w, ki * be.w);
+            Sh[(size_t)row * (DV / 4)] = x;
+        }
     }
 }
 
+int sm_count() {
+    static int n = 0;
+    if (n == 0) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            n = 148;
+    }
+    return n;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static bool tried = false;
+    if (!tried) {
+        tried = true;
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult qr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &qr) == cudaSuccess &&
+            qr == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
 template <int DK, int DV, typename Tin, typename TOut>
-static cudaError_t launch_decode_t(const DecodeArgs& a, cudaStream_t st) {
-    decode_step_kernel<DK, DV, Tin, TOut><<<a.B * a.H, 256, 0, st>>>(
-        static_cast<const Tin*>(a.q), static_cast<const Tin*>(a.k), static_cast<const Tin*>(a.v),
-        a.eta, a.g, a.eps, a.S, static_cast<TOut*>(a.o));
+cudaError_t launch_decode_t(const DecodeArgs& a, cudaStream_t st) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return cudaErrorNotSupported;
+    // the state as a 2-D fp32 matrix [B*H*Dk rows, Dv columns]; box = Dk rows x 64 columns
+    CUtensorMap ms;
+    cuuint64_t dims[2] = {(cuuint64_t)DV, (cuuint64_t)a.B * a.H * DK};
+    cuuint64_t strides[1] = {(cuuint64_t)DV * 4};
+    cuuint32_t box[2] = {NV, DK};
+    cuuint32_t estr[2] = {1, 1};
+    if (enc(&ms, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, a.S, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) !=
+        CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
+    const int units = a.B * a.H * (DV / NV);
+    int grid = units < 2 * sm_count() ? units : 2 * sm_count();
+    if ((units + grid - 1) / grid > MAX_UNITS_PER_CTA) grid = (units + MAX_UNITS_PER_CTA - 1) / MAX_UNITS_PER_CTA;
+    const size_t smem = sizeof(DecodeSmem<DK, Tin>) + 128;
+    cudaError_t e = cudaFuncSetAttribute(decode_step_kernel<DK, DV, Tin, TOut>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    decode_step_kernel<DK, DV, Tin, TOut><<<grid, NT, smem, st>>>(
+        ms, static_cast<const Tin*>(a.q), static_cast<const Tin*>(a.k), static_cast<const Tin*>(a.v), a.eta, a.g,
+        a.eps, a.S, static_cast<TOut*>(a.o), units);
     return cudaGetLastError();
 }
 
 template <int DK, int DV, typename Tin>
-static cudaError_t launch_decode_o(const DecodeArgs& a, cudaStream_t st) {
+cudaError_t launch_decode_o(const DecodeArgs& a, cudaStream_t st) {
     return a.out_bf16 ? launch_decode_t<DK, DV, Tin, __nv_bfloat16>(a, st)
                       : launch_decode_t<DK, DV, Tin, float>(a, st);
 }
 
 template <typename Tin>
-static cudaError_t launch_decode_d(const DecodeArgs& a, cudaStream_t st) {
+cudaError_t launch_decode_d(const DecodeArgs& a, cudaStream_t st) {
     if (a.Dk == 128 && a.Dv == 128) return launch_decode_o<128, 128, Tin>(a, st);
     if (a.Dk == 128 && a.Dv == 64) return launch_decode_o<128, 64, Tin>(a, st);
     if (a.Dk == 64 && a.Dv == 128) return launch_decode_o<64, 128, Tin>(a, st);
     return launch_decode_o<64, 64, Tin>(a, st);
 }
 
+}  // namespace
+
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st) {
     if (a.bf16) return launch_decode_d<__nv_bfloat16>(a, st);
     return launch_decode_d<float>(a, st);
+}
+
+cudaError_t decode_take_error(cudaStream_t st, unsigned int* flag) {
+    cudaError_t e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return e;
+    e = cudaMemcpyFromSymbol(flag, g_decode_error, sizeof(unsigned int));
+    if (e != cudaSuccess) return e;
+    const unsigned int zero = 0;
+    return cudaMemcpyToSymbol(g_decode_error, &zero, sizeof(unsigned int));
 }
 
 }  // namespace kla

@@ -57,6 +57,7 @@ cudaError_t launch_chunk_fwd_tc(const FwdArgs& a, cudaStream_t st);
 // Synchronise `st`, then read and clear the device error word of the tensor-core kernels
 // (non-zero when a bounded wait expired).
 cudaError_t tc_take_error(cudaStream_t st, unsigned int* flag);
+cudaError_t decode_take_error(cudaStream_t st, unsigned int* flag);
 // Record `msg` as the calling thread's last error (see kla_last_error) and return `status`.
 int set_last_error(int status, const char* msg);
 
