@@ -407,9 +407,12 @@ def bench_long(kla, WORKLOADS, make_inputs, dev, stream, rank, world, hbm_peak, 
     d = {k: (v.to(dev) if v is not None else None) for k, v in inp.items()}
     o = torch.empty(w.B, w.T, w.H, w.Dv, device=dev, dtype=torch.float32)
     ST = torch.empty(w.B, w.H, w.Dk, w.Dv, device=dev, dtype=torch.float32)
+    # few heads, long sequences: the library's segmented path (workspace allocated once here)
+    need = kla.lib().kla_chunk_fwd_workspace(w.B, w.T, w.H, w.Dk, w.Dv, 64, 1)
+    ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
 
     def run():
-        kla.chunk_fwd(d["q"], d["k"], d["v"], d["eta"], d["g"], w.eps, d["S0"], o=o, S_T=ST)
+        kla.chunk_fwd(d["q"], d["k"], d["v"], d["eta"], d["g"], w.eps, d["S0"], o=o, S_T=ST, workspace=ws)
 
     run()
     torch.cuda.synchronize()
@@ -424,6 +427,7 @@ def bench_long(kla, WORKLOADS, make_inputs, dev, stream, rank, world, hbm_peak, 
     flops = fwd_flops_per_token_head(w.Dk) * w.B * w.T * w.H
     return {"workload": w.name, "value": tokens / (total_ms / 1e3), "unit": "tokens/s",
             "steps": nsteps, "ms_per_step": total_ms / nsteps, "l2": "inputs larger than L2",
+            "gpu_launches_per_step": 3 if need > 0 else 1, "segmented": need > 0,
             "roofline": {"bound": "hbm", "achieved": alg / mean_s / 1e9, "peak": hbm_peak, "unit": "GB/s",
                          "frac": alg / mean_s / 1e9 / hbm_peak,
                          "tensor_frac": flops / mean_s / 1e12 / tc_peak}}

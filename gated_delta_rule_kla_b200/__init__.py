@@ -110,13 +110,17 @@ def _stream(device, stream):
 
 
 def chunk_fwd(q, k, v, eta, g, eps=1e-6, S0=None, *, o=None, S_T=None, save_chunk_states=False,
-              output_final_state=True, out_dtype=torch.float32, stream=None):
+              output_final_state=True, out_dtype=torch.float32, stream=None, segmented=True,
+              workspace=None):
     """Chunkwise prefill (section 4, Propositions 3-4).
 
     q, k: [B,T,H,Dk]; v: [B,T,H,Dv] (bf16 or fp32, same dtype); eta, g: [B,T,H] fp32;
     S0: [B,H,Dk,Dv] fp32 or None.  o is written in `out_dtype` (fp32 by default; a bf16
     store rounds each output once).  Returns (o, S_T) or (o, S_T, S_chunks) when
     save_chunk_states (S_chunks: [B,H,ceil(T/64),Dk,Dv], the state at each chunk start).
+    For long sequences over few heads the library splits each sequence into segments run in
+    parallel; that path needs the workspace kla_chunk_fwd_workspace() reports, allocated
+    here unless `workspace` is given (segmented=False keeps the single-pass path).
     """
     dev = k.device
     B, T, H, Dk = k.shape
@@ -134,9 +138,14 @@ def chunk_fwd(q, k, v, eta, g, eps=1e-6, S0=None, *, o=None, S_T=None, save_chun
     Sc = None
     if save_chunk_states:
         Sc = torch.empty(B, H, (T + CHUNK - 1) // CHUNK, Dk, Dv, device=dev, dtype=torch.float32)
-    st = lib().kla_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(eta), _ptr(g), float(eps), _ptr(S0),
-                             _ptr(o), _ptr(S_T), _ptr(Sc), B, T, H, Dk, Dv, CHUNK, _dtype_code(k),
-                             _dtype_code(o), None, 0, _stream(dev, stream))
+    L = lib()
+    need = L.kla_chunk_fwd_workspace(B, T, H, Dk, Dv, CHUNK, _dtype_code(k)) if segmented else 0
+    if need > 0 and (workspace is None or workspace.numel() < need):
+        workspace = torch.empty(need, device=dev, dtype=torch.uint8)
+    ws_ptr, ws_n = (_ptr(workspace), workspace.numel()) if need > 0 else (None, 0)
+    st = L.kla_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(eta), _ptr(g), float(eps), _ptr(S0),
+                         _ptr(o), _ptr(S_T), _ptr(Sc), B, T, H, Dk, Dv, CHUNK, _dtype_code(k),
+                         _dtype_code(o), ws_ptr, ws_n, _stream(dev, stream))
     _check(st, "kla_chunk_fwd")
     return (o, S_T, Sc) if save_chunk_states else (o, S_T)
 

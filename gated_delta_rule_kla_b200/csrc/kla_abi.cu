@@ -106,15 +106,16 @@ const char* kla_last_error(void) { return g_last_error.c_str(); }
 int kla_version(void) { return 100; }
 
 size_t kla_chunk_fwd_workspace(int B, int T, int H, int Dk, int Dv, int chunk, int dtype) {
-    (void)B; (void)T; (void)H; (void)Dk; (void)Dv; (void)chunk; (void)dtype;
-    return 0;
+    if (B < 1 || H < 1 || T < 1 || chunk != kla::kChunkLen) return 0;
+    kla::FwdArgs a{};
+    a.B = B; a.T = T; a.H = H; a.Dk = Dk; a.Dv = Dv; a.bf16 = dtype == KLA_BF16;
+    return kla::chunk_fwd_tc_segmented_workspace(a);
 }
 
 kla_status kla_chunk_fwd(const void* q, const void* k, const void* v, const float* eta,
                          const float* g, float eps, const float* S0, void* o, float* S_T,
                          float* S_chunks, int B, int T, int H, int Dk, int Dv, int chunk,
                          int dtype, int out_dtype, void* ws, size_t ws_bytes, void* stream) {
-    (void)ws; (void)ws_bytes;
     kla_status st = check_common(B, T, H, Dk, Dv, chunk, dtype, out_dtype, eps);
     if (st != KLA_OK) return st;
     if (T > 0) {
@@ -133,8 +134,19 @@ kla_status kla_chunk_fwd(const void* q, const void* k, const void* v, const floa
     }
     kla::FwdArgs a{q, k, v, eta, g, eps, S0, o, S_T, S_chunks, B, T, H, Dk, Dv, dtype == KLA_BF16,
                    out_dtype == KLA_BF16};
-    cudaError_t e = kla::chunk_fwd_tc_supported(a) ? kla::launch_chunk_fwd_tc(a, s)
-                                                   : kla::launch_chunk_fwd_simt(a, s);
+    cudaError_t e;
+    if (kla::chunk_fwd_tc_supported(a)) {
+        // long sequences over few heads: the segmented path when the caller gave its workspace
+        const size_t need = kla::chunk_fwd_tc_segmented_workspace(a);
+        if (need > 0 && ws != nullptr && ws_bytes >= need) {
+            if (!aligned16(ws)) return fail(KLA_ERR_INVALID_ARG, "ws must be 16-byte aligned");
+            e = kla::launch_chunk_fwd_tc_segmented(a, ws, s);
+        } else {
+            e = kla::launch_chunk_fwd_tc(a, s);
+        }
+    } else {
+        e = kla::launch_chunk_fwd_simt(a, s);
+    }
     if (e != cudaSuccess) return cuda_fail(e, "kla_chunk_fwd launch");
     return KLA_OK;
 }
@@ -181,7 +193,7 @@ kla_status kla_chunk_bwd(const void* q, const void* k, const void* v, const floa
         float* Sc_ws = reinterpret_cast<float*>(w + off[0]);
         kla::FwdArgs fa{q, k, v, eta, g, eps, S0, nullptr, nullptr, Sc_ws, B, T, H, Dk, Dv,
                         dtype == KLA_BF16, false};
-        e = kla::launch_chunk_fwd_simt(fa, s);
+        e = kla::chunk_fwd_tc_supported(fa) ? kla::launch_chunk_fwd_tc(fa, s) : kla::launch_chunk_fwd_simt(fa, s);
         if (e != cudaSuccess) return cuda_fail(e, "kla_chunk_bwd state recompute");
         Sc = Sc_ws;
     }

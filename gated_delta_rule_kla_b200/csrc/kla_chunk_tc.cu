@@ -201,12 +201,26 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int row = tid & 127;  // TMEM lane owned with the other thread of the pair
     const int ch = tid >> 7;    // which half of an epilogue's columns this thread takes
     const int H = a.H, T = a.T;
-    const int b = blockIdx.x / H, h = blockIdx.x % H;
-    const int NC = (T + CH - 1) / CH;
+    const int NCtot = (T + CH - 1) / CH;
+    // segment handled by this CTA: chunks [c0, c1) of head (b, h); kind 1 = transition pass
+    const int nseg = a.nseg > 1 ? a.nseg : 1;
+    const bool segmented = a.nseg > 1;
+    const int segc = segmented ? a.seg_chunks : NCtot;
+    const int head_idx = blockIdx.x / nseg, seg = blockIdx.x % nseg;
+    const int BH = gridDim.x / nseg;
+    const int b = head_idx / H, h = head_idx % H;
+    const bool ident = blockIdx.y == 1;
+    const int c0 = seg * segc, c1 = min(NCtot, c0 + segc);
+    const int NC = c1 > c0 ? c1 - c0 : 0;  // chunks of this CTA
     const uint32_t sbase = smem_u32(sm);
     const uint32_t bar_full0 = smem_u32(&ms->full[0]);
     const uint32_t bar_mma = smem_u32(&ms->mma);
-    const size_t state_off = ((size_t)b * H + h) * DK * DV;
+    const float* S0p = (a.S0 && !ident)
+                           ? a.S0 + (size_t)(segmented ? head_idx * nseg + seg : head_idx) * DK * DV
+                           : nullptr;
+    float* STp = a.S_T ? a.S_T + (size_t)(segmented ? ((size_t)blockIdx.y * BH + head_idx) * nseg + seg : head_idx) *
+                                     DK * DV
+                       : nullptr;
 
     if (tid == 0) {
         mbar_init(bar_full0, 1);
@@ -221,15 +235,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         tmem_alloc(smem_u32(&ms->tmem_base), 512);
         tmem_relinquish();
     }
-    // log-decays of chunk 0 (threads 0-63); their sum gives gamma_last of chunk 0
+    // log-decays of the first chunk (threads 0-63); their sum gives its gamma_last
     float g_next = 0.f, eta_next = 0.f;
-    if (tid < CH && tid < T) {
-        const size_t ti = tok_index(b, tid, h, T, H);
+    const bool first_valid = NC > 0 && c0 * CH + tid < T;
+    if (tid < CH && first_valid) {
+        const size_t ti = tok_index(b, c0 * CH + tid, h, T, H);
         g_next = a.g[ti];
         eta_next = a.eta[ti];
     }
     if (warp < 2) {
-        const float sg = warp_sum((tid < T) ? g_next : 0.f);
+        const float sg = warp_sum((tid < CH && first_valid) ? g_next : 0.f);
         if ((tid & 31) == 0) ms->gsum[warp] = sg;
     }
     tc_fence_before();
@@ -241,16 +256,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     // Initial state: this thread holds row dk = `row`, columns [64 ch, 64 ch + 64).
     {
         const float g0 = (NC > 0) ? __expf(ms->gsum[0] + ms->gsum[1]) : 1.f;
-        float4* sc0 = (a.S_chunks && NC > 0)
-                          ? reinterpret_cast<float4*>(a.S_chunks + (size_t)blockIdx.x * NC * DK * DV +
+        float4* sc0 = (a.S_chunks && NC > 0 && !ident)
+                          ? reinterpret_cast<float4*>(a.S_chunks + ((size_t)head_idx * NCtot + c0) * DK * DV +
                                                       (size_t)row * DV + 64 * ch)
                           : nullptr;
 #pragma unroll 1
         for (int q2 = 0; q2 < 2; ++q2) {
             float x[32];
-            if (a.S0) {
-                const float4* src =
-                    reinterpret_cast<const float4*>(a.S0 + state_off + (size_t)row * DV + 64 * ch + 32 * q2);
+            if (S0p) {
+                const float4* src = reinterpret_cast<const float4*>(S0p + (size_t)row * DV + 64 * ch + 32 * q2);
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
                     const float4 v4 = src[i];
@@ -258,7 +272,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 }
             } else {
 #pragma unroll
-                for (int i = 0; i < 32; ++i) x[i] = 0.f;
+                for (int i = 0; i < 32; ++i) x[i] = (ident && row == 64 * ch + 32 * q2 + i) ? 1.f : 0.f;
             }
             if (sc0) {
 #pragma unroll
@@ -289,12 +303,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         tma_load_4d(vv, &tm_v, bar, 0, h, t0, b);
         tma_load_4d(vv + 8192, &tm_v, bar, 64, h, t0, b);
     };
-    if (tid == 0 && NC > 0) issue_loads(0, 0);
+    if (tid == 0 && NC > 0) issue_loads(c0, 0);
 
     uint32_t mma_phase = 0;
     bool aborted = false;
-    int issued = (NC > 0) ? 0 : -1;  // last chunk whose tiles were requested
-    int landed = -1;                 // last chunk whose tiles were waited for
+    int issued = (NC > 0) ? c0 : c0 - 1;  // last chunk whose tiles were requested
+    int landed = c0 - 1;                  // last chunk whose tiles were waited for
 
     // Bounded wait on the MMA barrier shared by the whole CTA; false = give up.
     auto wait_mma = [&]() -> bool {
@@ -303,8 +317,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         return !__syncthreads_or(!ok);
     };
 
-    for (int c = 0; c < NC; ++c) {
-        const int st = c & 1;
+    for (int c = c0; c < c1; ++c) {
+        const int lc = c - c0;  // chunk index within this CTA's run
+        const int st = lc & 1;
         const int t0 = c * CH;
         const int n = min(CH, T - t0);
         uint8_t* qk = sm + OFF_QK + st * QK_STAGE;
@@ -315,15 +330,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (tid < CH) {
             ms->graw[tid] = (tid < n) ? g_next : 0.f;
             ms->eta[tid] = (tid < n) ? eta_next : 0.f;
-            if (c + 1 < NC && (c + 1) * CH + tid < T) {
+            if (c + 1 < c1 && (c + 1) * CH + tid < T) {
                 const size_t ti = tok_index(b, (c + 1) * CH + tid, h, T, H);
                 g_next = a.g[ti];
                 eta_next = a.eta[ti];
             }
         }
-        if (tid == 0 && c + 1 < NC) issue_loads(c + 1, st ^ 1);
-        if (c + 1 < NC) issued = c + 1;
-        const bool ok_tma = mbar_wait_bounded(bar_full0 + 8 * st, (c >> 1) & 1, kWaitLimitNs);
+        if (tid == 0 && c + 1 < c1) issue_loads(c + 1, st ^ 1);
+        if (c + 1 < c1) issued = c + 1;
+        const bool ok_tma = mbar_wait_bounded(bar_full0 + 8 * st, (lc >> 1) & 1, kWaitLimitNs);
         if (__syncthreads_or(!ok_tma)) { aborted = true; break; }
         landed = c;
 
@@ -365,7 +380,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 }
             const KaczCoef cf = kacz_coef(ms->eta[j], r2, a.eps);
             ms->bco[j] = cf.b;
-            ms->cco[j] = cf.c;
+            ms->cco[j] = ident ? 0.f : cf.c;  // the transition pass runs with zero values
             ms->invr[j] = cf.inv_r;
         }
         if (warp == 0) {  // inclusive prefix sum of g inside the chunk (2 tokens per lane)
@@ -551,7 +566,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             st_chunks_split(qk, qk + 16384, row, 4 * ch, 4, x);
         }
         if (warp < 2) {  // sum of the next chunk's log-decays (loaded at the top of this chunk)
-            const bool valid = (c + 1 < NC) && ((c + 1) * CH + tid < T);
+            const bool valid = (c + 1 < c1) && ((c + 1) * CH + tid < T);
             const float sg = warp_sum(valid ? g_next : 0.f);
             if ((tid & 31) == 0) ms->gsum[warp] = sg;
         }
@@ -588,10 +603,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         // ---- new state to bf16 hi/lo (thread pair = dk row) and outputs (thread pair = dv);
         // TMEM keeps gamma_last(next chunk) * S for the next chunk's accumulation
         {
-            const bool has_next = c + 1 < NC;
+            const bool has_next = c + 1 < c1;
             const float gN = has_next ? __expf(ms->gsum[0] + ms->gsum[1]) : 1.f;
-            float4* scn = (a.S_chunks && has_next)
-                              ? reinterpret_cast<float4*>(a.S_chunks + ((size_t)blockIdx.x * NC + c + 1) * DK * DV +
+            float4* scn = (a.S_chunks && has_next && !ident)
+                              ? reinterpret_cast<float4*>(a.S_chunks + ((size_t)head_idx * NCtot + c + 1) * DK * DV +
                                                           (size_t)row * DV + 64 * ch)
                               : nullptr;
 #pragma unroll 1
@@ -635,9 +650,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (tid == 0) atomicOr(&g_tc_error, 1u);
         // let TMA loads that may still be landing in shared memory finish first
         for (int cc = landed + 1; cc <= issued; ++cc)
-            (void)mbar_wait_bounded(bar_full0 + 8 * (cc & 1), (cc >> 1) & 1, kWaitLimitNs);
-    } else if (a.S_T) {
-        float4* dst = reinterpret_cast<float4*>(a.S_T + state_off + (size_t)row * DV + 64 * ch);
+            (void)mbar_wait_bounded(bar_full0 + 8 * ((cc - c0) & 1), ((cc - c0) >> 1) & 1, kWaitLimitNs);
+    } else if (STp) {
+        float4* dst = reinterpret_cast<float4*>(STp + (size_t)row * DV + 64 * ch);
 #pragma unroll 1
         for (int q2 = 0; q2 < 2; ++q2) {
             float x[32];
@@ -699,19 +714,159 @@ cudaError_t launch_chunk_fwd_tc(const FwdArgs& a, cudaStream_t st) {
     if (!make_map(&mq, a.q, a.B, a.T, a.H) || !make_map(&mk, a.k, a.B, a.T, a.H) ||
         !make_map(&mv, a.v, a.B, a.T, a.H))
         return cudaErrorInvalidValue;
+    const int nseg = a.nseg > 1 ? a.nseg : 1;
+    const dim3 grid(a.B * a.H * nseg, a.kinds > 1 ? a.kinds : 1);
     cudaError_t e;
     if (a.out_bf16) {
         e = cudaFuncSetAttribute(chunk_fwd_tc_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)SMEM_BYTES);
         if (e != cudaSuccess) return e;
-        chunk_fwd_tc_kernel<__nv_bfloat16><<<a.B * a.H, NTHREADS, SMEM_BYTES, st>>>(mq, mk, mv, a);
+        chunk_fwd_tc_kernel<__nv_bfloat16><<<grid, NTHREADS, SMEM_BYTES, st>>>(mq, mk, mv, a);
     } else {
         e = cudaFuncSetAttribute(chunk_fwd_tc_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)SMEM_BYTES);
         if (e != cudaSuccess) return e;
-        chunk_fwd_tc_kernel<float><<<a.B * a.H, NTHREADS, SMEM_BYTES, st>>>(mq, mk, mv, a);
+        chunk_fwd_tc_kernel<float><<<grid, NTHREADS, SMEM_BYTES, st>>>(mq, mk, mv, a);
     }
     return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------------------------
+// Segmented long-sequence forward.  The state map of a run of chunks is affine,
+// S_end = M S_start + N (the recurrence is linear in the state and in the values), so:
+//   pass 1: every segment twice in parallel -- from S = 0 with its values (gives N_s) and
+//           from S = I with zero values (gives M_s);
+//   scan:   S_{s+1} = M_s S_s + N_s per (b, h) in fp32, recording each segment's start;
+//   pass 2: every segment from its true start state, producing o (and S_chunks).
+// ------------------------------------------------------------------------------------
+namespace {
+
+constexpr int SCAN_LD = 129;  // padded row of M in shared memory
+
+__global__ void __launch_bounds__(256) seg_scan_kernel(const float* __restrict__ S0, const float* __restrict__ MN,
+                                                       float* __restrict__ Sstart, float* __restrict__ S_T, int BH,
+                                                       int nseg) {
+    extern __shared__ float scan_sm[];
+    float* Ss = scan_sm;             // 128 x 128 current state
+    float* Ms = Ss + DK * DV;        // 128 x SCAN_LD transition of the segment
+    const int head = blockIdx.x, tid = threadIdx.x;
+    const int tx = tid & 15, ty = tid >> 4;
+    const size_t SZ = (size_t)DK * DV;
+    for (int x = tid; x < DK * DV; x += 256) Ss[x] = S0 ? S0[head * SZ + x] : 0.f;
+    __syncthreads();
+    for (int sgm = 0; sgm < nseg; ++sgm) {
+        const float* M = MN + ((size_t)BH + head) * nseg * SZ + (size_t)sgm * SZ;   // kind 1
+        const float* N = MN + (size_t)head * nseg * SZ + (size_t)sgm * SZ;          // kind 0
+        float* out = Sstart + ((size_t)head * nseg + sgm) * SZ;
+        for (int x = tid; x < DK * DV; x += 256) {
+            out[x] = Ss[x];
+            Ms[(x / DV) * SCAN_LD + x % DV] = M[x];
+        }
+        __syncthreads();
+        float acc[8][8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+#pragma unroll
+            for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+#pragma unroll 2
+        for (int kk = 0; kk < DK; ++kk) {
+            float av[8], bv[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) av[i] = Ms[(ty + 16 * i) * SCAN_LD + kk];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) bv[j] = Ss[kk * DV + tx + 16 * j];
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+#pragma unroll
+                for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+        }
+        __syncthreads();  // every read of S and M is done
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int r = ty + 16 * i, c = tx + 16 * j;
+                Ss[r * DV + c] = acc[i][j] + N[r * DV + c];
+            }
+        __syncthreads();
+    }
+    if (S_T)
+        for (int x = tid; x < DK * DV; x += 256) S_T[head * SZ + x] = Ss[x];
+}
+
+int sm_count_tc() {
+    static int n = 0;
+    if (n == 0) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            n = 148;
+    }
+    return n;
+}
+
+// Segment count minimising a simple model of the run time in units of one chunk step:
+// pass 1 (two CTAs per segment) + pass 2 (one) + the scan (about one step per segment).
+int choose_nseg(int BH, int NC) {
+    const int sms = sm_count_tc();
+    auto waves = [&](long long ctas) { return (ctas + sms - 1) / sms; };
+    long long best_cost = (long long)NC;  // unsegmented: one CTA per head
+    int best = 1;
+    if (BH * 2 > sms) return 1;
+    for (int ns = 2; ns <= 64 && ns <= NC; ++ns) {
+        const long long per = (NC + ns - 1) / ns;
+        const long long cost = waves(2LL * BH * ns) * per + waves((long long)BH * ns) * per + ns;
+        if (cost < best_cost) {
+            best_cost = cost;
+            best = ns;
+        }
+    }
+    // require a clear gain before switching to three launches
+    return (best > 1 && best_cost * 4 < (long long)NC * 3) ? best : 1;
+}
+
+}  // namespace
+
+size_t chunk_fwd_tc_segmented_workspace(const FwdArgs& a) {
+    if (!(a.bf16 && a.Dk == 128 && a.Dv == 128 && a.T > 0)) return 0;  // shapes of the tensor-core path
+    const int NC = (a.T + CH - 1) / CH;
+    const int nseg = choose_nseg(a.B * a.H, NC);
+    if (nseg <= 1) return 0;
+    return (size_t)3 * a.B * a.H * nseg * DK * DV * sizeof(float);
+}
+
+cudaError_t launch_chunk_fwd_tc_segmented(const FwdArgs& a, void* ws, cudaStream_t st) {
+    const int NC = (a.T + CH - 1) / CH;
+    const int BH = a.B * a.H;
+    const int nseg = choose_nseg(BH, NC);
+    if (nseg <= 1) return launch_chunk_fwd_tc(a, st);
+    const int segc = (NC + nseg - 1) / nseg;
+    const int nseg_used = (NC + segc - 1) / segc;
+    const size_t SZ = (size_t)DK * DV;
+    float* MN = static_cast<float*>(ws);                  // [2, BH, nseg, DK, DV]
+    float* Sstart = MN + 2 * (size_t)BH * nseg_used * SZ;  // [BH, nseg, DK, DV]
+    FwdArgs p1 = a;
+    p1.S0 = nullptr;
+    p1.o = nullptr;
+    p1.S_T = MN;
+    p1.S_chunks = nullptr;
+    p1.nseg = nseg_used;
+    p1.seg_chunks = segc;
+    p1.kinds = 2;
+    cudaError_t e = launch_chunk_fwd_tc(p1, st);
+    if (e != cudaSuccess) return e;
+    const size_t scan_smem = sizeof(float) * (DK * DV + DK * SCAN_LD);
+    e = cudaFuncSetAttribute(seg_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)scan_smem);
+    if (e != cudaSuccess) return e;
+    seg_scan_kernel<<<BH, 256, scan_smem, st>>>(a.S0, MN, Sstart, a.S_T, BH, nseg_used);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    FwdArgs p2 = a;
+    p2.S0 = Sstart;
+    p2.S_T = nullptr;
+    p2.nseg = nseg_used;
+    p2.seg_chunks = segc;
+    p2.kinds = 1;
+    return launch_chunk_fwd_tc(p2, st);
 }
 
 cudaError_t tc_take_error(cudaStream_t st, unsigned int* flag) {

@@ -30,6 +30,11 @@ struct FwdArgs {
     int B, T, H, Dk, Dv;
     bool bf16;      // q, k, v are bf16 (else fp32)
     bool out_bf16;  // o is bf16 (else fp32)
+    // Segmented long-sequence mode (tensor-core kernel only).  nseg > 1 splits each sequence
+    // into nseg runs of seg_chunks chunks processed by separate CTAs; S0 and S_T then index
+    // [B*H, nseg, Dk, Dv] (S_T: [kinds, B*H, nseg, Dk, Dv]) and a second grid row (kind 1)
+    // runs each segment from the identity state with zero values (the segment's transition).
+    int nseg, seg_chunks, kinds;
 };
 
 struct BwdArgs {
@@ -54,6 +59,11 @@ cudaError_t launch_chunk_bwd_simt(const BwdArgs& a, cudaStream_t st);
 // Tensor-core (tcgen05) forward for bf16 inputs with Dk == Dv == 128.
 bool chunk_fwd_tc_supported(const FwdArgs& a);
 cudaError_t launch_chunk_fwd_tc(const FwdArgs& a, cudaStream_t st);
+// Workspace bytes of the segmented long-sequence forward for these sizes (0: not used).
+size_t chunk_fwd_tc_segmented_workspace(const FwdArgs& a);
+// Segmented forward: per-segment transitions in parallel, a scan over segments, then the
+// outputs of every segment from its true start state.  ws must hold the size above.
+cudaError_t launch_chunk_fwd_tc_segmented(const FwdArgs& a, void* ws, cudaStream_t st);
 // Synchronise `st`, then read and clear the device error word of the tensor-core kernels
 // (non-zero when a bounded wait expired).
 cudaError_t tc_take_error(cudaStream_t st, unsigned int* flag);

@@ -129,6 +129,24 @@ def test_fwd_long_context_workload_sampled_heads(kla, oracle_mod):
     assert rel_err(gST, rST) <= 2e-2
 
 
+@pytest.mark.parametrize("T,H,s0", [(4096 + 100, 2, True), (3000, 3, False)])
+def test_fwd_segmented_long_sequence(kla, oracle_mod, T, H, s0):
+    """Long sequences over few heads run as parallel segments chained by a scan."""
+    assert kla.lib().kla_chunk_fwd_workspace(1, T, H, 128, 128, 64, 1) > 0
+    inp = small_inputs(1, T, H, 128, 128, "bf16", seed=T + H, s0=s0, g_lo=-0.05)
+    d = {k: (v.cuda() if v is not None else None) for k, v in inp.items()}
+    o, ST, Sc = kla.chunk_fwd(d["q"], d["k"], d["v"], d["eta"], d["g"], 1e-6, d["S0"], save_chunk_states=True)
+    o1, ST1, Sc1 = kla.chunk_fwd(d["q"], d["k"], d["v"], d["eta"], d["g"], 1e-6, d["S0"], save_chunk_states=True,
+                                 segmented=False)
+    torch.cuda.synchronize()
+    kla.check_device_error()
+    ro, rST = oracle_mod.forward(*(np64(inp[k]) for k in ("q", "k", "v", "eta", "g")), 1e-6, np64(inp["S0"]))
+    assert rel_err(o, ro) <= 2e-2
+    assert rel_err(ST, rST) <= 2e-2
+    assert rel_err(o, np64(o1)) <= 1e-2
+    assert rel_err(Sc, np64(Sc1)) <= 1e-2
+
+
 def test_fwd_state_passing_equals_one_call(kla):
     """Checkpoint/resume: forward(T1) then forward(T2, S0=S_T1) == forward(T1+T2)."""
     inp = small_inputs(2, 320, 2, 128, 128, "f32", seed=5, g_lo=-0.05)
