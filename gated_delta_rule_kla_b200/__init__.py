@@ -110,7 +110,7 @@ def _stream(device, stream):
 
 
 def chunk_fwd(q, k, v, eta, g, eps=1e-6, S0=None, *, o=None, S_T=None, save_chunk_states=False,
-              output_final_state=True, out_dtype=torch.float32, stream=None, segmented=True,
+              output_final_state=True, out_dtype=torch.float32, stream=None, fused=False,
               workspace=None):
     """Chunkwise prefill (section 4, Propositions 3-4).
 
@@ -118,9 +118,11 @@ def chunk_fwd(q, k, v, eta, g, eps=1e-6, S0=None, *, o=None, S_T=None, save_chun
     S0: [B,H,Dk,Dv] fp32 or None.  o is written in `out_dtype` (fp32 by default; a bf16
     store rounds each output once).  Returns (o, S_T) or (o, S_T, S_chunks) when
     save_chunk_states (S_chunks: [B,H,ceil(T/64),Dk,Dv], the state at each chunk start).
-    For long sequences over few heads the library splits each sequence into segments run in
-    parallel; that path needs the workspace kla_chunk_fwd_workspace() reports, allocated
-    here unless `workspace` is given (segmented=False keeps the single-pass path).
+    bf16 inputs with Dk == Dv == 128 take the split path: a chunk-parallel preparation kernel
+    stores every chunk's state-independent operands in the workspace kla_chunk_fwd_workspace()
+    reports (allocated here unless `workspace` is given), then a sequential state pass (split
+    into parallel segments for long sequences over few heads).  fused=True passes no workspace,
+    which selects the one-kernel-per-head path.
     """
     dev = k.device
     B, T, H, Dk = k.shape
@@ -139,7 +141,7 @@ def chunk_fwd(q, k, v, eta, g, eps=1e-6, S0=None, *, o=None, S_T=None, save_chun
     if save_chunk_states:
         Sc = torch.empty(B, H, (T + CHUNK - 1) // CHUNK, Dk, Dv, device=dev, dtype=torch.float32)
     L = lib()
-    need = L.kla_chunk_fwd_workspace(B, T, H, Dk, Dv, CHUNK, _dtype_code(k)) if segmented else 0
+    need = 0 if fused else L.kla_chunk_fwd_workspace(B, T, H, Dk, Dv, CHUNK, _dtype_code(k))
     if need > 0 and (workspace is None or workspace.numel() < need):
         workspace = torch.empty(need, device=dev, dtype=torch.uint8)
     ws_ptr, ws_n = (_ptr(workspace), workspace.numel()) if need > 0 else (None, 0)

@@ -109,7 +109,7 @@ size_t kla_chunk_fwd_workspace(int B, int T, int H, int Dk, int Dv, int chunk, i
     if (B < 1 || H < 1 || T < 1 || chunk != kla::kChunkLen) return 0;
     kla::FwdArgs a{};
     a.B = B; a.T = T; a.H = H; a.Dk = Dk; a.Dv = Dv; a.bf16 = dtype == KLA_BF16;
-    return kla::chunk_fwd_tc_segmented_workspace(a);
+    return kla::chunk_fwd_split_workspace(a);
 }
 
 kla_status kla_chunk_fwd(const void* q, const void* k, const void* v, const float* eta,
@@ -136,11 +136,12 @@ kla_status kla_chunk_fwd(const void* q, const void* k, const void* v, const floa
                    out_dtype == KLA_BF16};
     cudaError_t e;
     if (kla::chunk_fwd_tc_supported(a)) {
-        // long sequences over few heads: the segmented path when the caller gave its workspace
-        const size_t need = kla::chunk_fwd_tc_segmented_workspace(a);
+        // With the workspace of kla_chunk_fwd_workspace: chunk-parallel preparation + state pass
+        // (segmented for long sequences over few heads).  Without it: the fused one-kernel path.
+        const size_t need = kla::chunk_fwd_split_workspace(a);
         if (need > 0 && ws != nullptr && ws_bytes >= need) {
             if (!aligned16(ws)) return fail(KLA_ERR_INVALID_ARG, "ws must be 16-byte aligned");
-            e = kla::launch_chunk_fwd_tc_segmented(a, ws, s);
+            e = kla::launch_chunk_fwd_split(a, ws, s);
         } else {
             e = kla::launch_chunk_fwd_tc(a, s);
         }
@@ -224,11 +225,12 @@ kla_status kla_decode_step(const void* q, const void* k, const void* v, const fl
 }
 
 kla_status kla_check_device_error(void* stream) {
-    unsigned int flag = 0, flag2 = 0;
+    unsigned int flag = 0, flag2 = 0, flag3 = 0;
     cudaError_t e = kla::tc_take_error(static_cast<cudaStream_t>(stream), &flag);
     if (e == cudaSuccess) e = kla::decode_take_error(static_cast<cudaStream_t>(stream), &flag2);
+    if (e == cudaSuccess) e = kla::split_take_error(static_cast<cudaStream_t>(stream), &flag3);
     if (e != cudaSuccess) return cuda_fail(e, "kla_check_device_error");
-    flag |= flag2 << 8;
+    flag |= (flag2 << 8) | (flag3 << 16);
     if (flag) return fail(KLA_ERR_TIMEOUT, "a kernel gave up on a bounded wait (flag %u)", flag);
     return KLA_OK;
 }

@@ -1,0 +1,918 @@
+// kla_chunk_split.cu -- chunkwise KLA forward split into a chunk-parallel preparation kernel
+// and a sequential state pass, both on the 5th-generation tensor cores (sm_100a).
+//
+// Same math as the fused kernel ("Kaczmarz Linear Attention", section 4, Propositions 3-4,
+// Eqs. 7-9, on unit keys khat = k/r with b = eta r^2/(r^2+eps), c = eta r/(r^2+eps)):
+//   P   = Gam o (Q Khat^T),   L = Diag(b)(Gam^- o Khat Khat^T),   T = (I + L)^{-1}
+//   W   = T Diag(b gamma) Khat,   U' = T Diag(c) V                      (independent of S)
+//   U   = U' - W S,   O = Diag(gamma) Q S + P U,   S' = gamma_last S + Ktil^T U,
+//   Ktil = Diag(delta) Khat,  delta_j = e^{G_last - G_j}.
+// Everything that does not depend on the incoming state -- P, W, U', Ktil and the decays --
+// is computed for all chunks at once by `chunk_prep_kernel` (one CTA per chunk, two CTAs per
+// SM) and written to a per-chunk record in the workspace, already in the shared-memory image
+// the MMAs read.  `chunk_state_kernel` then walks the chunks of each head in order and does
+// only what the state feeds: U = U' - W S, S' and O, with every A operand (S and U as bf16
+// hi/lo pairs) held in TMEM, so a step is two dependent MMA groups and two short epilogues.
+//
+// State-pass TMEM (lane = dv throughout, 512 columns):
+//   [0,128)   S^T master, fp32, pre-scaled by the coming chunk's gamma_last
+//   [128,192) S^T hi bf16, [192,256) S^T lo     -- A operand, K = dk
+//   [256,320) U^T accumulator fp32 (col = token)
+//   [320,352) U^T hi bf16, [352,384) U^T lo     -- A operand, K = token
+//   [384,448) O1 = S^T Q^T,  [448,512) O2 = U^T P^T;   o = gamma o O1 + O2
+#include <cuda.h>
+#include <string.h>
+
+#include "kla_device.cuh"
+#include "kla_launch.h"
+#include "kla_sm100.cuh"
+#include "kla_tc_common.cuh"
+
+namespace kla {
+
+__device__ unsigned int g_split_error = 0;
+
+namespace {
+
+using namespace sm100;
+using namespace tcc;
+
+constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s
+
+// ---- per-chunk record in the workspace (byte offsets); tiles use the 128-byte swizzle
+constexpr uint32_t REC_W = 0;        // -W^T bf16: 128 dk rows x 64 tokens          16 KB
+constexpr uint32_t REC_KT = 16384;   // Ktil hi: [64 tokens x 64 dk] x 2 blocks        16 KB
+constexpr uint32_t REC_KTLO = 32768; // Ktil lo                                        16 KB
+constexpr uint32_t REC_P = 49152;    // P hi [64 x 64], then P lo                       16 KB
+constexpr uint32_t REC_UP = 65536;   // U' fp32 [64 tokens][128 dv]                      32 KB
+constexpr uint32_t REC_TILES = 98304;
+constexpr uint32_t REC_SC = REC_TILES;  // gamma[64], then gamma_last of the next chunk  512 B
+constexpr uint32_t REC_SCB = 512;
+constexpr size_t REC_BYTES = REC_TILES + REC_SCB;
+
+// =====================================================================================
+// Preparation kernel: one chunk per CTA.
+// =====================================================================================
+constexpr int PT = 256;
+constexpr int kPrepIssuer = 128;
+constexpr uint32_t P_QK = 0;       // [Q; K] tile (32 KB), later U' fp32
+constexpr uint32_t P_V = 32768;    // V tile (16 KB), later -W^T
+constexpr uint32_t P_P = 49152;    // P hi/lo (16 KB)
+constexpr uint32_t P_Z = 65536;    // L/T fp32 -> T' T'' hi/lo -> Ktil hi/lo (32 KB)
+constexpr uint32_t P_MISC = 98304;
+constexpr uint32_t P_SMEM = P_MISC + 3072 + 1024;
+constexpr uint32_t PM_G = 0, PM_W = 64, PM_U = 128;  // TMEM columns (256 allocated)
+
+struct PrepMisc {
+    uint64_t full, mma;
+    uint32_t tmem_base, pad[3];
+    float sc[128];  // record scalars: gamma[64], gamma_last(next chunk)
+    float G[CH], gam[CH], del[CH], bco[CH], cco[CH], invr[CH], graw[CH], eta[CH], pk[CH];
+    float gsum[2], grange;
+};
+static_assert(sizeof(PrepMisc) <= 3072, "prep scalars");
+
+__global__ void __launch_bounds__(PT, 2)
+    chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                      const __grid_constant__ CUtensorMap tm_v, FwdArgs a, uint8_t* __restrict__ recs) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    PrepMisc* ms = reinterpret_cast<PrepMisc*>(sm + P_MISC);
+    float* Lf = reinterpret_cast<float*>(sm + P_Z);
+    float* Toff = Lf + 64 * LDL;
+    float* Xs = Toff + 6 * 256;
+
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int row = tid & 127, ch = tid >> 7;
+    const int H = a.H, T = a.T;
+    const int NC = (T + CH - 1) / CH;
+    const int c = blockIdx.x, head = blockIdx.y;
+    const int b = head / H, h = head % H;
+    const int t0 = c * CH, n = min(CH, T - t0);
+    uint8_t* rec = recs + ((size_t)head * NC + c) * REC_BYTES;
+    const uint32_t sbase = smem_u32(sm);
+    const uint32_t bar_full = smem_u32(&ms->full), bar_mma = smem_u32(&ms->mma);
+
+    if (tid == 0) {
+        mbar_init(bar_full, 1);
+        mbar_init(bar_mma, 1);
+        fence_mbar_init();
+        mbar_expect_tx(bar_full, 6 * 8192);
+        tma_load_4d(sbase + P_QK, &tm_q, bar_full, 0, h, t0, b);
+        tma_load_4d(sbase + P_QK + 16384, &tm_q, bar_full, 64, h, t0, b);
+        tma_load_4d(sbase + P_QK + 8192, &tm_k, bar_full, 0, h, t0, b);
+        tma_load_4d(sbase + P_QK + 24576, &tm_k, bar_full, 64, h, t0, b);
+        tma_load_4d(sbase + P_V, &tm_v, bar_full, 0, h, t0, b);
+        tma_load_4d(sbase + P_V + 8192, &tm_v, bar_full, 64, h, t0, b);
+    }
+    if (warp == 0) {
+        tmem_alloc(smem_u32(&ms->tmem_base), 256);
+        tmem_relinquish();
+    }
+    if (tid < CH) {
+        const bool live = tid < n;
+        const size_t ti = tok_index(b, t0 + (live ? tid : 0), h, T, H);
+        ms->graw[tid] = live ? a.g[ti] : 0.f;
+        ms->eta[tid] = live ? a.eta[ti] : 0.f;
+    } else if (tid < 2 * CH) {  // log-decays of the next chunk: its gamma_last
+        const int j = tid - CH;
+        const bool live = (c + 1 < NC) && ((c + 1) * CH + j < T);
+        const float gn = live ? a.g[tok_index(b, (c + 1) * CH + j, h, T, H)] : 0.f;
+        const float sg = warp_sum(gn);
+        if ((tid & 31) == 0) ms->gsum[warp - 2] = sg;
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = ms->tmem_base;
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    const uint8_t* qk = sm + P_QK;
+    const uint32_t qk_a = sbase + P_QK, v_a = sbase + P_V;
+
+    bool ok = mbar_wait_bounded(bar_full, 0, kWaitNs);
+    if (__syncthreads_or(!ok)) {
+        if (tid == 0) atomicOr(&g_split_error, 1u);
+        goto done;
+    }
+    // ---- MMA: Gram = [Q; K] K^T (lane = token; Q rows 0-63, K rows 64-127)
+    if (tid == kPrepIssuer) {
+        tc_fence_after();
+        const uint32_t ig = idesc_bf16(128, 64, false, false);
+#pragma unroll
+        for (int s = 0; s < 8; ++s) {
+            const uint32_t off = (s >> 2) * 16384 + (s & 3) * 32;
+            mma_bf16(tmem + PM_G, smem_desc(qk_a + off, 16, 1024), smem_desc(qk_a + off + 8192, 16, 1024), ig,
+                     s > 0);
+        }
+        mma_commit(bar_mma);
+    }
+    // key norms and Kaczmarz coefficients (thread 64 + j reads key row j)
+    if (tid >= CH && tid < 2 * CH) {
+        const int j = tid - CH;
+        float r2 = 0.f;
+#pragma unroll
+        for (int blk = 0; blk < 2; ++blk)
+#pragma unroll
+            for (int c8 = 0; c8 < 8; ++c8) {  // chunk order rotated by row: no bank conflicts
+                const int cc = (c8 + j) & 7;
+                float f[8];
+                unpack_bf16x8(*reinterpret_cast<const uint4*>(qk + blk * 16384 + 8192 + j * 128 + cc * 16), f);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) r2 = fmaf(f[e], f[e], r2);
+            }
+        const KaczCoef cf = kacz_coef(ms->eta[j], r2, a.eps);
+        ms->bco[j] = cf.b;
+        ms->cco[j] = cf.c;
+        ms->invr[j] = cf.inv_r;
+    }
+    if (warp == 0) {  // inclusive prefix sum of g inside the chunk (2 tokens per lane)
+        const int l = tid;
+        const float x0 = ms->graw[2 * l], x1 = ms->graw[2 * l + 1];
+        float s = x0 + x1;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const float y = __shfl_up_sync(0xffffffffu, s, o);
+            if (l >= o) s += y;
+        }
+        const float excl = s - (x0 + x1);
+        const float G0 = excl + x0, G1 = excl + x0 + x1;
+        ms->G[2 * l] = G0;
+        ms->G[2 * l + 1] = G1;
+        float gr = fmaxf(fabsf(G0), fabsf(G1));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) gr = fmaxf(gr, __shfl_xor_sync(0xffffffffu, gr, o));
+        if (l == 0) ms->grange = gr;
+    }
+    __syncthreads();
+    {
+        // e^{G_i - G_j} = gamma_i * e^{-G_j} while every |G_j| < 80; otherwise the exact exp of
+        // the difference.  Uniform over the CTA.
+        const bool factored = ms->grange < 80.f;
+        if (tid < CH) {
+            const float gm = __expf(ms->G[tid]);
+            ms->gam[tid] = gm;
+            ms->sc[tid] = gm;
+            ms->del[tid] = __expf(ms->G[CH - 1] - ms->G[tid]);  // G is flat past the last token
+            ms->pk[tid] = factored ? __expf(-ms->G[tid]) * ms->invr[tid] : 0.f;
+        } else if (tid == CH) {
+            ms->sc[CH] = __expf(ms->gsum[0] + ms->gsum[1]);
+        }
+        ok = mbar_wait_bounded(bar_mma, 0, kWaitNs);
+        if (__syncthreads_or(!ok)) {
+            if (tid == 0) atomicOr(&g_split_error, 1u);
+            goto done;
+        }
+        tc_fence_after();
+
+        // ---- Gram epilogue: P (rows 0-63, hi/lo bf16) and L (rows 64-127, fp32); 32 columns each
+        float x[32];
+        tmem_ld32(tmem + lane_base + PM_G + 32 * ch, x);
+        tmem_ld_wait();
+        if (row < CH) {
+            const int i = row;
+            if (factored) {
+                const float gi = ms->gam[i];
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const int j = 32 * ch + e;
+                    x[e] = (j <= i) ? gi * x[e] * ms->pk[j] : 0.f;
+                }
+            } else {
+                const float Gi = ms->G[i];
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const int j = 32 * ch + e;
+                    x[e] = (j <= i) ? __expf(Gi - ms->G[j]) * x[e] * ms->invr[j] : 0.f;
+                }
+            }
+            st_chunks_split(sm + P_P, sm + P_P + 8192, i, 4 * ch, 4, x);
+        } else {
+            const int i = row - CH;
+            const float bi = ms->bco[i] * ms->invr[i];
+            if (factored) {
+                const float bgi = bi * ms->gam[i];
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const int j = 32 * ch + e;
+                    x[e] = (j < i) ? bgi * x[e] * ms->pk[j] : 0.f;
+                }
+            } else {
+                const float Gi = ms->G[i];
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const int j = 32 * ch + e;
+                    x[e] = (j < i) ? bi * __expf(Gi - ms->G[j]) * x[e] * ms->invr[j] : 0.f;
+                }
+            }
+            float4* lrow = reinterpret_cast<float4*>(Lf + i * LDL + 32 * ch);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) lrow[q] = make_float4(x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    invert_unit_lower64<PT>(Lf, Toff, Xs, tid);
+    // ---- T' = T Diag(b gamma / r), T'' = T Diag(c): thread -> row tid/4, 16 columns
+    {
+        const int i = tid >> 2, qq = tid & 3, I = i >> 4;
+        float tv[16];
+        if (qq <= I) {
+            const float* src = (qq == I) ? (Lf + i * LDL + 16 * qq) : (Toff + toff_block(I, qq) * 256 + (i & 15) * 16);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const float4 t4 = *reinterpret_cast<const float4*>(src + 4 * q);
+                tv[4 * q] = t4.x; tv[4 * q + 1] = t4.y; tv[4 * q + 2] = t4.z; tv[4 * q + 3] = t4.w;
+            }
+        } else {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) tv[e] = 0.f;
+        }
+        __syncthreads();  // T is read; the tiles below overwrite it
+        float v[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            const int j = 16 * qq + e;
+            v[e] = tv[e] * (ms->bco[j] * ms->gam[j] * ms->invr[j]);
+        }
+        st_chunks_split(sm + P_Z, sm + P_Z + 8192, i, 2 * qq, 2, v);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) v[e] = tv[e] * ms->cco[16 * qq + e];
+        st_chunks_split(sm + P_Z + 16384, sm + P_Z + 24576, i, 2 * qq, 2, v);
+    }
+    fence_proxy_async();
+    __syncthreads();
+    // ---- MMA: W^T = K^T T'^T (lane = dk) and U'^T = V^T T''^T (lane = dv)
+    if (tid == kPrepIssuer) {
+        tc_fence_after();
+        const uint32_t iw = idesc_bf16(128, 64, true, false);
+#pragma unroll
+        for (int part = 0; part < 2; ++part)
+#pragma unroll
+            for (int s = 0; s < 4; ++s)
+                mma_bf16(tmem + PM_W, smem_desc(qk_a + 8192 + s * 2048, 16384, 1024),
+                         smem_desc(sbase + P_Z + part * 8192 + s * 32, 16, 1024), iw, (part | s) > 0);
+#pragma unroll
+        for (int part = 0; part < 2; ++part)
+#pragma unroll
+            for (int s = 0; s < 4; ++s)
+                mma_bf16(tmem + PM_U, smem_desc(v_a + s * 2048, 8192, 1024),
+                         smem_desc(sbase + P_Z + 16384 + part * 8192 + s * 32, 16, 1024), iw, (part | s) > 0);
+        mma_commit(bar_mma);
+    }
+    ok = mbar_wait_bounded(bar_mma, 1, kWaitNs);
+    if (__syncthreads_or(!ok)) {
+        if (tid == 0) atomicOr(&g_split_error, 1u);
+        goto done;
+    }
+    tc_fence_after();
+    {
+        // ---- -W^T to bf16 over the consumed V tile; Ktil = Diag(delta / r) K hi/lo over T tiles
+        float x[32], u[32];
+        tmem_ld32(tmem + lane_base + PM_W + 32 * ch, x);
+        tmem_ld32(tmem + lane_base + PM_U + 32 * ch, u);
+        tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) x[e] = -x[e];
+        st_chunks_bf16(sm + P_V, row, 4 * ch, 4, x);
+        {
+            const int j = tid >> 2, blk = (tid >> 1) & 1, cq = 4 * (tid & 1);
+            const float sc = ms->del[j] * ms->invr[j];
+#pragma unroll
+            for (int c4 = 0; c4 < 4; ++c4) {
+                const int cc = cq + ((c4 + j) & 3);  // rotated by row: no bank conflicts
+                float f[8], hi[8], lo[8];
+                const uint32_t off = (uint32_t)(j * 128 + cc * 16);  // same swizzle phase: (64 + j) & 7 == j & 7
+                unpack_bf16x8(*reinterpret_cast<const uint4*>(qk + blk * 16384 + 8192 + off), f);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) split_bf16(f[e] * sc, hi[e], lo[e]);
+                uint4 uh, ul;
+                uh.x = pack_bf16x2(hi[0], hi[1]); uh.y = pack_bf16x2(hi[2], hi[3]);
+                uh.z = pack_bf16x2(hi[4], hi[5]); uh.w = pack_bf16x2(hi[6], hi[7]);
+                ul.x = pack_bf16x2(lo[0], lo[1]); ul.y = pack_bf16x2(lo[2], lo[3]);
+                ul.z = pack_bf16x2(lo[4], lo[5]); ul.w = pack_bf16x2(lo[6], lo[7]);
+                *reinterpret_cast<uint4*>(sm + P_Z + blk * 8192 + off) = uh;
+                *reinterpret_cast<uint4*>(sm + P_Z + 16384 + blk * 8192 + off) = ul;
+            }
+        }
+        __syncthreads();  // the [Q; K] tile is consumed: U' goes over it
+        // ---- U' fp32 as [token][dv] (thread = dv lane, 32 tokens)
+        float* up = reinterpret_cast<float*>(sm + P_QK);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) up[(32 * ch + e) * DV + row] = u[e];
+    }
+    fence_proxy_async();
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0) {
+        bulk_store(rec + REC_W, sbase + P_V, 16384);
+        bulk_store(rec + REC_KT, sbase + P_Z, 32768);
+        bulk_store(rec + REC_P, sbase + P_P, 16384);
+        bulk_store(rec + REC_UP, sbase + P_QK, 32768);
+        bulk_store(rec + REC_SC, smem_u32(ms->sc), REC_SCB);
+        bulk_commit();
+        bulk_wait_all();
+    }
+done:
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 256);
+    }
+}
+
+// =====================================================================================
+// State pass: one CTA per (b, h) [segment, kind], chunks in order.  Warp-specialised:
+// warps 0-7 run the epilogues (thread pair = one TMEM lane = one dv column, the two threads
+// splitting the columns), warp 8 issues the MMAs.  The two sides meet on mbarriers:
+//   issuer -> epilogue: bar_u (U^T ready in TMEM), bar_s (S^T updated), bar_o (O1, O2 ready)
+//   epilogue -> issuer: s_ready (S hi/lo written), u_ready (U hi/lo written), o_free (O read)
+// so an MMA issue, which blocks its thread while the tensor pipe drains, never delays an
+// epilogue.  Per chunk c the issuer runs  U(c) | O1(c) | S(c) O2(c)  and the epilogue warps
+//   U epi(c) -> S hi/lo(c+1) [releases U(c+1)] -> S master rescale -> O epi(c) -> o via TMA.
+// =====================================================================================
+constexpr int ST = 288;
+constexpr int kIssuerWarp = 8;
+constexpr int kLoader = 32;           // thread that issues every load and store of the stage
+constexpr uint32_t S_STAGE = 114688;  // Q 16 KB + the record's tiles (96 KB)
+constexpr uint32_t SO_Q = 0, SO_W = 16384, SO_KT = 32768, SO_KTLO = 49152, SO_P = 65536, SO_PLO = 73728,
+                   SO_UP = 81920;
+static_assert(SO_W == REC_W + 16384 && SO_KT == REC_KT + 16384 && SO_KTLO == REC_KTLO + 16384 &&
+                  SO_P == REC_P + 16384 && SO_UP == REC_UP + 16384,
+              "stage mirrors the record");
+constexpr uint32_t EARLY_BYTES = S_STAGE - SO_KT;        // Ktil, P, U': free once chunk c's MMAs finish
+constexpr uint32_t LATE_BYTES = 16384 + 16384 + REC_SCB;  // Q, W, scalars: after the o tile left
+constexpr uint32_t S_SC = 2 * S_STAGE;  // 2 x 512 B record scalars
+constexpr uint32_t S_MISC = S_SC + 2 * REC_SCB;
+constexpr uint32_t S_SMEM = S_MISC + 128 + 1024;
+constexpr uint32_t TM_S = 0, TM_SH = 128, TM_SL = 192, TM_U = 256, TM_UH = 320, TM_UL = 352, TM_O1 = 384,
+                   TM_O2 = 448;
+
+struct StateMisc {
+    uint64_t full[2];
+    uint64_t bar_u, bar_s, bar_o;        // tcgen05.commit arrivals
+    uint64_t s_ready, u_ready, o_free;   // one arrival per epilogue warp
+    uint32_t tmem_base, abort;
+    float gsum[2];
+};
+
+// Pack 32 fp32 values (consecutive K indices) into 16 bf16x2 hi words and 16 lo words.
+__device__ __forceinline__ void split_pack32(const float (&x)[32], uint32_t (&hp)[16], uint32_t (&lp)[16]) {
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+        float h0, l0, h1, l1;
+        split_bf16(x[2 * e], h0, l0);
+        split_bf16(x[2 * e + 1], h1, l1);
+        hp[e] = pack_bf16x2(h0, h1);
+        lp[e] = pack_bf16x2(l0, l1);
+    }
+}
+
+// Barrier over the 256 epilogue threads (named barrier 1) returning the OR of `pred`.
+__device__ __forceinline__ bool epi_bar_or(bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.b32 p, %1, 0;\n\t"
+        "bar.red.or.pred q, 1, 256, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)pred)
+        : "memory");
+    return r != 0;
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+// Raise the expected transaction bytes of the current phase without arriving.
+__device__ __forceinline__ void mbar_expect_tx_only(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void tma_store_4d(const void* tmap, uint32_t src, int c0, int c1, int c2, int c3) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.global.shared::cta.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(
+            reinterpret_cast<uint64_t>(tmap)),
+        "r"(src), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+        : "memory");
+}
+__device__ __forceinline__ void bulk_wait_read_all() {
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+
+template <typename TOut>
+__global__ void __launch_bounds__(ST, 1)
+    chunk_state_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_o, FwdArgs a,
+                       const uint8_t* __restrict__ recs) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    StateMisc* ms = reinterpret_cast<StateMisc*>(sm + S_MISC);
+
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int row = tid & 127;        // TMEM lane = dv (epilogue warps)
+    const int ch = (tid >> 7) & 1;    // half of every epilogue's columns
+    const int H = a.H, T = a.T;
+    const int NCtot = (T + CH - 1) / CH;
+    const int nseg = a.nseg > 1 ? a.nseg : 1;
+    const bool segmented = a.nseg > 1;
+    const int segc = segmented ? a.seg_chunks : NCtot;
+    const int head_idx = blockIdx.x / nseg, seg = blockIdx.x % nseg;
+    const int BH = gridDim.x / nseg;
+    const int b = head_idx / H, h = head_idx % H;
+    const bool ident = blockIdx.y == 1;  // transition pass: identity start, zero values, no outputs
+    const int c0 = seg * segc, c1 = min(NCtot, c0 + segc);
+    const int NC = c1 > c0 ? c1 - c0 : 0;
+    const uint32_t sbase = smem_u32(sm);
+    const uint32_t bar_full0 = smem_u32(&ms->full[0]);
+    const uint32_t bar_u = smem_u32(&ms->bar_u), bar_s = smem_u32(&ms->bar_s), bar_o = smem_u32(&ms->bar_o);
+    const uint32_t s_ready = smem_u32(&ms->s_ready), u_ready = smem_u32(&ms->u_ready),
+                   o_free = smem_u32(&ms->o_free);
+    const float* S0p = (a.S0 && !ident)
+                           ? a.S0 + (size_t)(segmented ? head_idx * nseg + seg : head_idx) * DK * DV
+                           : nullptr;
+    float* STp = a.S_T ? a.S_T + (size_t)(segmented ? ((size_t)blockIdx.y * BH + head_idx) * nseg + seg : head_idx) *
+                                     DK * DV
+                       : nullptr;
+    float* Sc = (a.S_chunks && !ident) ? a.S_chunks + (size_t)head_idx * NCtot * DK * DV : nullptr;
+    const bool write_o = !ident && a.o != nullptr;
+
+    if (tid == 0) {
+        mbar_init(bar_full0, 1);
+        mbar_init(bar_full0 + 8, 1);
+        mbar_init(bar_u, 1);
+        mbar_init(bar_s, 1);
+        mbar_init(bar_o, 1);
+        mbar_init(s_ready, 8);
+        mbar_init(u_ready, 8);
+        mbar_init(o_free, 8);
+        ms->abort = 0;
+        fence_mbar_init();
+        prefetch_tmap(&tm_q);
+        if (write_o) prefetch_tmap(&tm_o);
+    }
+    if (warp == 0) {
+        tmem_alloc(smem_u32(&ms->tmem_base), 512);
+        tmem_relinquish();
+    }
+    if (warp < 2) {  // gamma_last of the first chunk
+        const bool live = NC > 0 && c0 * CH + tid < T;
+        const float gv = live ? a.g[tok_index(b, c0 * CH + tid, h, T, H)] : 0.f;
+        const float sg = warp_sum(gv);
+        if ((tid & 31) == 0) ms->gsum[warp] = sg;
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = ms->tmem_base;
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+
+    // Stage loads: the early part (Ktil, P, U') and the late part (Q, W, scalars) of chunk c.
+    auto load_early = [&](int c, int st) {
+        const uint32_t bar = bar_full0 + 8 * st;
+        const uint32_t base = sbase + st * S_STAGE;
+        const uint8_t* rec = recs + ((size_t)head_idx * NCtot + c) * REC_BYTES;
+        mbar_expect_tx_only(bar, EARLY_BYTES);
+#pragma unroll
+        for (int p = 0; p < 5; ++p) bulk_load(base + SO_KT + p * 16384, rec + REC_KT + p * 16384, 16384, bar);
+    };
+    auto load_late = [&](int c, int st) {
+        const uint32_t bar = bar_full0 + 8 * st;
+        const uint32_t base = sbase + st * S_STAGE;
+        const uint8_t* rec = recs + ((size_t)head_idx * NCtot + c) * REC_BYTES;
+        mbar_expect_tx(bar, LATE_BYTES);  // the one arrival of the phase
+        tma_load_4d(base + SO_Q, &tm_q, bar, 0, h, c * CH, b);
+        tma_load_4d(base + SO_Q + 8192, &tm_q, bar, 64, h, c * CH, b);
+        bulk_load(base + SO_W, rec + REC_W, 16384, bar);
+        bulk_load(sbase + S_SC + st * REC_SCB, rec + REC_SC, REC_SCB, bar);
+    };
+    int issued = c0 - 1;  // (loader) last chunk whose late part was requested
+    if (tid == kLoader) {
+        for (int i = 0; i < min(NC, 2); ++i) {
+            load_early(c0 + i, i);
+            load_late(c0 + i, i);
+            issued = c0 + i;
+        }
+    }
+    __syncwarp();
+
+    bool aborted = false;
+    if (warp == kIssuerWarp) {
+        // ================================ MMA issuer ================================
+        if ((tid & 31) == 0) {
+            const uint32_t iu = idesc_bf16(128, 64, false, true);
+            const uint32_t io = idesc_bf16(128, 64, false, false);
+            const uint32_t is = idesc_bf16(128, 128, false, true);
+            for (int c = c0; c < c1 && !aborted; ++c) {
+                const int lc = c - c0, st = lc & 1;
+                const uint32_t stg = sbase + st * S_STAGE;
+                if (!mbar_wait_bounded(bar_full0 + 8 * st, (lc >> 1) & 1, kWaitNs) ||
+                    !mbar_wait_bounded(s_ready, lc & 1, kWaitNs)) {
+                    aborted = true;
+                    break;
+                }
+                tc_fence_after();
+                // U^T = -(S^T W^T)   (the record holds -W^T; U' is added in the epilogue)
+#pragma unroll
+                for (int part = 0; part < 2; ++part)
+#pragma unroll
+                    for (int s = 0; s < 8; ++s)
+                        mma_bf16_ts(tmem + TM_U, tmem + (part ? TM_SL : TM_SH) + 8 * s,
+                                    smem_desc(stg + SO_W + s * 2048, 8192, 1024), iu, (part | s) > 0);
+                mma_commit(bar_u);
+                // O1 = S^T Q^T, once the previous chunk's outputs are read
+                if (lc > 0 && !mbar_wait_bounded(o_free, (lc - 1) & 1, kWaitNs)) {
+                    aborted = true;
+                    break;
+                }
+                tc_fence_after();
+#pragma unroll
+                for (int part = 0; part < 2; ++part)
+#pragma unroll
+                    for (int s = 0; s < 8; ++s)
+                        mma_bf16_ts(tmem + TM_O1, tmem + (part ? TM_SL : TM_SH) + 8 * s,
+                                    smem_desc(stg + SO_Q + (s >> 2) * 8192 + (s & 3) * 32, 16, 1024), io,
+                                    (part | s) > 0);
+                // S^T += U^T Ktil (N = 128), then O2 = U^T P^T; hi x hi, hi x lo, lo x hi
+                if (!mbar_wait_bounded(u_ready, lc & 1, kWaitNs)) {
+                    aborted = true;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t ua[3] = {TM_UH, TM_UH, TM_UL};
+                const uint32_t kb[3] = {stg + SO_KT, stg + SO_KTLO, stg + SO_KT};
+                const uint32_t pb[3] = {stg + SO_P, stg + SO_PLO, stg + SO_P};
+#pragma unroll
+                for (int p = 0; p < 3; ++p)
+#pragma unroll
+                    for (int s = 0; s < 4; ++s)
+                        mma_bf16_ts(tmem + TM_S, tmem + ua[p] + 8 * s, smem_desc(kb[p] + s * 2048, 8192, 1024), is,
+                                    1);
+                mma_commit(bar_s);
+#pragma unroll
+                for (int p = 0; p < 3; ++p)
+#pragma unroll
+                    for (int s = 0; s < 4; ++s)
+                        mma_bf16_ts(tmem + TM_O2, tmem + ua[p] + 8 * s, smem_desc(pb[p] + s * 32, 16, 1024), io,
+                                    (p | s) > 0);
+                mma_commit(bar_o);
+            }
+            if (aborted) atomicOr(&ms->abort, 1u);
+        }
+        __syncwarp();
+    } else {
+        // ================================ epilogue warps ================================
+        // Initial state: thread (dv = row, half ch) holds dk in [64 ch, 64 ch + 64).
+        {
+            const float g0 = NC > 0 ? __expf(ms->gsum[0] + ms->gsum[1]) : 1.f;
+#pragma unroll 1
+            for (int q2 = 0; q2 < 2; ++q2) {
+                const int dk0 = 64 * ch + 32 * q2;
+                float x[32];
+#pragma unroll
+                for (int e = 0; e < 32; ++e)
+                    x[e] = S0p ? S0p[(size_t)(dk0 + e) * DV + row] : ((ident && dk0 + e == row) ? 1.f : 0.f);
+                if (Sc && NC > 0) {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) Sc[((size_t)c0 * DK + dk0 + e) * DV + row] = x[e];
+                }
+                uint32_t hp[16], lp[16];
+                split_pack32(x, hp, lp);
+                tmem_st16u(tmem + lane_base + TM_SH + 32 * ch + 16 * q2, hp);
+                tmem_st16u(tmem + lane_base + TM_SL + 32 * ch + 16 * q2, lp);
+#pragma unroll
+                for (int e = 0; e < 32; ++e) x[e] *= g0;
+                tmem_st32(tmem + lane_base + TM_S + 64 * ch + 32 * q2, x);
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if ((tid & 31) == 0) mbar_arrive(s_ready);
+        }
+        for (int c = c0; c < c1; ++c) {
+            const int lc = c - c0, st = lc & 1;
+            const uint8_t* stg_p = sm + st * S_STAGE;
+            const bool has_next = c + 1 < c1;
+            // ---- U epilogue: U = U' + acc, to bf16 hi/lo A operands (thread = dv, 32 tokens)
+            {
+                const bool ok = mbar_wait_bounded(bar_u, lc & 1, kWaitNs);
+                if (epi_bar_or(!ok)) { aborted = true; break; }
+                tc_fence_after();
+                float x[32];
+                tmem_ld32(tmem + lane_base + TM_U + 32 * ch, x);
+                tmem_ld_wait();
+                if (!ident) {
+                    const float* up = reinterpret_cast<const float*>(stg_p + SO_UP);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) x[e] += up[(32 * ch + e) * DV + row];
+                }
+                uint32_t hp[16], lp[16];
+                split_pack32(x, hp, lp);
+                tmem_st16u(tmem + lane_base + TM_UH + 16 * ch, hp);
+                tmem_st16u(tmem + lane_base + TM_UL + 16 * ch, lp);
+                tmem_st_wait();  // also covers the previous chunk's master rescale
+                tc_fence_before();
+                __syncwarp();
+                if ((tid & 31) == 0) mbar_arrive(u_ready);
+            }
+            // ---- state epilogue: S_{c+1} to hi/lo (releases U(c+1)), then the fp32 master
+            //      pre-scaled by the next gamma_last
+            {
+                const bool ok = mbar_wait_bounded(bar_s, lc & 1, kWaitNs);
+                if (epi_bar_or(!ok)) { aborted = true; break; }
+                tc_fence_after();
+                if (has_next) {
+                    float x0[32], x1[32];
+                    tmem_ld32(tmem + lane_base + TM_S + 64 * ch, x0);
+                    tmem_ld32(tmem + lane_base + TM_S + 64 * ch + 32, x1);
+                    tmem_ld_wait();
+                    {
+                        uint32_t hp[16], lp[16];
+                        split_pack32(x0, hp, lp);
+                        tmem_st16u(tmem + lane_base + TM_SH + 32 * ch, hp);
+                        tmem_st16u(tmem + lane_base + TM_SL + 32 * ch, lp);
+                        split_pack32(x1, hp, lp);
+                        tmem_st16u(tmem + lane_base + TM_SH + 32 * ch + 16, hp);
+                        tmem_st16u(tmem + lane_base + TM_SL + 32 * ch + 16, lp);
+                    }
+                    tmem_st_wait();
+                    tc_fence_before();
+                    __syncwarp();
+                    if ((tid & 31) == 0) mbar_arrive(s_ready);
+                    if (Sc) {
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) {
+                            Sc[((size_t)(c + 1) * DK + 64 * ch + e) * DV + row] = x0[e];
+                            Sc[((size_t)(c + 1) * DK + 64 * ch + 32 + e) * DV + row] = x1[e];
+                        }
+                    }
+                    const float gN = reinterpret_cast<const float*>(sm + S_SC + st * REC_SCB)[CH];
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        x0[e] *= gN;
+                        x1[e] *= gN;
+                    }
+                    tmem_st32(tmem + lane_base + TM_S + 64 * ch, x0);
+                    tmem_st32(tmem + lane_base + TM_S + 64 * ch + 32, x1);
+                }
+            }
+            // ---- output epilogue: o = gamma o O1 + O2 staged as [token][dv] over the consumed
+            //      Q and W tiles, then one TMA store
+            {
+                const bool ok = mbar_wait_bounded(bar_o, lc & 1, kWaitNs);
+                if (epi_bar_or(!ok)) { aborted = true; break; }
+                tc_fence_after();
+                // every MMA of chunk c is done: Ktil, P, U' of this stage can take chunk c + 2
+                if (tid == kLoader && c + 2 < c1) load_early(c + 2, st);
+                __syncwarp();
+                if (write_o) {
+                    const float* gm = reinterpret_cast<const float*>(sm + S_SC + st * REC_SCB);
+                    TOut* stage_o = reinterpret_cast<TOut*>(sm + st * S_STAGE + SO_Q);
+                    float o1[32], o2[32];
+                    tmem_ld32(tmem + lane_base + TM_O1 + 32 * ch, o1);
+                    tmem_ld32(tmem + lane_base + TM_O2 + 32 * ch, o2);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const int t = 32 * ch + e;
+                        stage_o[t * DV + row] = from_f32<TOut>(fmaf(gm[t], o1[e], o2[e]));
+                    }
+                    fence_proxy_async();
+                }
+                tc_fence_before();
+                __syncwarp();
+                if ((tid & 31) == 0) mbar_arrive(o_free);
+                if (tid == kLoader) {
+                    if (!mbar_wait_bounded(o_free, lc & 1, kWaitNs)) {
+                        atomicOr(&ms->abort, 1u);
+                    } else {
+                        if (write_o) {
+                            tma_store_4d(&tm_o, sbase + st * S_STAGE + SO_Q, 0, h, c * CH, b);
+                            bulk_commit();
+                            bulk_wait_read_all();
+                        }
+                        if (c + 2 < c1) {
+                            load_late(c + 2, st);
+                            issued = c + 2;
+                        }
+                    }
+                }
+                __syncwarp();
+            }
+        }
+    }
+
+    __syncthreads();
+    if (aborted || ms->abort) {
+        if (tid == 0) atomicOr(&g_split_error, 1u);
+        if (tid == kLoader) {  // let loads that may still be landing in shared memory finish
+            for (int cc = max(c0, issued - 1); cc <= issued; ++cc)
+                (void)mbar_wait_bounded(bar_full0 + 8 * ((cc - c0) & 1), ((cc - c0) >> 1) & 1, kWaitNs);
+        }
+    } else if (NC > 0 && warp < kIssuerWarp && STp) {
+        tc_fence_after();
+#pragma unroll 1
+        for (int q2 = 0; q2 < 2; ++q2) {
+            const int dk0 = 64 * ch + 32 * q2;
+            float x[32];
+            tmem_ld32(tmem + lane_base + TM_S + 64 * ch + 32 * q2, x);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) STp[(size_t)(dk0 + e) * DV + row] = x[e];
+        }
+    }
+    bulk_wait_all();  // stores of this thread complete before exit
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+int sm_count() {
+    static int n = 0;
+    if (n == 0) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            n = 148;
+    }
+    return n;
+}
+
+// Segments per head for the state pass: minimise, in units of one state step,
+// pass 1 (two CTAs per segment, one CTA per SM) + pass 2 + the fp32 scan (~7 steps per segment).
+int choose_nseg_split(int BH, int NC) {
+    const int sms = sm_count();
+    auto waves = [&](long long ctas) { return (ctas + sms - 1) / sms; };
+    const long long base = waves(BH) * (long long)NC;
+    long long best_cost = base;
+    int best = 1;
+    for (int ns = 2; ns <= 64 && ns <= NC; ++ns) {
+        const long long per = (NC + ns - 1) / ns;
+        const long long cost = waves(2LL * BH * ns) * per + waves((long long)BH * ns) * per + 7LL * ns;
+        if (cost < best_cost) {
+            best_cost = cost;
+            best = ns;
+        }
+    }
+    return (best > 1 && best_cost * 4 < base * 3) ? best : 1;
+}
+
+size_t align1k(size_t x) { return (x + 1023) & ~size_t(1023); }
+
+struct SplitLayout {
+    size_t rec_bytes, seg_off, total;
+    int nseg, segc;
+};
+
+SplitLayout split_layout(const FwdArgs& a) {
+    SplitLayout L{};
+    const int NC = (a.T + CH - 1) / CH;
+    const int BH = a.B * a.H;
+    L.rec_bytes = align1k((size_t)BH * NC * REC_BYTES);
+    L.seg_off = L.rec_bytes;
+    const int ns = choose_nseg_split(BH, NC);
+    if (ns > 1) {
+        L.segc = (NC + ns - 1) / ns;
+        L.nseg = (NC + L.segc - 1) / L.segc;
+        L.total = L.seg_off + (size_t)3 * BH * L.nseg * DK * DV * sizeof(float);
+    } else {
+        L.nseg = 1;
+        L.segc = NC;
+        L.total = L.seg_off;
+    }
+    return L;
+}
+
+// 4-D map over the [B, T, H, 128] output (fp32 or bf16) for TMA stores of one chunk's rows of
+// one (b, h): box = 128 features x 64 tokens, no swizzle.
+bool make_out_map(CUtensorMap* m, void* base, int B, int T, int H, bool bf16) {
+    EncodeTiledFn enc = get_encode_fn();
+    if (!enc) return false;
+    const cuuint64_t elt = bf16 ? 2 : 4;
+    cuuint64_t dims[4] = {(cuuint64_t)128, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
+    cuuint64_t strides[3] = {128 * elt, (cuuint64_t)H * 128 * elt, (cuuint64_t)T * H * 128 * elt};
+    cuuint32_t box[4] = {128, 1, 64, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, base, dims,
+                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                     CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <typename TOut>
+cudaError_t launch_state(const CUtensorMap& mq, const FwdArgs& a, const uint8_t* recs, dim3 grid, cudaStream_t st) {
+    CUtensorMap mo;
+    memset(&mo, 0, sizeof(mo));
+    if (a.o != nullptr && !make_out_map(&mo, a.o, a.B, a.T, a.H, a.out_bf16)) return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(chunk_state_kernel<TOut>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)S_SMEM);
+    if (e != cudaSuccess) return e;
+    chunk_state_kernel<TOut><<<grid, ST, S_SMEM, st>>>(mq, mo, a, recs);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t chunk_fwd_split_workspace(const FwdArgs& a) {
+    if (!(a.bf16 && a.Dk == 128 && a.Dv == 128 && a.T > 0)) return 0;
+    return split_layout(a).total;
+}
+
+cudaError_t launch_chunk_fwd_split(const FwdArgs& a, void* ws, cudaStream_t st) {
+    CUtensorMap mq, mk, mv;
+    if (!make_map(&mq, a.q, a.B, a.T, a.H) || !make_map(&mk, a.k, a.B, a.T, a.H) ||
+        !make_map(&mv, a.v, a.B, a.T, a.H))
+        return cudaErrorInvalidValue;
+    const SplitLayout L = split_layout(a);
+    const int NC = (a.T + CH - 1) / CH;
+    const int BH = a.B * a.H;
+    uint8_t* recs = static_cast<uint8_t*>(ws);
+    cudaError_t e = cudaFuncSetAttribute(chunk_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)P_SMEM);
+    if (e != cudaSuccess) return e;
+    chunk_prep_kernel<<<dim3(NC, BH), PT, P_SMEM, st>>>(mq, mk, mv, a, recs);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    auto state = [&](const FwdArgs& f, dim3 grid) {
+        return f.out_bf16 ? launch_state<__nv_bfloat16>(mq, f, recs, grid, st)
+                          : launch_state<float>(mq, f, recs, grid, st);
+    };
+    if (L.nseg <= 1) {
+        FwdArgs f = a;
+        f.nseg = 1;
+        f.seg_chunks = NC;
+        f.kinds = 1;
+        return state(f, dim3(BH, 1));
+    }
+    const size_t SZ = (size_t)DK * DV;
+    float* MN = reinterpret_cast<float*>(recs + L.seg_off);  // [2, BH, nseg, DK, DV]
+    float* Sstart = MN + 2 * (size_t)BH * L.nseg * SZ;        // [BH, nseg, DK, DV]
+    FwdArgs p1 = a;
+    p1.S0 = nullptr;
+    p1.o = nullptr;
+    p1.S_T = MN;
+    p1.S_chunks = nullptr;
+    p1.nseg = L.nseg;
+    p1.seg_chunks = L.segc;
+    p1.kinds = 2;
+    if ((e = state(p1, dim3(BH * L.nseg, 2))) != cudaSuccess) return e;
+    if ((e = launch_seg_scan(a.S0, MN, Sstart, a.S_T, BH, L.nseg, st)) != cudaSuccess) return e;
+    FwdArgs p2 = a;
+    p2.S0 = Sstart;
+    p2.S_T = nullptr;
+    p2.nseg = L.nseg;
+    p2.seg_chunks = L.segc;
+    p2.kinds = 1;
+    return state(p2, dim3(BH * L.nseg, 1));
+}
+
+cudaError_t split_take_error(cudaStream_t st, unsigned int* flag) {
+    cudaError_t e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return e;
+    e = cudaMemcpyFromSymbol(flag, g_split_error, sizeof(unsigned int));
+    if (e != cudaSuccess) return e;
+    const unsigned int zero = 0;
+    return cudaMemcpyToSymbol(g_split_error, &zero, sizeof(unsigned int));
+}
+
+}  // namespace kla

@@ -35,6 +35,7 @@
 #include "kla_device.cuh"
 #include "kla_launch.h"
 #include "kla_sm100.cuh"
+#include "kla_tc_common.cuh"
 
 namespace kla {
 
@@ -43,8 +44,8 @@ __device__ unsigned int g_tc_error = 0;
 namespace {
 
 using namespace sm100;
+using namespace tcc;
 
-constexpr int DK = 128, DV = 128, CH = 64;
 constexpr int NTHREADS = 256;
 constexpr int kIssuer = 128;  // thread that issues the MMAs (warp 4: idle during the scalar prep)
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
@@ -60,7 +61,6 @@ constexpr uint32_t OFF_P = 163840;      // 16 KB: P hi [64 x 64], P lo
 constexpr uint32_t OFF_Z = 180224;      // 32 KB: L/T fp32 -> T' T'' hi/lo -> Ktil hi/lo
 constexpr uint32_t OFF_MISC = 212992;   // barriers, TMEM slot, per-token scalars
 constexpr uint32_t SMEM_BYTES = OFF_MISC + 4096 + 1024;  // + alignment slack
-constexpr int LDL = 68;                 // row stride (floats) of the fp32 L/T buffer, 16-B rows
 
 // TMEM columns
 constexpr uint32_t TM_G = 0, TM_SQ = 64, TM_W = 128, TM_U = 192, TM_S = 256, TM_PU = 384;
@@ -75,116 +75,6 @@ struct Misc {
     float gsum[2];  // per-warp sums of the next chunk's log-decays
     float grange;   // max |G_j| over the current chunk
 };
-
-__device__ __forceinline__ size_t tok_index(int b, int t, int h, int T, int H) {
-    return ((size_t)b * T + t) * H + h;
-}
-
-// Off-diagonal 16x16 block (I, J), I > J, of T in the Toff buffer: blocks ordered by
-// distance d = I - J, then by J: (1,0) (2,1) (3,2) (2,0) (3,1) (3,0).
-__device__ __forceinline__ int toff_block(int I, int J) {
-    const int d = I - J;
-    return (d == 1 ? 0 : (d == 2 ? 3 : 5)) + J;
-}
-
-// T = (I + L)^{-1} of the unit lower-triangular 64x64 matrix of Eq. (7), by blockwise
-// forward substitution (Appendix B.2) on 16x16 blocks.  L: fp32, rows of LDL floats,
-// strictly lower (upper part zero).
-//   diagonal blocks  D_I = (I + L_II)^{-1}: column by column (64 threads), written over L_II
-//   off-diagonal     T_IJ = -D_I sum_{K=J}^{I-1} L_IK T_KJ (T_JJ = D_J), by distance
-//                    d = I - J = 1, 2, 3, into Toff (6 blocks of 16x16); L stays intact.
-// X is scratch for 3 x 256 floats.  All NTHREADS threads must call it.
-__device__ __forceinline__ void invert_unit_lower64(float* Lf, float* Toff, float* X, int tid) {
-    if (tid < 64) {
-        const int base = 16 * (tid >> 4), l = tid & 15;
-        float x[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            float a0 = 0.f, a1 = 0.f;
-#pragma unroll
-            for (int j = 0; j + 1 < i; j += 2) {
-                a0 = fmaf(Lf[(base + i) * LDL + base + j], x[j], a0);
-                a1 = fmaf(Lf[(base + i) * LDL + base + j + 1], x[j + 1], a1);
-            }
-            if (i & 1) a0 = fmaf(Lf[(base + i) * LDL + base + i - 1], x[i - 1], a0);
-            x[i] = (i < l) ? 0.f : ((i == l) ? 1.f : -(a0 + a1));
-        }
-        __syncwarp();
-#pragma unroll
-        for (int i = 0; i < 16; ++i) Lf[(base + i) * LDL + base + l] = x[i];
-    }
-    __syncthreads();
-#pragma unroll 1
-    for (int d = 1; d < 4; ++d) {
-        const int njobs = 64 * (4 - d);  // (block, row, column quad)
-        for (int job = tid; job < njobs; job += NTHREADS) {
-            const int J = job >> 6, I = J + d, r = (job >> 2) & 15, cq = job & 3;
-            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-            for (int K = J; K < I; ++K) {
-                const float* tk = (K == J) ? (Lf + 16 * J * LDL + 16 * J) : (Toff + toff_block(K, J) * 256);
-                const int ldt = (K == J) ? LDL : 16;
-#pragma unroll
-                for (int m = 0; m < 16; ++m) {
-                    const float l = Lf[(16 * I + r) * LDL + 16 * K + m];
-                    const float4 t = *reinterpret_cast<const float4*>(tk + m * ldt + 4 * cq);
-                    acc.x = fmaf(l, t.x, acc.x);
-                    acc.y = fmaf(l, t.y, acc.y);
-                    acc.z = fmaf(l, t.z, acc.z);
-                    acc.w = fmaf(l, t.w, acc.w);
-                }
-            }
-            *reinterpret_cast<float4*>(X + job * 4) = acc;
-        }
-        __syncthreads();
-        for (int job = tid; job < njobs; job += NTHREADS) {
-            const int J = job >> 6, I = J + d, r = (job >> 2) & 15, cq = job & 3;
-            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-            for (int m = 0; m < 16; ++m) {
-                const float l = Lf[(16 * I + r) * LDL + 16 * I + m];  // D_I
-                const float4 x = *reinterpret_cast<const float4*>(X + ((J << 6) + (m << 2) + cq) * 4);
-                acc.x = fmaf(l, x.x, acc.x);
-                acc.y = fmaf(l, x.y, acc.y);
-                acc.z = fmaf(l, x.z, acc.z);
-                acc.w = fmaf(l, x.w, acc.w);
-            }
-            *reinterpret_cast<float4*>(Toff + toff_block(I, J) * 256 + r * 16 + 4 * cq) =
-                make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
-        }
-        __syncthreads();
-    }
-}
-
-// Write chunks [c0, c0 + n) of row r of a swizzled bf16 block from 8*n fp32 values.
-__device__ __forceinline__ void st_chunks_bf16(uint8_t* block, int r, int c0, int n, const float* v) {
-#pragma unroll
-    for (int c = 0; c < n; ++c) {
-        uint4 u;
-        u.x = pack_bf16x2(v[8 * c + 0], v[8 * c + 1]);
-        u.y = pack_bf16x2(v[8 * c + 2], v[8 * c + 3]);
-        u.z = pack_bf16x2(v[8 * c + 4], v[8 * c + 5]);
-        u.w = pack_bf16x2(v[8 * c + 6], v[8 * c + 7]);
-        *reinterpret_cast<uint4*>(block + sw128_off(r, c0 + c)) = u;
-    }
-}
-
-// Split 8*n fp32 values into hi/lo bf16 and write chunks [c0, c0 + n) of row r of two blocks.
-__device__ __forceinline__ void st_chunks_split(uint8_t* hi_block, uint8_t* lo_block, int r, int c0, int n,
-                                                const float* v) {
-#pragma unroll
-    for (int c = 0; c < n; ++c) {
-        float h[8], l[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) split_bf16(v[8 * c + e], h[e], l[e]);
-        uint4 uh, ul;
-        uh.x = pack_bf16x2(h[0], h[1]); uh.y = pack_bf16x2(h[2], h[3]);
-        uh.z = pack_bf16x2(h[4], h[5]); uh.w = pack_bf16x2(h[6], h[7]);
-        ul.x = pack_bf16x2(l[0], l[1]); ul.y = pack_bf16x2(l[2], l[3]);
-        ul.z = pack_bf16x2(l[4], l[5]); ul.w = pack_bf16x2(l[6], l[7]);
-        *reinterpret_cast<uint4*>(hi_block + sw128_off(r, c0 + c)) = uh;
-        *reinterpret_cast<uint4*>(lo_block + sw128_off(r, c0 + c)) = ul;
-    }
-}
 
 template <typename TOut>
 __global__ void __launch_bounds__(NTHREADS, 1)
@@ -461,7 +351,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         tc_fence_before();
         __syncthreads();
-        invert_unit_lower64(Lf, Toff, Xs, tid);
+        invert_unit_lower64<NTHREADS>(Lf, Toff, Xs, tid);
         // ---- T' = T Diag(b gamma / r), T'' = T Diag(c): thread -> row tid/4, 16 columns
         {
             const int i = tid >> 2, qq = tid & 3, I = i >> 4;
@@ -670,11 +560,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
 }
 
-// ---------------------------------------------------------------- host side
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+}  // namespace
 
+// ---------------------------------------------------------------- host side
 EncodeTiledFn get_encode_fn() {
     static EncodeTiledFn fn = nullptr;
     static bool tried = false;
@@ -689,7 +577,6 @@ EncodeTiledFn get_encode_fn() {
     return fn;
 }
 
-// 4-D map over a [B, T, H, 128] bf16 tensor; box = 64 tokens x 64 features of one (b, h).
 bool make_map(CUtensorMap* m, const void* base, int B, int T, int H) {
     EncodeTiledFn enc = get_encode_fn();
     if (!enc) return false;
@@ -702,8 +589,6 @@ bool make_map(CUtensorMap* m, const void* base, int B, int T, int H) {
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
-
-}  // namespace
 
 bool chunk_fwd_tc_supported(const FwdArgs& a) {
     return a.bf16 && a.Dk == 128 && a.Dv == 128 && a.T > 0 && get_encode_fn() != nullptr;
@@ -827,6 +712,15 @@ int choose_nseg(int BH, int NC) {
 
 }  // namespace
 
+cudaError_t launch_seg_scan(const float* S0, const float* MN, float* Sstart, float* S_T, int BH, int nseg,
+                            cudaStream_t st) {
+    const size_t scan_smem = sizeof(float) * (DK * DV + DK * SCAN_LD);
+    cudaError_t e = cudaFuncSetAttribute(seg_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)scan_smem);
+    if (e != cudaSuccess) return e;
+    seg_scan_kernel<<<BH, 256, scan_smem, st>>>(S0, MN, Sstart, S_T, BH, nseg);
+    return cudaGetLastError();
+}
+
 size_t chunk_fwd_tc_segmented_workspace(const FwdArgs& a) {
     if (!(a.bf16 && a.Dk == 128 && a.Dv == 128 && a.T > 0)) return 0;  // shapes of the tensor-core path
     const int NC = (a.T + CH - 1) / CH;
@@ -855,11 +749,7 @@ cudaError_t launch_chunk_fwd_tc_segmented(const FwdArgs& a, void* ws, cudaStream
     p1.kinds = 2;
     cudaError_t e = launch_chunk_fwd_tc(p1, st);
     if (e != cudaSuccess) return e;
-    const size_t scan_smem = sizeof(float) * (DK * DV + DK * SCAN_LD);
-    e = cudaFuncSetAttribute(seg_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)scan_smem);
-    if (e != cudaSuccess) return e;
-    seg_scan_kernel<<<BH, 256, scan_smem, st>>>(a.S0, MN, Sstart, a.S_T, BH, nseg_used);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = launch_seg_scan(a.S0, MN, Sstart, a.S_T, BH, nseg_used, st)) != cudaSuccess) return e;
     FwdArgs p2 = a;
     p2.S0 = Sstart;
     p2.S_T = nullptr;

@@ -64,6 +64,17 @@ size_t chunk_fwd_tc_segmented_workspace(const FwdArgs& a);
 // Segmented forward: per-segment transitions in parallel, a scan over segments, then the
 // outputs of every segment from its true start state.  ws must hold the size above.
 cudaError_t launch_chunk_fwd_tc_segmented(const FwdArgs& a, void* ws, cudaStream_t st);
+// Sequential fp32 scan over segments: S_{s+1} = M_s S_s + N_s per head, recording each
+// segment's start in Sstart [BH, nseg, Dk, Dv] (MN: [2, BH, nseg, Dk, Dv], N first) and the
+// final state in S_T (may be null).
+cudaError_t launch_seg_scan(const float* S0, const float* MN, float* Sstart, float* S_T, int BH, int nseg,
+                            cudaStream_t st);
+// Split tensor-core forward: a chunk-parallel preparation kernel writes every chunk's
+// state-independent operands to the workspace, then a sequential state pass (segmented for
+// long sequences over few heads).  Workspace bytes for these sizes (0: shapes not supported).
+size_t chunk_fwd_split_workspace(const FwdArgs& a);
+cudaError_t launch_chunk_fwd_split(const FwdArgs& a, void* ws, cudaStream_t st);
+cudaError_t split_take_error(cudaStream_t st, unsigned int* flag);
 // Synchronise `st`, then read and clear the device error word of the tensor-core kernels
 // (non-zero when a bounded wait expired).
 cudaError_t tc_take_error(cudaStream_t st, unsigned int* flag);

@@ -1,0 +1,139 @@
+// kla_tc_common.cuh -- pieces shared by the tensor-core chunk kernels: sizes, the blocked
+// 64x64 unit-lower-triangular inverse, swizzled bf16 tile writers and the TMA map builder.
+#pragma once
+
+#include <cuda.h>
+
+#include "kla_sm100.cuh"
+
+namespace kla {
+
+// cuTensorMapEncodeTiled, fetched from the driver at run time (null when there is no driver).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn get_encode_fn();
+// 4-D map over a [B, T, H, 128] bf16 tensor; box = 64 tokens x 64 features of one (b, h),
+// 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, int B, int T, int H);
+
+namespace tcc {
+
+using namespace sm100;
+
+constexpr int DK = 128, DV = 128, CH = 64;
+constexpr int LDL = 68;  // row stride (floats) of the fp32 L/T buffer, 16-B rows
+
+__device__ __forceinline__ size_t tok_index(int b, int t, int h, int T, int H) {
+    return ((size_t)b * T + t) * H + h;
+}
+
+// Off-diagonal 16x16 block (I, J), I > J, of T in the Toff buffer: blocks ordered by
+// distance d = I - J, then by J: (1,0) (2,1) (3,2) (2,0) (3,1) (3,0).
+__device__ __forceinline__ int toff_block(int I, int J) {
+    const int d = I - J;
+    return (d == 1 ? 0 : (d == 2 ? 3 : 5)) + J;
+}
+
+// T = (I + L)^{-1} of the unit lower-triangular 64x64 matrix of Eq. (7), by blockwise
+// forward substitution (Appendix B.2) on 16x16 blocks.  L: fp32, rows of LDL floats,
+// strictly lower (upper part zero).
+//   diagonal blocks  D_I = (I + L_II)^{-1}: column by column (64 threads), written over L_II
+//   off-diagonal     T_IJ = -D_I sum_{K=J}^{I-1} L_IK T_KJ (T_JJ = D_J), by distance
+//                    d = I - J = 1, 2, 3, into Toff (6 blocks of 16x16); L stays intact.
+// X is scratch for 3 x 256 floats.  All NT threads of the CTA must call it.
+template <int NT>
+__device__ __forceinline__ void invert_unit_lower64(float* Lf, float* Toff, float* X, int tid) {
+    if (tid < 64) {
+        const int base = 16 * (tid >> 4), l = tid & 15;
+        float x[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+            for (int j = 0; j + 1 < i; j += 2) {
+                a0 = fmaf(Lf[(base + i) * LDL + base + j], x[j], a0);
+                a1 = fmaf(Lf[(base + i) * LDL + base + j + 1], x[j + 1], a1);
+            }
+            if (i & 1) a0 = fmaf(Lf[(base + i) * LDL + base + i - 1], x[i - 1], a0);
+            x[i] = (i < l) ? 0.f : ((i == l) ? 1.f : -(a0 + a1));
+        }
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) Lf[(base + i) * LDL + base + l] = x[i];
+    }
+    __syncthreads();
+#pragma unroll 1
+    for (int d = 1; d < 4; ++d) {
+        const int njobs = 64 * (4 - d);  // (block, row, column quad)
+        for (int job = tid; job < njobs; job += NT) {
+            const int J = job >> 6, I = J + d, r = (job >> 2) & 15, cq = job & 3;
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int K = J; K < I; ++K) {
+                const float* tk = (K == J) ? (Lf + 16 * J * LDL + 16 * J) : (Toff + toff_block(K, J) * 256);
+                const int ldt = (K == J) ? LDL : 16;
+#pragma unroll
+                for (int m = 0; m < 16; ++m) {
+                    const float l = Lf[(16 * I + r) * LDL + 16 * K + m];
+                    const float4 t = *reinterpret_cast<const float4*>(tk + m * ldt + 4 * cq);
+                    acc.x = fmaf(l, t.x, acc.x);
+                    acc.y = fmaf(l, t.y, acc.y);
+                    acc.z = fmaf(l, t.z, acc.z);
+                    acc.w = fmaf(l, t.w, acc.w);
+                }
+            }
+            *reinterpret_cast<float4*>(X + job * 4) = acc;
+        }
+        __syncthreads();
+        for (int job = tid; job < njobs; job += NT) {
+            const int J = job >> 6, I = J + d, r = (job >> 2) & 15, cq = job & 3;
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int m = 0; m < 16; ++m) {
+                const float l = Lf[(16 * I + r) * LDL + 16 * I + m];  // D_I
+                const float4 x = *reinterpret_cast<const float4*>(X + ((J << 6) + (m << 2) + cq) * 4);
+                acc.x = fmaf(l, x.x, acc.x);
+                acc.y = fmaf(l, x.y, acc.y);
+                acc.z = fmaf(l, x.z, acc.z);
+                acc.w = fmaf(l, x.w, acc.w);
+            }
+            *reinterpret_cast<float4*>(Toff + toff_block(I, J) * 256 + r * 16 + 4 * cq) =
+                make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
+        }
+        __syncthreads();
+    }
+}
+
+// Write chunks [c0, c0 + n) of row r of a swizzled bf16 block from 8*n fp32 values.
+__device__ __forceinline__ void st_chunks_bf16(uint8_t* block, int r, int c0, int n, const float* v) {
+#pragma unroll
+    for (int c = 0; c < n; ++c) {
+        uint4 u;
+        u.x = pack_bf16x2(v[8 * c + 0], v[8 * c + 1]);
+        u.y = pack_bf16x2(v[8 * c + 2], v[8 * c + 3]);
+        u.z = pack_bf16x2(v[8 * c + 4], v[8 * c + 5]);
+        u.w = pack_bf16x2(v[8 * c + 6], v[8 * c + 7]);
+        *reinterpret_cast<uint4*>(block + sw128_off(r, c0 + c)) = u;
+    }
+}
+
+// Split 8*n fp32 values into hi/lo bf16 and write chunks [c0, c0 + n) of row r of two blocks.
+__device__ __forceinline__ void st_chunks_split(uint8_t* hi_block, uint8_t* lo_block, int r, int c0, int n,
+                                                const float* v) {
+#pragma unroll
+    for (int c = 0; c < n; ++c) {
+        float h[8], l[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) split_bf16(v[8 * c + e], h[e], l[e]);
+        uint4 uh, ul;
+        uh.x = pack_bf16x2(h[0], h[1]); uh.y = pack_bf16x2(h[2], h[3]);
+        uh.z = pack_bf16x2(h[4], h[5]); uh.w = pack_bf16x2(h[6], h[7]);
+        ul.x = pack_bf16x2(l[0], l[1]); ul.y = pack_bf16x2(l[2], l[3]);
+        ul.z = pack_bf16x2(l[4], l[5]); ul.w = pack_bf16x2(l[6], l[7]);
+        *reinterpret_cast<uint4*>(hi_block + sw128_off(r, c0 + c)) = uh;
+        *reinterpret_cast<uint4*>(lo_block + sw128_off(r, c0 + c)) = ul;
+    }
+}
+
+}  // namespace tcc
+}  // namespace kla

@@ -84,8 +84,14 @@ int kla_version(void);
  *   S_T          out  [B,H,Dk,Dv] fp32 final state, or NULL.  May alias S0.
  *   S_chunks     out  [B,H,ceil(T/chunk),Dk,Dv] fp32 state at the start of every chunk, or
  *                     NULL.  Passing it to kla_chunk_bwd saves the backward's recompute.
- *   ws, ws_bytes      caller workspace of at least kla_chunk_fwd_workspace() bytes (the
- *                     forward currently needs none; ws may then be NULL).
+ *   ws, ws_bytes      caller workspace (device memory, 16-byte aligned, owned by the caller,
+ *                     contents need not be initialised), or NULL.  With at least
+ *                     kla_chunk_fwd_workspace() bytes, bf16 inputs with Dk == Dv == 128 run the
+ *                     split path: a chunk-parallel kernel stores every chunk's state-independent
+ *                     operands there (about 97 KiB per chunk and head), then a sequential state
+ *                     pass consumes them (segmented, for long sequences over few heads).  With
+ *                     NULL or a smaller buffer the forward still runs, as one fused kernel per
+ *                     head.  The workspace must not be shared with a concurrent call.
  * Returns KLA_OK or an error status; on error nothing is launched.
  */
 size_t kla_chunk_fwd_workspace(int B, int T, int H, int Dk, int Dv, int chunk, int dtype);

@@ -137,7 +137,7 @@ def test_fwd_segmented_long_sequence(kla, oracle_mod, T, H, s0):
     d = {k: (v.cuda() if v is not None else None) for k, v in inp.items()}
     o, ST, Sc = kla.chunk_fwd(d["q"], d["k"], d["v"], d["eta"], d["g"], 1e-6, d["S0"], save_chunk_states=True)
     o1, ST1, Sc1 = kla.chunk_fwd(d["q"], d["k"], d["v"], d["eta"], d["g"], 1e-6, d["S0"], save_chunk_states=True,
-                                 segmented=False)
+                                 fused=True)
     torch.cuda.synchronize()
     kla.check_device_error()
     ro, rST = oracle_mod.forward(*(np64(inp[k]) for k in ("q", "k", "v", "eta", "g")), 1e-6, np64(inp["S0"]))
@@ -145,6 +145,33 @@ def test_fwd_segmented_long_sequence(kla, oracle_mod, T, H, s0):
     assert rel_err(ST, rST) <= 2e-2
     assert rel_err(o, np64(o1)) <= 1e-2
     assert rel_err(Sc, np64(Sc1)) <= 1e-2
+
+
+@pytest.mark.parametrize("B,T,H,s0,g_lo,out_bf16", [(1, 1, 1, True, -0.5, False), (1, 64, 2, False, -0.5, False),
+                                                    (2, 191, 3, True, -0.05, True), (1, 700, 1, True, -3.0, False)])
+def test_fwd_split_and_fused_paths_agree(kla, oracle_mod, B, T, H, s0, g_lo, out_bf16):
+    """The split path (chunk-parallel preparation + state pass, with the workspace) and the
+    fused one-kernel path both match the oracle, including the per-chunk states."""
+    inp = small_inputs(B, T, H, 128, 128, "bf16", seed=T + 11 * H, s0=s0, g_lo=g_lo)
+    d = {k: (v.cuda() if v is not None else None) for k, v in inp.items()}
+    odt = torch.bfloat16 if out_bf16 else torch.float32
+    outs = {}
+    for fused in (False, True):
+        outs[fused] = kla.chunk_fwd(d["q"], d["k"], d["v"], d["eta"], d["g"], 1e-6, d["S0"], save_chunk_states=True,
+                                    out_dtype=odt, fused=fused)
+    torch.cuda.synchronize()
+    kla.check_device_error()
+    ro, rST = oracle_mod.forward(*(np64(inp[k]) for k in ("q", "k", "v", "eta", "g")), 1e-6, np64(inp["S0"]))
+    for fused, (o, ST, Sc) in outs.items():
+        if out_bf16:  # a bf16 store is the fp32 result rounded once
+            o32 = kla.chunk_fwd(d["q"], d["k"], d["v"], d["eta"], d["g"], 1e-6, d["S0"], fused=fused)[0]
+            torch.testing.assert_close(o, o32.to(torch.bfloat16), rtol=0, atol=0)
+            o = o32
+        assert rel_err(o, ro) <= 2e-2, fused
+        assert rel_err(ST, rST) <= 2e-2, fused
+    assert rel_err(outs[False][2], np64(outs[True][2])) <= 1e-2  # chunk-start states
+    if s0:
+        torch.testing.assert_close(outs[False][2][:, :, 0], d["S0"])  # chunk 0 starts from S0
 
 
 def test_fwd_state_passing_equals_one_call(kla):
