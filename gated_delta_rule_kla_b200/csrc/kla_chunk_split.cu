@@ -364,16 +364,24 @@ done:
 // =====================================================================================
 // State pass: one CTA per (b, h) [segment, kind], chunks in order.  Warp-specialised:
 // warps 0-7 run the epilogues (thread pair = one TMEM lane = one dv column, the two threads
-// splitting the columns), warp 8 issues the MMAs.  The two sides meet on mbarriers:
+// splitting the columns), warp 8 issues the MMAs, warp 9 moves the stages in and the outputs
+// out.  They meet on mbarriers:
 //   issuer -> epilogue: bar_u (U^T ready in TMEM), bar_s (S^T updated), bar_o (O1, O2 ready)
-//   epilogue -> issuer: s_ready (S hi/lo written), u_ready (U hi/lo written), o_free (O read)
-// so an MMA issue, which blocks its thread while the tensor pipe drains, never delays an
-// epilogue.  Per chunk c the issuer runs  U(c) | O1(c) | S(c) O2(c)  and the epilogue warps
-//   U epi(c) -> S hi/lo(c+1) [releases U(c+1)] -> S master rescale -> O epi(c) -> o via TMA.
+//   epilogue -> issuer: s_ready[2], u_ready[2] (each half of the S, U operands written),
+//                       o_free (O read and the o tile staged)
+// bar_o and o_free, which the loader also waits on, come one per stage: a phase of either
+// cannot come round again before the loader has refilled that stage, so the loader's parity
+// waits never alias even when it runs late.
+// An MMA issue blocks its thread while the tensor pipe drains, so no epilogue work sits on the
+// issuing warp; and the S and U operands are released in halves, so the first K steps of the
+// MMA that consumes them run while the epilogue finishes the second half.  Per chunk c:
+//   issuer    U(c) [2 halves] | O1(c) | S(c) [2 halves] O2(c)
+//   epilogue  U epi(c) -> S hi/lo(c+1) -> master rescale -> O epi(c)
+//   loader    refill of chunk c's stage with chunk c + 2 (Ktil, P, U' once chunk c's MMAs are
+//             done; Q, W and scalars once the o tile has left by TMA store)
 // =====================================================================================
-constexpr int ST = 288;
-constexpr int kIssuerWarp = 8;
-constexpr int kLoader = 32;           // thread that issues every load and store of the stage
+constexpr int ST = 320;
+constexpr int kIssuerWarp = 8, kLoaderWarp = 9;
 constexpr uint32_t S_STAGE = 114688;  // Q 16 KB + the record's tiles (96 KB)
 constexpr uint32_t SO_Q = 0, SO_W = 16384, SO_KT = 32768, SO_KTLO = 49152, SO_P = 65536, SO_PLO = 73728,
                    SO_UP = 81920;
@@ -390,36 +398,22 @@ constexpr uint32_t TM_S = 0, TM_SH = 128, TM_SL = 192, TM_U = 256, TM_UH = 320, 
 
 struct StateMisc {
     uint64_t full[2];
-    uint64_t bar_u, bar_s, bar_o;        // tcgen05.commit arrivals
-    uint64_t s_ready, u_ready, o_free;   // one arrival per epilogue warp
+    uint64_t bar_u, bar_s, bar_o[2];              // tcgen05.commit arrivals (bar_o per stage)
+    uint64_t s_ready[2], u_ready[2], o_free[2];   // one arrival per epilogue warp (o_free per stage)
     uint32_t tmem_base, abort;
     float gsum[2];
 };
 
-// Pack 32 fp32 values (consecutive K indices) into 16 bf16x2 hi words and 16 lo words.
-__device__ __forceinline__ void split_pack32(const float (&x)[32], uint32_t (&hp)[16], uint32_t (&lp)[16]) {
+// Split fp32 values into bf16 hi + lo words, two consecutive K indices per 32-bit word (the
+// lower index in the low half): hi = rn(x), lo = rn(x - hi).
+template <int N>
+__device__ __forceinline__ void split_pack(const float* x, uint32_t* hp, uint32_t* lp) {
 #pragma unroll
-    for (int e = 0; e < 16; ++e) {
-        float h0, l0, h1, l1;
-        split_bf16(x[2 * e], h0, l0);
-        split_bf16(x[2 * e + 1], h1, l1);
-        hp[e] = pack_bf16x2(h0, h1);
-        lp[e] = pack_bf16x2(l0, l1);
+    for (int e = 0; e < N / 2; ++e) {
+        const uint32_t hw = pack_bf16x2(x[2 * e], x[2 * e + 1]);
+        hp[e] = hw;
+        lp[e] = pack_bf16x2(x[2 * e] - __uint_as_float(hw << 16), x[2 * e + 1] - __uint_as_float(hw & 0xffff0000u));
     }
-}
-
-// Barrier over the 256 epilogue threads (named barrier 1) returning the OR of `pred`.
-__device__ __forceinline__ bool epi_bar_or(bool pred) {
-    uint32_t r;
-    asm volatile(
-        "{\n\t.reg .pred p, q;\n\t"
-        "setp.ne.b32 p, %1, 0;\n\t"
-        "bar.red.or.pred q, 1, 256, p;\n\t"
-        "selp.u32 %0, 1, 0, q;\n\t}"
-        : "=r"(r)
-        : "r"((uint32_t)pred)
-        : "memory");
-    return r != 0;
 }
 
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
@@ -439,6 +433,13 @@ __device__ __forceinline__ void tma_store_4d(const void* tmap, uint32_t src, int
 __device__ __forceinline__ void bulk_wait_read_all() {
     asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
+// Epilogue warp: make this warp's TMEM stores visible to the MMA issuer, then arrive once.
+__device__ __forceinline__ void epi_signal(uint32_t bar, int tid) {
+    tmem_st_wait();
+    tc_fence_before();
+    __syncwarp();
+    if ((tid & 31) == 0) mbar_arrive(bar);
+}
 
 template <typename TOut>
 __global__ void __launch_bounds__(ST, 1)
@@ -448,7 +449,7 @@ __global__ void __launch_bounds__(ST, 1)
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     StateMisc* ms = reinterpret_cast<StateMisc*>(sm + S_MISC);
 
-    const int tid = threadIdx.x, warp = tid >> 5;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int row = tid & 127;        // TMEM lane = dv (epilogue warps)
     const int ch = (tid >> 7) & 1;    // half of every epilogue's columns
     const int H = a.H, T = a.T;
@@ -464,9 +465,9 @@ __global__ void __launch_bounds__(ST, 1)
     const int NC = c1 > c0 ? c1 - c0 : 0;
     const uint32_t sbase = smem_u32(sm);
     const uint32_t bar_full0 = smem_u32(&ms->full[0]);
-    const uint32_t bar_u = smem_u32(&ms->bar_u), bar_s = smem_u32(&ms->bar_s), bar_o = smem_u32(&ms->bar_o);
-    const uint32_t s_ready = smem_u32(&ms->s_ready), u_ready = smem_u32(&ms->u_ready),
-                   o_free = smem_u32(&ms->o_free);
+    const uint32_t bar_u = smem_u32(&ms->bar_u), bar_s = smem_u32(&ms->bar_s), bar_o0 = smem_u32(&ms->bar_o[0]);
+    const uint32_t s_ready0 = smem_u32(&ms->s_ready[0]), u_ready0 = smem_u32(&ms->u_ready[0]),
+                   o_free0 = smem_u32(&ms->o_free[0]);
     const float* S0p = (a.S0 && !ident)
                            ? a.S0 + (size_t)(segmented ? head_idx * nseg + seg : head_idx) * DK * DV
                            : nullptr;
@@ -481,14 +482,16 @@ __global__ void __launch_bounds__(ST, 1)
         mbar_init(bar_full0 + 8, 1);
         mbar_init(bar_u, 1);
         mbar_init(bar_s, 1);
-        mbar_init(bar_o, 1);
-        mbar_init(s_ready, 8);
-        mbar_init(u_ready, 8);
-        mbar_init(o_free, 8);
+        mbar_init(bar_o0, 1);
+        mbar_init(bar_o0 + 8, 1);
+        mbar_init(s_ready0, 8);
+        mbar_init(s_ready0 + 8, 8);
+        mbar_init(u_ready0, 8);
+        mbar_init(u_ready0 + 8, 8);
+        mbar_init(o_free0, 8);
+        mbar_init(o_free0 + 8, 8);
         ms->abort = 0;
         fence_mbar_init();
-        prefetch_tmap(&tm_q);
-        if (write_o) prefetch_tmap(&tm_o);
     }
     if (warp == 0) {
         tmem_alloc(smem_u32(&ms->tmem_base), 512);
@@ -498,7 +501,7 @@ __global__ void __launch_bounds__(ST, 1)
         const bool live = NC > 0 && c0 * CH + tid < T;
         const float gv = live ? a.g[tok_index(b, c0 * CH + tid, h, T, H)] : 0.f;
         const float sg = warp_sum(gv);
-        if ((tid & 31) == 0) ms->gsum[warp] = sg;
+        if (lane == 0) ms->gsum[warp] = sg;
     }
     tc_fence_before();
     __syncthreads();
@@ -506,61 +509,99 @@ __global__ void __launch_bounds__(ST, 1)
     const uint32_t tmem = ms->tmem_base;
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
 
-    // Stage loads: the early part (Ktil, P, U') and the late part (Q, W, scalars) of chunk c.
-    auto load_early = [&](int c, int st) {
-        const uint32_t bar = bar_full0 + 8 * st;
-        const uint32_t base = sbase + st * S_STAGE;
-        const uint8_t* rec = recs + ((size_t)head_idx * NCtot + c) * REC_BYTES;
-        mbar_expect_tx_only(bar, EARLY_BYTES);
-#pragma unroll
-        for (int p = 0; p < 5; ++p) bulk_load(base + SO_KT + p * 16384, rec + REC_KT + p * 16384, 16384, bar);
-    };
-    auto load_late = [&](int c, int st) {
-        const uint32_t bar = bar_full0 + 8 * st;
-        const uint32_t base = sbase + st * S_STAGE;
-        const uint8_t* rec = recs + ((size_t)head_idx * NCtot + c) * REC_BYTES;
-        mbar_expect_tx(bar, LATE_BYTES);  // the one arrival of the phase
-        tma_load_4d(base + SO_Q, &tm_q, bar, 0, h, c * CH, b);
-        tma_load_4d(base + SO_Q + 8192, &tm_q, bar, 64, h, c * CH, b);
-        bulk_load(base + SO_W, rec + REC_W, 16384, bar);
-        bulk_load(sbase + S_SC + st * REC_SCB, rec + REC_SC, REC_SCB, bar);
-    };
-    int issued = c0 - 1;  // (loader) last chunk whose late part was requested
-    if (tid == kLoader) {
-        for (int i = 0; i < min(NC, 2); ++i) {
-            load_early(c0 + i, i);
-            load_late(c0 + i, i);
-            issued = c0 + i;
-        }
-    }
-    __syncwarp();
-
     bool aborted = false;
-    if (warp == kIssuerWarp) {
+    if (warp == kLoaderWarp) {
+        // ================================ loader ================================
+        if (lane == 0) {
+            prefetch_tmap(&tm_q);
+            if (write_o) prefetch_tmap(&tm_o);
+            // The early part (Ktil, P, U') and the late part (Q, W, scalars) of chunk c; the
+            // late part carries the phase's one arrival.
+            auto load_early = [&](int c, int st) {
+                const uint32_t bar = bar_full0 + 8 * st;
+                const uint32_t base = sbase + st * S_STAGE;
+                const uint8_t* rec = recs + ((size_t)head_idx * NCtot + c) * REC_BYTES;
+                mbar_expect_tx_only(bar, EARLY_BYTES);
+#pragma unroll
+                for (int p = 0; p < 5; ++p)
+                    bulk_load(base + SO_KT + p * 16384, rec + REC_KT + p * 16384, 16384, bar);
+            };
+            auto load_late = [&](int c, int st) {
+                const uint32_t bar = bar_full0 + 8 * st;
+                const uint32_t base = sbase + st * S_STAGE;
+                const uint8_t* rec = recs + ((size_t)head_idx * NCtot + c) * REC_BYTES;
+                mbar_expect_tx(bar, LATE_BYTES);
+                tma_load_4d(base + SO_Q, &tm_q, bar, 0, h, c * CH, b);
+                tma_load_4d(base + SO_Q + 8192, &tm_q, bar, 64, h, c * CH, b);
+                bulk_load(base + SO_W, rec + REC_W, 16384, bar);
+                bulk_load(sbase + S_SC + st * REC_SCB, rec + REC_SC, REC_SCB, bar);
+            };
+            int early = c0 - 1, late = c0 - 1;  // last chunk of each part requested
+            for (int i = 0; i < min(NC, 2); ++i) {
+                load_early(c0 + i, i);
+                load_late(c0 + i, i);
+                early = late = c0 + i;
+            }
+            for (int c = c0; c < c1; ++c) {
+                const int lc = c - c0, st = lc & 1;
+                // every MMA of chunk c done: Ktil, P, U' of its stage can take chunk c + 2
+                if (!mbar_wait_bounded(bar_o0 + 8 * st, (lc >> 1) & 1, kWaitNs)) { aborted = true; break; }
+                if (c + 2 < c1) {
+                    load_early(c + 2, st);
+                    early = c + 2;
+                }
+                // o tile staged and every scalar read: store it, then the rest of the stage
+                if (!mbar_wait_bounded(o_free0 + 8 * st, (lc >> 1) & 1, kWaitNs)) { aborted = true; break; }
+                if (write_o) {
+                    tma_store_4d(&tm_o, sbase + st * S_STAGE + SO_Q, 0, h, c * CH, b);
+                    bulk_commit();
+                    bulk_wait_read_all();
+                }
+                if (c + 2 < c1) {
+                    load_late(c + 2, st);
+                    late = c + 2;
+                }
+            }
+            if (aborted) {
+                atomicOr(&ms->abort, 1u);
+                // let loads that may still be landing in shared memory finish (a phase whose late
+                // part was never requested cannot complete: wait out its early bytes instead)
+                for (int cc = max(c0, late - 1); cc <= early; ++cc)
+                    (void)mbar_wait_bounded(bar_full0 + 8 * ((cc - c0) & 1), ((cc - c0) >> 1) & 1,
+                                            cc <= late ? kWaitNs : 20000000ull);
+            }
+            bulk_wait_all();
+        }
+        __syncwarp();
+    } else if (warp == kIssuerWarp) {
         // ================================ MMA issuer ================================
-        if ((tid & 31) == 0) {
+        if (lane == 0) {
             const uint32_t iu = idesc_bf16(128, 64, false, true);
             const uint32_t io = idesc_bf16(128, 64, false, false);
             const uint32_t is = idesc_bf16(128, 128, false, true);
             for (int c = c0; c < c1 && !aborted; ++c) {
                 const int lc = c - c0, st = lc & 1;
                 const uint32_t stg = sbase + st * S_STAGE;
-                if (!mbar_wait_bounded(bar_full0 + 8 * st, (lc >> 1) & 1, kWaitNs) ||
-                    !mbar_wait_bounded(s_ready, lc & 1, kWaitNs)) {
-                    aborted = true;
-                    break;
+                if (!mbar_wait_bounded(bar_full0 + 8 * st, (lc >> 1) & 1, kWaitNs)) { aborted = true; break; }
+                // U^T = -(S^T W^T) (the record holds -W^T; U' is added in the epilogue).  K steps
+                // {0,1,4,5} read the first half of each thread's S columns, {2,3,6,7} the second.
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    if (!mbar_wait_bounded(s_ready0 + 8 * half, lc & 1, kWaitNs)) { aborted = true; break; }
+                    tc_fence_after();
+#pragma unroll
+                    for (int part = 0; part < 2; ++part)
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const int s = 2 * half + (j & 1) + 4 * (j >> 1);
+                            mma_bf16_ts(tmem + TM_U, tmem + (part ? TM_SL : TM_SH) + 8 * s,
+                                        smem_desc(stg + SO_W + s * 2048, 8192, 1024), iu, (half | part | j) > 0);
+                        }
                 }
-                tc_fence_after();
-                // U^T = -(S^T W^T)   (the record holds -W^T; U' is added in the epilogue)
-#pragma unroll
-                for (int part = 0; part < 2; ++part)
-#pragma unroll
-                    for (int s = 0; s < 8; ++s)
-                        mma_bf16_ts(tmem + TM_U, tmem + (part ? TM_SL : TM_SH) + 8 * s,
-                                    smem_desc(stg + SO_W + s * 2048, 8192, 1024), iu, (part | s) > 0);
+                if (aborted) break;
                 mma_commit(bar_u);
                 // O1 = S^T Q^T, once the previous chunk's outputs are read
-                if (lc > 0 && !mbar_wait_bounded(o_free, (lc - 1) & 1, kWaitNs)) {
+                if (lc > 0 && !mbar_wait_bounded(o_free0 + 8 * (st ^ 1), ((lc - 1) >> 1) & 1, kWaitNs)) {
                     aborted = true;
                     break;
                 }
@@ -572,29 +613,34 @@ __global__ void __launch_bounds__(ST, 1)
                         mma_bf16_ts(tmem + TM_O1, tmem + (part ? TM_SL : TM_SH) + 8 * s,
                                     smem_desc(stg + SO_Q + (s >> 2) * 8192 + (s & 3) * 32, 16, 1024), io,
                                     (part | s) > 0);
-                // S^T += U^T Ktil (N = 128), then O2 = U^T P^T; hi x hi, hi x lo, lo x hi
-                if (!mbar_wait_bounded(u_ready, lc & 1, kWaitNs)) {
-                    aborted = true;
-                    break;
-                }
-                tc_fence_after();
+                // S^T += U^T Ktil (N = 128): K steps {0,2} (first half of each thread's tokens),
+                // then {1,3}; products hi x hi, hi x lo, lo x hi
                 const uint32_t ua[3] = {TM_UH, TM_UH, TM_UL};
                 const uint32_t kb[3] = {stg + SO_KT, stg + SO_KTLO, stg + SO_KT};
                 const uint32_t pb[3] = {stg + SO_P, stg + SO_PLO, stg + SO_P};
 #pragma unroll
-                for (int p = 0; p < 3; ++p)
+                for (int half = 0; half < 2; ++half) {
+                    if (!mbar_wait_bounded(u_ready0 + 8 * half, lc & 1, kWaitNs)) { aborted = true; break; }
+                    tc_fence_after();
 #pragma unroll
-                    for (int s = 0; s < 4; ++s)
-                        mma_bf16_ts(tmem + TM_S, tmem + ua[p] + 8 * s, smem_desc(kb[p] + s * 2048, 8192, 1024), is,
-                                    1);
+                    for (int p = 0; p < 3; ++p)
+#pragma unroll
+                        for (int j = 0; j < 2; ++j) {
+                            const int s = half + 2 * j;
+                            mma_bf16_ts(tmem + TM_S, tmem + ua[p] + 8 * s, smem_desc(kb[p] + s * 2048, 8192, 1024),
+                                        is, 1);
+                        }
+                }
+                if (aborted) break;
                 mma_commit(bar_s);
+                // O2 = U^T P^T
 #pragma unroll
                 for (int p = 0; p < 3; ++p)
 #pragma unroll
                     for (int s = 0; s < 4; ++s)
                         mma_bf16_ts(tmem + TM_O2, tmem + ua[p] + 8 * s, smem_desc(pb[p] + s * 32, 16, 1024), io,
                                     (p | s) > 0);
-                mma_commit(bar_o);
+                mma_commit(bar_o0 + 8 * st);
             }
             if (aborted) atomicOr(&ms->abort, 1u);
         }
@@ -616,49 +662,48 @@ __global__ void __launch_bounds__(ST, 1)
                     for (int e = 0; e < 32; ++e) Sc[((size_t)c0 * DK + dk0 + e) * DV + row] = x[e];
                 }
                 uint32_t hp[16], lp[16];
-                split_pack32(x, hp, lp);
+                split_pack<32>(x, hp, lp);
                 tmem_st16u(tmem + lane_base + TM_SH + 32 * ch + 16 * q2, hp);
                 tmem_st16u(tmem + lane_base + TM_SL + 32 * ch + 16 * q2, lp);
 #pragma unroll
                 for (int e = 0; e < 32; ++e) x[e] *= g0;
                 tmem_st32(tmem + lane_base + TM_S + 64 * ch + 32 * q2, x);
             }
-            tmem_st_wait();
-            tc_fence_before();
-            __syncwarp();
-            if ((tid & 31) == 0) mbar_arrive(s_ready);
+            epi_signal(s_ready0, tid);
+            if (lane == 0) mbar_arrive(s_ready0 + 8);
         }
         for (int c = c0; c < c1; ++c) {
             const int lc = c - c0, st = lc & 1;
             const uint8_t* stg_p = sm + st * S_STAGE;
             const bool has_next = c + 1 < c1;
-            // ---- U epilogue: U = U' + acc, to bf16 hi/lo A operands (thread = dv, 32 tokens)
+            // ---- U epilogue: U = U' + acc to bf16 hi/lo A operands (thread = dv, tokens
+            //      32 ch .. + 32), released in two halves of 16 tokens
             {
                 const bool ok = mbar_wait_bounded(bar_u, lc & 1, kWaitNs);
-                if (epi_bar_or(!ok)) { aborted = true; break; }
+                if (__any_sync(0xffffffffu, !ok)) { aborted = true; break; }
                 tc_fence_after();
                 float x[32];
                 tmem_ld32(tmem + lane_base + TM_U + 32 * ch, x);
                 tmem_ld_wait();
-                if (!ident) {
-                    const float* up = reinterpret_cast<const float*>(stg_p + SO_UP);
+                const float* up = reinterpret_cast<const float*>(stg_p + SO_UP);
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) x[e] += up[(32 * ch + e) * DV + row];
+                for (int half = 0; half < 2; ++half) {
+                    if (!ident) {
+#pragma unroll
+                        for (int e = 16 * half; e < 16 * half + 16; ++e) x[e] += up[(32 * ch + e) * DV + row];
+                    }
+                    uint32_t hp[8], lp[8];
+                    split_pack<16>(x + 16 * half, hp, lp);
+                    tmem_st8u(tmem + lane_base + TM_UH + 16 * ch + 8 * half, hp);
+                    tmem_st8u(tmem + lane_base + TM_UL + 16 * ch + 8 * half, lp);
+                    epi_signal(u_ready0 + 8 * half, tid);  // the first also covers the master rescale
                 }
-                uint32_t hp[16], lp[16];
-                split_pack32(x, hp, lp);
-                tmem_st16u(tmem + lane_base + TM_UH + 16 * ch, hp);
-                tmem_st16u(tmem + lane_base + TM_UL + 16 * ch, lp);
-                tmem_st_wait();  // also covers the previous chunk's master rescale
-                tc_fence_before();
-                __syncwarp();
-                if ((tid & 31) == 0) mbar_arrive(u_ready);
             }
-            // ---- state epilogue: S_{c+1} to hi/lo (releases U(c+1)), then the fp32 master
-            //      pre-scaled by the next gamma_last
+            // ---- state epilogue: S_{c+1} to hi/lo in two halves (releasing U(c+1)), then the
+            //      fp32 master pre-scaled by the next gamma_last
             {
                 const bool ok = mbar_wait_bounded(bar_s, lc & 1, kWaitNs);
-                if (epi_bar_or(!ok)) { aborted = true; break; }
+                if (__any_sync(0xffffffffu, !ok)) { aborted = true; break; }
                 tc_fence_after();
                 if (has_next) {
                     float x0[32], x1[32];
@@ -667,17 +712,15 @@ __global__ void __launch_bounds__(ST, 1)
                     tmem_ld_wait();
                     {
                         uint32_t hp[16], lp[16];
-                        split_pack32(x0, hp, lp);
+                        split_pack<32>(x0, hp, lp);
                         tmem_st16u(tmem + lane_base + TM_SH + 32 * ch, hp);
                         tmem_st16u(tmem + lane_base + TM_SL + 32 * ch, lp);
-                        split_pack32(x1, hp, lp);
+                        epi_signal(s_ready0, tid);
+                        split_pack<32>(x1, hp, lp);
                         tmem_st16u(tmem + lane_base + TM_SH + 32 * ch + 16, hp);
                         tmem_st16u(tmem + lane_base + TM_SL + 32 * ch + 16, lp);
+                        epi_signal(s_ready0 + 8, tid);
                     }
-                    tmem_st_wait();
-                    tc_fence_before();
-                    __syncwarp();
-                    if ((tid & 31) == 0) mbar_arrive(s_ready);
                     if (Sc) {
 #pragma unroll
                         for (int e = 0; e < 32; ++e) {
@@ -696,14 +739,11 @@ __global__ void __launch_bounds__(ST, 1)
                 }
             }
             // ---- output epilogue: o = gamma o O1 + O2 staged as [token][dv] over the consumed
-            //      Q and W tiles, then one TMA store
+            //      Q and W tiles; the loader stores it
             {
-                const bool ok = mbar_wait_bounded(bar_o, lc & 1, kWaitNs);
-                if (epi_bar_or(!ok)) { aborted = true; break; }
+                const bool ok = mbar_wait_bounded(bar_o0 + 8 * st, (lc >> 1) & 1, kWaitNs);
+                if (__any_sync(0xffffffffu, !ok)) { aborted = true; break; }
                 tc_fence_after();
-                // every MMA of chunk c is done: Ktil, P, U' of this stage can take chunk c + 2
-                if (tid == kLoader && c + 2 < c1) load_early(c + 2, st);
-                __syncwarp();
                 if (write_o) {
                     const float* gm = reinterpret_cast<const float*>(sm + S_SC + st * REC_SCB);
                     TOut* stage_o = reinterpret_cast<TOut*>(sm + st * S_STAGE + SO_Q);
@@ -720,34 +760,15 @@ __global__ void __launch_bounds__(ST, 1)
                 }
                 tc_fence_before();
                 __syncwarp();
-                if ((tid & 31) == 0) mbar_arrive(o_free);
-                if (tid == kLoader) {
-                    if (!mbar_wait_bounded(o_free, lc & 1, kWaitNs)) {
-                        atomicOr(&ms->abort, 1u);
-                    } else {
-                        if (write_o) {
-                            tma_store_4d(&tm_o, sbase + st * S_STAGE + SO_Q, 0, h, c * CH, b);
-                            bulk_commit();
-                            bulk_wait_read_all();
-                        }
-                        if (c + 2 < c1) {
-                            load_late(c + 2, st);
-                            issued = c + 2;
-                        }
-                    }
-                }
-                __syncwarp();
+                if (lane == 0) mbar_arrive(o_free0 + 8 * st);
             }
         }
+        if (aborted && lane == 0) atomicOr(&ms->abort, 1u);
     }
 
     __syncthreads();
-    if (aborted || ms->abort) {
+    if (ms->abort) {
         if (tid == 0) atomicOr(&g_split_error, 1u);
-        if (tid == kLoader) {  // let loads that may still be landing in shared memory finish
-            for (int cc = max(c0, issued - 1); cc <= issued; ++cc)
-                (void)mbar_wait_bounded(bar_full0 + 8 * ((cc - c0) & 1), ((cc - c0) >> 1) & 1, kWaitNs);
-        }
     } else if (NC > 0 && warp < kIssuerWarp && STp) {
         tc_fence_after();
 #pragma unroll 1
@@ -760,7 +781,6 @@ __global__ void __launch_bounds__(ST, 1)
             for (int e = 0; e < 32; ++e) STp[(size_t)(dk0 + e) * DV + row] = x[e];
         }
     }
-    bulk_wait_all();  // stores of this thread complete before exit
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
