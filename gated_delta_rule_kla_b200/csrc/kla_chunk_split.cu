@@ -60,7 +60,7 @@ constexpr uint32_t P_V = 32768;    // V tile (16 KB), later -W^T
 constexpr uint32_t P_P = 49152;    // P hi/lo (16 KB)
 constexpr uint32_t P_Z = 65536;    // L/T fp32 -> T' T'' hi/lo -> Ktil hi/lo (32 KB)
 constexpr uint32_t P_MISC = 98304;
-constexpr uint32_t P_SMEM = P_MISC + 3072 + 1024;
+constexpr uint32_t P_SMEM = P_MISC + 4096 + 1024;
 constexpr uint32_t PM_G = 0, PM_W = 64, PM_U = 128;  // TMEM columns (256 allocated)
 
 struct PrepMisc {
@@ -68,9 +68,10 @@ struct PrepMisc {
     uint32_t tmem_base, pad[3];
     float sc[128];  // record scalars: gamma[64], gamma_last(next chunk)
     float G[CH], gam[CH], del[CH], bco[CH], cco[CH], invr[CH], graw[CH], eta[CH], pk[CH];
+    float wsc[CH];  // b gamma / r: column scale of T'
     float gsum[2], grange;
 };
-static_assert(sizeof(PrepMisc) <= 3072, "prep scalars");
+static_assert(sizeof(PrepMisc) <= 4096, "prep scalars");
 
 __global__ void __launch_bounds__(PT, 2)
     chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -78,9 +79,8 @@ __global__ void __launch_bounds__(PT, 2)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     PrepMisc* ms = reinterpret_cast<PrepMisc*>(sm + P_MISC);
-    float* Lf = reinterpret_cast<float*>(sm + P_Z);
-    float* Toff = Lf + 64 * LDL;
-    float* Xs = Toff + 6 * 256;
+    float* Lf = reinterpret_cast<float*>(sm + P_Z);  // 64 x LDL fp32: L, then T in place
+    float* Xs = Lf + 64 * LDL;                         // 1024 floats of scratch for the inverse
 
     const int tid = threadIdx.x, warp = tid >> 5;
     const int row = tid & 127, ch = tid >> 7;
@@ -194,6 +194,7 @@ __global__ void __launch_bounds__(PT, 2)
             ms->sc[tid] = gm;
             ms->del[tid] = __expf(ms->G[CH - 1] - ms->G[tid]);  // G is flat past the last token
             ms->pk[tid] = factored ? __expf(-ms->G[tid]) * ms->invr[tid] : 0.f;
+            ms->wsc[tid] = ms->bco[tid] * gm * ms->invr[tid];
         } else if (tid == CH) {
             ms->sc[CH] = __expf(ms->gsum[0] + ms->gsum[1]);
         }
@@ -251,29 +252,24 @@ __global__ void __launch_bounds__(PT, 2)
     }
     tc_fence_before();
     __syncthreads();
-    invert_unit_lower64<PT>(Lf, Toff, Xs, tid);
-    // ---- T' = T Diag(b gamma / r), T'' = T Diag(c): thread -> row tid/4, 16 columns
+    invert_unit_lower64_doubling<PT>(Lf, Xs, tid);
+    // ---- T' = T Diag(b gamma / r), T'' = T Diag(c): thread -> row tid/4, 16 columns (T is zero
+    //      above its diagonal)
     {
-        const int i = tid >> 2, qq = tid & 3, I = i >> 4;
+        const int i = tid >> 2, qq = tid & 3;
         float tv[16];
-        if (qq <= I) {
-            const float* src = (qq == I) ? (Lf + i * LDL + 16 * qq) : (Toff + toff_block(I, qq) * 256 + (i & 15) * 16);
+        {
+            const float* src = Lf + i * LDL + 16 * qq;
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 const float4 t4 = *reinterpret_cast<const float4*>(src + 4 * q);
                 tv[4 * q] = t4.x; tv[4 * q + 1] = t4.y; tv[4 * q + 2] = t4.z; tv[4 * q + 3] = t4.w;
             }
-        } else {
-#pragma unroll
-            for (int e = 0; e < 16; ++e) tv[e] = 0.f;
         }
         __syncthreads();  // T is read; the tiles below overwrite it
         float v[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-            const int j = 16 * qq + e;
-            v[e] = tv[e] * (ms->bco[j] * ms->gam[j] * ms->invr[j]);
-        }
+        for (int e = 0; e < 16; ++e) v[e] = tv[e] * ms->wsc[16 * qq + e];
         st_chunks_split(sm + P_Z, sm + P_Z + 8192, i, 2 * qq, 2, v);
 #pragma unroll
         for (int e = 0; e < 16; ++e) v[e] = tv[e] * ms->cco[16 * qq + e];
@@ -350,7 +346,7 @@ __global__ void __launch_bounds__(PT, 2)
         bulk_store(rec + REC_UP, sbase + P_QK, 32768);
         bulk_store(rec + REC_SC, smem_u32(ms->sc), REC_SCB);
         bulk_commit();
-        bulk_wait_all();
+        bulk_wait_read();  // shared memory may be released; the writes land before the grid ends
     }
 done:
     tc_fence_before();
@@ -429,9 +425,6 @@ __device__ __forceinline__ void tma_store_4d(const void* tmap, uint32_t src, int
             reinterpret_cast<uint64_t>(tmap)),
         "r"(src), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
         : "memory");
-}
-__device__ __forceinline__ void bulk_wait_read_all() {
-    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
 // Epilogue warp: make this warp's TMEM stores visible to the MMA issuer, then arrive once.
 __device__ __forceinline__ void epi_signal(uint32_t bar, int tid) {
@@ -555,7 +548,7 @@ __global__ void __launch_bounds__(ST, 1)
                 if (write_o) {
                     tma_store_4d(&tm_o, sbase + st * S_STAGE + SO_Q, 0, h, c * CH, b);
                     bulk_commit();
-                    bulk_wait_read_all();
+                    bulk_wait_read();
                 }
                 if (c + 2 < c1) {
                     load_late(c + 2, st);

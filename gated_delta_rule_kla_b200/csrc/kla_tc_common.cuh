@@ -104,6 +104,74 @@ __device__ __forceinline__ void invert_unit_lower64(float* Lf, float* Toff, floa
     }
 }
 
+// T = (I + L)^{-1} of the unit lower-triangular 64x64 matrix of Eq. (7), in place, by
+// recursive doubling on the block form of the inverse (a rearrangement of the forward
+// substitution of Appendix B.2):
+//   [A 0; C B]^{-1} = [A^{-1} 0; -B^{-1} C A^{-1}  B^{-1}].
+// Level 0 inverts the eight 8x8 diagonal blocks by substitution (64 threads); levels 8, 16, 32
+// then join pairs of inverted s x s blocks, writing -T_B (L_BA T_A) over L_BA, with every thread
+// computing PER = 32 s / NT adjacent outputs of each product.  On entry Lf holds L (rows of
+// LDL floats, zero on and above the diagonal); on exit it holds T, ones on the diagonal.
+// X is scratch for 1024 floats.  All NT (= 256) threads of the CTA must call it.
+template <int S, int NT>
+__device__ __forceinline__ void inverse_join_level(float* Lf, float* X, int tid) {
+    constexpr int PER = 32 * S / NT;  // outputs per thread: 1, 2, 4 for S = 8, 16, 32
+    static_assert(PER >= 1 && PER <= 4 && S % PER == 0, "join level shape");
+    const int idx = tid * PER;
+    const int p = idx / (S * S), rem = idx % (S * S), i = rem / S, j0 = rem % S;
+    const int A0 = 2 * S * p, B0 = A0 + S;
+    float acc[PER];
+#pragma unroll
+    for (int e = 0; e < PER; ++e) acc[e] = 0.f;
+    // X_p = L_BA T_A   (T_A lower triangular: zero above its diagonal)
+#pragma unroll 8
+    for (int k = 0; k < S; ++k) {
+        const float l = Lf[(B0 + i) * LDL + A0 + k];
+        const float* t = Lf + (A0 + k) * LDL + A0 + j0;
+#pragma unroll
+        for (int e = 0; e < PER; ++e) acc[e] = fmaf(l, t[e], acc[e]);
+    }
+#pragma unroll
+    for (int e = 0; e < PER; ++e) X[idx + e] = acc[e];
+    __syncthreads();
+    // T_BA = -T_B X_p, over L_BA (whose reads are all done)
+#pragma unroll
+    for (int e = 0; e < PER; ++e) acc[e] = 0.f;
+#pragma unroll 8
+    for (int k = 0; k < S; ++k) {
+        const float l = Lf[(B0 + i) * LDL + B0 + k];
+        const float* x = X + p * S * S + k * S + j0;
+#pragma unroll
+        for (int e = 0; e < PER; ++e) acc[e] = fmaf(l, x[e], acc[e]);
+    }
+#pragma unroll
+    for (int e = 0; e < PER; ++e) Lf[(B0 + i) * LDL + A0 + j0 + e] = -acc[e];
+    __syncthreads();
+}
+
+template <int NT>
+__device__ __forceinline__ void invert_unit_lower64_doubling(float* Lf, float* X, int tid) {
+    static_assert(NT == 256, "the join levels assume 256 threads");
+    if (tid < 64) {  // 8x8 diagonal block tid / 8, column tid % 8
+        const int base = 8 * (tid >> 3), c = tid & 7;
+        float x[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            float s = 0.f;
+#pragma unroll
+            for (int j = 0; j < i; ++j) s = fmaf(Lf[(base + i) * LDL + base + j], x[j], s);
+            x[i] = (i < c) ? 0.f : ((i == c) ? 1.f : -s);
+        }
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < 8; ++i) Lf[(base + i) * LDL + base + c] = x[i];
+    }
+    __syncthreads();
+    inverse_join_level<8, NT>(Lf, X, tid);
+    inverse_join_level<16, NT>(Lf, X, tid);
+    inverse_join_level<32, NT>(Lf, X, tid);
+}
+
 // Write chunks [c0, c0 + n) of row r of a swizzled bf16 block from 8*n fp32 values.
 __device__ __forceinline__ void st_chunks_bf16(uint8_t* block, int r, int c0, int n, const float* v) {
 #pragma unroll
