@@ -51,29 +51,29 @@ constexpr uint32_t REC_SCB = 512;
 constexpr size_t REC_BYTES = REC_TILES + REC_SCB;
 
 // =====================================================================================
-// Preparation kernel: one chunk per CTA.
+// Preparation kernel: one chunk per CTA, three CTAs per SM.  Shared memory holds only the
+// inputs and the MMA operands; every output goes from registers straight to its record.
 // =====================================================================================
 constexpr int PT = 256;
 constexpr int kPrepIssuer = 128;
-constexpr uint32_t P_QK = 0;       // [Q; K] tile (32 KB), later U' fp32
-constexpr uint32_t P_V = 32768;    // V tile (16 KB), later -W^T
-constexpr uint32_t P_P = 49152;    // P hi/lo (16 KB)
-constexpr uint32_t P_Z = 65536;    // L/T fp32 -> T' T'' hi/lo -> Ktil hi/lo (32 KB)
-constexpr uint32_t P_MISC = 98304;
-constexpr uint32_t P_SMEM = P_MISC + 4096 + 1024;
-constexpr uint32_t PM_G = 0, PM_W = 64, PM_U = 128;  // TMEM columns (256 allocated)
+constexpr uint32_t P_QK = 0;       // [Q; K] tile (32 KB); after the Gram MMA, T' hi/lo over Q
+constexpr uint32_t P_V = 32768;    // V tile (16 KB)
+constexpr uint32_t P_Z = 49152;    // L/T fp32 (64 x LDL) + 1024 floats scratch; then T'' hi/lo
+constexpr uint32_t P_MISC = P_Z + 64 * LDL * 4 + 4096;
+constexpr uint32_t P_SMEM = P_MISC + 3072 + 1024;
+static_assert(P_MISC % 1024 == 0, "prep scalars alignment");
+constexpr uint32_t PM_G = 0, PM_W = 0, PM_U = 64;  // TMEM columns (128 allocated); W reuses G's
 
 struct PrepMisc {
     uint64_t full, mma;
     uint32_t tmem_base, pad[3];
-    float sc[128];  // record scalars: gamma[64], gamma_last(next chunk)
     float G[CH], gam[CH], del[CH], bco[CH], cco[CH], invr[CH], graw[CH], eta[CH], pk[CH];
     float wsc[CH];  // b gamma / r: column scale of T'
     float gsum[2], grange;
 };
-static_assert(sizeof(PrepMisc) <= 4096, "prep scalars");
+static_assert(sizeof(PrepMisc) <= 3072, "prep scalars");
 
-__global__ void __launch_bounds__(PT, 2)
+__global__ void __launch_bounds__(PT, 3)
     chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, FwdArgs a, uint8_t* __restrict__ recs) {
     extern __shared__ uint8_t smem_raw[];
@@ -93,6 +93,18 @@ __global__ void __launch_bounds__(PT, 2)
     const uint32_t sbase = smem_u32(sm);
     const uint32_t bar_full = smem_u32(&ms->full), bar_mma = smem_u32(&ms->mma);
 
+    // per-token gates first: their latency overlaps the barrier set-up and the tile loads
+    float g_own = 0.f, eta_own = 0.f, g_next = 0.f;
+    if (tid < CH) {
+        if (tid < n) {
+            const size_t ti = tok_index(b, t0 + tid, h, T, H);
+            g_own = a.g[ti];
+            eta_own = a.eta[ti];
+        }
+    } else if (tid < 2 * CH) {
+        const int j = tid - CH;
+        if (c + 1 < NC && (c + 1) * CH + j < T) g_next = a.g[tok_index(b, (c + 1) * CH + j, h, T, H)];
+    }
     if (tid == 0) {
         mbar_init(bar_full, 1);
         mbar_init(bar_mma, 1);
@@ -106,19 +118,14 @@ __global__ void __launch_bounds__(PT, 2)
         tma_load_4d(sbase + P_V + 8192, &tm_v, bar_full, 64, h, t0, b);
     }
     if (warp == 0) {
-        tmem_alloc(smem_u32(&ms->tmem_base), 256);
+        tmem_alloc(smem_u32(&ms->tmem_base), 128);
         tmem_relinquish();
     }
     if (tid < CH) {
-        const bool live = tid < n;
-        const size_t ti = tok_index(b, t0 + (live ? tid : 0), h, T, H);
-        ms->graw[tid] = live ? a.g[ti] : 0.f;
-        ms->eta[tid] = live ? a.eta[ti] : 0.f;
-    } else if (tid < 2 * CH) {  // log-decays of the next chunk: its gamma_last
-        const int j = tid - CH;
-        const bool live = (c + 1 < NC) && ((c + 1) * CH + j < T);
-        const float gn = live ? a.g[tok_index(b, (c + 1) * CH + j, h, T, H)] : 0.f;
-        const float sg = warp_sum(gn);
+        ms->graw[tid] = g_own;
+        ms->eta[tid] = eta_own;
+    } else if (tid < 2 * CH) {  // the next chunk's gamma_last
+        const float sg = warp_sum(g_next);
         if ((tid & 31) == 0) ms->gsum[warp - 2] = sg;
     }
     tc_fence_before();
@@ -191,12 +198,12 @@ __global__ void __launch_bounds__(PT, 2)
         if (tid < CH) {
             const float gm = __expf(ms->G[tid]);
             ms->gam[tid] = gm;
-            ms->sc[tid] = gm;
+            reinterpret_cast<float*>(rec + REC_SC)[tid] = gm;
             ms->del[tid] = __expf(ms->G[CH - 1] - ms->G[tid]);  // G is flat past the last token
             ms->pk[tid] = factored ? __expf(-ms->G[tid]) * ms->invr[tid] : 0.f;
             ms->wsc[tid] = ms->bco[tid] * gm * ms->invr[tid];
         } else if (tid == CH) {
-            ms->sc[CH] = __expf(ms->gsum[0] + ms->gsum[1]);
+            reinterpret_cast<float*>(rec + REC_SC)[CH] = __expf(ms->gsum[0] + ms->gsum[1]);
         }
         ok = mbar_wait_bounded(bar_mma, 0, kWaitNs);
         if (__syncthreads_or(!ok)) {
@@ -205,7 +212,8 @@ __global__ void __launch_bounds__(PT, 2)
         }
         tc_fence_after();
 
-        // ---- Gram epilogue: P (rows 0-63, hi/lo bf16) and L (rows 64-127, fp32); 32 columns each
+        // ---- Gram epilogue: P (rows 0-63, hi/lo bf16, to the record) and L (rows 64-127,
+        //      fp32); 32 columns each
         float x[32];
         tmem_ld32(tmem + lane_base + PM_G + 32 * ch, x);
         tmem_ld_wait();
@@ -226,7 +234,7 @@ __global__ void __launch_bounds__(PT, 2)
                     x[e] = (j <= i) ? __expf(Gi - ms->G[j]) * x[e] * ms->invr[j] : 0.f;
                 }
             }
-            st_chunks_split(sm + P_P, sm + P_P + 8192, i, 4 * ch, 4, x);
+            st_chunks_split(rec + REC_P, rec + REC_P + 8192, i, 4 * ch, 4, x);
         } else {
             const int i = row - CH;
             const float bi = ms->bco[i] * ms->invr[i];
@@ -253,8 +261,8 @@ __global__ void __launch_bounds__(PT, 2)
     tc_fence_before();
     __syncthreads();
     invert_unit_lower64_doubling<PT>(Lf, Xs, tid);
-    // ---- T' = T Diag(b gamma / r), T'' = T Diag(c): thread -> row tid/4, 16 columns (T is zero
-    //      above its diagonal)
+    // ---- T' = T Diag(b gamma / r) over the Q slots of the [Q; K] tile, T'' = T Diag(c) over
+    //      L/T: thread -> row tid/4, 16 columns (T is zero above its diagonal)
     {
         const int i = tid >> 2, qq = tid & 3;
         float tv[16];
@@ -266,16 +274,17 @@ __global__ void __launch_bounds__(PT, 2)
                 tv[4 * q] = t4.x; tv[4 * q + 1] = t4.y; tv[4 * q + 2] = t4.z; tv[4 * q + 3] = t4.w;
             }
         }
-        __syncthreads();  // T is read; the tiles below overwrite it
+        __syncthreads();  // T is read; T'' overwrites it
         float v[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) v[e] = tv[e] * ms->wsc[16 * qq + e];
-        st_chunks_split(sm + P_Z, sm + P_Z + 8192, i, 2 * qq, 2, v);
+        st_chunks_split(sm + P_QK, sm + P_QK + 16384, i, 2 * qq, 2, v);
 #pragma unroll
         for (int e = 0; e < 16; ++e) v[e] = tv[e] * ms->cco[16 * qq + e];
-        st_chunks_split(sm + P_Z + 16384, sm + P_Z + 24576, i, 2 * qq, 2, v);
+        st_chunks_split(sm + P_Z, sm + P_Z + 8192, i, 2 * qq, 2, v);
     }
     fence_proxy_async();
+    tc_fence_before();
     __syncthreads();
     // ---- MMA: W^T = K^T T'^T (lane = dk) and U'^T = V^T T''^T (lane = dv)
     if (tid == kPrepIssuer) {
@@ -286,13 +295,13 @@ __global__ void __launch_bounds__(PT, 2)
 #pragma unroll
             for (int s = 0; s < 4; ++s)
                 mma_bf16(tmem + PM_W, smem_desc(qk_a + 8192 + s * 2048, 16384, 1024),
-                         smem_desc(sbase + P_Z + part * 8192 + s * 32, 16, 1024), iw, (part | s) > 0);
+                         smem_desc(qk_a + part * 16384 + s * 32, 16, 1024), iw, (part | s) > 0);
 #pragma unroll
         for (int part = 0; part < 2; ++part)
 #pragma unroll
             for (int s = 0; s < 4; ++s)
                 mma_bf16(tmem + PM_U, smem_desc(v_a + s * 2048, 8192, 1024),
-                         smem_desc(sbase + P_Z + 16384 + part * 8192 + s * 32, 16, 1024), iw, (part | s) > 0);
+                         smem_desc(sbase + P_Z + part * 8192 + s * 32, 16, 1024), iw, (part | s) > 0);
         mma_commit(bar_mma);
     }
     ok = mbar_wait_bounded(bar_mma, 1, kWaitNs);
@@ -302,58 +311,43 @@ __global__ void __launch_bounds__(PT, 2)
     }
     tc_fence_after();
     {
-        // ---- -W^T to bf16 over the consumed V tile; Ktil = Diag(delta / r) K hi/lo over T tiles
-        float x[32], u[32];
+        // ---- -W^T (thread = dk row, 32 tokens), U' as [token][dv] rows, Ktil hi/lo: all to the record
+        float x[32];
         tmem_ld32(tmem + lane_base + PM_W + 32 * ch, x);
-        tmem_ld32(tmem + lane_base + PM_U + 32 * ch, u);
         tmem_ld_wait();
 #pragma unroll
         for (int e = 0; e < 32; ++e) x[e] = -x[e];
-        st_chunks_bf16(sm + P_V, row, 4 * ch, 4, x);
-        {
-            const int j = tid >> 2, blk = (tid >> 1) & 1, cq = 4 * (tid & 1);
-            const float sc = ms->del[j] * ms->invr[j];
+        st_chunks_bf16(rec + REC_W, row, 4 * ch, 4, x);
+        tmem_ld32(tmem + lane_base + PM_U + 32 * ch, x);
+        tmem_ld_wait();
+        float* up = reinterpret_cast<float*>(rec + REC_UP);
 #pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4) {
-                const int cc = cq + ((c4 + j) & 3);  // rotated by row: no bank conflicts
-                float f[8], hi[8], lo[8];
-                const uint32_t off = (uint32_t)(j * 128 + cc * 16);  // same swizzle phase: (64 + j) & 7 == j & 7
-                unpack_bf16x8(*reinterpret_cast<const uint4*>(qk + blk * 16384 + 8192 + off), f);
+        for (int e = 0; e < 32; ++e) up[(32 * ch + e) * DV + row] = x[e];
+        const int j = tid >> 2, blk = (tid >> 1) & 1, cq = 4 * (tid & 1);
+        const float sc = ms->del[j] * ms->invr[j];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) split_bf16(f[e] * sc, hi[e], lo[e]);
-                uint4 uh, ul;
-                uh.x = pack_bf16x2(hi[0], hi[1]); uh.y = pack_bf16x2(hi[2], hi[3]);
-                uh.z = pack_bf16x2(hi[4], hi[5]); uh.w = pack_bf16x2(hi[6], hi[7]);
-                ul.x = pack_bf16x2(lo[0], lo[1]); ul.y = pack_bf16x2(lo[2], lo[3]);
-                ul.z = pack_bf16x2(lo[4], lo[5]); ul.w = pack_bf16x2(lo[6], lo[7]);
-                *reinterpret_cast<uint4*>(sm + P_Z + blk * 8192 + off) = uh;
-                *reinterpret_cast<uint4*>(sm + P_Z + 16384 + blk * 8192 + off) = ul;
-            }
+        for (int c4 = 0; c4 < 4; ++c4) {
+            const int cc = cq + ((c4 + j) & 3);  // rotated by row: no bank conflicts
+            float f[8], hi[8], lo[8];
+            const uint32_t off = (uint32_t)(j * 128 + cc * 16);  // same swizzle phase: (64 + j) & 7 == j & 7
+            unpack_bf16x8(*reinterpret_cast<const uint4*>(qk + blk * 16384 + 8192 + off), f);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) split_bf16(f[e] * sc, hi[e], lo[e]);
+            uint4 uh, ul;
+            uh.x = pack_bf16x2(hi[0], hi[1]); uh.y = pack_bf16x2(hi[2], hi[3]);
+            uh.z = pack_bf16x2(hi[4], hi[5]); uh.w = pack_bf16x2(hi[6], hi[7]);
+            ul.x = pack_bf16x2(lo[0], lo[1]); ul.y = pack_bf16x2(lo[2], lo[3]);
+            ul.z = pack_bf16x2(lo[4], lo[5]); ul.w = pack_bf16x2(lo[6], lo[7]);
+            *reinterpret_cast<uint4*>(rec + REC_KT + blk * 8192 + off) = uh;
+            *reinterpret_cast<uint4*>(rec + REC_KTLO + blk * 8192 + off) = ul;
         }
-        __syncthreads();  // the [Q; K] tile is consumed: U' goes over it
-        // ---- U' fp32 as [token][dv] (thread = dv lane, 32 tokens)
-        float* up = reinterpret_cast<float*>(sm + P_QK);
-#pragma unroll
-        for (int e = 0; e < 32; ++e) up[(32 * ch + e) * DV + row] = u[e];
-    }
-    fence_proxy_async();
-    tc_fence_before();
-    __syncthreads();
-    if (tid == 0) {
-        bulk_store(rec + REC_W, sbase + P_V, 16384);
-        bulk_store(rec + REC_KT, sbase + P_Z, 32768);
-        bulk_store(rec + REC_P, sbase + P_P, 16384);
-        bulk_store(rec + REC_UP, sbase + P_QK, 32768);
-        bulk_store(rec + REC_SC, smem_u32(ms->sc), REC_SCB);
-        bulk_commit();
-        bulk_wait_read();  // shared memory may be released; the writes land before the grid ends
     }
 done:
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
-        tmem_dealloc(tmem, 256);
+        tmem_dealloc(tmem, 128);
     }
 }
 
