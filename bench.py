@@ -256,9 +256,10 @@ def gpu_arm(args, rank, world, local_rank):
     d = {k: (v.to(dev) if v is not None else None) for k, v in inp.items()}
     o = torch.empty(w.B, w.T, w.H, w.Dv, device=dev, dtype=torch.float32)
     ST = torch.empty(w.B, w.H, w.Dk, w.Dv, device=dev, dtype=torch.float32)
+    ws = kla.fwd_workspace(d["k"], d["v"])  # the split path's per-chunk records, allocated once
 
     def prefill():
-        kla.chunk_fwd(d["q"], d["k"], d["v"], d["eta"], d["g"], w.eps, d["S0"], o=o, S_T=ST)
+        kla.chunk_fwd(d["q"], d["k"], d["v"], d["eta"], d["g"], w.eps, d["S0"], o=o, S_T=ST, workspace=ws)
 
     sampler = ClockSampler(local_rank)
     for _ in range(args.warmup):
@@ -280,6 +281,7 @@ def gpu_arm(args, rank, world, local_rank):
         mean_s = statistics.mean(ms) / 1e3
         achieved_gbs = alg_bytes / mean_s / 1e9
         achieved_tf = alg_flops / mean_s / 1e12
+        stages = time_fwd_stages(kla, d, w, ws, o, ST, flush, stream, 3 if args.quick else 10)
 
         extra = {}
         parts = set(args.parts.split(",")) if not args.skip_extra else set()
@@ -315,16 +317,38 @@ def gpu_arm(args, rank, world, local_rank):
                    "parallelism": f"{world} independent replica(s), no collective"},
         "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
                      "frac": achieved_gbs / hbm_peak, "peak_kind": peaks_kind,
+                     "scope": "one kla_chunk_fwd call: chunk_prep_kernel + chunk_state_kernel",
                      "traffic": recorded_traffic("chunk_fwd_prefill_b8_t2048_h8_d128"),
-                     "alg_bytes_per_launch": alg_bytes, "kernel_us": mean_s * 1e6,
+                     "alg_bytes_per_launch": alg_bytes, "kernel_us": mean_s * 1e6, "stages": stages,
                      "tensor": {"achieved": achieved_tf, "peak": tc_peak, "unit": "TFLOP/s",
                                 "frac": achieved_tf / tc_peak, "alg_flops_per_launch": alg_flops}},
         "e2e": e2e,
-        "gpu_launches": args.steps,
+        "gpu_launches": 2 * args.steps,
         "clocks": clocks,
     }
     line.update(extra)
     return line
+
+
+def time_fwd_stages(kla, d, w, ws, o, ST, flush, stream, nsteps):
+    """Each stage of the split forward timed on its own with CUDA events on the launching
+    stream (L2 flushed before every step): the preparation kernel and the state pass."""
+    import torch
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(nsteps)]
+    for i in range(nsteps):
+        flush()
+        ev[i][0].record(stream)
+        kla.chunk_fwd_prep(d["q"], d["k"], d["v"], d["eta"], d["g"], w.eps, ws)
+        ev[i][1].record(stream)
+        kla.chunk_fwd_state(d["q"], d["g"], d["S0"], ws, o=o, S_T=ST)
+        ev[i][2].record(stream)
+    torch.cuda.synchronize()
+    prep = statistics.median(e[0].elapsed_time(e[1]) for e in ev) * 1e3
+    state = statistics.median(e[1].elapsed_time(e[2]) for e in ev) * 1e3
+    tot = prep + state
+    return {"chunk_prep_kernel": {"us": prep, "share": prep / tot},
+            "chunk_state_kernel": {"us": state, "share": state / tot},
+            "dominant": "chunk_prep_kernel" if prep >= state else "chunk_state_kernel"}
 
 
 def bench_decode(kla, WORKLOADS, make_inputs, dev, stream, flush, rank, world, hbm_peak, args):
@@ -373,10 +397,11 @@ def bench_train(kla, WORKLOADS, make_inputs, dev, stream, flush, rank, world, hb
     dO = d["dO"].to(d["q"].dtype)
     ws = torch.empty(kla.lib().kla_chunk_bwd_workspace(w.B, w.T, w.H, w.Dk, w.Dv, 64, 1, 1),
                      dtype=torch.uint8, device=dev)
+    fws = kla.fwd_workspace(d["k"], d["v"])
 
     def step():
         _, _, Sc = kla.chunk_fwd(d["q"], d["k"], d["v"], d["eta"], d["g"], w.eps, d["S0"],
-                                 save_chunk_states=True)
+                                 save_chunk_states=True, workspace=fws)
         kla.chunk_bwd(d["q"], d["k"], d["v"], d["eta"], d["g"], dO, w.eps, d["S0"], None, Sc, workspace=ws)
 
     nsteps = 2 if args.quick else 5
@@ -392,7 +417,8 @@ def bench_train(kla, WORKLOADS, make_inputs, dev, stream, flush, rank, world, hb
     elt = d["q"].element_size()
     alg = fwd_bytes(w.B, w.T, w.H, w.Dk, w.Dv, elt, False) + bwd_bytes(w.B, w.T, w.H, w.Dk, w.Dv, elt)
     return {"workload": w.name, "value": tokens / (total_ms / 1e3), "unit": "tokens/s",
-            "steps": nsteps, "ms_per_step": total_ms / nsteps, "gpu_launches_per_step": 4,
+            "steps": nsteps, "ms_per_step": total_ms / nsteps,
+            "gpu_launches_per_step": 5,  # forward: preparation + state pass; backward: 3 kernels
             "roofline": {"bound": "tensor", "achieved": flops / mean_s / 1e12, "peak": tc_peak,
                          "unit": "TFLOP/s", "frac": flops / mean_s / 1e12 / tc_peak,
                          "hbm_frac": alg / mean_s / 1e9 / hbm_peak, "alg_flops_per_step": flops,
@@ -407,9 +433,9 @@ def bench_long(kla, WORKLOADS, make_inputs, dev, stream, rank, world, hbm_peak, 
     d = {k: (v.to(dev) if v is not None else None) for k, v in inp.items()}
     o = torch.empty(w.B, w.T, w.H, w.Dv, device=dev, dtype=torch.float32)
     ST = torch.empty(w.B, w.H, w.Dk, w.Dv, device=dev, dtype=torch.float32)
-    # few heads, long sequences: the library's segmented path (workspace allocated once here)
-    need = kla.lib().kla_chunk_fwd_workspace(w.B, w.T, w.H, w.Dk, w.Dv, 64, 1)
-    ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    # few heads, long sequences: the split path with a segmented state pass (workspace
+    # allocated once here)
+    ws = kla.fwd_workspace(d["k"], d["v"])
 
     def run():
         kla.chunk_fwd(d["q"], d["k"], d["v"], d["eta"], d["g"], w.eps, d["S0"], o=o, S_T=ST, workspace=ws)
@@ -427,7 +453,8 @@ def bench_long(kla, WORKLOADS, make_inputs, dev, stream, rank, world, hbm_peak, 
     flops = fwd_flops_per_token_head(w.Dk) * w.B * w.T * w.H
     return {"workload": w.name, "value": tokens / (total_ms / 1e3), "unit": "tokens/s",
             "steps": nsteps, "ms_per_step": total_ms / nsteps, "l2": "inputs larger than L2",
-            "gpu_launches_per_step": 3 if need > 0 else 1, "segmented": need > 0,
+            # preparation, transition pass, segment scan, output pass
+            "gpu_launches_per_step": 4,
             "roofline": {"bound": "hbm", "achieved": alg / mean_s / 1e9, "peak": hbm_peak, "unit": "GB/s",
                          "frac": alg / mean_s / 1e9 / hbm_peak,
                          "tensor_frac": flops / mean_s / 1e12 / tc_peak}}

@@ -55,6 +55,10 @@ def lib():
         L.kla_chunk_fwd_workspace.restype = sz
         L.kla_chunk_fwd.argtypes = [vp, vp, vp, fp, fp, f, fp, vp, fp, fp, i, i, i, i, i, i, i, i, vp, sz, vp]
         L.kla_chunk_fwd.restype = i
+        L.kla_chunk_fwd_prep.argtypes = [vp, vp, vp, fp, fp, f, i, i, i, i, i, i, i, vp, sz, vp]
+        L.kla_chunk_fwd_prep.restype = i
+        L.kla_chunk_fwd_state.argtypes = [vp, fp, fp, vp, fp, fp, i, i, i, i, i, i, i, i, vp, sz, vp]
+        L.kla_chunk_fwd_state.restype = i
         L.kla_chunk_bwd_workspace.argtypes = [i, i, i, i, i, i, i, i]
         L.kla_chunk_bwd_workspace.restype = sz
         L.kla_chunk_bwd.argtypes = [vp, vp, vp, fp, fp, f, fp, vp, fp, fp, vp, vp, vp, fp, fp, fp,
@@ -150,6 +154,52 @@ def chunk_fwd(q, k, v, eta, g, eps=1e-6, S0=None, *, o=None, S_T=None, save_chun
                          _dtype_code(o), ws_ptr, ws_n, _stream(dev, stream))
     _check(st, "kla_chunk_fwd")
     return (o, S_T, Sc) if save_chunk_states else (o, S_T)
+
+
+def fwd_workspace(k, v):
+    """A workspace for kla_chunk_fwd / its two stages, sized for k [B,T,H,Dk] and v (None when
+    the shapes take no workspace)."""
+    B, T, H, Dk = k.shape
+    need = lib().kla_chunk_fwd_workspace(B, T, H, Dk, v.shape[-1], CHUNK, _dtype_code(k))
+    return torch.empty(need, device=k.device, dtype=torch.uint8) if need > 0 else None
+
+
+def chunk_fwd_prep(q, k, v, eta, g, eps, workspace, *, stream=None):
+    """First stage of the split forward: every chunk's state-independent operands into
+    `workspace` (from fwd_workspace).  bf16 inputs with Dk == Dv == 128."""
+    dev = k.device
+    B, T, H, Dk = k.shape
+    Dv = v.shape[-1]
+    _need(q, "q", dev, k.dtype, (B, T, H, Dk)); _need(v, "v", dev, k.dtype, (B, T, H, Dv))
+    _need(eta, "eta", dev, torch.float32, (B, T, H)); _need(g, "g", dev, torch.float32, (B, T, H))
+    _need(workspace, "workspace", dev, torch.uint8)
+    L = lib()
+    st = L.kla_chunk_fwd_prep(_ptr(q), _ptr(k), _ptr(v), _ptr(eta), _ptr(g), float(eps), B, T, H, Dk, Dv,
+                              CHUNK, _dtype_code(k), _ptr(workspace), workspace.numel(), _stream(dev, stream))
+    _check(st, "kla_chunk_fwd_prep")
+
+
+def chunk_fwd_state(q, g, S0, workspace, *, Dv=None, o=None, S_T=None, S_chunks=None,
+                    out_dtype=torch.float32, stream=None):
+    """Second stage of the split forward: the state pass over the records that chunk_fwd_prep
+    left in `workspace`.  Writes o, S_T, S_chunks when given (allocates o and S_T when None)."""
+    dev = q.device
+    B, T, H, Dk = q.shape
+    Dv = Dk if Dv is None else Dv
+    _need(g, "g", dev, torch.float32, (B, T, H)); _need(S0, "S0", dev, torch.float32, (B, H, Dk, Dv))
+    if o is None:
+        o = torch.empty(B, T, H, Dv, device=dev, dtype=out_dtype)
+    if S_T is None:
+        S_T = torch.empty(B, H, Dk, Dv, device=dev, dtype=torch.float32)
+    _need(o, "o", dev, None, (B, T, H, Dv)); _need(S_T, "S_T", dev, torch.float32, (B, H, Dk, Dv))
+    _need(S_chunks, "S_chunks", dev, torch.float32, (B, H, (T + CHUNK - 1) // CHUNK, Dk, Dv))
+    _need(workspace, "workspace", dev, torch.uint8)
+    L = lib()
+    st = L.kla_chunk_fwd_state(_ptr(q), _ptr(g), _ptr(S0), _ptr(o), _ptr(S_T), _ptr(S_chunks), B, T, H, Dk, Dv,
+                               CHUNK, _dtype_code(q), _dtype_code(o), _ptr(workspace), workspace.numel(),
+                               _stream(dev, stream))
+    _check(st, "kla_chunk_fwd_state")
+    return o, S_T
 
 
 def chunk_bwd(q, k, v, eta, g, dO, eps=1e-6, S0=None, dS_T=None, S_chunks=None, *, stream=None,

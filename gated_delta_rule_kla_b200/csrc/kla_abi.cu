@@ -152,6 +152,52 @@ kla_status kla_chunk_fwd(const void* q, const void* k, const void* v, const floa
     return KLA_OK;
 }
 
+static kla_status split_stage_checks(int B, int T, int H, int Dk, int Dv, int chunk, int dtype, int out_dtype,
+                                     float eps, void* ws, size_t ws_bytes, const char* name, kla::FwdArgs* a) {
+    kla_status st = check_common(B, T, H, Dk, Dv, chunk, dtype, out_dtype, eps);
+    if (st != KLA_OK) return st;
+    if (T < 1) return fail(KLA_ERR_INVALID_ARG, "%s needs T >= 1 (got %d)", name, T);
+    a->B = B; a->T = T; a->H = H; a->Dk = Dk; a->Dv = Dv; a->eps = eps;
+    a->bf16 = dtype == KLA_BF16; a->out_bf16 = out_dtype == KLA_BF16;
+    if (!(a->bf16 && Dk == 128 && Dv == 128))
+        return fail(KLA_ERR_UNSUPPORTED, "%s needs bf16 inputs with Dk == Dv == 128", name);
+    const size_t need = kla::chunk_fwd_split_workspace(*a);
+    if (ws == nullptr || ws_bytes < need)
+        return fail(KLA_ERR_WORKSPACE, "%s needs %zu workspace bytes (got %zu)", name, need,
+                    ws == nullptr ? (size_t)0 : ws_bytes);
+    if (!aligned16(ws)) return fail(KLA_ERR_INVALID_ARG, "ws must be 16-byte aligned");
+    return KLA_OK;
+}
+
+kla_status kla_chunk_fwd_prep(const void* q, const void* k, const void* v, const float* eta,
+                              const float* g, float eps, int B, int T, int H, int Dk, int Dv,
+                              int chunk, int dtype, void* ws, size_t ws_bytes, void* stream) {
+    kla::FwdArgs a{};
+    kla_status st = split_stage_checks(B, T, H, Dk, Dv, chunk, dtype, KLA_F32, eps, ws, ws_bytes,
+                                       "kla_chunk_fwd_prep", &a);
+    if (st != KLA_OK) return st;
+    REQUIRE_PTR(q); REQUIRE_PTR(k); REQUIRE_PTR(v); REQUIRE_PTR(eta); REQUIRE_PTR(g);
+    a.q = q; a.k = k; a.v = v; a.eta = eta; a.g = g;
+    cudaError_t e = kla::launch_chunk_fwd_split_prep(a, ws, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "kla_chunk_fwd_prep launch");
+    return KLA_OK;
+}
+
+kla_status kla_chunk_fwd_state(const void* q, const float* g, const float* S0, void* o, float* S_T,
+                               float* S_chunks, int B, int T, int H, int Dk, int Dv, int chunk,
+                               int dtype, int out_dtype, void* ws, size_t ws_bytes, void* stream) {
+    kla::FwdArgs a{};
+    kla_status st = split_stage_checks(B, T, H, Dk, Dv, chunk, dtype, out_dtype, 0.f, ws, ws_bytes,
+                                       "kla_chunk_fwd_state", &a);
+    if (st != KLA_OK) return st;
+    REQUIRE_PTR(q); REQUIRE_PTR(g);
+    OPTIONAL_PTR(S0); OPTIONAL_PTR(o); OPTIONAL_PTR(S_T); OPTIONAL_PTR(S_chunks);
+    a.q = q; a.g = g; a.S0 = S0; a.o = o; a.S_T = S_T; a.S_chunks = S_chunks;
+    cudaError_t e = kla::launch_chunk_fwd_split_state(a, ws, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "kla_chunk_fwd_state launch");
+    return KLA_OK;
+}
+
 size_t kla_chunk_bwd_workspace(int B, int T, int H, int Dk, int Dv, int chunk, int dtype,
                                int have_S_chunks) {
     (void)chunk; (void)dtype;

@@ -867,19 +867,25 @@ size_t chunk_fwd_split_workspace(const FwdArgs& a) {
     return split_layout(a).total;
 }
 
-cudaError_t launch_chunk_fwd_split(const FwdArgs& a, void* ws, cudaStream_t st) {
+cudaError_t launch_chunk_fwd_split_prep(const FwdArgs& a, void* ws, cudaStream_t st) {
     CUtensorMap mq, mk, mv;
     if (!make_map(&mq, a.q, a.B, a.T, a.H) || !make_map(&mk, a.k, a.B, a.T, a.H) ||
         !make_map(&mv, a.v, a.B, a.T, a.H))
         return cudaErrorInvalidValue;
+    const int NC = (a.T + CH - 1) / CH;
+    cudaError_t e = cudaFuncSetAttribute(chunk_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)P_SMEM);
+    if (e != cudaSuccess) return e;
+    chunk_prep_kernel<<<dim3(NC, a.B * a.H), PT, P_SMEM, st>>>(mq, mk, mv, a, static_cast<uint8_t*>(ws));
+    return cudaGetLastError();
+}
+
+cudaError_t launch_chunk_fwd_split_state(const FwdArgs& a, void* ws, cudaStream_t st) {
+    CUtensorMap mq;
+    if (!make_map(&mq, a.q, a.B, a.T, a.H)) return cudaErrorInvalidValue;
     const SplitLayout L = split_layout(a);
     const int NC = (a.T + CH - 1) / CH;
     const int BH = a.B * a.H;
     uint8_t* recs = static_cast<uint8_t*>(ws);
-    cudaError_t e = cudaFuncSetAttribute(chunk_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)P_SMEM);
-    if (e != cudaSuccess) return e;
-    chunk_prep_kernel<<<dim3(NC, BH), PT, P_SMEM, st>>>(mq, mk, mv, a, recs);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
     auto state = [&](const FwdArgs& f, dim3 grid) {
         return f.out_bf16 ? launch_state<__nv_bfloat16>(mq, f, recs, grid, st)
                           : launch_state<float>(mq, f, recs, grid, st);
@@ -902,7 +908,8 @@ cudaError_t launch_chunk_fwd_split(const FwdArgs& a, void* ws, cudaStream_t st) 
     p1.nseg = L.nseg;
     p1.seg_chunks = L.segc;
     p1.kinds = 2;
-    if ((e = state(p1, dim3(BH * L.nseg, 2))) != cudaSuccess) return e;
+    cudaError_t e = state(p1, dim3(BH * L.nseg, 2));
+    if (e != cudaSuccess) return e;
     if ((e = launch_seg_scan(a.S0, MN, Sstart, a.S_T, BH, L.nseg, st)) != cudaSuccess) return e;
     FwdArgs p2 = a;
     p2.S0 = Sstart;
@@ -911,6 +918,15 @@ cudaError_t launch_chunk_fwd_split(const FwdArgs& a, void* ws, cudaStream_t st) 
     p2.seg_chunks = L.segc;
     p2.kinds = 1;
     return state(p2, dim3(BH * L.nseg, 1));
+}
+
+cudaError_t launch_chunk_fwd_split(const FwdArgs& a, void* ws, cudaStream_t st) {
+    cudaError_t e = launch_chunk_fwd_split_prep(a, ws, st);
+    return e == cudaSuccess ? launch_chunk_fwd_split_state(a, ws, st) : e;
+}
+
+int chunk_fwd_split_state_launches(const FwdArgs& a) {
+    return split_layout(a).nseg > 1 ? 3 : 1;
 }
 
 cudaError_t split_take_error(cudaStream_t st, unsigned int* flag) {

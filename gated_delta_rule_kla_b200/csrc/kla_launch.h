@@ -74,6 +74,10 @@ cudaError_t launch_seg_scan(const float* S0, const float* MN, float* Sstart, flo
 // long sequences over few heads).  Workspace bytes for these sizes (0: shapes not supported).
 size_t chunk_fwd_split_workspace(const FwdArgs& a);
 cudaError_t launch_chunk_fwd_split(const FwdArgs& a, void* ws, cudaStream_t st);
+// The two stages of the split path: the chunk-parallel preparation (writes the per-chunk
+// records into ws) and the state pass that reads them.
+cudaError_t launch_chunk_fwd_split_prep(const FwdArgs& a, void* ws, cudaStream_t st);
+cudaError_t launch_chunk_fwd_split_state(const FwdArgs& a, void* ws, cudaStream_t st);
 cudaError_t split_take_error(cudaStream_t st, unsigned int* flag);
 // Synchronise `st`, then read and clear the device error word of the tensor-core kernels
 // (non-zero when a bounded wait expired).

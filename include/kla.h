@@ -101,6 +101,30 @@ kla_status kla_chunk_fwd(const void *q, const void *k, const void *v, const floa
                          int dtype, int out_dtype, void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * kla_chunk_fwd_prep, kla_chunk_fwd_state -- the two stages of kla_chunk_fwd's split path, for
+ * callers that schedule them separately (for example, preparing the next layer's chunks on
+ * another stream, or timing each stage).  Same math as kla_chunk_fwd ("Kaczmarz Linear
+ * Attention", section 4, Eqs. 7-9): _prep computes, for every chunk in parallel, everything that
+ * does not depend on the incoming state (key norms and Kaczmarz coefficients, decays, the UT
+ * transform inverse, W, U', the decayed keys, the masked scores) and stores it in ws; _state then
+ * runs the sequential state pass from ws.  Together they equal one kla_chunk_fwd call with that
+ * workspace, bit for bit.
+ *   Arguments as for kla_chunk_fwd.  Only dtype == KLA_BF16 with Dk == Dv == 128 and T >= 1 is
+ *   supported (KLA_ERR_UNSUPPORTED / KLA_ERR_INVALID_ARG otherwise).  ws (device, 16-byte
+ *   aligned, at least kla_chunk_fwd_workspace() bytes, owned by the caller) is required
+ *   (KLA_ERR_WORKSPACE otherwise); _state must get the same ws, q, g and sizes as the _prep
+ *   call it follows, ordered after it (same stream, or an event), with ws untouched between.
+ * Returns KLA_OK or an error status; on error nothing is launched.
+ */
+kla_status kla_chunk_fwd_prep(const void *q, const void *k, const void *v, const float *eta,
+                              const float *g, float eps, int B, int T, int H, int Dk, int Dv,
+                              int chunk, int dtype, void *ws, size_t ws_bytes, void *stream);
+kla_status kla_chunk_fwd_state(const void *q, const float *g, const float *S0, void *o,
+                               float *S_T, float *S_chunks, int B, int T, int H, int Dk, int Dv,
+                               int chunk, int dtype, int out_dtype, void *ws, size_t ws_bytes,
+                               void *stream);
+
+/*
  * kla_chunk_bwd -- gradients of the chunkwise forward.
  * The paper gives no backward; this one differentiates the forward above exactly (same
  * result as reverse-mode differentiation of the tokenwise recurrence).  Given the upstream

@@ -60,6 +60,22 @@ def test_fwd_rejects_before_launch(L, kw, code):
     assert len(L.kla_last_error()) > 0
 
 
+def test_fwd_stages_reject_before_launch(L):
+    need = L.kla_chunk_fwd_workspace(2, 300, 3, 128, 128, 64, 1)
+    assert need >= 2 * 3 * 5 * 98816  # one record of ~97 KiB per chunk and head
+    prep = lambda dtype=1, Dk=128, T=300, ws=FAKE, n=need: L.kla_chunk_fwd_prep(
+        FAKE, FAKE, FAKE, FAKE, FAKE, 1e-6, 2, T, 3, Dk, 128, 64, dtype, ws, n, None)
+    state = lambda dtype=1, ws=FAKE, n=need, q=FAKE: L.kla_chunk_fwd_state(
+        q, FAKE, None, FAKE, None, None, 2, 300, 3, 128, 128, 64, dtype, 0, ws, n, None)
+    assert prep(dtype=0) == UNSUPPORTED and prep(Dk=64) == UNSUPPORTED
+    assert prep(T=0) == INVALID
+    assert prep(ws=None) == WORKSPACE and prep(n=need - 1) == WORKSPACE
+    assert state(dtype=0) == UNSUPPORTED and state(ws=None) == WORKSPACE
+    assert state(q=None) == INVALID and state(ws=MISALIGNED) == INVALID
+    assert b"aligned" in L.kla_last_error()
+    assert state(ws=None) == WORKSPACE and b"kla_chunk_fwd_state" in L.kla_last_error()
+
+
 def test_bwd_workspace_checked(L):
     need = L.kla_chunk_bwd_workspace(2, 100, 3, 64, 128, 64, 1, 0)
     ntok = 2 * 100 * 3

@@ -174,6 +174,24 @@ def test_fwd_split_and_fused_paths_agree(kla, oracle_mod, B, T, H, s0, g_lo, out
         torch.testing.assert_close(outs[False][2][:, :, 0], d["S0"])  # chunk 0 starts from S0
 
 
+@pytest.mark.parametrize("B,T,H", [(2, 300, 3), (1, 4096 + 100, 2)])
+def test_fwd_prep_and_state_stages_equal_one_call(kla, B, T, H):
+    """kla_chunk_fwd_prep then kla_chunk_fwd_state is kla_chunk_fwd with the same workspace,
+    bit for bit (the second shape takes the segmented state pass)."""
+    inp = small_inputs(B, T, H, 128, 128, "bf16", seed=T + H, g_lo=-0.05)
+    d = {k: (v.cuda() if v is not None else None) for k, v in inp.items()}
+    ws = kla.fwd_workspace(d["k"], d["v"])
+    o, ST, Sc = kla.chunk_fwd(d["q"], d["k"], d["v"], d["eta"], d["g"], 1e-6, d["S0"], save_chunk_states=True,
+                              workspace=ws)
+    ws2 = kla.fwd_workspace(d["k"], d["v"])
+    Sc2 = torch.empty_like(Sc)
+    kla.chunk_fwd_prep(d["q"], d["k"], d["v"], d["eta"], d["g"], 1e-6, ws2)
+    o2, ST2 = kla.chunk_fwd_state(d["q"], d["g"], d["S0"], ws2, S_chunks=Sc2)
+    torch.cuda.synchronize()
+    kla.check_device_error()
+    assert torch.equal(o, o2) and torch.equal(ST, ST2) and torch.equal(Sc, Sc2)
+
+
 def test_fwd_state_passing_equals_one_call(kla):
     """Checkpoint/resume: forward(T1) then forward(T2, S0=S_T1) == forward(T1+T2)."""
     inp = small_inputs(2, 320, 2, 128, 128, "f32", seed=5, g_lo=-0.05)
