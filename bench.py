@@ -461,44 +461,74 @@ def bench_long(kla, WORKLOADS, make_inputs, dev, stream, rank, world, hbm_peak, 
 
 
 def bench_e2e(kla, w, inp, dev, stream, rank, world, args):
-    """Same metric through the public API from pinned host buffers: H2D of the step's
-    inputs, kla_chunk_fwd, D2H of the result, all inside the timed region."""
+    """Same metric through the public API from pinned host buffers: every step's inputs go
+    host -> device, kla_chunk_fwd runs, and o and S_T come back device -> host, all inside the
+    timed region.  Steps are pipelined the way a serving loop would run them: two buffer sets,
+    inputs of step i + 1 copied on their own stream while step i computes and its results
+    are copied back, so the two copy directions and the kernels overlap."""
     import torch
     names = ["q", "k", "v", "eta", "g"]
     host = {n: inp[n].pin_memory() for n in names}
-    devb = {n: torch.empty_like(host[n], device=dev) for n in names}
-    o_h = torch.empty(w.B, w.T, w.H, w.Dv, dtype=torch.float32).pin_memory()
-    ST_h = torch.empty(w.B, w.H, w.Dk, w.Dv, dtype=torch.float32).pin_memory()
+    nbuf = 2
+    devb = [{n: torch.empty_like(host[n], device=dev) for n in names} for _ in range(nbuf)]
+    outs = [(torch.empty(w.B, w.T, w.H, w.Dv, device=dev), torch.empty(w.B, w.H, w.Dk, w.Dv, device=dev))
+            for _ in range(nbuf)]
+    o_h = [torch.empty(w.B, w.T, w.H, w.Dv, dtype=torch.float32).pin_memory() for _ in range(nbuf)]
+    ST_h = [torch.empty(w.B, w.H, w.Dk, w.Dv, dtype=torch.float32).pin_memory() for _ in range(nbuf)]
+    ws = kla.fwd_workspace(devb[0]["k"], devb[0]["v"])
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev = lambda: torch.cuda.Event()
+    in_ready = [ev() for _ in range(nbuf)]
+    in_free = [ev() for _ in range(nbuf)]    # the step that used this input set has computed
+    out_ready = [ev() for _ in range(nbuf)]  # o, S_T of this set computed
+    out_free = [ev() for _ in range(nbuf)]   # o, S_T of this set copied back
 
-    def step():
-        for n in names:
-            devb[n].copy_(host[n], non_blocking=True)
-        o, ST = kla.chunk_fwd(devb["q"], devb["k"], devb["v"], devb["eta"], devb["g"], w.eps, None)
-        o_h.copy_(o, non_blocking=True)
-        ST_h.copy_(ST, non_blocking=True)
+    def run(nsteps):
+        for i in range(nsteps):
+            j = i % nbuf
+            with torch.cuda.stream(s_in):
+                if i >= nbuf:
+                    s_in.wait_event(in_free[j])
+                for n in names:
+                    devb[j][n].copy_(host[n], non_blocking=True)
+                in_ready[j].record(s_in)
+            stream.wait_event(in_ready[j])
+            if i >= nbuf:
+                stream.wait_event(out_free[j])
+            o, ST = outs[j]
+            kla.chunk_fwd(devb[j]["q"], devb[j]["k"], devb[j]["v"], devb[j]["eta"], devb[j]["g"], w.eps, None,
+                          o=o, S_T=ST, workspace=ws, stream=stream)
+            in_free[j].record(stream)
+            out_ready[j].record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(out_ready[j])
+                o_h[j].copy_(o, non_blocking=True)
+                ST_h[j].copy_(ST, non_blocking=True)
+                out_free[j].record(s_out)
+        stream.wait_stream(s_in)
+        stream.wait_stream(s_out)
 
-    step()
+    run(2)
     torch.cuda.synchronize()
     barrier(world)
-    nsteps = 3 if args.quick else 10
+    nsteps = 4 if args.quick else 12
     st, en = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     st.record(stream)
-    for _ in range(nsteps):
-        step()
+    s_in.wait_stream(stream)
+    s_out.wait_stream(stream)
+    run(nsteps)
     en.record(stream)
     torch.cuda.synchronize()
     barrier(world)
     ms = max_over_ranks(st.elapsed_time(en), world)
     tokens = sum_over_ranks(float(w.B * w.T), world) * nsteps
     h2d = sum(host[n].numel() * host[n].element_size() for n in names)
-    d2h = o_h.numel() * o_h.element_size() + ST_h.numel() * 4
+    d2h = o_h[0].numel() * o_h[0].element_size() + ST_h[0].numel() * 4
     return {"value": tokens / (ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h, "steps": nsteps}
+            "d2h_bytes_per_step": d2h, "steps": nsteps,
+            "pipelining": "2 buffer sets; H2D, kernels and D2H on separate streams"}
 
 
-# ---------------------------------------------------------------------------------------
-# CPU oracle arm and CPU baseline
-# ---------------------------------------------------------------------------------------
 def oracle_sample(workload_name, npairs, seed_offset=0):
     """Inputs of `npairs` (b, h) pairs of the workload, as fp64 arrays [npairs, T, 1, D]."""
     import numpy as np

@@ -234,7 +234,7 @@ __global__ void __launch_bounds__(PT, 3)
                     x[e] = (j <= i) ? __expf(Gi - ms->G[j]) * x[e] * ms->invr[j] : 0.f;
                 }
             }
-            st_chunks_split(rec + REC_P, rec + REC_P + 8192, i, 4 * ch, 4, x);
+            st_chunks_split_global(rec + REC_P, rec + REC_P + 8192, i, 4 * ch, 4, x);
         } else {
             const int i = row - CH;
             const float bi = ms->bco[i] * ms->invr[i];
@@ -317,29 +317,31 @@ __global__ void __launch_bounds__(PT, 3)
         tmem_ld_wait();
 #pragma unroll
         for (int e = 0; e < 32; ++e) x[e] = -x[e];
-        st_chunks_bf16(rec + REC_W, row, 4 * ch, 4, x);
+        st_chunks_bf16_global(rec + REC_W, row, 4 * ch, 4, x);
         tmem_ld32(tmem + lane_base + PM_U + 32 * ch, x);
         tmem_ld_wait();
         float* up = reinterpret_cast<float*>(rec + REC_UP);
 #pragma unroll
         for (int e = 0; e < 32; ++e) up[(32 * ch + e) * DV + row] = x[e];
+        // Ktil row j, dk block blk, logical chunks cq .. cq + 3, in pairs (one 32-byte store
+        // each); the pair order alternates with blk so the two blocks' reads of a row (16 KB
+        // apart, same banks) do not collide
         const int j = tid >> 2, blk = (tid >> 1) & 1, cq = 4 * (tid & 1);
         const float sc = ms->del[j] * ms->invr[j];
+        const uint8_t* krow = qk + blk * 16384 + 8192 + j * 128;  // K row j: swizzle phase (64 + j) & 7 == j & 7
 #pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
-            const int cc = cq + ((c4 + j) & 3);  // rotated by row: no bank conflicts
-            float f[8], hi[8], lo[8];
-            const uint32_t off = (uint32_t)(j * 128 + cc * 16);  // same swizzle phase: (64 + j) & 7 == j & 7
-            unpack_bf16x8(*reinterpret_cast<const uint4*>(qk + blk * 16384 + 8192 + off), f);
+        for (int pp = 0; pp < 2; ++pp) {
+            const int c = cq + 2 * ((pp + blk) & 1);
+            float f[16];
+            unpack_bf16x8(*reinterpret_cast<const uint4*>(krow + ((c ^ (j & 7)) << 4)), f);
+            unpack_bf16x8(*reinterpret_cast<const uint4*>(krow + (((c + 1) ^ (j & 7)) << 4)), f + 8);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) split_bf16(f[e] * sc, hi[e], lo[e]);
-            uint4 uh, ul;
-            uh.x = pack_bf16x2(hi[0], hi[1]); uh.y = pack_bf16x2(hi[2], hi[3]);
-            uh.z = pack_bf16x2(hi[4], hi[5]); uh.w = pack_bf16x2(hi[6], hi[7]);
-            ul.x = pack_bf16x2(lo[0], lo[1]); ul.y = pack_bf16x2(lo[2], lo[3]);
-            ul.z = pack_bf16x2(lo[4], lo[5]); ul.w = pack_bf16x2(lo[6], lo[7]);
-            *reinterpret_cast<uint4*>(rec + REC_KT + blk * 8192 + off) = uh;
-            *reinterpret_cast<uint4*>(rec + REC_KTLO + blk * 8192 + off) = ul;
+            for (int e = 0; e < 16; ++e) f[e] *= sc;
+            uint4 h0, l0, h1, l1;
+            split_chunk8(f, h0, l0);
+            split_chunk8(f + 8, h1, l1);
+            st_pair_sw128_global(rec + REC_KT + blk * 8192, j, c, h0, h1);
+            st_pair_sw128_global(rec + REC_KTLO + blk * 8192, j, c, l0, l1);
         }
     }
 done:

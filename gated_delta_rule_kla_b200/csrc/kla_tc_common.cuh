@@ -172,6 +172,55 @@ __device__ __forceinline__ void invert_unit_lower64_doubling(float* Lf, float* X
     inverse_join_level<32, NT>(Lf, X, tid);
 }
 
+// Store the 16-byte chunks c and c + 1 (c even) of row r of a 128B-swizzled [rows x 64] bf16
+// block in global memory with one 32-byte store: under the swizzle they are the two halves of
+// one aligned 32-byte sector (physical chunks c ^ (r & 7) and that ^ 1), in either order.
+// `block` must be 32-byte aligned.
+__device__ __forceinline__ void st_pair_sw128_global(uint8_t* block, int r, int c, uint4 a, uint4 b) {
+    const int p = c ^ (r & 7);
+    uint8_t* dst = block + r * 128 + ((p & ~1) << 4);
+    const uint4 f = (p & 1) ? b : a, g = (p & 1) ? a : b;
+    asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(dst), "r"(f.x), "r"(f.y),
+                 "r"(f.z), "r"(f.w), "r"(g.x), "r"(g.y), "r"(g.z), "r"(g.w)
+                 : "memory");
+}
+
+// bf16 hi/lo words of 8 fp32 values (one 16-byte chunk of each of the two blocks).
+__device__ __forceinline__ void split_chunk8(const float* v, uint4& uh, uint4& ul) {
+    float h[8], l[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) split_bf16(v[e], h[e], l[e]);
+    uh.x = pack_bf16x2(h[0], h[1]); uh.y = pack_bf16x2(h[2], h[3]);
+    uh.z = pack_bf16x2(h[4], h[5]); uh.w = pack_bf16x2(h[6], h[7]);
+    ul.x = pack_bf16x2(l[0], l[1]); ul.y = pack_bf16x2(l[2], l[3]);
+    ul.z = pack_bf16x2(l[4], l[5]); ul.w = pack_bf16x2(l[6], l[7]);
+}
+
+// Global versions of st_chunks_split / st_chunks_bf16 for an even count of chunks starting
+// at an even chunk: 32-byte stores, whole sectors.
+__device__ __forceinline__ void st_chunks_split_global(uint8_t* hi_block, uint8_t* lo_block, int r, int c0, int n,
+                                                       const float* v) {
+#pragma unroll
+    for (int c = 0; c < n; c += 2) {
+        uint4 h0, l0, h1, l1;
+        split_chunk8(v + 8 * c, h0, l0);
+        split_chunk8(v + 8 * c + 8, h1, l1);
+        st_pair_sw128_global(hi_block, r, c0 + c, h0, h1);
+        st_pair_sw128_global(lo_block, r, c0 + c, l0, l1);
+    }
+}
+__device__ __forceinline__ void st_chunks_bf16_global(uint8_t* block, int r, int c0, int n, const float* v) {
+#pragma unroll
+    for (int c = 0; c < n; c += 2) {
+        uint4 a, b;
+        a.x = pack_bf16x2(v[8 * c + 0], v[8 * c + 1]); a.y = pack_bf16x2(v[8 * c + 2], v[8 * c + 3]);
+        a.z = pack_bf16x2(v[8 * c + 4], v[8 * c + 5]); a.w = pack_bf16x2(v[8 * c + 6], v[8 * c + 7]);
+        b.x = pack_bf16x2(v[8 * c + 8], v[8 * c + 9]); b.y = pack_bf16x2(v[8 * c + 10], v[8 * c + 11]);
+        b.z = pack_bf16x2(v[8 * c + 12], v[8 * c + 13]); b.w = pack_bf16x2(v[8 * c + 14], v[8 * c + 15]);
+        st_pair_sw128_global(block, r, c0 + c, a, b);
+    }
+}
+
 // Write chunks [c0, c0 + n) of row r of a swizzled bf16 block from 8*n fp32 values.
 __device__ __forceinline__ void st_chunks_bf16(uint8_t* block, int r, int c0, int n, const float* v) {
 #pragma unroll
