@@ -790,7 +790,7 @@ int sm_count() {
 }
 
 // Segments per head for the state pass: minimise, in units of one state step,
-// pass 1 (two CTAs per segment, one CTA per SM) + pass 2 + the fp32 scan (~7 steps per segment).
+// pass 1 (two CTAs per segment, one CTA per SM) + pass 2 + the fp32 scan (~1 step per segment).
 int choose_nseg_split(int BH, int NC) {
     const int sms = sm_count();
     auto waves = [&](long long ctas) { return (ctas + sms - 1) / sms; };
@@ -799,7 +799,7 @@ int choose_nseg_split(int BH, int NC) {
     int best = 1;
     for (int ns = 2; ns <= 64 && ns <= NC; ++ns) {
         const long long per = (NC + ns - 1) / ns;
-        const long long cost = waves(2LL * BH * ns) * per + waves((long long)BH * ns) * per + 7LL * ns;
+        const long long cost = waves(2LL * BH * ns) * per + waves((long long)BH * ns) * per + ns;
         if (cost < best_cost) {
             best_cost = cost;
             best = ns;

@@ -628,55 +628,51 @@ namespace {
 
 constexpr int SCAN_LD = 129;  // padded row of M in shared memory
 
+// One CTA per (head, 16-column slice of the state): the columns of S evolve independently,
+// S_{s+1}[:, cols] = M_s S_s[:, cols] + N_s[:, cols].
+constexpr int SCAN_W = 16;  // state columns per CTA
+
 __global__ void __launch_bounds__(256) seg_scan_kernel(const float* __restrict__ S0, const float* __restrict__ MN,
                                                        float* __restrict__ Sstart, float* __restrict__ S_T, int BH,
                                                        int nseg) {
     extern __shared__ float scan_sm[];
-    float* Ss = scan_sm;             // 128 x 128 current state
-    float* Ms = Ss + DK * DV;        // 128 x SCAN_LD transition of the segment
-    const int head = blockIdx.x, tid = threadIdx.x;
-    const int tx = tid & 15, ty = tid >> 4;
+    float* Ms = scan_sm;                 // 128 x SCAN_LD transition of the segment
+    float* Ss = Ms + DK * SCAN_LD;       // 128 x SCAN_W current state columns
+    const int head = blockIdx.x, c0 = blockIdx.y * SCAN_W, tid = threadIdx.x;
+    const int tx = tid & (SCAN_W - 1), ty = tid >> 4;  // column, row group (rows ty + 16 i)
     const size_t SZ = (size_t)DK * DV;
-    for (int x = tid; x < DK * DV; x += 256) Ss[x] = S0 ? S0[head * SZ + x] : 0.f;
-    __syncthreads();
+    for (int x = tid; x < DK * SCAN_W; x += 256) {
+        const int r = x / SCAN_W, c = x % SCAN_W;
+        Ss[x] = S0 ? S0[head * SZ + (size_t)r * DV + c0 + c] : 0.f;
+    }
     for (int sgm = 0; sgm < nseg; ++sgm) {
         const float* M = MN + ((size_t)BH + head) * nseg * SZ + (size_t)sgm * SZ;   // kind 1
         const float* N = MN + (size_t)head * nseg * SZ + (size_t)sgm * SZ;          // kind 0
         float* out = Sstart + ((size_t)head * nseg + sgm) * SZ;
-        for (int x = tid; x < DK * DV; x += 256) {
-            out[x] = Ss[x];
-            Ms[(x / DV) * SCAN_LD + x % DV] = M[x];
+        for (int x = tid; x < DK * DV / 4; x += 256) {
+            const float4 m4 = reinterpret_cast<const float4*>(M)[x];
+            float* dst = Ms + (4 * x / DV) * SCAN_LD + (4 * x) % DV;
+            dst[0] = m4.x; dst[1] = m4.y; dst[2] = m4.z; dst[3] = m4.w;
         }
-        __syncthreads();
-        float acc[8][8];
+        __syncthreads();  // M and the current columns are in place
+        for (int x = tid; x < DK * SCAN_W; x += 256) out[(size_t)(x / SCAN_W) * DV + c0 + x % SCAN_W] = Ss[x];
+        float acc[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-#pragma unroll
-            for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
-#pragma unroll 2
+        for (int i = 0; i < 8; ++i) acc[i] = N[(size_t)(ty + 16 * i) * DV + c0 + tx];
+#pragma unroll 4
         for (int kk = 0; kk < DK; ++kk) {
-            float av[8], bv[8];
+            const float b = Ss[kk * SCAN_W + tx];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) av[i] = Ms[(ty + 16 * i) * SCAN_LD + kk];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) bv[j] = Ss[kk * DV + tx + 16 * j];
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-#pragma unroll
-                for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+            for (int i = 0; i < 8; ++i) acc[i] = fmaf(Ms[(ty + 16 * i) * SCAN_LD + kk], b, acc[i]);
         }
         __syncthreads();  // every read of S and M is done
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const int r = ty + 16 * i, c = tx + 16 * j;
-                Ss[r * DV + c] = acc[i][j] + N[r * DV + c];
-            }
+        for (int i = 0; i < 8; ++i) Ss[(ty + 16 * i) * SCAN_W + tx] = acc[i];
         __syncthreads();
     }
     if (S_T)
-        for (int x = tid; x < DK * DV; x += 256) S_T[head * SZ + x] = Ss[x];
+        for (int x = tid; x < DK * SCAN_W; x += 256)
+            S_T[head * SZ + (size_t)(x / SCAN_W) * DV + c0 + x % SCAN_W] = Ss[x];
 }
 
 int sm_count_tc() {
@@ -714,10 +710,10 @@ int choose_nseg(int BH, int NC) {
 
 cudaError_t launch_seg_scan(const float* S0, const float* MN, float* Sstart, float* S_T, int BH, int nseg,
                             cudaStream_t st) {
-    const size_t scan_smem = sizeof(float) * (DK * DV + DK * SCAN_LD);
+    const size_t scan_smem = sizeof(float) * (DK * SCAN_LD + DK * SCAN_W);
     cudaError_t e = cudaFuncSetAttribute(seg_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)scan_smem);
     if (e != cudaSuccess) return e;
-    seg_scan_kernel<<<BH, 256, scan_smem, st>>>(S0, MN, Sstart, S_T, BH, nseg);
+    seg_scan_kernel<<<dim3(BH, DV / SCAN_W), 256, scan_smem, st>>>(S0, MN, Sstart, S_T, BH, nseg);
     return cudaGetLastError();
 }
 
