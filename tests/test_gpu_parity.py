@@ -192,6 +192,54 @@ def test_fwd_prep_and_state_stages_equal_one_call(kla, B, T, H):
     assert torch.equal(o, o2) and torch.equal(ST, ST2) and torch.equal(Sc, Sc2)
 
 
+def test_fwd_split_more_heads_than_sms(kla, oracle_mod):
+    """B*H = 200 heads: the state pass needs two waves of CTAs; sampled heads vs the oracle."""
+    inp = small_inputs(2, 150, 100, 128, 128, "bf16", seed=77, g_lo=-0.2)
+    d = {k: (v.cuda() if v is not None else None) for k, v in inp.items()}
+    o, ST = kla.chunk_fwd(d["q"], d["k"], d["v"], d["eta"], d["g"], 1e-6, d["S0"])
+    torch.cuda.synchronize()
+    kla.check_device_error()
+    pairs = [(0, 0), (0, 99), (1, 37), (1, 99)]
+    args = [heads_slice(np64(inp[k]), pairs) for k in ("q", "k", "v", "eta", "g")]
+    ro, rST = oracle_mod.forward(*args, 1e-6, heads_slice(np64(inp["S0"]), pairs, state=True))
+    assert rel_err(heads_slice(np64(o), pairs), ro) <= 2e-2
+    assert rel_err(heads_slice(np64(ST), pairs, state=True), rST) <= 2e-2
+
+
+def test_fwd_split_zero_norm_key_and_zero_eta(kla, oracle_mod):
+    """Split path edge cases: a key of zero norm with eps = 0 skips its write, eta = 0 only
+    decays, and a chunk of only masked-out writes leaves the state decayed."""
+    inp = small_inputs(1, 200, 2, 128, 128, "bf16", seed=13, g_lo=-0.1)
+    inp["k"][0, 3] = 0.0
+    inp["k"][0, 100, 1] = 0.0
+    inp["eta"][0, 64:128] = 0.0
+    d = {k: (v.cuda() if v is not None else None) for k, v in inp.items()}
+    o, ST = kla.chunk_fwd(d["q"], d["k"], d["v"], d["eta"], d["g"], 0.0, d["S0"])
+    torch.cuda.synchronize()
+    kla.check_device_error()
+    ro, rST = oracle_mod.forward(*(np64(inp[k]) for k in ("q", "k", "v", "eta", "g")), 0.0, np64(inp["S0"]))
+    assert rel_err(o, ro) <= 2e-2
+    assert rel_err(ST, rST) <= 2e-2
+
+
+def test_fwd_segmented_in_place_state_and_bf16_out(kla, oracle_mod):
+    """Segmented state pass with S_T written over S0 and a bf16 readout."""
+    T, H = 4096 + 37, 2
+    inp = small_inputs(1, T, H, 128, 128, "bf16", seed=19, g_lo=-0.05)
+    d = {k: (v.cuda() if v is not None else None) for k, v in inp.items()}
+    S = d["S0"].clone()
+    o16, S_out = kla.chunk_fwd(d["q"], d["k"], d["v"], d["eta"], d["g"], 1e-6, S, S_T=S, out_dtype=torch.bfloat16)
+    o32, ST32 = kla.chunk_fwd(d["q"], d["k"], d["v"], d["eta"], d["g"], 1e-6, d["S0"])
+    torch.cuda.synchronize()
+    kla.check_device_error()
+    assert S_out.data_ptr() == S.data_ptr()
+    torch.testing.assert_close(o16, o32.to(torch.bfloat16), rtol=0, atol=0)
+    torch.testing.assert_close(S, ST32, rtol=0, atol=0)
+    ro, rST = oracle_mod.forward(*(np64(inp[k]) for k in ("q", "k", "v", "eta", "g")), 1e-6, np64(inp["S0"]))
+    assert rel_err(o32, ro) <= 2e-2
+    assert rel_err(S, rST) <= 2e-2
+
+
 def test_fwd_state_passing_equals_one_call(kla):
     """Checkpoint/resume: forward(T1) then forward(T2, S0=S_T1) == forward(T1+T2)."""
     inp = small_inputs(2, 320, 2, 128, 128, "f32", seed=5, g_lo=-0.05)
