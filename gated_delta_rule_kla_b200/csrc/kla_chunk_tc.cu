@@ -617,12 +617,11 @@ cudaError_t launch_chunk_fwd_tc(const FwdArgs& a, cudaStream_t st) {
 }
 
 // ------------------------------------------------------------------------------------
-// Segmented long-sequence forward.  The state map of a run of chunks is affine,
-// S_end = M S_start + N (the recurrence is linear in the state and in the values), so:
-//   pass 1: every segment twice in parallel -- from S = 0 with its values (gives N_s) and
-//           from S = I with zero values (gives M_s);
-//   scan:   S_{s+1} = M_s S_s + N_s per (b, h) in fp32, recording each segment's start;
-//   pass 2: every segment from its true start state, producing o (and S_chunks).
+// Scan over segments for the segmented state pass (kla_chunk_split.cu).  The state map of a
+// run of chunks is affine, S_end = M S_start + N (the recurrence is linear in the state and
+// in the values): pass 1 runs every segment from S = 0 with its values (gives N_s) and from
+// S = I with zero values (gives M_s); this scan chains S_{s+1} = M_s S_s + N_s per (b, h) in
+// fp32, recording each segment's start; pass 2 runs every segment from its true start.
 // ------------------------------------------------------------------------------------
 namespace {
 
@@ -675,37 +674,6 @@ __global__ void __launch_bounds__(256) seg_scan_kernel(const float* __restrict__
             S_T[head * SZ + (size_t)(x / SCAN_W) * DV + c0 + x % SCAN_W] = Ss[x];
 }
 
-int sm_count_tc() {
-    static int n = 0;
-    if (n == 0) {
-        int dev = 0;
-        if (cudaGetDevice(&dev) != cudaSuccess ||
-            cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
-            n = 148;
-    }
-    return n;
-}
-
-// Segment count minimising a simple model of the run time in units of one chunk step:
-// pass 1 (two CTAs per segment) + pass 2 (one) + the scan (about one step per segment).
-int choose_nseg(int BH, int NC) {
-    const int sms = sm_count_tc();
-    auto waves = [&](long long ctas) { return (ctas + sms - 1) / sms; };
-    long long best_cost = (long long)NC;  // unsegmented: one CTA per head
-    int best = 1;
-    if (BH * 2 > sms) return 1;
-    for (int ns = 2; ns <= 64 && ns <= NC; ++ns) {
-        const long long per = (NC + ns - 1) / ns;
-        const long long cost = waves(2LL * BH * ns) * per + waves((long long)BH * ns) * per + ns;
-        if (cost < best_cost) {
-            best_cost = cost;
-            best = ns;
-        }
-    }
-    // require a clear gain before switching to three launches
-    return (best > 1 && best_cost * 4 < (long long)NC * 3) ? best : 1;
-}
-
 }  // namespace
 
 cudaError_t launch_seg_scan(const float* S0, const float* MN, float* Sstart, float* S_T, int BH, int nseg,
@@ -715,44 +683,6 @@ cudaError_t launch_seg_scan(const float* S0, const float* MN, float* Sstart, flo
     if (e != cudaSuccess) return e;
     seg_scan_kernel<<<dim3(BH, DV / SCAN_W), 256, scan_smem, st>>>(S0, MN, Sstart, S_T, BH, nseg);
     return cudaGetLastError();
-}
-
-size_t chunk_fwd_tc_segmented_workspace(const FwdArgs& a) {
-    if (!(a.bf16 && a.Dk == 128 && a.Dv == 128 && a.T > 0)) return 0;  // shapes of the tensor-core path
-    const int NC = (a.T + CH - 1) / CH;
-    const int nseg = choose_nseg(a.B * a.H, NC);
-    if (nseg <= 1) return 0;
-    return (size_t)3 * a.B * a.H * nseg * DK * DV * sizeof(float);
-}
-
-cudaError_t launch_chunk_fwd_tc_segmented(const FwdArgs& a, void* ws, cudaStream_t st) {
-    const int NC = (a.T + CH - 1) / CH;
-    const int BH = a.B * a.H;
-    const int nseg = choose_nseg(BH, NC);
-    if (nseg <= 1) return launch_chunk_fwd_tc(a, st);
-    const int segc = (NC + nseg - 1) / nseg;
-    const int nseg_used = (NC + segc - 1) / segc;
-    const size_t SZ = (size_t)DK * DV;
-    float* MN = static_cast<float*>(ws);                  // [2, BH, nseg, DK, DV]
-    float* Sstart = MN + 2 * (size_t)BH * nseg_used * SZ;  // [BH, nseg, DK, DV]
-    FwdArgs p1 = a;
-    p1.S0 = nullptr;
-    p1.o = nullptr;
-    p1.S_T = MN;
-    p1.S_chunks = nullptr;
-    p1.nseg = nseg_used;
-    p1.seg_chunks = segc;
-    p1.kinds = 2;
-    cudaError_t e = launch_chunk_fwd_tc(p1, st);
-    if (e != cudaSuccess) return e;
-    if ((e = launch_seg_scan(a.S0, MN, Sstart, a.S_T, BH, nseg_used, st)) != cudaSuccess) return e;
-    FwdArgs p2 = a;
-    p2.S0 = Sstart;
-    p2.S_T = nullptr;
-    p2.nseg = nseg_used;
-    p2.seg_chunks = segc;
-    p2.kinds = 1;
-    return launch_chunk_fwd_tc(p2, st);
 }
 
 cudaError_t tc_take_error(cudaStream_t st, unsigned int* flag) {

@@ -30,7 +30,7 @@ struct FwdArgs {
     int B, T, H, Dk, Dv;
     bool bf16;      // q, k, v are bf16 (else fp32)
     bool out_bf16;  // o is bf16 (else fp32)
-    // Segmented long-sequence mode (tensor-core kernel only).  nseg > 1 splits each sequence
+    // Segmented long-sequence mode (tensor-core kernels).  nseg > 1 splits each sequence
     // into nseg runs of seg_chunks chunks processed by separate CTAs; S0 and S_T then index
     // [B*H, nseg, Dk, Dv] (S_T: [kinds, B*H, nseg, Dk, Dv]) and a second grid row (kind 1)
     // runs each segment from the identity state with zero values (the segment's transition).
@@ -59,11 +59,6 @@ cudaError_t launch_chunk_bwd_simt(const BwdArgs& a, cudaStream_t st);
 // Tensor-core (tcgen05) forward for bf16 inputs with Dk == Dv == 128.
 bool chunk_fwd_tc_supported(const FwdArgs& a);
 cudaError_t launch_chunk_fwd_tc(const FwdArgs& a, cudaStream_t st);
-// Workspace bytes of the segmented long-sequence forward for these sizes (0: not used).
-size_t chunk_fwd_tc_segmented_workspace(const FwdArgs& a);
-// Segmented forward: per-segment transitions in parallel, a scan over segments, then the
-// outputs of every segment from its true start state.  ws must hold the size above.
-cudaError_t launch_chunk_fwd_tc_segmented(const FwdArgs& a, void* ws, cudaStream_t st);
 // Sequential fp32 scan over segments: S_{s+1} = M_s S_s + N_s per head, recording each
 // segment's start in Sstart [BH, nseg, Dk, Dv] (MN: [2, BH, nseg, Dk, Dv], N first) and the
 // final state in S_T (may be null).
