@@ -120,14 +120,29 @@ __device__ __forceinline__ void inverse_join_level(float* Lf, float* X, int tid)
     const int idx = tid * PER;
     const int p = idx / (S * S), rem = idx % (S * S), i = rem / S, j0 = rem % S;
     const int A0 = 2 * S * p, B0 = A0 + S;
+    // PER adjacent floats at a 4*PER-byte aligned address (rows of LDL = 68 floats, j0 a
+    // multiple of PER, block offsets multiples of 8): one vector load.
+    auto ld = [](const float* p, float (&v)[PER]) {
+        if constexpr (PER == 4) {
+            const float4 t = *reinterpret_cast<const float4*>(p);
+            v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
+        } else if constexpr (PER == 2) {
+            const float2 t = *reinterpret_cast<const float2*>(p);
+            v[0] = t.x; v[1] = t.y;
+        } else {
+            v[0] = *p;
+        }
+    };
     float acc[PER];
 #pragma unroll
     for (int e = 0; e < PER; ++e) acc[e] = 0.f;
     // X_p = L_BA T_A   (T_A lower triangular: zero above its diagonal)
+    const float* lrow = Lf + (B0 + i) * LDL;
 #pragma unroll 8
     for (int k = 0; k < S; ++k) {
-        const float l = Lf[(B0 + i) * LDL + A0 + k];
-        const float* t = Lf + (A0 + k) * LDL + A0 + j0;
+        const float l = lrow[A0 + k];
+        float t[PER];
+        ld(Lf + (A0 + k) * LDL + A0 + j0, t);
 #pragma unroll
         for (int e = 0; e < PER; ++e) acc[e] = fmaf(l, t[e], acc[e]);
     }
@@ -139,13 +154,20 @@ __device__ __forceinline__ void inverse_join_level(float* Lf, float* X, int tid)
     for (int e = 0; e < PER; ++e) acc[e] = 0.f;
 #pragma unroll 8
     for (int k = 0; k < S; ++k) {
-        const float l = Lf[(B0 + i) * LDL + B0 + k];
-        const float* x = X + p * S * S + k * S + j0;
+        const float l = lrow[B0 + k];
+        float x[PER];
+        ld(X + p * S * S + k * S + j0, x);
 #pragma unroll
         for (int e = 0; e < PER; ++e) acc[e] = fmaf(l, x[e], acc[e]);
     }
-#pragma unroll
-    for (int e = 0; e < PER; ++e) Lf[(B0 + i) * LDL + A0 + j0 + e] = -acc[e];
+    float* dst = Lf + (B0 + i) * LDL + A0 + j0;
+    if constexpr (PER == 4) {
+        *reinterpret_cast<float4*>(dst) = make_float4(-acc[0], -acc[1], -acc[2], -acc[3]);
+    } else if constexpr (PER == 2) {
+        *reinterpret_cast<float2*>(dst) = make_float2(-acc[0], -acc[1]);
+    } else {
+        dst[0] = -acc[0];
+    }
     __syncthreads();
 }
 
