@@ -92,25 +92,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int ch = tid >> 7;    // which half of an epilogue's columns this thread takes
     const int H = a.H, T = a.T;
     const int NCtot = (T + CH - 1) / CH;
-    // segment handled by this CTA: chunks [c0, c1) of head (b, h); kind 1 = transition pass
-    const int nseg = a.nseg > 1 ? a.nseg : 1;
-    const bool segmented = a.nseg > 1;
-    const int segc = segmented ? a.seg_chunks : NCtot;
-    const int head_idx = blockIdx.x / nseg, seg = blockIdx.x % nseg;
-    const int BH = gridDim.x / nseg;
+    // one CTA per head (b, h), every chunk [c0, c1) of its sequence in order
+    const int head_idx = blockIdx.x;
     const int b = head_idx / H, h = head_idx % H;
-    const bool ident = blockIdx.y == 1;
-    const int c0 = seg * segc, c1 = min(NCtot, c0 + segc);
-    const int NC = c1 > c0 ? c1 - c0 : 0;  // chunks of this CTA
+    const int c0 = 0, c1 = NCtot;
+    const int NC = NCtot;
     const uint32_t sbase = smem_u32(sm);
     const uint32_t bar_full0 = smem_u32(&ms->full[0]);
     const uint32_t bar_mma = smem_u32(&ms->mma);
-    const float* S0p = (a.S0 && !ident)
-                           ? a.S0 + (size_t)(segmented ? head_idx * nseg + seg : head_idx) * DK * DV
-                           : nullptr;
-    float* STp = a.S_T ? a.S_T + (size_t)(segmented ? ((size_t)blockIdx.y * BH + head_idx) * nseg + seg : head_idx) *
-                                     DK * DV
-                       : nullptr;
+    const float* S0p = a.S0 ? a.S0 + (size_t)head_idx * DK * DV : nullptr;
+    float* STp = a.S_T ? a.S_T + (size_t)head_idx * DK * DV : nullptr;
 
     if (tid == 0) {
         mbar_init(bar_full0, 1);
@@ -146,7 +137,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     // Initial state: this thread holds row dk = `row`, columns [64 ch, 64 ch + 64).
     {
         const float g0 = (NC > 0) ? __expf(ms->gsum[0] + ms->gsum[1]) : 1.f;
-        float4* sc0 = (a.S_chunks && NC > 0 && !ident)
+        float4* sc0 = (a.S_chunks && NC > 0)
                           ? reinterpret_cast<float4*>(a.S_chunks + ((size_t)head_idx * NCtot + c0) * DK * DV +
                                                       (size_t)row * DV + 64 * ch)
                           : nullptr;
@@ -162,7 +153,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 }
             } else {
 #pragma unroll
-                for (int i = 0; i < 32; ++i) x[i] = (ident && row == 64 * ch + 32 * q2 + i) ? 1.f : 0.f;
+                for (int i = 0; i < 32; ++i) x[i] = 0.f;
             }
             if (sc0) {
 #pragma unroll
@@ -270,7 +261,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 }
             const KaczCoef cf = kacz_coef(ms->eta[j], r2, a.eps);
             ms->bco[j] = cf.b;
-            ms->cco[j] = ident ? 0.f : cf.c;  // the transition pass runs with zero values
+            ms->cco[j] = cf.c;
             ms->invr[j] = cf.inv_r;
         }
         if (warp == 0) {  // inclusive prefix sum of g inside the chunk (2 tokens per lane)
@@ -495,7 +486,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         {
             const bool has_next = c + 1 < c1;
             const float gN = has_next ? __expf(ms->gsum[0] + ms->gsum[1]) : 1.f;
-            float4* scn = (a.S_chunks && has_next && !ident)
+            float4* scn = (a.S_chunks && has_next)
                               ? reinterpret_cast<float4*>(a.S_chunks + ((size_t)head_idx * NCtot + c + 1) * DK * DV +
                                                           (size_t)row * DV + 64 * ch)
                               : nullptr;
@@ -599,8 +590,7 @@ cudaError_t launch_chunk_fwd_tc(const FwdArgs& a, cudaStream_t st) {
     if (!make_map(&mq, a.q, a.B, a.T, a.H) || !make_map(&mk, a.k, a.B, a.T, a.H) ||
         !make_map(&mv, a.v, a.B, a.T, a.H))
         return cudaErrorInvalidValue;
-    const int nseg = a.nseg > 1 ? a.nseg : 1;
-    const dim3 grid(a.B * a.H * nseg, a.kinds > 1 ? a.kinds : 1);
+    const dim3 grid(a.B * a.H);
     cudaError_t e;
     if (a.out_bf16) {
         e = cudaFuncSetAttribute(chunk_fwd_tc_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -30,7 +30,7 @@ struct FwdArgs {
     int B, T, H, Dk, Dv;
     bool bf16;      // q, k, v are bf16 (else fp32)
     bool out_bf16;  // o is bf16 (else fp32)
-    // Segmented long-sequence mode (tensor-core kernels).  nseg > 1 splits each sequence
+    // Segmented long-sequence mode (split state pass only).  nseg > 1 splits each sequence
     // into nseg runs of seg_chunks chunks processed by separate CTAs; S0 and S_T then index
     // [B*H, nseg, Dk, Dv] (S_T: [kinds, B*H, nseg, Dk, Dv]) and a second grid row (kind 1)
     // runs each segment from the identity state with zero values (the segment's transition).
