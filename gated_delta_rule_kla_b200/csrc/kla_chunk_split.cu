@@ -380,8 +380,7 @@ constexpr uint32_t SO_Q = 0, SO_W = 16384, SO_KT = 32768, SO_KTLO = 49152, SO_P 
 static_assert(SO_W == REC_W + 16384 && SO_KT == REC_KT + 16384 && SO_KTLO == REC_KTLO + 16384 &&
                   SO_P == REC_P + 16384 && SO_UP == REC_UP + 16384,
               "stage mirrors the record");
-constexpr uint32_t EARLY_BYTES = S_STAGE - SO_KT;        // Ktil, P, U': free once chunk c's MMAs finish
-constexpr uint32_t LATE_BYTES = 16384 + 16384 + REC_SCB;  // Q, W, scalars: after the o tile left
+static_assert(S_STAGE - SO_KT == 32768 + 16384 + 32768, "early part: Ktil, P, U'");
 constexpr uint32_t S_SC = 2 * S_STAGE;  // 2 x 512 B record scalars
 constexpr uint32_t S_MISC = S_SC + 2 * REC_SCB;
 constexpr uint32_t S_SMEM = S_MISC + 128 + 1024;
@@ -465,6 +464,9 @@ __global__ void __launch_bounds__(ST, 1)
                        : nullptr;
     float* Sc = (a.S_chunks && !ident) ? a.S_chunks + (size_t)head_idx * NCtot * DK * DV : nullptr;
     const bool write_o = !ident && a.o != nullptr;
+    // Without outputs (the transition pass of the segmented mode) Q, P and the O products are not
+    // needed; with zero values (its identity kind) neither is U'.
+    const bool need_vals = !ident;
 
     if (tid == 0) {
         mbar_init(bar_full0, 1);
@@ -506,22 +508,30 @@ __global__ void __launch_bounds__(ST, 1)
             if (write_o) prefetch_tmap(&tm_o);
             // The early part (Ktil, P, U') and the late part (Q, W, scalars) of chunk c; the
             // late part carries the phase's one arrival.
+            const uint32_t early_bytes = 32768 + (write_o ? 16384 : 0) + (need_vals ? 32768 : 0);
+            const uint32_t late_bytes = 16384 + REC_SCB + (write_o ? 16384 : 0);
             auto load_early = [&](int c, int st) {
                 const uint32_t bar = bar_full0 + 8 * st;
                 const uint32_t base = sbase + st * S_STAGE;
                 const uint8_t* rec = recs + ((size_t)head_idx * NCtot + c) * REC_BYTES;
-                mbar_expect_tx_only(bar, EARLY_BYTES);
-#pragma unroll
-                for (int p = 0; p < 5; ++p)
-                    bulk_load(base + SO_KT + p * 16384, rec + REC_KT + p * 16384, 16384, bar);
+                mbar_expect_tx_only(bar, early_bytes);
+                bulk_load(base + SO_KT, rec + REC_KT, 16384, bar);
+                bulk_load(base + SO_KTLO, rec + REC_KTLO, 16384, bar);
+                if (write_o) bulk_load(base + SO_P, rec + REC_P, 16384, bar);
+                if (need_vals) {
+                    bulk_load(base + SO_UP, rec + REC_UP, 16384, bar);
+                    bulk_load(base + SO_UP + 16384, rec + REC_UP + 16384, 16384, bar);
+                }
             };
             auto load_late = [&](int c, int st) {
                 const uint32_t bar = bar_full0 + 8 * st;
                 const uint32_t base = sbase + st * S_STAGE;
                 const uint8_t* rec = recs + ((size_t)head_idx * NCtot + c) * REC_BYTES;
-                mbar_expect_tx(bar, LATE_BYTES);
-                tma_load_4d(base + SO_Q, &tm_q, bar, 0, h, c * CH, b);
-                tma_load_4d(base + SO_Q + 8192, &tm_q, bar, 64, h, c * CH, b);
+                mbar_expect_tx(bar, late_bytes);
+                if (write_o) {
+                    tma_load_4d(base + SO_Q, &tm_q, bar, 0, h, c * CH, b);
+                    tma_load_4d(base + SO_Q + 8192, &tm_q, bar, 64, h, c * CH, b);
+                }
                 bulk_load(base + SO_W, rec + REC_W, 16384, bar);
                 bulk_load(sbase + S_SC + st * REC_SCB, rec + REC_SC, REC_SCB, bar);
             };
@@ -590,18 +600,20 @@ __global__ void __launch_bounds__(ST, 1)
                 if (aborted) break;
                 mma_commit(bar_u);
                 // O1 = S^T Q^T, once the previous chunk's outputs are read
-                if (lc > 0 && !mbar_wait_bounded(o_free0 + 8 * (st ^ 1), ((lc - 1) >> 1) & 1, kWaitNs)) {
-                    aborted = true;
-                    break;
+                if (write_o) {
+                    if (lc > 0 && !mbar_wait_bounded(o_free0 + 8 * (st ^ 1), ((lc - 1) >> 1) & 1, kWaitNs)) {
+                        aborted = true;
+                        break;
+                    }
+                    tc_fence_after();
+#pragma unroll
+                    for (int part = 0; part < 2; ++part)
+#pragma unroll
+                        for (int s = 0; s < 8; ++s)
+                            mma_bf16_ts(tmem + TM_O1, tmem + (part ? TM_SL : TM_SH) + 8 * s,
+                                        smem_desc(stg + SO_Q + (s >> 2) * 8192 + (s & 3) * 32, 16, 1024), io,
+                                        (part | s) > 0);
                 }
-                tc_fence_after();
-#pragma unroll
-                for (int part = 0; part < 2; ++part)
-#pragma unroll
-                    for (int s = 0; s < 8; ++s)
-                        mma_bf16_ts(tmem + TM_O1, tmem + (part ? TM_SL : TM_SH) + 8 * s,
-                                    smem_desc(stg + SO_Q + (s >> 2) * 8192 + (s & 3) * 32, 16, 1024), io,
-                                    (part | s) > 0);
                 // S^T += U^T Ktil (N = 128): K steps {0,2} (first half of each thread's tokens),
                 // then {1,3}; products hi x hi, hi x lo, lo x hi
                 const uint32_t ua[3] = {TM_UH, TM_UH, TM_UL};
@@ -623,12 +635,14 @@ __global__ void __launch_bounds__(ST, 1)
                 if (aborted) break;
                 mma_commit(bar_s);
                 // O2 = U^T P^T
+                if (write_o) {
 #pragma unroll
-                for (int p = 0; p < 3; ++p)
+                    for (int p = 0; p < 3; ++p)
 #pragma unroll
-                    for (int s = 0; s < 4; ++s)
-                        mma_bf16_ts(tmem + TM_O2, tmem + ua[p] + 8 * s, smem_desc(pb[p] + s * 32, 16, 1024), io,
-                                    (p | s) > 0);
+                        for (int s = 0; s < 4; ++s)
+                            mma_bf16_ts(tmem + TM_O2, tmem + ua[p] + 8 * s, smem_desc(pb[p] + s * 32, 16, 1024), io,
+                                        (p | s) > 0);
+                }
                 mma_commit(bar_o0 + 8 * st);
             }
             if (aborted) atomicOr(&ms->abort, 1u);
