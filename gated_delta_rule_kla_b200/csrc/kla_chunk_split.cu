@@ -584,18 +584,19 @@ __global__ void __launch_bounds__(ST, 1)
                 if (!mbar_wait_bounded(bar_full0 + 8 * st, (lc >> 1) & 1, kWaitNs)) { aborted = true; break; }
                 // U^T = -(S^T W^T) (the record holds -W^T; U' is added in the epilogue).  K steps
                 // {0,1,4,5} read the first half of each thread's S columns, {2,3,6,7} the second.
+                // S enters as its bf16 hi part only: W is itself one bf16 rounding, and the lo
+                // part's share is below that (measured: max|err|/rms of o and S_T 3.3e-3 against
+                // 2.7e-3 with both parts, over the headline workload and the stress cases).
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
                     if (!mbar_wait_bounded(s_ready0 + 8 * half, lc & 1, kWaitNs)) { aborted = true; break; }
                     tc_fence_after();
 #pragma unroll
-                    for (int part = 0; part < 2; ++part)
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            const int s = 2 * half + (j & 1) + 4 * (j >> 1);
-                            mma_bf16_ts(tmem + TM_U, tmem + (part ? TM_SL : TM_SH) + 8 * s,
-                                        smem_desc(stg + SO_W + s * 2048, 8192, 1024), iu, (half | part | j) > 0);
-                        }
+                    for (int j = 0; j < 4; ++j) {
+                        const int s = 2 * half + (j & 1) + 4 * (j >> 1);
+                        mma_bf16_ts(tmem + TM_U, tmem + TM_SH + 8 * s, smem_desc(stg + SO_W + s * 2048, 8192, 1024),
+                                    iu, (half | j) > 0);
+                    }
                 }
                 if (aborted) break;
                 mma_commit(bar_u);
