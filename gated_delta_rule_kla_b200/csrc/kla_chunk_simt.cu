@@ -18,6 +18,7 @@
 // owns one slice of NV value columns of one (b, h) and walks the chunks in order.
 #include "kla_device.cuh"
 #include "kla_launch.h"
+#include "kla_tc_common.cuh"
 
 namespace kla {
 namespace {
@@ -289,7 +290,7 @@ constexpr size_t fwd_smem_bytes() {
 // Per chunk (newest first) with incoming state S (from S_chunks) and dS' the gradient
 // w.r.t. the chunk's outgoing state:
 //   dU  = (Gam o Q Khat^T)^T dO + Diag(delta) Khat dS'
-//   dR  = (I + L)^{-T} dU                                  (back substitution)
+//   dR  = (I + L)^{-T} dU = T^T dU,  T = (I + L)^{-1} inverted once per chunk (doubling)
 //   dS  = gamma_last dS' + Q^T Diag(gamma) dO - Khat^T Diag(b gamma) dR   (carried on)
 //   dV  = Diag(c) dR,  dc_i = dR_i . v_i
 //   D   = -dR U^T (strictly lower) -> db_i += sum_t D_it (Gam o KK)_it,
@@ -331,6 +332,9 @@ __global__ void __launch_bounds__(NT, 1) chunk_bwd_simt_kernel(BwdArgs a) {
     float* dbs = dGs + C;
     float* dcs = dbs + C;
     float* red = dcs + C;  // 8
+    float* Tf = red + 8;                // C x tcc::LDL   T = (I + L)^{-1}  (16-byte aligned)
+    float* Xinv = Tf + C * tcc::LDL;    // 1024           scratch of the inverse
+    float* Tmp = Xinv + 1024;           // C x LDV        U = T R and dR = T^T dU before copy-back
 
     const int v0 = blockIdx.x * NV, h = blockIdx.y, b = blockIdx.z;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -426,19 +430,26 @@ __global__ void __launch_bounds__(NT, 1) chunk_bwd_simt_kernel(BwdArgs a) {
             Us[i * LDV + j] -= bs[i] * gams[i] * Xs[i * LDV + j];
         }
         __syncthreads();
-        // forward substitution -> U
+        // T = (I + Diag(b) Lh)^{-1} (Lh is zero on and above the diagonal; rows past the last
+        // token are unit rows), then U = T R
+        for (int x = tid; x < C * C; x += NT) {
+            const int i = x / C, j = x % C;
+            Tf[i * tcc::LDL + j] = bs[i] * Lh[i * LDC + j];
+        }
+        __syncthreads();
+        tcc::invert_unit_lower64_doubling<NT>(Tf, Xinv, tid);
         {
-            const int col = tid >> 3, part = tid & 7;
-            for (int i = 1; i < n; ++i) {
-                const float bi = bs[i];
-                float s = 0.f;
-                for (int j = part; j < i; j += 8) s = fmaf(Lh[i * LDC + j], Us[j * LDV + col], s);
-                s += __shfl_xor_sync(0xffffffffu, s, 1);
-                s += __shfl_xor_sync(0xffffffffu, s, 2);
-                s += __shfl_xor_sync(0xffffffffu, s, 4);
-                if (part == 0) Us[i * LDV + col] -= bi * s;
-                __syncthreads();
-            }
+            float au[4][2];
+            zero(au);
+            gemm_acc<C, 4, 2, 16, 16>(au, ty, tx, [&](int i, int j) { return Tf[i * tcc::LDL + j]; },
+                                      [&](int j, int c) { return Us[j * LDV + c]; });
+#pragma unroll
+            for (int m = 0; m < 4; ++m)
+#pragma unroll
+                for (int nn = 0; nn < 2; ++nn) Tmp[(ty + 16 * m) * LDV + tx + 16 * nn] = au[m][nn];
+            __syncthreads();
+            for (int x = tid; x < C * NV; x += NT) Us[(x / NV) * LDV + x % NV] = Tmp[(x / NV) * LDV + x % NV];
+            __syncthreads();
         }
         // dU = P^T dO + Diag(delta) Khat dS'
         {
@@ -455,19 +466,19 @@ __global__ void __launch_bounds__(NT, 1) chunk_bwd_simt_kernel(BwdArgs a) {
                 }
         }
         __syncthreads();
-        // back substitution (I + L)^T dR = dU
+        // dR = T^T dU
         {
-            const int col = tid >> 3, part = tid & 7;
-            for (int i = n - 2; i >= 0; --i) {
-                float s = 0.f;
-                for (int j = i + 1 + part; j < n; j += 8)
-                    s = fmaf(bs[j] * Lh[j * LDC + i], dRs[j * LDV + col], s);
-                s += __shfl_xor_sync(0xffffffffu, s, 1);
-                s += __shfl_xor_sync(0xffffffffu, s, 2);
-                s += __shfl_xor_sync(0xffffffffu, s, 4);
-                if (part == 0) dRs[i * LDV + col] -= s;
-                __syncthreads();
-            }
+            float ar[4][2];
+            zero(ar);
+            gemm_acc<C, 4, 2, 16, 16>(ar, ty, tx, [&](int i, int j) { return Tf[j * tcc::LDL + i]; },
+                                      [&](int j, int c) { return dRs[j * LDV + c]; });
+#pragma unroll
+            for (int m = 0; m < 4; ++m)
+#pragma unroll
+                for (int nn = 0; nn < 2; ++nn) Tmp[(ty + 16 * m) * LDV + tx + 16 * nn] = ar[m][nn];
+            __syncthreads();
+            for (int x = tid; x < C * NV; x += NT) dRs[(x / NV) * LDV + x % NV] = Tmp[(x / NV) * LDV + x % NV];
+            __syncthreads();
         }
         // Row scalars (one warp per row, one column per lane) and dv.
         for (int i = warp; i < n; i += NT / 32) {
@@ -650,8 +661,8 @@ __global__ void __launch_bounds__(NT, 1) chunk_bwd_simt_kernel(BwdArgs a) {
 
 template <int DK>
 constexpr size_t bwd_smem_bytes() {
-    return sizeof(float) *
-           (2 * C * (DK + 1) + 2 * DK * 33 + 6 * C * 33 + 2 * C * (C + 1) + 9 * C + 8);
+    return sizeof(float) * (2 * C * (DK + 1) + 2 * DK * 33 + 6 * C * 33 + 2 * C * (C + 1) + 9 * C + 8 +
+                            C * tcc::LDL + 1024 + C * 33);
 }
 
 // dq to the output type; dk and deta from the unit-key gradients:
