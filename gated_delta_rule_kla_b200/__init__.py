@@ -61,6 +61,8 @@ def lib():
         L.kla_chunk_fwd_state.restype = i
         L.kla_chunk_bwd_workspace.argtypes = [i, i, i, i, i, i, i, i]
         L.kla_chunk_bwd_workspace.restype = sz
+        L.kla_chunk_bwd_workspace_min.argtypes = [i, i, i, i, i, i, i, i]
+        L.kla_chunk_bwd_workspace_min.restype = sz
         L.kla_chunk_bwd.argtypes = [vp, vp, vp, fp, fp, f, fp, vp, fp, fp, vp, vp, vp, fp, fp, fp,
                                     i, i, i, i, i, i, i, i, vp, sz, vp]
         L.kla_chunk_bwd.restype = i
@@ -203,12 +205,14 @@ def chunk_fwd_state(q, g, S0, workspace, *, Dv=None, o=None, S_T=None, S_chunks=
 
 
 def chunk_bwd(q, k, v, eta, g, dO, eps=1e-6, S0=None, dS_T=None, S_chunks=None, *, stream=None,
-              workspace=None, out_dtype=torch.float32):
+              workspace=None, out_dtype=torch.float32, cuda_cores=False):
     """Gradients of the chunkwise forward w.r.t. q, k, v, eta, g and S0.
 
     dO: [B,T,H,Dv] (same dtype as q); dS_T: [B,H,Dk,Dv] fp32 or None; S_chunks: the
     array chunk_fwd(save_chunk_states=True) returned for the same inputs, or None.
-    dq, dk, dv are written in `out_dtype` (fp32 by default).
+    dq, dk, dv are written in `out_dtype` (fp32 by default).  bf16 inputs with
+    Dk == Dv == 128 run on the tensor cores unless `cuda_cores` is set (the workspace is then
+    sized for the CUDA-core backward, which the library runs with a smaller workspace).
     Returns dict(dq, dk, dv, deta, dg, dS0).
     """
     dev = k.device
@@ -227,8 +231,9 @@ def chunk_bwd(q, k, v, eta, g, dO, eps=1e-6, S0=None, dS_T=None, S_chunks=None, 
                deta=torch.empty_like(eta), dg=torch.empty_like(g),
                dS0=torch.empty(B, H, Dk, Dv, device=dev, dtype=torch.float32))
     L = lib()
-    need = L.kla_chunk_bwd_workspace(B, T, H, Dk, Dv, CHUNK, _dtype_code(k), int(S_chunks is not None))
-    if workspace is None or workspace.numel() < need:
+    size = L.kla_chunk_bwd_workspace_min if cuda_cores else L.kla_chunk_bwd_workspace
+    need = size(B, T, H, Dk, Dv, CHUNK, _dtype_code(k), int(S_chunks is not None))
+    if workspace is None or workspace.numel() < need or (cuda_cores and workspace.numel() > need):
         workspace = torch.empty(max(need, 16), device=dev, dtype=torch.uint8)
     st = L.kla_chunk_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(eta), _ptr(g), float(eps), _ptr(S0), _ptr(dO),
                          _ptr(dS_T), _ptr(S_chunks), _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]),

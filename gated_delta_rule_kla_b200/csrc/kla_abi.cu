@@ -8,6 +8,7 @@
 
 #include "kla.h"
 #include "kla_launch.h"
+#include "kla_tc_common.cuh"
 
 namespace {
 
@@ -61,6 +62,11 @@ kla_status check_common(int B, int T, int H, int Dk, int Dv, int chunk, int dtyp
     do {                                                                                       \
         if (!aligned16(p)) return fail(KLA_ERR_INVALID_ARG, "%s must be 16-byte aligned", #p); \
     } while (0)
+
+// Shapes the tensor-core backward serves (bf16, Dk == Dv == 128).
+bool tc_bwd_shape(int T, int Dk, int Dv, int dtype) {
+    return dtype == KLA_BF16 && Dk == 128 && Dv == 128 && T >= 1;
+}
 
 size_t bwd_ws_layout(int B, int T, int H, int Dk, int Dv, bool have_S_chunks, size_t* off) {
     const size_t NC = (size_t)(T + kla::kChunkLen - 1) / kla::kChunkLen;
@@ -198,12 +204,20 @@ kla_status kla_chunk_fwd_state(const void* q, const float* g, const float* S0, v
     return KLA_OK;
 }
 
-size_t kla_chunk_bwd_workspace(int B, int T, int H, int Dk, int Dv, int chunk, int dtype,
-                               int have_S_chunks) {
+size_t kla_chunk_bwd_workspace_min(int B, int T, int H, int Dk, int Dv, int chunk, int dtype,
+                                   int have_S_chunks) {
     (void)chunk; (void)dtype;
     if (B < 1 || H < 1 || T < 0) return 0;
     size_t off[5];
     return bwd_ws_layout(B, T, H, Dk, Dv, have_S_chunks != 0, off);
+}
+
+size_t kla_chunk_bwd_workspace(int B, int T, int H, int Dk, int Dv, int chunk, int dtype,
+                               int have_S_chunks) {
+    const size_t simt = kla_chunk_bwd_workspace_min(B, T, H, Dk, Dv, chunk, dtype, have_S_chunks);
+    if (!tc_bwd_shape(T, Dk, Dv, dtype)) return simt;
+    const size_t tc = kla::chunk_bwd_tc_workspace(B, T, H, have_S_chunks != 0);
+    return tc > simt ? tc : simt;
 }
 
 kla_status kla_chunk_bwd(const void* q, const void* k, const void* v, const float* eta,
@@ -232,8 +246,17 @@ kla_status kla_chunk_bwd(const void* q, const void* k, const void* v, const floa
         return fail(KLA_ERR_WORKSPACE, "kla_chunk_bwd needs %zu workspace bytes (got %zu)", need,
                     ws == nullptr ? (size_t)0 : ws_bytes);
     if (!aligned16(ws)) return fail(KLA_ERR_INVALID_ARG, "ws must be 16-byte aligned");
+    cudaError_t e;
+    if (tc_bwd_shape(T, Dk, Dv, dtype) && kla::get_encode_fn() != nullptr &&
+        ws_bytes >= kla::chunk_bwd_tc_workspace(B, T, H, S_chunks != nullptr)) {
+        kla::BwdTcArgs ta{q, k, v, eta, g, eps, S0, dO, dS_T, S_chunks, dq, dk, dv, deta, dg, dS0,
+                          B, T, H, out_dtype == KLA_BF16};
+        e = kla::launch_chunk_bwd_tc(ta, ws, ws_bytes, s);
+        if (e != cudaSuccess) return cuda_fail(e, "kla_chunk_bwd (tensor cores)");
+        return KLA_OK;
+    }
     char* w = static_cast<char*>(ws);
-    cudaError_t e = cudaMemsetAsync(w + off[1], 0, off[4] - off[1], s);
+    e = cudaMemsetAsync(w + off[1], 0, off[4] - off[1], s);
     if (e != cudaSuccess) return cuda_fail(e, "kla_chunk_bwd workspace clear");
     const float* Sc = S_chunks;
     if (Sc == nullptr) {
@@ -271,12 +294,13 @@ kla_status kla_decode_step(const void* q, const void* k, const void* v, const fl
 }
 
 kla_status kla_check_device_error(void* stream) {
-    unsigned int flag = 0, flag2 = 0, flag3 = 0;
+    unsigned int flag = 0, flag2 = 0, flag3 = 0, flag4 = 0;
     cudaError_t e = kla::tc_take_error(static_cast<cudaStream_t>(stream), &flag);
     if (e == cudaSuccess) e = kla::decode_take_error(static_cast<cudaStream_t>(stream), &flag2);
     if (e == cudaSuccess) e = kla::split_take_error(static_cast<cudaStream_t>(stream), &flag3);
+    if (e == cudaSuccess) e = kla::bwd_tc_take_error(static_cast<cudaStream_t>(stream), &flag4);
     if (e != cudaSuccess) return cuda_fail(e, "kla_check_device_error");
-    flag |= (flag2 << 8) | (flag3 << 16);
+    flag |= (flag2 << 8) | (flag3 << 16) | (flag4 << 24);
     if (flag) return fail(KLA_ERR_TIMEOUT, "a kernel gave up on a bounded wait (flag %u)", flag);
     return KLA_OK;
 }

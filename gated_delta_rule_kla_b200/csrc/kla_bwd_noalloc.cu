@@ -54,7 +54,7 @@ kla_status kla_chunk_bwd_noalloc(const void* q, const void* k, const void* v, co
                                  float* deta, float* dg, float* dS0, int B, int T, int H, int Dk, int Dv,
                                  int chunk, int dtype, int out_dtype, void* stream) {
     // Size check first, before touching the device: the scratch replaces the workspace.
-    const size_t need = kla_chunk_bwd_workspace(B, T, H, Dk, Dv, chunk, dtype, S_chunks != nullptr);
+    const size_t need = kla_chunk_bwd_workspace_min(B, T, H, Dk, Dv, chunk, dtype, S_chunks != nullptr);
     if (need > kNoallocScratchBytes) {
         // The regular entry point reports the same condition with its own message; run its
         // validation so argument errors keep their usual status, then report the size.

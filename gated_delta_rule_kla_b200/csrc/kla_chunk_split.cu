@@ -39,16 +39,7 @@ using namespace tcc;
 
 constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s
 
-// ---- per-chunk record in the workspace (byte offsets); tiles use the 128-byte swizzle
-constexpr uint32_t REC_W = 0;        // -W^T bf16: 128 dk rows x 64 tokens          16 KB
-constexpr uint32_t REC_KT = 16384;   // Ktil hi: [64 tokens x 64 dk] x 2 blocks        16 KB
-constexpr uint32_t REC_KTLO = 32768; // Ktil lo                                        16 KB
-constexpr uint32_t REC_P = 49152;    // P hi [64 x 64], then P lo                       16 KB
-constexpr uint32_t REC_UP = 65536;   // U' fp32 [64 tokens][128 dv]                      32 KB
-constexpr uint32_t REC_TILES = 98304;
-constexpr uint32_t REC_SC = REC_TILES;  // gamma[64], then gamma_last of the next chunk  512 B
-constexpr uint32_t REC_SCB = 512;
-constexpr size_t REC_BYTES = REC_TILES + REC_SCB;
+// The per-chunk record layout (REC_*) is defined in kla_tc_common.cuh.
 
 // =====================================================================================
 // Preparation kernel: one chunk per CTA, three CTAs per SM.  Shared memory holds only the
@@ -69,7 +60,7 @@ struct PrepMisc {
     uint32_t tmem_base, pad[3];
     float G[CH], gam[CH], del[CH], bco[CH], cco[CH], invr[CH], graw[CH], eta[CH], pk[CH];
     float wsc[CH];  // b gamma / r: column scale of T'
-    float gsum[2], grange;
+    float gsum[2], gprev[2], grange;
 };
 static_assert(sizeof(PrepMisc) <= 3072, "prep scalars");
 
@@ -94,7 +85,7 @@ __global__ void __launch_bounds__(PT, 3)
     const uint32_t bar_full = smem_u32(&ms->full), bar_mma = smem_u32(&ms->mma);
 
     // per-token gates first: their latency overlaps the barrier set-up and the tile loads
-    float g_own = 0.f, eta_own = 0.f, g_next = 0.f;
+    float g_own = 0.f, eta_own = 0.f, g_next = 0.f, g_prev = 0.f;
     if (tid < CH) {
         if (tid < n) {
             const size_t ti = tok_index(b, t0 + tid, h, T, H);
@@ -104,6 +95,8 @@ __global__ void __launch_bounds__(PT, 3)
     } else if (tid < 2 * CH) {
         const int j = tid - CH;
         if (c + 1 < NC && (c + 1) * CH + j < T) g_next = a.g[tok_index(b, (c + 1) * CH + j, h, T, H)];
+    } else if (tid < 3 * CH) {  // the previous chunk (always full) for the reverse pass
+        if (c > 0) g_prev = a.g[tok_index(b, (c - 1) * CH + tid - 2 * CH, h, T, H)];
     }
     if (tid == 0) {
         mbar_init(bar_full, 1);
@@ -127,6 +120,9 @@ __global__ void __launch_bounds__(PT, 3)
     } else if (tid < 2 * CH) {  // the next chunk's gamma_last
         const float sg = warp_sum(g_next);
         if ((tid & 31) == 0) ms->gsum[warp - 2] = sg;
+    } else if (tid < 3 * CH) {  // the previous chunk's gamma_last
+        const float sg = warp_sum(g_prev);
+        if ((tid & 31) == 0) ms->gprev[warp - 4] = sg;
     }
     tc_fence_before();
     __syncthreads();
@@ -204,6 +200,8 @@ __global__ void __launch_bounds__(PT, 3)
             ms->wsc[tid] = ms->bco[tid] * gm * ms->invr[tid];
         } else if (tid == CH) {
             reinterpret_cast<float*>(rec + REC_SC)[CH] = __expf(ms->gsum[0] + ms->gsum[1]);
+        } else if (tid == CH + 1) {
+            reinterpret_cast<float*>(rec + REC_SC)[CH + 1] = __expf(ms->gprev[0] + ms->gprev[1]);
         }
         ok = mbar_wait_bounded(bar_mma, 0, kWaitNs);
         if (__syncthreads_or(!ok)) {
@@ -275,6 +273,10 @@ __global__ void __launch_bounds__(PT, 3)
             }
         }
         __syncthreads();  // T is read; T'' overwrites it
+        if (a.T_chunks) {
+            uint8_t* tt = static_cast<uint8_t*>(a.T_chunks) + ((size_t)head * NC + c) * 16384;
+            st_chunks_split_global(tt, tt + 8192, i, 2 * qq, 2, tv);
+        }
         float v[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) v[e] = tv[e] * ms->wsc[16 * qq + e];
@@ -395,25 +397,6 @@ struct StateMisc {
     float gsum[2];
 };
 
-// Split fp32 values into bf16 hi + lo words, two consecutive K indices per 32-bit word (the
-// lower index in the low half): hi = rn(x), lo = rn(x - hi).
-template <int N>
-__device__ __forceinline__ void split_pack(const float* x, uint32_t* hp, uint32_t* lp) {
-#pragma unroll
-    for (int e = 0; e < N / 2; ++e) {
-        const uint32_t hw = pack_bf16x2(x[2 * e], x[2 * e + 1]);
-        hp[e] = hw;
-        lp[e] = pack_bf16x2(x[2 * e] - __uint_as_float(hw << 16), x[2 * e + 1] - __uint_as_float(hw & 0xffff0000u));
-    }
-}
-
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-// Raise the expected transaction bytes of the current phase without arriving.
-__device__ __forceinline__ void mbar_expect_tx_only(uint32_t bar, uint32_t bytes) {
-    asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
-}
 __device__ __forceinline__ void tma_store_4d(const void* tmap, uint32_t src, int c0, int c1, int c2, int c3) {
     asm volatile(
         "cp.async.bulk.tensor.4d.global.shared::cta.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(
@@ -421,14 +404,6 @@ __device__ __forceinline__ void tma_store_4d(const void* tmap, uint32_t src, int
         "r"(src), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
         : "memory");
 }
-// Epilogue warp: make this warp's TMEM stores visible to the MMA issuer, then arrive once.
-__device__ __forceinline__ void epi_signal(uint32_t bar, int tid) {
-    tmem_st_wait();
-    tc_fence_before();
-    __syncwarp();
-    if ((tid & 31) == 0) mbar_arrive(bar);
-}
-
 template <typename TOut>
 __global__ void __launch_bounds__(ST, 1)
     chunk_state_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_o, FwdArgs a,
@@ -690,11 +665,16 @@ __global__ void __launch_bounds__(ST, 1)
                 tmem_ld32(tmem + lane_base + TM_U + 32 * ch, x);
                 tmem_ld_wait();
                 const float* up = reinterpret_cast<const float*>(stg_p + SO_UP);
+                float* Uc = (a.U_chunks && !ident) ? a.U_chunks + ((size_t)head_idx * NCtot + c) * CH * DV : nullptr;
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
                     if (!ident) {
 #pragma unroll
                         for (int e = 16 * half; e < 16 * half + 16; ++e) x[e] += up[(32 * ch + e) * DV + row];
+                    }
+                    if (Uc) {
+#pragma unroll
+                        for (int e = 16 * half; e < 16 * half + 16; ++e) Uc[(32 * ch + e) * DV + row] = x[e];
                     }
                     uint32_t hp[8], lp[8];
                     split_pack<16>(x + 16 * half, hp, lp);
@@ -922,6 +902,7 @@ cudaError_t launch_chunk_fwd_split_state(const FwdArgs& a, void* ws, cudaStream_
     p1.o = nullptr;
     p1.S_T = MN;
     p1.S_chunks = nullptr;
+    p1.U_chunks = nullptr;
     p1.nseg = L.nseg;
     p1.seg_chunks = L.segc;
     p1.kinds = 2;

@@ -35,6 +35,12 @@ struct FwdArgs {
     // [B*H, nseg, Dk, Dv] (S_T: [kinds, B*H, nseg, Dk, Dv]) and a second grid row (kind 1)
     // runs each segment from the identity state with zero values (the segment's transition).
     int nseg, seg_chunks, kinds;
+    // Extra outputs of the split path for the tensor-core backward (both may be null):
+    // U_chunks [B*H, NC, 64, Dv] fp32, each chunk's U = T (Diag(c) V - Diag(b gamma) Khat S)
+    // (state pass); T_chunks [B*H, NC] x 16 KB, each chunk's T = (I + L)^{-1} as bf16 hi then lo
+    // [64 x 64] tiles, rows of T in the 128-byte swizzle (preparation kernel).
+    float* U_chunks;
+    void* T_chunks;
 };
 
 struct BwdArgs {
@@ -52,6 +58,26 @@ struct BwdArgs {
     bool bf16;      // q, k, v, dO are bf16 (else fp32)
     bool out_bf16;  // dq, dk, dv are bf16 (else fp32)
 };
+
+// Tensor-core backward (bf16 inputs, Dk == Dv == 128).
+struct BwdTcArgs {
+    const void *q, *k, *v;
+    const float *eta, *g;
+    float eps;
+    const float* S0;        // may be null (zero state)
+    const void* dO;         // bf16, [B,T,H,Dv]
+    const float* dS_T;      // may be null
+    const float* S_chunks;  // may be null (then recomputed into the workspace)
+    void *dq, *dk, *dv;
+    float *deta, *dg, *dS0;
+    int B, T, H;
+    bool out_bf16;
+};
+// Workspace bytes of the tensor-core backward: the split forward's records and, per chunk and
+// head, T (16 KB), U (32 KB), lambda (64 KB), dR (32 KB) and, without S_chunks, S (64 KB).
+size_t chunk_bwd_tc_workspace(int B, int T, int H, bool have_S_chunks);
+cudaError_t launch_chunk_bwd_tc(const BwdTcArgs& a, void* ws, size_t ws_bytes, cudaStream_t st);
+cudaError_t bwd_tc_take_error(cudaStream_t st, unsigned int* flag);
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st);
 cudaError_t launch_chunk_fwd_simt(const FwdArgs& a, cudaStream_t st);

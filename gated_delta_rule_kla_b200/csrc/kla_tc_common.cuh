@@ -274,5 +274,52 @@ __device__ __forceinline__ void st_chunks_split(uint8_t* hi_block, uint8_t* lo_b
     }
 }
 
+
+// ---- per-chunk record of the split forward's preparation kernel (byte offsets in the
+//      workspace); tiles use the 128-byte swizzle
+constexpr uint32_t REC_W = 0;        // -W^T bf16: 128 dk rows x 64 tokens          16 KB
+constexpr uint32_t REC_KT = 16384;   // Ktil hi: [64 tokens x 64 dk] x 2 blocks        16 KB
+constexpr uint32_t REC_KTLO = 32768; // Ktil lo                                        16 KB
+constexpr uint32_t REC_P = 49152;    // P hi [64 x 64], then P lo                       16 KB
+constexpr uint32_t REC_UP = 65536;   // U' fp32 [64 tokens][128 dv]                      32 KB
+constexpr uint32_t REC_TILES = 98304;
+constexpr uint32_t REC_SC = REC_TILES;  // gamma[64], gamma_last of the next chunk, of the previous chunk  512 B
+constexpr uint32_t REC_SCB = 512;
+constexpr size_t REC_BYTES = REC_TILES + REC_SCB;
+
+// Split fp32 values into bf16 hi + lo words, two consecutive K indices per 32-bit word (the
+// lower index in the low half): hi = rn(x), lo = rn(x - hi).
+template <int N>
+__device__ __forceinline__ void split_pack(const float* x, uint32_t* hp, uint32_t* lp) {
+#pragma unroll
+    for (int e = 0; e < N / 2; ++e) {
+        const uint32_t hw = pack_bf16x2(x[2 * e], x[2 * e + 1]);
+        hp[e] = hw;
+        lp[e] = pack_bf16x2(x[2 * e] - __uint_as_float(hw << 16), x[2 * e + 1] - __uint_as_float(hw & 0xffff0000u));
+    }
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+// Raise the expected transaction bytes of the current phase without arriving.
+__device__ __forceinline__ void mbar_expect_tx_only(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+// Pack fp32 pairs into bf16 words (hi part only), the lower K index in the low half.
+template <int N>
+__device__ __forceinline__ void pack_hi(const float* x, uint32_t* hp) {
+#pragma unroll
+    for (int e = 0; e < N / 2; ++e) hp[e] = pack_bf16x2(x[2 * e], x[2 * e + 1]);
+}
+
+// Epilogue warp: make this warp's TMEM stores visible to the MMA issuer, then arrive once.
+__device__ __forceinline__ void epi_signal(uint32_t bar, int tid) {
+    tmem_st_wait();
+    tc_fence_before();
+    __syncwarp();
+    if ((tid & 31) == 0) mbar_arrive(bar);
+}
+
 }  // namespace tcc
 }  // namespace kla

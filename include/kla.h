@@ -134,11 +134,20 @@ kla_status kla_chunk_fwd_state(const void *q, const float *g, const float *S0, v
  * same inputs, or NULL to recompute it inside the workspace.
  * Gradient of k at a key of exactly zero norm: the normalised-key form used on the GPU has
  * no finite limit there; dk is returned as zero for such tokens (all other gradients exact).
- * ws, ws_bytes: caller workspace of at least kla_chunk_bwd_workspace() bytes (required).
+ * ws, ws_bytes: caller workspace (device, 16-byte aligned, owned by the caller, contents need
+ * not be initialised) of at least kla_chunk_bwd_workspace_min() bytes (required; smaller is
+ * KLA_ERR_WORKSPACE).  With at least kla_chunk_bwd_workspace() bytes, bf16 inputs with
+ * Dk == Dv == 128 run on the tensor cores: the split forward's preparation and state pass are
+ * recomputed into ws (about 241 KiB per chunk and head, plus 64 KiB without S_chunks), a
+ * reverse state pass carries the state gradient chunk by chunk, and a chunk-parallel kernel
+ * forms every gradient.  With less, and for every other shape, the CUDA-core backward runs.
+ * The workspace must not be shared with a concurrent call.
  * Every output is fully overwritten.
  */
 size_t kla_chunk_bwd_workspace(int B, int T, int H, int Dk, int Dv, int chunk, int dtype,
                                int have_S_chunks);
+size_t kla_chunk_bwd_workspace_min(int B, int T, int H, int Dk, int Dv, int chunk, int dtype,
+                                   int have_S_chunks);
 kla_status kla_chunk_bwd(const void *q, const void *k, const void *v, const float *eta,
                          const float *g, float eps, const float *S0, const void *dO,
                          const float *dS_T, const float *S_chunks, void *dq, void *dk, void *dv,

@@ -380,6 +380,78 @@ def test_bwd_small(kla, oracle_mod, B, T, H, Dk, Dv, dtype, s0, with_dST):
         assert rel_err(gr[name], ref[name]) <= TOL[dtype], name
 
 
+BWD_TC_CASES = [
+    # B, T, H, s0, g_lo, with dS_T
+    (1, 64, 1, True, -0.5, True),
+    (2, 130, 3, True, -0.01, True),   # long memory: the state gradient crosses every chunk
+    (1, 333, 2, False, -0.5, False),
+    (1, 150, 2, True, -2.0, True),    # in-chunk decay down to ~e^-64
+    (1, 200, 2, True, -4.0, False),   # beyond e^-80 inside a chunk
+]
+
+
+@pytest.mark.parametrize("B,T,H,s0,g_lo,with_dST", BWD_TC_CASES)
+def test_bwd_tensor_core_and_cuda_core_paths_match_oracle(kla, oracle_mod, B, T, H, s0, g_lo, with_dST):
+    """bf16, d = 128: the tensor-core backward (default workspace) and the CUDA-core backward
+    (minimum workspace) both against the fp64 oracle."""
+    inp = small_inputs(B, T, H, 128, 128, "bf16", seed=T + 7 * H, s0=s0, g_lo=g_lo)
+    gen = torch.Generator().manual_seed(T + 1)
+    dO = torch.randn(B, T, H, 128, generator=gen).to(torch.bfloat16)
+    dST = torch.randn(B, H, 128, 128, generator=gen) if with_dST else None
+    d = {k: (v.cuda() if v is not None else None) for k, v in inp.items()}
+    args = (d["q"], d["k"], d["v"], d["eta"], d["g"], dO.cuda(), 1e-6, d["S0"],
+            dST.cuda() if dST is not None else None)
+    g_tc = kla.chunk_bwd(*args)
+    g_cc = kla.chunk_bwd(*args, cuda_cores=True)
+    torch.cuda.synchronize()
+    kla.check_device_error()
+    ref = oracle_mod.backward(*(np64(inp[k]) for k in ("q", "k", "v", "eta", "g")), 1e-6, np64(inp["S0"]),
+                              np64(dO), np64(dST))
+    for name in GRADS:
+        assert rel_err(g_tc[name], ref[name]) <= 2e-2, ("tensor cores", name)
+        assert rel_err(g_cc[name], ref[name]) <= 2e-2, ("cuda cores", name)
+
+
+def test_bwd_tensor_cores_zero_norm_key_and_zero_eta(kla, oracle_mod):
+    inp = small_inputs(1, 140, 2, 128, 128, "bf16", seed=41)
+    inp["k"][0, 5, 0] = 0
+    inp["k"][0, 70, 1] = 0
+    inp["eta"][0, 9, :] = 0
+    inp["eta"][0, 100, 0] = 0
+    dO = torch.randn(1, 140, 2, 128, generator=torch.Generator().manual_seed(5)).to(torch.bfloat16)
+    d = {k: v.cuda() for k, v in inp.items()}
+    gr = kla.chunk_bwd(d["q"], d["k"], d["v"], d["eta"], d["g"], dO.cuda(), 1e-6, d["S0"])
+    torch.cuda.synchronize()
+    ref = oracle_mod.backward(*(np64(inp[k]) for k in ("q", "k", "v", "eta", "g")), 1e-6, np64(inp["S0"]),
+                              np64(dO), None)
+    for name in GRADS:
+        if name == "dk":  # the unit-key form returns zero for the zero-norm keys (documented)
+            got = np64(gr[name]).copy()
+            want = np.array(ref[name], copy=True)
+            for (t, hh) in ((5, 0), (70, 1)):
+                assert np.all(got[0, t, hh] == 0)
+                want[0, t, hh] = 0
+            assert rel_err(got, want) <= 2e-2, name
+        else:
+            assert rel_err(gr[name], ref[name]) <= 2e-2, name
+
+
+def test_bwd_tensor_cores_more_heads_than_sms(kla, oracle_mod):
+    B, T, H = 10, 70, 16  # 160 reverse-pass CTAs: more than one wave
+    inp = small_inputs(B, T, H, 128, 128, "bf16", seed=77)
+    dO = torch.randn(B, T, H, 128, generator=torch.Generator().manual_seed(6)).to(torch.bfloat16)
+    d = {k: v.cuda() for k, v in inp.items()}
+    gr = kla.chunk_bwd(d["q"], d["k"], d["v"], d["eta"], d["g"], dO.cuda(), 1e-6, d["S0"])
+    torch.cuda.synchronize()
+    pairs = [(0, 0), (9, 15), (4, 7)]
+    args = [heads_slice(np64(inp[k]), pairs) for k in ("q", "k", "v", "eta", "g")]
+    ref = oracle_mod.backward(*args, 1e-6, heads_slice(np64(inp["S0"]), pairs, state=True),
+                              heads_slice(np64(dO), pairs), None)
+    for name in GRADS:
+        got = heads_slice(np64(gr[name]), pairs, state=(name == "dS0"))
+        assert rel_err(got, ref[name]) <= 2e-2, name
+
+
 def test_bwd_with_saved_chunk_states_matches_recompute(kla):
     inp = small_inputs(1, 190, 2, 128, 128, "bf16", seed=8)
     d = {k: v.cuda() for k, v in inp.items()}
