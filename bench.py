@@ -395,14 +395,15 @@ def bench_train(kla, WORKLOADS, make_inputs, dev, stream, flush, rank, world, hb
     inp = make_inputs(w)
     d = {k: (v.to(dev) if v is not None else None) for k, v in inp.items()}
     dO = d["dO"].to(d["q"].dtype)
-    ws = torch.empty(kla.lib().kla_chunk_bwd_workspace(w.B, w.T, w.H, w.Dk, w.Dv, 64, 1, 1),
-                     dtype=torch.uint8, device=dev)
-    fws = kla.fwd_workspace(d["k"], d["v"])
+    # one workspace shared by the training forward and the backward (kla_chunk_fwd_train,
+    # kla_chunk_bwd_after_train): the backward reuses the forward's records and tiles
+    ws = kla.train_workspace(d["k"], d["v"])
+    o = torch.empty(w.B, w.T, w.H, w.Dv, device=dev, dtype=torch.float32)
+    ST = torch.empty(w.B, w.H, w.Dk, w.Dv, device=dev, dtype=torch.float32)
 
     def step():
-        _, _, Sc = kla.chunk_fwd(d["q"], d["k"], d["v"], d["eta"], d["g"], w.eps, d["S0"],
-                                 save_chunk_states=True, workspace=fws)
-        kla.chunk_bwd(d["q"], d["k"], d["v"], d["eta"], d["g"], dO, w.eps, d["S0"], None, Sc, workspace=ws)
+        kla.chunk_fwd_train(d["q"], d["k"], d["v"], d["eta"], d["g"], w.eps, d["S0"], workspace=ws, o=o, S_T=ST)
+        kla.chunk_bwd_after_train(d["q"], d["k"], d["v"], d["eta"], d["g"], dO, ws, w.eps)
 
     nsteps = 2 if args.quick else 5
     step()
@@ -418,7 +419,8 @@ def bench_train(kla, WORKLOADS, make_inputs, dev, stream, flush, rank, world, hb
     alg = fwd_bytes(w.B, w.T, w.H, w.Dk, w.Dv, elt, False) + bwd_bytes(w.B, w.T, w.H, w.Dk, w.Dv, elt)
     return {"workload": w.name, "value": tokens / (total_ms / 1e3), "unit": "tokens/s",
             "steps": nsteps, "ms_per_step": total_ms / nsteps,
-            "gpu_launches_per_step": 5,  # forward: preparation + state pass; backward: 3 kernels
+            # forward: preparation + state pass; backward: reverse state pass + gradient kernel
+            "gpu_launches_per_step": 4,
             "roofline": {"bound": "tensor", "achieved": flops / mean_s / 1e12, "peak": tc_peak,
                          "unit": "TFLOP/s", "frac": flops / mean_s / 1e12 / tc_peak,
                          "hbm_frac": alg / mean_s / 1e9 / hbm_peak, "alg_flops_per_step": flops,

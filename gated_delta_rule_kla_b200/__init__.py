@@ -18,7 +18,8 @@ import os
 
 import torch
 
-__all__ = ["lib", "chunk_fwd", "chunk_bwd", "decode_step", "check_device_error", "KLAError", "CHUNK",
+__all__ = ["lib", "chunk_fwd", "chunk_bwd", "chunk_fwd_train", "chunk_bwd_after_train", "train_workspace",
+           "decode_step", "check_device_error", "KLAError", "CHUNK",
            "library_path"]
 
 CHUNK = 64
@@ -63,6 +64,11 @@ def lib():
         L.kla_chunk_bwd_workspace.restype = sz
         L.kla_chunk_bwd_workspace_min.argtypes = [i, i, i, i, i, i, i, i]
         L.kla_chunk_bwd_workspace_min.restype = sz
+        L.kla_chunk_fwd_train.argtypes = [vp, vp, vp, fp, fp, f, fp, vp, fp, i, i, i, i, i, i, i, i, vp, sz, vp]
+        L.kla_chunk_fwd_train.restype = i
+        L.kla_chunk_bwd_after_train.argtypes = [vp, vp, vp, fp, fp, f, vp, fp, vp, vp, vp, fp, fp, fp,
+                                                i, i, i, i, i, i, i, i, vp, sz, vp]
+        L.kla_chunk_bwd_after_train.restype = i
         L.kla_chunk_bwd.argtypes = [vp, vp, vp, fp, fp, f, fp, vp, fp, fp, vp, vp, vp, fp, fp, fp,
                                     i, i, i, i, i, i, i, i, vp, sz, vp]
         L.kla_chunk_bwd.restype = i
@@ -241,6 +247,61 @@ def chunk_bwd(q, k, v, eta, g, dO, eps=1e-6, S0=None, dS_T=None, S_chunks=None, 
                          _dtype_code(k), _dtype_code(out_dtype), _ptr(workspace), workspace.numel(),
                          _stream(dev, stream))
     _check(st, "kla_chunk_bwd")
+    return out
+
+
+def train_workspace(k, v):
+    """A workspace for chunk_fwd_train / chunk_bwd_after_train on these shapes (reusable)."""
+    B, T, H, Dk = k.shape
+    n = lib().kla_chunk_bwd_workspace(B, T, H, Dk, v.shape[-1], CHUNK, _dtype_code(k), 0)
+    return torch.empty(max(n, 16), device=k.device, dtype=torch.uint8)
+
+
+def chunk_fwd_train(q, k, v, eta, g, eps=1e-6, S0=None, *, workspace=None, o=None, S_T=None,
+                    out_dtype=torch.float32, stream=None):
+    """Training forward: (o, S_T, workspace), the workspace holding what chunk_bwd_after_train
+    needs for these inputs (kla_chunk_fwd_train)."""
+    dev = k.device
+    B, T, H, Dk = k.shape
+    Dv = v.shape[-1]
+    dt = k.dtype
+    _need(q, "q", dev, dt, (B, T, H, Dk)); _need(k, "k", dev, dt); _need(v, "v", dev, dt, (B, T, H, Dv))
+    _need(eta, "eta", dev, torch.float32, (B, T, H)); _need(g, "g", dev, torch.float32, (B, T, H))
+    _need(S0, "S0", dev, torch.float32, (B, H, Dk, Dv))
+    if o is None:
+        o = torch.empty(B, T, H, Dv, device=dev, dtype=out_dtype)
+    if S_T is None:
+        S_T = torch.empty(B, H, Dk, Dv, device=dev, dtype=torch.float32)
+    _need(o, "o", dev, None, (B, T, H, Dv)); _need(S_T, "S_T", dev, torch.float32, (B, H, Dk, Dv))
+    if workspace is None:
+        workspace = train_workspace(k, v)
+    st = lib().kla_chunk_fwd_train(_ptr(q), _ptr(k), _ptr(v), _ptr(eta), _ptr(g), float(eps), _ptr(S0), _ptr(o),
+                                   _ptr(S_T), B, T, H, Dk, Dv, CHUNK, _dtype_code(k), _dtype_code(o),
+                                   _ptr(workspace), workspace.numel(), _stream(dev, stream))
+    _check(st, "kla_chunk_fwd_train")
+    return o, S_T, workspace
+
+
+def chunk_bwd_after_train(q, k, v, eta, g, dO, workspace, eps=1e-6, dS_T=None, *, out_dtype=torch.float32,
+                          stream=None):
+    """Backward after chunk_fwd_train on the same inputs and workspace (kla_chunk_bwd_after_train).
+    Returns dict(dq, dk, dv, deta, dg, dS0)."""
+    dev = k.device
+    B, T, H, Dk = k.shape
+    Dv = v.shape[-1]
+    dt = k.dtype
+    _need(dO, "dO", dev, dt, (B, T, H, Dv)); _need(dS_T, "dS_T", dev, torch.float32, (B, H, Dk, Dv))
+    out = dict(dq=torch.empty(q.shape, device=dev, dtype=out_dtype),
+               dk=torch.empty(k.shape, device=dev, dtype=out_dtype),
+               dv=torch.empty(v.shape, device=dev, dtype=out_dtype),
+               deta=torch.empty_like(eta), dg=torch.empty_like(g),
+               dS0=torch.empty(B, H, Dk, Dv, device=dev, dtype=torch.float32))
+    st = lib().kla_chunk_bwd_after_train(_ptr(q), _ptr(k), _ptr(v), _ptr(eta), _ptr(g), float(eps), _ptr(dO),
+                                         _ptr(dS_T), _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]),
+                                         _ptr(out["deta"]), _ptr(out["dg"]), _ptr(out["dS0"]), B, T, H, Dk, Dv,
+                                         CHUNK, _dtype_code(k), _dtype_code(out_dtype), _ptr(workspace),
+                                         workspace.numel(), _stream(dev, stream))
+    _check(st, "kla_chunk_bwd_after_train")
     return out
 
 

@@ -68,6 +68,13 @@ bool tc_bwd_shape(int T, int Dk, int Dv, int dtype) {
     return dtype == KLA_BF16 && Dk == 128 && Dv == 128 && T >= 1;
 }
 
+// The backward (and the training forward) run on the tensor cores for their shapes when the
+// workspace holds the tensor-core layout; the decision depends only on the arguments.
+bool tc_bwd_path(int B, int T, int H, int Dk, int Dv, int dtype, size_t ws_bytes) {
+    return tc_bwd_shape(T, Dk, Dv, dtype) && kla::get_encode_fn() != nullptr &&
+           ws_bytes >= kla::chunk_bwd_tc_workspace(B, T, H, false);
+}
+
 size_t bwd_ws_layout(int B, int T, int H, int Dk, int Dv, bool have_S_chunks, size_t* off) {
     const size_t NC = (size_t)(T + kla::kChunkLen - 1) / kla::kChunkLen;
     const size_t ntok = (size_t)B * T * H;
@@ -220,15 +227,22 @@ size_t kla_chunk_bwd_workspace(int B, int T, int H, int Dk, int Dv, int chunk, i
     return tc > simt ? tc : simt;
 }
 
-kla_status kla_chunk_bwd(const void* q, const void* k, const void* v, const float* eta,
-                         const float* g, float eps, const float* S0, const void* dO,
-                         const float* dS_T, const float* S_chunks, void* dq, void* dk, void* dv,
-                         float* deta, float* dg, float* dS0, int B, int T, int H, int Dk, int Dv,
-                         int chunk, int dtype, int out_dtype, void* ws, size_t ws_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// Backward of every entry point.  after_train: ws holds what kla_chunk_fwd_train left there for
+// these inputs (the forward is not recomputed, S_chunks is ignored).
+kla_status bwd_impl(const void* q, const void* k, const void* v, const float* eta, const float* g,
+                    float eps, const float* S0, const void* dO, const float* dS_T, const float* S_chunks,
+                    void* dq, void* dk, void* dv, float* deta, float* dg, float* dS0, int B, int T, int H,
+                    int Dk, int Dv, int chunk, int dtype, int out_dtype, void* ws, size_t ws_bytes,
+                    void* stream, bool after_train, const char* name) {
     kla_status st = check_common(B, T, H, Dk, Dv, chunk, dtype, out_dtype, eps);
     if (st != KLA_OK) return st;
     REQUIRE_PTR(dS0);
     OPTIONAL_PTR(S0); OPTIONAL_PTR(dS_T); OPTIONAL_PTR(S_chunks);
+    if (after_train) S_chunks = nullptr;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const size_t sbytes = (size_t)B * H * Dk * Dv * sizeof(float);
     if (T == 0) {
@@ -243,16 +257,16 @@ kla_status kla_chunk_bwd(const void* q, const void* k, const void* v, const floa
     size_t off[5];
     const size_t need = bwd_ws_layout(B, T, H, Dk, Dv, S_chunks != nullptr, off);
     if (ws == nullptr || ws_bytes < need)
-        return fail(KLA_ERR_WORKSPACE, "kla_chunk_bwd needs %zu workspace bytes (got %zu)", need,
+        return fail(KLA_ERR_WORKSPACE, "%s needs %zu workspace bytes (got %zu)", name, need,
                     ws == nullptr ? (size_t)0 : ws_bytes);
     if (!aligned16(ws)) return fail(KLA_ERR_INVALID_ARG, "ws must be 16-byte aligned");
     cudaError_t e;
-    if (tc_bwd_shape(T, Dk, Dv, dtype) && kla::get_encode_fn() != nullptr &&
-        ws_bytes >= kla::chunk_bwd_tc_workspace(B, T, H, S_chunks != nullptr)) {
+    if (tc_bwd_path(B, T, H, Dk, Dv, dtype, ws_bytes)) {
         kla::BwdTcArgs ta{q, k, v, eta, g, eps, S0, dO, dS_T, S_chunks, dq, dk, dv, deta, dg, dS0,
                           B, T, H, out_dtype == KLA_BF16};
-        e = kla::launch_chunk_bwd_tc(ta, ws, ws_bytes, s);
-        if (e != cudaSuccess) return cuda_fail(e, "kla_chunk_bwd (tensor cores)");
+        e = after_train ? kla::launch_chunk_bwd_tc_reverse(ta, ws, ws_bytes, s)
+                        : kla::launch_chunk_bwd_tc(ta, ws, ws_bytes, s);
+        if (e != cudaSuccess) return cuda_fail(e, name);
         return KLA_OK;
     }
     char* w = static_cast<char*>(ws);
@@ -261,10 +275,12 @@ kla_status kla_chunk_bwd(const void* q, const void* k, const void* v, const floa
     const float* Sc = S_chunks;
     if (Sc == nullptr) {
         float* Sc_ws = reinterpret_cast<float*>(w + off[0]);
-        kla::FwdArgs fa{q, k, v, eta, g, eps, S0, nullptr, nullptr, Sc_ws, B, T, H, Dk, Dv,
-                        dtype == KLA_BF16, false};
-        e = kla::chunk_fwd_tc_supported(fa) ? kla::launch_chunk_fwd_tc(fa, s) : kla::launch_chunk_fwd_simt(fa, s);
-        if (e != cudaSuccess) return cuda_fail(e, "kla_chunk_bwd state recompute");
+        if (!after_train) {
+            kla::FwdArgs fa{q, k, v, eta, g, eps, S0, nullptr, nullptr, Sc_ws, B, T, H, Dk, Dv,
+                            dtype == KLA_BF16, false};
+            e = kla::chunk_fwd_tc_supported(fa) ? kla::launch_chunk_fwd_tc(fa, s) : kla::launch_chunk_fwd_simt(fa, s);
+            if (e != cudaSuccess) return cuda_fail(e, "kla_chunk_bwd state recompute");
+        }
         Sc = Sc_ws;
     }
     const size_t ntok = (size_t)B * T * H;
@@ -274,8 +290,64 @@ kla_status kla_chunk_bwd(const void* q, const void* k, const void* v, const floa
                    acc3, acc3 + ntok, acc3 + 2 * ntok, B, T, H, Dk, Dv, dtype == KLA_BF16,
                    out_dtype == KLA_BF16};
     e = kla::launch_chunk_bwd_simt(a, s);
-    if (e != cudaSuccess) return cuda_fail(e, "kla_chunk_bwd launch");
+    if (e != cudaSuccess) return cuda_fail(e, name);
     return KLA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+kla_status kla_chunk_bwd(const void* q, const void* k, const void* v, const float* eta,
+                         const float* g, float eps, const float* S0, const void* dO,
+                         const float* dS_T, const float* S_chunks, void* dq, void* dk, void* dv,
+                         float* deta, float* dg, float* dS0, int B, int T, int H, int Dk, int Dv,
+                         int chunk, int dtype, int out_dtype, void* ws, size_t ws_bytes, void* stream) {
+    return bwd_impl(q, k, v, eta, g, eps, S0, dO, dS_T, S_chunks, dq, dk, dv, deta, dg, dS0, B, T, H, Dk, Dv,
+                    chunk, dtype, out_dtype, ws, ws_bytes, stream, false, "kla_chunk_bwd");
+}
+
+kla_status kla_chunk_fwd_train(const void* q, const void* k, const void* v, const float* eta,
+                               const float* g, float eps, const float* S0, void* o, float* S_T, int B,
+                               int T, int H, int Dk, int Dv, int chunk, int dtype, int out_dtype, void* ws,
+                               size_t ws_bytes, void* stream) {
+    kla_status st = check_common(B, T, H, Dk, Dv, chunk, dtype, out_dtype, eps);
+    if (st != KLA_OK) return st;
+    if (T > 0) {
+        REQUIRE_PTR(q); REQUIRE_PTR(k); REQUIRE_PTR(v); REQUIRE_PTR(eta); REQUIRE_PTR(g);
+    }
+    OPTIONAL_PTR(S0); OPTIONAL_PTR(o); OPTIONAL_PTR(S_T);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (T == 0)  // nothing for the backward to keep: the plain forward's empty-sequence case
+        return kla_chunk_fwd(q, k, v, eta, g, eps, S0, o, S_T, nullptr, B, T, H, Dk, Dv, chunk, dtype,
+                             out_dtype, nullptr, 0, stream);
+    size_t off[5];
+    const size_t need = bwd_ws_layout(B, T, H, Dk, Dv, false, off);
+    if (ws == nullptr || ws_bytes < need)
+        return fail(KLA_ERR_WORKSPACE, "kla_chunk_fwd_train needs %zu workspace bytes (got %zu)", need,
+                    ws == nullptr ? (size_t)0 : ws_bytes);
+    if (!aligned16(ws)) return fail(KLA_ERR_INVALID_ARG, "ws must be 16-byte aligned");
+    kla::FwdArgs a{q, k, v, eta, g, eps, S0, o, S_T, nullptr, B, T, H, Dk, Dv, dtype == KLA_BF16,
+                   out_dtype == KLA_BF16};
+    cudaError_t e;
+    if (tc_bwd_path(B, T, H, Dk, Dv, dtype, ws_bytes)) {
+        e = kla::launch_chunk_fwd_train_tc(a, ws, ws_bytes, s);
+    } else {
+        // the CUDA-core backward's layout: the chunk states at the start of ws
+        a.S_chunks = reinterpret_cast<float*>(static_cast<char*>(ws) + off[0]);
+        e = kla::chunk_fwd_tc_supported(a) ? kla::launch_chunk_fwd_tc(a, s) : kla::launch_chunk_fwd_simt(a, s);
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "kla_chunk_fwd_train launch");
+    return KLA_OK;
+}
+
+kla_status kla_chunk_bwd_after_train(const void* q, const void* k, const void* v, const float* eta,
+                                     const float* g, float eps, const void* dO, const float* dS_T, void* dq,
+                                     void* dk, void* dv, float* deta, float* dg, float* dS0, int B, int T,
+                                     int H, int Dk, int Dv, int chunk, int dtype, int out_dtype, void* ws,
+                                     size_t ws_bytes, void* stream) {
+    return bwd_impl(q, k, v, eta, g, eps, nullptr, dO, dS_T, nullptr, dq, dk, dv, deta, dg, dS0, B, T, H, Dk,
+                    Dv, chunk, dtype, out_dtype, ws, ws_bytes, stream, true, "kla_chunk_bwd_after_train");
 }
 
 kla_status kla_decode_step(const void* q, const void* k, const void* v, const float* eta,

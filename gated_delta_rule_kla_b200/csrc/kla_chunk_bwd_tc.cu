@@ -73,6 +73,32 @@ __device__ __forceinline__ void st_row32<__nv_bfloat16>(__nv_bfloat16* dst, cons
     }
 }
 
+// Split 8 fp32 values into bf16 hi/lo and store them as 16-byte piece `cc` of row r of two
+// 128-byte-swizzled tiles.
+__device__ __forceinline__ void st_piece_split(uint8_t* hi_blk, uint8_t* lo_blk, int r, int cc, const float* x) {
+    uint4 hh, ll;
+    split_chunk8(x, hh, ll);
+    const uint32_t off = r * 128 + ((cc ^ (r & 7)) << 4);
+    *reinterpret_cast<uint4*>(hi_blk + off) = hh;
+    *reinterpret_cast<uint4*>(lo_blk + off) = ll;
+}
+template <typename TOut>
+__device__ __forceinline__ void st_piece8(TOut* dst, const float* x);
+template <>
+__device__ __forceinline__ void st_piece8<float>(float* dst, const float* x) {
+    reinterpret_cast<float4*>(dst)[0] = make_float4(x[0], x[1], x[2], x[3]);
+    reinterpret_cast<float4*>(dst)[1] = make_float4(x[4], x[5], x[6], x[7]);
+}
+template <>
+__device__ __forceinline__ void st_piece8<__nv_bfloat16>(__nv_bfloat16* dst, const float* x) {
+    uint4 w;
+    w.x = pack_bf16x2(x[0], x[1]);
+    w.y = pack_bf16x2(x[2], x[3]);
+    w.z = pack_bf16x2(x[4], x[5]);
+    w.w = pack_bf16x2(x[6], x[7]);
+    *reinterpret_cast<uint4*>(dst) = w;
+}
+
 // Device-side view of one backward call: inputs, outputs and the workspace arrays.
 struct BwdDev {
     const void *q, *k, *v;
@@ -80,11 +106,12 @@ struct BwdDev {
     float eps;
     const float* dS_T;
     const uint8_t* recs;   // forward preparation records [BH, NC]
-    const uint8_t* Tch;    // T hi/lo tiles [BH, NC] x 16 KB
-    const float* Sch;      // [BH, NC, DK, DV]
-    const float* Uch;      // [BH, NC, CH, DV]
-    float* Lam;            // [BH, NC, DK, DV]  gradient of each chunk's outgoing state
-    float* dR;             // [BH, NC, CH, DV]
+    // per chunk and head, bf16 hi then lo tile images in the 128-byte swizzle:
+    const uint8_t* Ttl;    // T: [64 rows of T][64]                                     16 KB
+    const uint8_t* Stl;    // incoming state S: [dk half][128 dv rows][64 dk]           64 KB
+    const uint8_t* Utl;    // U: [128 dv rows][64 tokens]                               32 KB
+    uint8_t* Ltl;          // lambda = dS' (gradient of the outgoing state), as S       64 KB
+    float* dR;             // [BH, NC, CH, DV] fp32
     void *dq, *dk, *dv;
     float *deta, *dg, *dS0;
     int B, T, H;
@@ -99,7 +126,8 @@ struct BwdDev {
 //   dR^T     = dU^T T
 // TMEM: [0,128) lambda^T master fp32, [128,192) lambda^T hi, [192,256) dU^T accumulator,
 // [256,288) dU^T hi, [288,320) dU^T lo, [320,352) (gamma dO)^T hi, [352,384) lo,
-// [384,448) dR^T accumulator, [448,512) lambda^T lo.
+// [384,448) dR^T accumulator, [448,512) lambda^T lo.  Every chunk's lambda leaves as bf16 hi/lo
+// tiles (thread = one dv row of 64 dk: 32-byte stores), the layout the gradient kernel reads.
 // =====================================================================================
 constexpr int RT = 320;
 constexpr int kRIssuer = 8, kRLoader = 9;
@@ -145,7 +173,7 @@ __global__ void __launch_bounds__(RT, 1)
     const uint32_t l_ready0 = smem_u32(&ms->l_ready[0]), u_ready0 = smem_u32(&ms->u_ready[0]),
                    gd_ready = smem_u32(&ms->gd_ready);
     const float* dST = a.dS_T ? a.dS_T + (size_t)head * DK * DV : nullptr;
-    float* Lam = a.Lam + (size_t)head * NC * DK * DV;
+    uint8_t* Ltl = a.Ltl + (size_t)head * NC * 65536;
     float* dRh = a.dR + (size_t)head * NC * CH * DV;
 
     if (tid == 0) {
@@ -193,7 +221,7 @@ __global__ void __launch_bounds__(RT, 1)
                 const uint8_t* rec = a.recs + ((size_t)head * NC + c) * REC_BYTES;
                 mbar_expect_tx(bar, kBytes);
                 bulk_load(base + SR_W, rec + REC_W, 65536, bar);
-                bulk_load(base + SR_T, a.Tch + ((size_t)head * NC + c) * 16384, 16384, bar);
+                bulk_load(base + SR_T, a.Ttl + ((size_t)head * NC + c) * 16384, 16384, bar);
                 bulk_load(sbase + R_SC + st * REC_SCB, rec + REC_SC, REC_SCB, bar);
                 tma_load_4d(base + SR_DO, &tm_do, bar, 0, h, c * CH, b);
                 tma_load_4d(base + SR_DO + 8192, &tm_do, bar, 64, h, c * CH, b);
@@ -312,8 +340,6 @@ __global__ void __launch_bounds__(RT, 1)
                 float x[32];
 #pragma unroll
                 for (int e = 0; e < 32; ++e) x[e] = dST ? dST[(size_t)(dk0 + e) * DV + row] : 0.f;
-#pragma unroll
-                for (int e = 0; e < 32; ++e) Lam[((size_t)(NC - 1) * DK + dk0 + e) * DV + row] = x[e];
                 uint32_t hp[16], lp[16];
                 split_pack<32>(x, hp, lp);
                 tmem_st16u(tmem + lane_base + TR_LH + 32 * ch + 16 * q2, hp);
@@ -324,29 +350,34 @@ __global__ void __launch_bounds__(RT, 1)
                 epi_signal(l_ready0 + 8 * q2, tid);
             }
         }
-        for (int lc = 0; lc < NC; ++lc) {
-            const int c = NC - 1 - lc, st = lc & 1;
-            const bool has_next = c > 0;
-            float gprev;
-            // ---- (gamma dO)^T hi/lo: thread = dv, tokens 32 ch .. + 32
-            {
-                const bool ok = mbar_wait_bounded(full0 + 8 * st, (lc >> 1) & 1, kWaitNs);
-                if (__any_sync(0xffffffffu, !ok)) { aborted = true; break; }
-                const float* sc = reinterpret_cast<const float*>(sm + R_SC + st * REC_SCB);
-                gprev = sc[CH + 1];  // gamma_last of chunk c - 1: the master's next pre-scale
-                const uint8_t* dob = sm + st * R_STAGE + SR_DO + (row >> 6) * 8192;
-                float x[32];
+        // (gamma dO)^T hi/lo for the chunk of processing index lc2 (thread = dv, tokens 32 ch ..
+        // + 32), and that chunk's gamma_last of chunk c - 1 for the master's next pre-scale; the
+        // signal also orders the master rescale before the Q product
+        float gprev = 1.f;
+        auto gamma_do = [&](int lc2) -> bool {
+            const int st2 = lc2 & 1;
+            const bool ok = mbar_wait_bounded(full0 + 8 * st2, (lc2 >> 1) & 1, kWaitNs);
+            if (__any_sync(0xffffffffu, !ok)) return false;
+            const float* sc = reinterpret_cast<const float*>(sm + R_SC + st2 * REC_SCB);
+            gprev = sc[CH + 1];
+            const uint8_t* dob = sm + st2 * R_STAGE + SR_DO + (row >> 6) * 8192;
+            float x[32];
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const int t = 32 * ch + e;
-                    x[e] = sc[t] * ld_sw128_bf16(dob, t, row & 63);
-                }
-                uint32_t hp[16], lp[16];
-                split_pack<32>(x, hp, lp);
-                tmem_st16u(tmem + lane_base + TR_GH + 16 * ch, hp);
-                tmem_st16u(tmem + lane_base + TR_GL + 16 * ch, lp);
-                epi_signal(gd_ready, tid);  // also orders the master rescale before the Q product
+            for (int e = 0; e < 32; ++e) {
+                const int t = 32 * ch + e;
+                x[e] = sc[t] * ld_sw128_bf16(dob, t, row & 63);
             }
+            uint32_t hp[16], lp[16];
+            split_pack<32>(x, hp, lp);
+            tmem_st16u(tmem + lane_base + TR_GH + 16 * ch, hp);
+            tmem_st16u(tmem + lane_base + TR_GL + 16 * ch, lp);
+            epi_signal(gd_ready, tid);
+            return true;
+        };
+        if (!gamma_do(0)) aborted = true;
+        for (int lc = 0; lc < NC && !aborted; ++lc) {
+            const int c = NC - 1 - lc;
+            const bool has_next = c > 0;
             // ---- dU epilogue: hi/lo A operands, released in two halves of 16 tokens
             {
                 const bool ok = mbar_wait_bounded(bar_u, lc & 1, kWaitNs);
@@ -363,9 +394,12 @@ __global__ void __launch_bounds__(RT, 1)
                     tmem_st8u(tmem + lane_base + TR_UL + 16 * ch + 8 * half, lp);
                     epi_signal(u_ready0 + 8 * half, tid);
                 }
+                // lambda_c (still the dU product's operand) to its tiles while the W product runs
+                st_tmem_row_global(tmem + lane_base + TR_LH + 32 * ch, tmem + lane_base + TR_LL + 32 * ch,
+                                   Ltl + (size_t)c * 65536 + ch * 16384, 32768, row);
             }
-            // ---- lambda epilogue: hi/lo of the next chunk's lambda in two halves, the chunk's
-            //      lambda to the workspace, then the master pre-scaled by gamma_last of chunk c - 1
+            // ---- lambda epilogue: hi/lo of the next chunk's lambda in two halves, the master
+            //      pre-scaled by gamma_last of chunk c - 1, the next chunk's gamma dO
             {
                 const bool ok = mbar_wait_bounded(bar_s, lc & 1, kWaitNs);
                 if (__any_sync(0xffffffffu, !ok)) { aborted = true; break; }
@@ -375,28 +409,28 @@ __global__ void __launch_bounds__(RT, 1)
                     tmem_ld32(tmem + lane_base + TR_L + 64 * ch, x0);
                     tmem_ld32(tmem + lane_base + TR_L + 64 * ch + 32, x1);
                     tmem_ld_wait();
-                    uint32_t hp[16], lp[16];
-                    split_pack<32>(x0, hp, lp);
-                    tmem_st16u(tmem + lane_base + TR_LH + 32 * ch, hp);
-                    tmem_st16u(tmem + lane_base + TR_LL + 32 * ch, lp);
-                    epi_signal(l_ready0, tid);
-                    split_pack<32>(x1, hp, lp);
-                    tmem_st16u(tmem + lane_base + TR_LH + 32 * ch + 16, hp);
-                    tmem_st16u(tmem + lane_base + TR_LL + 32 * ch + 16, lp);
-                    epi_signal(l_ready0 + 8, tid);
-                    float* Ln = Lam + (size_t)(c - 1) * DK * DV;
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        Ln[(size_t)(64 * ch + e) * DV + row] = x0[e];
-                        Ln[(size_t)(64 * ch + 32 + e) * DV + row] = x1[e];
+                    {
+                        uint32_t hp[16], lp[16];
+                        split_pack<32>(x0, hp, lp);
+                        tmem_st16u(tmem + lane_base + TR_LH + 32 * ch, hp);
+                        tmem_st16u(tmem + lane_base + TR_LL + 32 * ch, lp);
+                        epi_signal(l_ready0, tid);
+                        split_pack<32>(x1, hp, lp);
+                        tmem_st16u(tmem + lane_base + TR_LH + 32 * ch + 16, hp);
+                        tmem_st16u(tmem + lane_base + TR_LL + 32 * ch + 16, lp);
+                        epi_signal(l_ready0 + 8, tid);
                     }
+                    {
+                        float y[32];
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        x0[e] *= gprev;
-                        x1[e] *= gprev;
+                        for (int e = 0; e < 32; ++e) y[e] = x0[e] * gprev;
+                        tmem_st32(tmem + lane_base + TR_L + 64 * ch, y);
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) y[e] = x1[e] * gprev;
+                        tmem_st32(tmem + lane_base + TR_L + 64 * ch + 32, y);
                     }
-                    tmem_st32(tmem + lane_base + TR_L + 64 * ch, x0);
-                    tmem_st32(tmem + lane_base + TR_L + 64 * ch + 32, x1);
+                    if (!gamma_do(lc + 1)) { aborted = true; break; }
+
                 }
             }
             // ---- dR epilogue: dR as [token][dv] rows to the workspace
@@ -465,10 +499,12 @@ constexpr uint32_t G_QK = 0, G_DOR = 32768, G_DRL = 65536, G_UH = 81920, G_UL = 
 constexpr uint32_t TG_G = 0, TG_YA = 64, TG_YB = 128, TG_Z = 192, TG_L = 320, TG_X = 0;
 
 struct GradMisc {
-    uint64_t full, bar1, bar2, bar3;
+    uint64_t full, bar1, bar2, bar3, bar_lam;
     uint32_t tmem_base, factored;
     float G[CH], gam[CH], del[CH], ginv[CH], bco[CH], cco[CH], invr[CH], eta[CH], r2[CH], graw[CH];
-    float rowsum[CH], colsum[CH], rowB[CH], s_oq[CH], s_rx[CH], s_uk[CH], kd[CH], dc[CH], dr[CH], dGs[CH];
+    // decay-gradient row / column sums: one slot per contributing warp, added in a fixed order
+    float rs_part[4][CH], cs_part[4][CH];
+    float rowB[CH], s_oq[CH], s_rx[CH], s_uk[CH], kd[CH], dc[CH], dr[CH], dGs[CH];
     float red[8];
     float lamS;
 };
@@ -494,7 +530,7 @@ __global__ void __launch_bounds__(GT, 1)
     const size_t crow = (size_t)head * NC + c;  // chunk index in the workspace arrays
     const uint32_t sbase = smem_u32(sm);
     const uint32_t bar_full = smem_u32(&ms->full), bar1 = smem_u32(&ms->bar1), bar2 = smem_u32(&ms->bar2),
-                   bar3 = smem_u32(&ms->bar3);
+                   bar3 = smem_u32(&ms->bar3), bar_lam = smem_u32(&ms->bar_lam);
     // epilogue roles: TMEM lane quadrant and column half
     const int q4 = warp & 3, chh = warp >> 2;
     const bool top = q4 < 2;
@@ -503,128 +539,119 @@ __global__ void __launch_bounds__(GT, 1)
     uint32_t tmem = 0;
     bool ok = true;
     float dkh[64];  // dkhat of token ti_row, columns [64 chh, 64 chh + 64) (lower-half threads)
+    const int pr = tid >> 4, pc = tid & 15;  // 8-feature piece pc of rows pr + 16 j
+    const int hf = tid & 1;                   // column half when building the F / E operands
 
+    // ---- every input of the chunk requested at once: Q, K, dO by TMA; the S and U tile images
+    //      and dR (fp32, into the F/E area) by bulk copies; lambda follows once Z is done
     if (tid == 0) {
         mbar_init(bar_full, 1);
         mbar_init(bar1, 1);
         mbar_init(bar2, 1);
         mbar_init(bar3, 1);
+        mbar_init(bar_lam, 1);
         fence_mbar_init();
-        mbar_expect_tx(bar_full, 6 * 8192);
+        mbar_expect_tx(bar_full, 6 * 8192 + 65536 + 32768 + CH * DV * 4);
         tma_load_4d(sbase + G_QK, &tm_q, bar_full, 0, h, t0, b);
         tma_load_4d(sbase + G_QK + 16384, &tm_q, bar_full, 64, h, t0, b);
         tma_load_4d(sbase + G_QK + 8192, &tm_k, bar_full, 0, h, t0, b);
         tma_load_4d(sbase + G_QK + 24576, &tm_k, bar_full, 64, h, t0, b);
         tma_load_4d(sbase + G_DOR, &tm_do, bar_full, 0, h, t0, b);
         tma_load_4d(sbase + G_DOR + 16384, &tm_do, bar_full, 64, h, t0, b);
+        bulk_load(sbase + G_SL, a.Stl + crow * 65536, 65536, bar_full);
+        bulk_load(sbase + G_UH, a.Utl + crow * 32768, 32768, bar_full);
+        bulk_load(sbase + G_F, a.dR + crow * CH * DV, CH * DV * 4, bar_full);
     }
     if (warp == 0) {
         tmem_alloc(smem_u32(&ms->tmem_base), 512);
         tmem_relinquish();
     }
     if (tid < CH) {
-        ms->rowsum[tid] = 0.f;
-        ms->colsum[tid] = 0.f;
         ms->rowB[tid] = 0.f;
         ms->s_oq[tid] = 0.f;
         ms->s_rx[tid] = 0.f;
         ms->s_uk[tid] = 0.f;
         ms->kd[tid] = 0.f;
     }
-    // ---- per-token rows (4 threads per token, 32 features each): key norm, Kaczmarz
-    //      coefficients, dv = c dR, dc = dR . v, and the dR, U operand tiles
+    // Row-major [64][128] arrays are handled in 8-feature pieces: thread tid takes piece pc of
+    // rows pr + 16 j (16 consecutive threads share a row).
+    uint4 vraw[4];
     {
-        const int i = tid >> 2, qq = tid & 3;
-        const bool live = i < n;
-        const size_t ti = tok_index(b, t0 + (live ? i : 0), h, T, H);
-        float r2 = 0.f;
-        if (live) {
-            const uint4* kp =
-                reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.k) + ti * DK + 32 * qq);
+        uint4 kraw[4];
+        float etav[4], gv[4];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                float f[8];
-                unpack_bf16x8(kp[u], f);
+        for (int j = 0; j < 4; ++j) {
+            const int i = pr + 16 * j;
+            const bool live = i < n;
+            const size_t ti = tok_index(b, t0 + (live ? i : 0), h, T, H);
+            kraw[j] = live ? reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.k) + ti * DK)[pc]
+                           : make_uint4(0u, 0u, 0u, 0u);
+            vraw[j] = live ? reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.v) + ti * DV)[pc]
+                           : make_uint4(0u, 0u, 0u, 0u);
+            etav[j] = live ? a.eta[ti] : 0.f;
+            gv[j] = live ? a.g[ti] : 0.f;
+        }
 #pragma unroll
-                for (int e = 0; e < 8; ++e) r2 = fmaf(f[e], f[e], r2);
+        for (int j = 0; j < 4; ++j) {
+            const int i = pr + 16 * j;
+            float f[8];
+            unpack_bf16x8(kraw[j], f);
+            float r2 = 0.f;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) r2 = fmaf(f[e], f[e], r2);
+#pragma unroll
+            for (int o = 1; o < 16; o <<= 1) r2 += __shfl_xor_sync(0xffffffffu, r2, o);
+            const KaczCoef cf = kacz_coef(etav[j], r2, a.eps);
+            if (pc == 0) {
+                ms->graw[i] = gv[j];
+                ms->eta[i] = etav[j];
+                ms->r2[i] = r2;
+                ms->bco[i] = cf.b;
+                ms->cco[i] = cf.c;
+                ms->invr[i] = cf.inv_r;
             }
         }
-        r2 += __shfl_xor_sync(0xffffffffu, r2, 1);
-        r2 += __shfl_xor_sync(0xffffffffu, r2, 2);
-        const float eta_i = live ? a.eta[ti] : 0.f;
-        const float g_i = live ? a.g[ti] : 0.f;
-        const KaczCoef cf = kacz_coef(eta_i, r2, a.eps);
-        if (qq == 0) {
-            ms->graw[i] = g_i;
-            ms->eta[i] = eta_i;
-            ms->r2[i] = r2;
-            ms->bco[i] = cf.b;
-            ms->cco[i] = cf.c;
-            ms->invr[i] = cf.inv_r;
-        }
-        float x[32];
-        {
-            const float4* src = reinterpret_cast<const float4*>(a.dR + (crow * CH + i) * DV + 32 * qq);
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const float4 f = src[u];
-                x[4 * u] = f.x; x[4 * u + 1] = f.y; x[4 * u + 2] = f.z; x[4 * u + 3] = f.w;
-            }
-        }
-        float dcp = 0.f;
-        if (live) {
-            const uint4* vp = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.v) + ti * DV + 32 * qq);
-            float dvv[32];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                float f[8];
-                unpack_bf16x8(vp[u], f);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    dcp = fmaf(x[8 * u + e], f[e], dcp);
-                    dvv[8 * u + e] = cf.c * x[8 * u + e];
-                }
-            }
-            st_row32<TOut>(static_cast<TOut*>(a.dv) + ti * DV + 32 * qq, dvv);
-        }
-        dcp += __shfl_xor_sync(0xffffffffu, dcp, 1);
-        dcp += __shfl_xor_sync(0xffffffffu, dcp, 2);
-        if (qq == 0) ms->dc[i] = dcp;
-        st_chunks_split(sm + G_DOR + (qq >> 1) * 16384 + 8192, sm + G_DRL + (qq >> 1) * 8192, i, 4 * (qq & 1), 4, x);
-        {
-            const float4* src = reinterpret_cast<const float4*>(a.Uch + (crow * CH + i) * DV + 32 * qq);
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const float4 f = src[u];
-                x[4 * u] = f.x; x[4 * u + 1] = f.y; x[4 * u + 2] = f.z; x[4 * u + 3] = f.w;
-            }
-        }
-        st_chunks_split(sm + G_UH + (qq >> 1) * 8192, sm + G_UL + (qq >> 1) * 8192, i, 4 * (qq & 1), 4, x);
     }
-    // ---- S hi/lo tiles (thread = dk row rr, dv half hf); S stays in registers for <lambda, S>
-    float sv[64];
-    const int rr = tid >> 1, hf = tid & 1;
+    __syncthreads();
+    ok = mbar_wait_bounded(bar_full, 0, kWaitNs);
+    if (__syncthreads_or(!ok)) goto done;
+    // ---- dR: dv = c dR, dc = dR . v, and the dR hi (rows 64-127 of [dO; dR]) / lo tiles
     {
-        const float4* src = reinterpret_cast<const float4*>(a.Sch + (crow * DK + rr) * DV + 64 * hf);
+        const float* stg = reinterpret_cast<const float*>(sm + G_F);
 #pragma unroll
-        for (int u = 0; u < 16; ++u) {
-            const float4 f = src[u];
-            sv[4 * u] = f.x; sv[4 * u + 1] = f.y; sv[4 * u + 2] = f.z; sv[4 * u + 3] = f.w;
+        for (int j = 0; j < 4; ++j) {
+            const int i = pr + 16 * j;
+            const float4 f0 = *reinterpret_cast<const float4*>(stg + i * DV + 8 * pc);
+            const float4 f1 = *reinterpret_cast<const float4*>(stg + i * DV + 8 * pc + 4);
+            const float x[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
+            float vv[8];
+            unpack_bf16x8(vraw[j], vv);
+            float dcp = 0.f;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) dcp = fmaf(x[e], vv[e], dcp);
+#pragma unroll
+            for (int o = 1; o < 16; o <<= 1) dcp += __shfl_xor_sync(0xffffffffu, dcp, o);
+            if (pc == 0) ms->dc[i] = dcp;
+            if (i < n) {
+                const float ci = ms->cco[i];
+                float y[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) y[e] = ci * x[e];
+                st_piece8<TOut>(static_cast<TOut*>(a.dv) + tok_index(b, t0 + i, h, T, H) * DV + 8 * pc, y);
+            }
+            st_piece_split(sm + G_DOR + (pc >> 3) * 16384 + 8192, sm + G_DRL + (pc >> 3) * 8192, i, pc & 7, x);
         }
-        st_chunks_split(sm + G_SL + hf * 16384, sm + G_SL + 32768 + hf * 16384, rr, 0, 8, sv);
     }
     fence_proxy_async();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     tmem = ms->tmem_base;
-    ok = mbar_wait_bounded(bar_full, 0, kWaitNs);
-    if (__syncthreads_or(!ok)) goto done;
-    // ---- MMA group 1: Gram, Y / D, dO S^T and dR S^T
+    // ---- MMA group 1: Gram, Y / D, dO S^T and dR S^T (U and S as MN-major B operands)
     if (tid == 0) {
-        tc_fence_after();
         const uint32_t i64 = idesc_bf16(128, 64, false, false);
-        const uint32_t i128 = idesc_bf16(128, 128, false, false);
+        const uint32_t i64n = idesc_bf16(128, 64, false, true);
+        const uint32_t i128n = idesc_bf16(128, 128, false, true);
 #pragma unroll
         for (int s = 0; s < 8; ++s) {
             const uint32_t off = (s >> 2) * 16384 + (s & 3) * 32;
@@ -637,23 +664,21 @@ __global__ void __launch_bounds__(GT, 1)
 #pragma unroll
             for (int s = 0; s < 8; ++s)
                 mma_bf16(tmem + TG_YA, smem_desc(sbase + G_DOR + (s >> 2) * 16384 + (s & 3) * 32, 16, 1024),
-                         smem_desc(sbase + (p ? G_UL : G_UH) + (s >> 2) * 8192 + (s & 3) * 32, 16, 1024), i64,
-                         (p | s) > 0);
+                         smem_desc(sbase + (p ? G_UL : G_UH) + s * 2048, 8192, 1024), i64n, (p | s) > 0);
 #pragma unroll
         for (int s = 0; s < 8; ++s)
             mma_bf16(tmem + TG_YB, smem_desc(sbase + G_DRL - 8192 + (s >> 2) * 8192 + (s & 3) * 32, 16, 1024),
-                     smem_desc(sbase + G_UH + (s >> 2) * 8192 + (s & 3) * 32, 16, 1024), i64, s > 0);
+                     smem_desc(sbase + G_UH + s * 2048, 8192, 1024), i64n, s > 0);
         // [dO; dR hi] S^T with S hi, then S lo
 #pragma unroll
         for (int p = 0; p < 2; ++p)
 #pragma unroll
             for (int s = 0; s < 8; ++s)
                 mma_bf16(tmem + TG_Z, smem_desc(sbase + G_DOR + (s >> 2) * 16384 + (s & 3) * 32, 16, 1024),
-                         smem_desc(sbase + G_SL + p * 32768 + (s >> 2) * 16384 + (s & 3) * 32, 16, 1024), i128,
-                         (p | s) > 0);
+                         smem_desc(sbase + G_SL + p * 32768 + s * 2048, 16384, 1024), i128n, (p | s) > 0);
         mma_commit(bar1);
     }
-    // ---- meanwhile: the decays (warp 1) and lambda (into registers), <lambda, S>
+    // ---- meanwhile: the decays (warp 1); this thread's pieces of the S tiles for <lambda, S>
     if (warp == 1) {
         const float x0 = ms->graw[2 * lane], x1 = ms->graw[2 * lane + 1];
         float s = x0 + x1;
@@ -671,51 +696,23 @@ __global__ void __launch_bounds__(GT, 1)
         for (int o = 16; o > 0; o >>= 1) gr = fmaxf(gr, __shfl_xor_sync(0xffffffffu, gr, o));
         if (lane == 0) ms->factored = gr < 80.f ? 1u : 0u;
     }
-    float lv[64];
-    {
-        const float4* src = reinterpret_cast<const float4*>(a.Lam + (crow * DK + rr) * DV + 64 * hf);
+    uint4 spc[16];  // hi pieces 0-7 then lo pieces 0-7 (same element positions)
 #pragma unroll
-        for (int u = 0; u < 16; ++u) {
-            const float4 f = src[u];
-            lv[4 * u] = f.x; lv[4 * u + 1] = f.y; lv[4 * u + 2] = f.z; lv[4 * u + 3] = f.w;
-        }
-        float p = 0.f;
-#pragma unroll
-        for (int e = 0; e < 64; ++e) p = fmaf(lv[e], sv[e], p);
-        p = warp_sum(p);
-        if (lane == 0) ms->red[warp] = p;
-    }
+    for (int j = 0; j < 16; ++j) spc[j] = reinterpret_cast<const uint4*>(sm + G_SL)[tid + 256 * j];
     __syncthreads();
     if (tid < CH) {
         const float Gt = ms->G[tid];
         ms->gam[tid] = __expf(Gt);
         ms->del[tid] = __expf(ms->G[CH - 1] - Gt);  // G is flat past the last token
         ms->ginv[tid] = ms->factored ? __expf(-Gt) : 0.f;
-    } else if (tid == CH) {
-        float p = 0.f;
-#pragma unroll
-        for (int w = 0; w < GT / 32; ++w) p += ms->red[w];
-        ms->lamS = p;
     }
-    // ---- lambda hi/lo over S once group 1 is done, then MMA group 2: [junk; U] lambda^T
+    // ---- lambda tiles over S once group 1 is done (every thread has read its S pieces)
     ok = mbar_wait_bounded(bar1, 0, kWaitNs);
-    if (__syncthreads_or(!ok)) goto done;
-    st_chunks_split(sm + G_SL + hf * 16384, sm + G_SL + 32768 + hf * 16384, rr, 0, 8, lv);
     fence_proxy_async();
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
+    if (__syncthreads_or(!ok)) goto done;
     if (tid == 0) {
-        const uint32_t i128 = idesc_bf16(128, 128, false, false);
-        const uint32_t ua[3] = {G_UH, G_UH, G_UL};
-        const uint32_t lb[3] = {G_SL, G_SL + 32768, G_SL};
-#pragma unroll
-        for (int p = 0; p < 3; ++p)
-#pragma unroll
-            for (int s = 0; s < 8; ++s)
-                mma_bf16(tmem + TG_L, smem_desc(sbase + ua[p] - 8192 + (s >> 2) * 8192 + (s & 3) * 32, 16, 1024),
-                         smem_desc(sbase + lb[p] + (s >> 2) * 16384 + (s & 3) * 32, 16, 1024), i128, (p | s) > 0);
-        mma_commit(bar2);
+        mbar_expect_tx(bar_lam, 65536);
+        bulk_load(sbase + G_SL, a.Ltl + crow * 65536, 65536, bar_lam);
     }
     // ---- Gram and Y / D epilogue: F, E to shared memory; row and column sums of the decay
     //      gradient terms (Y o P and D o Diag(b) L), and the L part of db
@@ -756,7 +753,7 @@ __global__ void __launch_bounds__(GT, 1)
                 rs += dgv[e];
             }
         }
-        atomicAdd(&ms->rowsum[i], rs);
+        ms->rs_part[2 * (top ? 0 : 1) + chh][i] = rs;
         if (!top) atomicAdd(&ms->rowB[i], rb);
         // column sums over this warp's 32 rows: lane l ends with column 32 chh + l
 #pragma unroll
@@ -769,7 +766,48 @@ __global__ void __launch_bounds__(GT, 1)
                 dgv[k2] = keep + __shfl_xor_sync(0xffffffffu, send, off);
             }
         }
-        atomicAdd(&ms->colsum[32 * chh + lane], dgv[0]);
+        ms->cs_part[q4][32 * chh + lane] = dgv[0];
+    }
+    // ---- lambda landed: <lambda, S> from the tile pieces, then MMA group 2: [junk; U] lambda^T
+    //      (A: U as the upper M half of an MN-major operand, B: lambda MN-major)
+    ok = mbar_wait_bounded(bar_lam, 0, kWaitNs);
+    if (__syncthreads_or(!ok)) goto done;
+    {
+        float p = 0.f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const uint4 lh = reinterpret_cast<const uint4*>(sm + G_SL)[tid + 256 * j];
+            const uint4 ll = reinterpret_cast<const uint4*>(sm + G_SL)[tid + 256 * (j + 8)];
+            float a0[8], a1[8], b0[8], b1[8];
+            unpack_bf16x8(spc[j], a0);
+            unpack_bf16x8(spc[j + 8], a1);
+            unpack_bf16x8(lh, b0);
+            unpack_bf16x8(ll, b1);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) p = fmaf(a0[e] + a1[e], b0[e] + b1[e], p);
+        }
+        p = warp_sum(p);
+        if (lane == 0) ms->red[warp] = p;
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (tid == 0) {
+        const uint32_t i128nn = idesc_bf16(128, 128, true, true);
+        const uint32_t ua[3] = {G_UH, G_UH, G_UL};
+        const uint32_t lb[3] = {G_SL, G_SL + 32768, G_SL};
+#pragma unroll
+        for (int p = 0; p < 3; ++p)
+#pragma unroll
+            for (int s = 0; s < 8; ++s)
+                mma_bf16(tmem + TG_L, smem_desc(sbase + ua[p] - 16384 + s * 2048, 16384, 1024),
+                         smem_desc(sbase + lb[p] + s * 2048, 16384, 1024), i128nn, (p | s) > 0);
+        mma_commit(bar2);
+    } else if (tid == 32) {
+        float p = 0.f;
+#pragma unroll
+        for (int w = 0; w < GT / 32; ++w) p += ms->red[w];
+        ms->lamS = p;
     }
     // ---- X operands over the lambda tiles once group 2 is done:
     //      A1 = [F Diag(1/r); (E + E^T) Diag(1/r)],  A2 = [0; F^T]  (hi/lo, 128 rows x 64 tokens)
@@ -880,7 +918,9 @@ __global__ void __launch_bounds__(GT, 1)
         const float srx = ms->s_rx[i] * ir, suk = ms->s_uk[i] * ir, soq = ms->s_oq[i];
         const float db = ms->rowB[i] - gi * srx;
         const float dc = ms->dc[i];
-        ms->dGs[i] = gi * (soq - bi * srx) - de * suk + ms->rowsum[i] - ms->colsum[i];
+        const float rsum = (ms->rs_part[0][i] + ms->rs_part[1][i]) + (ms->rs_part[2][i] + ms->rs_part[3][i]);
+        const float csum = (ms->cs_part[0][i] + ms->cs_part[1][i]) + (ms->cs_part[2][i] + ms->cs_part[3][i]);
+        ms->dGs[i] = gi * (soq - bi * srx) - de * suk + rsum - csum;
         float extra = warp_sum(de * suk);  // delta_i = gamma_last / gamma_i feeds dG of the last token
         if (lane == 0) ms->red[warp] = extra;
         const float r2 = ms->r2[i], den = r2 + a.eps, et = ms->eta[i];
@@ -948,10 +988,11 @@ done:
 size_t align1k(size_t x) { return (x + 1023) & ~size_t(1023); }
 
 struct BwdLayout {
-    size_t fwd, T, U, Lam, dR, S, total;
+    size_t fwd, T, S, U, L, dR, total;
 };
 
-BwdLayout bwd_layout(int B, int T, int H, bool have_S) {
+// [forward records | T tiles | S tiles | U tiles | lambda tiles | dR], each 1 KB aligned
+BwdLayout bwd_layout(int B, int T, int H) {
     FwdArgs fa{};
     fa.B = B;
     fa.T = T;
@@ -964,14 +1005,14 @@ BwdLayout bwd_layout(int B, int T, int H, bool have_S) {
     L.fwd = 0;
     L.T = o;
     o += align1k(nch * 16384);
+    L.S = o;
+    o += align1k(nch * 65536);
     L.U = o;
-    o += align1k(nch * CH * DV * sizeof(float));
-    L.Lam = o;
-    o += align1k(nch * DK * DV * sizeof(float));
+    o += align1k(nch * 32768);
+    L.L = o;
+    o += align1k(nch * 65536);
     L.dR = o;
     o += align1k(nch * CH * DV * sizeof(float));
-    L.S = o;
-    if (!have_S) o += align1k(nch * DK * DV * sizeof(float));
     L.total = o;
     return L;
 }
@@ -989,39 +1030,27 @@ cudaError_t launch_grad(const CUtensorMap& mq, const CUtensorMap& mk, const CUte
 }  // namespace
 
 size_t chunk_bwd_tc_workspace(int B, int T, int H, bool have_S_chunks) {
+    (void)have_S_chunks;  // the tensor-core path recomputes the states as tiles in any case
     if (B < 1 || H < 1 || T < 1) return 0;
-    return bwd_layout(B, T, H, have_S_chunks).total;
+    return bwd_layout(B, T, H).total;
 }
 
-cudaError_t launch_chunk_bwd_tc(const BwdTcArgs& a, void* ws, size_t ws_bytes, cudaStream_t st) {
-    const BwdLayout L = bwd_layout(a.B, a.T, a.H, a.S_chunks != nullptr);
+cudaError_t launch_chunk_fwd_train_tc(const FwdArgs& f, void* ws, size_t ws_bytes, cudaStream_t st) {
+    const BwdLayout L = bwd_layout(f.B, f.T, f.H);
     if (ws == nullptr || ws_bytes < L.total) return cudaErrorInvalidValue;
     uint8_t* w = static_cast<uint8_t*>(ws);
-    float* Sws = a.S_chunks ? nullptr : reinterpret_cast<float*>(w + L.S);
-    // 1-2: the forward's records, T, S (unless given) and U
-    FwdArgs fa{};
-    fa.q = a.q;
-    fa.k = a.k;
-    fa.v = a.v;
-    fa.eta = a.eta;
-    fa.g = a.g;
-    fa.eps = a.eps;
-    fa.S0 = a.S0;
-    fa.o = nullptr;
-    fa.S_T = nullptr;
-    fa.S_chunks = Sws;
-    fa.B = a.B;
-    fa.T = a.T;
-    fa.H = a.H;
-    fa.Dk = fa.Dv = 128;
-    fa.bf16 = true;
-    fa.out_bf16 = false;
-    fa.U_chunks = reinterpret_cast<float*>(w + L.U);
-    fa.T_chunks = w + L.T;
+    FwdArgs fa = f;
+    fa.T_tiles = w + L.T;
+    fa.S_tiles = w + L.S;
+    fa.U_tiles = w + L.U;
     cudaError_t e = launch_chunk_fwd_split_prep(fa, w + L.fwd, st);
-    if (e != cudaSuccess) return e;
-    if ((e = launch_chunk_fwd_split_state(fa, w + L.fwd, st)) != cudaSuccess) return e;
-    // 3-4: reverse state pass and gradients
+    return e == cudaSuccess ? launch_chunk_fwd_split_state(fa, w + L.fwd, st) : e;
+}
+
+cudaError_t launch_chunk_bwd_tc_reverse(const BwdTcArgs& a, void* ws, size_t ws_bytes, cudaStream_t st) {
+    const BwdLayout L = bwd_layout(a.B, a.T, a.H);
+    if (ws == nullptr || ws_bytes < L.total) return cudaErrorInvalidValue;
+    uint8_t* w = static_cast<uint8_t*>(ws);
     CUtensorMap mq, mk, mdo;
     if (!make_map(&mq, a.q, a.B, a.T, a.H) || !make_map(&mk, a.k, a.B, a.T, a.H) ||
         !make_map(&mdo, a.dO, a.B, a.T, a.H))
@@ -1035,10 +1064,10 @@ cudaError_t launch_chunk_bwd_tc(const BwdTcArgs& a, void* ws, size_t ws_bytes, c
     d.eps = a.eps;
     d.dS_T = a.dS_T;
     d.recs = w + L.fwd;
-    d.Tch = w + L.T;
-    d.Sch = a.S_chunks ? a.S_chunks : Sws;
-    d.Uch = reinterpret_cast<const float*>(w + L.U);
-    d.Lam = reinterpret_cast<float*>(w + L.Lam);
+    d.Ttl = w + L.T;
+    d.Stl = w + L.S;
+    d.Utl = w + L.U;
+    d.Ltl = w + L.L;
     d.dR = reinterpret_cast<float*>(w + L.dR);
     d.dq = a.dq;
     d.dk = a.dk;
@@ -1050,12 +1079,33 @@ cudaError_t launch_chunk_bwd_tc(const BwdTcArgs& a, void* ws, size_t ws_bytes, c
     d.T = a.T;
     d.H = a.H;
     const int BH = a.B * a.H, NC = (a.T + CH - 1) / CH;
-    e = cudaFuncSetAttribute(chunk_bwd_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)R_SMEM);
+    cudaError_t e =
+        cudaFuncSetAttribute(chunk_bwd_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)R_SMEM);
     if (e != cudaSuccess) return e;
     chunk_bwd_state_kernel<<<BH, RT, R_SMEM, st>>>(mq, mdo, d);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     return a.out_bf16 ? launch_grad<__nv_bfloat16>(mq, mk, mdo, d, NC, BH, st)
                       : launch_grad<float>(mq, mk, mdo, d, NC, BH, st);
+}
+
+cudaError_t launch_chunk_bwd_tc(const BwdTcArgs& a, void* ws, size_t ws_bytes, cudaStream_t st) {
+    // 1-2: the forward's records and the T, S and U tiles (no o, S_T or fp32 states)
+    FwdArgs fa{};
+    fa.q = a.q;
+    fa.k = a.k;
+    fa.v = a.v;
+    fa.eta = a.eta;
+    fa.g = a.g;
+    fa.eps = a.eps;
+    fa.S0 = a.S0;
+    fa.B = a.B;
+    fa.T = a.T;
+    fa.H = a.H;
+    fa.Dk = fa.Dv = 128;
+    fa.bf16 = true;
+    cudaError_t e = launch_chunk_fwd_train_tc(fa, ws, ws_bytes, st);
+    // 3-4: reverse state pass and gradients
+    return e == cudaSuccess ? launch_chunk_bwd_tc_reverse(a, ws, ws_bytes, st) : e;
 }
 
 cudaError_t bwd_tc_take_error(cudaStream_t st, unsigned int* flag) {

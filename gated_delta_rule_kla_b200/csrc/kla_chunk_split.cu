@@ -273,8 +273,8 @@ __global__ void __launch_bounds__(PT, 3)
             }
         }
         __syncthreads();  // T is read; T'' overwrites it
-        if (a.T_chunks) {
-            uint8_t* tt = static_cast<uint8_t*>(a.T_chunks) + ((size_t)head * NC + c) * 16384;
+        if (a.T_tiles) {
+            uint8_t* tt = static_cast<uint8_t*>(a.T_tiles) + ((size_t)head * NC + c) * 16384;
             st_chunks_split_global(tt, tt + 8192, i, 2 * qq, 2, tv);
         }
         float v[16];
@@ -438,6 +438,8 @@ __global__ void __launch_bounds__(ST, 1)
                                      DK * DV
                        : nullptr;
     float* Sc = (a.S_chunks && !ident) ? a.S_chunks + (size_t)head_idx * NCtot * DK * DV : nullptr;
+    uint8_t* Stl = (a.S_tiles && !ident) ? static_cast<uint8_t*>(a.S_tiles) + (size_t)head_idx * NCtot * 65536 : nullptr;
+    uint8_t* Utl = (a.U_tiles && !ident) ? static_cast<uint8_t*>(a.U_tiles) + (size_t)head_idx * NCtot * 32768 : nullptr;
     const bool write_o = !ident && a.o != nullptr;
     // Without outputs (the transition pass of the segmented mode) Q, P and the O products are not
     // needed; with zero values (its identity kind) neither is U'.
@@ -665,16 +667,12 @@ __global__ void __launch_bounds__(ST, 1)
                 tmem_ld32(tmem + lane_base + TM_U + 32 * ch, x);
                 tmem_ld_wait();
                 const float* up = reinterpret_cast<const float*>(stg_p + SO_UP);
-                float* Uc = (a.U_chunks && !ident) ? a.U_chunks + ((size_t)head_idx * NCtot + c) * CH * DV : nullptr;
+                uint8_t* Ut = Utl ? Utl + (size_t)c * 32768 : nullptr;
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
                     if (!ident) {
 #pragma unroll
                         for (int e = 16 * half; e < 16 * half + 16; ++e) x[e] += up[(32 * ch + e) * DV + row];
-                    }
-                    if (Uc) {
-#pragma unroll
-                        for (int e = 16 * half; e < 16 * half + 16; ++e) Uc[(32 * ch + e) * DV + row] = x[e];
                     }
                     uint32_t hp[8], lp[8];
                     split_pack<16>(x + 16 * half, hp, lp);
@@ -682,6 +680,19 @@ __global__ void __launch_bounds__(ST, 1)
                     tmem_st8u(tmem + lane_base + TM_UL + 16 * ch + 8 * half, lp);
                     epi_signal(u_ready0 + 8 * half, tid);  // the first also covers the master rescale
                 }
+                // tile images for the backward, read back from TMEM while the S product runs: U(c)
+                // hi/lo and the chunk's incoming state S_c hi/lo (still the S operand)
+                if (Ut) {
+                    uint32_t wh[16], wl[16];
+                    tmem_ld16u(tmem + lane_base + TM_UH + 16 * ch, wh);
+                    tmem_ld16u(tmem + lane_base + TM_UL + 16 * ch, wl);
+                    tmem_ld_wait();
+                    st_words_sw128_global(Ut, row, 4 * ch, 4, wh);
+                    st_words_sw128_global(Ut + 16384, row, 4 * ch, 4, wl);
+                }
+                if (Stl)
+                    st_tmem_row_global(tmem + lane_base + TM_SH + 32 * ch, tmem + lane_base + TM_SL + 32 * ch,
+                                       Stl + (size_t)c * 65536 + ch * 16384, 32768, row);
             }
             // ---- state epilogue: S_{c+1} to hi/lo in two halves (releasing U(c+1)), then the
             //      fp32 master pre-scaled by the next gamma_last
@@ -712,6 +723,7 @@ __global__ void __launch_bounds__(ST, 1)
                             Sc[((size_t)(c + 1) * DK + 64 * ch + 32 + e) * DV + row] = x1[e];
                         }
                     }
+
                     const float gN = reinterpret_cast<const float*>(sm + S_SC + st * REC_SCB)[CH];
 #pragma unroll
                     for (int e = 0; e < 32; ++e) {
@@ -902,7 +914,8 @@ cudaError_t launch_chunk_fwd_split_state(const FwdArgs& a, void* ws, cudaStream_
     p1.o = nullptr;
     p1.S_T = MN;
     p1.S_chunks = nullptr;
-    p1.U_chunks = nullptr;
+    p1.S_tiles = nullptr;
+    p1.U_tiles = nullptr;
     p1.nseg = L.nseg;
     p1.seg_chunks = L.segc;
     p1.kinds = 2;

@@ -35,12 +35,14 @@ struct FwdArgs {
     // [B*H, nseg, Dk, Dv] (S_T: [kinds, B*H, nseg, Dk, Dv]) and a second grid row (kind 1)
     // runs each segment from the identity state with zero values (the segment's transition).
     int nseg, seg_chunks, kinds;
-    // Extra outputs of the split path for the tensor-core backward (both may be null):
-    // U_chunks [B*H, NC, 64, Dv] fp32, each chunk's U = T (Diag(c) V - Diag(b gamma) Khat S)
-    // (state pass); T_chunks [B*H, NC] x 16 KB, each chunk's T = (I + L)^{-1} as bf16 hi then lo
-    // [64 x 64] tiles, rows of T in the 128-byte swizzle (preparation kernel).
-    float* U_chunks;
-    void* T_chunks;
+    // Extra outputs of the split path for the tensor-core backward (all may be null), per chunk
+    // and head as bf16 hi then lo tile images in the 128-byte swizzle:
+    //   T_tiles  16 KB  T = (I + L)^{-1}: [64 rows of T][64]                   (preparation kernel)
+    //   S_tiles  64 KB  the chunk's incoming state: [dk half][128 dv rows][64 dk]     (state pass)
+    //   U_tiles  32 KB  U = T (Diag(c) V - Diag(b gamma) Khat S): [128 dv rows][64 tokens]
+    void* T_tiles;
+    void* S_tiles;
+    void* U_tiles;
 };
 
 struct BwdArgs {
@@ -77,6 +79,10 @@ struct BwdTcArgs {
 // head, T (16 KB), U (32 KB), lambda (64 KB), dR (32 KB) and, without S_chunks, S (64 KB).
 size_t chunk_bwd_tc_workspace(int B, int T, int H, bool have_S_chunks);
 cudaError_t launch_chunk_bwd_tc(const BwdTcArgs& a, void* ws, size_t ws_bytes, cudaStream_t st);
+// The two halves of launch_chunk_bwd_tc for a training step: the forward (o and S_T as `f` asks,
+// plus the backward's records and tiles in ws), then the backward from that ws.
+cudaError_t launch_chunk_fwd_train_tc(const FwdArgs& f, void* ws, size_t ws_bytes, cudaStream_t st);
+cudaError_t launch_chunk_bwd_tc_reverse(const BwdTcArgs& a, void* ws, size_t ws_bytes, cudaStream_t st);
 cudaError_t bwd_tc_take_error(cudaStream_t st, unsigned int* flag);
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st);

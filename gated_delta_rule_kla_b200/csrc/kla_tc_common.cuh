@@ -231,6 +231,31 @@ __device__ __forceinline__ void st_chunks_split_global(uint8_t* hi_block, uint8_
         st_pair_sw128_global(lo_block, r, c0 + c, l0, l1);
     }
 }
+// Packed bf16 words (two features per word, lower feature in the low half) as pieces
+// c0 .. c0 + n - 1 of row r of a 128-byte-swizzled global tile (c0 and n even).
+__device__ __forceinline__ void st_words_sw128_global(uint8_t* block, int r, int c0, int n, const uint32_t* w) {
+#pragma unroll
+    for (int c = 0; c < n; c += 2)
+        st_pair_sw128_global(block, r, c0 + c, make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]),
+                             make_uint4(w[4 * c + 4], w[4 * c + 5], w[4 * c + 6], w[4 * c + 7]));
+}
+// A thread's 32 TMEM columns of packed bf16 hi and lo words (64 features of its lane) as one
+// row of a global hi tile and the same row of the lo tile 'lo_off' bytes after it.
+__device__ __forceinline__ void st_tmem_row_global(uint32_t t_hi, uint32_t t_lo, uint8_t* block, uint32_t lo_off,
+                                                   int r) {
+    float h[32], l[32];
+    tmem_ld32(t_hi, h);
+    tmem_ld32(t_lo, l);
+    tmem_ld_wait();
+    uint32_t wh[32], wl[32];
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+        wh[e] = __float_as_uint(h[e]);
+        wl[e] = __float_as_uint(l[e]);
+    }
+    st_words_sw128_global(block, r, 0, 8, wh);
+    st_words_sw128_global(block + lo_off, r, 0, 8, wl);
+}
 __device__ __forceinline__ void st_chunks_bf16_global(uint8_t* block, int r, int c0, int n, const float* v) {
 #pragma unroll
     for (int c = 0; c < n; c += 2) {

@@ -138,9 +138,9 @@ kla_status kla_chunk_fwd_state(const void *q, const float *g, const float *S0, v
  * not be initialised) of at least kla_chunk_bwd_workspace_min() bytes (required; smaller is
  * KLA_ERR_WORKSPACE).  With at least kla_chunk_bwd_workspace() bytes, bf16 inputs with
  * Dk == Dv == 128 run on the tensor cores: the split forward's preparation and state pass are
- * recomputed into ws (about 241 KiB per chunk and head, plus 64 KiB without S_chunks), a
- * reverse state pass carries the state gradient chunk by chunk, and a chunk-parallel kernel
- * forms every gradient.  With less, and for every other shape, the CUDA-core backward runs.
+ * recomputed into ws (about 305 KiB per chunk and head; S_chunks is then not read), a reverse
+ * state pass carries the state gradient chunk by chunk, and a chunk-parallel kernel forms every
+ * gradient.  With less, and for every other shape, the CUDA-core backward runs.
  * The workspace must not be shared with a concurrent call.
  * Every output is fully overwritten.
  */
@@ -154,6 +154,34 @@ kla_status kla_chunk_bwd(const void *q, const void *k, const void *v, const floa
                          float *deta, float *dg, float *dS0, int B, int T, int H, int Dk,
                          int Dv, int chunk, int dtype, int out_dtype, void *ws, size_t ws_bytes,
                          void *stream);
+
+/*
+ * kla_chunk_fwd_train, kla_chunk_bwd_after_train -- a training step's forward and backward
+ * sharing one workspace, so the backward does not recompute the forward.  Same math as
+ * kla_chunk_fwd and kla_chunk_bwd ("Kaczmarz Linear Attention", section 4, Eqs. 7-9, and their
+ * exact derivative), same results bit for bit.
+ *   kla_chunk_fwd_train: arguments as kla_chunk_fwd without S_chunks; writes o and S_T (either
+ *     may be NULL) and leaves in ws what the backward needs: for bf16 inputs with
+ *     Dk == Dv == 128 and at least kla_chunk_bwd_workspace(..., have_S_chunks = 0) bytes, the
+ *     split forward's per-chunk records and every chunk's T, S and U as bf16 tile images;
+ *     otherwise (at least kla_chunk_bwd_workspace_min(..., 0) bytes) the chunk states.
+ *   kla_chunk_bwd_after_train: arguments as kla_chunk_bwd without S0 and S_chunks; must get the
+ *     same q, k, v, eta, g, eps, sizes, dtype, ws and ws_bytes as the kla_chunk_fwd_train call it
+ *     follows (ordered after it: same stream, or an event), with ws untouched in between.
+ * ws: device memory, 16-byte aligned, owned by the caller, contents need not be initialised;
+ * too small is KLA_ERR_WORKSPACE.  Returns KLA_OK or an error status; on error nothing is
+ * launched.
+ */
+kla_status kla_chunk_fwd_train(const void *q, const void *k, const void *v, const float *eta,
+                               const float *g, float eps, const float *S0, void *o, float *S_T,
+                               int B, int T, int H, int Dk, int Dv, int chunk, int dtype,
+                               int out_dtype, void *ws, size_t ws_bytes, void *stream);
+kla_status kla_chunk_bwd_after_train(const void *q, const void *k, const void *v, const float *eta,
+                                     const float *g, float eps, const void *dO, const float *dS_T,
+                                     void *dq, void *dk, void *dv, float *deta, float *dg,
+                                     float *dS0, int B, int T, int H, int Dk, int Dv, int chunk,
+                                     int dtype, int out_dtype, void *ws, size_t ws_bytes,
+                                     void *stream);
 
 /*
  * kla_decode_step -- one generated token: Algorithm 1 (left panel), lines 2-6 (readout

@@ -130,3 +130,19 @@ def test_product_and_oracle_share_no_code():
             text = open(os.path.join(ROOT, "oracle", f)).read()
             assert "gated_delta_rule_kla_b200" not in text
             assert "kla.h" not in text
+
+
+def test_train_pair_rejects_before_launch(L):
+    need = L.kla_chunk_bwd_workspace(2, 100, 3, 128, 128, 64, 1, 0)
+    small = L.kla_chunk_bwd_workspace_min(2, 100, 3, 128, 128, 64, 1, 0)
+    assert need > small  # bf16, d = 128: the tensor-core backward's layout
+    fwd = lambda ws=FAKE, n=need, q=FAKE, Dk=128: L.kla_chunk_fwd_train(
+        q, FAKE, FAKE, FAKE, FAKE, 1e-6, None, FAKE, None, 2, 100, 3, Dk, 128, 64, 1, 0, ws, n, None)
+    bwd = lambda ws=FAKE, n=need, dO=FAKE: L.kla_chunk_bwd_after_train(
+        FAKE, FAKE, FAKE, FAKE, FAKE, 1e-6, dO, None, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 2, 100, 3, 128, 128,
+        64, 1, 0, ws, n, None)
+    assert fwd(ws=None) == WORKSPACE and b"kla_chunk_fwd_train" in L.kla_last_error()
+    assert fwd(n=small - 1) == WORKSPACE
+    assert fwd(q=None) == INVALID and fwd(ws=MISALIGNED) == INVALID and fwd(Dk=96) == UNSUPPORTED
+    assert bwd(ws=None) == WORKSPACE and b"kla_chunk_bwd_after_train" in L.kla_last_error()
+    assert bwd(dO=None) == INVALID and bwd(n=small - 1) == WORKSPACE

@@ -452,6 +452,37 @@ def test_bwd_tensor_cores_more_heads_than_sms(kla, oracle_mod):
         assert rel_err(got, ref[name]) <= 2e-2, name
 
 
+@pytest.mark.parametrize("B,T,H,D,dtype,small_ws", [
+    (2, 150, 3, 128, "bf16", False),   # tensor-core layout: records and tiles shared
+    (2, 150, 3, 128, "bf16", True),    # minimum workspace: chunk states shared, CUDA-core backward
+    (1, 130, 2, 64, "f32", False),
+])
+def test_train_pair_equals_separate_calls(kla, B, T, H, D, dtype, small_ws):
+    """chunk_fwd_train + chunk_bwd_after_train give what chunk_fwd and chunk_bwd give."""
+    inp = small_inputs(B, T, H, D, D, dtype, seed=T + H, g_lo=-0.1)
+    d = {k: v.cuda() for k, v in inp.items()}
+    gen = torch.Generator().manual_seed(3)
+    dO = torch.randn(B, T, H, D, generator=gen).to(d["q"].dtype).cuda()
+    dST = torch.randn(B, H, D, D, generator=gen).cuda()
+    L = kla.lib()
+    size = L.kla_chunk_bwd_workspace_min if small_ws else L.kla_chunk_bwd_workspace
+    ws = torch.empty(size(B, T, H, D, D, 64, 1 if dtype == "bf16" else 0, 0), dtype=torch.uint8, device="cuda")
+    o1, S1, _ = kla.chunk_fwd_train(d["q"], d["k"], d["v"], d["eta"], d["g"], 1e-6, d["S0"], workspace=ws)
+    g1 = kla.chunk_bwd_after_train(d["q"], d["k"], d["v"], d["eta"], d["g"], dO, ws, 1e-6, dST)
+    # the minimum workspace runs the one-kernel forward, as chunk_fwd does without a workspace
+    o2, S2 = kla.chunk_fwd(d["q"], d["k"], d["v"], d["eta"], d["g"], 1e-6, d["S0"], fused=small_ws)
+    g2 = kla.chunk_bwd(d["q"], d["k"], d["v"], d["eta"], d["g"], dO, 1e-6, d["S0"], dST, cuda_cores=small_ws)
+    torch.cuda.synchronize()
+    kla.check_device_error()
+    assert torch.equal(o1, o2) and torch.equal(S1, S2)
+    for name in GRADS:
+        if dtype == "bf16" and not small_ws:
+            assert torch.equal(g1[name], g2[name]), name  # same kernels on the same tiles
+        else:  # fp32 atomics may add in another order
+            a, b = g1[name].double(), g2[name].double()
+            assert (a - b).abs().max().item() <= 1e-5 * (b.pow(2).mean().sqrt().item() + 1e-30), name
+
+
 def test_bwd_with_saved_chunk_states_matches_recompute(kla):
     inp = small_inputs(1, 190, 2, 128, 128, "bf16", seed=8)
     d = {k: v.cuda() for k, v in inp.items()}
