@@ -13,8 +13,12 @@
 // independent): Dk x 64 fp32.  A persistent grid with two CTAs per SM walks the units; a
 // single thread keeps up to STAGES - 1 units ahead in flight with 2-D TMA loads (plus 1-D
 // bulk copies of k, q and the unit's slice of v) into a ring of shared-memory stages, while
-// all threads reduce, update and store the current unit.  Waits are bounded; on expiry the
-// kernel records an error word (reported by kla_check_device_error) and stops.
+// all threads reduce and update the current unit; the updated tile goes back into its stage
+// and leaves by one 2-D TMA store once every warp has written its rows (an mbarrier, so no
+// warp waits for the store).  One block-wide barrier per unit: every lane finishes the
+// reductions for its own column group from per-warp partials kept in two buffers (by unit
+// parity).  Waits are bounded; on expiry the kernel records an error word (reported by
+// kla_check_device_error) and stops.
 #include <cuda.h>
 
 #include "kla_device.cuh"
@@ -37,17 +41,26 @@ constexpr int STAGES = 3;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
 constexpr int NW = NT / 32;       // warps
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void tma_store_2d(const void* tmap, uint32_t src, int c0, int c1) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(tmap)),
+                 "r"(src), "r"(c0), "r"(c1)
+                 : "memory");
+}
 constexpr int MAX_UNITS_PER_CTA = 64;
 
 template <int DK, typename Tin>
 struct DecodeSmem {
     float s[STAGES][DK][NV];                    // state tiles
     Tin kv[STAGES][DK], qv[STAGES][DK], vv[STAGES][NV];
-    float4 red_k[NW][CG], red_q[NW][CG];        // per-warp partial S^T k, S^T q
-    float4 be[CG];                              // beta * e for the unit's columns
-    float scal[2][NW];                          // per-warp partial ||k||^2, k.q
+    float4 red_k[2][NW][CG], red_q[2][NW][CG];  // per-warp partial S^T k, S^T q (by unit parity)
+    float scal[2][2][NW];                       // per-warp partial ||k||^2, k.q (by unit parity)
     float alpha[MAX_UNITS_PER_CTA], eta[MAX_UNITS_PER_CTA];
-    uint64_t full[STAGES];
+    uint64_t full[STAGES], done[STAGES];        // tile landed; every warp wrote its updated rows
 };
 
 template <int DK, int DV, typename Tin, typename TOut>
@@ -71,18 +84,13 @@ __global__ void __launch_bounds__(NT, 2)
     const int nmine = (blockIdx.x < units) ? (units - 1 - blockIdx.x) / stride + 1 : 0;
 
     if (tid == 0) {
-        for (int s = 0; s < STAGES; ++s) mbar_init(smem_u32(&sm.full[s]), 1);
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(smem_u32(&sm.full[s]), 1);
+            mbar_init(smem_u32(&sm.done[s]), NW);
+        }
         fence_mbar_init();
         prefetch_tmap(&tm_s);
     }
-    // the decay and gate of every unit this CTA will process, loaded once
-    if (tid < nmine) {
-        const int head = (blockIdx.x + tid * stride) / UPH;
-        sm.alpha[tid] = expf(g[head]);
-        sm.eta[tid] = eta[head];
-    }
-    __syncthreads();
-
     // one thread requests unit number i of this CTA into stage i % STAGES
     auto request = [&](int i) {
         const int u = blockIdx.x + i * stride;
@@ -95,21 +103,30 @@ __global__ void __launch_bounds__(NT, 2)
         bulk_load(smem_u32(&sm.qv[st][0]), q + (size_t)head * DK, kVecBytes, bar);
         bulk_load(smem_u32(&sm.vv[st][0]), v + (size_t)head * DV + v0, kVBytes, bar);
     };
-    if (tid == 0) {
+    if (tid == 0) {  // the first tiles are requested before anything else
         for (int i = 0; i < STAGES - 1 && i < nmine; ++i) request(i);
     }
+    // the decay and gate of every unit this CTA will process, loaded once
+    if (tid < nmine) {
+        const int head = (blockIdx.x + tid * stride) / UPH;
+        sm.alpha[tid] = expf(g[head]);
+        sm.eta[tid] = eta[head];
+    }
+    __syncthreads();
 
+
+    bool store_failed = false;  // tid 0: a store barrier expired (the next unit's check stops all)
     for (int i = 0; i < nmine; ++i) {
         const int u = blockIdx.x + i * stride;
         const int head = u / UPH, v0 = (u % UPH) * NV;
-        const int st = i % STAGES;
-        // keep STAGES - 1 units in flight; every thread finished reading stage (i - 1) % STAGES
-        // before the previous iteration's second barrier (the update uses registers only)
+        const int st = i % STAGES, par = i & 1;
+        // keep STAGES - 1 units in flight; the stage refilled now held unit i - 1, whose store
+        // was issued at the end of the previous iteration: let it finish reading first
         if (tid == 0 && i + STAGES - 1 < nmine) {
-            fence_proxy_async();
+            bulk_wait_read();
             request(i + STAGES - 1);
         }
-        const bool ok = mbar_wait_bounded(smem_u32(&sm.full[st]), (i / STAGES) & 1, kWaitLimitNs);
+        const bool ok = mbar_wait_bounded(smem_u32(&sm.full[st]), (i / STAGES) & 1, kWaitLimitNs) && !store_failed;
         if (__syncthreads_or(!ok)) {
             if (tid == 0) {
                 atomicOr(&g_decode_error, 1u);
@@ -128,7 +145,7 @@ __global__ void __launch_bounds__(NT, 2)
             kq = kx * qx;
         }
         float4 cur[RPT];
-        float kir[RPT];  // k rows of this thread, kept for the update (the stage is refilled early)
+        float kir[RPT];
         float4 pk = make_float4(0.f, 0.f, 0.f, 0.f), pq = pk;
 #pragma unroll
         for (int r = 0; r < RPT; ++r) {
@@ -150,35 +167,35 @@ __global__ void __launch_bounds__(NT, 2)
         kk = warp_sum(kk);
         kq = warp_sum(kq);
         if (lane < CG) {
-            sm.red_k[warp][lane] = pk;
-            sm.red_q[warp][lane] = pq;
+            sm.red_k[par][warp][lane] = pk;
+            sm.red_q[par][warp][lane] = pq;
         }
         if (lane == 0) {
-            sm.scal[0][warp] = kk;
-            sm.scal[1][warp] = kq;
+            sm.scal[par][0][warp] = kk;
+            sm.scal[par][1][warp] = kq;
         }
         __syncthreads();
+        // every lane: final sums, residual and beta e for its column group cg (== lane % 16)
         const float alpha = sm.alpha[i];
-        if (tid < CG) {  // final sums, residual and output for column group cg = tid
+        float4 be;
+        {
             float n2 = 0.f, kdq = 0.f;
             float4 sk = make_float4(0.f, 0.f, 0.f, 0.f), sq = sk;
 #pragma unroll
             for (int w = 0; w < NW; ++w) {
-                n2 += sm.scal[0][w];
-                kdq += sm.scal[1][w];
-                const float4 a = sm.red_k[w][tid], b = sm.red_q[w][tid];
+                n2 += sm.scal[par][0][w];
+                kdq += sm.scal[par][1][w];
+                const float4 a = sm.red_k[par][w][cg], b = sm.red_q[par][w][cg];
                 sk.x += a.x; sk.y += a.y; sk.z += a.z; sk.w += a.w;
                 sq.x += b.x; sq.y += b.y; sq.z += b.z; sq.w += b.w;
             }
             const float den = n2 + eps;
             const float beta = den > 0.f ? sm.eta[i] / den : 0.f;
-            float4 be;
-            be.x = beta * (to_f32(sm.vv[st][4 * tid + 0]) - alpha * sk.x);
-            be.y = beta * (to_f32(sm.vv[st][4 * tid + 1]) - alpha * sk.y);
-            be.z = beta * (to_f32(sm.vv[st][4 * tid + 2]) - alpha * sk.z);
-            be.w = beta * (to_f32(sm.vv[st][4 * tid + 3]) - alpha * sk.w);
-            sm.be[tid] = be;
-            if (o != nullptr) {  // o = alpha S^T q + (k.q) beta e
+            be.x = beta * (to_f32(sm.vv[st][4 * cg + 0]) - alpha * sk.x);
+            be.y = beta * (to_f32(sm.vv[st][4 * cg + 1]) - alpha * sk.y);
+            be.z = beta * (to_f32(sm.vv[st][4 * cg + 2]) - alpha * sk.z);
+            be.w = beta * (to_f32(sm.vv[st][4 * cg + 3]) - alpha * sk.w);
+            if (o != nullptr && tid < CG) {  // o = alpha S^T q + (k.q) beta e
                 TOut* oh = o + (size_t)head * DV + v0 + tid * 4;
                 oh[0] = from_f32<TOut>(fmaf(alpha, sq.x, kdq * be.x));
                 oh[1] = from_f32<TOut>(fmaf(alpha, sq.y, kdq * be.y));
@@ -186,10 +203,7 @@ __global__ void __launch_bounds__(NT, 2)
                 oh[3] = from_f32<TOut>(fmaf(alpha, sq.w, kdq * be.w));
             }
         }
-        __syncthreads();
-        // S <- alpha S + beta k e^T, written back in place from registers
-        const float4 be = sm.be[cg];
-        float4* Sh = reinterpret_cast<float4*>(S + (size_t)head * DK * DV + v0) + cg;
+        // S <- alpha S + beta k e^T into the stage, then out by one TMA store of the tile
 #pragma unroll
         for (int r = 0; r < RPT; ++r) {
             const int row = rg + r * RG;
@@ -199,9 +213,22 @@ __global__ void __launch_bounds__(NT, 2)
             x.y = fmaf(alpha, x.y, ki * be.y);
             x.z = fmaf(alpha, x.z, ki * be.z);
             x.w = fmaf(alpha, x.w, ki * be.w);
-            Sh[(size_t)row * (DV / 4)] = x;
+            *reinterpret_cast<float4*>(&sm.s[st][row][4 * cg]) = x;
+        }
+        fence_proxy_async();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&sm.done[st]));
+        if (tid == 0) {
+            if (!mbar_wait_bounded(smem_u32(&sm.done[st]), (i / STAGES) & 1, kWaitLimitNs)) {
+                atomicOr(&g_decode_error, 1u);
+                store_failed = true;
+            } else {
+                tma_store_2d(&tm_s, smem_u32(&sm.s[st][0][0]), v0, head * DK);
+                bulk_commit();
+            }
         }
     }
+    if (tid == 0) bulk_wait_all();  // every state tile has left shared memory and reached global
 }
 
 int sm_count() {
