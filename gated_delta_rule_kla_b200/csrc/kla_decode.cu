@@ -34,10 +34,21 @@ namespace {
 using namespace sm100;
 
 constexpr int NT = 256;
-constexpr int NV = 64;            // value columns per unit
-constexpr int CG = NV / 4;        // float4 column groups per unit (16)
-constexpr int RG = NT / CG;       // row groups (32)
-constexpr int STAGES = 3;
+#ifndef KLA_DECODE_NV
+#define KLA_DECODE_NV 64
+#endif
+#ifndef KLA_DECODE_STAGES
+#define KLA_DECODE_STAGES 3
+#endif
+#ifndef KLA_DECODE_CTAS
+#define KLA_DECODE_CTAS 2
+#endif
+constexpr int NV = KLA_DECODE_NV;         // value columns per unit
+constexpr int CG = NV / 4;                // float4 column groups per unit
+constexpr int RG = NT / CG;               // row groups
+constexpr int STAGES = KLA_DECODE_STAGES;
+constexpr int CTAS_PER_SM = KLA_DECODE_CTAS;
+static_assert(CG <= 32 && 32 % CG == 0, "column groups tile a warp");
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
 constexpr int NW = NT / 32;       // warps
@@ -64,7 +75,7 @@ struct DecodeSmem {
 };
 
 template <int DK, int DV, typename Tin, typename TOut>
-__global__ void __launch_bounds__(NT, 2)
+__global__ void __launch_bounds__(NT, CTAS_PER_SM)
     decode_step_kernel(const __grid_constant__ CUtensorMap tm_s, const Tin* __restrict__ q,
                        const Tin* __restrict__ k, const Tin* __restrict__ v, const float* __restrict__ eta,
                        const float* __restrict__ g, float eps, float* __restrict__ S, TOut* __restrict__ o,
@@ -159,11 +170,14 @@ __global__ void __launch_bounds__(NT, 2)
             pq.x = fmaf(cur[r].x, qi, pq.x); pq.y = fmaf(cur[r].y, qi, pq.y);
             pq.z = fmaf(cur[r].z, qi, pq.z); pq.w = fmaf(cur[r].w, qi, pq.w);
         }
-        // lanes c and c + 16 hold the same columns (two rows of the warp): fold them
-        pk.x += __shfl_xor_sync(0xffffffffu, pk.x, 16); pk.y += __shfl_xor_sync(0xffffffffu, pk.y, 16);
-        pk.z += __shfl_xor_sync(0xffffffffu, pk.z, 16); pk.w += __shfl_xor_sync(0xffffffffu, pk.w, 16);
-        pq.x += __shfl_xor_sync(0xffffffffu, pq.x, 16); pq.y += __shfl_xor_sync(0xffffffffu, pq.y, 16);
-        pq.z += __shfl_xor_sync(0xffffffffu, pq.z, 16); pq.w += __shfl_xor_sync(0xffffffffu, pq.w, 16);
+        // lanes c, c + CG, ... hold the same columns (several rows of the warp): fold them
+#pragma unroll
+        for (int o = CG; o < 32; o <<= 1) {
+            pk.x += __shfl_xor_sync(0xffffffffu, pk.x, o); pk.y += __shfl_xor_sync(0xffffffffu, pk.y, o);
+            pk.z += __shfl_xor_sync(0xffffffffu, pk.z, o); pk.w += __shfl_xor_sync(0xffffffffu, pk.w, o);
+            pq.x += __shfl_xor_sync(0xffffffffu, pq.x, o); pq.y += __shfl_xor_sync(0xffffffffu, pq.y, o);
+            pq.z += __shfl_xor_sync(0xffffffffu, pq.z, o); pq.w += __shfl_xor_sync(0xffffffffu, pq.w, o);
+        }
         kk = warp_sum(kk);
         kq = warp_sum(kq);
         if (lane < CG) {
@@ -275,7 +289,7 @@ cudaError_t launch_decode_t(const DecodeArgs& a, cudaStream_t st) {
         CUDA_SUCCESS)
         return cudaErrorInvalidValue;
     const int units = a.B * a.H * (DV / NV);
-    int grid = units < 2 * sm_count() ? units : 2 * sm_count();
+    int grid = units < CTAS_PER_SM * sm_count() ? units : CTAS_PER_SM * sm_count();
     if ((units + grid - 1) / grid > MAX_UNITS_PER_CTA) grid = (units + MAX_UNITS_PER_CTA - 1) / MAX_UNITS_PER_CTA;
     const size_t smem = sizeof(DecodeSmem<DK, Tin>) + 128;
     cudaError_t e = cudaFuncSetAttribute(decode_step_kernel<DK, DV, Tin, TOut>,
