@@ -512,6 +512,26 @@ def test_bwd_training_workload_sampled_heads(kla, oracle_mod):
         assert rel_err(got, ref[name]) <= 2e-2, name
 
 
+def test_bwd_long_context_sampled_heads(kla, oracle_mod):
+    """The tensor-core backward at the long-context shape (B=1, T=65536, H=16: 1024 chunks per
+    head through the reverse pass, the segmented forward recomputed inside), sampled heads
+    against the fp64 oracle."""
+    w = WORKLOADS["prefill_b1_t65536_h16_d128"]
+    inp = make_inputs(w)
+    d = {k: (v.cuda() if v is not None else None) for k, v in inp.items()}
+    dO = torch.randn(w.B, w.T, w.H, w.Dv, generator=torch.Generator().manual_seed(65)).to(torch.bfloat16)
+    gr = kla.chunk_bwd(d["q"], d["k"], d["v"], d["eta"], d["g"], dO.cuda(), w.eps, d["S0"])
+    torch.cuda.synchronize()
+    kla.check_device_error()
+    pairs = [(0, 5)]
+    args = [heads_slice(np64(inp[k]), pairs) for k in ("q", "k", "v", "eta", "g")]
+    ref = oracle_mod.backward(*args, w.eps, heads_slice(np64(inp["S0"]), pairs, state=True),
+                              heads_slice(np64(dO), pairs), None)
+    for name in GRADS:
+        got = heads_slice(np64(gr[name]), pairs, state=(name == "dS0"))
+        assert rel_err(got, ref[name]) <= 2e-2, name
+
+
 def test_bf16_outputs_are_rounded_fp32_outputs(kla):
     """out_dtype=bf16 stores round the same fp32 results once (forward, decode, backward)."""
     for Dk in (128, 64):
