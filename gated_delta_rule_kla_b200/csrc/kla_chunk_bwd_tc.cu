@@ -493,7 +493,7 @@ __global__ void __launch_bounds__(RT, 1)
 //   [0,128)   X (after the first two are read): lanes 0-63 F Khat, lanes 64-127
 //             (E + E^T) Khat + F^T Q
 // =====================================================================================
-constexpr int GT = 256;
+constexpr int GT = 512;
 constexpr uint32_t G_QK = 0, G_DOR = 32768, G_DRL = 65536, G_UH = 81920, G_UL = 98304, G_SL = 114688,
                    G_F = 180224, G_E = G_F + 64 * 65 * 4, G_MISC = G_E + 64 * 65 * 4;
 constexpr uint32_t TG_G = 0, TG_YA = 64, TG_YB = 128, TG_Z = 192, TG_L = 320, TG_X = 0;
@@ -502,10 +502,11 @@ struct GradMisc {
     uint64_t full, bar1, bar2, bar3, bar_lam;
     uint32_t tmem_base, factored;
     float G[CH], gam[CH], del[CH], ginv[CH], bco[CH], cco[CH], invr[CH], eta[CH], r2[CH], graw[CH];
-    // decay-gradient row / column sums: one slot per contributing warp, added in a fixed order
-    float rs_part[4][CH], cs_part[4][CH];
-    float rowB[CH], s_oq[CH], s_rx[CH], s_uk[CH], kd[CH], dc[CH], dr[CH], dGs[CH];
-    float red[8];
+    // per-token sums over several warps: one slot per contributing warp, added in a fixed order
+    float rs_part[8][CH], cs_part[4][CH];
+    float rowB_p[4][CH], s_oq_p[4][CH], s_rx_p[4][CH], s_uk_p[4][CH], kd_p[4][CH];
+    float kd[CH], dc[CH], dr[CH], dGs[CH];
+    float red[GT / 32];
     float lamS;
 };
 constexpr uint32_t G_SMEM = G_MISC + ((sizeof(GradMisc) + 127) / 128) * 128 + 1024;
@@ -531,16 +532,16 @@ __global__ void __launch_bounds__(GT, 1)
     const uint32_t sbase = smem_u32(sm);
     const uint32_t bar_full = smem_u32(&ms->full), bar1 = smem_u32(&ms->bar1), bar2 = smem_u32(&ms->bar2),
                    bar3 = smem_u32(&ms->bar3), bar_lam = smem_u32(&ms->bar_lam);
-    // epilogue roles: TMEM lane quadrant and column half
-    const int q4 = warp & 3, chh = warp >> 2;
+    // epilogue roles: TMEM lane quadrant and column quarter
+    const int q4 = warp & 3, cq = warp >> 2;
     const bool top = q4 < 2;
     const int ti_row = 32 * (q4 & 1) + lane;  // token of this thread's TMEM lane (both halves)
     const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
     uint32_t tmem = 0;
     bool ok = true;
-    float dkh[64];  // dkhat of token ti_row, columns [64 chh, 64 chh + 64) (lower-half threads)
-    const int pr = tid >> 4, pc = tid & 15;  // 8-feature piece pc of rows pr + 16 j
-    const int hf = tid & 1;                   // column half when building the F / E operands
+    float dkh[32];  // dkhat of token ti_row, columns [32 cq, 32 cq + 32) (lower-half threads)
+    const int pr = tid >> 4, pc = tid & 15;  // 8-feature piece pc of rows pr + 32 j
+    const int qq = tid & 3;                   // column quarter when building the F / E operands
 
     // ---- every input of the chunk requested at once: Q, K, dO by TMA; the S and U tile images
     //      and dR (fp32, into the F/E area) by bulk copies; lambda follows once Z is done
@@ -566,22 +567,15 @@ __global__ void __launch_bounds__(GT, 1)
         tmem_alloc(smem_u32(&ms->tmem_base), 512);
         tmem_relinquish();
     }
-    if (tid < CH) {
-        ms->rowB[tid] = 0.f;
-        ms->s_oq[tid] = 0.f;
-        ms->s_rx[tid] = 0.f;
-        ms->s_uk[tid] = 0.f;
-        ms->kd[tid] = 0.f;
-    }
     // Row-major [64][128] arrays are handled in 8-feature pieces: thread tid takes piece pc of
-    // rows pr + 16 j (16 consecutive threads share a row).
-    uint4 vraw[4];
+    // rows pr + 32 j (16 consecutive threads share a row).
+    uint4 vraw[2];
     {
-        uint4 kraw[4];
-        float etav[4], gv[4];
+        uint4 kraw[2];
+        float etav[2], gv[2];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int i = pr + 16 * j;
+        for (int j = 0; j < 2; ++j) {
+            const int i = pr + 32 * j;
             const bool live = i < n;
             const size_t ti = tok_index(b, t0 + (live ? i : 0), h, T, H);
             kraw[j] = live ? reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.k) + ti * DK)[pc]
@@ -592,8 +586,8 @@ __global__ void __launch_bounds__(GT, 1)
             gv[j] = live ? a.g[ti] : 0.f;
         }
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int i = pr + 16 * j;
+        for (int j = 0; j < 2; ++j) {
+            const int i = pr + 32 * j;
             float f[8];
             unpack_bf16x8(kraw[j], f);
             float r2 = 0.f;
@@ -619,8 +613,8 @@ __global__ void __launch_bounds__(GT, 1)
     {
         const float* stg = reinterpret_cast<const float*>(sm + G_F);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int i = pr + 16 * j;
+        for (int j = 0; j < 2; ++j) {
+            const int i = pr + 32 * j;
             const float4 f0 = *reinterpret_cast<const float4*>(stg + i * DV + 8 * pc);
             const float4 f1 = *reinterpret_cast<const float4*>(stg + i * DV + 8 * pc + 4);
             const float x[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
@@ -696,9 +690,9 @@ __global__ void __launch_bounds__(GT, 1)
         for (int o = 16; o > 0; o >>= 1) gr = fmaxf(gr, __shfl_xor_sync(0xffffffffu, gr, o));
         if (lane == 0) ms->factored = gr < 80.f ? 1u : 0u;
     }
-    uint4 spc[16];  // hi pieces 0-7 then lo pieces 0-7 (same element positions)
+    uint4 spc[8];  // hi pieces 0-3 then lo pieces 0-3 (same element positions)
 #pragma unroll
-    for (int j = 0; j < 16; ++j) spc[j] = reinterpret_cast<const uint4*>(sm + G_SL)[tid + 256 * j];
+    for (int j = 0; j < 8; ++j) spc[j] = reinterpret_cast<const uint4*>(sm + G_SL)[tid + GT * j];
     __syncthreads();
     if (tid < CH) {
         const float Gt = ms->G[tid];
@@ -715,58 +709,61 @@ __global__ void __launch_bounds__(GT, 1)
         bulk_load(sbase + G_SL, a.Ltl + crow * 65536, 65536, bar_lam);
     }
     // ---- Gram and Y / D epilogue: F, E to shared memory; row and column sums of the decay
-    //      gradient terms (Y o P and D o Diag(b) L), and the L part of db
+    //      gradient terms (Y o P and D o Diag(b) L), and the L part of db (16 columns a thread)
     {
         const int i = ti_row;
-        float gr[32], y[32], d2[32];
-        tmem_ld32(tmem + lane_base + TG_G + 32 * chh, gr);
-        tmem_ld32(tmem + lane_base + TG_YA + 32 * chh, y);
-        if (!top) tmem_ld32(tmem + lane_base + TG_YB + 32 * chh, d2);
+        uint32_t gru[16], yu[16], d2u[16];
+        tmem_ld16u(tmem + lane_base + TG_G + 16 * cq, gru);
+        tmem_ld16u(tmem + lane_base + TG_YA + 16 * cq, yu);
+        if (!top) tmem_ld16u(tmem + lane_base + TG_YB + 16 * cq, d2u);
         tmem_ld_wait();
         const bool fac = ms->factored != 0;
         const float Gi = ms->G[i], gi = ms->gam[i], ir = ms->invr[i], bi = ms->bco[i];
-        float rs = 0.f, rb = 0.f, dgv[32];
+        float rs = 0.f, rb = 0.f, dgv[16];
         if (top) {
             float* Fr = Fs + i * 65;
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-                const int t = 32 * chh + e;
+            for (int e = 0; e < 16; ++e) {
+                const int t = 16 * cq + e;
+                const float y = __uint_as_float(yu[e]);
                 const float gm = fac ? gi * ms->ginv[t] : __expf(Gi - ms->G[t]);
                 const float gam_it = (t <= i) ? gm : 0.f;
-                const float pm = gam_it * gr[e] * ms->invr[t];
-                Fr[t] = y[e] * gam_it;
-                dgv[e] = y[e] * pm;
+                const float pm = gam_it * __uint_as_float(gru[e]) * ms->invr[t];
+                Fr[t] = y * gam_it;
+                dgv[e] = y * pm;
                 rs += dgv[e];
             }
         } else {
             float* Er = Es + i * 65;
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-                const int t = 32 * chh + e;
+            for (int e = 0; e < 16; ++e) {
+                const int t = 16 * cq + e;
                 const float gm = fac ? gi * ms->ginv[t] : __expf(Gi - ms->G[t]);
                 const float gam_it = (t < i) ? gm : 0.f;
-                const float D = -(y[e] + d2[e]);
-                const float lh = gam_it * gr[e] * ir * ms->invr[t];
+                const float D = -(__uint_as_float(yu[e]) + __uint_as_float(d2u[e]));
+                const float lh = gam_it * __uint_as_float(gru[e]) * ir * ms->invr[t];
                 Er[t] = D * bi * gam_it;
                 dgv[e] = D * bi * lh;
                 rb = fmaf(D, lh, rb);
                 rs += dgv[e];
             }
+            ms->rowB_p[cq][i] = rb;
         }
-        ms->rs_part[2 * (top ? 0 : 1) + chh][i] = rs;
-        if (!top) atomicAdd(&ms->rowB[i], rb);
-        // column sums over this warp's 32 rows: lane l ends with column 32 chh + l
+        ms->rs_part[(top ? 0 : 4) + cq][i] = rs;
+        // column sums over this warp's 32 rows: lanes 2 m and 2 m + 1 end with column 16 cq + m
 #pragma unroll
-        for (int off = 16; off >= 1; off >>= 1) {
+        for (int off = 16; off >= 2; off >>= 1) {
             const bool up = (lane & off) != 0;
+            const int hv = off >> 1;  // values kept after this step
 #pragma unroll
-            for (int k2 = 0; k2 < off; ++k2) {
-                const float send = up ? dgv[k2] : dgv[k2 + off];
-                const float keep = up ? dgv[k2 + off] : dgv[k2];
+            for (int k2 = 0; k2 < hv; ++k2) {
+                const float send = up ? dgv[k2] : dgv[k2 + hv];
+                const float keep = up ? dgv[k2 + hv] : dgv[k2];
                 dgv[k2] = keep + __shfl_xor_sync(0xffffffffu, send, off);
             }
         }
-        ms->cs_part[q4][32 * chh + lane] = dgv[0];
+        dgv[0] += __shfl_xor_sync(0xffffffffu, dgv[0], 1);
+        if ((lane & 1) == 0) ms->cs_part[q4][16 * cq + (lane >> 1)] = dgv[0];
     }
     // ---- lambda landed: <lambda, S> from the tile pieces, then MMA group 2: [junk; U] lambda^T
     //      (A: U as the upper M half of an MN-major operand, B: lambda MN-major)
@@ -775,12 +772,12 @@ __global__ void __launch_bounds__(GT, 1)
     {
         float p = 0.f;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const uint4 lh = reinterpret_cast<const uint4*>(sm + G_SL)[tid + 256 * j];
-            const uint4 ll = reinterpret_cast<const uint4*>(sm + G_SL)[tid + 256 * (j + 8)];
+        for (int j = 0; j < 4; ++j) {
+            const uint4 lh = reinterpret_cast<const uint4*>(sm + G_SL)[tid + GT * j];
+            const uint4 ll = reinterpret_cast<const uint4*>(sm + G_SL)[tid + GT * (j + 4)];
             float a0[8], a1[8], b0[8], b1[8];
             unpack_bf16x8(spc[j], a0);
-            unpack_bf16x8(spc[j + 8], a1);
+            unpack_bf16x8(spc[j + 4], a1);
             unpack_bf16x8(lh, b0);
             unpack_bf16x8(ll, b1);
 #pragma unroll
@@ -814,26 +811,26 @@ __global__ void __launch_bounds__(GT, 1)
     ok = mbar_wait_bounded(bar2, 0, kWaitNs);
     if (__syncthreads_or(!ok)) goto done;
     {
-        const int r = tid >> 1;
-        float v1[32], v2[32];
+        const int r = tid >> 2;  // operand row; this thread's 16 tokens t = 16 qq + e
+        float v1[16], v2[16];
         if (r < CH) {
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-                const int t = 32 * hf + e;
+            for (int e = 0; e < 16; ++e) {
+                const int t = 16 * qq + e;
                 v1[e] = Fs[r * 65 + t] * ms->invr[t];
                 v2[e] = 0.f;
             }
         } else {
             const int i = r - CH;
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-                const int t = 32 * hf + e;
+            for (int e = 0; e < 16; ++e) {
+                const int t = 16 * qq + e;
                 v1[e] = (Es[i * 65 + t] + Es[t * 65 + i]) * ms->invr[t];
                 v2[e] = Fs[t * 65 + i];
             }
         }
-        st_chunks_split(sm + G_SL, sm + G_SL + 16384, r, 4 * hf, 4, v1);
-        st_chunks_split(sm + G_SL + 32768, sm + G_SL + 49152, r, 4 * hf, 4, v2);
+        st_chunks_split(sm + G_SL, sm + G_SL + 16384, r, 2 * qq, 2, v1);
+        st_chunks_split(sm + G_SL + 32768, sm + G_SL + 49152, r, 2 * qq, 2, v2);
     }
     fence_proxy_async();
     tc_fence_before();
@@ -852,7 +849,8 @@ __global__ void __launch_bounds__(GT, 1)
     ok = mbar_wait_bounded(bar3, 0, kWaitNs);
     if (__syncthreads_or(!ok)) goto done;
     tc_fence_after();
-    // ---- dq (upper lanes) and dkhat (lower lanes), with their row dot products
+    // ---- dq (upper lanes) and dkhat (lower lanes), 32 columns a thread, with their row dot
+    //      products (one slot per column quarter)
     {
         const int i = ti_row;
         const bool live = i < n;
@@ -860,54 +858,52 @@ __global__ void __launch_bounds__(GT, 1)
         const float gi = ms->gam[i];
         if (top) {
             float so = 0.f;
-            const uint8_t* qrow = sm + G_QK + chh * 16384;
-#pragma unroll 1
-            for (int p = 0; p < 2; ++p) {
-                float z[32], x[32];
-                tmem_ld32(tmem + lane_base + TG_Z + 64 * chh + 32 * p, z);
-                tmem_ld32(tmem + lane_base + TG_X + 64 * chh + 32 * p, x);
-                tmem_ld_wait();
+            const uint8_t* qrow = sm + G_QK + (cq >> 1) * 16384;
+            float z[32], x[32];
+            tmem_ld32(tmem + lane_base + TG_Z + 32 * cq, z);
+            tmem_ld32(tmem + lane_base + TG_X + 32 * cq, x);
+            tmem_ld_wait();
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    float f[8];
-                    ld_sw128_chunk(qrow, i, 4 * p + u, f);
+            for (int u = 0; u < 4; ++u) {
+                float f[8];
+                ld_sw128_chunk(qrow, i, 4 * (cq & 1) + u, f);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) so = fmaf(f[e], z[8 * u + e], so);
-                }
-#pragma unroll
-                for (int e = 0; e < 32; ++e) x[e] = fmaf(gi, z[e], x[e]);
-                if (live) st_row32<TOut>(static_cast<TOut*>(a.dq) + ti * DK + 64 * chh + 32 * p, x);
+                for (int e = 0; e < 8; ++e) so = fmaf(f[e], z[8 * u + e], so);
             }
-            atomicAdd(&ms->s_oq[i], so);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) x[e] = fmaf(gi, z[e], x[e]);
+            if (live) st_row32<TOut>(static_cast<TOut*>(a.dq) + ti * DK + 32 * cq, x);
+            ms->s_oq_p[cq][i] = so;
         } else {
             float srx = 0.f, suk = 0.f, kdp = 0.f;
             const float nbg = -ms->bco[i] * gi, de = ms->del[i];
-            const uint8_t* krow = sm + G_QK + chh * 16384 + 8192;
+            const uint8_t* krow = sm + G_QK + (cq >> 1) * 16384 + 8192;
 #pragma unroll
-            for (int p = 0; p < 2; ++p) {
-                float z[32], l[32], x[32];
-                tmem_ld32(tmem + lane_base + TG_Z + 64 * chh + 32 * p, z);
-                tmem_ld32(tmem + lane_base + TG_L + 64 * chh + 32 * p, l);
-                tmem_ld32(tmem + lane_base + TG_X + 64 * chh + 32 * p, x);
+            for (int p = 0; p < 2; ++p) {  // 16 columns at a time (register pressure)
+                uint32_t zu[16], lu[16], xu[16];
+                tmem_ld16u(tmem + lane_base + TG_Z + 32 * cq + 16 * p, zu);
+                tmem_ld16u(tmem + lane_base + TG_L + 32 * cq + 16 * p, lu);
+                tmem_ld16u(tmem + lane_base + TG_X + 32 * cq + 16 * p, xu);
                 tmem_ld_wait();
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
+                for (int u = 0; u < 2; ++u) {
                     float f[8];
-                    ld_sw128_chunk(krow, i, 4 * p + u, f);
+                    ld_sw128_chunk(krow, i, 4 * (cq & 1) + 2 * p + u, f);
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
                         const int k2 = 8 * u + e;
-                        const float d = fmaf(de, l[k2], fmaf(nbg, z[k2], x[k2]));
-                        dkh[32 * p + k2] = d;
-                        srx = fmaf(f[e], z[k2], srx);
-                        suk = fmaf(f[e], l[k2], suk);
+                        const float z = __uint_as_float(zu[k2]), l = __uint_as_float(lu[k2]);
+                        const float d = fmaf(de, l, fmaf(nbg, z, __uint_as_float(xu[k2])));
+                        dkh[16 * p + k2] = d;
+                        srx = fmaf(f[e], z, srx);
+                        suk = fmaf(f[e], l, suk);
                         kdp = fmaf(f[e], d, kdp);
                     }
                 }
             }
-            atomicAdd(&ms->s_rx[i], srx);
-            atomicAdd(&ms->s_uk[i], suk);
-            atomicAdd(&ms->kd[i], kdp);
+            ms->s_rx_p[cq][i] = srx;
+            ms->s_uk_p[cq][i] = suk;
+            ms->kd_p[cq][i] = kdp;
         }
     }
     __syncthreads();
@@ -915,11 +911,13 @@ __global__ void __launch_bounds__(GT, 1)
     if (tid < CH) {
         const int i = tid;
         const float ir = ms->invr[i], gi = ms->gam[i], bi = ms->bco[i], de = ms->del[i];
-        const float srx = ms->s_rx[i] * ir, suk = ms->s_uk[i] * ir, soq = ms->s_oq[i];
-        const float db = ms->rowB[i] - gi * srx;
+        auto sum4 = [&](const float (*v)[CH]) { return (v[0][i] + v[1][i]) + (v[2][i] + v[3][i]); };
+        const float srx = sum4(ms->s_rx_p) * ir, suk = sum4(ms->s_uk_p) * ir, soq = sum4(ms->s_oq_p);
+        const float db = sum4(ms->rowB_p) - gi * srx;
         const float dc = ms->dc[i];
-        const float rsum = (ms->rs_part[0][i] + ms->rs_part[1][i]) + (ms->rs_part[2][i] + ms->rs_part[3][i]);
-        const float csum = (ms->cs_part[0][i] + ms->cs_part[1][i]) + (ms->cs_part[2][i] + ms->cs_part[3][i]);
+        const float rsum = ((ms->rs_part[0][i] + ms->rs_part[1][i]) + (ms->rs_part[2][i] + ms->rs_part[3][i])) +
+                           ((ms->rs_part[4][i] + ms->rs_part[5][i]) + (ms->rs_part[6][i] + ms->rs_part[7][i]));
+        const float csum = sum4(ms->cs_part);
         ms->dGs[i] = gi * (soq - bi * srx) - de * suk + rsum - csum;
         float extra = warp_sum(de * suk);  // delta_i = gamma_last / gamma_i feeds dG of the last token
         if (lane == 0) ms->red[warp] = extra;
@@ -931,7 +929,7 @@ __global__ void __launch_bounds__(GT, 1)
             dr = (db * et * 2.f * r * a.eps + dc * et * (a.eps - r2)) / (den * den);
         }
         ms->dr[i] = dr;
-        ms->kd[i] *= ir;
+        ms->kd[i] = sum4(ms->kd_p) * ir;
         if (i < n) a.deta[tok_index(b, t0 + i, h, T, H)] = deta;
     }
     __syncthreads();
@@ -957,22 +955,19 @@ __global__ void __launch_bounds__(GT, 1)
         if (i < n) {
             const size_t ti = tok_index(b, t0 + i, h, T, H);
             const float ir = ms->invr[i], kd = ms->kd[i], dr = ms->dr[i];
-            const uint8_t* krow = sm + G_QK + chh * 16384 + 8192;
+            const uint8_t* krow = sm + G_QK + (cq >> 1) * 16384 + 8192;
+            float x[32];
 #pragma unroll
-            for (int p = 0; p < 2; ++p) {
-                float x[32];
+            for (int u = 0; u < 4; ++u) {
+                float f[8];
+                ld_sw128_chunk(krow, i, 4 * (cq & 1) + u, f);
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    float f[8];
-                    ld_sw128_chunk(krow, i, 4 * p + u, f);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const float kh = f[e] * ir;
-                        x[8 * u + e] = ir > 0.f ? fmaf(dkh[32 * p + 8 * u + e] - kh * kd, ir, kh * dr) : 0.f;
-                    }
+                for (int e = 0; e < 8; ++e) {
+                    const float kh = f[e] * ir;
+                    x[8 * u + e] = ir > 0.f ? fmaf(dkh[8 * u + e] - kh * kd, ir, kh * dr) : 0.f;
                 }
-                st_row32<TOut>(static_cast<TOut*>(a.dk) + ti * DK + 64 * chh + 32 * p, x);
             }
+            st_row32<TOut>(static_cast<TOut*>(a.dk) + ti * DK + 32 * cq, x);
         }
     }
 done:
