@@ -6,7 +6,7 @@
 // Diag(b gamma) Khat S) and lambda = dS' the gradient of the chunk's outgoing state:
 //   dU      = P^T dO + Ktil lambda,       dR = T^T dU
 //   dS      = gamma_last lambda + (Diag(gamma) Q)^T dO - W^T dU      (W^T dU = (b gamma Khat)^T dR)
-// so the reverse state recurrence needs only the forward's preparation records (P, Ktil, -W^T)
+// so the reverse state recurrence needs only the forward's preparation records (P, Ktil, -W)
 // and the chunk's dO and Q.  Then, for every chunk independently,
 //   Y = dO U^T,  D = -dR U^T,   F = Gam o Y (lower),  E = Diag(b) (Gam^- o D) (strictly lower)
 //   dq    = Diag(gamma) dO S^T + F Khat
@@ -136,7 +136,7 @@ constexpr uint32_t SR_DO = 0, SR_Q = 16384, SR_W = 32768, SR_KT = 49152, SR_KTLO
                    SR_T = 98304;
 static_assert(SR_KT - SR_W == REC_KT - REC_W && SR_KTLO - SR_W == REC_KTLO - REC_W && SR_P - SR_W == REC_P - REC_W &&
                   REC_P + 16384 - REC_W == 65536,
-              "the record's -W^T, Ktil and P tiles arrive as one 64 KB copy");
+              "the record's -W, Ktil and P tiles arrive as one 64 KB copy");
 static_assert(SR_T + 16384 == R_STAGE, "stage size");
 constexpr uint32_t R_SC = 2 * R_STAGE;
 constexpr uint32_t R_MISC = R_SC + 2 * REC_SCB;
@@ -254,7 +254,7 @@ __global__ void __launch_bounds__(RT, 1)
             const uint32_t i_dop = idesc_bf16(128, 64, true, true);   // dO^T (MN-major) x P (MN-major)
             const uint32_t i_lk = idesc_bf16(128, 64, false, false);  // lambda^T x Ktil^T (K-major)
             const uint32_t i_q = idesc_bf16(128, 128, false, true);   // (gamma dO)^T x Q (MN-major)
-            const uint32_t i_w = idesc_bf16(128, 128, false, false);  // dU^T x (-W) (K-major)
+            const uint32_t i_w = idesc_bf16(128, 128, false, true);   // dU^T x (-W) ([token][dk] tiles: MN-major)
             const uint32_t i_t = idesc_bf16(128, 64, false, true);    // dU^T x T (MN-major)
             for (int lc = 0; lc < NC && !aborted; ++lc) {
                 const int st = lc & 1;
@@ -308,7 +308,7 @@ __global__ void __launch_bounds__(RT, 1)
                         for (int j = 0; j < 2; ++j) {
                             const int s = half + 2 * j;
                             mma_bf16_ts(tmem + TR_L, tmem + (p ? TR_UL : TR_UH) + 8 * s,
-                                        smem_desc(stg + SR_W + s * 32, 16, 1024), i_w, 1);
+                                        smem_desc(stg + SR_W + s * 2048, 8192, 1024), i_w, 1);
                         }
                 }
                 if (aborted) break;

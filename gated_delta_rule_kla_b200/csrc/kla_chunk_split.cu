@@ -313,13 +313,15 @@ __global__ void __launch_bounds__(PT, 3)
     }
     tc_fence_after();
     {
-        // ---- -W^T (thread = dk row, 32 tokens), U' as [token][dv] rows, Ktil hi/lo: all to the record
+        // ---- -W (thread = dk column, 32 tokens) transposed to [token][dk] tiles over the consumed
+        //      V tile, then one bulk copy to the record; U' as [token][dv] rows and Ktil hi/lo
+        //      straight to the record
         float x[32];
         tmem_ld32(tmem + lane_base + PM_W + 32 * ch, x);
         tmem_ld_wait();
 #pragma unroll
         for (int e = 0; e < 32; ++e) x[e] = -x[e];
-        st_chunks_bf16_global(rec + REC_W, row, 4 * ch, 4, x);
+        st_w_tokens_smem(sm + P_V, row, 32 * ch, x, tid & 31);
         tmem_ld32(tmem + lane_base + PM_U + 32 * ch, x);
         tmem_ld_wait();
         float* up = reinterpret_cast<float*>(rec + REC_UP);
@@ -345,6 +347,13 @@ __global__ void __launch_bounds__(PT, 3)
             st_pair_sw128_global(rec + REC_KT + blk * 8192, j, c, h0, h1);
             st_pair_sw128_global(rec + REC_KTLO + blk * 8192, j, c, l0, l1);
         }
+        fence_proxy_async();
+        __syncthreads();
+        if (tid == 0) {
+            bulk_store(rec + REC_W, sbase + P_V, 16384);
+            bulk_commit();
+            bulk_wait_read();
+        }
     }
 done:
     tc_fence_before();
@@ -362,37 +371,43 @@ done:
 // out.  They meet on mbarriers:
 //   issuer -> epilogue: bar_u (U^T ready in TMEM), bar_s (S^T updated), bar_o (O1, O2 ready)
 //   epilogue -> issuer: s_ready[2], u_ready[2] (each half of the S, U operands written),
-//                       o_free (O read and the o tile staged)
+//                       o_read (O1 and O2 read out of TMEM)
+//   epilogue -> loader: o_free (the o tile staged)
 // bar_o and o_free, which the loader also waits on, come one per stage: a phase of either
 // cannot come round again before the loader has refilled that stage, so the loader's parity
 // waits never alias even when it runs late.
 // An MMA issue blocks its thread while the tensor pipe drains, so no epilogue work sits on the
 // issuing warp; and the S and U operands are released in halves, so the first K steps of the
 // MMA that consumes them run while the epilogue finishes the second half.  Per chunk c:
-//   issuer    U(c) [2 halves] | O1(c) | S(c) [2 halves] O2(c)
+//   issuer    [U | O1 hi](c) [2 halves] | O1 lo(c) | S(c) [2 halves] O2(c)
 //   epilogue  U epi(c) -> S hi/lo(c+1) -> master rescale -> O epi(c)
-//   loader    refill of chunk c's stage with chunk c + 2 (Ktil, P, U' once chunk c's MMAs are
-//             done; Q, W and scalars once the o tile has left by TMA store)
+//   loader    refill of chunk c's stage with chunk c + 2 (part A: -W, Q, P, U' once chunk c's
+//             MMAs are done; part B: Ktil and scalars once the o tile has left by TMA store)
 // =====================================================================================
 constexpr int ST = 320;
 constexpr int kIssuerWarp = 8, kLoaderWarp = 9;
 constexpr uint32_t S_STAGE = 114688;  // Q 16 KB + the record's tiles (96 KB)
-constexpr uint32_t SO_Q = 0, SO_W = 16384, SO_KT = 32768, SO_KTLO = 49152, SO_P = 65536, SO_PLO = 73728,
-                   SO_UP = 81920;
-static_assert(SO_W == REC_W + 16384 && SO_KT == REC_KT + 16384 && SO_KTLO == REC_KTLO + 16384 &&
-                  SO_P == REC_P + 16384 && SO_UP == REC_UP + 16384,
+// SO_WQ: [-W block 0 | Q block 0 | -W block 1 | Q block 1], 8 KB each ([64 tokens x 64 dk]),
+// so that one K-major descriptor over 128 rows reads -W then Q for the same 16 dk: the U and
+// O1 products share their A operand (S^T) and run as N = 128 MMAs.  The o tile is staged over
+// Ktil (32 KB) once the chunk's MMAs are done.
+constexpr uint32_t SO_WQ = 0, SO_KT = 32768, SO_KTLO = 49152, SO_P = 65536, SO_PLO = 73728, SO_UP = 81920;
+static_assert(SO_KT == REC_KT + 16384 && SO_KTLO == REC_KTLO + 16384 && SO_P == REC_P + 16384 &&
+                  SO_UP == REC_UP + 16384,
               "stage mirrors the record");
-static_assert(S_STAGE - SO_KT == 32768 + 16384 + 32768, "early part: Ktil, P, U'");
+static_assert(S_STAGE - SO_KT == 32768 + 16384 + 32768, "Ktil, P, U' fill the rest of the stage");
 constexpr uint32_t S_SC = 2 * S_STAGE;  // 2 x 512 B record scalars
 constexpr uint32_t S_MISC = S_SC + 2 * REC_SCB;
 constexpr uint32_t S_SMEM = S_MISC + 128 + 1024;
-constexpr uint32_t TM_S = 0, TM_SH = 128, TM_SL = 192, TM_U = 256, TM_UH = 320, TM_UL = 352, TM_O1 = 384,
+constexpr uint32_t TM_S = 0, TM_SH = 128, TM_SL = 192, TM_U = 256, TM_O1 = 320, TM_UH = 384, TM_UL = 416,
                    TM_O2 = 448;
+static_assert(TM_O1 == TM_U + 64, "U and O1 are one N = 128 accumulator");
 
 struct StateMisc {
-    uint64_t full[2];
+    uint64_t full_a[2], full_b[2];                // the two parts of each stage (TMA / bulk bytes)
     uint64_t bar_u, bar_s, bar_o[2];              // tcgen05.commit arrivals (bar_o per stage)
     uint64_t s_ready[2], u_ready[2], o_free[2];   // one arrival per epilogue warp (o_free per stage)
+    uint64_t o_read;                              // O1 and O2 read out of TMEM (one arrival per warp)
     uint32_t tmem_base, abort;
     float gsum[2];
 };
@@ -427,10 +442,10 @@ __global__ void __launch_bounds__(ST, 1)
     const int c0 = seg * segc, c1 = min(NCtot, c0 + segc);
     const int NC = c1 > c0 ? c1 - c0 : 0;
     const uint32_t sbase = smem_u32(sm);
-    const uint32_t bar_full0 = smem_u32(&ms->full[0]);
+    const uint32_t full_a0 = smem_u32(&ms->full_a[0]), full_b0 = smem_u32(&ms->full_b[0]);
     const uint32_t bar_u = smem_u32(&ms->bar_u), bar_s = smem_u32(&ms->bar_s), bar_o0 = smem_u32(&ms->bar_o[0]);
     const uint32_t s_ready0 = smem_u32(&ms->s_ready[0]), u_ready0 = smem_u32(&ms->u_ready[0]),
-                   o_free0 = smem_u32(&ms->o_free[0]);
+                   o_free0 = smem_u32(&ms->o_free[0]), o_read = smem_u32(&ms->o_read);
     const float* S0p = (a.S0 && !ident)
                            ? a.S0 + (size_t)(segmented ? head_idx * nseg + seg : head_idx) * DK * DV
                            : nullptr;
@@ -446,8 +461,10 @@ __global__ void __launch_bounds__(ST, 1)
     const bool need_vals = !ident;
 
     if (tid == 0) {
-        mbar_init(bar_full0, 1);
-        mbar_init(bar_full0 + 8, 1);
+        mbar_init(full_a0, 1);
+        mbar_init(full_a0 + 8, 1);
+        mbar_init(full_b0, 1);
+        mbar_init(full_b0 + 8, 1);
         mbar_init(bar_u, 1);
         mbar_init(bar_s, 1);
         mbar_init(bar_o0, 1);
@@ -458,6 +475,7 @@ __global__ void __launch_bounds__(ST, 1)
         mbar_init(u_ready0 + 8, 8);
         mbar_init(o_free0, 8);
         mbar_init(o_free0 + 8, 8);
+        mbar_init(o_read, 8);
         ms->abort = 0;
         fence_mbar_init();
     }
@@ -483,68 +501,71 @@ __global__ void __launch_bounds__(ST, 1)
         if (lane == 0) {
             prefetch_tmap(&tm_q);
             if (write_o) prefetch_tmap(&tm_o);
-            // The early part (Ktil, P, U') and the late part (Q, W, scalars) of chunk c; the
-            // late part carries the phase's one arrival.
-            const uint32_t early_bytes = 32768 + (write_o ? 16384 : 0) + (need_vals ? 32768 : 0);
-            const uint32_t late_bytes = 16384 + REC_SCB + (write_o ? 16384 : 0);
-            auto load_early = [&](int c, int st) {
-                const uint32_t bar = bar_full0 + 8 * st;
+            // Part A of chunk c (-W, Q, P, U': the operands of its first products) can land as soon
+            // as chunk c - 2's MMAs are done; part B (Ktil, needed from the S product on, and the
+            // scalars, read by the epilogues up to chunk c - 2's o tile) only after that tile,
+            // staged over Ktil, has left by TMA store.
+            const uint32_t a_bytes = 16384 + (write_o ? 32768 : 0) + (need_vals ? 32768 : 0);
+            const uint32_t b_bytes = 32768 + REC_SCB;
+            auto load_a = [&](int c, int st) {
+                const uint32_t bar = full_a0 + 8 * st;
                 const uint32_t base = sbase + st * S_STAGE;
                 const uint8_t* rec = recs + ((size_t)head_idx * NCtot + c) * REC_BYTES;
-                mbar_expect_tx_only(bar, early_bytes);
-                bulk_load(base + SO_KT, rec + REC_KT, 16384, bar);
-                bulk_load(base + SO_KTLO, rec + REC_KTLO, 16384, bar);
-                if (write_o) bulk_load(base + SO_P, rec + REC_P, 16384, bar);
+                mbar_expect_tx(bar, a_bytes);
+                bulk_load(base + SO_WQ, rec + REC_W, 8192, bar);
+                bulk_load(base + SO_WQ + 16384, rec + REC_W + 8192, 8192, bar);
+                if (write_o) {
+                    tma_load_4d(base + SO_WQ + 8192, &tm_q, bar, 0, h, c * CH, b);
+                    tma_load_4d(base + SO_WQ + 24576, &tm_q, bar, 64, h, c * CH, b);
+                    bulk_load(base + SO_P, rec + REC_P, 16384, bar);
+                }
                 if (need_vals) {
                     bulk_load(base + SO_UP, rec + REC_UP, 16384, bar);
                     bulk_load(base + SO_UP + 16384, rec + REC_UP + 16384, 16384, bar);
                 }
             };
-            auto load_late = [&](int c, int st) {
-                const uint32_t bar = bar_full0 + 8 * st;
+            auto load_b = [&](int c, int st) {
+                const uint32_t bar = full_b0 + 8 * st;
                 const uint32_t base = sbase + st * S_STAGE;
                 const uint8_t* rec = recs + ((size_t)head_idx * NCtot + c) * REC_BYTES;
-                mbar_expect_tx(bar, late_bytes);
-                if (write_o) {
-                    tma_load_4d(base + SO_Q, &tm_q, bar, 0, h, c * CH, b);
-                    tma_load_4d(base + SO_Q + 8192, &tm_q, bar, 64, h, c * CH, b);
-                }
-                bulk_load(base + SO_W, rec + REC_W, 16384, bar);
+                mbar_expect_tx(bar, b_bytes);
+                bulk_load(base + SO_KT, rec + REC_KT, 16384, bar);
+                bulk_load(base + SO_KTLO, rec + REC_KTLO, 16384, bar);
                 bulk_load(sbase + S_SC + st * REC_SCB, rec + REC_SC, REC_SCB, bar);
             };
-            int early = c0 - 1, late = c0 - 1;  // last chunk of each part requested
+            int last_a = c0 - 1, last_b = c0 - 1;  // last chunk of each part requested
             for (int i = 0; i < min(NC, 2); ++i) {
-                load_early(c0 + i, i);
-                load_late(c0 + i, i);
-                early = late = c0 + i;
+                load_a(c0 + i, i);
+                load_b(c0 + i, i);
+                last_a = last_b = c0 + i;
             }
             for (int c = c0; c < c1; ++c) {
                 const int lc = c - c0, st = lc & 1;
-                // every MMA of chunk c done: Ktil, P, U' of its stage can take chunk c + 2
+                // every MMA of chunk c done: part A of its stage can take chunk c + 2
                 if (!mbar_wait_bounded(bar_o0 + 8 * st, (lc >> 1) & 1, kWaitNs)) { aborted = true; break; }
                 if (c + 2 < c1) {
-                    load_early(c + 2, st);
-                    early = c + 2;
+                    load_a(c + 2, st);
+                    last_a = c + 2;
                 }
-                // o tile staged and every scalar read: store it, then the rest of the stage
+                // o tile staged and every scalar read: store it, then part B
                 if (!mbar_wait_bounded(o_free0 + 8 * st, (lc >> 1) & 1, kWaitNs)) { aborted = true; break; }
                 if (write_o) {
-                    tma_store_4d(&tm_o, sbase + st * S_STAGE + SO_Q, 0, h, c * CH, b);
+                    tma_store_4d(&tm_o, sbase + st * S_STAGE + SO_KT, 0, h, c * CH, b);
                     bulk_commit();
                     bulk_wait_read();
                 }
                 if (c + 2 < c1) {
-                    load_late(c + 2, st);
-                    late = c + 2;
+                    load_b(c + 2, st);
+                    last_b = c + 2;
                 }
             }
             if (aborted) {
                 atomicOr(&ms->abort, 1u);
-                // let loads that may still be landing in shared memory finish (a phase whose late
-                // part was never requested cannot complete: wait out its early bytes instead)
-                for (int cc = max(c0, late - 1); cc <= early; ++cc)
-                    (void)mbar_wait_bounded(bar_full0 + 8 * ((cc - c0) & 1), ((cc - c0) >> 1) & 1,
-                                            cc <= late ? kWaitNs : 20000000ull);
+                // let loads that may still be landing in shared memory finish
+                for (int cc = max(c0, last_a - 1); cc <= last_a; ++cc)
+                    (void)mbar_wait_bounded(full_a0 + 8 * ((cc - c0) & 1), ((cc - c0) >> 1) & 1, kWaitNs);
+                for (int cc = max(c0, last_b - 1); cc <= last_b; ++cc)
+                    (void)mbar_wait_bounded(full_b0 + 8 * ((cc - c0) & 1), ((cc - c0) >> 1) & 1, kWaitNs);
             }
             bulk_wait_all();
         }
@@ -552,51 +573,52 @@ __global__ void __launch_bounds__(ST, 1)
     } else if (warp == kIssuerWarp) {
         // ================================ MMA issuer ================================
         if (lane == 0) {
-            const uint32_t iu = idesc_bf16(128, 64, false, true);
+            const uint32_t iu = idesc_bf16(128, 64, false, false);
+            const uint32_t iuo = idesc_bf16(128, 128, false, false);
             const uint32_t io = idesc_bf16(128, 64, false, false);
             const uint32_t is = idesc_bf16(128, 128, false, true);
             for (int c = c0; c < c1 && !aborted; ++c) {
                 const int lc = c - c0, st = lc & 1;
                 const uint32_t stg = sbase + st * S_STAGE;
-                if (!mbar_wait_bounded(bar_full0 + 8 * st, (lc >> 1) & 1, kWaitNs)) { aborted = true; break; }
-                // U^T = -(S^T W^T) (the record holds -W^T; U' is added in the epilogue).  K steps
-                // {0,1,4,5} read the first half of each thread's S columns, {2,3,6,7} the second.
-                // S enters as its bf16 hi part only: W is itself one bf16 rounding, and the lo
-                // part's share is below that (measured: max|err|/rms of o and S_T 3.3e-3 against
-                // 2.7e-3 with both parts, over the headline workload and the stress cases).
+                if (!mbar_wait_bounded(full_a0 + 8 * st, (lc >> 1) & 1, kWaitNs)) { aborted = true; break; }
+                // [U^T | O1] = S^T [-W^T | Q^T] (N = 128; the record holds -W, U' is added in the
+                // epilogue), once the previous chunk's O1 and O2 are read.  K steps {0,1,4,5} read
+                // the first half of each thread's S columns, {2,3,6,7} the second.  U takes S as its
+                // bf16 hi part only: W is itself one bf16 rounding, and the lo part's share is
+                // below that (measured: max|err|/rms of o and S_T 3.3e-3 against 2.7e-3 with both
+                // parts, over the headline workload and the stress cases); O1 adds S lo x Q^T below.
+                // Without outputs the MMAs are U's alone (N = 64).
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
                     if (!mbar_wait_bounded(s_ready0 + 8 * half, lc & 1, kWaitNs)) { aborted = true; break; }
-                    tc_fence_after();
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const int s = 2 * half + (j & 1) + 4 * (j >> 1);
-                        mma_bf16_ts(tmem + TM_U, tmem + TM_SH + 8 * s, smem_desc(stg + SO_W + s * 2048, 8192, 1024),
-                                    iu, (half | j) > 0);
-                    }
-                }
-                if (aborted) break;
-                mma_commit(bar_u);
-                // O1 = S^T Q^T, once the previous chunk's outputs are read
-                if (write_o) {
-                    if (lc > 0 && !mbar_wait_bounded(o_free0 + 8 * (st ^ 1), ((lc - 1) >> 1) & 1, kWaitNs)) {
+                    if (half == 0 && write_o && lc > 0 && !mbar_wait_bounded(o_read, (lc - 1) & 1, kWaitNs)) {
                         aborted = true;
                         break;
                     }
                     tc_fence_after();
 #pragma unroll
-                    for (int part = 0; part < 2; ++part)
+                    for (int j = 0; j < 4; ++j) {
+                        const int s = 2 * half + (j & 1) + 4 * (j >> 1);
+                        mma_bf16_ts(tmem + TM_U, tmem + TM_SH + 8 * s,
+                                    smem_desc(stg + SO_WQ + (s >> 2) * 16384 + (s & 3) * 32, 16, 1024),
+                                    write_o ? iuo : iu, (half | j) > 0);
+                    }
+                }
+                if (aborted) break;
+                mma_commit(bar_u);
+                // O1 += S^T lo Q^T
+                if (write_o) {
 #pragma unroll
-                        for (int s = 0; s < 8; ++s)
-                            mma_bf16_ts(tmem + TM_O1, tmem + (part ? TM_SL : TM_SH) + 8 * s,
-                                        smem_desc(stg + SO_Q + (s >> 2) * 8192 + (s & 3) * 32, 16, 1024), io,
-                                        (part | s) > 0);
+                    for (int s = 0; s < 8; ++s)
+                        mma_bf16_ts(tmem + TM_O1, tmem + TM_SL + 8 * s,
+                                    smem_desc(stg + SO_WQ + 8192 + (s >> 2) * 16384 + (s & 3) * 32, 16, 1024), io, 1);
                 }
                 // S^T += U^T Ktil (N = 128): K steps {0,2} (first half of each thread's tokens),
                 // then {1,3}; products hi x hi, hi x lo, lo x hi
                 const uint32_t ua[3] = {TM_UH, TM_UH, TM_UL};
                 const uint32_t kb[3] = {stg + SO_KT, stg + SO_KTLO, stg + SO_KT};
                 const uint32_t pb[3] = {stg + SO_P, stg + SO_PLO, stg + SO_P};
+                if (!mbar_wait_bounded(full_b0 + 8 * st, (lc >> 1) & 1, kWaitNs)) { aborted = true; break; }
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
                     if (!mbar_wait_bounded(u_ready0 + 8 * half, lc & 1, kWaitNs)) { aborted = true; break; }
@@ -742,11 +764,12 @@ __global__ void __launch_bounds__(ST, 1)
                 tc_fence_after();
                 if (write_o) {
                     const float* gm = reinterpret_cast<const float*>(sm + S_SC + st * REC_SCB);
-                    TOut* stage_o = reinterpret_cast<TOut*>(sm + st * S_STAGE + SO_Q);
+                    TOut* stage_o = reinterpret_cast<TOut*>(sm + st * S_STAGE + SO_KT);
                     float o1[32], o2[32];
                     tmem_ld32(tmem + lane_base + TM_O1 + 32 * ch, o1);
                     tmem_ld32(tmem + lane_base + TM_O2 + 32 * ch, o2);
                     tmem_ld_wait();
+                    epi_signal(o_read, tid);  // the next chunk's [U | O1] product may start
 #pragma unroll
                     for (int e = 0; e < 32; ++e) {
                         const int t = 32 * ch + e;

@@ -268,6 +268,25 @@ __device__ __forceinline__ void st_chunks_bf16_global(uint8_t* block, int r, int
     }
 }
 
+// Write 32 tokens of one dk column, v[e] at token t0 + e, into a [64 tokens x 64 dk] x 2
+// swizzled bf16 tile pair in shared memory (block dk / 64), from a warp whose consecutive
+// lanes hold consecutive dk.  Lane pairs (dk even, dk + 1) trade values so that each lane
+// writes whole 32-bit words (two dk of one token): of each token pair (t, t + 4) the even
+// lane writes t and the odd lane t + 4, whose swizzled 64-byte runs use the other 16 banks.
+__device__ __forceinline__ void st_w_tokens_smem(uint8_t* base, int dk, int t0, const float* v, int lane) {
+    const int odd = lane & 1, dk0 = dk & ~1;
+    uint8_t* blk = base + (dk0 >> 6) * 8192;
+    const int col = dk0 & 63;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const int e0 = (i & 3) + 8 * (i >> 2);  // 0..3, 8..11, 16..19, 24..27
+        const float other = __shfl_xor_sync(0xffffffffu, odd ? v[e0] : v[e0 + 4], 1);
+        const uint32_t w = odd ? pack_bf16x2(other, v[e0 + 4]) : pack_bf16x2(v[e0], other);
+        const int t = t0 + e0 + 4 * odd;
+        *reinterpret_cast<uint32_t*>(blk + t * 128 + (((col >> 3) ^ (t & 7)) << 4) + (col & 7) * 2) = w;
+    }
+}
+
 // Write chunks [c0, c0 + n) of row r of a swizzled bf16 block from 8*n fp32 values.
 __device__ __forceinline__ void st_chunks_bf16(uint8_t* block, int r, int c0, int n, const float* v) {
 #pragma unroll
@@ -302,7 +321,7 @@ __device__ __forceinline__ void st_chunks_split(uint8_t* hi_block, uint8_t* lo_b
 
 // ---- per-chunk record of the split forward's preparation kernel (byte offsets in the
 //      workspace); tiles use the 128-byte swizzle
-constexpr uint32_t REC_W = 0;        // -W^T bf16: 128 dk rows x 64 tokens          16 KB
+constexpr uint32_t REC_W = 0;        // -W bf16: [64 tokens x 64 dk] x 2 blocks         16 KB
 constexpr uint32_t REC_KT = 16384;   // Ktil hi: [64 tokens x 64 dk] x 2 blocks        16 KB
 constexpr uint32_t REC_KTLO = 32768; // Ktil lo                                        16 KB
 constexpr uint32_t REC_P = 49152;    // P hi [64 x 64], then P lo                       16 KB
