@@ -171,6 +171,97 @@ __device__ __forceinline__ void inverse_join_level(float* Lf, float* X, int tid)
     __syncthreads();
 }
 
+// Join levels 16 and 32 with the triangles' zeros skipped.  The same sums as
+// inverse_join_level, term for term and in the same order (only products with a structural
+// zero factor are left out, so the results are bit-identical), with warp-uniform trip counts:
+// phase 1 (X = L_BA T_A, T_A[k][j] = 0 for k < j) gives each warp a group of columns j0.. and
+// runs k from j0; phase 2 (T_BA = -T_B X, T_B[i][k] = 0 for k > i) gives each warp a group of
+// rows and stops after the group's last row.  Operand rows are read as float4 (k four at a
+// time; every bound is a multiple of 4).  256 threads.
+__device__ __forceinline__ void inverse_join32_tri(float* Lf, float* X, int tid) {
+    const int w = tid >> 5, lane = tid & 31;
+    {  // warp w: columns 4w .. 4w + 3 of X, lane: row i
+        const int i = lane, j0 = 4 * w;
+        const float* lrow = Lf + (32 + i) * LDL;
+        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+        for (int k = j0; k < 32; k += 4) {
+            const float4 l4 = *reinterpret_cast<const float4*>(lrow + k);
+            const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const float4 t = *reinterpret_cast<const float4*>(Lf + (k + u) * LDL + j0);
+                a0 = fmaf(lv[u], t.x, a0);
+                a1 = fmaf(lv[u], t.y, a1);
+                a2 = fmaf(lv[u], t.z, a2);
+                a3 = fmaf(lv[u], t.w, a3);
+            }
+        }
+        *reinterpret_cast<float4*>(X + i * 32 + j0) = make_float4(a0, a1, a2, a3);
+    }
+    __syncthreads();
+    {  // warp w: rows 4w .. 4w + 3 of T_BA, lane: column j
+        const int j = lane, i0 = 4 * w;
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int k = 0; k < i0 + 4; k += 4) {
+            float tb[4][4];
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                const float4 t = *reinterpret_cast<const float4*>(Lf + (32 + i0 + r) * LDL + 32 + k);
+                tb[r][0] = t.x; tb[r][1] = t.y; tb[r][2] = t.z; tb[r][3] = t.w;
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const float x = X[(k + u) * 32 + j];
+#pragma unroll
+                for (int r = 0; r < 4; ++r) acc[r] = fmaf(tb[r][u], x, acc[r]);
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < 4; ++r) Lf[(32 + i0 + r) * LDL + j] = -acc[r];
+    }
+    __syncthreads();
+}
+
+__device__ __forceinline__ void inverse_join16_tri(float* Lf, float* X, int tid) {
+    const int w = tid >> 5, lane = tid & 31;
+    const int p = w >> 2, A0 = 32 * p, B0 = A0 + 16;
+    {  // warp: join p, columns 4 (w & 3) .. + 3; lane: row lane & 15, column pair lane >> 4
+        const int i = lane & 15, j0 = 4 * (w & 3), jc = j0 + 2 * (lane >> 4);
+        const float* lrow = Lf + (B0 + i) * LDL + A0;
+        float a0 = 0.f, a1 = 0.f;
+        for (int k = j0; k < 16; k += 4) {
+            const float4 l4 = *reinterpret_cast<const float4*>(lrow + k);
+            const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const float2 t = *reinterpret_cast<const float2*>(Lf + (A0 + k + u) * LDL + A0 + jc);
+                a0 = fmaf(lv[u], t.x, a0);
+                a1 = fmaf(lv[u], t.y, a1);
+            }
+        }
+        *reinterpret_cast<float2*>(X + p * 256 + i * 16 + jc) = make_float2(a0, a1);
+    }
+    __syncthreads();
+    {  // warp: join p, rows 4 (w & 3) .. + 3; lane: column lane & 15, row pair lane >> 4
+        const int j = lane & 15, i0 = 4 * (w & 3), ir = i0 + 2 * (lane >> 4);
+        float c0 = 0.f, c1 = 0.f;
+        for (int k = 0; k < i0 + 4; k += 4) {
+            const float4 t0 = *reinterpret_cast<const float4*>(Lf + (B0 + ir) * LDL + B0 + k);
+            const float4 t1 = *reinterpret_cast<const float4*>(Lf + (B0 + ir + 1) * LDL + B0 + k);
+            const float r0[4] = {t0.x, t0.y, t0.z, t0.w}, r1[4] = {t1.x, t1.y, t1.z, t1.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const float x = X[p * 256 + (k + u) * 16 + j];
+                c0 = fmaf(r0[u], x, c0);
+                c1 = fmaf(r1[u], x, c1);
+            }
+        }
+        Lf[(B0 + ir) * LDL + A0 + j] = -c0;
+        Lf[(B0 + ir + 1) * LDL + A0 + j] = -c1;
+    }
+    __syncthreads();
+}
+
 template <int NT>
 __device__ __forceinline__ void invert_unit_lower64_doubling(float* Lf, float* X, int tid) {
     static_assert(NT == 256, "the join levels assume 256 threads");
@@ -190,8 +281,8 @@ __device__ __forceinline__ void invert_unit_lower64_doubling(float* Lf, float* X
     }
     __syncthreads();
     inverse_join_level<8, NT>(Lf, X, tid);
-    inverse_join_level<16, NT>(Lf, X, tid);
-    inverse_join_level<32, NT>(Lf, X, tid);
+    inverse_join16_tri(Lf, X, tid);
+    inverse_join32_tri(Lf, X, tid);
 }
 
 // Store the 16-byte chunks c and c + 1 (c even) of row r of a 128B-swizzled [rows x 64] bf16
