@@ -149,24 +149,34 @@ __global__ void __launch_bounds__(PT, 3)
         }
         mma_commit(bar_mma);
     }
-    // key norms and Kaczmarz coefficients (thread 64 + j reads key row j)
-    if (tid >= CH && tid < 2 * CH) {
-        const int j = tid - CH;
-        float r2 = 0.f;
+    // key norms and Kaczmarz coefficients: four threads per key row j = tid / 4, thread q of the
+    // four summing 32 features (dk block q / 2, logical 16-byte chunks 4 (q & 1) .. + 3 of it, in
+    // an order rotated by q / 2 so that the eight lanes of a quarter warp -- rows j and j + 1,
+    // whose swizzle phases differ in parity -- hit eight different bank groups)
+    {
+        const int j = tid >> 2, q = tid & 3;
+        const uint8_t* krow = qk + (q >> 1) * 16384 + 8192 + j * 128;
+        float ra = 0.f, rb = 0.f;
 #pragma unroll
-        for (int blk = 0; blk < 2; ++blk)
+        for (int m = 0; m < 4; ++m) {
+            const int cc = 4 * (q & 1) + ((m + 2 * (q >> 1)) & 3);
+            float f[8];
+            unpack_bf16x8(*reinterpret_cast<const uint4*>(krow + ((cc ^ (j & 7)) << 4)), f);
 #pragma unroll
-            for (int c8 = 0; c8 < 8; ++c8) {  // chunk order rotated by row: no bank conflicts
-                const int cc = (c8 + j) & 7;
-                float f[8];
-                unpack_bf16x8(*reinterpret_cast<const uint4*>(qk + blk * 16384 + 8192 + j * 128 + cc * 16), f);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) r2 = fmaf(f[e], f[e], r2);
+            for (int e = 0; e < 8; e += 2) {
+                ra = fmaf(f[e], f[e], ra);
+                rb = fmaf(f[e + 1], f[e + 1], rb);
             }
-        const KaczCoef cf = kacz_coef(ms->eta[j], r2, a.eps);
-        ms->bco[j] = cf.b;
-        ms->cco[j] = cf.c;
-        ms->invr[j] = cf.inv_r;
+        }
+        float r2 = ra + rb;
+        r2 += __shfl_xor_sync(0xffffffffu, r2, 1);
+        r2 += __shfl_xor_sync(0xffffffffu, r2, 2);
+        if (q == 0) {
+            const KaczCoef cf = kacz_coef(ms->eta[j], r2, a.eps);
+            ms->bco[j] = cf.b;
+            ms->cco[j] = cf.c;
+            ms->invr[j] = cf.inv_r;
+        }
     }
     if (warp == 0) {  // inclusive prefix sum of g inside the chunk (2 tokens per lane)
         const int l = tid;
