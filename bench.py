@@ -257,6 +257,7 @@ def gpu_arm(args, rank, world, local_rank):
     o = torch.empty(w.B, w.T, w.H, w.Dv, device=dev, dtype=torch.float32)
     ST = torch.empty(w.B, w.H, w.Dk, w.Dv, device=dev, dtype=torch.float32)
     ws = kla.fwd_workspace(d["k"], d["v"])  # the split path's per-chunk records, allocated once
+    launches = kla.fwd_kernel_launches(d["k"], d["v"])  # 4: two slabs (prep + state pass each)
 
     def prefill():
         kla.chunk_fwd(d["q"], d["k"], d["v"], d["eta"], d["g"], w.eps, d["S0"], o=o, S_T=ST, workspace=ws)
@@ -317,13 +318,15 @@ def gpu_arm(args, rank, world, local_rank):
                    "parallelism": f"{world} independent replica(s), no collective"},
         "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
                      "frac": achieved_gbs / hbm_peak, "peak_kind": peaks_kind,
-                     "scope": "one kla_chunk_fwd call: chunk_prep_kernel + chunk_state_kernel",
+                     "scope": ("one kla_chunk_fwd call: chunk_prep_kernel + chunk_state_kernel"
+                               + (", as two slabs (slab 1's state pass concurrent with slab 2's"
+                                  " preparation)" if launches == 4 else "")),
                      "traffic": recorded_traffic("chunk_fwd_prefill_b8_t2048_h8_d128"),
                      "alg_bytes_per_launch": alg_bytes, "kernel_us": mean_s * 1e6, "stages": stages,
                      "tensor": {"achieved": achieved_tf, "peak": tc_peak, "unit": "TFLOP/s",
                                 "frac": achieved_tf / tc_peak, "alg_flops_per_launch": alg_flops}},
         "e2e": e2e,
-        "gpu_launches": 2 * args.steps,
+        "gpu_launches": launches * args.steps,
         "clocks": clocks,
     }
     line.update(extra)
@@ -413,6 +416,7 @@ def bench_train(kla, WORKLOADS, make_inputs, dev, stream, flush, rank, world, hb
         kla.chunk_bwd_after_train(d["q"], d["k"], d["v"], d["eta"], d["g"], dO, ws, w.eps)
 
     nsteps = 2 if args.quick else 5
+    launches = kla.fwd_kernel_launches(d["k"], d["v"]) + 2  # + reverse state pass, gradient kernel
     step()
     torch.cuda.synchronize()
     barrier(world)
@@ -426,8 +430,9 @@ def bench_train(kla, WORKLOADS, make_inputs, dev, stream, flush, rank, world, hb
     alg = fwd_bytes(w.B, w.T, w.H, w.Dk, w.Dv, elt, False) + bwd_bytes(w.B, w.T, w.H, w.Dk, w.Dv, elt)
     return {"workload": w.name, "value": tokens / (total_ms / 1e3), "unit": "tokens/s",
             "steps": nsteps, "ms_per_step": total_ms / nsteps,
-            # forward: preparation + state pass; backward: reverse state pass + gradient kernel
-            "gpu_launches_per_step": 4,
+            # forward: preparation + state pass (each twice with two slabs); backward: reverse
+            # state pass + gradient kernel
+            "gpu_launches_per_step": launches,
             "roofline": {"bound": "tensor", "achieved": flops / mean_s / 1e12, "peak": tc_peak,
                          "unit": "TFLOP/s", "frac": flops / mean_s / 1e12 / tc_peak,
                          "hbm_frac": alg / mean_s / 1e9 / hbm_peak, "alg_flops_per_step": flops,

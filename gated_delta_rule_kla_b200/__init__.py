@@ -54,6 +54,8 @@ def lib():
         L.kla_version.restype = i
         L.kla_chunk_fwd_workspace.argtypes = [i, i, i, i, i, i, i]
         L.kla_chunk_fwd_workspace.restype = sz
+        L.kla_chunk_fwd_kernel_launches.argtypes = [i, i, i, i, i, i, i]
+        L.kla_chunk_fwd_kernel_launches.restype = i
         L.kla_chunk_fwd.argtypes = [vp, vp, vp, fp, fp, f, fp, vp, fp, fp, i, i, i, i, i, i, i, i, vp, sz, vp]
         L.kla_chunk_fwd.restype = i
         L.kla_chunk_fwd_prep.argtypes = [vp, vp, vp, fp, fp, f, i, i, i, i, i, i, i, vp, sz, vp]
@@ -170,6 +172,12 @@ def fwd_workspace(k, v):
     B, T, H, Dk = k.shape
     need = lib().kla_chunk_fwd_workspace(B, T, H, Dk, v.shape[-1], CHUNK, _dtype_code(k))
     return torch.empty(need, device=k.device, dtype=torch.uint8) if need > 0 else None
+
+
+def fwd_kernel_launches(k, v):
+    """Kernels one chunk_fwd call with a workspace from fwd_workspace launches for k, v."""
+    B, T, H, Dk = k.shape
+    return lib().kla_chunk_fwd_kernel_launches(B, T, H, Dk, v.shape[-1], CHUNK, _dtype_code(k))
 
 
 def chunk_fwd_prep(q, k, v, eta, g, eps, workspace, *, stream=None):

@@ -125,6 +125,13 @@ size_t kla_chunk_fwd_workspace(int B, int T, int H, int Dk, int Dv, int chunk, i
     return kla::chunk_fwd_split_workspace(a);
 }
 
+int kla_chunk_fwd_kernel_launches(int B, int T, int H, int Dk, int Dv, int chunk, int dtype) {
+    if (B < 1 || H < 1 || T < 1 || chunk != kla::kChunkLen) return 0;
+    kla::FwdArgs a{};
+    a.B = B; a.T = T; a.H = H; a.Dk = Dk; a.Dv = Dv; a.bf16 = dtype == KLA_BF16;
+    return kla::chunk_fwd_split_workspace(a) > 0 ? kla::chunk_fwd_split_launches(a) : 1;
+}
+
 kla_status kla_chunk_fwd(const void* q, const void* k, const void* v, const float* eta,
                          const float* g, float eps, const float* S0, void* o, float* S_T,
                          float* S_chunks, int B, int T, int H, int Dk, int Dv, int chunk,

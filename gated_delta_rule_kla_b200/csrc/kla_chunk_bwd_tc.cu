@@ -1038,8 +1038,7 @@ cudaError_t launch_chunk_fwd_train_tc(const FwdArgs& f, void* ws, size_t ws_byte
     fa.T_tiles = w + L.T;
     fa.S_tiles = w + L.S;
     fa.U_tiles = w + L.U;
-    cudaError_t e = launch_chunk_fwd_split_prep(fa, w + L.fwd, st);
-    return e == cudaSuccess ? launch_chunk_fwd_split_state(fa, w + L.fwd, st) : e;
+    return launch_chunk_fwd_split(fa, w + L.fwd, st);  // two slabs when the heads are few
 }
 
 cudaError_t launch_chunk_bwd_tc_reverse(const BwdTcArgs& a, void* ws, size_t ws_bytes, cudaStream_t st) {

@@ -23,6 +23,10 @@
 #include <cuda.h>
 #include <string.h>
 
+#include <algorithm>
+#include <mutex>
+#include <unordered_map>
+
 #include "kla_device.cuh"
 #include "kla_launch.h"
 #include "kla_sm100.cuh"
@@ -66,7 +70,7 @@ static_assert(sizeof(PrepMisc) <= 3072, "prep scalars");
 
 __global__ void __launch_bounds__(PT, 3)
     chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                      const __grid_constant__ CUtensorMap tm_v, FwdArgs a, uint8_t* __restrict__ recs) {
+                      const __grid_constant__ CUtensorMap tm_v, FwdArgs a, uint8_t* __restrict__ recs, int cfirst) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     PrepMisc* ms = reinterpret_cast<PrepMisc*>(sm + P_MISC);
@@ -77,7 +81,7 @@ __global__ void __launch_bounds__(PT, 3)
     const int row = tid & 127, ch = tid >> 7;
     const int H = a.H, T = a.T;
     const int NC = (T + CH - 1) / CH;
-    const int c = blockIdx.x, head = blockIdx.y;
+    const int c = cfirst + blockIdx.x, head = blockIdx.y;
     const int b = head / H, h = head % H;
     const int t0 = c * CH, n = min(CH, T - t0);
     uint8_t* rec = recs + ((size_t)head * NC + c) * REC_BYTES;
@@ -444,12 +448,12 @@ __global__ void __launch_bounds__(ST, 1)
     const int NCtot = (T + CH - 1) / CH;
     const int nseg = a.nseg > 1 ? a.nseg : 1;
     const bool segmented = a.nseg > 1;
-    const int segc = segmented ? a.seg_chunks : NCtot;
+    const int segc = a.seg_chunks > 0 ? a.seg_chunks : NCtot;  // chunks of this run (segment or slab)
     const int head_idx = blockIdx.x / nseg, seg = blockIdx.x % nseg;
     const int BH = gridDim.x / nseg;
     const int b = head_idx / H, h = head_idx % H;
     const bool ident = blockIdx.y == 1;  // transition pass: identity start, zero values, no outputs
-    const int c0 = seg * segc, c1 = min(NCtot, c0 + segc);
+    const int c0 = (segmented ? 0 : a.chunk0) + seg * segc, c1 = min(NCtot, c0 + segc);
     const int NC = c1 > c0 ? c1 - c0 : 0;
     const uint32_t sbase = smem_u32(sm);
     const uint32_t full_a0 = smem_u32(&ms->full_a[0]), full_b0 = smem_u32(&ms->full_b[0]);
@@ -850,9 +854,47 @@ int choose_nseg_split(int BH, int NC) {
 
 size_t align1k(size_t x) { return (x + 1023) & ~size_t(1023); }
 
+// Two slabs: the state pass holds one SM per head for the whole sequence, so with few heads
+// most SMs idle while it runs.  Splitting the chunks into two slabs lets the second slab's
+// preparation run on those SMs while the first slab's state pass runs, the second state pass
+// starting from the first one's final state.  Cost model in
+// state steps (one chunk of the state pass, ~2.3 us here); a wave of preparation CTAs (three
+// per SM) takes kPrepWaveSteps of them (measured: ~18.7 us per wave).  Returns the first
+// slab's chunk count, or 0 for one run.
+// The first slab's preparation has the whole GPU: whole waves, and a last partial wave that
+// costs 0.45 + 0.55 x its fill (its CTAs share their SMs with fewer others); the second slab's
+// runs beside the state pass and spills onto its SMs when it ends, so it is counted fluidly.
+// Calibrated on the B=8 T=2048 H=8 and B=4 T=4096 H=16 forwards (sweeps of the split point:
+// optima at 20 of 32 and 41-42 of 64 chunks).
+constexpr double kPrepWaveSteps = 8.1;
+int choose_slab_split(int BH, int NC) {
+    const int sms = sm_count();
+    if (NC < 8 || 2 * BH > sms) return 0;
+    auto prep_all = [&](long long items) {
+        const long long slots = 3LL * sms, full = items / slots;
+        const double frac = (double)(items - full * slots) / slots;
+        return (full + (frac > 0 ? 0.45 + 0.55 * frac : 0.0)) * kPrepWaveSteps;
+    };
+    auto prep_beside = [&](double items) { return items / (3.0 * (sms - BH)) * kPrepWaveSteps; };
+    const double base = prep_all((long long)NC * BH) + NC;
+    double best = base;
+    int nc1 = 0;
+    for (int n1 = 2; n1 <= NC - 2; ++n1) {
+        const double t = prep_all((long long)n1 * BH) + std::max<double>(n1 + 2, prep_beside((double)(NC - n1) * BH)) +
+                         (NC - n1) + 2;
+        if (t < best) {
+            best = t;
+            nc1 = n1;
+        }
+    }
+    return best < 0.95 * base ? nc1 : 0;
+}
+
 struct SplitLayout {
     size_t rec_bytes, seg_off, total;
     int nseg, segc;
+    int nc1;          // chunks of the first slab (0: one run)
+    size_t slab_off;  // [B*H, Dk, Dv] fp32: the state between the slabs
 };
 
 SplitLayout split_layout(const FwdArgs& a) {
@@ -870,8 +912,31 @@ SplitLayout split_layout(const FwdArgs& a) {
         L.nseg = 1;
         L.segc = NC;
         L.total = L.seg_off;
+        L.nc1 = choose_slab_split(BH, NC);
+        if (L.nc1 > 0) {
+            L.slab_off = L.total;
+            L.total += (size_t)BH * DK * DV * sizeof(float);
+        }
     }
     return L;
+}
+
+// A stream per device for the second slab's preparation (created once).
+cudaError_t slab_stream(cudaStream_t* out) {
+    static std::mutex mu;
+    static std::unordered_map<int, cudaStream_t> streams;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = streams.find(dev);
+    if (it == streams.end()) {
+        cudaStream_t s = nullptr;
+        if ((e = cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking)) != cudaSuccess) return e;
+        it = streams.emplace(dev, s).first;
+    }
+    *out = it->second;
+    return cudaSuccess;
 }
 
 // 4-D map over the [B, T, H, 128] output (fp32 or bf16) for TMA stores of one chunk's rows of
@@ -909,16 +974,30 @@ size_t chunk_fwd_split_workspace(const FwdArgs& a) {
     return split_layout(a).total;
 }
 
-cudaError_t launch_chunk_fwd_split_prep(const FwdArgs& a, void* ws, cudaStream_t st) {
+namespace {
+// Preparation of chunks [cfirst, cfirst + count) of every head.
+cudaError_t launch_prep_range(const FwdArgs& a, void* ws, int cfirst, int count, cudaStream_t st) {
     CUtensorMap mq, mk, mv;
     if (!make_map(&mq, a.q, a.B, a.T, a.H) || !make_map(&mk, a.k, a.B, a.T, a.H) ||
         !make_map(&mv, a.v, a.B, a.T, a.H))
         return cudaErrorInvalidValue;
-    const int NC = (a.T + CH - 1) / CH;
     cudaError_t e = cudaFuncSetAttribute(chunk_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)P_SMEM);
     if (e != cudaSuccess) return e;
-    chunk_prep_kernel<<<dim3(NC, a.B * a.H), PT, P_SMEM, st>>>(mq, mk, mv, a, static_cast<uint8_t*>(ws));
+    chunk_prep_kernel<<<dim3(count, a.B * a.H), PT, P_SMEM, st>>>(mq, mk, mv, a, static_cast<uint8_t*>(ws), cfirst);
     return cudaGetLastError();
+}
+// One non-segmented state-pass run over chunks [f.chunk0, f.chunk0 + f.seg_chunks) of every head.
+cudaError_t launch_state_run(const FwdArgs& f, void* ws, cudaStream_t st) {
+    CUtensorMap mq;
+    if (!make_map(&mq, f.q, f.B, f.T, f.H)) return cudaErrorInvalidValue;
+    const uint8_t* recs = static_cast<const uint8_t*>(ws);
+    const dim3 grid(f.B * f.H, 1);
+    return f.out_bf16 ? launch_state<__nv_bfloat16>(mq, f, recs, grid, st) : launch_state<float>(mq, f, recs, grid, st);
+}
+}  // namespace
+
+cudaError_t launch_chunk_fwd_split_prep(const FwdArgs& a, void* ws, cudaStream_t st) {
+    return launch_prep_range(a, ws, 0, (a.T + CH - 1) / CH, st);
 }
 
 cudaError_t launch_chunk_fwd_split_state(const FwdArgs& a, void* ws, cudaStream_t st) {
@@ -937,6 +1016,7 @@ cudaError_t launch_chunk_fwd_split_state(const FwdArgs& a, void* ws, cudaStream_
         f.nseg = 1;
         f.seg_chunks = NC;
         f.kinds = 1;
+        f.chunk0 = 0;
         return state(f, dim3(BH, 1));
     }
     const size_t SZ = (size_t)DK * DV;
@@ -952,6 +1032,7 @@ cudaError_t launch_chunk_fwd_split_state(const FwdArgs& a, void* ws, cudaStream_
     p1.nseg = L.nseg;
     p1.seg_chunks = L.segc;
     p1.kinds = 2;
+    p1.chunk0 = 0;
     cudaError_t e = state(p1, dim3(BH * L.nseg, 2));
     if (e != cudaSuccess) return e;
     if ((e = launch_seg_scan(a.S0, MN, Sstart, a.S_T, BH, L.nseg, st)) != cudaSuccess) return e;
@@ -961,16 +1042,63 @@ cudaError_t launch_chunk_fwd_split_state(const FwdArgs& a, void* ws, cudaStream_
     p2.nseg = L.nseg;
     p2.seg_chunks = L.segc;
     p2.kinds = 1;
+    p2.chunk0 = 0;
     return state(p2, dim3(BH * L.nseg, 1));
 }
 
 cudaError_t launch_chunk_fwd_split(const FwdArgs& a, void* ws, cudaStream_t st) {
-    cudaError_t e = launch_chunk_fwd_split_prep(a, ws, st);
-    return e == cudaSuccess ? launch_chunk_fwd_split_state(a, ws, st) : e;
+    const SplitLayout L = split_layout(a);
+    if (L.nc1 <= 0) {
+        cudaError_t e = launch_chunk_fwd_split_prep(a, ws, st);
+        return e == cudaSuccess ? launch_chunk_fwd_split_state(a, ws, st) : e;
+    }
+    // Two slabs: prep(slab 1) then state(slab 1) on the caller's stream -- the state pass, next
+    // in the same queue, takes its SMs (one per head) first -- while prep(slab 2) runs on the
+    // side stream over the other SMs; state(slab 2) follows on the caller's stream once both are
+    // done.  The kernels of the two streams share no data and never wait on each other.
+    const int NC = (a.T + CH - 1) / CH;
+    float* Smid = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + L.slab_off);
+    cudaStream_t side = nullptr;
+    cudaEvent_t ev_prep = nullptr, ev_state = nullptr;
+    cudaError_t e = slab_stream(&side);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ev_prep, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ev_state, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = launch_prep_range(a, ws, 0, L.nc1, st);
+    if (e == cudaSuccess) e = cudaEventRecord(ev_prep, st);
+    if (e == cudaSuccess) {
+        FwdArgs f1 = a;
+        f1.nseg = 1;
+        f1.kinds = 1;
+        f1.chunk0 = 0;
+        f1.seg_chunks = L.nc1;
+        f1.S_T = Smid;
+        e = launch_state_run(f1, ws, st);
+    }
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(side, ev_prep, 0);
+    if (e == cudaSuccess) {
+        e = launch_prep_range(a, ws, L.nc1, NC - L.nc1, side);
+        // the caller's stream takes the side stream's work back whatever happens next
+        const cudaError_t er = cudaEventRecord(ev_state, side);
+        const cudaError_t ej = er == cudaSuccess ? cudaStreamWaitEvent(st, ev_state, 0) : er;
+        if (e == cudaSuccess) e = ej;
+    }
+    if (e == cudaSuccess) {
+        FwdArgs f2 = a;
+        f2.nseg = 1;
+        f2.kinds = 1;
+        f2.chunk0 = L.nc1;
+        f2.seg_chunks = NC - L.nc1;
+        f2.S0 = Smid;
+        e = launch_state_run(f2, ws, st);
+    }
+    if (ev_prep) cudaEventDestroy(ev_prep);  // released once the work that uses them is done
+    if (ev_state) cudaEventDestroy(ev_state);
+    return e;
 }
 
-int chunk_fwd_split_state_launches(const FwdArgs& a) {
-    return split_layout(a).nseg > 1 ? 3 : 1;
+int chunk_fwd_split_launches(const FwdArgs& a) {
+    const SplitLayout L = split_layout(a);
+    return L.nseg > 1 ? 4 : (L.nc1 > 0 ? 4 : 2);
 }
 
 cudaError_t split_take_error(cudaStream_t st, unsigned int* flag) {

@@ -43,6 +43,9 @@ struct FwdArgs {
     void* T_tiles;
     void* S_tiles;
     void* U_tiles;
+    // First chunk of a non-segmented state-pass run of seg_chunks chunks (0 for a whole
+    // sequence): the host splits a sequence into slabs handled by consecutive runs.
+    int chunk0;
 };
 
 struct BwdArgs {
@@ -101,6 +104,8 @@ cudaError_t launch_seg_scan(const float* S0, const float* MN, float* Sstart, flo
 // long sequences over few heads).  Workspace bytes for these sizes (0: shapes not supported).
 size_t chunk_fwd_split_workspace(const FwdArgs& a);
 cudaError_t launch_chunk_fwd_split(const FwdArgs& a, void* ws, cudaStream_t st);
+// Kernels one launch_chunk_fwd_split call launches (preparation and state passes).
+int chunk_fwd_split_launches(const FwdArgs& a);
 // The two stages of the split path: the chunk-parallel preparation (writes the per-chunk
 // records into ws) and the state pass that reads them.
 cudaError_t launch_chunk_fwd_split_prep(const FwdArgs& a, void* ws, cudaStream_t st);

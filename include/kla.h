@@ -92,9 +92,18 @@ int kla_version(void);
  *                     pass consumes them (segmented, for long sequences over few heads).  With
  *                     NULL or a smaller buffer the forward still runs, as one fused kernel per
  *                     head.  The workspace must not be shared with a concurrent call.
+ *                     When the heads are few (at most half the SMs), the split path runs the
+ *                     sequence as two slabs of chunks: the second slab's preparation runs on an
+ *                     internal stream of the device while the first slab's state pass runs on
+ *                     `stream`, which then waits for it before the second state pass (results
+ *                     are bit-identical to one run; the call stays ordered on `stream`).
  * Returns KLA_OK or an error status; on error nothing is launched.
  */
 size_t kla_chunk_fwd_workspace(int B, int T, int H, int Dk, int Dv, int chunk, int dtype);
+/* Number of kernels one kla_chunk_fwd call launches for these shapes when given at least
+ * kla_chunk_fwd_workspace() bytes of workspace (1 for shapes that take none); 0 for invalid
+ * shapes. */
+int kla_chunk_fwd_kernel_launches(int B, int T, int H, int Dk, int Dv, int chunk, int dtype);
 kla_status kla_chunk_fwd(const void *q, const void *k, const void *v, const float *eta,
                          const float *g, float eps, const float *S0, void *o, float *S_T,
                          float *S_chunks, int B, int T, int H, int Dk, int Dv, int chunk,

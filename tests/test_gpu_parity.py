@@ -174,12 +174,15 @@ def test_fwd_split_and_fused_paths_agree(kla, oracle_mod, B, T, H, s0, g_lo, out
         torch.testing.assert_close(outs[False][2][:, :, 0], d["S0"])  # chunk 0 starts from S0
 
 
-@pytest.mark.parametrize("B,T,H", [(2, 300, 3), (1, 4096 + 100, 2)])
-def test_fwd_prep_and_state_stages_equal_one_call(kla, B, T, H):
+@pytest.mark.parametrize("B,T,H,launches", [(2, 300, 3, 2), (1, 4096 + 100, 2, 4), (8, 1024, 8, 4)])
+def test_fwd_prep_and_state_stages_equal_one_call(kla, B, T, H, launches):
     """kla_chunk_fwd_prep then kla_chunk_fwd_state is kla_chunk_fwd with the same workspace,
-    bit for bit (the second shape takes the segmented state pass)."""
+    bit for bit.  The second shape takes the segmented state pass; the third runs kla_chunk_fwd
+    as two slabs (the first slab's state pass concurrent with the second slab's preparation),
+    against one state-pass run over the whole sequence here."""
     inp = small_inputs(B, T, H, 128, 128, "bf16", seed=T + H, g_lo=-0.05)
     d = {k: (v.cuda() if v is not None else None) for k, v in inp.items()}
+    assert kla.fwd_kernel_launches(d["k"], d["v"]) == launches
     ws = kla.fwd_workspace(d["k"], d["v"])
     o, ST, Sc = kla.chunk_fwd(d["q"], d["k"], d["v"], d["eta"], d["g"], 1e-6, d["S0"], save_chunk_states=True,
                               workspace=ws)
