@@ -295,6 +295,8 @@ def gpu_arm(args, rank, world, local_rank):
         if "long" in parts:
             extra["long_context"] = bench_long(kla, WORKLOADS, make_inputs, dev, stream, rank, world,
                                                hbm_peak, tc_peak, args)
+        if "direct" in parts:
+            extra["direct_beta"] = bench_direct(kla, w, d, ws, o, ST, flush, stream, world, hbm_peak, args)
 
     # ---------------- end-to-end through the public API with host buffers ----------------
     e2e = None if args.skip_e2e else bench_e2e(kla, w, inp, dev, stream, rank, world, args)
@@ -474,6 +476,33 @@ def bench_long(kla, WORKLOADS, make_inputs, dev, stream, rank, world, hbm_peak, 
                          "tensor_frac": flops / mean_s / 1e12 / tc_peak}}
 
 
+def bench_direct(kla, w, d, ws, o, ST, flush, stream, world, hbm_peak, args):
+    """The headline prefill with the direct write strength (beta_t = eta_t as given: the
+    Gated DeltaNet update, KLA_BETA_DIRECT): the same kernels, the coefficient map changed."""
+    import torch
+    eta = (d["eta"] / ((d["k"].float() ** 2).sum(-1) + 1.0)).contiguous()  # contractive writes
+
+    def prefill():
+        kla.chunk_fwd(d["q"], d["k"], d["v"], eta, d["g"], w.eps, d["S0"], o=o, S_T=ST, workspace=ws,
+                      beta="direct")
+
+    for _ in range(3):
+        flush()
+        prefill()
+    torch.cuda.synchronize()
+    nsteps = 5 if args.quick else 20
+    ms = time_steps(prefill, nsteps, flush, stream)
+    total_ms = max_over_ranks(sum(ms), world)
+    tokens = sum_over_ranks(float(w.B * w.T), world) * nsteps
+    mean_s = statistics.mean(ms) / 1e3
+    alg = fwd_bytes(w.B, w.T, w.H, w.Dk, w.Dv, d["q"].element_size(), d["S0"] is not None)
+    return {"workload": w.name, "beta": "direct", "value": tokens / (total_ms / 1e3), "unit": "tokens/s",
+            "steps": nsteps, "ms_per_step": total_ms / nsteps, "l2": "flushed between timed steps",
+            "gpu_launches_per_step": kla.fwd_kernel_launches(d["k"], d["v"]),
+            "roofline": {"bound": "hbm", "achieved": alg / mean_s / 1e9, "peak": hbm_peak, "unit": "GB/s",
+                         "frac": alg / mean_s / 1e9 / hbm_peak}}
+
+
 def bench_e2e(kla, w, inp, dev, stream, rank, world, args):
     """Same metric through the public API from pinned host buffers: every step's inputs go
     host -> device, kla_chunk_fwd runs, and o and S_T come back device -> host, all inside the
@@ -613,8 +642,8 @@ def parse(argv=None):
     ap.add_argument("--ref-pairs", type=int, default=8, help="(b,h) pairs per reference step")
     ap.add_argument("--cpu-pairs", type=int, default=64, help="(b,h) pairs in the CPU baseline sample")
     ap.add_argument("--skip-extra", action="store_true", help="headline prefill only")
-    ap.add_argument("--parts", default="decode,train,long",
-                    help="sub-measurements after the headline prefill (comma list of decode,train,long)")
+    ap.add_argument("--parts", default="decode,train,long,direct",
+                    help="sub-measurements after the headline prefill (comma list of decode,train,long,direct)")
     ap.add_argument("--skip-e2e", action="store_true", help="omit the host-buffer end-to-end leg")
     ap.add_argument("--skip-cpu", action="store_true", help="omit the CPU baseline")
     ap.add_argument("--quick", action="store_true", help="fewer decode/train steps (smoke runs)")

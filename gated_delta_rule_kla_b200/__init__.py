@@ -24,6 +24,7 @@ __all__ = ["lib", "chunk_fwd", "chunk_bwd", "chunk_fwd_train", "chunk_bwd_after_
 
 CHUNK = 64
 KLA_F32, KLA_BF16 = 0, 1
+KLA_BETA_DIRECT = 0x100  # OR-ed into the input dtype code: beta_t = eta_t as given
 _PKG = os.path.dirname(os.path.abspath(__file__))
 library_path = os.path.join(_PKG, "libkla.so")
 _lib = None
@@ -102,6 +103,14 @@ def _dtype_code(t):
     raise TypeError(f"expected bfloat16 or float32, got {dt}")
 
 
+def _in_code(t, beta):
+    """Input dtype code with the write-strength mode: "kaczmarz" (beta_t = eta_t / (||k_t||^2 +
+    eps), Eq. 3) or "direct" (beta_t = eta_t as given: the Gated DeltaNet update)."""
+    if beta not in ("kaczmarz", "direct"):
+        raise ValueError(f"beta must be 'kaczmarz' or 'direct', got {beta!r}")
+    return _dtype_code(t) | (KLA_BETA_DIRECT if beta == "direct" else 0)
+
+
 def _need(t, name, device, dtype=None, shape=None):
     if t is None:
         return None
@@ -125,7 +134,7 @@ def _stream(device, stream):
 
 def chunk_fwd(q, k, v, eta, g, eps=1e-6, S0=None, *, o=None, S_T=None, save_chunk_states=False,
               output_final_state=True, out_dtype=torch.float32, stream=None, fused=False,
-              workspace=None):
+              workspace=None, beta="kaczmarz"):
     """Chunkwise prefill (section 4, Propositions 3-4).
 
     q, k: [B,T,H,Dk]; v: [B,T,H,Dv] (bf16 or fp32, same dtype); eta, g: [B,T,H] fp32;
@@ -136,7 +145,9 @@ def chunk_fwd(q, k, v, eta, g, eps=1e-6, S0=None, *, o=None, S_T=None, save_chun
     stores every chunk's state-independent operands in the workspace kla_chunk_fwd_workspace()
     reports (allocated here unless `workspace` is given), then a sequential state pass (split
     into parallel segments for long sequences over few heads).  fused=True passes no workspace,
-    which selects the one-kernel-per-head path.
+    which selects the one-kernel-per-head path.  beta="direct" takes eta as the write strength
+    itself (beta_t = eta_t, the Gated DeltaNet update) instead of the Kaczmarz step; the other
+    entry points take the same keyword.
     """
     dev = k.device
     B, T, H, Dk = k.shape
@@ -160,7 +171,7 @@ def chunk_fwd(q, k, v, eta, g, eps=1e-6, S0=None, *, o=None, S_T=None, save_chun
         workspace = torch.empty(need, device=dev, dtype=torch.uint8)
     ws_ptr, ws_n = (_ptr(workspace), workspace.numel()) if need > 0 else (None, 0)
     st = L.kla_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(eta), _ptr(g), float(eps), _ptr(S0),
-                         _ptr(o), _ptr(S_T), _ptr(Sc), B, T, H, Dk, Dv, CHUNK, _dtype_code(k),
+                         _ptr(o), _ptr(S_T), _ptr(Sc), B, T, H, Dk, Dv, CHUNK, _in_code(k, beta),
                          _dtype_code(o), ws_ptr, ws_n, _stream(dev, stream))
     _check(st, "kla_chunk_fwd")
     return (o, S_T, Sc) if save_chunk_states else (o, S_T)
@@ -180,7 +191,7 @@ def fwd_kernel_launches(k, v):
     return lib().kla_chunk_fwd_kernel_launches(B, T, H, Dk, v.shape[-1], CHUNK, _dtype_code(k))
 
 
-def chunk_fwd_prep(q, k, v, eta, g, eps, workspace, *, stream=None):
+def chunk_fwd_prep(q, k, v, eta, g, eps, workspace, *, stream=None, beta="kaczmarz"):
     """First stage of the split forward: every chunk's state-independent operands into
     `workspace` (from fwd_workspace).  bf16 inputs with Dk == Dv == 128."""
     dev = k.device
@@ -191,7 +202,7 @@ def chunk_fwd_prep(q, k, v, eta, g, eps, workspace, *, stream=None):
     _need(workspace, "workspace", dev, torch.uint8)
     L = lib()
     st = L.kla_chunk_fwd_prep(_ptr(q), _ptr(k), _ptr(v), _ptr(eta), _ptr(g), float(eps), B, T, H, Dk, Dv,
-                              CHUNK, _dtype_code(k), _ptr(workspace), workspace.numel(), _stream(dev, stream))
+                              CHUNK, _in_code(k, beta), _ptr(workspace), workspace.numel(), _stream(dev, stream))
     _check(st, "kla_chunk_fwd_prep")
 
 
@@ -219,7 +230,7 @@ def chunk_fwd_state(q, g, S0, workspace, *, Dv=None, o=None, S_T=None, S_chunks=
 
 
 def chunk_bwd(q, k, v, eta, g, dO, eps=1e-6, S0=None, dS_T=None, S_chunks=None, *, stream=None,
-              workspace=None, out_dtype=torch.float32, cuda_cores=False):
+              workspace=None, out_dtype=torch.float32, cuda_cores=False, beta="kaczmarz"):
     """Gradients of the chunkwise forward w.r.t. q, k, v, eta, g and S0.
 
     dO: [B,T,H,Dv] (same dtype as q); dS_T: [B,H,Dk,Dv] fp32 or None; S_chunks: the
@@ -252,7 +263,7 @@ def chunk_bwd(q, k, v, eta, g, dO, eps=1e-6, S0=None, dS_T=None, S_chunks=None, 
     st = L.kla_chunk_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(eta), _ptr(g), float(eps), _ptr(S0), _ptr(dO),
                          _ptr(dS_T), _ptr(S_chunks), _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]),
                          _ptr(out["deta"]), _ptr(out["dg"]), _ptr(out["dS0"]), B, T, H, Dk, Dv, CHUNK,
-                         _dtype_code(k), _dtype_code(out_dtype), _ptr(workspace), workspace.numel(),
+                         _in_code(k, beta), _dtype_code(out_dtype), _ptr(workspace), workspace.numel(),
                          _stream(dev, stream))
     _check(st, "kla_chunk_bwd")
     return out
@@ -266,7 +277,7 @@ def train_workspace(k, v):
 
 
 def chunk_fwd_train(q, k, v, eta, g, eps=1e-6, S0=None, *, workspace=None, o=None, S_T=None,
-                    out_dtype=torch.float32, stream=None):
+                    out_dtype=torch.float32, stream=None, beta="kaczmarz"):
     """Training forward: (o, S_T, workspace), the workspace holding what chunk_bwd_after_train
     needs for these inputs (kla_chunk_fwd_train)."""
     dev = k.device
@@ -284,14 +295,14 @@ def chunk_fwd_train(q, k, v, eta, g, eps=1e-6, S0=None, *, workspace=None, o=Non
     if workspace is None:
         workspace = train_workspace(k, v)
     st = lib().kla_chunk_fwd_train(_ptr(q), _ptr(k), _ptr(v), _ptr(eta), _ptr(g), float(eps), _ptr(S0), _ptr(o),
-                                   _ptr(S_T), B, T, H, Dk, Dv, CHUNK, _dtype_code(k), _dtype_code(o),
+                                   _ptr(S_T), B, T, H, Dk, Dv, CHUNK, _in_code(k, beta), _dtype_code(o),
                                    _ptr(workspace), workspace.numel(), _stream(dev, stream))
     _check(st, "kla_chunk_fwd_train")
     return o, S_T, workspace
 
 
 def chunk_bwd_after_train(q, k, v, eta, g, dO, workspace, eps=1e-6, dS_T=None, *, out_dtype=torch.float32,
-                          stream=None):
+                          stream=None, beta="kaczmarz"):
     """Backward after chunk_fwd_train on the same inputs and workspace (kla_chunk_bwd_after_train).
     Returns dict(dq, dk, dv, deta, dg, dS0)."""
     dev = k.device
@@ -307,13 +318,14 @@ def chunk_bwd_after_train(q, k, v, eta, g, dO, workspace, eps=1e-6, dS_T=None, *
     st = lib().kla_chunk_bwd_after_train(_ptr(q), _ptr(k), _ptr(v), _ptr(eta), _ptr(g), float(eps), _ptr(dO),
                                          _ptr(dS_T), _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]),
                                          _ptr(out["deta"]), _ptr(out["dg"]), _ptr(out["dS0"]), B, T, H, Dk, Dv,
-                                         CHUNK, _dtype_code(k), _dtype_code(out_dtype), _ptr(workspace),
+                                         CHUNK, _in_code(k, beta), _dtype_code(out_dtype), _ptr(workspace),
                                          workspace.numel(), _stream(dev, stream))
     _check(st, "kla_chunk_bwd_after_train")
     return out
 
 
-def decode_step(q, k, v, eta, g, S, eps=1e-6, *, o=None, out_dtype=torch.float32, stream=None):
+def decode_step(q, k, v, eta, g, S, eps=1e-6, *, o=None, out_dtype=torch.float32, stream=None,
+                beta="kaczmarz"):
     """One decode token for every (b, h): q, k [B,H,Dk]; v [B,H,Dv]; eta, g [B,H] fp32;
     S [B,H,Dk,Dv] fp32 updated in place.  Returns o [B,H,Dv]."""
     dev = S.device
@@ -326,7 +338,7 @@ def decode_step(q, k, v, eta, g, S, eps=1e-6, *, o=None, out_dtype=torch.float32
         o = torch.empty(B, H, Dv, device=dev, dtype=out_dtype)
     _need(o, "o", dev, None, (B, H, Dv))
     st = lib().kla_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(eta), _ptr(g), float(eps), _ptr(S), _ptr(o),
-                               B, H, Dk, Dv, _dtype_code(k), _dtype_code(o), _stream(dev, stream))
+                               B, H, Dk, Dv, _in_code(k, beta), _dtype_code(o), _stream(dev, stream))
     _check(st, "kla_decode_step")
     return o
 

@@ -7,6 +7,7 @@
 #include <string>
 
 #include "kla.h"
+#include "kla_device.cuh"
 #include "kla_launch.h"
 #include "kla_tc_common.cuh"
 
@@ -30,6 +31,16 @@ kla_status cuda_fail(cudaError_t e, const char* where) {
 }
 
 bool aligned16(const void* p) { return p == nullptr || (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// KLA_BETA_DIRECT rides in a dtype argument: take it off (leaving the element type) and say
+// whether it was set.  The kernels learn it as eps = kla::kBetaDirect, a value the checks
+// below never let through otherwise.
+bool take_beta_flag(int& dtype) {
+    const bool direct = (dtype & KLA_BETA_DIRECT) != 0;
+    dtype &= ~KLA_BETA_DIRECT;
+    return direct;
+}
+float kernel_eps(float eps, bool direct) { return direct ? kla::kBetaDirect : eps; }
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
@@ -119,6 +130,7 @@ const char* kla_last_error(void) { return g_last_error.c_str(); }
 int kla_version(void) { return 100; }
 
 size_t kla_chunk_fwd_workspace(int B, int T, int H, int Dk, int Dv, int chunk, int dtype) {
+    take_beta_flag(dtype);
     if (B < 1 || H < 1 || T < 1 || chunk != kla::kChunkLen) return 0;
     kla::FwdArgs a{};
     a.B = B; a.T = T; a.H = H; a.Dk = Dk; a.Dv = Dv; a.bf16 = dtype == KLA_BF16;
@@ -126,6 +138,7 @@ size_t kla_chunk_fwd_workspace(int B, int T, int H, int Dk, int Dv, int chunk, i
 }
 
 int kla_chunk_fwd_kernel_launches(int B, int T, int H, int Dk, int Dv, int chunk, int dtype) {
+    take_beta_flag(dtype);
     if (B < 1 || H < 1 || T < 1 || chunk != kla::kChunkLen) return 0;
     kla::FwdArgs a{};
     a.B = B; a.T = T; a.H = H; a.Dk = Dk; a.Dv = Dv; a.bf16 = dtype == KLA_BF16;
@@ -136,6 +149,7 @@ kla_status kla_chunk_fwd(const void* q, const void* k, const void* v, const floa
                          const float* g, float eps, const float* S0, void* o, float* S_T,
                          float* S_chunks, int B, int T, int H, int Dk, int Dv, int chunk,
                          int dtype, int out_dtype, void* ws, size_t ws_bytes, void* stream) {
+    const bool direct = take_beta_flag(dtype);
     kla_status st = check_common(B, T, H, Dk, Dv, chunk, dtype, out_dtype, eps);
     if (st != KLA_OK) return st;
     if (T > 0) {
@@ -152,8 +166,8 @@ kla_status kla_chunk_fwd(const void* q, const void* k, const void* v, const floa
         }
         return KLA_OK;
     }
-    kla::FwdArgs a{q, k, v, eta, g, eps, S0, o, S_T, S_chunks, B, T, H, Dk, Dv, dtype == KLA_BF16,
-                   out_dtype == KLA_BF16};
+    kla::FwdArgs a{q, k, v, eta, g, kernel_eps(eps, direct), S0, o, S_T, S_chunks, B, T, H, Dk, Dv,
+                   dtype == KLA_BF16, out_dtype == KLA_BF16};
     cudaError_t e;
     if (kla::chunk_fwd_tc_supported(a)) {
         // With the workspace of kla_chunk_fwd_workspace: chunk-parallel preparation + state pass
@@ -192,10 +206,12 @@ static kla_status split_stage_checks(int B, int T, int H, int Dk, int Dv, int ch
 kla_status kla_chunk_fwd_prep(const void* q, const void* k, const void* v, const float* eta,
                               const float* g, float eps, int B, int T, int H, int Dk, int Dv,
                               int chunk, int dtype, void* ws, size_t ws_bytes, void* stream) {
+    const bool direct = take_beta_flag(dtype);
     kla::FwdArgs a{};
     kla_status st = split_stage_checks(B, T, H, Dk, Dv, chunk, dtype, KLA_F32, eps, ws, ws_bytes,
                                        "kla_chunk_fwd_prep", &a);
     if (st != KLA_OK) return st;
+    a.eps = kernel_eps(eps, direct);
     REQUIRE_PTR(q); REQUIRE_PTR(k); REQUIRE_PTR(v); REQUIRE_PTR(eta); REQUIRE_PTR(g);
     a.q = q; a.k = k; a.v = v; a.eta = eta; a.g = g;
     cudaError_t e = kla::launch_chunk_fwd_split_prep(a, ws, static_cast<cudaStream_t>(stream));
@@ -206,6 +222,7 @@ kla_status kla_chunk_fwd_prep(const void* q, const void* k, const void* v, const
 kla_status kla_chunk_fwd_state(const void* q, const float* g, const float* S0, void* o, float* S_T,
                                float* S_chunks, int B, int T, int H, int Dk, int Dv, int chunk,
                                int dtype, int out_dtype, void* ws, size_t ws_bytes, void* stream) {
+    take_beta_flag(dtype);  // the state pass reads the preparation's coefficients
     kla::FwdArgs a{};
     kla_status st = split_stage_checks(B, T, H, Dk, Dv, chunk, dtype, out_dtype, 0.f, ws, ws_bytes,
                                        "kla_chunk_fwd_state", &a);
@@ -220,7 +237,8 @@ kla_status kla_chunk_fwd_state(const void* q, const float* g, const float* S0, v
 
 size_t kla_chunk_bwd_workspace_min(int B, int T, int H, int Dk, int Dv, int chunk, int dtype,
                                    int have_S_chunks) {
-    (void)chunk; (void)dtype;
+    (void)chunk;
+    take_beta_flag(dtype);
     if (B < 1 || H < 1 || T < 0) return 0;
     size_t off[5];
     return bwd_ws_layout(B, T, H, Dk, Dv, have_S_chunks != 0, off);
@@ -228,6 +246,7 @@ size_t kla_chunk_bwd_workspace_min(int B, int T, int H, int Dk, int Dv, int chun
 
 size_t kla_chunk_bwd_workspace(int B, int T, int H, int Dk, int Dv, int chunk, int dtype,
                                int have_S_chunks) {
+    take_beta_flag(dtype);
     const size_t simt = kla_chunk_bwd_workspace_min(B, T, H, Dk, Dv, chunk, dtype, have_S_chunks);
     if (!tc_bwd_shape(T, Dk, Dv, dtype)) return simt;
     const size_t tc = kla::chunk_bwd_tc_workspace(B, T, H, have_S_chunks != 0);
@@ -245,7 +264,9 @@ kla_status bwd_impl(const void* q, const void* k, const void* v, const float* et
                     void* dq, void* dk, void* dv, float* deta, float* dg, float* dS0, int B, int T, int H,
                     int Dk, int Dv, int chunk, int dtype, int out_dtype, void* ws, size_t ws_bytes,
                     void* stream, bool after_train, const char* name) {
+    const bool direct = take_beta_flag(dtype);
     kla_status st = check_common(B, T, H, Dk, Dv, chunk, dtype, out_dtype, eps);
+    const float keps = kernel_eps(eps, direct);
     if (st != KLA_OK) return st;
     REQUIRE_PTR(dS0);
     OPTIONAL_PTR(S0); OPTIONAL_PTR(dS_T); OPTIONAL_PTR(S_chunks);
@@ -269,7 +290,7 @@ kla_status bwd_impl(const void* q, const void* k, const void* v, const float* et
     if (!aligned16(ws)) return fail(KLA_ERR_INVALID_ARG, "ws must be 16-byte aligned");
     cudaError_t e;
     if (tc_bwd_path(B, T, H, Dk, Dv, dtype, ws_bytes)) {
-        kla::BwdTcArgs ta{q, k, v, eta, g, eps, S0, dO, dS_T, S_chunks, dq, dk, dv, deta, dg, dS0,
+        kla::BwdTcArgs ta{q, k, v, eta, g, keps, S0, dO, dS_T, S_chunks, dq, dk, dv, deta, dg, dS0,
                           B, T, H, out_dtype == KLA_BF16};
         e = after_train ? kla::launch_chunk_bwd_tc_reverse(ta, ws, ws_bytes, s)
                         : kla::launch_chunk_bwd_tc(ta, ws, ws_bytes, s);
@@ -283,7 +304,7 @@ kla_status bwd_impl(const void* q, const void* k, const void* v, const float* et
     if (Sc == nullptr) {
         float* Sc_ws = reinterpret_cast<float*>(w + off[0]);
         if (!after_train) {
-            kla::FwdArgs fa{q, k, v, eta, g, eps, S0, nullptr, nullptr, Sc_ws, B, T, H, Dk, Dv,
+            kla::FwdArgs fa{q, k, v, eta, g, keps, S0, nullptr, nullptr, Sc_ws, B, T, H, Dk, Dv,
                             dtype == KLA_BF16, false};
             e = kla::chunk_fwd_tc_supported(fa) ? kla::launch_chunk_fwd_tc(fa, s) : kla::launch_chunk_fwd_simt(fa, s);
             if (e != cudaSuccess) return cuda_fail(e, "kla_chunk_bwd state recompute");
@@ -292,7 +313,7 @@ kla_status bwd_impl(const void* q, const void* k, const void* v, const float* et
     }
     const size_t ntok = (size_t)B * T * H;
     float* acc3 = reinterpret_cast<float*>(w + off[3]);
-    kla::BwdArgs a{q, k, v, eta, g, eps, Sc, dO, dS_T, dq, dk, dv, deta, dg, dS0,
+    kla::BwdArgs a{q, k, v, eta, g, keps, Sc, dO, dS_T, dq, dk, dv, deta, dg, dS0,
                    reinterpret_cast<float*>(w + off[1]), reinterpret_cast<float*>(w + off[2]),
                    acc3, acc3 + ntok, acc3 + 2 * ntok, B, T, H, Dk, Dv, dtype == KLA_BF16,
                    out_dtype == KLA_BF16};
@@ -318,6 +339,7 @@ kla_status kla_chunk_fwd_train(const void* q, const void* k, const void* v, cons
                                const float* g, float eps, const float* S0, void* o, float* S_T, int B,
                                int T, int H, int Dk, int Dv, int chunk, int dtype, int out_dtype, void* ws,
                                size_t ws_bytes, void* stream) {
+    const bool direct = take_beta_flag(dtype);
     kla_status st = check_common(B, T, H, Dk, Dv, chunk, dtype, out_dtype, eps);
     if (st != KLA_OK) return st;
     if (T > 0) {
@@ -326,16 +348,16 @@ kla_status kla_chunk_fwd_train(const void* q, const void* k, const void* v, cons
     OPTIONAL_PTR(S0); OPTIONAL_PTR(o); OPTIONAL_PTR(S_T);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (T == 0)  // nothing for the backward to keep: the plain forward's empty-sequence case
-        return kla_chunk_fwd(q, k, v, eta, g, eps, S0, o, S_T, nullptr, B, T, H, Dk, Dv, chunk, dtype,
-                             out_dtype, nullptr, 0, stream);
+        return kla_chunk_fwd(q, k, v, eta, g, eps, S0, o, S_T, nullptr, B, T, H, Dk, Dv, chunk,
+                             dtype | (direct ? KLA_BETA_DIRECT : 0), out_dtype, nullptr, 0, stream);
     size_t off[5];
     const size_t need = bwd_ws_layout(B, T, H, Dk, Dv, false, off);
     if (ws == nullptr || ws_bytes < need)
         return fail(KLA_ERR_WORKSPACE, "kla_chunk_fwd_train needs %zu workspace bytes (got %zu)", need,
                     ws == nullptr ? (size_t)0 : ws_bytes);
     if (!aligned16(ws)) return fail(KLA_ERR_INVALID_ARG, "ws must be 16-byte aligned");
-    kla::FwdArgs a{q, k, v, eta, g, eps, S0, o, S_T, nullptr, B, T, H, Dk, Dv, dtype == KLA_BF16,
-                   out_dtype == KLA_BF16};
+    kla::FwdArgs a{q, k, v, eta, g, kernel_eps(eps, direct), S0, o, S_T, nullptr, B, T, H, Dk, Dv,
+                   dtype == KLA_BF16, out_dtype == KLA_BF16};
     cudaError_t e;
     if (tc_bwd_path(B, T, H, Dk, Dv, dtype, ws_bytes)) {
         e = kla::launch_chunk_fwd_train_tc(a, ws, ws_bytes, s);
@@ -360,12 +382,13 @@ kla_status kla_chunk_bwd_after_train(const void* q, const void* k, const void* v
 kla_status kla_decode_step(const void* q, const void* k, const void* v, const float* eta,
                            const float* g, float eps, float* S, void* o, int B, int H, int Dk,
                            int Dv, int dtype, int out_dtype, void* stream) {
+    const bool direct = take_beta_flag(dtype);
     kla_status st = check_common(B, 0, H, Dk, Dv, kla::kChunkLen, dtype, out_dtype, eps);
     if (st != KLA_OK) return st;
     REQUIRE_PTR(q); REQUIRE_PTR(k); REQUIRE_PTR(v); REQUIRE_PTR(eta); REQUIRE_PTR(g);
     REQUIRE_PTR(S);
     OPTIONAL_PTR(o);
-    kla::DecodeArgs a{q, k, v, eta, g, eps, S, o, B, H, Dk, Dv, dtype == KLA_BF16,
+    kla::DecodeArgs a{q, k, v, eta, g, kernel_eps(eps, direct), S, o, B, H, Dk, Dv, dtype == KLA_BF16,
                       out_dtype == KLA_BF16};
     cudaError_t e = kla::launch_decode(a, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "kla_decode_step launch");

@@ -925,8 +925,13 @@ __global__ void __launch_bounds__(GT, 1)
         float deta = 0.f, dr = 0.f;
         if (ir > 0.f) {
             const float r = r2 * ir;
-            deta = db * r2 / den + dc * r / den;
-            dr = (db * et * 2.f * r * a.eps + dc * et * (a.eps - r2)) / (den * den);
+            if (a.eps < 0.f) {  // direct: b = eta r^2, c = eta r
+                deta = db * r2 + dc * r;
+                dr = db * et * 2.f * r + dc * et;
+            } else {            // Kaczmarz: b = eta r^2 / (r^2 + eps), c = eta r / (r^2 + eps)
+                deta = db * r2 / den + dc * r / den;
+                dr = (db * et * 2.f * r * a.eps + dc * et * (a.eps - r2)) / (den * den);
+            }
         }
         ms->dr[i] = dr;
         ms->kd[i] = sum4(ms->kd_p) * ir;

@@ -690,7 +690,8 @@ __global__ void __launch_bounds__(256) bwd_finalize_kernel(BwdArgs a, size_t nto
     r2 = warp_sum(r2);
     const float r = sqrtf(r2);
     const float den = r2 + a.eps;
-    const bool live = den > 0.f && r > 0.f;
+    const bool direct = a.eps < 0.f;  // beta = eta as given: b = eta r^2, c = eta r
+    const bool live = (direct || den > 0.f) && r > 0.f;
     const float inv_r = live ? 1.f / r : 0.f;
     float kd = 0.f;
 #pragma unroll
@@ -698,7 +699,10 @@ __global__ void __launch_bounds__(256) bwd_finalize_kernel(BwdArgs a, size_t nto
     kd = warp_sum(kd);
     const float db = a.acc_db[w], dc = a.acc_dc[w], et = a.eta[w];
     float deta = 0.f, dr = 0.f;
-    if (live) {
+    if (live && direct) {
+        deta = db * r2 + dc * r;
+        dr = db * et * 2.f * r + dc * et;
+    } else if (live) {
         deta = db * r2 / den + dc * r / den;
         dr = (db * et * 2.f * r * a.eps + dc * et * (a.eps - r2)) / (den * den);
     }

@@ -203,8 +203,8 @@ __global__ void __launch_bounds__(NT, CTAS_PER_SM)
                 sk.x += a.x; sk.y += a.y; sk.z += a.z; sk.w += a.w;
                 sq.x += b.x; sq.y += b.y; sq.z += b.z; sq.w += b.w;
             }
-            const float den = n2 + eps;
-            const float beta = den > 0.f ? sm.eta[i] / den : 0.f;
+            const float den = n2 + eps;  // eps < 0: the direct write strength beta = eta
+            const float beta = eps < 0.f ? sm.eta[i] : (den > 0.f ? sm.eta[i] / den : 0.f);
             be.x = beta * (to_f32(sm.vv[st][4 * cg + 0]) - alpha * sk.x);
             be.y = beta * (to_f32(sm.vv[st][4 * cg + 1]) - alpha * sk.y);
             be.z = beta * (to_f32(sm.vv[st][4 * cg + 2]) - alpha * sk.z);

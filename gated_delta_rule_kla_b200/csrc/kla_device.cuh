@@ -33,10 +33,27 @@ __device__ __forceinline__ float warp_sum(float x) {
 struct KaczCoef {
     float b, c, inv_r;
 };
+// eps < 0 is never a Kaczmarz stabiliser (the C ABI rejects it): the library passes
+// kBetaDirect to the kernels to select the direct write strength beta = eta as given.
+constexpr float kBetaDirect = -1.f;
+// Coefficients of the unit-key form (k = r khat): the write beta k k^T = b khat khat^T and the
+// value injection beta k = c khat.  Kaczmarz (Eq. 3): beta = eta / (r^2 + eps), so
+// b = eta r^2 / (r^2 + eps), c = eta r / (r^2 + eps); direct: beta = eta, b = eta r^2, c = eta r.
+// A zero key writes nothing in either mode.
 __device__ __forceinline__ KaczCoef kacz_coef(float eta, float r2, float eps) {
     KaczCoef out;
+    const float r = sqrtf(r2);
+    if (eps < 0.f) {
+        if (r > 0.f) {
+            out.b = eta * r2;
+            out.c = eta * r;
+            out.inv_r = 1.f / r;
+        } else {
+            out.b = out.c = out.inv_r = 0.f;
+        }
+        return out;
+    }
     float den = r2 + eps;
-    float r = sqrtf(r2);
     if (den > 0.f && r > 0.f) {
         out.b = eta * r2 / den;
         out.c = eta * r / den;

@@ -7,10 +7,10 @@
  *     beta_t = eta_t / (||k_t||^2 + eps)          section 3.1, Eq. (3)
  *     alpha_t = exp(g_t)                           (g is the log-decay)
  *     Sbar = alpha_t S_{t-1};  e_t = v_t - Sbar^T k_t
- *     S_t  = Sbar + beta_t k_t e_t^T               Algorithm 1 (left panel), lines 2-5
+ *     S_t  = Sbar + beta_t k_t e_t^T               Algorithm 1 (left panel)
  *     o_t  = S_t^T q_t                             section 2 readout
  *
- * The readout uses q exactly as passed.  Algorithm 1, line 6 divides by ||q_t||; because o
+ * The readout uses q exactly as passed.  Algorithm 1's readout divides by ||q_t||; because o
  * is linear in q, a caller who wants that form passes q_t / ||q_t||.  No 1/sqrt(Dk) scale
  * and no key normalisation is applied (normalising k would turn KLA into GDN).
  * When ||k_t||^2 + eps == 0 the write is skipped (beta_t = 0); the paper is silent there.
@@ -30,7 +30,12 @@
  *     S0 to S_T).  The last chunk may be partial.  eps >= 0.  g <= 0 is the intended range
  *     (the decay factors exp(G_i - G_j) are then <= 1); g > 0 is accepted without an
  *     accuracy guarantee.
- *   - dtype selects the element type of the inputs q, k, v (and dO): KLA_F32 or KLA_BF16.
+ *   - dtype selects the element type of the inputs q, k, v (and dO): KLA_F32 or KLA_BF16,
+ *     optionally OR-ed with KLA_BETA_DIRECT.  That flag takes the write strength as given,
+ *     beta_t = eta_t (the Gated DeltaNet update, or any beta the caller computes), instead of
+ *     the Kaczmarz step beta_t = eta_t / (||k_t||^2 + eps); eps is then unused (it must still
+ *     be >= 0).  Every entry point taking dtype accepts the flag (the workspace and launch-count
+ *     queries ignore it); the backward then differentiates the direct map.
  *     out_dtype selects the element type of the outputs o (and dq, dk, dv): KLA_F32 or
  *     KLA_BF16.  eta, g, S0, S_T, S, dS_T, deta, dg, dS0 are always fp32, as is the state.
  *     Outputs are computed in fp32 and rounded once on store; with heavy-tailed outputs a
@@ -61,6 +66,9 @@ typedef enum {
 } kla_status;
 
 typedef enum { KLA_F32 = 0, KLA_BF16 = 1 } kla_dtype;
+
+/* OR into a dtype argument: beta_t = eta_t as given (see the conventions above). */
+#define KLA_BETA_DIRECT 0x100
 
 /* Static string naming a status code (never NULL). */
 const char *kla_status_string(int status);
@@ -193,7 +201,7 @@ kla_status kla_chunk_bwd_after_train(const void *q, const void *k, const void *v
                                      void *stream);
 
 /*
- * kla_decode_step -- one generated token: Algorithm 1 (left panel), lines 2-6 (readout
+ * kla_decode_step -- one generated token: Algorithm 1 (left panel), update and readout (readout
  * without the 1/||q|| factor, as above), for every (b, h) at once.
  *
  *   q, k    in     [B,H,Dk] of `dtype`      v   in  [B,H,Dv] of `dtype`

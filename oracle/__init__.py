@@ -41,6 +41,12 @@ def _check(rc, name):
         raise RuntimeError(f"{name} failed with code {rc}")
 
 
+def _direct(beta):
+    if beta not in ("kaczmarz", "direct"):
+        raise ValueError(f"beta must be 'kaczmarz' or 'direct', got {beta!r}")
+    return 1 if beta == "direct" else 0
+
+
 class OracleLib:
     """ctypes view of one build of kla_oracle.c."""
 
@@ -49,19 +55,22 @@ class OracleLib:
         dp = ctypes.POINTER(ctypes.c_double)
         i = ctypes.c_int
         d = ctypes.c_double
-        lib.kla_oracle_forward.argtypes = [i, i, i, i, i, dp, dp, dp, dp, dp, d, dp, dp, dp]
-        lib.kla_oracle_decode_step.argtypes = [i, i, i, i, dp, dp, dp, dp, dp, d, dp, dp]
-        lib.kla_oracle_backward.argtypes = [i, i, i, i, i, dp, dp, dp, dp, dp, d, dp, dp, dp,
+        # each takes `int direct` after eps: beta_t = eta_t as given instead of Eq. (3)
+        lib.kla_oracle_forward.argtypes = [i, i, i, i, i, dp, dp, dp, dp, dp, d, i, dp, dp, dp]
+        lib.kla_oracle_decode_step.argtypes = [i, i, i, i, dp, dp, dp, dp, dp, d, i, dp, dp]
+        lib.kla_oracle_backward.argtypes = [i, i, i, i, i, dp, dp, dp, dp, dp, d, i, dp, dp, dp,
                                             dp, dp, dp, dp, dp, dp, i]
-        lib.kla_oracle_chunk_forward.argtypes = [i, i, i, i, i, dp, dp, dp, dp, dp, d, dp, i, dp, dp]
+        lib.kla_oracle_chunk_forward.argtypes = [i, i, i, i, i, dp, dp, dp, dp, dp, d, i, dp, i, dp, dp]
         for f in (lib.kla_oracle_forward, lib.kla_oracle_decode_step, lib.kla_oracle_backward,
                   lib.kla_oracle_chunk_forward):
             f.restype = ctypes.c_int
         self.lib = lib
         self.path = path
 
-    def forward(self, q, k, v, eta, g, eps, S0=None):
+    def forward(self, q, k, v, eta, g, eps, S0=None, beta="kaczmarz"):
         """Token recurrence. q,k [B,T,H,Dk]; v [B,T,H,Dv]; eta,g [B,T,H]; S0 [B,H,Dk,Dv].
+        beta="direct" takes beta_t = eta_t as given (the Gated DeltaNet update) instead of
+        Eq. (3); the other methods take the same keyword.
 
         Returns (o [B,T,H,Dv], S_T [B,H,Dk,Dv]) in float64.
         """
@@ -71,11 +80,11 @@ class OracleLib:
         o = np.zeros((B, T, H, Dv))
         ST = np.zeros((B, H, Dk, Dv))
         rc = self.lib.kla_oracle_forward(B, T, H, Dk, Dv, _ptr(q), _ptr(k), _ptr(v), _ptr(eta),
-                                         _ptr(g), float(eps), _ptr(S0), _ptr(o), _ptr(ST))
+                                         _ptr(g), float(eps), _direct(beta), _ptr(S0), _ptr(o), _ptr(ST))
         _check(rc, "kla_oracle_forward")
         return o, ST
 
-    def decode_step(self, q, k, v, eta, g, eps, S):
+    def decode_step(self, q, k, v, eta, g, eps, S, beta="kaczmarz"):
         """One token step per head. q,k [B,H,Dk]; v [B,H,Dv]; eta,g [B,H]; S [B,H,Dk,Dv].
 
         Returns (o [B,H,Dv], S_new) without modifying the argument S.
@@ -86,11 +95,11 @@ class OracleLib:
         Dv = v.shape[-1]
         o = np.zeros((B, H, Dv))
         rc = self.lib.kla_oracle_decode_step(B, H, Dk, Dv, _ptr(q), _ptr(k), _ptr(v), _ptr(eta),
-                                             _ptr(g), float(eps), _ptr(S), _ptr(o))
+                                             _ptr(g), float(eps), _direct(beta), _ptr(S), _ptr(o))
         _check(rc, "kla_oracle_decode_step")
         return o, S
 
-    def backward(self, q, k, v, eta, g, eps, S0, dO, dS_T=None, ckpt=64):
+    def backward(self, q, k, v, eta, g, eps, S0, dO, dS_T=None, ckpt=64, beta="kaczmarz"):
         """Gradients of <o, dO> + <S_T, dS_T> w.r.t. every input.
 
         Returns a dict with dq, dk, dv, deta, dg, dS0 (float64).
@@ -101,14 +110,14 @@ class OracleLib:
         out = dict(dq=np.zeros((B, T, H, Dk)), dk=np.zeros((B, T, H, Dk)), dv=np.zeros((B, T, H, Dv)),
                    deta=np.zeros((B, T, H)), dg=np.zeros((B, T, H)), dS0=np.zeros((B, H, Dk, Dv)))
         rc = self.lib.kla_oracle_backward(B, T, H, Dk, Dv, _ptr(q), _ptr(k), _ptr(v), _ptr(eta),
-                                          _ptr(g), float(eps), _ptr(S0), _ptr(dO), _ptr(dS_T),
+                                          _ptr(g), float(eps), _direct(beta), _ptr(S0), _ptr(dO), _ptr(dS_T),
                                           _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]),
                                           _ptr(out["deta"]), _ptr(out["dg"]), _ptr(out["dS0"]),
                                           int(ckpt))
         _check(rc, "kla_oracle_backward")
         return out
 
-    def chunk_forward(self, q, k, v, eta, g, eps, S0=None, chunk=64):
+    def chunk_forward(self, q, k, v, eta, g, eps, S0=None, chunk=64, beta="kaczmarz"):
         """Chunkwise form (Eqs. 7-9) in fp64; used only to cross-check `forward`."""
         q, k, v, eta, g, S0 = map(_f64, (q, k, v, eta, g, S0))
         B, T, H, Dk = k.shape
@@ -116,7 +125,7 @@ class OracleLib:
         o = np.zeros((B, T, H, Dv))
         ST = np.zeros((B, H, Dk, Dv))
         rc = self.lib.kla_oracle_chunk_forward(B, T, H, Dk, Dv, _ptr(q), _ptr(k), _ptr(v), _ptr(eta),
-                                               _ptr(g), float(eps), _ptr(S0), int(chunk), _ptr(o),
+                                               _ptr(g), float(eps), _direct(beta), _ptr(S0), int(chunk), _ptr(o),
                                                _ptr(ST))
         _check(rc, "kla_oracle_chunk_forward")
         return o, ST

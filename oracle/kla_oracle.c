@@ -18,6 +18,11 @@
  *     Kaczmarz", section 2, writes alpha_t = exp(g_t)).
  *     If ||k_t||^2 + eps == 0 the write is skipped (beta_t = 0); the paper is
  *     silent on that case.
+ *     With direct != 0 every function takes the write strength as given,
+ *     beta_t = eta_t: the Gated DeltaNet update that the paper starts from
+ *     (section 3.3 contrasts its beta with the Kaczmarz step; the blog "From
+ *     Gated DeltaNet to Kaczmarz" writes the same recurrence with a learned
+ *     beta); eps is then unused.
  *   - kla_oracle_backward: reverse-mode differentiation of the same token
  *     recurrence.  The paper gives no backward; this one is derived by hand
  *     from the forward above (chain rule, one token at a time, newest first)
@@ -41,8 +46,10 @@
 #define IDX_GATE(b, t, h, T, H) (((size_t)(b) * (T) + (t)) * (H) + (h))
 #define IDX_STATE(b, h, H, Dk, Dv) (((size_t)(b) * (H) + (h)) * (size_t)(Dk) * (Dv))
 
-/* Eq. (3): beta = eta / (||k||^2 + eps); zero when the denominator is zero. */
-static double kaczmarz_beta(double eta, double knorm2, double eps) {
+/* Eq. (3): beta = eta / (||k||^2 + eps); zero when the denominator is zero.
+ * direct: beta = eta (the Gated DeltaNet write strength). */
+static double kaczmarz_beta(double eta, double knorm2, double eps, int direct) {
+    if (direct) return eta;
     double den = knorm2 + eps;
     return den != 0.0 ? eta / den : 0.0;
 }
@@ -50,11 +57,11 @@ static double kaczmarz_beta(double eta, double knorm2, double eps) {
 /* One tokenwise step of Algorithm 1 (left panel), in place on S (Dk x Dv).
  * e (length Dv) is scratch.  Writes o (length Dv) when o != NULL. */
 static void token_step(double *S, const double *q, const double *k, const double *v, double eta,
-                       double g, double eps, int Dk, int Dv, double *e, double *o) {
+                       double g, double eps, int direct, int Dk, int Dv, double *e, double *o) {
     double alpha = exp(g);
     double n = 0.0;
     for (int i = 0; i < Dk; ++i) n += k[i] * k[i];
-    double beta = kaczmarz_beta(eta, n, eps);
+    double beta = kaczmarz_beta(eta, n, eps, direct);
     /* Sbar = alpha S */
     for (size_t x = 0; x < (size_t)Dk * Dv; ++x) S[x] *= alpha;
     /* e = v - Sbar^T k */
@@ -82,7 +89,7 @@ static void gather_token(const double *src, int b, int t, int h, int T, int H, i
 }
 
 int kla_oracle_forward(int B, int T, int H, int Dk, int Dv, const double *q, const double *k,
-                       const double *v, const double *eta, const double *g, double eps,
+                       const double *v, const double *eta, const double *g, double eps, int direct,
                        const double *S0, double *o, double *S_T) {
     if (B < 0 || T < 0 || H < 0 || Dk <= 0 || Dv <= 0) return 1;
     int npairs = B * H;
@@ -109,7 +116,7 @@ int kla_oracle_forward(int B, int T, int H, int Dk, int Dv, const double *q, con
                 gather_token(k, b, t, h, T, H, Dk, kt);
                 gather_token(v, b, t, h, T, H, Dv, vt);
                 size_t gi = IDX_GATE(b, t, h, T, H);
-                token_step(S, qt, kt, vt, eta[gi], g[gi], eps, Dk, Dv, e, ot);
+                token_step(S, qt, kt, vt, eta[gi], g[gi], eps, direct, Dk, Dv, e, ot);
                 if (o) memcpy(o + IDX_TOK(b, t, h, 0, T, H, Dv), ot, sizeof(double) * (size_t)Dv);
             }
             if (S_T) memcpy(S_T + IDX_STATE(b, h, H, Dk, Dv), S, sizeof(double) * (size_t)Dk * Dv);
@@ -122,7 +129,7 @@ int kla_oracle_forward(int B, int T, int H, int Dk, int Dv, const double *q, con
 /* One decode step: Algorithm 1 (left panel) once per (b, h), S updated in place.
  * q, k: [B, H, Dk]; v, o: [B, H, Dv]; eta, g: [B, H]; S: [B, H, Dk, Dv]. */
 int kla_oracle_decode_step(int B, int H, int Dk, int Dv, const double *q, const double *k,
-                           const double *v, const double *eta, const double *g, double eps,
+                           const double *v, const double *eta, const double *g, double eps, int direct,
                            double *S, double *o) {
     if (B < 0 || H < 0 || Dk <= 0 || Dv <= 0) return 1;
     int npairs = B * H;
@@ -136,7 +143,7 @@ int kla_oracle_decode_step(int B, int H, int Dk, int Dv, const double *q, const 
             continue;
         }
         token_step(S + (size_t)p * Dk * Dv, q + (size_t)p * Dk, k + (size_t)p * Dk,
-                   v + (size_t)p * Dv, eta[p], g[p], eps, Dk, Dv, e, o ? o + (size_t)p * Dv : NULL);
+                   v + (size_t)p * Dv, eta[p], g[p], eps, direct, Dk, Dv, e, o ? o + (size_t)p * Dv : NULL);
         free(e);
     }
     return bad ? 2 : 0;
@@ -152,6 +159,7 @@ int kla_oracle_decode_step(int B, int H, int Dk, int Dv, const double *q, const 
  *   dv     = de                            (e = v - Sbar^T k)
  *   dn     = -dbeta * beta / (n + eps)     (n = ||k||^2)
  *   deta   = dbeta / (n + eps)
+ *   (direct: beta = eta, so dn = 0 and deta = dbeta)
  *   dk     = beta G e - Sbar de + 2 k dn
  *   dSbar  = G - k de^T
  *   dg     = alpha <dSbar, S_{t-1}>_F      (Sbar = exp(g) S_{t-1})
@@ -161,7 +169,7 @@ int kla_oracle_decode_step(int B, int H, int Dk, int Dv, const double *q, const 
  * States S_{t-1} are recomputed from checkpoints taken every `ckpt` tokens.
  */
 int kla_oracle_backward(int B, int T, int H, int Dk, int Dv, const double *q, const double *k,
-                        const double *v, const double *eta, const double *g, double eps,
+                        const double *v, const double *eta, const double *g, double eps, int direct,
                         const double *S0, const double *dO, const double *dS_T, double *dq,
                         double *dk, double *dv, double *deta, double *dg, double *dS0,
                         int ckpt) {
@@ -198,7 +206,7 @@ int kla_oracle_backward(int B, int T, int H, int Dk, int Dv, const double *q, co
                     gather_token(k, b, t, h, T, H, Dk, kt);
                     gather_token(v, b, t, h, T, H, Dv, vt);
                     size_t gi = IDX_GATE(b, t, h, T, H);
-                    token_step(S, qt, kt, vt, eta[gi], g[gi], eps, Dk, Dv, e, NULL);
+                    token_step(S, qt, kt, vt, eta[gi], g[gi], eps, direct, Dk, Dv, e, NULL);
                 }
             }
             if (dS_T) memcpy(G, dS_T + IDX_STATE(b, h, H, Dk, Dv), sizeof(double) * SS);
@@ -215,7 +223,7 @@ int kla_oracle_backward(int B, int T, int H, int Dk, int Dv, const double *q, co
                     gather_token(k, b, t, h, T, H, Dk, kt);
                     gather_token(v, b, t, h, T, H, Dv, vt);
                     size_t gi = IDX_GATE(b, t, h, T, H);
-                    token_step(Sn, qt, kt, vt, eta[gi], g[gi], eps, Dk, Dv, e, NULL);
+                    token_step(Sn, qt, kt, vt, eta[gi], g[gi], eps, direct, Dk, Dv, e, NULL);
                 }
                 for (int t = t1 - 1; t >= t0; --t) {
                     const double *Sprev = blk + (size_t)(t - t0) * SS;
@@ -229,7 +237,7 @@ int kla_oracle_backward(int B, int T, int H, int Dk, int Dv, const double *q, co
                     double n = 0.0;
                     for (int i = 0; i < Dk; ++i) n += kt[i] * kt[i];
                     double den = n + eps;
-                    double beta = kaczmarz_beta(eta[gi], n, eps);
+                    double beta = kaczmarz_beta(eta[gi], n, eps, direct);
                     /* e = v - Sbar^T k, Sbar = alpha S_{t-1} */
                     for (int j = 0; j < Dv; ++j) {
                         double s = 0.0;
@@ -254,7 +262,9 @@ int kla_oracle_backward(int B, int T, int H, int Dk, int Dv, const double *q, co
                         dbeta += s * e[j];
                     }
                     double dn = 0.0, detat = 0.0;
-                    if (den != 0.0) {
+                    if (direct) {
+                        detat = dbeta;
+                    } else if (den != 0.0) {
                         dn = -dbeta * beta / den;
                         detat = dbeta / den;
                     }
@@ -308,7 +318,7 @@ int kla_oracle_backward(int B, int T, int H, int Dk, int Dv, const double *q, co
  */
 int kla_oracle_chunk_forward(int B, int T, int H, int Dk, int Dv, const double *q,
                              const double *k, const double *v, const double *eta,
-                             const double *g, double eps, const double *S0, int C, double *o,
+                             const double *g, double eps, int direct, const double *S0, int C, double *o,
                              double *S_T) {
     if (B < 0 || T < 0 || H < 0 || Dk <= 0 || Dv <= 0 || C <= 0) return 1;
     int npairs = B * H;
@@ -347,7 +357,7 @@ int kla_oracle_chunk_forward(int B, int T, int H, int Dk, int Dv, const double *
                     gprev = gam[i];
                     double kn = 0.0;
                     for (int x = 0; x < Dk; ++x) kn += K[(size_t)i * Dk + x] * K[(size_t)i * Dk + x];
-                    bet[i] = kaczmarz_beta(eta[gi], kn, eps);
+                    bet[i] = kaczmarz_beta(eta[gi], kn, eps, direct);
                 }
                 /* strictly lower L = B (A^- o K K^T), stored in Mx */
                 for (int i = 0; i < n; ++i)

@@ -576,3 +576,87 @@ def test_bwd_empty_sequence(kla):
     gr = kla.chunk_bwd(z, z, z, gz, gz, z, 1e-6, None, dST)
     torch.cuda.synchronize()
     torch.testing.assert_close(gr["dS0"], dST, rtol=0, atol=0)
+
+
+# ---------------------------------------------------------------------------------------
+# direct write strength: beta_t = eta_t as given (the Gated DeltaNet update), selected by
+# KLA_BETA_DIRECT in the dtype argument (beta="direct" in the binding)
+# ---------------------------------------------------------------------------------------
+def direct_eta(inp):
+    """A direct write strength that keeps every write a contraction for these keys:
+    beta_t = eta_t / (||k_t||^2 + 1), computed on the CPU from the rounded keys."""
+    k = inp["k"].double()
+    return (inp["eta"].double() / ((k * k).sum(-1) + 1.0)).float()
+
+
+@pytest.mark.parametrize("B,T,H,Dk,Dv,dtype,fused", [
+    (1, 150, 2, 128, 128, "bf16", False),   # split path (preparation + state pass)
+    (2, 130, 3, 128, 128, "bf16", True),    # fused one-kernel-per-head path
+    (8, 1024, 8, 128, 128, "bf16", False),  # two slabs
+    (1, 100, 2, 64, 128, "f32", False),     # CUDA-core path
+])
+def test_fwd_direct_beta_matches_oracle(kla, oracle_mod, B, T, H, Dk, Dv, dtype, fused):
+    inp = small_inputs(B, T, H, Dk, Dv, dtype, seed=T + 5 * H, g_lo=-0.2)
+    inp["eta"] = direct_eta(inp)
+    d = {k: (v.cuda() if v is not None else None) for k, v in inp.items()}
+    o, ST = kla.chunk_fwd(d["q"], d["k"], d["v"], d["eta"], d["g"], 1e-6, d["S0"], fused=fused, beta="direct")
+    torch.cuda.synchronize()
+    kla.check_device_error()
+    ro, rST = oracle_mod.forward(*(np64(inp[k]) for k in ("q", "k", "v", "eta", "g")), 1e-6, np64(inp["S0"]),
+                                 beta="direct")
+    assert rel_err(o, ro) <= TOL[dtype]
+    assert rel_err(ST, rST) <= TOL[dtype]
+
+
+def test_direct_beta_with_kaczmarz_eta_equals_kaczmarz(kla):
+    """beta="direct" fed eta / (||k||^2 + eps) is the Kaczmarz forward (split path, bf16)."""
+    inp = small_inputs(2, 300, 3, 128, 128, "bf16", seed=77)
+    d = {k: (v.cuda() if v is not None else None) for k, v in inp.items()}
+    eps = 1e-3
+    kk = d["k"].float()
+    eta_d = (d["eta"] / ((kk * kk).sum(-1) + eps)).contiguous()
+    o1, S1 = kla.chunk_fwd(d["q"], d["k"], d["v"], d["eta"], d["g"], eps, d["S0"])
+    o2, S2 = kla.chunk_fwd(d["q"], d["k"], d["v"], eta_d, d["g"], eps, d["S0"], beta="direct")
+    torch.cuda.synchronize()
+    assert rel_err(o2, np64(o1)) <= 1e-3
+    assert rel_err(S2, np64(S1)) <= 1e-3
+
+
+@pytest.mark.parametrize("B,T,H,Dk,Dv,dtype", [(1, 150, 2, 128, 128, "bf16"), (1, 97, 2, 64, 64, "f32")])
+def test_bwd_direct_beta_matches_oracle(kla, oracle_mod, B, T, H, Dk, Dv, dtype):
+    """Both backward paths (tensor cores with the default workspace for bf16 d = 128, CUDA
+    cores otherwise or with the minimum workspace) in the direct mode."""
+    inp = small_inputs(B, T, H, Dk, Dv, dtype, seed=T + 9 * H, g_lo=-0.2)
+    inp["eta"] = direct_eta(inp)
+    gen = torch.Generator().manual_seed(T + 2)
+    dO = torch.randn(B, T, H, Dv, generator=gen).to(inp["q"].dtype)
+    dST = torch.randn(B, H, Dk, Dv, generator=gen)
+    d = {k: (v.cuda() if v is not None else None) for k, v in inp.items()}
+    args = (d["q"], d["k"], d["v"], d["eta"], d["g"], dO.cuda(), 1e-6, d["S0"], dST.cuda())
+    runs = {"default": kla.chunk_bwd(*args, beta="direct"),
+            "cuda cores": kla.chunk_bwd(*args, cuda_cores=True, beta="direct")}
+    torch.cuda.synchronize()
+    kla.check_device_error()
+    ref = oracle_mod.backward(*(np64(inp[k]) for k in ("q", "k", "v", "eta", "g")), 1e-6, np64(inp["S0"]),
+                              np64(dO), np64(dST), beta="direct")
+    for path, gr in runs.items():
+        for name in GRADS:
+            assert rel_err(gr[name], ref[name]) <= TOL[dtype], (path, name)
+
+
+@pytest.mark.parametrize("Dk,Dv,dtype", [(128, 128, "bf16"), (64, 128, "f32")])
+def test_decode_direct_beta_matches_oracle(kla, oracle_mod, Dk, Dv, dtype):
+    w = Workload("dec", "decode", B=3, T=12, H=5, Dk=Dk, Dv=Dv, dtype=dtype, key_mode="scaled",
+                 gate_mode="uniform", s0="normal", seed=Dk + 2 * Dv)
+    inp = make_inputs(w)
+    kk = inp["k"].double()
+    eta = (inp["eta"].double() / ((kk * kk).sum(-1) + 1.0)).float()
+    S = inp["S0"].cuda().clone()
+    Sref = np64(inp["S0"])
+    for t in range(w.T):
+        o = kla.decode_step(inp["q"][t].cuda(), inp["k"][t].cuda(), inp["v"][t].cuda(), eta[t].cuda(),
+                            inp["g"][t].cuda(), S, w.eps, beta="direct")
+        ro, Sref = oracle_mod.decode_step(np64(inp["q"][t]), np64(inp["k"][t]), np64(inp["v"][t]), np64(eta[t]),
+                                          np64(inp["g"][t]), w.eps, Sref, beta="direct")
+        assert rel_err(o, ro) <= TOL[dtype]
+    assert rel_err(S, Sref) <= TOL[dtype]

@@ -36,6 +36,16 @@ def _backward_pins(mod):
         yield lambda T=T, ck=ck, eps=eps: pins.test_backward_finite_differences(mod, T, ck, eps)
 
 
+def _direct_pins(mod):
+    yield lambda: pins.test_direct_mode_with_kaczmarz_eta_equals_kaczmarz_mode(mod)
+    yield lambda: pins.test_direct_mode_inverse_norm_beta_projects(mod)
+
+
+def _direct_backward_pins(mod):
+    for T, ck in ((7, 3), (5, 64)):
+        yield lambda T=T, ck=ck: pins.test_direct_backward_finite_differences(mod, T, ck)
+
+
 def _chunk_pins(mod):
     for C in (2, 3, 8, 64):
         yield lambda C=C: pins.test_chunk_form_matches_token_form(mod, C)
@@ -49,8 +59,15 @@ MUTATIONS = [
      "for (int j = 0; j < Dv; ++j) S[(size_t)i * Dv + j] -= beta * k[i] * e[j];", _forward_pins),
     ("readout_transposed", "for (int i = 0; i < Dk; ++i) s += S[(size_t)i * Dv + j] * q[i];",
      "for (int i = 0; i < Dk; ++i) s += S[(size_t)j * Dk + i] * q[i];", _forward_pins),
-    ("beta_uses_norm_not_square", "double beta = kaczmarz_beta(eta, n, eps);",
-     "double beta = kaczmarz_beta(eta, sqrt(n), eps);", _forward_pins),
+    ("beta_uses_norm_not_square", "double beta = kaczmarz_beta(eta, n, eps, direct);",
+     "double beta = kaczmarz_beta(eta, sqrt(n), eps, direct);", _forward_pins),
+    ("direct_mode_normalises_anyway", "    if (direct) return eta;",
+     "    if (direct) return eta / (knorm2 + 1.0);", _direct_pins),
+    ("bwd_direct_deta_halved", "                        detat = dbeta;\n",
+     "                        detat = 0.5 * dbeta;\n", _direct_backward_pins),
+    ("bwd_direct_keeps_norm_term", "                        detat = dbeta;\n",
+     "                        detat = dbeta;\n                        dn = -dbeta * beta / den;\n",
+     _direct_backward_pins),
     ("bwd_dk_drops_norm_term", "dkt[i] = beta * s - Sbde[i] + 2.0 * kt[i] * dn;",
      "dkt[i] = beta * s - Sbde[i];", _backward_pins),
     ("bwd_dg_drops_alpha", "dgt *= alpha;", "dgt *= 1.0;", _backward_pins),

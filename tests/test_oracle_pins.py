@@ -401,3 +401,76 @@ def test_backward_without_dST_and_zero_S0(oracle_mod):
     # o is linear in q, so <dq, q> = <o, dO> exactly
     o, _ = oracle_mod.forward(q, k, v, eta, g, 1e-3, None)
     assert abs(np.sum(g1["dq"] * q) - np.sum(o * dO)) <= 1e-12 * max(1.0, abs(np.sum(o * dO)))
+
+
+# ---------------------------------------------------------------------------------------
+# Direct write strength (beta_t = eta_t as given: the Gated DeltaNet update KLA starts
+# from, section 3.3).  Pinned against the Kaczmarz mode, which the pins above fix:
+#   direct(eta' = eta / (||k||^2 + eps)) == Kaczmarz(eta), token by token.
+# ---------------------------------------------------------------------------------------
+def test_direct_mode_with_kaczmarz_eta_equals_kaczmarz_mode(oracle_mod):
+    rng = np.random.default_rng(300)
+    q, k, v, eta, g, S0 = _rand_inputs(rng, 2, 11, 3, 5, 4, key_lo=0.1, key_hi=10.0)
+    for eps in (0.0, 1e-3, 0.7):
+        n = np.sum(k * k, axis=-1)
+        o1, S1 = oracle_mod.forward(q, k, v, eta, g, eps, S0)
+        o2, S2 = oracle_mod.forward(q, k, v, eta / (n + eps), g, 123.0, S0, beta="direct")  # eps unused
+        np.testing.assert_allclose(o2, o1, rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(S2, S1, rtol=1e-12, atol=1e-12)
+        c1, cS1 = oracle_mod.chunk_forward(q, k, v, eta / (n + eps), g, 5.0, S0, chunk=4, beta="direct")
+        np.testing.assert_allclose(c1, o1, rtol=1e-10, atol=1e-11)
+        np.testing.assert_allclose(cS1, S1, rtol=1e-10, atol=1e-11)
+
+
+# Gated DeltaNet as a projection: with beta_t = 1 / ||k_t||^2 the write is the exact
+# projection S_t^T k_t = v_t (Theorem 1 read for GDN), for any decay.
+def test_direct_mode_inverse_norm_beta_projects(oracle_mod):
+    rng = np.random.default_rng(301)
+    q, k, v, _, g, S0 = _rand_inputs(rng, 2, 10, 2, 6, 3, key_lo=0.2, key_hi=5.0, g_lo=-1.5)
+    beta = 1.0 / np.sum(k * k, axis=-1)
+    S = S0.copy()
+    for t in range(k.shape[1]):
+        _, S = oracle_mod.decode_step(q[:, t], k[:, t], v[:, t], beta[:, t], g[:, t], 0.0, S, beta="direct")
+        readout = np.einsum("bhij,bhi->bhj", S, k[:, t])
+        np.testing.assert_allclose(readout, v[:, t], rtol=0, atol=1e-12 * (1 + np.abs(v[:, t]).max()))
+
+
+def test_direct_decode_step_equals_forward_T1(oracle_mod):
+    rng = np.random.default_rng(302)
+    q, k, v, eta, g, S0 = _rand_inputs(rng, 2, 1, 3, 4, 5)
+    o, ST = oracle_mod.forward(q, k, v, eta, g, 1e-6, S0, beta="direct")
+    o2, S2 = oracle_mod.decode_step(q[:, 0], k[:, 0], v[:, 0], eta[:, 0], g[:, 0], 1e-6, S0, beta="direct")
+    np.testing.assert_array_equal(o[:, 0], o2)
+    np.testing.assert_array_equal(ST, S2)
+
+
+@pytest.mark.parametrize("T,ckpt", [(7, 3), (5, 64)])
+def test_direct_backward_finite_differences(oracle_mod, T, ckpt):
+    rng = np.random.default_rng(310 + T)
+    B, H, Dk, Dv = 1, 2, 3, 4
+    q, k, v, eta, g, S0 = _rand_inputs(rng, B, T, H, Dk, Dv, key_lo=0.5, key_hi=1.5, s0=0.5)
+    eta = 0.3 * eta  # beta = eta as given: keep the writes contractive for these key norms
+    dO = rng.standard_normal((B, T, H, Dv))
+    dST = rng.standard_normal((B, H, Dk, Dv))
+    grads = oracle_mod.backward(q, k, v, eta, g, 0.0, S0, dO, dST, ckpt=ckpt, beta="direct")
+    args = dict(q=q, k=k, v=v, eta=eta, g=g, S0=S0)
+
+    def loss(a):
+        o, ST = oracle_mod.forward(a["q"], a["k"], a["v"], a["eta"], a["g"], 0.0, a["S0"], beta="direct")
+        return float(np.sum(o * dO) + np.sum(ST * dST))
+
+    hstep = 1e-6
+    for name in args:
+        x = args[name]
+        fd = np.zeros_like(x)
+        it = np.nditer(x, flags=["multi_index"])
+        for _ in it:
+            idx = it.multi_index
+            a_p = {kk: vv.copy() for kk, vv in args.items()}
+            a_m = {kk: vv.copy() for kk, vv in args.items()}
+            a_p[name][idx] += hstep
+            a_m[name][idx] -= hstep
+            fd[idx] = (loss(a_p) - loss(a_m)) / (2 * hstep)
+        got = grads["d" + name]
+        err = np.abs(got - fd).max() / max(np.abs(fd).max(), 1e-3)
+        assert err <= 1e-6, (name, err)
