@@ -378,22 +378,51 @@ def bench_decode(kla, WORKLOADS, make_inputs, dev, stream, flush, rank, world, h
     S_sets[0].copy_(inp["S0"].to(dev))
     torch.cuda.synchronize()
     barrier(world)
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
-    for t in range(steps):
-        tok = t // NSETS
-        evs[t][0].record(stream)
-        kla.decode_step(q[tok], k[tok], v[tok], eta[tok], g[tok], S_sets[t % NSETS], w.eps, o=o)
-        evs[t][1].record(stream)
+
+    def all_steps():
+        for t in range(steps):
+            tok = t // NSETS
+            kla.decode_step(q[tok], k[tok], v[tok], eta[tok], g[tok], S_sets[t % NSETS], w.eps, o=o)
+
+    # The steps are captured once in a CUDA graph and replayed, as a serving loop would run
+    # them: one host launch per step costs about as much as the step itself, so timed eagerly
+    # the number would follow the host CPU.  Events bracket the whole replay.
+    timing = "one CUDA graph of every step, events around the replay"
+    try:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=torch.cuda.Stream(dev)):  # captured off the default stream
+            all_steps()
+    except Exception as exc:  # capture unavailable: per-step events on eager launches
+        graph, timing = None, f"per-step events on eager launches (graph capture failed: {type(exc).__name__})"
+    for S_, S0_ in zip(S_sets, [inp["S0"]] * NSETS):
+        S_.copy_(S0_.to(dev))
     torch.cuda.synchronize()
     barrier(world)
-    ms = [a.elapsed_time(b) for a, b in evs]
+    if graph is not None:
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ev0.record(stream)
+        graph.replay()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        ms = [ev0.elapsed_time(ev1) / steps] * steps
+        del graph
+    else:
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        for t in range(steps):
+            tok = t // NSETS
+            evs[t][0].record(stream)
+            kla.decode_step(q[tok], k[tok], v[tok], eta[tok], g[tok], S_sets[t % NSETS], w.eps, o=o)
+            evs[t][1].record(stream)
+        torch.cuda.synchronize()
+        ms = [a.elapsed_time(b) for a, b in evs]
+    barrier(world)
     total_ms = max_over_ranks(sum(ms), world)
     tokens = sum_over_ranks(float(w.B), world) * steps
     mean_s = statistics.mean(ms) / 1e3
     alg = decode_bytes(w.B, w.H, w.Dk, w.Dv, q.element_size())
     gbs = alg / mean_s / 1e9
     return {"workload": w.name, "value": tokens / (total_ms / 1e3), "unit": "tokens/s",
-            "steps": steps, "us_per_step": total_ms * 1e3 / steps, "gpu_launches": steps,
+            "steps": steps, "us_per_step": total_ms * 1e3 / steps, "gpu_launches": steps, "timing": timing,
             "l2": "inputs larger than L2 (4 sequence groups' states cycled, 268 MB)",
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s",
                          "frac": gbs / hbm_peak, "alg_bytes_per_launch": alg,
