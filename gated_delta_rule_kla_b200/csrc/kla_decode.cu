@@ -102,6 +102,12 @@ __global__ void __launch_bounds__(NT, CTAS_PER_SM)
         fence_mbar_init();
         prefetch_tmap(&tm_s);
     }
+    // Launched with programmatic stream serialization: the set-up above touches only shared
+    // memory, so it may overlap the previous kernel's tail; the state, inputs and gates it
+    // produced are read only after this wait.  The next step may then be scheduled (it waits in
+    // the same way for this one to finish).
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     // one thread requests unit number i of this CTA into stage i % STAGES
     auto request = [&](int i) {
         const int u = blockIdx.x + i * stride;
@@ -295,10 +301,19 @@ cudaError_t launch_decode_t(const DecodeArgs& a, cudaStream_t st) {
     cudaError_t e = cudaFuncSetAttribute(decode_step_kernel<DK, DV, Tin, TOut>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    decode_step_kernel<DK, DV, Tin, TOut><<<grid, NT, smem, st>>>(
-        ms, static_cast<const Tin*>(a.q), static_cast<const Tin*>(a.k), static_cast<const Tin*>(a.v), a.eta, a.g,
-        a.eps, a.S, static_cast<TOut*>(a.o), units);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(NT);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // overlap the previous kernel's tail
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, decode_step_kernel<DK, DV, Tin, TOut>, ms, static_cast<const Tin*>(a.q),
+                              static_cast<const Tin*>(a.k), static_cast<const Tin*>(a.v), a.eta, a.g, a.eps, a.S,
+                              static_cast<TOut*>(a.o), units);
 }
 
 template <int DK, int DV, typename Tin>
