@@ -18,8 +18,9 @@ import os
 
 import torch
 
-__all__ = ["lib", "chunk_fwd", "chunk_bwd", "chunk_fwd_train", "chunk_bwd_after_train", "train_workspace",
-           "decode_step", "check_device_error", "KLAError", "CHUNK",
+__all__ = ["lib", "chunk_fwd", "chunk_fwd_prep", "chunk_fwd_state", "fwd_workspace", "fwd_kernel_launches",
+           "chunk_bwd", "chunk_fwd_train", "chunk_bwd_after_train", "train_workspace",
+           "decode_step", "check_device_error", "KLAError", "CHUNK", "KLA_BETA_DIRECT",
            "library_path"]
 
 CHUNK = 64
