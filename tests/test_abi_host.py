@@ -146,3 +146,39 @@ def test_train_pair_rejects_before_launch(L):
     assert fwd(q=None) == INVALID and fwd(ws=MISALIGNED) == INVALID and fwd(Dk=96) == UNSUPPORTED
     assert bwd(ws=None) == WORKSPACE and b"kla_chunk_bwd_after_train" in L.kla_last_error()
     assert bwd(dO=None) == INVALID and bwd(n=small - 1) == WORKSPACE
+
+
+DIRECT = 0x100  # KLA_BETA_DIRECT
+
+
+def test_direct_beta_flag_is_stripped_and_still_validated(L):
+    """KLA_BETA_DIRECT rides in dtype: the queries ignore it, the entry points accept it with
+    a valid element type, and validation (element type, eps >= 0) still applies."""
+    for B, T, H in [(8, 2048, 8), (2, 300, 3), (1, 65536, 16)]:
+        assert L.kla_chunk_fwd_workspace(B, T, H, 128, 128, 64, 1 | DIRECT) == \
+            L.kla_chunk_fwd_workspace(B, T, H, 128, 128, 64, 1)
+        assert L.kla_chunk_fwd_kernel_launches(B, T, H, 128, 128, 64, 1 | DIRECT) == \
+            L.kla_chunk_fwd_kernel_launches(B, T, H, 128, 128, 64, 1)
+        assert L.kla_chunk_bwd_workspace(B, T, H, 128, 128, 64, 1 | DIRECT, 0) == \
+            L.kla_chunk_bwd_workspace(B, T, H, 128, 128, 64, 1, 0)
+    assert _fwd(L, dtype=7 | DIRECT) == UNSUPPORTED      # not an element type even without the flag
+    assert _fwd(L, dtype=1 | 0x200) == UNSUPPORTED       # an unknown flag bit
+    assert _fwd(L, dtype=1 | DIRECT, eps=-1.0) == INVALID  # eps is unused in the direct mode, still >= 0
+    assert _fwd(L, dtype=1 | DIRECT, q=None) == INVALID
+    st = L.kla_decode_step(FAKE, FAKE, FAKE, FAKE, FAKE, -0.5, FAKE, None, 4, 2, 128, 128, 1 | DIRECT, 0, None)
+    assert st == INVALID
+
+
+def test_forward_launch_plan(L):
+    """Kernels per kla_chunk_fwd call with a full workspace: two slabs (preparation and state pass
+    each twice) when the heads fill at most half the SMs and there are enough chunks; the
+    segmented pass (preparation, transition pass, scan, output pass) for long sequences over
+    few heads; one preparation and one state pass otherwise; the fused kernel (1) for shapes
+    that take no workspace.  (Without a GPU the library plans for 148 SMs.)"""
+    cases = [((8, 2048, 8), 4), ((4, 4096, 16), 4), ((8, 1024, 8), 4),   # two slabs
+             ((1, 65536, 16), 4),                                       # segmented
+             ((2, 300, 3), 2), ((16, 2048, 16), 2), ((1, 256, 2), 2)]   # one run
+    for (B, T, H), n in cases:
+        assert L.kla_chunk_fwd_kernel_launches(B, T, H, 128, 128, 64, 1) == n, (B, T, H)
+    assert L.kla_chunk_fwd_kernel_launches(1, 300, 2, 64, 64, 64, 0) == 1  # fp32 d = 64: one kernel
+    assert L.kla_chunk_fwd_kernel_launches(0, 300, 2, 128, 128, 64, 1) == 0  # invalid shape
