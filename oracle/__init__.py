@@ -61,8 +61,15 @@ class OracleLib:
         lib.kla_oracle_backward.argtypes = [i, i, i, i, i, dp, dp, dp, dp, dp, d, i, dp, dp, dp,
                                             dp, dp, dp, dp, dp, dp, i]
         lib.kla_oracle_chunk_forward.argtypes = [i, i, i, i, i, dp, dp, dp, dp, dp, d, i, dp, i, dp, dp]
+        # diagonal gating: g is [B, T, H, Dk] (decode: [B, H, Dk]); the backward has no checkpoints
+        lib.kla_oracle_forward_diag.argtypes = [i, i, i, i, i, dp, dp, dp, dp, dp, d, i, dp, dp, dp]
+        lib.kla_oracle_decode_step_diag.argtypes = [i, i, i, i, dp, dp, dp, dp, dp, d, i, dp, dp]
+        lib.kla_oracle_backward_diag.argtypes = [i, i, i, i, i, dp, dp, dp, dp, dp, d, i, dp, dp, dp,
+                                                 dp, dp, dp, dp, dp, dp]
+        lib.kla_oracle_chunk_forward_diag.argtypes = [i, i, i, i, i, dp, dp, dp, dp, dp, d, i, dp, i, dp, dp]
         for f in (lib.kla_oracle_forward, lib.kla_oracle_decode_step, lib.kla_oracle_backward,
-                  lib.kla_oracle_chunk_forward):
+                  lib.kla_oracle_chunk_forward, lib.kla_oracle_forward_diag, lib.kla_oracle_decode_step_diag,
+                  lib.kla_oracle_backward_diag, lib.kla_oracle_chunk_forward_diag):
             f.restype = ctypes.c_int
         self.lib = lib
         self.path = path
@@ -130,6 +137,58 @@ class OracleLib:
         _check(rc, "kla_oracle_chunk_forward")
         return o, ST
 
+    # ---- diagonal gating ("Kaczmarz Linear Attention", App. A.5, B.5): g per key channel ----
+    def forward_diag(self, q, k, v, eta, g, eps, S0=None, beta="kaczmarz"):
+        """Token recurrence with the decay Diag(exp(g_t)), g [B,T,H,Dk]; returns (o, S_T)."""
+        q, k, v, eta, g, S0 = map(_f64, (q, k, v, eta, g, S0))
+        B, T, H, Dk = k.shape
+        Dv = v.shape[-1]
+        o = np.zeros((B, T, H, Dv))
+        ST = np.zeros((B, H, Dk, Dv))
+        rc = self.lib.kla_oracle_forward_diag(B, T, H, Dk, Dv, _ptr(q), _ptr(k), _ptr(v), _ptr(eta), _ptr(g),
+                                              float(eps), _direct(beta), _ptr(S0), _ptr(o), _ptr(ST))
+        _check(rc, "kla_oracle_forward_diag")
+        return o, ST
+
+    def decode_step_diag(self, q, k, v, eta, g, eps, S, beta="kaczmarz"):
+        """One diagonal-gated token step per head, g [B,H,Dk]; returns (o, S_new)."""
+        q, k, v, eta, g = map(_f64, (q, k, v, eta, g))
+        S = _f64(S).copy()
+        B, H, Dk = k.shape
+        Dv = v.shape[-1]
+        o = np.zeros((B, H, Dv))
+        rc = self.lib.kla_oracle_decode_step_diag(B, H, Dk, Dv, _ptr(q), _ptr(k), _ptr(v), _ptr(eta), _ptr(g),
+                                                  float(eps), _direct(beta), _ptr(S), _ptr(o))
+        _check(rc, "kla_oracle_decode_step_diag")
+        return o, S
+
+    def backward_diag(self, q, k, v, eta, g, eps, S0, dO, dS_T=None, beta="kaczmarz"):
+        """Gradients of <o, dO> + <S_T, dS_T>; dg is [B,T,H,Dk]."""
+        q, k, v, eta, g, S0, dO, dS_T = map(_f64, (q, k, v, eta, g, S0, dO, dS_T))
+        B, T, H, Dk = k.shape
+        Dv = v.shape[-1]
+        out = dict(dq=np.zeros((B, T, H, Dk)), dk=np.zeros((B, T, H, Dk)), dv=np.zeros((B, T, H, Dv)),
+                   deta=np.zeros((B, T, H)), dg=np.zeros((B, T, H, Dk)), dS0=np.zeros((B, H, Dk, Dv)))
+        rc = self.lib.kla_oracle_backward_diag(B, T, H, Dk, Dv, _ptr(q), _ptr(k), _ptr(v), _ptr(eta), _ptr(g),
+                                               float(eps), _direct(beta), _ptr(S0), _ptr(dO), _ptr(dS_T),
+                                               _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]),
+                                               _ptr(out["deta"]), _ptr(out["dg"]), _ptr(out["dS0"]))
+        _check(rc, "kla_oracle_backward_diag")
+        return out
+
+    def chunk_forward_diag(self, q, k, v, eta, g, eps, S0=None, chunk=64, beta="kaczmarz"):
+        """Chunk form of the diagonal-gated recurrence; used only to cross-check forward_diag."""
+        q, k, v, eta, g, S0 = map(_f64, (q, k, v, eta, g, S0))
+        B, T, H, Dk = k.shape
+        Dv = v.shape[-1]
+        o = np.zeros((B, T, H, Dv))
+        ST = np.zeros((B, H, Dk, Dv))
+        rc = self.lib.kla_oracle_chunk_forward_diag(B, T, H, Dk, Dv, _ptr(q), _ptr(k), _ptr(v), _ptr(eta), _ptr(g),
+                                                    float(eps), _direct(beta), _ptr(S0), int(chunk), _ptr(o),
+                                                    _ptr(ST))
+        _check(rc, "kla_oracle_chunk_forward_diag")
+        return o, ST
+
 
 _default = None
 
@@ -155,6 +214,22 @@ def backward(*a, **kw):
 
 def chunk_forward(*a, **kw):
     return _load().chunk_forward(*a, **kw)
+
+
+def forward_diag(*a, **kw):
+    return _load().forward_diag(*a, **kw)
+
+
+def decode_step_diag(*a, **kw):
+    return _load().decode_step_diag(*a, **kw)
+
+
+def backward_diag(*a, **kw):
+    return _load().backward_diag(*a, **kw)
+
+
+def chunk_forward_diag(*a, **kw):
+    return _load().chunk_forward_diag(*a, **kw)
 
 
 def threads() -> int:

@@ -415,3 +415,299 @@ int kla_oracle_chunk_forward(int B, int T, int H, int Dk, int Dv, const double *
     }
     return bad ? 2 : 0;
 }
+
+/*
+ * Diagonal gating ("Kaczmarz Linear Attention", Appendix A.5 and B.5): the decay is the
+ * per-key-channel operator D_t = Diag(alpha_t), alpha_t = exp(g_t) with g_t in R^{Dk}:
+ *     Sdec = Diag(alpha_t) S_{t-1}
+ *     e_t  = v_t - Sdec^T k_t
+ *     S_t  = Sdec + beta_t k_t e_t^T      (beta_t unchanged: A.5's decay-agnostic remark)
+ *     o_t  = S_t^T q_t
+ * g is laid out [B, T, H, Dk].  Not yet a row of the CUDA library: these functions exist so that
+ * its diagonal-gated kernels can be checked against them.
+ */
+static void diag_token_step(double *S, const double *q, const double *k, const double *v, double eta,
+                            const double *gvec, double eps, int direct, int Dk, int Dv, double *resid,
+                            double *out) {
+    double knorm2 = 0.0;
+    for (int r = 0; r < Dk; ++r) knorm2 += k[r] * k[r];
+    const double bt = kaczmarz_beta(eta, knorm2, eps, direct);
+    for (int r = 0; r < Dk; ++r) {
+        const double ar = exp(gvec[r]);
+        for (int c = 0; c < Dv; ++c) S[(size_t)r * Dv + c] *= ar;
+    }
+    for (int c = 0; c < Dv; ++c) {
+        double acc = 0.0;
+        for (int r = 0; r < Dk; ++r) acc += k[r] * S[(size_t)r * Dv + c];
+        resid[c] = v[c] - acc;
+    }
+    for (int r = 0; r < Dk; ++r) {
+        const double w = bt * k[r];
+        for (int c = 0; c < Dv; ++c) S[(size_t)r * Dv + c] += w * resid[c];
+    }
+    if (out) {
+        for (int c = 0; c < Dv; ++c) {
+            double acc = 0.0;
+            for (int r = 0; r < Dk; ++r) acc += q[r] * S[(size_t)r * Dv + c];
+            out[c] = acc;
+        }
+    }
+}
+
+int kla_oracle_forward_diag(int B, int T, int H, int Dk, int Dv, const double *q, const double *k,
+                            const double *v, const double *eta, const double *g, double eps, int direct,
+                            const double *S0, double *o, double *ST) {
+    if (B < 0 || T < 0 || H < 0 || Dk <= 0 || Dv <= 0) return 1;
+    int bad = 0;
+    const size_t SS = (size_t)Dk * Dv;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int p = 0; p < B * H; ++p) {
+        const int b = p / H, h = p % H;
+        double *S = (double *)malloc(sizeof(double) * SS);
+        double *tmp = (double *)malloc(sizeof(double) * (size_t)(3 * Dk + 3 * Dv));
+        if (!S || !tmp) {
+#pragma omp atomic write
+            bad = 1;
+        } else {
+            double *qv = tmp, *kv = qv + Dk, *gv = kv + Dk, *vv = gv + Dk, *res = vv + Dv, *ov = res + Dv;
+            if (S0) memcpy(S, S0 + IDX_STATE(b, h, H, Dk, Dv), sizeof(double) * SS);
+            else memset(S, 0, sizeof(double) * SS);
+            for (int t = 0; t < T; ++t) {
+                gather_token(q, b, t, h, T, H, Dk, qv);
+                gather_token(k, b, t, h, T, H, Dk, kv);
+                gather_token(v, b, t, h, T, H, Dv, vv);
+                gather_token(g, b, t, h, T, H, Dk, gv);
+                diag_token_step(S, qv, kv, vv, eta[IDX_GATE(b, t, h, T, H)], gv, eps, direct, Dk, Dv, res,
+                                o ? ov : NULL);
+                if (o) memcpy(o + IDX_TOK(b, t, h, 0, T, H, Dv), ov, sizeof(double) * (size_t)Dv);
+            }
+            if (ST) memcpy(ST + IDX_STATE(b, h, H, Dk, Dv), S, sizeof(double) * SS);
+        }
+        free(S); free(tmp);
+    }
+    return bad ? 2 : 0;
+}
+
+int kla_oracle_decode_step_diag(int B, int H, int Dk, int Dv, const double *q, const double *k,
+                                const double *v, const double *eta, const double *g, double eps, int direct,
+                                double *S, double *o) {
+    if (B < 0 || H < 0 || Dk <= 0 || Dv <= 0) return 1;
+    int bad = 0;
+#pragma omp parallel for schedule(static)
+    for (int p = 0; p < B * H; ++p) {
+        double *res = (double *)malloc(sizeof(double) * (size_t)Dv);
+        if (!res) {
+#pragma omp atomic write
+            bad = 1;
+            continue;
+        }
+        diag_token_step(S + (size_t)p * Dk * Dv, q + (size_t)p * Dk, k + (size_t)p * Dk, v + (size_t)p * Dv, eta[p],
+                        g + (size_t)p * Dk, eps, direct, Dk, Dv, res, o ? o + (size_t)p * Dv : NULL);
+        free(res);
+    }
+    return bad ? 2 : 0;
+}
+
+/*
+ * Backward of the diagonal-gated recurrence, newest token first, with Lambda = dL/dS_t:
+ *   Lambda += q do^T;  dq = S_t do;  de = beta Lambda^T k;  dbeta = k^T Lambda e;  dv = de
+ *   dn, deta as for scalar gating (Kaczmarz or direct beta)
+ *   dk = beta Lambda e - Sdec de + 2 k dn
+ *   dSdec = Lambda - k de^T
+ *   dg[r] = alpha[r] sum_c dSdec[r][c] S_{t-1}[r][c]     (one entry per key channel)
+ *   Lambda <- Diag(alpha) dSdec
+ * States are recomputed forward from S0 for every token (plain, slow: the sizes the tests use
+ * are tiny).
+ */
+int kla_oracle_backward_diag(int B, int T, int H, int Dk, int Dv, const double *q, const double *k,
+                             const double *v, const double *eta, const double *g, double eps, int direct,
+                             const double *S0, const double *dO, const double *dS_T, double *dq, double *dk,
+                             double *dv, double *deta, double *dg, double *dS0) {
+    if (B < 0 || T < 0 || H < 0 || Dk <= 0 || Dv <= 0) return 1;
+    int bad = 0;
+    const size_t SS = (size_t)Dk * Dv;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int p = 0; p < B * H; ++p) {
+        const int b = p / H, h = p % H;
+        double *states = (double *)malloc(sizeof(double) * SS * (size_t)(T + 1));
+        double *Lam = (double *)malloc(sizeof(double) * SS);
+        double *tmp = (double *)malloc(sizeof(double) * (size_t)(5 * Dk + 4 * Dv));
+        if (!states || !Lam || !tmp) {
+#pragma omp atomic write
+            bad = 1;
+        } else {
+            double *qv = tmp, *kv = qv + Dk, *gv = kv + Dk, *dqv = gv + Dk, *dkv = dqv + Dk;
+            double *vv = dkv + Dk, *res = vv + Dv, *dov = res + Dv, *dres = dov + Dv;
+            if (S0) memcpy(states, S0 + IDX_STATE(b, h, H, Dk, Dv), sizeof(double) * SS);
+            else memset(states, 0, sizeof(double) * SS);
+            for (int t = 0; t < T; ++t) {  /* states[t] = S_t (states[0] = S0) */
+                memcpy(states + (size_t)(t + 1) * SS, states + (size_t)t * SS, sizeof(double) * SS);
+                gather_token(q, b, t, h, T, H, Dk, qv);
+                gather_token(k, b, t, h, T, H, Dk, kv);
+                gather_token(v, b, t, h, T, H, Dv, vv);
+                gather_token(g, b, t, h, T, H, Dk, gv);
+                diag_token_step(states + (size_t)(t + 1) * SS, qv, kv, vv, eta[IDX_GATE(b, t, h, T, H)], gv, eps,
+                                direct, Dk, Dv, res, NULL);
+            }
+            if (dS_T) memcpy(Lam, dS_T + IDX_STATE(b, h, H, Dk, Dv), sizeof(double) * SS);
+            else memset(Lam, 0, sizeof(double) * SS);
+            for (int t = T - 1; t >= 0; --t) {
+                const double *Sp = states + (size_t)t * SS, *Sc = states + (size_t)(t + 1) * SS;
+                gather_token(q, b, t, h, T, H, Dk, qv);
+                gather_token(k, b, t, h, T, H, Dk, kv);
+                gather_token(v, b, t, h, T, H, Dv, vv);
+                gather_token(g, b, t, h, T, H, Dk, gv);
+                gather_token(dO, b, t, h, T, H, Dv, dov);
+                const size_t gi = IDX_GATE(b, t, h, T, H);
+                double knorm2 = 0.0;
+                for (int r = 0; r < Dk; ++r) knorm2 += kv[r] * kv[r];
+                const double kden = knorm2 + eps;
+                const double bt = kaczmarz_beta(eta[gi], knorm2, eps, direct);
+                for (int c = 0; c < Dv; ++c) {  /* residual against the decayed state */
+                    double acc = 0.0;
+                    for (int r = 0; r < Dk; ++r) acc += kv[r] * exp(gv[r]) * Sp[(size_t)r * Dv + c];
+                    res[c] = vv[c] - acc;
+                }
+                for (int r = 0; r < Dk; ++r)
+                    for (int c = 0; c < Dv; ++c) Lam[(size_t)r * Dv + c] += qv[r] * dov[c];
+                for (int r = 0; r < Dk; ++r) {
+                    double acc = 0.0;
+                    for (int c = 0; c < Dv; ++c) acc += Sc[(size_t)r * Dv + c] * dov[c];
+                    dqv[r] = acc;
+                }
+                double dbt = 0.0;
+                for (int c = 0; c < Dv; ++c) {
+                    double acc = 0.0;
+                    for (int r = 0; r < Dk; ++r) acc += Lam[(size_t)r * Dv + c] * kv[r];
+                    dres[c] = bt * acc;
+                    dbt += acc * res[c];
+                }
+                double dnorm = 0.0, det = 0.0;
+                if (direct) det = dbt;
+                else if (kden != 0.0) { dnorm = -dbt * bt / kden; det = dbt / kden; }
+                for (int r = 0; r < Dk; ++r) {
+                    const double ar = exp(gv[r]);
+                    double a1 = 0.0, a2 = 0.0;
+                    for (int c = 0; c < Dv; ++c) {
+                        a1 += Lam[(size_t)r * Dv + c] * res[c];
+                        a2 += ar * Sp[(size_t)r * Dv + c] * dres[c];
+                    }
+                    dkv[r] = bt * a1 - a2 + 2.0 * kv[r] * dnorm;
+                }
+                for (int r = 0; r < Dk; ++r) {
+                    const double ar = exp(gv[r]);
+                    double acc = 0.0;
+                    for (int c = 0; c < Dv; ++c) {
+                        const size_t x = (size_t)r * Dv + c;
+                        const double dsd = Lam[x] - kv[r] * dres[c];
+                        acc += dsd * Sp[x];
+                        Lam[x] = ar * dsd;
+                    }
+                    dg[IDX_TOK(b, t, h, r, T, H, Dk)] = ar * acc;
+                }
+                memcpy(dq + IDX_TOK(b, t, h, 0, T, H, Dk), dqv, sizeof(double) * (size_t)Dk);
+                memcpy(dk + IDX_TOK(b, t, h, 0, T, H, Dk), dkv, sizeof(double) * (size_t)Dk);
+                memcpy(dv + IDX_TOK(b, t, h, 0, T, H, Dv), dres, sizeof(double) * (size_t)Dv);
+                deta[gi] = det;
+            }
+            memcpy(dS0 + IDX_STATE(b, h, H, Dk, Dv), Lam, sizeof(double) * SS);
+        }
+        free(states); free(Lam); free(tmp);
+    }
+    return bad ? 2 : 0;
+}
+
+/*
+ * Chunk form of the diagonal-gated recurrence (Appendix B.5: the scalar decay products become
+ * elementwise).  Per chunk, G_i = sum_{r<=i} g_r per channel; for i > j the decayed Gram is
+ * A_ij = sum_c k_i[c] k_j[c] exp(G_i[c] - G_j[c]); then, solving by forward substitution,
+ *     u_i = beta_i (v_i - S0^T (exp(G_i) o k_i)) - beta_i sum_{j<i} A_ij u_j
+ *     o_i = S0^T (exp(G_i) o q_i) + sum_{j<=i} [sum_c q_i[c] k_j[c] exp(G_i[c] - G_j[c])] u_j
+ *     S_end = Diag(exp(G_C)) S0 + sum_j Diag(exp(G_C - G_j)) k_j u_j^T
+ * Used only to check the token form above.
+ */
+int kla_oracle_chunk_forward_diag(int B, int T, int H, int Dk, int Dv, const double *q, const double *k,
+                                  const double *v, const double *eta, const double *g, double eps, int direct,
+                                  const double *S0, int C, double *o, double *ST) {
+    if (B < 0 || T < 0 || H < 0 || Dk <= 0 || Dv <= 0 || C <= 0) return 1;
+    int bad = 0;
+    const size_t SS = (size_t)Dk * Dv;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int p = 0; p < B * H; ++p) {
+        const int b = p / H, h = p % H;
+        double *S = (double *)malloc(sizeof(double) * SS);
+        double *Gc = (double *)malloc(sizeof(double) * (size_t)C * Dk);
+        double *uu = (double *)malloc(sizeof(double) * (size_t)C * Dv);
+        double *bb = (double *)malloc(sizeof(double) * (size_t)C);
+        double *Snew = (double *)malloc(sizeof(double) * SS);
+        if (!S || !Gc || !uu || !bb || !Snew) {
+#pragma omp atomic write
+            bad = 1;
+        } else {
+            if (S0) memcpy(S, S0 + IDX_STATE(b, h, H, Dk, Dv), sizeof(double) * SS);
+            else memset(S, 0, sizeof(double) * SS);
+            for (int t0 = 0; t0 < T; t0 += C) {
+                const int n = T - t0 < C ? T - t0 : C;
+                for (int i = 0; i < n; ++i) {
+                    const double *ki = k + IDX_TOK(b, t0 + i, h, 0, T, H, Dk);
+                    double kn = 0.0;
+                    for (int r = 0; r < Dk; ++r) {
+                        const double gr = g[IDX_TOK(b, t0 + i, h, r, T, H, Dk)];
+                        Gc[(size_t)i * Dk + r] = (i ? Gc[(size_t)(i - 1) * Dk + r] : 0.0) + gr;
+                        kn += ki[r] * ki[r];
+                    }
+                    bb[i] = kaczmarz_beta(eta[IDX_GATE(b, t0 + i, h, T, H)], kn, eps, direct);
+                }
+                for (int i = 0; i < n; ++i) {
+                    const double *ki = k + IDX_TOK(b, t0 + i, h, 0, T, H, Dk);
+                    const double *vi = v + IDX_TOK(b, t0 + i, h, 0, T, H, Dv);
+                    for (int c = 0; c < Dv; ++c) {
+                        double acc = 0.0;
+                        for (int r = 0; r < Dk; ++r) acc += exp(Gc[(size_t)i * Dk + r]) * ki[r] * S[(size_t)r * Dv + c];
+                        uu[(size_t)i * Dv + c] = bb[i] * (vi[c] - acc);
+                    }
+                    for (int j = 0; j < i; ++j) {
+                        const double *kj = k + IDX_TOK(b, t0 + j, h, 0, T, H, Dk);
+                        double aij = 0.0;
+                        for (int r = 0; r < Dk; ++r)
+                            aij += ki[r] * kj[r] * exp(Gc[(size_t)i * Dk + r] - Gc[(size_t)j * Dk + r]);
+                        for (int c = 0; c < Dv; ++c) uu[(size_t)i * Dv + c] -= bb[i] * aij * uu[(size_t)j * Dv + c];
+                    }
+                }
+                if (o) {
+                    for (int i = 0; i < n; ++i) {
+                        const double *qi = q + IDX_TOK(b, t0 + i, h, 0, T, H, Dk);
+                        double *oi = o + IDX_TOK(b, t0 + i, h, 0, T, H, Dv);
+                        for (int c = 0; c < Dv; ++c) {
+                            double acc = 0.0;
+                            for (int r = 0; r < Dk; ++r) acc += exp(Gc[(size_t)i * Dk + r]) * qi[r] * S[(size_t)r * Dv + c];
+                            oi[c] = acc;
+                        }
+                        for (int j = 0; j <= i; ++j) {
+                            const double *kj = k + IDX_TOK(b, t0 + j, h, 0, T, H, Dk);
+                            double sij = 0.0;
+                            for (int r = 0; r < Dk; ++r)
+                                sij += qi[r] * kj[r] * exp(Gc[(size_t)i * Dk + r] - Gc[(size_t)j * Dk + r]);
+                            for (int c = 0; c < Dv; ++c) oi[c] += sij * uu[(size_t)j * Dv + c];
+                        }
+                    }
+                }
+                for (int r = 0; r < Dk; ++r) {
+                    const double gl = Gc[(size_t)(n - 1) * Dk + r];
+                    for (int c = 0; c < Dv; ++c) {
+                        double acc = exp(gl) * S[(size_t)r * Dv + c];
+                        for (int j = 0; j < n; ++j) {
+                            const double kjr = k[IDX_TOK(b, t0 + j, h, r, T, H, Dk)];
+                            acc += exp(gl - Gc[(size_t)j * Dk + r]) * kjr * uu[(size_t)j * Dv + c];
+                        }
+                        Snew[(size_t)r * Dv + c] = acc;
+                    }
+                }
+                memcpy(S, Snew, sizeof(double) * SS);
+            }
+            if (ST) memcpy(ST + IDX_STATE(b, h, H, Dk, Dv), S, sizeof(double) * SS);
+        }
+        free(S); free(Gc); free(uu); free(bb); free(Snew);
+    }
+    return bad ? 2 : 0;
+}

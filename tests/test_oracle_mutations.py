@@ -46,6 +46,25 @@ def _direct_backward_pins(mod):
         yield lambda T=T, ck=ck: pins.test_direct_backward_finite_differences(mod, T, ck)
 
 
+def _diag_forward_pins(mod):
+    for eps in (1e-6, 0.5):
+        yield lambda eps=eps: pins.test_diag_relaxed_interpolation(mod, eps)
+    for C in (3, 8):
+        yield lambda C=C: pins.test_diag_chunk_form_matches_token_form(mod, C)
+
+
+def _diag_backward_pins(mod):
+    for beta, eps in (("kaczmarz", 1e-2), ("direct", 0.0)):
+        yield lambda beta=beta, eps=eps: pins.test_diag_backward_finite_differences(mod, beta, eps)
+    yield lambda: pins.test_diag_uniform_channels_equal_scalar_gating(mod, "kaczmarz")
+
+
+def _diag_chunk_pins(mod):
+    yield lambda: pins.test_diag_uniform_channels_equal_scalar_gating(mod, "kaczmarz")
+    for C in (3, 8):
+        yield lambda C=C: pins.test_diag_chunk_form_matches_token_form(mod, C)
+
+
 def _chunk_pins(mod):
     for C in (2, 3, 8, 64):
         yield lambda C=C: pins.test_chunk_form_matches_token_form(mod, C)
@@ -74,6 +93,15 @@ MUTATIONS = [
     ("bwd_dq_uses_previous_state", "for (int j = 0; j < Dv; ++j) s += Scur[(size_t)i * Dv + j] * dot[j];",
      "for (int j = 0; j < Dv; ++j) s += Sprev[(size_t)i * Dv + j] * dot[j];", _backward_pins),
     ("bwd_de_drops_beta", "de[j] = beta * s;", "de[j] = s;", _backward_pins),
+    ("diag_one_channel_decay_for_all", "        const double ar = exp(gvec[r]);",
+     "        const double ar = exp(gvec[0]);", _diag_forward_pins),
+    ("diag_bwd_dg_drops_alpha", "dg[IDX_TOK(b, t, h, r, T, H, Dk)] = ar * acc;",
+     "dg[IDX_TOK(b, t, h, r, T, H, Dk)] = acc;", _diag_backward_pins),
+    ("diag_bwd_state_gradient_not_decayed", "                        Lam[x] = ar * dsd;",
+     "                        Lam[x] = dsd;", _diag_backward_pins),
+    ("diag_chunk_ratio_inverted",
+     "aij += ki[r] * kj[r] * exp(Gc[(size_t)i * Dk + r] - Gc[(size_t)j * Dk + r]);",
+     "aij += ki[r] * kj[r] * exp(Gc[(size_t)j * Dk + r] - Gc[(size_t)i * Dk + r]);", _diag_chunk_pins),
     ("chunk_decay_ratio_inverted", "val = bet[i] * (gam[i] / gam[j]) * kk;",
      "val = bet[i] * (gam[j] / gam[i]) * kk;", _chunk_pins),
     ("chunk_substitution_sign", "U[(size_t)i * Dv + c2] -= l * U[(size_t)j * Dv + c2];",

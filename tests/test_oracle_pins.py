@@ -474,3 +474,122 @@ def test_direct_backward_finite_differences(oracle_mod, T, ckpt):
         got = grads["d" + name]
         err = np.abs(got - fd).max() / max(np.abs(fd).max(), 1e-3)
         assert err <= 1e-6, (name, err)
+
+
+# ---------------------------------------------------------------------------------------
+# Diagonal gating (Appendix A.5 and B.5): the decay Diag(exp(g_t)) per key channel.  The
+# oracle's diagonal-gated functions are pinned by: equality with the scalar-gated oracle when
+# every channel decays alike (forward, chunk form, backward with dg summed over channels),
+# Theorem 1's projection and Proposition 2's interpolation for any per-channel decay (A.5:
+# the derivation never uses how the decayed state was produced), the chunk form of B.5, and
+# finite differences.
+# ---------------------------------------------------------------------------------------
+def _diag_g(rng, shape_btH, Dk, lo=-1.0):
+    return rng.uniform(lo, 0.0, shape_btH + (Dk,))
+
+
+@pytest.mark.parametrize("beta", ["kaczmarz", "direct"])
+def test_diag_uniform_channels_equal_scalar_gating(oracle_mod, beta):
+    rng = np.random.default_rng(400)
+    q, k, v, eta, g, S0 = _rand_inputs(rng, 2, 9, 2, 5, 3, key_lo=0.4, key_hi=2.0, s0=0.5)
+    if beta == "direct":
+        eta = 0.3 * eta
+    gd = np.repeat(g[..., None], 5, axis=-1)
+    eps = 1e-3
+    o1, S1 = oracle_mod.forward(q, k, v, eta, g, eps, S0, beta=beta)
+    o2, S2 = oracle_mod.forward_diag(q, k, v, eta, gd, eps, S0, beta=beta)
+    np.testing.assert_allclose(o2, o1, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(S2, S1, rtol=1e-12, atol=1e-13)
+    o3, S3 = oracle_mod.chunk_forward_diag(q, k, v, eta, gd, eps, S0, chunk=4, beta=beta)
+    np.testing.assert_allclose(o3, o1, rtol=1e-10, atol=1e-11)
+    np.testing.assert_allclose(S3, S1, rtol=1e-10, atol=1e-11)
+    dO = rng.standard_normal(o1.shape)
+    dST = rng.standard_normal(S1.shape)
+    r1 = oracle_mod.backward(q, k, v, eta, g, eps, S0, dO, dST, beta=beta)
+    r2 = oracle_mod.backward_diag(q, k, v, eta, gd, eps, S0, dO, dST, beta=beta)
+    for name in ("dq", "dk", "dv", "deta", "dS0"):
+        np.testing.assert_allclose(r2[name], r1[name], rtol=1e-10, atol=1e-11, err_msg=name)
+    np.testing.assert_allclose(r2["dg"].sum(-1), r1["dg"], rtol=1e-10, atol=1e-11)
+
+
+def test_diag_hard_projection_any_decay(oracle_mod):
+    rng = np.random.default_rng(401)
+    q, k, v, _, _, S0 = _rand_inputs(rng, 2, 10, 2, 6, 3, key_lo=0.1, key_hi=10.0)
+    g = _diag_g(rng, k.shape[:3], 6, lo=-3.0)
+    eta = np.ones(k.shape[:3])
+    S = S0.copy()
+    for t in range(k.shape[1]):
+        _, S = oracle_mod.decode_step_diag(q[:, t], k[:, t], v[:, t], eta[:, t], g[:, t], 0.0, S)
+        readout = np.einsum("bhij,bhi->bhj", S, k[:, t])
+        np.testing.assert_allclose(readout, v[:, t], rtol=0, atol=1e-12 * (1 + np.abs(v[:, t]).max()))
+
+
+@pytest.mark.parametrize("eps", [1e-6, 0.5])
+def test_diag_relaxed_interpolation(oracle_mod, eps):
+    rng = np.random.default_rng(402)
+    q, k, v, eta, _, S0 = _rand_inputs(rng, 1, 8, 3, 4, 5)
+    g = _diag_g(rng, k.shape[:3], 4, lo=-2.0)
+    S = S0.copy()
+    for t in range(k.shape[1]):
+        Sdec = np.exp(g[:, t])[..., None] * S      # the decayed state, Diag(alpha_t) S_{t-1}
+        _, S = oracle_mod.decode_step_diag(q[:, t], k[:, t], v[:, t], eta[:, t], g[:, t], eps, S)
+        n = np.sum(k[:, t] ** 2, axis=-1)
+        c = (eta[:, t] * n / (n + eps))[..., None]
+        lhs = np.einsum("bhij,bhi->bhj", S, k[:, t])
+        rhs = (1 - c) * np.einsum("bhij,bhi->bhj", Sdec, k[:, t]) + c * v[:, t]
+        np.testing.assert_allclose(lhs, rhs, rtol=1e-11, atol=1e-12)
+
+
+@pytest.mark.parametrize("C", [1, 3, 8, 64])
+def test_diag_chunk_form_matches_token_form(oracle_mod, C):
+    rng = np.random.default_rng(403 + C)
+    q, k, v, eta, _, S0 = _rand_inputs(rng, 2, 70, 2, 5, 4, key_lo=0.3, key_hi=3.0)
+    g = _diag_g(rng, k.shape[:3], 5, lo=-1.5)
+    o1, S1 = oracle_mod.forward_diag(q, k, v, eta, g, 1e-6, S0)
+    o2, S2 = oracle_mod.chunk_forward_diag(q, k, v, eta, g, 1e-6, S0, chunk=C)
+    np.testing.assert_allclose(o2, o1, rtol=1e-9, atol=1e-10)
+    np.testing.assert_allclose(S2, S1, rtol=1e-9, atol=1e-10)
+
+
+def test_diag_decode_step_equals_forward_T1(oracle_mod):
+    rng = np.random.default_rng(404)
+    q, k, v, eta, _, S0 = _rand_inputs(rng, 2, 1, 3, 4, 5)
+    g = _diag_g(rng, k.shape[:3], 4)
+    o, ST = oracle_mod.forward_diag(q, k, v, eta, g, 1e-6, S0)
+    o2, S2 = oracle_mod.decode_step_diag(q[:, 0], k[:, 0], v[:, 0], eta[:, 0], g[:, 0], 1e-6, S0)
+    np.testing.assert_array_equal(o[:, 0], o2)
+    np.testing.assert_array_equal(ST, S2)
+
+
+@pytest.mark.parametrize("beta,eps", [("kaczmarz", 1e-2), ("direct", 0.0)])
+def test_diag_backward_finite_differences(oracle_mod, beta, eps):
+    rng = np.random.default_rng(410)
+    B, T, H, Dk, Dv = 1, 6, 2, 3, 4
+    q, k, v, eta, _, S0 = _rand_inputs(rng, B, T, H, Dk, Dv, key_lo=0.5, key_hi=1.5, s0=0.5)
+    g = _diag_g(rng, (B, T, H), Dk, lo=-1.0)
+    if beta == "direct":
+        eta = 0.3 * eta
+    dO = rng.standard_normal((B, T, H, Dv))
+    dST = rng.standard_normal((B, H, Dk, Dv))
+    grads = oracle_mod.backward_diag(q, k, v, eta, g, eps, S0, dO, dST, beta=beta)
+    args = dict(q=q, k=k, v=v, eta=eta, g=g, S0=S0)
+
+    def loss(a):
+        o, ST = oracle_mod.forward_diag(a["q"], a["k"], a["v"], a["eta"], a["g"], eps, a["S0"], beta=beta)
+        return float(np.sum(o * dO) + np.sum(ST * dST))
+
+    hstep = 1e-6
+    for name in args:
+        x = args[name]
+        fd = np.zeros_like(x)
+        it = np.nditer(x, flags=["multi_index"])
+        for _ in it:
+            idx = it.multi_index
+            a_p = {kk: vv.copy() for kk, vv in args.items()}
+            a_m = {kk: vv.copy() for kk, vv in args.items()}
+            a_p[name][idx] += hstep
+            a_m[name][idx] -= hstep
+            fd[idx] = (loss(a_p) - loss(a_m)) / (2 * hstep)
+        got = grads["d" + name]
+        err = np.abs(got - fd).max() / max(np.abs(fd).max(), 1e-3)
+        assert err <= 1e-6, (name, err)
