@@ -20,7 +20,8 @@ import torch
 
 __all__ = ["lib", "chunk_fwd", "chunk_fwd_prep", "chunk_fwd_state", "fwd_workspace", "fwd_kernel_launches",
            "chunk_bwd", "chunk_fwd_train", "chunk_bwd_after_train", "train_workspace",
-           "decode_step", "check_device_error", "KLAError", "CHUNK", "KLA_BETA_DIRECT",
+           "decode_step", "check_device_error", "debug_inject_wait_timeout",
+           "chunk_fwd_diag", "chunk_bwd_diag", "decode_step_diag", "KLAError", "CHUNK", "KLA_BETA_DIRECT",
            "library_path"]
 
 CHUNK = 64
@@ -80,6 +81,17 @@ def lib():
         L.kla_decode_step.restype = i
         L.kla_check_device_error.argtypes = [vp]
         L.kla_check_device_error.restype = i
+        L.kla_debug_inject_wait_timeout.argtypes = []
+        L.kla_debug_inject_wait_timeout.restype = None
+        L.kla_chunk_fwd_diag.argtypes = [vp, vp, vp, fp, fp, f, fp, vp, fp, i, i, i, i, i, i, i, i, vp]
+        L.kla_chunk_fwd_diag.restype = i
+        L.kla_chunk_bwd_diag_workspace.argtypes = [i, i, i, i, i, i, i]
+        L.kla_chunk_bwd_diag_workspace.restype = sz
+        L.kla_chunk_bwd_diag.argtypes = [vp, vp, vp, fp, fp, f, fp, vp, fp, vp, vp, vp, fp, fp, fp,
+                                         i, i, i, i, i, i, i, i, vp, sz, vp]
+        L.kla_chunk_bwd_diag.restype = i
+        L.kla_decode_step_diag.argtypes = [vp, vp, vp, fp, fp, f, fp, vp, i, i, i, i, i, i, vp]
+        L.kla_decode_step_diag.restype = i
         _lib = L
     return _lib
 
@@ -342,6 +354,82 @@ def decode_step(q, k, v, eta, g, S, eps=1e-6, *, o=None, out_dtype=torch.float32
                                B, H, Dk, Dv, _in_code(k, beta), _dtype_code(o), _stream(dev, stream))
     _check(st, "kla_decode_step")
     return o
+
+
+def chunk_fwd_diag(q, k, v, eta, g, eps=1e-6, S0=None, *, o=None, S_T=None, out_dtype=torch.float32,
+                   stream=None, beta="kaczmarz"):
+    """Prefill with diagonal (per-key-channel) gating (Appendix A.5, B.5): g is [B,T,H,Dk] fp32,
+    the decay of token t is Diag(exp(g_t)).  Other arguments as chunk_fwd.  Returns (o, S_T)."""
+    dev = k.device
+    B, T, H, Dk = k.shape
+    Dv = v.shape[-1]
+    dt = k.dtype
+    _need(q, "q", dev, dt, (B, T, H, Dk)); _need(k, "k", dev, dt); _need(v, "v", dev, dt, (B, T, H, Dv))
+    _need(eta, "eta", dev, torch.float32, (B, T, H)); _need(g, "g", dev, torch.float32, (B, T, H, Dk))
+    _need(S0, "S0", dev, torch.float32, (B, H, Dk, Dv))
+    if o is None:
+        o = torch.empty(B, T, H, Dv, device=dev, dtype=out_dtype)
+    _need(o, "o", dev, None, (B, T, H, Dv))
+    if S_T is None:
+        S_T = torch.empty(B, H, Dk, Dv, device=dev, dtype=torch.float32)
+    _need(S_T, "S_T", dev, torch.float32, (B, H, Dk, Dv))
+    st = lib().kla_chunk_fwd_diag(_ptr(q), _ptr(k), _ptr(v), _ptr(eta), _ptr(g), float(eps), _ptr(S0), _ptr(o),
+                                  _ptr(S_T), B, T, H, Dk, Dv, CHUNK, _in_code(k, beta), _dtype_code(o),
+                                  _stream(dev, stream))
+    _check(st, "kla_chunk_fwd_diag")
+    return o, S_T
+
+
+def chunk_bwd_diag(q, k, v, eta, g, dO, eps=1e-6, S0=None, dS_T=None, *, workspace=None,
+                   out_dtype=torch.float32, stream=None, beta="kaczmarz"):
+    """Gradients of chunk_fwd_diag (dg is [B,T,H,Dk]).  Returns dict(dq, dk, dv, deta, dg, dS0)."""
+    dev = k.device
+    B, T, H, Dk = k.shape
+    Dv = v.shape[-1]
+    dt = k.dtype
+    _need(q, "q", dev, dt, (B, T, H, Dk)); _need(k, "k", dev, dt); _need(v, "v", dev, dt, (B, T, H, Dv))
+    _need(eta, "eta", dev, torch.float32, (B, T, H)); _need(g, "g", dev, torch.float32, (B, T, H, Dk))
+    _need(S0, "S0", dev, torch.float32, (B, H, Dk, Dv)); _need(dO, "dO", dev, dt, (B, T, H, Dv))
+    _need(dS_T, "dS_T", dev, torch.float32, (B, H, Dk, Dv))
+    out = dict(dq=torch.empty(q.shape, device=dev, dtype=out_dtype),
+               dk=torch.empty(k.shape, device=dev, dtype=out_dtype),
+               dv=torch.empty(v.shape, device=dev, dtype=out_dtype),
+               deta=torch.empty_like(eta), dg=torch.empty_like(g),
+               dS0=torch.empty(B, H, Dk, Dv, device=dev, dtype=torch.float32))
+    L = lib()
+    need = L.kla_chunk_bwd_diag_workspace(B, T, H, Dk, Dv, CHUNK, _dtype_code(k))
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(max(need, 16), device=dev, dtype=torch.uint8)
+    st = L.kla_chunk_bwd_diag(_ptr(q), _ptr(k), _ptr(v), _ptr(eta), _ptr(g), float(eps), _ptr(S0), _ptr(dO),
+                              _ptr(dS_T), _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]), _ptr(out["deta"]),
+                              _ptr(out["dg"]), _ptr(out["dS0"]), B, T, H, Dk, Dv, CHUNK, _in_code(k, beta),
+                              _dtype_code(out_dtype), _ptr(workspace), workspace.numel(), _stream(dev, stream))
+    _check(st, "kla_chunk_bwd_diag")
+    return out
+
+
+def decode_step_diag(q, k, v, eta, g, S, eps=1e-6, *, o=None, out_dtype=torch.float32, stream=None,
+                     beta="kaczmarz"):
+    """One decode token with diagonal gating: g is [B,H,Dk] fp32; otherwise as decode_step."""
+    dev = S.device
+    B, H, Dk, Dv = S.shape
+    dt = k.dtype
+    _need(q, "q", dev, dt, (B, H, Dk)); _need(k, "k", dev, dt, (B, H, Dk)); _need(v, "v", dev, dt, (B, H, Dv))
+    _need(eta, "eta", dev, torch.float32, (B, H)); _need(g, "g", dev, torch.float32, (B, H, Dk))
+    _need(S, "S", dev, torch.float32, (B, H, Dk, Dv))
+    if o is None:
+        o = torch.empty(B, H, Dv, device=dev, dtype=out_dtype)
+    _need(o, "o", dev, None, (B, H, Dv))
+    st = lib().kla_decode_step_diag(_ptr(q), _ptr(k), _ptr(v), _ptr(eta), _ptr(g), float(eps), _ptr(S), _ptr(o),
+                                    B, H, Dk, Dv, _in_code(k, beta), _dtype_code(o), _stream(dev, stream))
+    _check(st, "kla_decode_step_diag")
+    return o
+
+
+def debug_inject_wait_timeout():
+    """Failure injection for tests: the next decode_step's kernel lets its first bounded wait
+    expire (nothing is stored), so check_device_error then raises KLAError(KLA_ERR_TIMEOUT)."""
+    lib().kla_debug_inject_wait_timeout()
 
 
 def check_device_error(stream=None, device=None):

@@ -30,25 +30,9 @@ def _nvcc() -> str:
     raise RuntimeError("nvcc not found; install the CUDA 12.9 toolkit or set NVCC")
 
 
-def _cutlass_include():
-    """CuTe/CUTLASS headers vendored with flashinfer (header-only, used for sm100 descriptors)."""
-    try:
-        import site
-        for sp in site.getsitepackages():
-            p = os.path.join(sp, "flashinfer", "data", "cutlass", "include")
-            if os.path.isdir(os.path.join(p, "cute")):
-                return p
-    except Exception:
-        pass
-    return None
-
-
 def _flags():
     f = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-I" + INCLUDE, "-I" + CSRC,
          "--expt-relaxed-constexpr", "-Xptxas", "-O3"] + ARCH
-    cut = _cutlass_include()
-    if cut:
-        f.append("-I" + cut)
     if os.environ.get("KLA_PTXAS_VERBOSE"):
         f += ["-Xptxas", "-v"]
     return f

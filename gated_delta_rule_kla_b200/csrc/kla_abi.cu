@@ -4,6 +4,7 @@
 #include <stdint.h>
 #include <stdio.h>
 
+#include <atomic>
 #include <string>
 
 #include "kla.h"
@@ -12,6 +13,9 @@
 #include "kla_tc_common.cuh"
 
 namespace {
+
+// Set by kla_debug_inject_wait_timeout, taken (and cleared) by the next kla_decode_step.
+std::atomic<int> g_inject_timeout{0};
 
 thread_local std::string g_last_error;
 
@@ -84,6 +88,27 @@ bool tc_bwd_shape(int T, int Dk, int Dv, int dtype) {
 bool tc_bwd_path(int B, int T, int H, int Dk, int Dv, int dtype, size_t ws_bytes) {
     return tc_bwd_shape(T, Dk, Dv, dtype) && kla::get_encode_fn() != nullptr &&
            ws_bytes >= kla::chunk_bwd_tc_workspace(B, T, H, false);
+}
+
+// Diagonal-gated backward: [S at every internal chunk start | acc_dq | acc_dkh | acc_dG (per
+// channel) | acc_db, acc_dc]; everything after the states is zeroed on every call.
+size_t diag_bwd_ws_layout(int B, int T, int H, int Dk, int Dv, size_t* off) {
+    const size_t CDl = (size_t)kla::diag_chunk_len();
+    const size_t NC = ((size_t)T + CDl - 1) / CDl;
+    const size_t ntok = (size_t)B * T * H;
+    size_t o = 0;
+    off[0] = o;
+    o += align256((size_t)B * H * NC * Dk * Dv * sizeof(float));
+    off[1] = o;
+    o += align256(ntok * Dk * sizeof(float));
+    off[2] = o;
+    o += align256(ntok * Dk * sizeof(float));
+    off[3] = o;
+    o += align256(ntok * Dk * sizeof(float));
+    off[4] = o;
+    o += align256(2 * ntok * sizeof(float));
+    off[5] = o;
+    return o;
 }
 
 size_t bwd_ws_layout(int B, int T, int H, int Dk, int Dv, bool have_S_chunks, size_t* off) {
@@ -389,11 +414,107 @@ kla_status kla_decode_step(const void* q, const void* k, const void* v, const fl
     REQUIRE_PTR(S);
     OPTIONAL_PTR(o);
     kla::DecodeArgs a{q, k, v, eta, g, kernel_eps(eps, direct), S, o, B, H, Dk, Dv, dtype == KLA_BF16,
-                      out_dtype == KLA_BF16};
+                      out_dtype == KLA_BF16, g_inject_timeout.exchange(0) != 0};
     cudaError_t e = kla::launch_decode(a, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "kla_decode_step launch");
     return KLA_OK;
 }
+
+kla_status kla_decode_step_diag(const void* q, const void* k, const void* v, const float* eta,
+                                const float* g, float eps, float* S, void* o, int B, int H, int Dk,
+                                int Dv, int dtype, int out_dtype, void* stream) {
+    const bool direct = take_beta_flag(dtype);
+    kla_status st = check_common(B, 0, H, Dk, Dv, kla::kChunkLen, dtype, out_dtype, eps);
+    if (st != KLA_OK) return st;
+    REQUIRE_PTR(q); REQUIRE_PTR(k); REQUIRE_PTR(v); REQUIRE_PTR(eta); REQUIRE_PTR(g);
+    REQUIRE_PTR(S);
+    OPTIONAL_PTR(o);
+    kla::DecodeArgs a{q, k, v, eta, g, kernel_eps(eps, direct), S, o, B, H, Dk, Dv, dtype == KLA_BF16,
+                      out_dtype == KLA_BF16, false, true};
+    cudaError_t e = kla::launch_decode(a, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "kla_decode_step_diag launch");
+    return KLA_OK;
+}
+
+kla_status kla_chunk_fwd_diag(const void* q, const void* k, const void* v, const float* eta,
+                              const float* g, float eps, const float* S0, void* o, float* S_T, int B,
+                              int T, int H, int Dk, int Dv, int chunk, int dtype, int out_dtype,
+                              void* stream) {
+    const bool direct = take_beta_flag(dtype);
+    kla_status st = check_common(B, T, H, Dk, Dv, chunk, dtype, out_dtype, eps);
+    if (st != KLA_OK) return st;
+    if (T > 0) {
+        REQUIRE_PTR(q); REQUIRE_PTR(k); REQUIRE_PTR(v); REQUIRE_PTR(eta); REQUIRE_PTR(g);
+    }
+    OPTIONAL_PTR(S0); OPTIONAL_PTR(o); OPTIONAL_PTR(S_T);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (T == 0) {
+        if (S_T != nullptr && S_T != S0) {
+            const size_t bytes = (size_t)B * H * Dk * Dv * sizeof(float);
+            cudaError_t e = S0 ? cudaMemcpyAsync(S_T, S0, bytes, cudaMemcpyDeviceToDevice, s)
+                               : cudaMemsetAsync(S_T, 0, bytes, s);
+            if (e != cudaSuccess) return cuda_fail(e, "kla_chunk_fwd_diag(T=0)");
+        }
+        return KLA_OK;
+    }
+    kla::FwdArgs a{q, k, v, eta, g, kernel_eps(eps, direct), S0, o, S_T, nullptr, B, T, H, Dk, Dv,
+                   dtype == KLA_BF16, out_dtype == KLA_BF16};
+    cudaError_t e = kla::launch_chunk_fwd_diag(a, s);
+    if (e != cudaSuccess) return cuda_fail(e, "kla_chunk_fwd_diag launch");
+    return KLA_OK;
+}
+
+size_t kla_chunk_bwd_diag_workspace(int B, int T, int H, int Dk, int Dv, int chunk, int dtype) {
+    (void)chunk;
+    take_beta_flag(dtype);
+    if (B < 1 || H < 1 || T < 0) return 0;
+    size_t off[6];
+    return diag_bwd_ws_layout(B, T, H, Dk, Dv, off);
+}
+
+kla_status kla_chunk_bwd_diag(const void* q, const void* k, const void* v, const float* eta,
+                              const float* g, float eps, const float* S0, const void* dO,
+                              const float* dS_T, void* dq, void* dk, void* dv, float* deta, float* dg,
+                              float* dS0, int B, int T, int H, int Dk, int Dv, int chunk, int dtype,
+                              int out_dtype, void* ws, size_t ws_bytes, void* stream) {
+    const bool direct = take_beta_flag(dtype);
+    kla_status st = check_common(B, T, H, Dk, Dv, chunk, dtype, out_dtype, eps);
+    if (st != KLA_OK) return st;
+    REQUIRE_PTR(dS0);
+    OPTIONAL_PTR(S0); OPTIONAL_PTR(dS_T);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (T == 0) {
+        const size_t sbytes = (size_t)B * H * Dk * Dv * sizeof(float);
+        cudaError_t e = dS_T ? cudaMemcpyAsync(dS0, dS_T, sbytes, cudaMemcpyDeviceToDevice, s)
+                             : cudaMemsetAsync(dS0, 0, sbytes, s);
+        if (e != cudaSuccess) return cuda_fail(e, "kla_chunk_bwd_diag(T=0)");
+        return KLA_OK;
+    }
+    REQUIRE_PTR(q); REQUIRE_PTR(k); REQUIRE_PTR(v); REQUIRE_PTR(eta); REQUIRE_PTR(g);
+    REQUIRE_PTR(dO); REQUIRE_PTR(dq); REQUIRE_PTR(dk); REQUIRE_PTR(dv); REQUIRE_PTR(deta);
+    REQUIRE_PTR(dg);
+    size_t off[6];
+    const size_t need = diag_bwd_ws_layout(B, T, H, Dk, Dv, off);
+    if (ws == nullptr || ws_bytes < need)
+        return fail(KLA_ERR_WORKSPACE, "kla_chunk_bwd_diag needs %zu workspace bytes (got %zu)", need,
+                    ws == nullptr ? (size_t)0 : ws_bytes);
+    if (!aligned16(ws)) return fail(KLA_ERR_INVALID_ARG, "ws must be 16-byte aligned");
+    char* w = static_cast<char*>(ws);
+    cudaError_t e = cudaMemsetAsync(w + off[1], 0, off[5] - off[1], s);
+    if (e != cudaSuccess) return cuda_fail(e, "kla_chunk_bwd_diag workspace clear");
+    const size_t ntok = (size_t)B * T * H;
+    float* acc_b = reinterpret_cast<float*>(w + off[4]);
+    kla::BwdArgs a{q, k, v, eta, g, kernel_eps(eps, direct), reinterpret_cast<const float*>(w + off[0]), dO, dS_T,
+                   dq, dk, dv, deta, dg, dS0, reinterpret_cast<float*>(w + off[1]),
+                   reinterpret_cast<float*>(w + off[2]), acc_b, acc_b + ntok,
+                   reinterpret_cast<float*>(w + off[3]), B, T, H, Dk, Dv, dtype == KLA_BF16,
+                   out_dtype == KLA_BF16};
+    e = kla::launch_chunk_bwd_diag(a, S0, s);
+    if (e != cudaSuccess) return cuda_fail(e, "kla_chunk_bwd_diag launch");
+    return KLA_OK;
+}
+
+void kla_debug_inject_wait_timeout(void) { g_inject_timeout.store(1); }
 
 kla_status kla_check_device_error(void* stream) {
     unsigned int flag = 0, flag2 = 0, flag3 = 0, flag4 = 0;

@@ -53,7 +53,9 @@ kla_status kla_chunk_bwd_noalloc(const void* q, const void* k, const void* v, co
                                  const float* dS_T, const float* S_chunks, void* dq, void* dk, void* dv,
                                  float* deta, float* dg, float* dS0, int B, int T, int H, int Dk, int Dv,
                                  int chunk, int dtype, int out_dtype, void* stream) {
-    // Size check first, before touching the device: the scratch replaces the workspace.
+    // Size check first, before touching the device: the scratch replaces the workspace.  The
+    // bound is the CUDA-core backward's size; kla_chunk_bwd picks the tensor cores by itself
+    // when their larger layout also fits the scratch.
     const size_t need = kla_chunk_bwd_workspace_min(B, T, H, Dk, Dv, chunk, dtype, S_chunks != nullptr);
     if (need > kNoallocScratchBytes) {
         // The regular entry point reports the same condition with its own message; run its

@@ -636,6 +636,31 @@ __global__ void __launch_bounds__(GT, 1)
             st_piece_split(sm + G_DOR + (pc >> 3) * 16384 + 8192, sm + G_DRL + (pc >> 3) * 8192, i, pc & 7, x);
         }
     }
+    // ---- keys of zero norm.  There the write vanishes and the exact gradient is
+    //      dk_t = beta_t Gbar_t v_t (Gbar_t: gradient of the state after token t; Eq. (3) with
+    //      ||k_t|| = 0 gives beta_t = eta_t / eps).  The unit-key U holds 0 in column t, and that
+    //      column only ever meets khat_t = 0, except in row t of dkhat.  With u_t = beta_t v_t
+    //      put in its place, row t of dkhat (F^T Q + E^T Khat + delta_t U lambda^T) is exactly
+    //      dk_t, and every other result is unchanged.
+    {
+        const uint32_t z0 = __ballot_sync(0xffffffffu, lane < n && ms->r2[lane] == 0.f);
+        const uint32_t z1 = __ballot_sync(0xffffffffu, lane + 32 < n && ms->r2[lane + 32] == 0.f);
+        uint64_t zm = ((uint64_t)z1 << 32) | z0;
+        while (zm) {
+            const int t = __ffsll((long long)zm) - 1;
+            zm &= zm - 1;
+            const float bt = a.eps < 0.f ? ms->eta[t] : (a.eps > 0.f ? ms->eta[t] / a.eps : 0.f);
+            if (tid < DV && bt != 0.f) {
+                const float vt = __bfloat162float(
+                    static_cast<const __nv_bfloat16*>(a.v)[tok_index(b, t0 + t, h, T, H) * DV + tid]);
+                float hi, lo;
+                split_bf16(bt * vt, hi, lo);
+                const uint32_t off = tid * 128 + ((((uint32_t)t >> 3) ^ (uint32_t)(tid & 7)) << 4) + (t & 7) * 2;
+                *reinterpret_cast<__nv_bfloat16*>(sm + G_UH + off) = __float2bfloat16_rn(hi);
+                *reinterpret_cast<__nv_bfloat16*>(sm + G_UL + off) = __float2bfloat16_rn(lo);
+            }
+        }
+    }
     fence_proxy_async();
     tc_fence_before();
     __syncthreads();
@@ -954,7 +979,8 @@ __global__ void __launch_bounds__(GT, 1)
         if (2 * lane < n) a.dg[tok_index(b, t0 + 2 * lane, h, T, H)] = s;
         if (2 * lane + 1 < n) a.dg[tok_index(b, t0 + 2 * lane + 1, h, T, H)] = s - x0;
     }
-    // ---- dk = (dkhat - khat (khat . dkhat)) / r + khat dr
+    // ---- dk = (dkhat - khat (khat . dkhat)) / r + khat dr; at a zero-norm key dkhat already
+    //      is dk (the substitution in U above)
     if (!top) {
         const int i = ti_row;
         if (i < n) {
@@ -969,7 +995,7 @@ __global__ void __launch_bounds__(GT, 1)
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
                     const float kh = f[e] * ir;
-                    x[8 * u + e] = ir > 0.f ? fmaf(dkh[8 * u + e] - kh * kd, ir, kh * dr) : 0.f;
+                    x[8 * u + e] = ir > 0.f ? fmaf(dkh[8 * u + e] - kh * kd, ir, kh * dr) : dkh[8 * u + e];
                 }
             }
             st_row32<TOut>(static_cast<TOut*>(a.dk) + ti * DK + 32 * cq, x);

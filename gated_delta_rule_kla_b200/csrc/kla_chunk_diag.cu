@@ -1,0 +1,784 @@
+// kla_chunk_diag.cu -- KLA with diagonal (per-key-channel) gating on CUDA cores (fp32).
+//
+// "Kaczmarz Linear Attention", Appendix A.5 (the Kaczmarz step is decay-agnostic) and B.5 (the
+// chunk form under a diagonal decay): the decay of token t is Diag(alpha_t) with
+// alpha_t = exp(g_t), g_t in R^{Dk} (one log-decay per key channel), so per head
+//   Sbar = Diag(alpha_t) S_{t-1};  e_t = v_t - Sbar^T k_t;  S_t = Sbar + beta_t k_t e_t^T;
+//   o_t = S_t^T q_t,  beta_t = eta_t / (||k_t||^2 + eps)  (or eta_t as given, direct mode).
+//
+// Chunk form on unit keys (k = r khat, b = eta r^2/(r^2+eps), c = eta r/(r^2+eps) as for scalar
+// gating), with G_i = sum_{s<=i} g_s the per-channel log-decay inside the chunk and
+// E_ij = exp(G_i - G_j) (a vector over channels, j <= i, every factor <= 1 for g <= 0):
+//   L_ij = b_i sum_c khat_i[c] khat_j[c] E_ij[c]   (j < i)      P_ij = sum_c q_i[c] khat_j[c] E_ij[c]
+//   (I + L) U = Diag(c) V - Diag(b) (Khat o Gam) S                 Gam_i = exp(G_i)
+//   O = (Q o Gam) S + P U
+//   S' = Diag(Gam_last) S + (Khat o Del)^T U                       Del_j = exp(G_last - G_j)
+// Unlike scalar gating, the decay cannot be taken out of the channel sums, so the chunk's
+// pairwise factors are formed channel by channel.  The kernels use 16-token chunks: every factor
+// is then exp of a non-positive number (no rescaling reference that could overflow, whatever the
+// decay), and the pairwise work per token stays small.
+//
+// Columns of V, U, O, S are independent, so a CTA owns NV value columns of one (b, h) and walks
+// the chunks in order (forward) or newest first (backward, from the chunk-start states the
+// forward kernel saved in the workspace).  The backward's column-coupled gradients (dq, dkhat,
+// db, dc, dG per channel) are partial sums over a CTA's columns, added atomically into fp32
+// accumulators; a finishing kernel maps (dkhat, db, dc) to (dk, deta) and the per-channel dG to
+// dg by a reverse cumulative sum inside each 16-token chunk.
+#include "kla_device.cuh"
+#include "kla_launch.h"
+
+namespace kla {
+namespace {
+
+constexpr int CD = 16;               // internal chunk length of the diagonal-gated kernels
+constexpr int NP = CD * (CD + 1) / 2;  // pairs j <= i inside a chunk
+constexpr int NT = 256;
+
+__device__ __forceinline__ size_t tok_index(int b, int t, int h, int T, int H) {
+    return ((size_t)b * T + t) * H + h;
+}
+__device__ __forceinline__ int pair_index(int i, int j) { return i * (i + 1) / 2 + j; }
+
+// Rows of one 16-token chunk: unit keys, queries, raw log-decays (into Gs, summed afterwards)
+// and the per-token coefficients.  One warp per row; rows past the sequence are zero (they then
+// contribute nothing and the decays stay flat).
+template <int DK, typename Tin>
+__device__ __forceinline__ void load_rows(const FwdArgs& a, int b, int h, int t0, int n, float* Ks, float* Qs,
+                                          float* Gs, float* bs, float* cs, float* us) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    constexpr int PER = DK / 32, LDK = DK + 1;
+    const Tin* q = static_cast<const Tin*>(a.q);
+    const Tin* k = static_cast<const Tin*>(a.k);
+    for (int i = warp; i < CD; i += NT / 32) {
+        if (i < n) {
+            const size_t ti = tok_index(b, t0 + i, h, a.T, a.H);
+            float kv[PER];
+            float r2 = 0.f;
+#pragma unroll
+            for (int u = 0; u < PER; ++u) {
+                kv[u] = to_f32(k[ti * DK + lane + 32 * u]);
+                r2 = fmaf(kv[u], kv[u], r2);
+            }
+            r2 = warp_sum(r2);
+            const float et = a.eta[ti];
+            const KaczCoef cf = kacz_coef(et, r2, a.eps);
+#pragma unroll
+            for (int u = 0; u < PER; ++u) {
+                Ks[i * LDK + lane + 32 * u] = kv[u] * cf.inv_r;
+                Qs[i * LDK + lane + 32 * u] = to_f32(q[ti * DK + lane + 32 * u]);
+                Gs[i * DK + lane + 32 * u] = a.g[ti * DK + lane + 32 * u];
+            }
+            if (lane == 0) {
+                bs[i] = cf.b;
+                cs[i] = cf.c;
+                // value coefficient of U in the backward: c, except at a key of zero norm, where
+                // U's row takes beta v (it meets only khat = 0 there, and row i of dkhat then
+                // equals the exact dk = beta Gbar_i v_i)
+                if (us) us[i] = r2 == 0.f ? (a.eps < 0.f ? et : (a.eps > 0.f ? et / a.eps : 0.f)) : cf.c;
+            }
+        } else {
+#pragma unroll
+            for (int u = 0; u < PER; ++u) {
+                Ks[i * LDK + lane + 32 * u] = 0.f;
+                Qs[i * LDK + lane + 32 * u] = 0.f;
+                Gs[i * DK + lane + 32 * u] = 0.f;
+            }
+            if (lane == 0) {
+                bs[i] = 0.f;
+                cs[i] = 0.f;
+                if (us) us[i] = 0.f;
+            }
+        }
+    }
+}
+
+// Inclusive per-channel prefix sum of the log-decays over the chunk (one thread per channel).
+template <int DK>
+__device__ __forceinline__ void cumsum_rows(float* Gs) {
+    if (threadIdx.x < DK) {
+        float acc = 0.f;
+#pragma unroll
+        for (int i = 0; i < CD; ++i) {
+            acc += Gs[i * DK + threadIdx.x];
+            Gs[i * DK + threadIdx.x] = acc;
+        }
+    }
+}
+
+// Chunk Gram matrices from the pairwise per-channel decays: A_ij = sum_c khat_i khat_j E_ij
+// (j < i) and P_ij = sum_c q_i khat_j E_ij (j <= i).  One warp per pair, lanes over channels.
+// When Es is given the factors E_ij[c] are also kept there ([pair][channel]).
+template <int DK>
+__device__ __forceinline__ void chunk_grams(const float* Ks, const float* Qs, const float* Gs, float* Am, float* Pm,
+                                            float* Es) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    constexpr int PER = DK / 32, LDK = DK + 1, LDC = CD + 1;
+    for (int p = warp; p < NP; p += NT / 32) {
+        int i = 0;
+        while ((i + 1) * (i + 2) / 2 <= p) ++i;
+        const int j = p - i * (i + 1) / 2;
+        float sa = 0.f, sp = 0.f;
+#pragma unroll
+        for (int u = 0; u < PER; ++u) {
+            const int c = lane + 32 * u;
+            const float e = __expf(Gs[i * DK + c] - Gs[j * DK + c]);
+            if (Es) Es[p * DK + c] = e;
+            const float kj = Ks[j * LDK + c] * e;
+            sa = fmaf(Ks[i * LDK + c], kj, sa);
+            sp = fmaf(Qs[i * LDK + c], kj, sp);
+        }
+        sa = warp_sum(sa);
+        sp = warp_sum(sp);
+        if (lane == 0) {
+            Am[i * LDC + j] = (j < i) ? sa : 0.f;
+            Pm[i * LDC + j] = sp;
+            if (j < i) {
+                Am[j * LDC + i] = 0.f;
+                Pm[j * LDC + i] = 0.f;
+            } else {
+                Am[i * LDC + i] = 0.f;
+            }
+        }
+    }
+}
+
+// ------------------------------------------------------------------------------------
+// Forward: grid (Dv / NV, H, B); S_chunks (optional) receives the state at the start of every
+// 16-token chunk, [B, H, ceil(T/16), Dk, Dv] (the backward's input).
+// ------------------------------------------------------------------------------------
+template <int DK>
+constexpr size_t diag_fwd_smem_bytes() {
+    constexpr int NV = 64;
+    return sizeof(float) * (3 * CD * (DK + 1) + CD * DK + DK * (NV + 1) + 2 * CD * (NV + 1) + 2 * CD * (CD + 1) +
+                            2 * CD);
+}
+
+template <int DK, typename Tin, typename TOut>
+__global__ void __launch_bounds__(NT, 1) chunk_fwd_diag_kernel(FwdArgs a) {
+    constexpr int NV = 64;
+    constexpr int LDK = DK + 1, LDV = NV + 1, LDC = CD + 1;
+    constexpr int TMS = DK / 16;
+    extern __shared__ float sm[];
+    float* Ks = sm;               // CD x LDK  unit keys
+    float* Qs = Ks + CD * LDK;    // CD x LDK  queries
+    float* Ws = Qs + CD * LDK;    // CD x LDK  khat o Gam, later khat o Del
+    float* Gs = Ws + CD * LDK;    // CD x DK   log-decay prefix (per channel)
+    float* Ss = Gs + CD * DK;     // DK x LDV  state slice
+    float* Rs = Ss + DK * LDV;    // CD x LDV  c V -> R -> U
+    float* Xs = Rs + CD * LDV;    // CD x LDV  (Khat o Gam) S
+    float* Lm = Xs + CD * LDV;    // CD x LDC  L, then P
+    float* Pm = Lm + CD * LDC;    // CD x LDC
+    float* bs = Pm + CD * LDC;
+    float* cs = bs + CD;
+
+    const int v0 = blockIdx.x * NV, h = blockIdx.y, b = blockIdx.z;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int tx = tid & 15, ty = tid >> 4;
+    const int T = a.T, H = a.H, Dv = a.Dv;
+    const Tin* v = static_cast<const Tin*>(a.v);
+    TOut* o = static_cast<TOut*>(a.o);
+    const size_t sbase = ((size_t)b * H + h) * DK * Dv;
+    const int NC = (T + CD - 1) / CD;
+
+    for (int x = tid; x < DK * NV; x += NT) {
+        const int r = x / NV, c = x % NV;
+        Ss[r * LDV + c] = a.S0 ? a.S0[sbase + (size_t)r * Dv + v0 + c] : 0.f;
+    }
+
+    for (int ci = 0; ci < NC; ++ci) {
+        const int t0 = ci * CD;
+        const int n = min(CD, T - t0);
+        __syncthreads();
+        if (a.S_chunks) {
+            float* dst = a.S_chunks + (((size_t)b * H + h) * NC + ci) * DK * Dv;
+            for (int x = tid; x < DK * NV; x += NT) {
+                const int r = x / NV, c = x % NV;
+                dst[(size_t)r * Dv + v0 + c] = Ss[r * LDV + c];
+            }
+        }
+        load_rows<DK, Tin>(a, b, h, t0, n, Ks, Qs, Gs, bs, cs, nullptr);
+        __syncthreads();
+        cumsum_rows<DK>(Gs);
+        // c V into Rs
+        for (int i = warp; i < CD; i += NT / 32) {
+            for (int j = lane; j < NV; j += 32) {
+                float val = 0.f;
+                if (i < n) val = cs[i] * to_f32(v[tok_index(b, t0 + i, h, T, H) * Dv + v0 + j]);
+                Rs[i * LDV + j] = val;
+            }
+        }
+        __syncthreads();
+        chunk_grams<DK>(Ks, Qs, Gs, Lm, Pm, nullptr);
+        for (int x = tid; x < CD * DK; x += NT) {  // khat o Gam
+            const int i = x / DK, c = x % DK;
+            Ws[i * LDK + c] = Ks[i * LDK + c] * __expf(Gs[i * DK + c]);
+        }
+        __syncthreads();
+        // X = (Khat o Gam) S: one row per ty, four columns per thread
+        {
+            float ax[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+            for (int d = 0; d < DK; ++d) {
+                const float w = Ws[ty * LDK + d];
+#pragma unroll
+                for (int nn = 0; nn < 4; ++nn) ax[nn] = fmaf(w, Ss[d * LDV + tx + 16 * nn], ax[nn]);
+            }
+#pragma unroll
+            for (int nn = 0; nn < 4; ++nn) Xs[ty * LDV + tx + 16 * nn] = ax[nn];
+        }
+        __syncthreads();
+        // R = c V - Diag(b) X; L = Diag(b) A
+        for (int x = tid; x < CD * NV; x += NT) {
+            const int i = x / NV, j = x % NV;
+            Rs[i * LDV + j] -= bs[i] * Xs[i * LDV + j];
+        }
+        if (tid < CD * CD) {
+            const int i = tid / CD, j = tid % CD;
+            Lm[i * LDC + j] *= bs[i];
+        }
+        __syncthreads();
+        // Forward substitution (I + L) U = R, row by row (Appendix B.2)
+        {
+            const int col = tid >> 2, part = tid & 3;
+            for (int i = 1; i < n; ++i) {
+                if (col < NV) {
+                    float s = 0.f;
+                    for (int j = part; j < i; j += 4) s = fmaf(Lm[i * LDC + j], Rs[j * LDV + col], s);
+                    s += __shfl_xor_sync(0xffffffffu, s, 1);
+                    s += __shfl_xor_sync(0xffffffffu, s, 2);
+                    if (part == 0) Rs[i * LDV + col] -= s;
+                }
+                __syncthreads();
+            }
+        }
+        // O = (Q o Gam) S + P U
+        if (o != nullptr) {
+            float ao[4] = {0.f, 0.f, 0.f, 0.f};
+            const int i = ty;
+#pragma unroll 4
+            for (int d = 0; d < DK; ++d) {
+                const float w = Qs[i * LDK + d] * __expf(Gs[i * DK + d]);
+#pragma unroll
+                for (int nn = 0; nn < 4; ++nn) ao[nn] = fmaf(w, Ss[d * LDV + tx + 16 * nn], ao[nn]);
+            }
+#pragma unroll
+            for (int t = 0; t < CD; ++t) {
+                const float p = Pm[i * LDC + t];
+#pragma unroll
+                for (int nn = 0; nn < 4; ++nn) ao[nn] = fmaf(p, Rs[t * LDV + tx + 16 * nn], ao[nn]);
+            }
+            if (i < n) {
+                TOut* orow = o + tok_index(b, t0 + i, h, T, H) * Dv + v0;
+#pragma unroll
+                for (int nn = 0; nn < 4; ++nn) orow[tx + 16 * nn] = from_f32<TOut>(ao[nn]);
+            }
+        }
+        // khat o Del, Del_j = exp(G_last - G_j)
+        for (int x = tid; x < CD * DK; x += NT) {
+            const int i = x / DK, c = x % DK;
+            Ws[i * LDK + c] = Ks[i * LDK + c] * __expf(Gs[(n - 1) * DK + c] - Gs[i * DK + c]);
+        }
+        __syncthreads();
+        // S' = Diag(Gam_last) S + (Khat o Del)^T U
+        {
+            float as[TMS][4];
+#pragma unroll
+            for (int m = 0; m < TMS; ++m)
+#pragma unroll
+                for (int nn = 0; nn < 4; ++nn) as[m][nn] = 0.f;
+#pragma unroll
+            for (int t = 0; t < CD; ++t) {
+                float uu[4];
+#pragma unroll
+                for (int nn = 0; nn < 4; ++nn) uu[nn] = Rs[t * LDV + tx + 16 * nn];
+#pragma unroll
+                for (int m = 0; m < TMS; ++m) {
+                    const float w = Ws[t * LDK + ty + 16 * m];
+#pragma unroll
+                    for (int nn = 0; nn < 4; ++nn) as[m][nn] = fmaf(w, uu[nn], as[m][nn]);
+                }
+            }
+#pragma unroll
+            for (int m = 0; m < TMS; ++m) {
+                const int r = ty + 16 * m;
+                const float gl_r = __expf(Gs[(n - 1) * DK + r]);
+#pragma unroll
+                for (int nn = 0; nn < 4; ++nn) {
+                    float* sp = &Ss[r * LDV + tx + 16 * nn];
+                    *sp = fmaf(gl_r, *sp, as[m][nn]);
+                }
+            }
+        }
+    }
+    __syncthreads();
+    if (a.S_T) {
+        for (int x = tid; x < DK * NV; x += NT) {
+            const int r = x / NV, c = x % NV;
+            a.S_T[sbase + (size_t)r * Dv + v0 + c] = Ss[r * LDV + c];
+        }
+    }
+}
+
+// ------------------------------------------------------------------------------------
+// Backward.  Per chunk (newest first) with incoming state S and lambda = dS' (gradient of the
+// outgoing state), Gam_i = exp(G_i), Del_j = exp(G_last - G_j) (vectors over channels):
+//   dU  = P^T dO + (Khat o Del) lambda,   dR = (I + L)^{-T} dU (back substitution)
+//   dS  = Diag(Gam_last) lambda + (Q o Gam)^T dO - (Diag(b) (Khat o Gam))^T dR     (carried on)
+//   dv  = Diag(c) dR,  dc_i = dR_i . v_i
+//   Y   = dO U^T (lower),  D = -dR U^T (strictly lower)
+//   Z1 = dO S^T, Z2 = dR S^T, Z3 = U lambda^T                     (rows: tokens, columns: channels)
+//   F1_i = sum_{j<=i} Y_ij khat_j o E_ij     F2_j = sum_{i>=j} Y_ij q_i o E_ij
+//   F3_i = sum_{j<i}  D_ij khat_j o E_ij     F4_j = sum_{i>j}  D_ij b_i khat_i o E_ij
+//   dq_i    = Gam_i o Z1_i + F1_i
+//   dkhat_i = -b_i Gam_i o Z2_i + Del_i o Z3_i + F2_i + b_i F3_i + F4_i
+//   db_i    = sum_{j<i} D_ij A_ij - (khat_i o Gam_i) . Z2_i
+//   dG_i    = Gam_i o q_i o Z1_i + q_i o F1_i - b_i Gam_i o khat_i o Z2_i - khat_i o F2_i
+//             + b_i khat_i o F3_i - khat_i o F4_i - Del_i o khat_i o Z3_i
+//   dG_last += sum_j Del_j o khat_j o Z3_j + Gam_last o rowsum(lambda o S)
+// ------------------------------------------------------------------------------------
+template <int DK>
+constexpr size_t diag_bwd_smem_bytes() {
+    constexpr int NV = 32;
+    return sizeof(float) * (2 * CD * (DK + 1) + CD * DK + NP * DK + 2 * DK * (NV + 1) + 4 * CD * (NV + 1) +
+                            5 * CD * (CD + 1) + 4 * CD + 8 + DK);
+}
+
+template <int DK, typename Tin, typename TOut>
+__global__ void __launch_bounds__(NT, 1) chunk_bwd_diag_kernel(BwdArgs a, FwdArgs f) {
+    constexpr int NV = 32;
+    constexpr int LDK = DK + 1, LDV = NV + 1, LDC = CD + 1;
+    constexpr int TMK = DK / 16;
+    constexpr int EPT = CD * DK / NT;  // (token, channel) elements per thread
+    extern __shared__ float sm[];
+    float* Ks = sm;               // CD x LDK  unit keys
+    float* Qs = Ks + CD * LDK;    // CD x LDK
+    float* Gs = Qs + CD * LDK;    // CD x DK   log-decay prefix
+    float* Es = Gs + CD * DK;     // NP x DK   E_ij per channel
+    float* Ss = Es + NP * DK;     // DK x LDV  incoming state slice
+    float* dSs = Ss + DK * LDV;   // DK x LDV  gradient of the outgoing state slice
+    float* Us = dSs + DK * LDV;   // CD x LDV  cV -> R -> U
+    float* dRs = Us + CD * LDV;   // CD x LDV  dU -> dR
+    float* dOs = dRs + CD * LDV;  // CD x LDV
+    float* Xs = dOs + CD * LDV;   // CD x LDV  (Khat o Gam) S, then (Khat o Del) lambda
+    float* Am = Xs + CD * LDV;    // CD x LDC  A (strictly lower, without b)
+    float* Lm = Am + CD * LDC;    // CD x LDC  L = Diag(b) A
+    float* Pm = Lm + CD * LDC;    // CD x LDC
+    float* Ym = Pm + CD * LDC;    // CD x LDC  Y = dO U^T (lower)
+    float* Dm = Ym + CD * LDC;    // CD x LDC  D = -dR U^T (strictly lower)
+    float* bs = Dm + CD * LDC;
+    float* cs = bs + CD;
+    float* us = cs + CD;
+    float* dbs = us + CD;
+    float* red = dbs + CD;        // 8
+    float* lsS = red + 8;         // DK: row sums of lambda o S over this slice
+
+    const int v0 = blockIdx.x * NV, h = blockIdx.y, b = blockIdx.z;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int tx = tid & 15, ty = tid >> 4;
+    const int T = a.T, H = a.H, Dv = a.Dv;
+    const Tin* v = static_cast<const Tin*>(a.v);
+    const Tin* dO = static_cast<const Tin*>(a.dO);
+    TOut* dv = static_cast<TOut*>(a.dv);
+    const size_t sbase = ((size_t)b * H + h) * DK * Dv;
+    const int NC = (T + CD - 1) / CD;
+
+    for (int x = tid; x < DK * NV; x += NT) {
+        const int r = x / NV, c = x % NV;
+        dSs[r * LDV + c] = a.dS_T ? a.dS_T[sbase + (size_t)r * Dv + v0 + c] : 0.f;
+    }
+
+    for (int ci = NC - 1; ci >= 0; --ci) {
+        const int t0 = ci * CD;
+        const int n = min(CD, T - t0);
+        __syncthreads();
+        load_rows<DK, Tin>(f, b, h, t0, n, Ks, Qs, Gs, bs, cs, us);
+        {
+            const float* src = a.S_chunks + (((size_t)b * H + h) * NC + ci) * DK * Dv;
+            for (int x = tid; x < DK * NV; x += NT) {
+                const int r = x / NV, c = x % NV;
+                Ss[r * LDV + c] = src[(size_t)r * Dv + v0 + c];
+            }
+        }
+        for (int x = tid; x < CD * NV; x += NT) {  // one column per lane
+            const int i = x / NV, j = x % NV;
+            float uv = 0.f, dov = 0.f;
+            if (i < n) {
+                const size_t ti = tok_index(b, t0 + i, h, T, H);
+                uv = to_f32(v[ti * Dv + v0 + j]);
+                dov = to_f32(dO[ti * Dv + v0 + j]);
+            }
+            Us[i * LDV + j] = uv;  // scaled by its coefficient below
+            dOs[i * LDV + j] = dov;
+        }
+        if (tid < CD) dbs[tid] = 0.f;
+        __syncthreads();
+        cumsum_rows<DK>(Gs);
+        for (int x = tid; x < CD * NV; x += NT) {
+            const int i = x / NV, j = x % NV;
+            Us[i * LDV + j] *= us[i];
+        }
+        __syncthreads();
+        chunk_grams<DK>(Ks, Qs, Gs, Am, Pm, Es);
+        // X = (Khat o Gam) S and the lambda o S row sums
+        {
+            float ax[2] = {0.f, 0.f};
+#pragma unroll 4
+            for (int d = 0; d < DK; ++d) {
+                const float w = Ks[ty * LDK + d] * __expf(Gs[ty * DK + d]);
+#pragma unroll
+                for (int nn = 0; nn < 2; ++nn) ax[nn] = fmaf(w, Ss[d * LDV + tx + 16 * nn], ax[nn]);
+            }
+#pragma unroll
+            for (int nn = 0; nn < 2; ++nn) Xs[ty * LDV + tx + 16 * nn] = ax[nn];
+        }
+        if (tid < DK) {
+            float p = 0.f;
+#pragma unroll 8
+            for (int c = 0; c < NV; ++c) p = fmaf(dSs[tid * LDV + c], Ss[tid * LDV + c], p);
+            lsS[tid] = p;
+        }
+        __syncthreads();
+        for (int x = tid; x < CD * NV; x += NT) {
+            const int i = x / NV, j = x % NV;
+            Us[i * LDV + j] -= bs[i] * Xs[i * LDV + j];
+        }
+        if (tid < CD * CD) {
+            const int i = tid / CD, j = tid % CD;
+            Lm[i * LDC + j] = bs[i] * Am[i * LDC + j];
+        }
+        __syncthreads();
+        // U = (I + L)^{-1} R, row by row
+        {
+            const int col = tid >> 3, part = tid & 7;
+            for (int i = 1; i < n; ++i) {
+                float s = 0.f;
+                for (int j = part; j < i; j += 8) s = fmaf(Lm[i * LDC + j], Us[j * LDV + col], s);
+                s += __shfl_xor_sync(0xffffffffu, s, 1);
+                s += __shfl_xor_sync(0xffffffffu, s, 2);
+                s += __shfl_xor_sync(0xffffffffu, s, 4);
+                if (part == 0) Us[i * LDV + col] -= s;
+                __syncthreads();
+            }
+        }
+        // dU = P^T dO + (Khat o Del) lambda
+        {
+            float ad[2] = {0.f, 0.f};
+            const int i = ty;
+#pragma unroll 4
+            for (int d = 0; d < DK; ++d) {
+                const float w = Ks[i * LDK + d] * __expf(Gs[(n - 1) * DK + d] - Gs[i * DK + d]);
+#pragma unroll
+                for (int nn = 0; nn < 2; ++nn) ad[nn] = fmaf(w, dSs[d * LDV + tx + 16 * nn], ad[nn]);
+            }
+#pragma unroll
+            for (int t = 0; t < CD; ++t) {
+                const float p = Pm[t * LDC + i];
+#pragma unroll
+                for (int nn = 0; nn < 2; ++nn) ad[nn] = fmaf(p, dOs[t * LDV + tx + 16 * nn], ad[nn]);
+            }
+#pragma unroll
+            for (int nn = 0; nn < 2; ++nn) dRs[i * LDV + tx + 16 * nn] = ad[nn];
+        }
+        __syncthreads();
+        // dR = (I + L)^{-T} dU, newest row first
+        {
+            const int col = tid >> 3, part = tid & 7;
+            for (int j = n - 2; j >= 0; --j) {
+                float s = 0.f;
+                for (int i = j + 1 + part; i < n; i += 8) s = fmaf(Lm[i * LDC + j], dRs[i * LDV + col], s);
+                s += __shfl_xor_sync(0xffffffffu, s, 1);
+                s += __shfl_xor_sync(0xffffffffu, s, 2);
+                s += __shfl_xor_sync(0xffffffffu, s, 4);
+                if (part == 0) dRs[j * LDV + col] -= s;
+                __syncthreads();
+            }
+        }
+        // dv, dc; Y = dO U^T, D = -dR U^T; then db's D o A part
+        for (int i = warp; i < n; i += NT / 32) {
+            const size_t ti = tok_index(b, t0 + i, h, T, H);
+            const float dr = dRs[i * LDV + lane];
+            dv[ti * Dv + v0 + lane] = from_f32<TOut>(cs[i] * dr);
+            const float s_rv = warp_sum(dr * to_f32(v[ti * Dv + v0 + lane]));
+            if (lane == 0) atomicAdd(&a.acc_dc[ti], s_rv);
+        }
+        {
+            const int i = ty, j = tx;  // 16 x 16 = 256 threads
+            float y = 0.f, dd = 0.f;
+#pragma unroll 8
+            for (int c = 0; c < NV; ++c) {
+                const float uj = Us[j * LDV + c];
+                y = fmaf(dOs[i * LDV + c], uj, y);
+                dd = fmaf(dRs[i * LDV + c], uj, dd);
+            }
+            Ym[i * LDC + j] = (j <= i) ? y : 0.f;
+            Dm[i * LDC + j] = (j < i) ? -dd : 0.f;
+        }
+        __syncthreads();
+        if (tid < CD) {
+            float s = 0.f;
+            for (int j = 0; j < tid; ++j) s = fmaf(Dm[tid * LDC + j], Am[tid * LDC + j], s);
+            atomicAdd(&dbs[tid], s);
+        }
+        // per (token, channel): dq, dkhat and dG partials (this thread: token ty, channels
+        // tx + 16 u)
+        {
+            const int i = ty;
+            float zq[EPT], zr[EPT], zl[EPT];
+#pragma unroll
+            for (int u = 0; u < EPT; ++u) zq[u] = zr[u] = zl[u] = 0.f;
+            // Z1 = dO S^T, Z2 = dR S^T, Z3 = U lambda^T (contraction over this CTA's columns)
+#pragma unroll 4
+            for (int c = 0; c < NV; ++c) {
+                const float o_ = dOs[i * LDV + c], r_ = dRs[i * LDV + c], u_ = Us[i * LDV + c];
+#pragma unroll
+                for (int u = 0; u < EPT; ++u) {
+                    const int d = tx + 16 * u;
+                    zq[u] = fmaf(o_, Ss[d * LDV + c], zq[u]);
+                    zr[u] = fmaf(r_, Ss[d * LDV + c], zr[u]);
+                    zl[u] = fmaf(u_, dSs[d * LDV + c], zl[u]);
+                }
+            }
+            float f1[EPT], f2[EPT], f3[EPT], f4[EPT];
+#pragma unroll
+            for (int u = 0; u < EPT; ++u) f1[u] = f2[u] = f3[u] = f4[u] = 0.f;
+            for (int j = 0; j <= i; ++j) {  // F1, F3: row i against earlier tokens j
+                const float y = Ym[i * LDC + j], dd = Dm[i * LDC + j];
+                const float* E = Es + pair_index(i, j) * DK;
+#pragma unroll
+                for (int u = 0; u < EPT; ++u) {
+                    const int d = tx + 16 * u;
+                    const float ke = Ks[j * LDK + d] * E[d];
+                    f1[u] = fmaf(y, ke, f1[u]);
+                    f3[u] = fmaf(dd, ke, f3[u]);
+                }
+            }
+            for (int r = i; r < n; ++r) {  // F2, F4: column i against later tokens r
+                const float y = Ym[r * LDC + i], dd = Dm[r * LDC + i] * bs[r];
+                const float* E = Es + pair_index(r, i) * DK;
+#pragma unroll
+                for (int u = 0; u < EPT; ++u) {
+                    const int d = tx + 16 * u;
+                    f2[u] = fmaf(y, Qs[r * LDK + d] * E[d], f2[u]);
+                    f4[u] = fmaf(dd, Ks[r * LDK + d] * E[d], f4[u]);
+                }
+            }
+            float kgz = 0.f;
+            if (i < n) {
+                const size_t ti = tok_index(b, t0 + i, h, T, H);
+                const float bi = bs[i];
+#pragma unroll
+                for (int u = 0; u < EPT; ++u) {
+                    const int d = tx + 16 * u;
+                    const float G = Gs[i * DK + d], Gl = Gs[(n - 1) * DK + d];
+                    const float gam = __expf(G), del = __expf(Gl - G);
+                    const float qd = Qs[i * LDK + d], kd = Ks[i * LDK + d];
+                    const float dq = fmaf(gam, zq[u], f1[u]);
+                    const float dk = -bi * gam * zr[u] + del * zl[u] + f2[u] + bi * f3[u] + f4[u];
+                    float dG = gam * qd * zq[u] + qd * f1[u] - bi * gam * kd * zr[u] - kd * f2[u] + bi * kd * f3[u] -
+                               kd * f4[u] - del * kd * zl[u];
+                    kgz = fmaf(kd * gam, zr[u], kgz);
+                    atomicAdd(&a.acc_dq[ti * DK + d], dq);
+                    atomicAdd(&a.acc_dkh[ti * DK + d], dk);
+                    atomicAdd(&a.acc_dG[ti * DK + d], dG);
+                    // the outgoing decays (Del_j and Gam_last) feed dG of the chunk's last token
+                    const size_t tl = tok_index(b, t0 + n - 1, h, T, H);
+                    float extra = del * kd * zl[u];
+                    if (i == n - 1) extra += __expf(Gl) * lsS[d];
+                    atomicAdd(&a.acc_dG[tl * DK + d], extra);
+                }
+            }
+            // db: - (khat_i o Gam_i) . Z2_i (this thread's channels, then the row's 16 threads)
+            kgz += __shfl_xor_sync(0xffffffffu, kgz, 1);
+            kgz += __shfl_xor_sync(0xffffffffu, kgz, 2);
+            kgz += __shfl_xor_sync(0xffffffffu, kgz, 4);
+            kgz += __shfl_xor_sync(0xffffffffu, kgz, 8);
+            if (tx == 0 && i < n) atomicAdd(&dbs[i], -kgz);
+        }
+        // new lambda = Diag(Gam_last) lambda + (Q o Gam)^T dO - (Diag(b) (Khat o Gam))^T dR
+        {
+            float as[TMK][2];
+#pragma unroll
+            for (int m = 0; m < TMK; ++m) as[m][0] = as[m][1] = 0.f;
+#pragma unroll
+            for (int t = 0; t < CD; ++t) {
+                float o2[2], r2[2];
+#pragma unroll
+                for (int nn = 0; nn < 2; ++nn) {
+                    o2[nn] = dOs[t * LDV + tx + 16 * nn];
+                    r2[nn] = -bs[t] * dRs[t * LDV + tx + 16 * nn];
+                }
+#pragma unroll
+                for (int m = 0; m < TMK; ++m) {
+                    const int r = ty + 16 * m;
+                    const float gm = __expf(Gs[t * DK + r]);
+                    const float wq = Qs[t * LDK + r] * gm, wk = Ks[t * LDK + r] * gm;
+#pragma unroll
+                    for (int nn = 0; nn < 2; ++nn) as[m][nn] = fmaf(wq, o2[nn], fmaf(wk, r2[nn], as[m][nn]));
+                }
+            }
+            __syncthreads();
+#pragma unroll
+            for (int m = 0; m < TMK; ++m) {
+                const int r = ty + 16 * m;
+                const float gl_r = __expf(Gs[(n - 1) * DK + r]);
+#pragma unroll
+                for (int nn = 0; nn < 2; ++nn) {
+                    float* sp = &dSs[r * LDV + tx + 16 * nn];
+                    *sp = fmaf(gl_r, *sp, as[m][nn]);
+                }
+            }
+        }
+        __syncthreads();
+        if (tid < n) atomicAdd(&a.acc_db[tok_index(b, t0 + tid, h, T, H)], dbs[tid]);
+    }
+    __syncthreads();
+    for (int x = tid; x < DK * NV; x += NT) {
+        const int r = x / NV, c = x % NV;
+        a.dS0[sbase + (size_t)r * Dv + v0 + c] = dSs[r * LDV + c];
+    }
+}
+
+// dq to the output type; dk and deta from the unit-key gradients (as for scalar gating):
+//   deta = db r^2/den + dc r/den,  dr = db eta 2 r eps/den^2 + dc eta (eps - r^2)/den^2
+//   dk   = (dkhat - khat (khat . dkhat)) / r + khat dr;  at a key of zero norm dkhat already is dk
+template <int DK, typename Tin, typename TOut>
+__global__ void __launch_bounds__(256) diag_finalize_kernel(BwdArgs a, size_t ntok) {
+    const size_t w = (size_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (w >= ntok) return;
+    constexpr int PER = DK / 32;
+    const Tin* k = static_cast<const Tin*>(a.k);
+    TOut* dq = static_cast<TOut*>(a.dq);
+    TOut* dk = static_cast<TOut*>(a.dk);
+    float kv[PER], dkh[PER];
+    float r2 = 0.f;
+#pragma unroll
+    for (int u = 0; u < PER; ++u) {
+        kv[u] = to_f32(k[w * DK + lane + 32 * u]);
+        dkh[u] = a.acc_dkh[w * DK + lane + 32 * u];
+        r2 = fmaf(kv[u], kv[u], r2);
+        dq[w * DK + lane + 32 * u] = from_f32<TOut>(a.acc_dq[w * DK + lane + 32 * u]);
+    }
+    r2 = warp_sum(r2);
+    const float r = sqrtf(r2);
+    const float den = r2 + a.eps;
+    const bool direct = a.eps < 0.f;
+    const bool live = (direct || den > 0.f) && r > 0.f;
+    const float inv_r = live ? 1.f / r : 0.f;
+    float kd = 0.f;
+#pragma unroll
+    for (int u = 0; u < PER; ++u) kd = fmaf(kv[u] * inv_r, dkh[u], kd);
+    kd = warp_sum(kd);
+    const float db = a.acc_db[w], dc = a.acc_dc[w], et = a.eta[w];
+    float deta = 0.f, dr = 0.f;
+    if (live && direct) {
+        deta = db * r2 + dc * r;
+        dr = db * et * 2.f * r + dc * et;
+    } else if (live) {
+        deta = db * r2 / den + dc * r / den;
+        dr = (db * et * 2.f * r * a.eps + dc * et * (a.eps - r2)) / (den * den);
+    }
+#pragma unroll
+    for (int u = 0; u < PER; ++u) {
+        const float kh = kv[u] * inv_r;
+        const float val = live ? (dkh[u] - kh * kd) * inv_r + kh * dr : dkh[u];
+        dk[w * DK + lane + 32 * u] = from_f32<TOut>(val);
+    }
+    if (lane == 0) a.deta[w] = deta;
+}
+
+// dg_r[c] = sum_{i >= r} dG_i[c] inside each 16-token chunk (one thread per chunk and channel).
+template <int DK>
+__global__ void diag_dg_kernel(BwdArgs a) {
+    const int NC = (a.T + CD - 1) / CD;
+    const size_t id = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const size_t total = (size_t)a.B * a.H * NC * DK;
+    if (id >= total) return;
+    const int c = (int)(id % DK);
+    const size_t ch = id / DK;
+    const int h = (int)(ch % a.H);
+    const int ci = (int)((ch / a.H) % NC);
+    const int b = (int)(ch / ((size_t)a.H * NC));
+    const int t0 = ci * CD;
+    const int n = min(CD, a.T - t0);
+    float acc = 0.f;
+    for (int i = n - 1; i >= 0; --i) {
+        const size_t ti = tok_index(b, t0 + i, h, a.T, a.H) * DK + c;
+        acc += a.acc_dG[ti];
+        a.dg[ti] = acc;
+    }
+}
+
+template <int DK, typename Tin, typename TOut>
+cudaError_t diag_fwd_launch(const FwdArgs& a, cudaStream_t st) {
+    const size_t smem = diag_fwd_smem_bytes<DK>();
+    cudaError_t e = cudaFuncSetAttribute(chunk_fwd_diag_kernel<DK, Tin, TOut>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    chunk_fwd_diag_kernel<DK, Tin, TOut><<<dim3(a.Dv / 64, a.H, a.B), NT, smem, st>>>(a);
+    return cudaGetLastError();
+}
+
+template <int DK, typename Tin, typename TOut>
+cudaError_t diag_bwd_launch(const BwdArgs& a, const FwdArgs& f, cudaStream_t st) {
+    const size_t smem = diag_bwd_smem_bytes<DK>();
+    cudaError_t e = cudaFuncSetAttribute(chunk_bwd_diag_kernel<DK, Tin, TOut>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    chunk_bwd_diag_kernel<DK, Tin, TOut><<<dim3(a.Dv / 32, a.H, a.B), NT, smem, st>>>(a, f);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    const size_t ntok = (size_t)a.B * a.T * a.H;
+    diag_finalize_kernel<DK, Tin, TOut><<<(unsigned)((ntok + 7) / 8), 256, 0, st>>>(a, ntok);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    const size_t nth = (size_t)a.B * a.H * ((a.T + CD - 1) / CD) * DK;
+    diag_dg_kernel<DK><<<(unsigned)((nth + 255) / 256), 256, 0, st>>>(a);
+    return cudaGetLastError();
+}
+
+template <int DK, typename Tin>
+cudaError_t diag_fwd_o(const FwdArgs& a, cudaStream_t st) {
+    return a.out_bf16 ? diag_fwd_launch<DK, Tin, __nv_bfloat16>(a, st) : diag_fwd_launch<DK, Tin, float>(a, st);
+}
+template <int DK, typename Tin>
+cudaError_t diag_bwd_o(const BwdArgs& a, const FwdArgs& f, cudaStream_t st) {
+    return a.out_bf16 ? diag_bwd_launch<DK, Tin, __nv_bfloat16>(a, f, st) : diag_bwd_launch<DK, Tin, float>(a, f, st);
+}
+
+}  // namespace
+
+int diag_chunk_len() { return CD; }
+
+cudaError_t launch_chunk_fwd_diag(const FwdArgs& a, cudaStream_t st) {
+    if (a.bf16) return a.Dk == 128 ? diag_fwd_o<128, __nv_bfloat16>(a, st) : diag_fwd_o<64, __nv_bfloat16>(a, st);
+    return a.Dk == 128 ? diag_fwd_o<128, float>(a, st) : diag_fwd_o<64, float>(a, st);
+}
+
+// The backward: the forward kernel first writes every 16-token chunk's starting state into
+// a.S_chunks (the workspace), then the reverse pass, the finishing kernel and the dg scan.
+// The accumulators in `a` must be zeroed before this is called.
+cudaError_t launch_chunk_bwd_diag(const BwdArgs& a, const float* S0, cudaStream_t st) {
+    FwdArgs f{};
+    f.q = a.q;
+    f.k = a.k;
+    f.v = a.v;
+    f.eta = a.eta;
+    f.g = a.g;
+    f.eps = a.eps;
+    f.S0 = S0;
+    f.o = nullptr;
+    f.S_T = nullptr;
+    f.S_chunks = const_cast<float*>(a.S_chunks);
+    f.B = a.B;
+    f.T = a.T;
+    f.H = a.H;
+    f.Dk = a.Dk;
+    f.Dv = a.Dv;
+    f.bf16 = a.bf16;
+    f.out_bf16 = false;
+    cudaError_t e = launch_chunk_fwd_diag(f, st);
+    if (e != cudaSuccess) return e;
+    if (a.bf16) return a.Dk == 128 ? diag_bwd_o<128, __nv_bfloat16>(a, f, st) : diag_bwd_o<64, __nv_bfloat16>(a, f, st);
+    return a.Dk == 128 ? diag_bwd_o<128, float>(a, f, st) : diag_bwd_o<64, float>(a, f, st);
+}
+
+}  // namespace kla

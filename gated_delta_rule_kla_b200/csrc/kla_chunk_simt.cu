@@ -62,7 +62,8 @@ __device__ __forceinline__ void load_qk_rows(const Tin* __restrict__ q, const Ti
                                              const float* __restrict__ eta,
                                              const float* __restrict__ g, float eps, int b, int h,
                                              int t0, int n, int T, int H, float* Ks, float* Qs,
-                                             int ldk, float* graw, float* bs, float* cs) {
+                                             int ldk, float* graw, float* bs, float* cs,
+                                             float* us = nullptr) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     constexpr int PER = DK / 32;
     for (int i = warp; i < C; i += NT / 32) {
@@ -88,6 +89,10 @@ __device__ __forceinline__ void load_qk_rows(const Tin* __restrict__ q, const Ti
                 graw[i] = g[ti];
                 bs[i] = cf.b;
                 cs[i] = cf.c;
+                // value coefficient of U for the backward: c, except at a key of zero norm,
+                // where U's row takes beta v (it meets only khat = 0 there, but row i of dkhat
+                // then equals the exact dk = beta Gbar v)
+                if (us) us[i] = r2 == 0.f ? (eps < 0.f ? eta[ti] : (eps > 0.f ? eta[ti] / eps : 0.f)) : cf.c;
             }
         } else {
 #pragma unroll
@@ -99,6 +104,7 @@ __device__ __forceinline__ void load_qk_rows(const Tin* __restrict__ q, const Ti
                 graw[i] = 0.f;
                 bs[i] = 0.f;
                 cs[i] = 0.f;
+                if (us) us[i] = 0.f;
             }
         }
     }
@@ -333,6 +339,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_bwd_simt_kernel(BwdArgs a) {
     float* dcs = dbs + C;
     float* red = dcs + C;  // 8
     float* Tf = red + 8;                // C x tcc::LDL   T = (I + L)^{-1}  (16-byte aligned)
+    float* ucs = Tf + C * tcc::LDL + 1024 + C * LDV;  // C   value coefficient of U
     float* Xinv = Tf + C * tcc::LDL;    // 1024           scratch of the inverse
     float* Tmp = Xinv + 1024;           // C x LDV        U = T R and dR = T^T dU before copy-back
 
@@ -357,7 +364,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_bwd_simt_kernel(BwdArgs a) {
         const int t0 = ci * C;
         const int n = min(C, T - t0);
         __syncthreads();
-        load_qk_rows<DK, Tin>(q, k, a.eta, a.g, a.eps, b, h, t0, n, T, H, Ks, Qs, LDK, graw, bs, cs);
+        load_qk_rows<DK, Tin>(q, k, a.eta, a.g, a.eps, b, h, t0, n, T, H, Ks, Qs, LDK, graw, bs, cs, ucs);
         {
             const float* src = a.S_chunks + (((size_t)b * H + h) * NC + ci) * DK * Dv;
             for (int x = tid; x < DK * NV; x += NT) {
@@ -375,7 +382,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_bwd_simt_kernel(BwdArgs a) {
             float cv = 0.f, dov = 0.f;
             if (i < n) {
                 const size_t ti = tok_index(b, t0 + i, h, T, H);
-                cv = cs[i] * to_f32(v[ti * Dv + v0 + lane]);
+                cv = ucs[i] * to_f32(v[ti * Dv + v0 + lane]);
                 dov = to_f32(dO[ti * Dv + v0 + lane]);
             }
             Us[i * LDV + lane] = cv;
@@ -662,13 +669,14 @@ __global__ void __launch_bounds__(NT, 1) chunk_bwd_simt_kernel(BwdArgs a) {
 template <int DK>
 constexpr size_t bwd_smem_bytes() {
     return sizeof(float) * (2 * C * (DK + 1) + 2 * DK * 33 + 6 * C * 33 + 2 * C * (C + 1) + 9 * C + 8 +
-                            C * tcc::LDL + 1024 + C * 33);
+                            C * tcc::LDL + 1024 + C * 33 + C);
 }
 
 // dq to the output type; dk and deta from the unit-key gradients:
 //   b = eta r^2/(r^2+eps), c = eta r/(r^2+eps), khat = k/r
 //   deta = db r^2/den + dc r/den,  dr = db eta 2 r eps/den^2 + dc eta (eps - r^2)/den^2
 //   dk   = (dkhat - khat (khat . dkhat)) / r + khat dr
+// At a key of zero norm the accumulated dkhat already is dk (U's row there was beta v).
 template <int DK, typename Tin, typename TOut>
 __global__ void __launch_bounds__(256) bwd_finalize_kernel(BwdArgs a, size_t ntok) {
     const size_t w = (size_t)blockIdx.x * 8 + (threadIdx.x >> 5);
@@ -709,7 +717,7 @@ __global__ void __launch_bounds__(256) bwd_finalize_kernel(BwdArgs a, size_t nto
 #pragma unroll
     for (int u = 0; u < PER; ++u) {
         const float kh = kv[u] * inv_r;
-        const float val = live ? (dkh[u] - kh * kd) * inv_r + kh * dr : 0.f;
+        const float val = live ? (dkh[u] - kh * kd) * inv_r + kh * dr : dkh[u];
         dk[w * DK + lane + 32 * u] = from_f32<TOut>(val);
     }
     if (lane == 0) a.deta[w] = deta;

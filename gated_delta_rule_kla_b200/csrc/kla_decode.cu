@@ -50,6 +50,7 @@ constexpr int STAGES = KLA_DECODE_STAGES;
 constexpr int CTAS_PER_SM = KLA_DECODE_CTAS;
 static_assert(CG <= 32 && 32 % CG == 0, "column groups tile a warp");
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
+constexpr uint64_t kInjectedWaitNs = 20000000ull;  // 20 ms: the injected wait (below)
 
 constexpr int NW = NT / 32;       // warps
 
@@ -67,19 +68,24 @@ constexpr int MAX_UNITS_PER_CTA = 64;
 template <int DK, typename Tin>
 struct DecodeSmem {
     float s[STAGES][DK][NV];                    // state tiles
+    float gv[STAGES][DK];                       // diagonal gating: the head's per-channel log-decay
     Tin kv[STAGES][DK], qv[STAGES][DK], vv[STAGES][NV];
     float4 red_k[2][NW][CG], red_q[2][NW][CG];  // per-warp partial S^T k, S^T q (by unit parity)
     float scal[2][2][NW];                       // per-warp partial ||k||^2, k.q (by unit parity)
     float alpha[MAX_UNITS_PER_CTA], eta[MAX_UNITS_PER_CTA];
     uint64_t full[STAGES], done[STAGES];        // tile landed; every warp wrote its updated rows
+    uint64_t never;                             // failure injection: a barrier nothing completes
 };
 
-template <int DK, int DV, typename Tin, typename TOut>
+// DIAG: diagonal gating ("Kaczmarz Linear Attention", App. A.5): g is [B, H, Dk] and row i of
+// the state decays by alpha_i = exp(g_i), so alpha_i folds into k_i and q_i in the reductions
+// (S-bar^T k = S^T (alpha o k)) and into the update of row i.
+template <int DK, int DV, typename Tin, typename TOut, bool DIAG>
 __global__ void __launch_bounds__(NT, CTAS_PER_SM)
     decode_step_kernel(const __grid_constant__ CUtensorMap tm_s, const Tin* __restrict__ q,
                        const Tin* __restrict__ k, const Tin* __restrict__ v, const float* __restrict__ eta,
                        const float* __restrict__ g, float eps, float* __restrict__ S, TOut* __restrict__ o,
-                       int units) {
+                       int units, int inject_timeout) {
     constexpr int RPT = DK / RG;   // rows per thread
     constexpr int UPH = DV / NV;   // units per head
     constexpr uint32_t kTileBytes = DK * NV * 4;
@@ -99,6 +105,7 @@ __global__ void __launch_bounds__(NT, CTAS_PER_SM)
             mbar_init(smem_u32(&sm.full[s]), 1);
             mbar_init(smem_u32(&sm.done[s]), NW);
         }
+        mbar_init(smem_u32(&sm.never), 1);
         fence_mbar_init();
         prefetch_tmap(&tm_s);
     }
@@ -114,8 +121,9 @@ __global__ void __launch_bounds__(NT, CTAS_PER_SM)
         const int head = u / UPH, v0 = (u % UPH) * NV;
         const int st = i % STAGES;
         const uint32_t bar = smem_u32(&sm.full[st]);
-        mbar_expect_tx(bar, kTileBytes + 2 * kVecBytes + kVBytes);
+        mbar_expect_tx(bar, kTileBytes + 2 * kVecBytes + kVBytes + (DIAG ? DK * 4 : 0));
         tma_load_2d(smem_u32(&sm.s[st][0][0]), &tm_s, bar, v0, head * DK);
+        if (DIAG) bulk_load(smem_u32(&sm.gv[st][0]), g + (size_t)head * DK, DK * 4, bar);
         bulk_load(smem_u32(&sm.kv[st][0]), k + (size_t)head * DK, kVecBytes, bar);
         bulk_load(smem_u32(&sm.qv[st][0]), q + (size_t)head * DK, kVecBytes, bar);
         bulk_load(smem_u32(&sm.vv[st][0]), v + (size_t)head * DV + v0, kVBytes, bar);
@@ -126,7 +134,7 @@ __global__ void __launch_bounds__(NT, CTAS_PER_SM)
     // the decay and gate of every unit this CTA will process, loaded once
     if (tid < nmine) {
         const int head = (blockIdx.x + tid * stride) / UPH;
-        sm.alpha[tid] = expf(g[head]);
+        sm.alpha[tid] = DIAG ? 1.f : expf(g[head]);
         sm.eta[tid] = eta[head];
     }
     __syncthreads();
@@ -143,7 +151,11 @@ __global__ void __launch_bounds__(NT, CTAS_PER_SM)
             bulk_wait_read();
             request(i + STAGES - 1);
         }
-        const bool ok = mbar_wait_bounded(smem_u32(&sm.full[st]), (i / STAGES) & 1, kWaitLimitNs) && !store_failed;
+        bool ok = mbar_wait_bounded(smem_u32(&sm.full[st]), (i / STAGES) & 1, kWaitLimitNs) && !store_failed;
+        // failure injection (kla_debug_inject_wait_timeout): the first unit also waits on a
+        // barrier that no thread and no copy completes, so that bounded wait expires and the
+        // error path below runs exactly as for a lost copy
+        if (inject_timeout && i == 0) ok = mbar_wait_bounded(smem_u32(&sm.never), 0, kInjectedWaitNs) && ok;
         if (__syncthreads_or(!ok)) {
             if (tid == 0) {
                 atomicOr(&g_decode_error, 1u);
@@ -162,15 +174,16 @@ __global__ void __launch_bounds__(NT, CTAS_PER_SM)
             kq = kx * qx;
         }
         float4 cur[RPT];
-        float kir[RPT];
+        float kir[RPT], air[RPT];
         float4 pk = make_float4(0.f, 0.f, 0.f, 0.f), pq = pk;
 #pragma unroll
         for (int r = 0; r < RPT; ++r) {
             const int row = rg + r * RG;
             cur[r] = *reinterpret_cast<const float4*>(&sm.s[st][row][4 * cg]);
-            const float ki = to_f32(sm.kv[st][row]);
-            kir[r] = ki;
-            const float qi = to_f32(sm.qv[st][row]);
+            air[r] = DIAG ? expf(sm.gv[st][row]) : 1.f;
+            kir[r] = to_f32(sm.kv[st][row]);
+            const float ki = DIAG ? air[r] * kir[r] : kir[r];
+            const float qi = DIAG ? air[r] * to_f32(sm.qv[st][row]) : to_f32(sm.qv[st][row]);
             pk.x = fmaf(cur[r].x, ki, pk.x); pk.y = fmaf(cur[r].y, ki, pk.y);
             pk.z = fmaf(cur[r].z, ki, pk.z); pk.w = fmaf(cur[r].w, ki, pk.w);
             pq.x = fmaf(cur[r].x, qi, pq.x); pq.y = fmaf(cur[r].y, qi, pq.y);
@@ -228,11 +241,12 @@ __global__ void __launch_bounds__(NT, CTAS_PER_SM)
         for (int r = 0; r < RPT; ++r) {
             const int row = rg + r * RG;
             const float ki = kir[r];
+            const float ar = DIAG ? air[r] : alpha;
             float4 x = cur[r];
-            x.x = fmaf(alpha, x.x, ki * be.x);
-            x.y = fmaf(alpha, x.y, ki * be.y);
-            x.z = fmaf(alpha, x.z, ki * be.z);
-            x.w = fmaf(alpha, x.w, ki * be.w);
+            x.x = fmaf(ar, x.x, ki * be.x);
+            x.y = fmaf(ar, x.y, ki * be.y);
+            x.z = fmaf(ar, x.z, ki * be.z);
+            x.w = fmaf(ar, x.w, ki * be.w);
             *reinterpret_cast<float4*>(&sm.s[st][row][4 * cg]) = x;
         }
         fence_proxy_async();
@@ -280,7 +294,7 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-template <int DK, int DV, typename Tin, typename TOut>
+template <int DK, int DV, typename Tin, typename TOut, bool DIAG>
 cudaError_t launch_decode_t(const DecodeArgs& a, cudaStream_t st) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return cudaErrorNotSupported;
@@ -298,7 +312,7 @@ cudaError_t launch_decode_t(const DecodeArgs& a, cudaStream_t st) {
     int grid = units < CTAS_PER_SM * sm_count() ? units : CTAS_PER_SM * sm_count();
     if ((units + grid - 1) / grid > MAX_UNITS_PER_CTA) grid = (units + MAX_UNITS_PER_CTA - 1) / MAX_UNITS_PER_CTA;
     const size_t smem = sizeof(DecodeSmem<DK, Tin>) + 128;
-    cudaError_t e = cudaFuncSetAttribute(decode_step_kernel<DK, DV, Tin, TOut>,
+    cudaError_t e = cudaFuncSetAttribute(decode_step_kernel<DK, DV, Tin, TOut, DIAG>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
@@ -311,15 +325,18 @@ cudaError_t launch_decode_t(const DecodeArgs& a, cudaStream_t st) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, decode_step_kernel<DK, DV, Tin, TOut>, ms, static_cast<const Tin*>(a.q),
+    return cudaLaunchKernelEx(&cfg, decode_step_kernel<DK, DV, Tin, TOut, DIAG>, ms, static_cast<const Tin*>(a.q),
                               static_cast<const Tin*>(a.k), static_cast<const Tin*>(a.v), a.eta, a.g, a.eps, a.S,
-                              static_cast<TOut*>(a.o), units);
+                              static_cast<TOut*>(a.o), units, a.inject_timeout ? 1 : 0);
 }
 
 template <int DK, int DV, typename Tin>
 cudaError_t launch_decode_o(const DecodeArgs& a, cudaStream_t st) {
-    return a.out_bf16 ? launch_decode_t<DK, DV, Tin, __nv_bfloat16>(a, st)
-                      : launch_decode_t<DK, DV, Tin, float>(a, st);
+    if (a.diag)
+        return a.out_bf16 ? launch_decode_t<DK, DV, Tin, __nv_bfloat16, true>(a, st)
+                          : launch_decode_t<DK, DV, Tin, float, true>(a, st);
+    return a.out_bf16 ? launch_decode_t<DK, DV, Tin, __nv_bfloat16, false>(a, st)
+                      : launch_decode_t<DK, DV, Tin, float, false>(a, st);
 }
 
 template <typename Tin>

@@ -17,6 +17,8 @@ struct DecodeArgs {
     int B, H, Dk, Dv;
     bool bf16;      // q, k, v are bf16 (else fp32)
     bool out_bf16;  // o is bf16 (else fp32)
+    bool inject_timeout;  // failure injection: every CTA's first wait expires (nothing is stored)
+    bool diag = false;    // g is [B, H, Dk]: one log-decay per key channel (diagonal gating)
 };
 
 struct FwdArgs {
@@ -89,6 +91,13 @@ cudaError_t launch_chunk_bwd_tc_reverse(const BwdTcArgs& a, void* ws, size_t ws_
 cudaError_t bwd_tc_take_error(cudaStream_t st, unsigned int* flag);
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st);
+// Diagonal (per-key-channel) gating on CUDA cores: g is [B, T, H, Dk].  The kernels work in
+// chunks of diag_chunk_len() tokens; S_chunks of the forward (optional) and of the backward
+// (required: the workspace region the backward launcher fills first) are per such chunk.  The
+// backward's acc_dG is [B, T, H, Dk]; every accumulator must be zeroed before the launch.
+int diag_chunk_len();
+cudaError_t launch_chunk_fwd_diag(const FwdArgs& a, cudaStream_t st);
+cudaError_t launch_chunk_bwd_diag(const BwdArgs& a, const float* S0, cudaStream_t st);
 cudaError_t launch_chunk_fwd_simt(const FwdArgs& a, cudaStream_t st);
 cudaError_t launch_chunk_bwd_simt(const BwdArgs& a, cudaStream_t st);
 // Tensor-core (tcgen05) forward for bf16 inputs with Dk == Dv == 128.

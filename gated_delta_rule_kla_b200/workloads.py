@@ -20,6 +20,8 @@ workload dtype (round-to-nearest-even for bf16); eta, g, S0, dO stay fp32.
   eta         = sigmoid(N(0, 1))
   g           ~ U(-0.5, 0)            (gate_mode "uniform")
               = -softplus(N(0,1))*0.1 (gate_mode "softplus")
+              ~ U(gate_lo, 0) per key channel, shape [..., Dk]
+                                      (gate_mode "diag": diagonal gating, App. A.5)
   S0          = 0 or 0.02 * N(0, 1)
   dO          ~ N(0, 1)               (training workload only)
 """
@@ -45,6 +47,7 @@ class Workload:
     seed: int
     eps: float = 1e-6
     chunk: int = 64
+    gate_lo: float = -0.5  # lower end of the per-channel log-decays (gate_mode "diag")
 
     def with_(self, **kw) -> "Workload":
         return replace(self, **kw)
@@ -69,13 +72,21 @@ WORKLOADS = {
     "train_b4_t4096_h16_d128": Workload("train_b4_t4096_h16_d128", "train", B=4, T=4096, H=16,
                                         Dk=128, Dv=128, dtype="bf16", key_mode="scaled",
                                         gate_mode="uniform", s0="zero", seed=4),
+    # diagonal (per-key-channel) gating on the prefill and decode shapes above
+    "prefill_diag_b8_t2048_h8_d128": Workload("prefill_diag_b8_t2048_h8_d128", "fwd", B=8, T=2048, H=8,
+                                              Dk=128, Dv=128, dtype="bf16", key_mode="unit_scaled",
+                                              gate_mode="diag", s0="zero", seed=5),
+    "decode_diag_b64_h16_d128_x1024": Workload("decode_diag_b64_h16_d128_x1024", "decode", B=64, T=1024,
+                                               H=16, Dk=128, Dv=128, dtype="bf16", key_mode="scaled",
+                                               gate_mode="diag", s0="normal", seed=6),
 }
 
 
 def make_inputs(w: Workload, device=None):
     """Draw the inputs of workload `w`.
 
-    Sequence workloads return q, k [B,T,H,Dk], v [B,T,H,Dv], eta, g [B,T,H],
+    Sequence workloads return q, k [B,T,H,Dk], v [B,T,H,Dv], eta, g [B,T,H] (diagonal gating:
+    g [B,T,H,Dk]),
     S0 [B,H,Dk,Dv] (None when zero) and, for training, dO [B,T,H,Dv].
     Decode returns the same tensors with the step axis first: q, k [T,B,H,Dk],
     v [T,B,H,Dv], eta, g [T,B,H].
@@ -102,6 +113,8 @@ def make_inputs(w: Workload, device=None):
         g = torch.empty(*tok, dtype=f64).uniform_(-0.5, 0.0, generator=gen)
     elif w.gate_mode == "softplus":
         g = -torch.nn.functional.softplus(torch.randn(*tok, generator=gen, dtype=f64)) * 0.1
+    elif w.gate_mode == "diag":
+        g = torch.empty(*tok, w.Dk, dtype=f64).uniform_(w.gate_lo, 0.0, generator=gen)
     else:
         raise ValueError(w.gate_mode)
     if w.s0 == "normal":

@@ -149,8 +149,9 @@ kla_status kla_chunk_fwd_state(const void *q, const float *g, const float *S0, v
  * input: dq, dk, dv (of `out_dtype`), deta, dg ([B,T,H] fp32) and dS0 ([B,H,Dk,Dv] fp32;
  * written even when S0 is NULL).  S_chunks may be the array kla_chunk_fwd wrote for the
  * same inputs, or NULL to recompute it inside the workspace.
- * Gradient of k at a key of exactly zero norm: the normalised-key form used on the GPU has
- * no finite limit there; dk is returned as zero for such tokens (all other gradients exact).
+ * At a key of exactly zero norm the write vanishes but dk does not: it is returned exactly,
+ * dk_t = beta_t Gbar_t v_t with beta_t = eta_t / eps (eta_t in the direct mode; 0 when
+ * eps == 0) and Gbar_t the gradient of the state after token t.
  * ws, ws_bytes: caller workspace (device, 16-byte aligned, owned by the caller, contents need
  * not be initialised) of at least kla_chunk_bwd_workspace_min() bytes (required; smaller is
  * KLA_ERR_WORKSPACE).  With at least kla_chunk_bwd_workspace() bytes, bf16 inputs with
@@ -215,12 +216,62 @@ kla_status kla_decode_step(const void *q, const void *k, const void *v, const fl
                            int Dv, int dtype, int out_dtype, void *stream);
 
 /*
+ * Diagonal (per-key-channel) gating -- "Kaczmarz Linear Attention", Appendix A.5 (the Kaczmarz
+ * step does not depend on how the decayed state was produced) and Appendix B.5 (the chunk form
+ * under a diagonal decay).  The decay of token t is Diag(alpha_t), alpha_t = exp(g_t) with one
+ * log-decay per key channel:
+ *     Sbar = Diag(alpha_t) S_{t-1};  e_t = v_t - Sbar^T k_t;  S_t = Sbar + beta_t k_t e_t^T;
+ *     o_t = S_t^T q_t,  beta_t as for kla_chunk_fwd (Kaczmarz step, or KLA_BETA_DIRECT).
+ * Arguments, conventions and error behaviour are those of the scalar-gated entry points above,
+ * except that g (and dg) are [B, T, H, Dk] fp32 (decode: [B, H, Dk]).  The chunk entry points
+ * run on CUDA cores in fp32 (16-token internal chunks, so every decay factor exp(G_i - G_j) is
+ * formed directly, channel by channel, and stays <= 1 for g <= 0); the decode step is the
+ * TMA-pipelined kernel of kla_decode_step with the per-channel decay folded in.
+ *
+ * kla_chunk_fwd_diag   -- prefill: o ([B,T,H,Dv] of out_dtype, or NULL) and S_T ([B,H,Dk,Dv]
+ *                         fp32, or NULL; may alias S0) from S0 (NULL = zero state).  No workspace.
+ * kla_chunk_bwd_diag   -- gradients of <o, dO> + <S_T, dS_T> with respect to q, k, v, eta, g
+ *                         (dg per channel, [B,T,H,Dk]) and S0; dS_T may be NULL.  ws: device,
+ *                         16-byte aligned, caller-owned, at least kla_chunk_bwd_diag_workspace()
+ *                         bytes (the state at every internal chunk start plus fp32
+ *                         accumulators, cleared by the call), else KLA_ERR_WORKSPACE.  At a key
+ *                         of zero norm dk is exact, as for kla_chunk_bwd.
+ * kla_decode_step_diag -- one token for every (b, h); S [B,H,Dk,Dv] updated in place.
+ * Returns KLA_OK or an error status; on error nothing is launched.
+ */
+kla_status kla_chunk_fwd_diag(const void *q, const void *k, const void *v, const float *eta,
+                              const float *g, float eps, const float *S0, void *o, float *S_T,
+                              int B, int T, int H, int Dk, int Dv, int chunk, int dtype,
+                              int out_dtype, void *stream);
+size_t kla_chunk_bwd_diag_workspace(int B, int T, int H, int Dk, int Dv, int chunk, int dtype);
+kla_status kla_chunk_bwd_diag(const void *q, const void *k, const void *v, const float *eta,
+                              const float *g, float eps, const float *S0, const void *dO,
+                              const float *dS_T, void *dq, void *dk, void *dv, float *deta,
+                              float *dg, float *dS0, int B, int T, int H, int Dk, int Dv,
+                              int chunk, int dtype, int out_dtype, void *ws, size_t ws_bytes,
+                              void *stream);
+kla_status kla_decode_step_diag(const void *q, const void *k, const void *v, const float *eta,
+                                const float *g, float eps, float *S, void *o, int B, int H,
+                                int Dk, int Dv, int dtype, int out_dtype, void *stream);
+
+/*
  * kla_check_device_error -- synchronises `stream`, then reads and clears the library's
  * device error word.  Returns KLA_ERR_TIMEOUT if a kernel gave up on a bounded internal
  * wait since the last check (its outputs are then invalid), KLA_ERR_CUDA if the stream
  * reports an error, KLA_OK otherwise.  Not part of the paper: a failure-detection hook.
  */
 kla_status kla_check_device_error(void *stream);
+
+/*
+ * kla_debug_inject_wait_timeout -- failure injection for tests of the path above.  The next
+ * kla_decode_step call (on any thread) launches its kernel so that every CTA's first bounded
+ * wait is on a barrier that nothing completes; after about 20 ms that wait expires, the kernel
+ * lets the loads it already issued land, stores nothing (S keeps its input values, o is not
+ * written) and records the expiry, which kla_check_device_error then reports as
+ * KLA_ERR_TIMEOUT.  No copy is cut short and nothing faults: the context stays usable and the
+ * following calls run normally.  One-shot; has no effect until called.  Not part of the paper.
+ */
+void kla_debug_inject_wait_timeout(void);
 
 /*
  * kla_chunk_bwd_noalloc -- kla_chunk_bwd for callers that cannot allocate device memory.
@@ -234,11 +285,17 @@ kla_status kla_check_device_error(void *stream);
  * it until the process exits).  It calls no cudaMalloc, cudaFree or allocating routine;
  * inputs and outputs are still the caller's, exactly as for kla_chunk_bwd, and the result is
  * the same.
- *   - Limit: calls whose kla_chunk_bwd_workspace() size exceeds KLA_NOALLOC_SCRATCH_BYTES are
- *     rejected with KLA_ERR_WORKSPACE before anything is launched (about 16K token-heads at
- *     Dk = Dv = 128 without S_chunks; passing S_chunks roughly doubles that).
+ *   - Limit: a call is accepted when kla_chunk_bwd_workspace_min() for its sizes is at most
+ *     KLA_NOALLOC_SCRATCH_BYTES (about 16K token-heads at Dk = Dv = 128 without S_chunks,
+ *     about 32K with it); larger calls are rejected with KLA_ERR_WORKSPACE before anything is
+ *     launched.  Which backward runs follows kla_chunk_bwd's rule for a workspace of
+ *     KLA_NOALLOC_SCRATCH_BYTES: bf16 inputs with Dk == Dv == 128 run on the tensor cores when
+ *     kla_chunk_bwd_workspace() also fits (about 6K token-heads), otherwise the CUDA-core
+ *     backward runs (same results within the tolerance, about ten times slower).
  *   - The first call on each device looks up the scratch array's device address (with that
- *     device current); make that first call before any stream capture begins.
+ *     device current) and caches it for the life of the process; make that first call before
+ *     any stream capture begins.  The cached address does not survive cudaDeviceReset: do not
+ *     call this entry point on a device after resetting it.
  *   - All calls on a device share the one array and the library clears what must start at
  *     zero on every call.  Calls that may overlap on the GPU (different streams, or host
  *     threads without ordering) race on the shared scratch: serialise them.

@@ -390,6 +390,40 @@ def test_backward_finite_differences(oracle_mod, T, ckpt, eps):
         assert err <= 1e-6, (name, err)
 
 
+@pytest.mark.parametrize("beta,eps", [("kaczmarz", 0.3), ("kaczmarz", 1e-2), ("direct", 0.0)])
+def test_backward_zero_norm_key_finite_differences(oracle_mod, beta, eps):
+    """At a key of exactly zero norm the write vanishes, but dk there is not zero:
+    dk_t = beta_t Gbar_t v_t (the only first-order term of beta k e^T).  Central differences
+    around k_t = 0 in every direction."""
+    rng = np.random.default_rng(420 + int(eps * 100))
+    B, T, H, Dk, Dv = 1, 6, 1, 3, 4
+    q, k, v, eta, g, S0 = _rand_inputs(rng, B, T, H, Dk, Dv, key_lo=0.5, key_hi=1.5, s0=0.5)
+    if beta == "direct":
+        eta = 0.3 * eta
+    zt = (1, 4)
+    for t in zt:
+        k[0, t, 0] = 0.0
+    dO = rng.standard_normal((B, T, H, Dv))
+    dST = rng.standard_normal((B, H, Dk, Dv))
+    grads = oracle_mod.backward(q, k, v, eta, g, eps, S0, dO, dST, beta=beta)
+
+    def loss(kk):
+        o, ST = oracle_mod.forward(q, kk, v, eta, g, eps, S0, beta=beta)
+        return float(np.sum(o * dO) + np.sum(ST * dST))
+
+    hstep = 1e-6
+    for t in zt:
+        fd = np.zeros(Dk)
+        for c in range(Dk):
+            kp, km = k.copy(), k.copy()
+            kp[0, t, 0, c] += hstep
+            km[0, t, 0, c] -= hstep
+            fd[c] = (loss(kp) - loss(km)) / (2 * hstep)
+        got = grads["dk"][0, t, 0]
+        assert np.abs(fd).max() > 1e-3  # the gradient there is genuinely nonzero
+        assert np.abs(got - fd).max() <= 1e-6 * np.abs(fd).max(), (t, got, fd)
+
+
 def test_backward_without_dST_and_zero_S0(oracle_mod):
     rng = np.random.default_rng(200)
     q, k, v, eta, g, _ = _rand_inputs(rng, 1, 6, 1, 3, 2)

@@ -23,7 +23,8 @@ def test_shapes_layout_and_dtypes(name):
     dt = torch.bfloat16 if ws.dtype == "bf16" else torch.float32
     assert d["q"].shape == tok + (ws.Dk,) and d["k"].shape == tok + (ws.Dk,) and d["v"].shape == tok + (ws.Dv,)
     assert d["q"].dtype == d["k"].dtype == d["v"].dtype == dt
-    assert d["eta"].shape == tok and d["g"].shape == tok
+    gshape = tok + (ws.Dk,) if ws.gate_mode == "diag" else tok
+    assert d["eta"].shape == tok and d["g"].shape == gshape
     assert d["eta"].dtype == d["g"].dtype == torch.float32
     if ws.s0 == "normal":
         assert d["S0"].shape == (ws.B, ws.H, ws.Dk, ws.Dv) and d["S0"].dtype == torch.float32
@@ -73,3 +74,15 @@ def test_gates_eta_and_initial_state():
     assert abs(float(gs.mean()) + 0.08066) < 0.003                   # -0.1 E[softplus(N(0,1))]
     S0 = make_inputs(small("decode_b64_h16_d128_x1024", T=4))["S0"].double()
     assert abs(float(S0.std()) - 0.02) < 0.001 and abs(float(S0.mean())) < 0.001
+
+
+def test_diagonal_gates_per_channel_uniform():
+    w = small("prefill_diag_b8_t2048_h8_d128", T=256, B=2)
+    g = make_inputs(w)["g"].double()
+    assert g.shape == (2, 256, w.H, w.Dk)
+    assert float(g.min()) >= w.gate_lo and float(g.max()) <= 0.0
+    assert abs(float(g.mean()) - w.gate_lo / 2) < 0.01
+    # channels are drawn independently: the decay differs across the key channels of a token
+    assert float(g.std(dim=-1).mean()) > 0.1
+    g4 = make_inputs(w.with_(gate_lo=-4.0))["g"].double()
+    assert float(g4.min()) >= -4.0 and abs(float(g4.mean()) + 2.0) < 0.05

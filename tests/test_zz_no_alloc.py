@@ -4,8 +4,9 @@ Callers such as CUDA-graph captures that must not allocate, plugins whose host f
 all device memory, or latency-critical paths cannot hand kla_chunk_bwd a workspace.  For them
 the library offers kla_chunk_bwd_noalloc, which uses a fixed scratch array compiled into
 libkla.so.  These tests call it through the C ABI and check that it returns what
-kla_chunk_bwd returns, on two calls in a row with different shapes and dtypes, so leftovers
-of the first call in the shared scratch would show up in the second.  The file name makes
+kla_chunk_bwd returns, on several calls in a row with different shapes, dtypes and backward
+paths (the tensor-core path twice on the same shape), so leftovers of an earlier call in the
+shared scratch would show up in a later one.  The file name makes
 pytest collect it last.
 """
 import ctypes
@@ -48,6 +49,18 @@ def test_noalloc_rejects_problems_larger_than_its_scratch():
     assert b"static scratch" in L.kla_last_error()
 
 
+def test_noalloc_limit_is_the_cuda_core_size():
+    """The call is accepted when the CUDA-core layout fits the scratch; the tensor-core layout
+    decides only which backward runs.  At bf16 B=1 T=8192 H=1 d=128 the two straddle the
+    scratch size (so that call runs the CUDA-core backward); at T=130 H=2 both fit."""
+    _, L = _lib()
+    cap = L.kla_chunk_bwd_noalloc_scratch_bytes()
+    assert L.kla_chunk_bwd_workspace_min(1, 8192, 1, 128, 128, 64, KLA_BF16, 0) <= cap
+    assert L.kla_chunk_bwd_workspace(1, 8192, 1, 128, 128, 64, KLA_BF16, 0) > cap
+    assert L.kla_chunk_bwd_workspace(1, 130, 2, 128, 128, 64, KLA_BF16, 0) <= cap
+    assert L.kla_chunk_bwd_workspace_min(1, 16384, 1, 128, 128, 64, KLA_BF16, 0) > cap
+
+
 def _rel_err(got, ref):
     got = got.detach().double().cpu()
     ref = ref.detach().double().cpu()
@@ -61,8 +74,15 @@ def test_noalloc_backward_matches_workspace_backward_on_two_calls():
         pytest.skip("no CUDA device")
     kla, L = _lib()
     dev = torch.device("cuda", 0)
-    cases = [(2, 200, 2, 128, "f32", 31), (1, 130, 3, 64, "bf16", 32)]
+    # In order: CUDA-core shapes (fp32, then bf16 d = 64); the tensor-core backward (bf16
+    # d = 128, both layouts fit) right after a different shape and then again, so stale bytes
+    # from an earlier call would show; a shape whose tensor-core layout does not fit (the
+    # CUDA-core backward on the scratch).
+    cases = [(2, 200, 2, 128, "f32", 31), (1, 130, 3, 64, "bf16", 32), (1, 130, 2, 128, "bf16", 33),
+             (1, 130, 2, 128, "bf16", 34), (1, 8192, 1, 128, "bf16", 35)]
     for B, T, H, D, dtype, seed in cases:
+        tensor_cores = dtype == "bf16" and D == 128 and \
+            L.kla_chunk_bwd_workspace(B, T, H, D, D, 64, KLA_BF16, 0) <= L.kla_chunk_bwd_noalloc_scratch_bytes()
         w = Workload("noalloc", "train", B=B, T=T, H=H, Dk=D, Dv=D, dtype=dtype, key_mode="scaled",
                      gate_mode="uniform", s0="normal", seed=seed)
         inp = make_inputs(w)
@@ -84,3 +104,5 @@ def test_noalloc_backward_matches_workspace_backward_on_two_calls():
         for name in ("dq", "dk", "dv", "deta", "dg", "dS0"):
             assert torch.isfinite(out[name]).all(), name
             assert _rel_err(out[name], ref[name]) <= TOL[dtype], name
+            if tensor_cores:  # the tensor-core backward is deterministic: same bits as with a workspace
+                assert torch.equal(out[name], ref[name]), name
