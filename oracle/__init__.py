@@ -13,6 +13,12 @@ may import this package.  The CUDA library shares no code with it.
 Parity status: forward pinned (Theorem 1, Propositions 1-2, Eq. (4), the
 recurrent form of Table 6, classical Kaczmarz, the chunk form, a hand-worked
 example, exact rational arithmetic); backward pinned by finite differences only.
+
+``oracle.gates`` (plain numpy, fp64) is the oracle of the gate prologue: the write gate
+eta_t = sigmoid(x_t . w_eta + b_eta) of section 3.3, the log-decay g_t = -softplus(x_t . w_g +
+b_g) (a reading: the pages print no projection for g) and the query normalisation of
+Algorithm 1's readout; pinned by closed forms, asymptotics, affinity of the logits, the
+normalised readout against this package's recurrence, and finite differences.
 """
 import ctypes
 import os
