@@ -278,6 +278,7 @@ def gpu_arm(args, rank, world, local_rank):
         tokens = sum_over_ranks(float(w.B * w.T), world) * args.steps
         elt = d["q"].element_size()
         alg_bytes = fwd_bytes(w.B, w.T, w.H, w.Dk, w.Dv, elt, d["S0"] is not None)
+        alg_bytes_bf16_o = fwd_bytes(w.B, w.T, w.H, w.Dk, w.Dv, elt, d["S0"] is not None, out_elt=2)
         alg_flops = fwd_flops_per_token_head(w.Dk) * w.B * w.T * w.H
         mean_s = statistics.mean(ms) / 1e3
         achieved_gbs = alg_bytes / mean_s / 1e9
@@ -297,6 +298,11 @@ def gpu_arm(args, rank, world, local_rank):
                                                hbm_peak, tc_peak, args)
         if "direct" in parts:
             extra["direct_beta"] = bench_direct(kla, w, d, ws, o, ST, flush, stream, world, hbm_peak, args)
+        if "diag" in parts:
+            extra["diagonal_gating"] = bench_diag(kla, WORKLOADS, make_inputs, dev, stream, flush, rank, world,
+                                                  hbm_peak, peaks, args)
+        if "gates" in parts:
+            extra["gate_prologue"] = bench_gates(kla, dev, stream, flush, rank, world, hbm_peak, args)
 
     # ---------------- end-to-end through the public API with host buffers ----------------
     e2e = None if args.skip_e2e else bench_e2e(kla, w, inp, dev, stream, rank, world, args)
@@ -325,6 +331,10 @@ def gpu_arm(args, rank, world, local_rank):
                                   " preparation)" if launches == 4 else "")),
                      "traffic": recorded_traffic("chunk_fwd_prefill_b8_t2048_h8_d128"),
                      "alg_bytes_per_launch": alg_bytes, "kernel_us": mean_s * 1e6, "stages": stages,
+                     # the same call counted with a bf16 o (1032 B per token-head): the output
+                     # store the scope table fixes, below the fp32 o this call writes
+                     "alg_bytes_bf16_o": alg_bytes_bf16_o,
+                     "frac_bf16_o": alg_bytes_bf16_o / mean_s / 1e9 / hbm_peak,
                      "tensor": {"achieved": achieved_tf, "peak": tc_peak, "unit": "TFLOP/s",
                                 "frac": achieved_tf / tc_peak, "alg_flops_per_launch": alg_flops}},
         "e2e": e2e,
@@ -356,9 +366,11 @@ def time_fwd_stages(kla, d, w, ws, o, ST, flush, stream, nsteps):
             "dominant": "chunk_prep_kernel" if prep >= state else "chunk_state_kernel"}
 
 
-def bench_decode(kla, WORKLOADS, make_inputs, dev, stream, flush, rank, world, hbm_peak, args):
+def bench_decode(kla, WORKLOADS, make_inputs, dev, stream, flush, rank, world, hbm_peak, args,
+                 wname="decode_b64_h16_d128_x1024", step_fn=None, traffic_key="decode_b64_h16_d128"):
     import torch
-    w = WORKLOADS["decode_b64_h16_d128_x1024"]
+    step_fn = step_fn or kla.decode_step
+    w = WORKLOADS[wname]
     w = w.with_(seed=w.seed + 1000 * rank)
     inp = make_inputs(w)
     q, k, v = inp["q"].to(dev), inp["k"].to(dev), inp["v"].to(dev)
@@ -374,7 +386,7 @@ def bench_decode(kla, WORKLOADS, make_inputs, dev, stream, flush, rank, world, h
     o = torch.empty(w.B, w.H, w.Dv, device=dev, dtype=torch.float32)
     steps = w.T if not args.quick else 64
     for t in range(8):
-        kla.decode_step(q[t], k[t], v[t], eta[t], g[t], S_sets[0], w.eps, o=o)
+        step_fn(q[t], k[t], v[t], eta[t], g[t], S_sets[0], w.eps, o=o)
     S_sets[0].copy_(inp["S0"].to(dev))
     torch.cuda.synchronize()
     barrier(world)
@@ -382,7 +394,7 @@ def bench_decode(kla, WORKLOADS, make_inputs, dev, stream, flush, rank, world, h
     def all_steps():
         for t in range(steps):
             tok = t // NSETS
-            kla.decode_step(q[tok], k[tok], v[tok], eta[tok], g[tok], S_sets[t % NSETS], w.eps, o=o)
+            step_fn(q[tok], k[tok], v[tok], eta[tok], g[tok], S_sets[t % NSETS], w.eps, o=o)
 
     # The steps are captured once in a CUDA graph and replayed, as a serving loop would run
     # them: one host launch per step costs about as much as the step itself, so timed eagerly
@@ -413,7 +425,7 @@ def bench_decode(kla, WORKLOADS, make_inputs, dev, stream, flush, rank, world, h
         for t in range(steps):
             tok = t // NSETS
             evs[t][0].record(stream)
-            kla.decode_step(q[tok], k[tok], v[tok], eta[tok], g[tok], S_sets[t % NSETS], w.eps, o=o)
+            step_fn(q[tok], k[tok], v[tok], eta[tok], g[tok], S_sets[t % NSETS], w.eps, o=o)
             evs[t][1].record(stream)
         torch.cuda.synchronize()
         ms = [a.elapsed_time(b) for a, b in evs]
@@ -422,13 +434,15 @@ def bench_decode(kla, WORKLOADS, make_inputs, dev, stream, flush, rank, world, h
     tokens = sum_over_ranks(float(w.B), world) * steps
     mean_s = statistics.mean(ms) / 1e3
     alg = decode_bytes(w.B, w.H, w.Dk, w.Dv, q.element_size())
+    if g.dim() == 4:  # diagonal gating: one log-decay per key channel
+        alg += w.B * w.H * (w.Dk - 1) * 4
     gbs = alg / mean_s / 1e9
     return {"workload": w.name, "value": tokens / (total_ms / 1e3), "unit": "tokens/s",
             "steps": steps, "us_per_step": total_ms * 1e3 / steps, "gpu_launches": steps, "timing": timing,
             "l2": "inputs larger than L2 (4 sequence groups' states cycled, 268 MB)",
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s",
                          "frac": gbs / hbm_peak, "alg_bytes_per_launch": alg,
-                         "traffic": recorded_traffic("decode_b64_h16_d128")}}
+                         "traffic": recorded_traffic(traffic_key)}}
 
 
 def bench_train(kla, WORKLOADS, make_inputs, dev, stream, flush, rank, world, hbm_peak, tc_peak, args):
@@ -492,6 +506,10 @@ def bench_long(kla, WORKLOADS, make_inputs, dev, stream, rank, world, hbm_peak, 
     barrier(world)
     nsteps = 2 if args.quick else 3
     ms = time_steps(run, nsteps, lambda: None, stream)  # inputs (403 MB) exceed L2
+    # the preparation and the segmented state pass (transition pass, segment scan, output pass)
+    # timed on their own
+    stages = time_fwd_stages(kla, d, w, ws, o, ST, lambda: None, stream, nsteps)
+    stages["chunk_state_kernel"]["includes"] = "transition pass + seg_scan_kernel + output pass"
     barrier(world)
     total_ms = max_over_ranks(sum(ms), world)
     tokens = sum_over_ranks(float(w.B * w.T), world) * nsteps
@@ -501,7 +519,7 @@ def bench_long(kla, WORKLOADS, make_inputs, dev, stream, rank, world, hbm_peak, 
     return {"workload": w.name, "value": tokens / (total_ms / 1e3), "unit": "tokens/s",
             "steps": nsteps, "ms_per_step": total_ms / nsteps, "l2": "inputs larger than L2",
             # preparation, transition pass, segment scan, output pass
-            "gpu_launches_per_step": 4,
+            "gpu_launches_per_step": 4, "stages": stages,
             "roofline": {"bound": "hbm", "achieved": alg / mean_s / 1e9, "peak": hbm_peak, "unit": "GB/s",
                          "frac": alg / mean_s / 1e9 / hbm_peak,
                          "tensor_frac": flops / mean_s / 1e12 / tc_peak}}
@@ -532,6 +550,117 @@ def bench_direct(kla, w, d, ws, o, ST, flush, stream, world, hbm_peak, args):
             "gpu_launches_per_step": kla.fwd_kernel_launches(d["k"], d["v"]),
             "roofline": {"bound": "hbm", "achieved": alg / mean_s / 1e9, "peak": hbm_peak, "unit": "GB/s",
                          "frac": alg / mean_s / 1e9 / hbm_peak}}
+
+
+def fp32_alu_peak_tflops(peaks):
+    """fp32 FMA peak of the CUDA cores: 148 SMs x 128 fp32 lanes x 2 FLOP per FMA at the
+    maximum SM clock (the unit counts and clock of the part; no measured figure exists)."""
+    return 148 * 128 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
+
+
+def bench_diag(kla, WORKLOADS, make_inputs, dev, stream, flush, rank, world, hbm_peak, peaks, args):
+    """Diagonal (per-key-channel) gating (App. A.5, B.5): the headline prefill shape through
+    kla_chunk_fwd_diag, its backward kla_chunk_bwd_diag, and the decode shape through
+    kla_decode_step_diag (same timing as the scalar decode leg)."""
+    import torch
+    w = WORKLOADS["prefill_diag_b8_t2048_h8_d128"]
+    w = w.with_(seed=w.seed + 1000 * rank)
+    inp = make_inputs(w)
+    d = {k: (v.to(dev) if v is not None else None) for k, v in inp.items()}
+    o = torch.empty(w.B, w.T, w.H, w.Dv, device=dev, dtype=torch.float32)
+    ST = torch.empty(w.B, w.H, w.Dk, w.Dv, device=dev, dtype=torch.float32)
+    dO = torch.randn(w.B, w.T, w.H, w.Dv, device=dev).to(d["q"].dtype)
+    L = kla.lib()
+    wsb = torch.empty(L.kla_chunk_bwd_diag_workspace(w.B, w.T, w.H, w.Dk, w.Dv, 64, 1), device=dev,
+                      dtype=torch.uint8)
+
+    def fwd():
+        kla.chunk_fwd_diag(d["q"], d["k"], d["v"], d["eta"], d["g"], w.eps, d["S0"], o=o, S_T=ST)
+
+    def bwd():
+        kla.chunk_bwd_diag(d["q"], d["k"], d["v"], d["eta"], d["g"], dO, w.eps, d["S0"], workspace=wsb)
+
+    for _ in range(3):
+        flush()
+        fwd()
+    bwd()
+    torch.cuda.synchronize()
+    barrier(world)
+    nf = 3 if args.quick else 10
+    ms_f = time_steps(fwd, nf, flush, stream)
+    ms_b = time_steps(bwd, 2 if args.quick else 3, flush, stream)
+    barrier(world)
+    tf_f = max_over_ranks(sum(ms_f), world) / nf
+    tf_b = max_over_ranks(sum(ms_b), world) / len(ms_b)
+    tokens = sum_over_ranks(float(w.B * w.T), world)
+    elt = d["q"].element_size()
+    # bytes as for scalar gating, plus the per-channel log-decays (Dk fp32 per token-head)
+    alg = fwd_bytes(w.B, w.T, w.H, w.Dk, w.Dv, elt, False) + w.B * w.T * w.H * (w.Dk - 1) * 4
+    flops = fwd_flops_per_token_head(w.Dk) * w.B * w.T * w.H
+    alu = fp32_alu_peak_tflops(peaks)
+    mean_f = statistics.mean(ms_f) / 1e3
+    out = {"workload": w.name, "value": tokens / (tf_f / 1e3), "unit": "tokens/s", "steps": nf,
+           "ms_per_step": tf_f, "l2": "flushed between timed steps", "gpu_launches_per_step": 1,
+           "roofline": {"bound": "alu", "achieved": flops / mean_f / 1e12, "peak": alu, "unit": "TFLOP/s",
+                        "frac": flops / mean_f / 1e12 / alu,
+                        "peak_kind": "derived: 148 SMs x 128 fp32 FMA lanes x 2 x max SM clock",
+                        "hbm_frac": alg / mean_f / 1e9 / hbm_peak, "alg_bytes_per_launch": alg,
+                        "alg_flops_per_launch": flops},
+           "backward": {"value": tokens / (tf_b / 1e3), "unit": "tokens/s", "ms_per_step": tf_b,
+                        "gpu_launches_per_step": 4,
+                        "what": "kla_chunk_bwd_diag: forward state recompute, reverse pass, finish, dg scan"}}
+    out["decode"] = bench_decode(kla, WORKLOADS, make_inputs, dev, stream, flush, rank, world, hbm_peak, args,
+                                 wname="decode_diag_b64_h16_d128_x1024", step_fn=kla.decode_step_diag,
+                                 traffic_key="decode_diag_b64_h16_d128")
+    return out
+
+
+def bench_gates(kla, dev, stream, flush, rank, world, hbm_peak, args):
+    """The gate prologue on the headline's tokens (N = B T = 16384, D = 1024 = 8 heads x 128,
+    H = 8, q normalised for Dk = 128): kla_gate_prologue and kla_gate_prologue_bwd."""
+    import torch
+    from gated_delta_rule_kla_b200.workloads import make_gate_inputs
+    N, D, H, Dk = 8 * 2048, 1024, 8, 128
+    gi = make_gate_inputs(N, D, H, Dk, "bf16", seed=31 + 1000 * rank, device=dev)
+    deta = torch.randn(N, H, device=dev)
+    dg = torch.randn(N, H, device=dev)
+    dqh = torch.randn(N, H, Dk, device=dev)
+    res = {}
+
+    def fwd():
+        res["f"] = kla.gate_prologue(gi["x"], gi["W"], gi["bias"], gi["q"])
+
+    fwd()
+
+    def bwd():
+        kla.gate_prologue_bwd(gi["x"], gi["W"], res["f"][0], res["f"][1], deta, dg, gi["q"], dqh)
+
+    for _ in range(3):
+        flush()
+        fwd()
+        bwd()
+    torch.cuda.synchronize()
+    barrier(world)
+    n = 5 if args.quick else 20
+    ms_f = time_steps(fwd, n, flush, stream)
+    ms_b = time_steps(bwd, n, flush, stream)
+    barrier(world)
+    tf = max_over_ranks(sum(ms_f), world) / n
+    tb = max_over_ranks(sum(ms_b), world) / n
+    # forward: x, W, q in; eta, g, qhat out.  backward: x, W, q, eta, g, deta, dg, dqhat in;
+    # dx, dq, dW, dbias out (fp32), plus the per-tile partial sums written and read once
+    fb = N * D * 2 + 2 * H * D * 2 + 2 * N * H * Dk * 2 + 2 * N * H * 4
+    bb = N * D * 2 + N * H * Dk * 2 + 4 * N * H * 4 + N * H * Dk * 4 + N * D * 4 + N * H * Dk * 4
+    tokens = sum_over_ranks(float(N), world)
+    return {"shape": {"N": N, "D": D, "H": H, "Dk": Dk, "dtype": "bf16"},
+            "value": tokens / (tf / 1e3), "unit": "tokens/s", "us_per_call": tf * 1e3,
+            "gpu_launches_per_step": 1, "l2": "flushed between timed steps",
+            "roofline": {"bound": "hbm", "achieved": fb / (tf / 1e3) / 1e9, "peak": hbm_peak, "unit": "GB/s",
+                         "frac": fb / (tf / 1e3) / 1e9 / hbm_peak, "alg_bytes_per_launch": fb},
+            "backward": {"us_per_call": tb * 1e3, "gpu_launches_per_step": 2,
+                         "roofline": {"bound": "hbm", "achieved": bb / (tb / 1e3) / 1e9, "peak": hbm_peak,
+                                      "unit": "GB/s", "frac": bb / (tb / 1e3) / 1e9 / hbm_peak,
+                                      "alg_bytes_per_launch": bb}}}
 
 
 def bench_e2e(kla, w, inp, dev, stream, rank, world, args):
@@ -670,11 +799,13 @@ def parse(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["kla", "reference"], default="kla")
     ap.add_argument("--workload", default="prefill_b8_t2048_h8_d128")
-    ap.add_argument("--ref-pairs", type=int, default=8, help="(b,h) pairs per reference step")
+    ap.add_argument("--ref-pairs", type=int, default=16,
+                    help="(b,h) pairs per reference step (at least the host's cores, so none idles)")
     ap.add_argument("--cpu-pairs", type=int, default=64, help="(b,h) pairs in the CPU baseline sample")
     ap.add_argument("--skip-extra", action="store_true", help="headline prefill only")
-    ap.add_argument("--parts", default="decode,train,long,direct",
-                    help="sub-measurements after the headline prefill (comma list of decode,train,long,direct)")
+    ap.add_argument("--parts", default="decode,train,long,direct,diag,gates",
+                    help="sub-measurements after the headline prefill (comma list of "
+                         "decode,train,long,direct,diag,gates)")
     ap.add_argument("--skip-e2e", action="store_true", help="omit the host-buffer end-to-end leg")
     ap.add_argument("--skip-cpu", action="store_true", help="omit the CPU baseline")
     ap.add_argument("--quick", action="store_true", help="fewer decode/train steps (smoke runs)")

@@ -21,7 +21,7 @@ import torch
 __all__ = ["lib", "chunk_fwd", "chunk_fwd_prep", "chunk_fwd_state", "fwd_workspace", "fwd_kernel_launches",
            "chunk_bwd", "chunk_fwd_train", "chunk_bwd_after_train", "train_workspace",
            "decode_step", "check_device_error", "debug_inject_wait_timeout",
-           "chunk_fwd_diag", "chunk_bwd_diag", "decode_step_diag", "KLAError", "CHUNK", "KLA_BETA_DIRECT",
+           "chunk_fwd_diag", "chunk_bwd_diag", "decode_step_diag", "gate_prologue", "gate_prologue_bwd", "KLAError", "CHUNK", "KLA_BETA_DIRECT",
            "library_path"]
 
 CHUNK = 64
@@ -92,6 +92,13 @@ def lib():
         L.kla_chunk_bwd_diag.restype = i
         L.kla_decode_step_diag.argtypes = [vp, vp, vp, fp, fp, f, fp, vp, i, i, i, i, i, i, vp]
         L.kla_decode_step_diag.restype = i
+        L.kla_gate_prologue.argtypes = [vp, vp, fp, vp, fp, fp, vp, i, i, i, i, i, vp]
+        L.kla_gate_prologue.restype = i
+        L.kla_gate_prologue_bwd_workspace.argtypes = [i, i, i]
+        L.kla_gate_prologue_bwd_workspace.restype = sz
+        L.kla_gate_prologue_bwd.argtypes = [vp, vp, fp, fp, vp, fp, fp, fp, fp, fp, fp, fp, i, i, i, i, i, vp, sz,
+                                            vp]
+        L.kla_gate_prologue_bwd.restype = i
         _lib = L
     return _lib
 
@@ -424,6 +431,61 @@ def decode_step_diag(q, k, v, eta, g, S, eps=1e-6, *, o=None, out_dtype=torch.fl
                                     B, H, Dk, Dv, _in_code(k, beta), _dtype_code(o), _stream(dev, stream))
     _check(st, "kla_decode_step_diag")
     return o
+
+
+def gate_prologue(x, W, bias, q=None, *, stream=None):
+    """Gates of every head from the token vectors (section 3.3): x [..., D], W [2H, D] (same
+    dtype, bf16 or fp32), bias [2H] fp32 -> eta = sigmoid(x W_eta^T + b_eta), g = -softplus(x W_g^T
+    + b_g), both [..., H] fp32; with q [..., H, Dk] also qhat = q / ||q|| (Algorithm 1's readout).
+    Returns (eta, g) or (eta, g, qhat)."""
+    dev = x.device
+    D = x.shape[-1]
+    lead = tuple(x.shape[:-1])
+    N = int(torch.tensor(lead).prod().item()) if lead else 1
+    H = W.shape[0] // 2
+    dt = x.dtype
+    _need(x, "x", dev, dt); _need(W, "W", dev, dt, (2 * H, D)); _need(bias, "bias", dev, torch.float32, (2 * H,))
+    Dk = 0
+    qhat = None
+    if q is not None:
+        Dk = q.shape[-1]
+        _need(q, "q", dev, dt, lead + (H, Dk))
+        qhat = torch.empty_like(q)
+    eta = torch.empty(lead + (H,), device=dev, dtype=torch.float32)
+    g = torch.empty(lead + (H,), device=dev, dtype=torch.float32)
+    st = lib().kla_gate_prologue(_ptr(x), _ptr(W), _ptr(bias), _ptr(q), _ptr(eta), _ptr(g), _ptr(qhat), N, D, H,
+                                 Dk, _dtype_code(x), _stream(dev, stream))
+    _check(st, "kla_gate_prologue")
+    return (eta, g) if q is None else (eta, g, qhat)
+
+
+def gate_prologue_bwd(x, W, eta, g, deta, dg, q=None, dqhat=None, *, stream=None):
+    """Backward of gate_prologue from its outputs (eta, g) and the upstream gradients.
+    Returns dict(dx, dW, dbias) (+ dq when q is given), all fp32."""
+    dev = x.device
+    D = x.shape[-1]
+    lead = tuple(x.shape[:-1])
+    N = int(torch.tensor(lead).prod().item()) if lead else 1
+    H = W.shape[0] // 2
+    dt = x.dtype
+    _need(x, "x", dev, dt); _need(W, "W", dev, dt, (2 * H, D))
+    for t, n in ((eta, "eta"), (g, "g"), (deta, "deta"), (dg, "dg")):
+        _need(t, n, dev, torch.float32, lead + (H,))
+    Dk = 0
+    out = dict(dx=torch.empty(lead + (D,), device=dev, dtype=torch.float32),
+               dW=torch.empty(2 * H, D, device=dev, dtype=torch.float32),
+               dbias=torch.empty(2 * H, device=dev, dtype=torch.float32))
+    if q is not None:
+        Dk = q.shape[-1]
+        _need(q, "q", dev, dt, lead + (H, Dk)); _need(dqhat, "dqhat", dev, torch.float32, lead + (H, Dk))
+        out["dq"] = torch.empty(lead + (H, Dk), device=dev, dtype=torch.float32)
+    L = lib()
+    ws = torch.empty(max(L.kla_gate_prologue_bwd_workspace(N, D, H), 16), device=dev, dtype=torch.uint8)
+    st = L.kla_gate_prologue_bwd(_ptr(x), _ptr(W), _ptr(eta), _ptr(g), _ptr(q), _ptr(deta), _ptr(dg), _ptr(dqhat),
+                                 _ptr(out["dx"]), _ptr(out["dW"]), _ptr(out["dbias"]), _ptr(out.get("dq")), N, D,
+                                 H, Dk, _dtype_code(x), _ptr(ws), ws.numel(), _stream(dev, stream))
+    _check(st, "kla_gate_prologue_bwd")
+    return out
 
 
 def debug_inject_wait_timeout():

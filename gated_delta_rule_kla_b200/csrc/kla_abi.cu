@@ -514,16 +514,76 @@ kla_status kla_chunk_bwd_diag(const void* q, const void* k, const void* v, const
     return KLA_OK;
 }
 
+static kla_status gate_checks(int N, int D, int H, int Dk, int dtype, bool with_q) {
+    if (N < 0 || D < 1 || H < 1)
+        return fail(KLA_ERR_INVALID_ARG, "sizes must satisfy N>=0, D>=1, H>=1 (got N=%d D=%d H=%d)", N, D, H);
+    if (H > 64) return fail(KLA_ERR_UNSUPPORTED, "at most 64 heads (got H=%d)", H);
+    if (dtype != KLA_F32 && dtype != KLA_BF16)
+        return fail(KLA_ERR_UNSUPPORTED, "dtype must be KLA_F32 or KLA_BF16 (got %d)", dtype);
+    if (dtype == KLA_BF16 && D % 8 != 0)
+        return fail(KLA_ERR_UNSUPPORTED, "bf16 rows must be 16-byte multiples: D %% 8 == 0 (got D=%d)", D);
+    if (dtype == KLA_F32 && D % 4 != 0)
+        return fail(KLA_ERR_UNSUPPORTED, "fp32 rows must be 16-byte multiples: D %% 4 == 0 (got D=%d)", D);
+    if (with_q && Dk != 64 && Dk != 128) return fail(KLA_ERR_UNSUPPORTED, "Dk must be 64 or 128 (got %d)", Dk);
+    return KLA_OK;
+}
+
+kla_status kla_gate_prologue(const void* x, const void* W, const float* bias, const void* q, float* eta, float* g,
+                             void* q_hat, int N, int D, int H, int Dk, int dtype, void* stream) {
+    if ((q == nullptr) != (q_hat == nullptr))
+        return fail(KLA_ERR_INVALID_ARG, "q and q_hat must be given together (or both NULL)");
+    kla_status st = gate_checks(N, D, H, Dk, dtype, q != nullptr);
+    if (st != KLA_OK) return st;
+    if (N == 0) return KLA_OK;
+    REQUIRE_PTR(x); REQUIRE_PTR(W); REQUIRE_PTR(bias); REQUIRE_PTR(eta); REQUIRE_PTR(g);
+    OPTIONAL_PTR(q); OPTIONAL_PTR(q_hat);
+    kla::GateArgs a{x, W, bias, q, eta, g, q_hat, N, D, H, Dk, dtype == KLA_BF16};
+    cudaError_t e = kla::launch_gate_prologue(a, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "kla_gate_prologue launch");
+    return KLA_OK;
+}
+
+size_t kla_gate_prologue_bwd_workspace(int N, int D, int H) {
+    if (N < 0 || D < 1 || H < 1) return 0;
+    return kla::gate_bwd_workspace(N, D, H);
+}
+
+kla_status kla_gate_prologue_bwd(const void* x, const void* W, const float* eta, const float* g, const void* q,
+                                 const float* deta, const float* dg, const float* dq_hat, float* dx, float* dW,
+                                 float* dbias, float* dq, int N, int D, int H, int Dk, int dtype, void* ws,
+                                 size_t ws_bytes, void* stream) {
+    if ((q == nullptr) != (dq_hat == nullptr) || (q == nullptr) != (dq == nullptr))
+        return fail(KLA_ERR_INVALID_ARG, "q, dq_hat and dq must be given together (or all NULL)");
+    kla_status st = gate_checks(N, D, H, Dk, dtype, q != nullptr);
+    if (st != KLA_OK) return st;
+    REQUIRE_PTR(dW); REQUIRE_PTR(dbias);
+    if (N > 0) {
+        REQUIRE_PTR(x); REQUIRE_PTR(W); REQUIRE_PTR(eta); REQUIRE_PTR(g); REQUIRE_PTR(deta); REQUIRE_PTR(dg);
+        REQUIRE_PTR(dx);
+    }
+    OPTIONAL_PTR(q); OPTIONAL_PTR(dq_hat); OPTIONAL_PTR(dq);
+    const size_t need = kla::gate_bwd_workspace(N, D, H);
+    if (N > 0 && (ws == nullptr || ws_bytes < need))
+        return fail(KLA_ERR_WORKSPACE, "kla_gate_prologue_bwd needs %zu workspace bytes (got %zu)", need,
+                    ws == nullptr ? (size_t)0 : ws_bytes);
+    if (!aligned16(ws)) return fail(KLA_ERR_INVALID_ARG, "ws must be 16-byte aligned");
+    kla::GateBwdArgs a{x, W, eta, g, deta, dg, q, dq_hat, dx, dW, dbias, dq, N, D, H, Dk, dtype == KLA_BF16};
+    cudaError_t e = kla::launch_gate_prologue_bwd(a, ws, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "kla_gate_prologue_bwd launch");
+    return KLA_OK;
+}
+
 void kla_debug_inject_wait_timeout(void) { g_inject_timeout.store(1); }
 
 kla_status kla_check_device_error(void* stream) {
-    unsigned int flag = 0, flag2 = 0, flag3 = 0, flag4 = 0;
+    unsigned int flag = 0, flag2 = 0, flag3 = 0, flag4 = 0, flag5 = 0;
     cudaError_t e = kla::tc_take_error(static_cast<cudaStream_t>(stream), &flag);
     if (e == cudaSuccess) e = kla::decode_take_error(static_cast<cudaStream_t>(stream), &flag2);
     if (e == cudaSuccess) e = kla::split_take_error(static_cast<cudaStream_t>(stream), &flag3);
     if (e == cudaSuccess) e = kla::bwd_tc_take_error(static_cast<cudaStream_t>(stream), &flag4);
+    if (e == cudaSuccess) e = kla::gates_take_error(static_cast<cudaStream_t>(stream), &flag5);
     if (e != cudaSuccess) return cuda_fail(e, "kla_check_device_error");
-    flag |= (flag2 << 8) | (flag3 << 16) | (flag4 << 24);
+    flag |= (flag2 << 8) | (flag3 << 16) | (flag4 << 24) | (flag5 << 4);
     if (flag) return fail(KLA_ERR_TIMEOUT, "a kernel gave up on a bounded wait (flag %u)", flag);
     return KLA_OK;
 }

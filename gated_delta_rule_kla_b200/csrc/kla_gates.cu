@@ -1,0 +1,434 @@
+// kla_gates.cu -- the gate prologue: the per-token inputs of the KLA recurrence that come from
+// the layer's token vector x_t ("Kaczmarz Linear Attention", section 3.3: eta_t is a
+// sigmoid-activated linear projection of the input token; alpha_t = exp(g_t)):
+//   z_t   = W x_t + bias                    W [2H, D]: rows 0..H-1 eta, rows H..2H-1 decay
+//   eta_t = sigmoid(z_t[0:H])               (write gate, one per head)
+//   g_t   = -softplus(z_t[H:2H])            (log-decay, <= 0)
+//   qhat  = q / ||q||  per (token, head)    (Algorithm 1's readout divides by ||q_t||; o is
+//                                            linear in q, so the recurrence on qhat is that
+//                                            readout; a zero query gives qhat = 0)
+// x is read once for all heads, which is why this is its own kernel rather than part of the
+// per-(chunk, head) preparation kernel (that would read each token's x once per head).
+//
+// bf16 with D % 64 == 0 and 2H in {16, 32, ..., 256}: one CTA per 128 tokens runs the
+// projection on the tensor cores (tcgen05, M = 128 tokens, N = 2H, K = D in 64-wide steps
+// through a 4-stage TMA ring), the activations in the TMEM epilogue, and the query
+// normalisation on the warps that neither load nor issue.  Other shapes and fp32: CUDA cores.
+//
+// Backward (CUDA cores): with dz = [deta * eta (1 - eta), dg * expm1(g)] (d(-softplus z)/dz =
+// -sigmoid(z) = expm1(g)),  dx = dz W,  dW = dz^T x,  dbias = sum_t dz,
+// dq = (dqhat - qhat (qhat . dqhat)) / ||q||.  dW and dbias are summed per 64-token tile into
+// the workspace and then over tiles in a fixed order (deterministic).
+#include <cuda.h>
+
+#include "kla_device.cuh"
+#include "kla_launch.h"
+#include "kla_sm100.cuh"
+#include "kla_tc_common.cuh"
+
+namespace kla {
+
+__device__ unsigned int g_gates_error = 0;
+
+namespace {
+
+using namespace sm100;
+
+constexpr uint64_t kWaitNs = 2000000000ull;
+constexpr int GM = 128;    // tokens per CTA
+constexpr int GKT = 64;    // K elements per stage (128 bytes of bf16)
+constexpr int GST = 4;     // stages
+constexpr int GTH = 256;   // threads: warps 0-3 epilogue, 4 loader, 5 MMA issuer; q rows on 0-3, 6, 7
+
+__device__ __forceinline__ float sigmoidf_(float z) { return 1.f / (1.f + __expf(-z)); }
+__device__ __forceinline__ float softplusf_(float z) { return fmaxf(z, 0.f) + log1pf(__expf(-fabsf(z))); }
+
+// q rows (token, head) of tokens [tok0, tok0 + ntok), warp-strided: qhat = q / ||q||.
+template <typename Tin>
+__device__ __forceinline__ void normalize_rows(const Tin* q, Tin* qhat, size_t tok0, int ntok, int H, int Dk,
+                                               int wid, int nwarps) {
+    const int lane = threadIdx.x & 31;
+    const int per = Dk / 32;
+    for (int r = wid; r < ntok * H; r += nwarps) {
+        const size_t base = (tok0 * H + r) * (size_t)Dk;
+        float x[4];
+        float s = 0.f;
+        for (int u = 0; u < per; ++u) {
+            x[u] = to_f32(q[base + lane + 32 * u]);
+            s = fmaf(x[u], x[u], s);
+        }
+        s = warp_sum(s);
+        const float inv = s > 0.f ? rsqrtf(s) : 0.f;
+        for (int u = 0; u < per; ++u) qhat[base + lane + 32 * u] = from_f32<Tin>(x[u] * inv);
+    }
+}
+
+// ------------------------------------------------------------------------------------
+// Tensor-core projection (bf16).  Stage s: x tile [128 tokens x 64] (16 KB) then the W tile
+// [NW rows x 64] (NW * 128 bytes, rounded up to 1 KB), both K-major with the 128-byte swizzle.
+// ------------------------------------------------------------------------------------
+struct GateBars {
+    uint64_t full[GST], empty[GST], done;
+    uint32_t tmem_base;
+};
+
+__global__ void __launch_bounds__(GTH, 1)
+    gate_prologue_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
+                            const float* __restrict__ bias, float* __restrict__ eta, float* __restrict__ g,
+                            const __nv_bfloat16* __restrict__ q, __nv_bfloat16* __restrict__ qhat, int N, int D,
+                            int H, int Dk, uint32_t w_bytes, uint32_t tmem_cols) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t stage_bytes = 16384 + w_bytes;
+    GateBars* bars = reinterpret_cast<GateBars*>(sm + GST * stage_bytes);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int NW = 2 * H, KT = D / GKT;
+    const int tok0 = blockIdx.x * GM;
+    const int ntok = min(GM, N - tok0);
+    const uint32_t sbase = smem_u32(sm);
+
+    if (tid == 0) {
+        for (int s = 0; s < GST; ++s) {
+            mbar_init(smem_u32(&bars->full[s]), 1);
+            mbar_init(smem_u32(&bars->empty[s]), 1);
+        }
+        mbar_init(smem_u32(&bars->done), 1);
+        fence_mbar_init();
+        prefetch_tmap(&tm_x);
+        prefetch_tmap(&tm_w);
+    }
+    if (warp == 0) {
+        tmem_alloc(smem_u32(&bars->tmem_base), tmem_cols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = bars->tmem_base;
+    bool ok = true;
+
+    if (warp == 4) {
+        if (lane == 0) {  // loader
+            for (int kt = 0; kt < KT && ok; ++kt) {
+                const int s = kt % GST;
+                if (kt >= GST) ok = mbar_wait_bounded(smem_u32(&bars->empty[s]), ((kt / GST) - 1) & 1, kWaitNs);
+                if (!ok) break;
+                const uint32_t full = smem_u32(&bars->full[s]);
+                mbar_expect_tx(full, 16384 + (uint32_t)NW * 128);
+                tma_load_2d(sbase + s * stage_bytes, &tm_x, full, kt * GKT, tok0);
+                tma_load_2d(sbase + s * stage_bytes + 16384, &tm_w, full, kt * GKT, 0);
+            }
+        }
+    } else if (warp == 5) {
+        if (lane == 0) {  // MMA issuer: Z[token][j] = sum_k x[token][k] W[j][k]
+            const uint32_t idesc = idesc_bf16(GM, NW, false, false);
+            for (int kt = 0; kt < KT && ok; ++kt) {
+                const int s = kt % GST;
+                ok = mbar_wait_bounded(smem_u32(&bars->full[s]), (kt / GST) & 1, kWaitNs);
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t a = sbase + s * stage_bytes, bw = a + 16384;
+#pragma unroll
+                for (int k = 0; k < GKT / 16; ++k)
+                    mma_bf16(tmem, smem_desc(a + 32 * k, 16, 1024), smem_desc(bw + 32 * k, 16, 1024), idesc,
+                             (kt | k) > 0);
+                mma_commit(smem_u32(&bars->empty[s]));
+            }
+            mma_commit(smem_u32(&bars->done));
+        }
+    }
+    // query normalisation on the other warps while the projection runs
+    if (q != nullptr && warp != 4 && warp != 5)
+        normalize_rows<__nv_bfloat16>(q, qhat, (size_t)tok0, ntok, H, Dk, warp < 4 ? warp : warp - 2, 6);
+    if (warp < 4) {  // epilogue: lane = token
+        const bool got = mbar_wait_bounded(smem_u32(&bars->done), 0, kWaitNs);
+        if (__any_sync(0xffffffffu, !got)) {
+            ok = false;
+        } else {
+            tc_fence_after();
+            const int t = 32 * warp + lane;
+            const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
+            for (int c0 = 0; c0 < NW; c0 += 16) {
+                uint32_t z[16];
+                tmem_ld16u(tmem + lane_base + c0, z);
+                tmem_ld_wait();
+                if (t < ntok) {
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const int j = c0 + e;
+                        const float zz = __uint_as_float(z[e]) + bias[j];
+                        if (j < H)
+                            eta[(size_t)(tok0 + t) * H + j] = sigmoidf_(zz);
+                        else
+                            g[(size_t)(tok0 + t) * H + (j - H)] = -softplusf_(zz);
+                    }
+                }
+            }
+        }
+    }
+    if (!ok) atomicOr(&g_gates_error, 1u);
+    tc_fence_before();
+    __syncthreads();
+    // a stage that never completed leaves no copy in flight: the loader stops before issuing
+    // past an expired wait, and every issued copy completes its own barrier
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, tmem_cols);
+    }
+}
+
+// ------------------------------------------------------------------------------------
+// CUDA-core projection: one warp per token, outputs in groups of 8.
+// ------------------------------------------------------------------------------------
+template <typename Tin>
+__global__ void __launch_bounds__(256) gate_prologue_simt_kernel(const Tin* __restrict__ x, const Tin* __restrict__ W,
+                                                                 const float* __restrict__ bias, float* __restrict__ eta,
+                                                                 float* __restrict__ g, const Tin* __restrict__ q,
+                                                                 Tin* __restrict__ qhat, int N, int D, int H, int Dk) {
+    const int lane = threadIdx.x & 31;
+    const size_t t = (size_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (t >= (size_t)N) return;
+    const int NW = 2 * H;
+    const Tin* xr = x + t * D;
+    for (int j0 = 0; j0 < NW; j0 += 8) {
+        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        for (int d = lane; d < D; d += 32) {
+            const float xv = to_f32(xr[d]);
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                if (j0 + e < NW) acc[e] = fmaf(xv, to_f32(W[(size_t)(j0 + e) * D + d]), acc[e]);
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] = warp_sum(acc[e]);
+        if (lane < 8 && j0 + lane < NW) {
+            float zz = 0.f;
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                if (e == lane) zz = acc[e];
+            const int j = j0 + lane;
+            zz += bias[j];
+            if (j < H)
+                eta[t * H + j] = sigmoidf_(zz);
+            else
+                g[t * H + (j - H)] = -softplusf_(zz);
+        }
+    }
+    if (q != nullptr) normalize_rows<Tin>(q, qhat, t, 1, H, Dk, 0, 1);
+}
+
+// ------------------------------------------------------------------------------------
+// Backward, per tile of 64 tokens: dz to shared memory; dx = dz W; partial dW, dbias of the
+// tile to the workspace; dq from dqhat.
+// ------------------------------------------------------------------------------------
+constexpr int BT = 64;    // tokens per tile
+constexpr int BD = 128;   // x / W columns per pass
+
+template <typename Tin>
+__global__ void __launch_bounds__(256) gate_bwd_tile_kernel(const Tin* __restrict__ x, const Tin* __restrict__ W,
+                                                            const float* __restrict__ eta, const float* __restrict__ g,
+                                                            const float* __restrict__ deta, const float* __restrict__ dg,
+                                                            const Tin* __restrict__ q, const float* __restrict__ dqhat,
+                                                            float* __restrict__ dx, float* __restrict__ dq,
+                                                            float* __restrict__ part_w, float* __restrict__ part_b,
+                                                            int N, int D, int H, int Dk) {
+    extern __shared__ float smf[];
+    const int NW = 2 * H;
+    float* dz = smf;                   // [BT][NW]
+    float* xs = dz + BT * NW;          // [BT][BD + 1]
+    float* wsh = xs + BT * (BD + 1);   // [NW][BD + 1]
+    const int tid = threadIdx.x;
+    const int tile = blockIdx.x;
+    const int t0 = tile * BT;
+    const int nt = min(BT, N - t0);
+    for (int i = tid; i < BT * NW; i += 256) {
+        const int t = i / NW, j = i % NW;
+        float v = 0.f;
+        if (t < nt) {
+            const size_t o = (size_t)(t0 + t) * H;
+            if (j < H) {
+                const float e = eta[o + j];
+                v = deta[o + j] * e * (1.f - e);
+            } else {
+                v = dg[o + j - H] * expm1f(g[o + j - H]);
+            }
+        }
+        dz[i] = v;
+    }
+    __syncthreads();
+    if (tid < NW) {  // dbias partial, fixed order over the tile's tokens
+        float s = 0.f;
+        for (int t = 0; t < BT; ++t) s += dz[t * NW + tid];
+        part_b[(size_t)tile * NW + tid] = s;
+    }
+    for (int d0 = 0; d0 < D; d0 += BD) {
+        const int nd = min(BD, D - d0);
+        __syncthreads();
+        for (int i = tid; i < BT * BD; i += 256) {
+            const int t = i / BD, c = i % BD;
+            xs[t * (BD + 1) + c] = (t < nt && c < nd) ? to_f32(x[(size_t)(t0 + t) * D + d0 + c]) : 0.f;
+        }
+        for (int i = tid; i < NW * BD; i += 256) {
+            const int j = i / BD, c = i % BD;
+            wsh[j * (BD + 1) + c] = c < nd ? to_f32(W[(size_t)j * D + d0 + c]) : 0.f;
+        }
+        __syncthreads();
+        // dx[t][c] = sum_j dz[t][j] W[j][c]: thread = column c (128) x token half
+        {
+            const int c = tid & (BD - 1), th = tid >> 7;
+            if (c < nd) {
+                for (int t = th; t < nt; t += 2) {
+                    float s = 0.f;
+                    for (int j = 0; j < NW; ++j) s = fmaf(dz[t * NW + j], wsh[j * (BD + 1) + c], s);
+                    dx[(size_t)(t0 + t) * D + d0 + c] = s;
+                }
+            }
+        }
+        // dW partial [j][c] = sum_t dz[t][j] x[t][c]
+        for (int i = tid; i < NW * BD; i += 256) {
+            const int j = i / BD, c = i % BD;
+            if (c < nd) {
+                float s = 0.f;
+                for (int t = 0; t < BT; ++t) s = fmaf(dz[t * NW + j], xs[t * (BD + 1) + c], s);
+                part_w[((size_t)tile * NW + j) * D + d0 + c] = s;
+            }
+        }
+    }
+    // dq = (dqhat - qhat (qhat . dqhat)) / ||q||, one warp per (token, head)
+    if (q != nullptr) {
+        const int lane = tid & 31, wid = tid >> 5;
+        const int per = Dk / 32;
+        for (int r = wid; r < nt * H; r += 8) {
+            const size_t base = ((size_t)t0 * H + r) * Dk;
+            float qv[4], dv[4];
+            float s = 0.f, p = 0.f;
+            for (int u = 0; u < per; ++u) {
+                qv[u] = to_f32(q[base + lane + 32 * u]);
+                dv[u] = dqhat[base + lane + 32 * u];
+                s = fmaf(qv[u], qv[u], s);
+                p = fmaf(qv[u], dv[u], p);
+            }
+            s = warp_sum(s);
+            p = warp_sum(p);
+            const float inv = s > 0.f ? rsqrtf(s) : 0.f;  // 1 / ||q||
+            // qhat . dqhat = p / ||q||
+            for (int u = 0; u < per; ++u) dq[base + lane + 32 * u] = inv * (dv[u] - qv[u] * inv * (p * inv));
+        }
+    }
+}
+
+// dW[j][d] = sum over tiles (fixed order), dbias[j] likewise.
+__global__ void gate_bwd_reduce_kernel(const float* __restrict__ part_w, const float* __restrict__ part_b,
+                                       float* __restrict__ dW, float* __restrict__ db, int ntile, int NW, int D) {
+    const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const size_t total = (size_t)NW * D;
+    if (i < total) {
+        float s = 0.f;
+        for (int t = 0; t < ntile; ++t) s += part_w[(size_t)t * total + i];
+        dW[i] = s;
+    }
+    if (i < (size_t)NW) {
+        float s = 0.f;
+        for (int t = 0; t < ntile; ++t) s += part_b[(size_t)t * NW + i];
+        db[i] = s;
+    }
+}
+
+bool gate_tc_shape(const GateArgs& a) {
+    return a.bf16 && a.D % GKT == 0 && a.H % 8 == 0 && 2 * a.H <= 256 && a.N >= 1;
+}
+
+}  // namespace
+
+size_t gate_bwd_workspace(int N, int D, int H) {
+    const size_t ntile = ((size_t)N + BT - 1) / BT;
+    return ntile * 2 * H * ((size_t)D + 1) * sizeof(float);
+}
+
+cudaError_t launch_gate_prologue(const GateArgs& a, cudaStream_t st) {
+    if (a.N == 0) return cudaSuccess;
+    if (gate_tc_shape(a)) {
+        EncodeTiledFn enc = get_encode_fn();
+        if (enc != nullptr) {
+            const int NW = 2 * a.H;
+            CUtensorMap mx, mw;
+            const cuuint64_t dx[2] = {(cuuint64_t)a.D, (cuuint64_t)a.N};
+            const cuuint64_t sx[1] = {(cuuint64_t)a.D * 2};
+            const cuuint32_t bx[2] = {GKT, GM};
+            const cuuint64_t dw[2] = {(cuuint64_t)a.D, (cuuint64_t)NW};
+            const cuuint32_t bw[2] = {GKT, (cuuint32_t)NW};
+            const cuuint32_t es[2] = {1, 1};
+            if (enc(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(a.x), dx, sx, bx, es,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS ||
+                enc(&mw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(a.W), dw, sx, bw, es,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+                return cudaErrorInvalidValue;
+            const uint32_t w_bytes = ((uint32_t)NW * 128 + 1023) & ~1023u;
+            uint32_t cols = 32;
+            while (cols < (uint32_t)NW) cols <<= 1;
+            const size_t smem = 1024 + GST * (16384 + (size_t)w_bytes) + sizeof(GateBars);
+            cudaError_t e = cudaFuncSetAttribute(gate_prologue_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 (int)smem);
+            if (e != cudaSuccess) return e;
+            gate_prologue_tc_kernel<<<(a.N + GM - 1) / GM, GTH, smem, st>>>(
+                mx, mw, a.bias, a.eta, a.g, static_cast<const __nv_bfloat16*>(a.q),
+                static_cast<__nv_bfloat16*>(a.qhat), a.N, a.D, a.H, a.Dk, w_bytes, cols);
+            return cudaGetLastError();
+        }
+    }
+    const unsigned grid = (unsigned)(((size_t)a.N + 7) / 8);
+    if (a.bf16)
+        gate_prologue_simt_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
+            static_cast<const __nv_bfloat16*>(a.x), static_cast<const __nv_bfloat16*>(a.W), a.bias, a.eta, a.g,
+            static_cast<const __nv_bfloat16*>(a.q), static_cast<__nv_bfloat16*>(a.qhat), a.N, a.D, a.H, a.Dk);
+    else
+        gate_prologue_simt_kernel<float><<<grid, 256, 0, st>>>(
+            static_cast<const float*>(a.x), static_cast<const float*>(a.W), a.bias, a.eta, a.g,
+            static_cast<const float*>(a.q), static_cast<float*>(a.qhat), a.N, a.D, a.H, a.Dk);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gate_prologue_bwd(const GateBwdArgs& a, void* ws, cudaStream_t st) {
+    if (a.N == 0) {
+        cudaError_t e = cudaMemsetAsync(a.dW, 0, (size_t)2 * a.H * a.D * sizeof(float), st);
+        if (e == cudaSuccess) e = cudaMemsetAsync(a.db, 0, (size_t)2 * a.H * sizeof(float), st);
+        return e;
+    }
+    const int NW = 2 * a.H;
+    const int ntile = (a.N + BT - 1) / BT;
+    float* part_w = static_cast<float*>(ws);
+    float* part_b = part_w + (size_t)ntile * NW * a.D;
+    const size_t smem = sizeof(float) * ((size_t)BT * NW + (size_t)BT * (BD + 1) + (size_t)NW * (BD + 1));
+    cudaError_t e;
+    if (a.bf16) {
+        e = cudaFuncSetAttribute(gate_bwd_tile_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)smem);
+        if (e != cudaSuccess) return e;
+        gate_bwd_tile_kernel<__nv_bfloat16><<<ntile, 256, smem, st>>>(
+            static_cast<const __nv_bfloat16*>(a.x), static_cast<const __nv_bfloat16*>(a.W), a.eta, a.g, a.deta, a.dg,
+            static_cast<const __nv_bfloat16*>(a.q), a.dqhat, a.dx, a.dq, part_w, part_b, a.N, a.D, a.H, a.Dk);
+    } else {
+        e = cudaFuncSetAttribute(gate_bwd_tile_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        gate_bwd_tile_kernel<float><<<ntile, 256, smem, st>>>(
+            static_cast<const float*>(a.x), static_cast<const float*>(a.W), a.eta, a.g, a.deta, a.dg,
+            static_cast<const float*>(a.q), a.dqhat, a.dx, a.dq, part_w, part_b, a.N, a.D, a.H, a.Dk);
+    }
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    const size_t total = (size_t)NW * a.D;
+    gate_bwd_reduce_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(part_w, part_b, a.dW, a.db, ntile, NW,
+                                                                            a.D);
+    return cudaGetLastError();
+}
+
+cudaError_t gates_take_error(cudaStream_t st, unsigned int* flag) {
+    cudaError_t e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return e;
+    e = cudaMemcpyFromSymbol(flag, g_gates_error, sizeof(unsigned int));
+    if (e != cudaSuccess) return e;
+    const unsigned int zero = 0;
+    return cudaMemcpyToSymbol(g_gates_error, &zero, sizeof(unsigned int));
+}
+
+}  // namespace kla

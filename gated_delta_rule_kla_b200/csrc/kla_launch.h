@@ -91,6 +91,34 @@ cudaError_t launch_chunk_bwd_tc_reverse(const BwdTcArgs& a, void* ws, size_t ws_
 cudaError_t bwd_tc_take_error(cudaStream_t st, unsigned int* flag);
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st);
+
+// Gate prologue: eta = sigmoid(z[:, :H]), g = -softplus(z[:, H:]) with z = x W^T + bias, and
+// (when q is given) qhat = q / ||q|| per (token, head).  x [N, D], W [2H, D], q/qhat [N, H, Dk]
+// in the input type; bias [2H], eta, g [N, H] fp32.
+struct GateArgs {
+    const void *x, *W;
+    const float* bias;
+    const void* q;  // may be null (then qhat is not written)
+    float *eta, *g;
+    void* qhat;
+    int N, D, H, Dk;
+    bool bf16;
+};
+// Backward of the prologue from its outputs eta, g and the upstream gradients; writes
+// dx [N, D], dW [2H, D], dbias [2H], and dq [N, H, Dk] when q is given (all fp32).
+struct GateBwdArgs {
+    const void *x, *W;
+    const float *eta, *g, *deta, *dg;
+    const void* q;
+    const float* dqhat;
+    float *dx, *dW, *db, *dq;
+    int N, D, H, Dk;
+    bool bf16;
+};
+cudaError_t launch_gate_prologue(const GateArgs& a, cudaStream_t st);
+size_t gate_bwd_workspace(int N, int D, int H);
+cudaError_t launch_gate_prologue_bwd(const GateBwdArgs& a, void* ws, cudaStream_t st);
+cudaError_t gates_take_error(cudaStream_t st, unsigned int* flag);
 // Diagonal (per-key-channel) gating on CUDA cores: g is [B, T, H, Dk].  The kernels work in
 // chunks of diag_chunk_len() tokens; S_chunks of the forward (optional) and of the backward
 // (required: the workspace region the backward launcher fills first) are per such chunk.  The

@@ -24,6 +24,11 @@ workload dtype (round-to-nearest-even for bf16); eta, g, S0, dO stay fp32.
                                       (gate_mode "diag": diagonal gating, App. A.5)
   S0          = 0 or 0.02 * N(0, 1)
   dO          ~ N(0, 1)               (training workload only)
+
+Gate prologue (make_gate_inputs): token vectors x ~ N(0, 1) [N, D]; projections
+W ~ N(0, 1/D) [2H, D] (unit-variance logits); bias_eta ~ N(0, 1), bias_g ~ N(0, 1) - 2 (so
+that -softplus keeps most decays mild); q ~ N(0, 1) [N, H, Dk] with a spread of norms
+(each row times a log-uniform factor on [0.1, 10]).
 """
 from dataclasses import dataclass, replace
 import math
@@ -128,4 +133,22 @@ def make_inputs(w: Workload, device=None):
         out["dO"] = torch.randn(w.B, w.T, w.H, w.Dv, generator=gen, dtype=f64).float()
     if device is not None:
         out = {key: (t.to(device) if t is not None else None) for key, t in out.items()}
+    return out
+
+
+def make_gate_inputs(N, D, H, Dk, dtype, seed, device=None):
+    """Seeded inputs of the gate prologue (see the module docstring): x [N, D], W [2H, D] and
+    q [N, H, Dk] in `dtype` ("f32" or "bf16"), bias [2H] fp32."""
+    gen = torch.Generator(device="cpu").manual_seed(seed)
+    f64 = torch.float64
+    tdt = torch.float32 if dtype == "f32" else torch.bfloat16
+    x = torch.randn(N, D, generator=gen, dtype=f64)
+    W = torch.randn(2 * H, D, generator=gen, dtype=f64) / math.sqrt(D)
+    bias = torch.randn(2 * H, generator=gen, dtype=f64)
+    bias[H:] -= 2.0
+    q = torch.randn(N, H, Dk, generator=gen, dtype=f64)
+    q = q * torch.exp(torch.empty(N, H, 1, dtype=f64).uniform_(math.log(0.1), math.log(10.0), generator=gen))
+    out = dict(x=x.to(tdt), W=W.to(tdt), bias=bias.float(), q=q.to(tdt))
+    if device is not None:
+        out = {key: t.to(device) for key, t in out.items()}
     return out

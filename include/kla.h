@@ -255,6 +255,42 @@ kla_status kla_decode_step_diag(const void *q, const void *k, const void *v, con
                                 int Dk, int Dv, int dtype, int out_dtype, void *stream);
 
 /*
+ * kla_gate_prologue -- the per-token inputs of the recurrence computed from the layer's token
+ * vectors, for every head at once ("Kaczmarz Linear Attention", section 3.3: the write gate is a
+ * sigmoid-activated linear projection of the input token; alpha_t = exp(g_t)):
+ *     z_t = W x_t + bias,  eta_t[h] = sigmoid(z_t[h]),  g_t[h] = -softplus(z_t[H + h])
+ * and, when q is given, qhat = q / ||q|| per (token, head) (Algorithm 1's readout divides by
+ * ||q_t||; o is linear in q, so the recurrence run on qhat gives that readout; a zero query
+ * gives qhat = 0).  The pages print no projection for g: the one here is a reading (a linear
+ * projection through -softplus, so that g <= 0).
+ *   x      in   [N, D] of `dtype` (N = B*T tokens; D % 8 == 0 for bf16, % 4 for fp32)
+ *   W      in   [2H, D] of `dtype`: rows 0..H-1 project eta, rows H..2H-1 project g
+ *   bias   in   [2H] fp32
+ *   q      in   [N, H, Dk] of `dtype`, or NULL (no normalisation); Dk in {64, 128}
+ *   eta, g out  [N, H] fp32
+ *   q_hat  out  [N, H, Dk] of `dtype` (NULL exactly when q is NULL)
+ * 1 <= H <= 64.  bf16 with D % 64 == 0 and H % 8 == 0 runs the projection on the tensor cores
+ * (fp32 accumulation); other shapes and fp32 on CUDA cores.  Returns KLA_OK or an error status;
+ * on error nothing is launched.
+ *
+ * kla_gate_prologue_bwd -- gradients of <eta, deta> + <g, dg> (+ <q_hat, dq_hat>) with respect
+ * to x, W, bias (and q), from the prologue's own outputs eta and g for the same x, W, bias:
+ *     dz = [deta * eta (1 - eta), dg * expm1(g)],  dx = dz W,  dW = dz^T x,  dbias = sum_t dz,
+ *     dq = (dq_hat - q_hat (q_hat . dq_hat)) / ||q||   (zero where q is zero)
+ * deta, dg [N, H], dq_hat [N, H, Dk] fp32 in; dx [N, D], dW [2H, D], dbias [2H], dq [N, H, Dk]
+ * fp32 out (q, dq_hat and dq all given or all NULL).  ws: device, 16-byte aligned,
+ * caller-owned, at least kla_gate_prologue_bwd_workspace() bytes (per-tile partial sums of dW
+ * and dbias, added in a fixed order: the result is deterministic).
+ */
+kla_status kla_gate_prologue(const void *x, const void *W, const float *bias, const void *q, float *eta,
+                             float *g, void *q_hat, int N, int D, int H, int Dk, int dtype, void *stream);
+size_t kla_gate_prologue_bwd_workspace(int N, int D, int H);
+kla_status kla_gate_prologue_bwd(const void *x, const void *W, const float *eta, const float *g,
+                                 const void *q, const float *deta, const float *dg, const float *dq_hat,
+                                 float *dx, float *dW, float *dbias, float *dq, int N, int D, int H, int Dk,
+                                 int dtype, void *ws, size_t ws_bytes, void *stream);
+
+/*
  * kla_check_device_error -- synchronises `stream`, then reads and clears the library's
  * device error word.  Returns KLA_ERR_TIMEOUT if a kernel gave up on a bounded internal
  * wait since the last check (its outputs are then invalid), KLA_ERR_CUDA if the stream
