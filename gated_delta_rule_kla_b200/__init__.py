@@ -83,7 +83,9 @@ def lib():
         L.kla_check_device_error.restype = i
         L.kla_debug_inject_wait_timeout.argtypes = []
         L.kla_debug_inject_wait_timeout.restype = None
-        L.kla_chunk_fwd_diag.argtypes = [vp, vp, vp, fp, fp, f, fp, vp, fp, i, i, i, i, i, i, i, i, vp]
+        L.kla_chunk_fwd_diag_workspace.argtypes = [i, i, i, i, i, i, i]
+        L.kla_chunk_fwd_diag_workspace.restype = sz
+        L.kla_chunk_fwd_diag.argtypes = [vp, vp, vp, fp, fp, f, fp, vp, fp, i, i, i, i, i, i, i, i, vp, sz, vp]
         L.kla_chunk_fwd_diag.restype = i
         L.kla_chunk_bwd_diag_workspace.argtypes = [i, i, i, i, i, i, i]
         L.kla_chunk_bwd_diag_workspace.restype = sz
@@ -364,9 +366,11 @@ def decode_step(q, k, v, eta, g, S, eps=1e-6, *, o=None, out_dtype=torch.float32
 
 
 def chunk_fwd_diag(q, k, v, eta, g, eps=1e-6, S0=None, *, o=None, S_T=None, out_dtype=torch.float32,
-                   stream=None, beta="kaczmarz"):
+                   stream=None, beta="kaczmarz", workspace=None, fused=False):
     """Prefill with diagonal (per-key-channel) gating (Appendix A.5, B.5): g is [B,T,H,Dk] fp32,
-    the decay of token t is Diag(exp(g_t)).  Other arguments as chunk_fwd.  Returns (o, S_T)."""
+    the decay of token t is Diag(exp(g_t)).  Other arguments as chunk_fwd.  The split path's
+    workspace (kla_chunk_fwd_diag_workspace) is allocated here unless given; fused=True passes
+    none (the one-kernel path).  Returns (o, S_T)."""
     dev = k.device
     B, T, H, Dk = k.shape
     Dv = v.shape[-1]
@@ -380,9 +384,14 @@ def chunk_fwd_diag(q, k, v, eta, g, eps=1e-6, S0=None, *, o=None, S_T=None, out_
     if S_T is None:
         S_T = torch.empty(B, H, Dk, Dv, device=dev, dtype=torch.float32)
     _need(S_T, "S_T", dev, torch.float32, (B, H, Dk, Dv))
-    st = lib().kla_chunk_fwd_diag(_ptr(q), _ptr(k), _ptr(v), _ptr(eta), _ptr(g), float(eps), _ptr(S0), _ptr(o),
-                                  _ptr(S_T), B, T, H, Dk, Dv, CHUNK, _in_code(k, beta), _dtype_code(o),
-                                  _stream(dev, stream))
+    L = lib()
+    need = 0 if fused else L.kla_chunk_fwd_diag_workspace(B, T, H, Dk, Dv, CHUNK, _dtype_code(k))
+    if need > 0 and (workspace is None or workspace.numel() < need):
+        workspace = torch.empty(need, device=dev, dtype=torch.uint8)
+    ws_ptr, ws_n = (_ptr(workspace), workspace.numel()) if need > 0 else (None, 0)
+    st = L.kla_chunk_fwd_diag(_ptr(q), _ptr(k), _ptr(v), _ptr(eta), _ptr(g), float(eps), _ptr(S0), _ptr(o),
+                              _ptr(S_T), B, T, H, Dk, Dv, CHUNK, _in_code(k, beta), _dtype_code(o), ws_ptr, ws_n,
+                              _stream(dev, stream))
     _check(st, "kla_chunk_fwd_diag")
     return o, S_T
 

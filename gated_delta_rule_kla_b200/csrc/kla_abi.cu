@@ -91,7 +91,8 @@ bool tc_bwd_path(int B, int T, int H, int Dk, int Dv, int dtype, size_t ws_bytes
 }
 
 // Diagonal-gated backward: [S at every internal chunk start | acc_dq | acc_dkh | acc_dG (per
-// channel) | acc_db, acc_dc]; everything after the states is zeroed on every call.
+// channel) | acc_db, acc_dc | the split forward's records]; the accumulators are zeroed on
+// every call.
 size_t diag_bwd_ws_layout(int B, int T, int H, int Dk, int Dv, size_t* off) {
     const size_t CDl = (size_t)kla::diag_chunk_len();
     const size_t NC = ((size_t)T + CDl - 1) / CDl;
@@ -108,6 +109,8 @@ size_t diag_bwd_ws_layout(int B, int T, int H, int Dk, int Dv, size_t* off) {
     off[4] = o;
     o += align256(2 * ntok * sizeof(float));
     off[5] = o;
+    o += align256(kla::diag_fwd_workspace(B, T, H, Dk, Dv));
+    off[6] = o;
     return o;
 }
 
@@ -436,10 +439,17 @@ kla_status kla_decode_step_diag(const void* q, const void* k, const void* v, con
     return KLA_OK;
 }
 
+size_t kla_chunk_fwd_diag_workspace(int B, int T, int H, int Dk, int Dv, int chunk, int dtype) {
+    take_beta_flag(dtype);
+    if (B < 1 || H < 1 || T < 1 || chunk != kla::kChunkLen || (Dk != 64 && Dk != 128) || (Dv != 64 && Dv != 128))
+        return 0;
+    return kla::diag_fwd_workspace(B, T, H, Dk, Dv);
+}
+
 kla_status kla_chunk_fwd_diag(const void* q, const void* k, const void* v, const float* eta,
                               const float* g, float eps, const float* S0, void* o, float* S_T, int B,
                               int T, int H, int Dk, int Dv, int chunk, int dtype, int out_dtype,
-                              void* stream) {
+                              void* ws, size_t ws_bytes, void* stream) {
     const bool direct = take_beta_flag(dtype);
     kla_status st = check_common(B, T, H, Dk, Dv, chunk, dtype, out_dtype, eps);
     if (st != KLA_OK) return st;
@@ -457,9 +467,10 @@ kla_status kla_chunk_fwd_diag(const void* q, const void* k, const void* v, const
         }
         return KLA_OK;
     }
+    if (!aligned16(ws)) return fail(KLA_ERR_INVALID_ARG, "ws must be 16-byte aligned");
     kla::FwdArgs a{q, k, v, eta, g, kernel_eps(eps, direct), S0, o, S_T, nullptr, B, T, H, Dk, Dv,
                    dtype == KLA_BF16, out_dtype == KLA_BF16};
-    cudaError_t e = kla::launch_chunk_fwd_diag(a, s);
+    cudaError_t e = kla::launch_chunk_fwd_diag(a, ws, ws == nullptr ? 0 : ws_bytes, s);
     if (e != cudaSuccess) return cuda_fail(e, "kla_chunk_fwd_diag launch");
     return KLA_OK;
 }
@@ -468,7 +479,7 @@ size_t kla_chunk_bwd_diag_workspace(int B, int T, int H, int Dk, int Dv, int chu
     (void)chunk;
     take_beta_flag(dtype);
     if (B < 1 || H < 1 || T < 0) return 0;
-    size_t off[6];
+    size_t off[7];
     return diag_bwd_ws_layout(B, T, H, Dk, Dv, off);
 }
 
@@ -493,7 +504,7 @@ kla_status kla_chunk_bwd_diag(const void* q, const void* k, const void* v, const
     REQUIRE_PTR(q); REQUIRE_PTR(k); REQUIRE_PTR(v); REQUIRE_PTR(eta); REQUIRE_PTR(g);
     REQUIRE_PTR(dO); REQUIRE_PTR(dq); REQUIRE_PTR(dk); REQUIRE_PTR(dv); REQUIRE_PTR(deta);
     REQUIRE_PTR(dg);
-    size_t off[6];
+    size_t off[7];
     const size_t need = diag_bwd_ws_layout(B, T, H, Dk, Dv, off);
     if (ws == nullptr || ws_bytes < need)
         return fail(KLA_ERR_WORKSPACE, "kla_chunk_bwd_diag needs %zu workspace bytes (got %zu)", need,
@@ -509,7 +520,7 @@ kla_status kla_chunk_bwd_diag(const void* q, const void* k, const void* v, const
                    reinterpret_cast<float*>(w + off[2]), acc_b, acc_b + ntok,
                    reinterpret_cast<float*>(w + off[3]), B, T, H, Dk, Dv, dtype == KLA_BF16,
                    out_dtype == KLA_BF16};
-    e = kla::launch_chunk_bwd_diag(a, S0, s);
+    e = kla::launch_chunk_bwd_diag(a, S0, w + off[5], need - off[5], s);
     if (e != cudaSuccess) return cuda_fail(e, "kla_chunk_bwd_diag launch");
     return KLA_OK;
 }
@@ -582,6 +593,9 @@ kla_status kla_check_device_error(void* stream) {
     if (e == cudaSuccess) e = kla::split_take_error(static_cast<cudaStream_t>(stream), &flag3);
     if (e == cudaSuccess) e = kla::bwd_tc_take_error(static_cast<cudaStream_t>(stream), &flag4);
     if (e == cudaSuccess) e = kla::gates_take_error(static_cast<cudaStream_t>(stream), &flag5);
+    unsigned int flag6 = 0;
+    if (e == cudaSuccess) e = kla::diag_take_error(static_cast<cudaStream_t>(stream), &flag6);
+    flag5 |= flag6 << 1;
     if (e != cudaSuccess) return cuda_fail(e, "kla_check_device_error");
     flag |= (flag2 << 8) | (flag3 << 16) | (flag4 << 24) | (flag5 << 4);
     if (flag) return fail(KLA_ERR_TIMEOUT, "a kernel gave up on a bounded wait (flag %u)", flag);

@@ -26,9 +26,15 @@
 // dg by a reverse cumulative sum inside each 16-token chunk.
 #include "kla_device.cuh"
 #include "kla_launch.h"
+#include "kla_sm100.cuh"
 
 namespace kla {
+
+__device__ unsigned int g_diag_error = 0;
+
 namespace {
+
+using namespace sm100;
 
 constexpr int CD = 16;               // internal chunk length of the diagonal-gated kernels
 constexpr int NP = CD * (CD + 1) / 2;  // pairs j <= i inside a chunk
@@ -340,7 +346,7 @@ template <int DK>
 constexpr size_t diag_bwd_smem_bytes() {
     constexpr int NV = 32;
     return sizeof(float) * (2 * CD * (DK + 1) + CD * DK + NP * DK + 2 * DK * (NV + 1) + 4 * CD * (NV + 1) +
-                            5 * CD * (CD + 1) + 4 * CD + 8 + DK);
+                            5 * CD * (CD + 1) + 4 * CD + 8 + DK + CD * DK);
 }
 
 template <int DK, typename Tin, typename TOut>
@@ -371,6 +377,7 @@ __global__ void __launch_bounds__(NT, 1) chunk_bwd_diag_kernel(BwdArgs a, FwdArg
     float* dbs = us + CD;
     float* red = dbs + CD;        // 8
     float* lsS = red + 8;         // DK: row sums of lambda o S over this slice
+    float* xs = lsS + DK;         // CD x DK: per-token terms of the last token's dG
 
     const int v0 = blockIdx.x * NV, h = blockIdx.y, b = blockIdx.z;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -580,12 +587,13 @@ __global__ void __launch_bounds__(NT, 1) chunk_bwd_diag_kernel(BwdArgs a, FwdArg
                     atomicAdd(&a.acc_dq[ti * DK + d], dq);
                     atomicAdd(&a.acc_dkh[ti * DK + d], dk);
                     atomicAdd(&a.acc_dG[ti * DK + d], dG);
-                    // the outgoing decays (Del_j and Gam_last) feed dG of the chunk's last token
-                    const size_t tl = tok_index(b, t0 + n - 1, h, T, H);
-                    float extra = del * kd * zl[u];
-                    if (i == n - 1) extra += __expf(Gl) * lsS[d];
-                    atomicAdd(&a.acc_dG[tl * DK + d], extra);
+                    // the outgoing decays Del_j feed dG of the chunk's last token: summed over
+                    // the chunk's tokens below, one atomic per channel
+                    xs[i * DK + d] = del * kd * zl[u];
                 }
+            } else {
+#pragma unroll
+                for (int u = 0; u < EPT; ++u) xs[i * DK + tx + 16 * u] = 0.f;
             }
             // db: - (khat_i o Gam_i) . Z2_i (this thread's channels, then the row's 16 threads)
             kgz += __shfl_xor_sync(0xffffffffu, kgz, 1);
@@ -593,6 +601,12 @@ __global__ void __launch_bounds__(NT, 1) chunk_bwd_diag_kernel(BwdArgs a, FwdArg
             kgz += __shfl_xor_sync(0xffffffffu, kgz, 4);
             kgz += __shfl_xor_sync(0xffffffffu, kgz, 8);
             if (tx == 0 && i < n) atomicAdd(&dbs[i], -kgz);
+        }
+        __syncthreads();
+        if (tid < DK) {  // dG of the last token: sum_j Del_j o khat_j o Z3_j + Gam_last o rowsum(lambda o S)
+            float e = __expf(Gs[(n - 1) * DK + tid]) * lsS[tid];
+            for (int r = 0; r < n; ++r) e += xs[r * DK + tid];
+            atomicAdd(&a.acc_dG[tok_index(b, t0 + n - 1, h, T, H) * DK + tid], e);
         }
         // new lambda = Diag(Gam_last) lambda + (Q o Gam)^T dO - (Diag(b) (Khat o Gam))^T dR
         {
@@ -709,6 +723,280 @@ __global__ void diag_dg_kernel(BwdArgs a) {
     }
 }
 
+// ------------------------------------------------------------------------------------
+// Split forward.  `diag_prep_kernel` (one CTA per 16-token chunk and head, all at once) forms
+// everything that does not depend on the incoming state and stores it as an fp32 record:
+//   W  = T Diag(b) (Khat o Gam)   [16][DK]     T = (I + L)^{-1}
+//   QG = Q o Gam                  [16][DK]
+//   KD = Khat o Del               [16][DK]
+//   P                             [16][16]
+//   GC = Gam_last                 [DK]
+//   UP = T Diag(c) V              [DV/64][16][64]   (in 64-column slices)
+// `diag_state_kernel` then walks each head's chunks in order on a 64-column slice of the state:
+//   U = UP - W S,   O = QG S + P U,   S' = Diag(GC) S + KD^T U,
+// with the records double-buffered in shared memory by bulk copies.
+// ------------------------------------------------------------------------------------
+template <int DK, int DV>
+struct DiagRec {
+    static constexpr int kHead = 3 * CD * DK + CD * CD + DK;  // W, QG, KD, P, GC (floats)
+    static constexpr int kSlice = CD * 64;                     // one 64-column slice of UP
+    static constexpr int kFloats = kHead + (DV / 64) * kSlice;
+    static constexpr int W = 0, QG = CD * DK, KD = 2 * CD * DK, P = 3 * CD * DK, GC = 3 * CD * DK + CD * CD,
+                         UP = kHead;
+};
+
+template <int DK, int DV, typename Tin>
+__global__ void __launch_bounds__(NT) diag_prep_kernel(FwdArgs a, float* __restrict__ recs) {
+    using R = DiagRec<DK, DV>;
+    constexpr int LDK = DK + 1, LDC = CD + 1, LDV = DV + 1;
+    extern __shared__ float sm[];
+    float* Ks = sm;               // CD x LDK  unit keys
+    float* Qs = Ks + CD * LDK;    // CD x LDK  queries
+    float* Bk = Qs + CD * LDK;    // CD x LDK  b_j khat_j o Gam_j
+    float* Gs = Bk + CD * LDK;    // CD x DK   log-decay prefix
+    float* Vs = Gs + CD * DK;     // CD x LDV  c_j v_j
+    float* Am = Vs + CD * LDV;    // CD x LDC
+    float* Pm = Am + CD * LDC;    // CD x LDC
+    float* Tm = Pm + CD * LDC;    // CD x LDC  T = (I + L)^{-1}
+    float* bs = Tm + CD * LDC;
+    float* cs = bs + CD;
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int ci = blockIdx.x, head = blockIdx.y;
+    const int b = head / a.H, h = head % a.H;
+    const int NC = (a.T + CD - 1) / CD;
+    const int t0 = ci * CD, n = min(CD, a.T - t0);
+    float* rec = recs + ((size_t)head * NC + ci) * R::kFloats;
+    const Tin* v = static_cast<const Tin*>(a.v);
+
+    load_rows<DK, Tin>(a, b, h, t0, n, Ks, Qs, Gs, bs, cs, nullptr);
+    __syncthreads();
+    cumsum_rows<DK>(Gs);
+    for (int x = tid; x < CD * DV; x += NT) {
+        const int i = x / DV, j = x % DV;
+        Vs[i * LDV + j] = i < n ? cs[i] * to_f32(v[tok_index(b, t0 + i, h, a.T, a.H) * DV + j]) : 0.f;
+    }
+    __syncthreads();
+    chunk_grams<DK>(Ks, Qs, Gs, Am, Pm, nullptr);
+    // elementwise operands: Bk (for W), and the QG, KD, GC records
+    for (int x = tid; x < CD * DK; x += NT) {
+        const int i = x / DK, c = x % DK;
+        const float G = Gs[i * DK + c], Gl = Gs[(CD - 1) * DK + c];  // G is flat past the last token
+        const float gam = __expf(G);
+        const float kh = Ks[i * LDK + c];
+        Bk[i * LDK + c] = bs[i] * kh * gam;
+        rec[R::QG + x] = Qs[i * LDK + c] * gam;
+        rec[R::KD + x] = kh * __expf(Gl - G);
+        if (i == 0) rec[R::GC + c] = __expf(Gl);
+    }
+    __syncthreads();
+    // T = (I + Diag(b) A)^{-1}: lane j of warp 0 builds column j by forward substitution;
+    // the other warps store P
+    if (warp == 0) {
+        if (lane < CD) {
+            const int j = lane;
+            float col[CD];
+#pragma unroll
+            for (int i = 0; i < CD; ++i) {
+                float s = 0.f;
+#pragma unroll
+                for (int m = 0; m < i; ++m) s = fmaf(Am[i * LDC + m], col[m], s);
+                col[i] = (i < j) ? 0.f : ((i == j) ? 1.f : -bs[i] * s);
+            }
+#pragma unroll
+            for (int i = 0; i < CD; ++i) Tm[i * LDC + j] = col[i];
+        }
+    } else {
+        for (int x = tid - 32; x < CD * CD; x += NT - 32) rec[R::P + x] = Pm[(x / CD) * LDC + x % CD];
+    }
+    __syncthreads();
+    // W = T Bk and UP = T Vs (T is unit lower triangular)
+    {
+        const int i = tid >> 4, cx = tid & 15;
+#pragma unroll 4
+        for (int u = 0; u < DK / 16; ++u) {
+            const int c = cx + 16 * u;
+            float s = 0.f;
+            for (int j = 0; j <= i; ++j) s = fmaf(Tm[i * LDC + j], Bk[j * LDK + c], s);
+            rec[R::W + i * DK + c] = s;
+        }
+#pragma unroll 4
+        for (int u = 0; u < DV / 16; ++u) {
+            const int c = cx + 16 * u;
+            float s = 0.f;
+            for (int j = 0; j <= i; ++j) s = fmaf(Tm[i * LDC + j], Vs[j * LDV + c], s);
+            rec[R::UP + (c >> 6) * R::kSlice + i * 64 + (c & 63)] = s;
+        }
+    }
+}
+
+template <int DK, int DV>
+constexpr size_t diag_prep_smem_bytes() {
+    return sizeof(float) * (3 * CD * (DK + 1) + CD * DK + CD * (DV + 1) + 3 * CD * (CD + 1) + 2 * CD);
+}
+
+template <int DK, int DV>
+constexpr size_t diag_state_smem_bytes() {
+    using R = DiagRec<DK, DV>;
+    return 128 + sizeof(float) * ((size_t)DK * 64 + 2 * (R::kHead + R::kSlice) + CD * 64) + 64;
+}
+
+template <int DK, int DV, typename TOut>
+__global__ void __launch_bounds__(NT, 1) diag_state_kernel(FwdArgs a, const float* __restrict__ recs) {
+    using R = DiagRec<DK, DV>;
+    constexpr uint32_t kHeadBytes = R::kHead * 4, kSliceBytes = R::kSlice * 4;
+    constexpr int kStage = R::kHead + R::kSlice;
+    static_assert(kHeadBytes % 16 == 0 && kSliceBytes % 16 == 0, "bulk copy sizes");
+    extern __shared__ uint8_t smem_raw[];
+    float* sm = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+    float* Ss = sm;                     // DK x 64 state slice
+    float* stg = Ss + DK * 64;          // 2 stages: [record head | UP slice]
+    float* Us = stg + 2 * kStage;       // CD x 64
+    uint64_t* full = reinterpret_cast<uint64_t*>(Us + CD * 64);
+
+    const int tid = threadIdx.x;
+    const int sl = blockIdx.x, v0 = sl * 64, h = blockIdx.y, b = blockIdx.z;
+    const int T = a.T, H = a.H;
+    const int NC = (T + CD - 1) / CD;
+    const size_t head = (size_t)b * H + h;
+    const size_t sbase = head * DK * DV;
+    const float* hrec = recs + head * NC * R::kFloats;
+    TOut* o = static_cast<TOut*>(a.o);
+
+    auto request = [&](int c, int st) {
+        const uint32_t bar = smem_u32(&full[st]);
+        const float* r = hrec + (size_t)c * R::kFloats;
+        mbar_expect_tx(bar, kHeadBytes + kSliceBytes);
+        bulk_load(smem_u32(stg + st * kStage), r, kHeadBytes, bar);
+        bulk_load(smem_u32(stg + st * kStage + R::kHead), r + R::UP + sl * R::kSlice, kSliceBytes, bar);
+    };
+    if (tid == 0) {
+        mbar_init(smem_u32(&full[0]), 1);
+        mbar_init(smem_u32(&full[1]), 1);
+        fence_mbar_init();
+        for (int c = 0; c < min(NC, 2); ++c) request(c, c);
+    }
+    for (int x = tid; x < DK * 64; x += NT) {
+        const int r = x >> 6, c = x & 63;
+        Ss[x] = a.S0 ? a.S0[sbase + (size_t)r * DV + v0 + c] : 0.f;
+    }
+    __syncthreads();
+
+    const int i = tid >> 4, cx = 4 * (tid & 15);  // row (token) and the four columns of this thread
+    bool ok = true;
+    for (int ci = 0; ci < NC; ++ci) {
+        const int st = ci & 1;
+        const int t0 = ci * CD, n = min(CD, T - t0);
+        const bool got = mbar_wait_bounded(smem_u32(&full[st]), (ci >> 1) & 1, 2000000000ull);
+        if (__syncthreads_or(!got)) { ok = false; break; }
+        const float* rs = stg + st * kStage;
+        if (a.S_chunks) {
+            float* dst = a.S_chunks + (head * NC + ci) * DK * DV;
+            for (int x = tid; x < DK * 16; x += NT) {
+                const int r = x >> 4, c4 = 4 * (x & 15);
+                *reinterpret_cast<float4*>(dst + (size_t)r * DV + v0 + c4) =
+                    *reinterpret_cast<const float4*>(Ss + r * 64 + c4);
+            }
+        }
+        // U = UP - W S and O1 = QG S (row i, columns cx .. cx + 3)
+        float4 u = *reinterpret_cast<const float4*>(rs + R::kHead + i * 64 + cx);
+        float4 oo = make_float4(0.f, 0.f, 0.f, 0.f);
+        {
+            const float* wr = rs + R::W + i * DK;
+            const float* qr = rs + R::QG + i * DK;
+#pragma unroll 8
+            for (int d = 0; d < DK; ++d) {
+                const float w = wr[d], q = qr[d];
+                const float4 s4 = *reinterpret_cast<const float4*>(Ss + d * 64 + cx);
+                u.x = fmaf(-w, s4.x, u.x); u.y = fmaf(-w, s4.y, u.y);
+                u.z = fmaf(-w, s4.z, u.z); u.w = fmaf(-w, s4.w, u.w);
+                oo.x = fmaf(q, s4.x, oo.x); oo.y = fmaf(q, s4.y, oo.y);
+                oo.z = fmaf(q, s4.z, oo.z); oo.w = fmaf(q, s4.w, oo.w);
+            }
+        }
+        *reinterpret_cast<float4*>(Us + i * 64 + cx) = u;
+        __syncthreads();
+        // O = O1 + P U (row i)
+        if (o != nullptr) {
+            const float* pr = rs + R::P + i * CD;
+#pragma unroll
+            for (int t = 0; t < CD; ++t) {
+                const float p = pr[t];
+                const float4 ut = *reinterpret_cast<const float4*>(Us + t * 64 + cx);
+                oo.x = fmaf(p, ut.x, oo.x); oo.y = fmaf(p, ut.y, oo.y);
+                oo.z = fmaf(p, ut.z, oo.z); oo.w = fmaf(p, ut.w, oo.w);
+            }
+            if (i < n) {
+                TOut* orow = o + tok_index(b, t0 + i, h, T, H) * DV + v0 + cx;
+                orow[0] = from_f32<TOut>(oo.x);
+                orow[1] = from_f32<TOut>(oo.y);
+                orow[2] = from_f32<TOut>(oo.z);
+                orow[3] = from_f32<TOut>(oo.w);
+            }
+        }
+        // S' = Diag(GC) S + KD^T U: rows i + 16 m of the state, columns cx .. cx + 3
+        {
+            float4 acc[DK / 16];
+#pragma unroll
+            for (int m = 0; m < DK / 16; ++m) {
+                const int r = i + 16 * m;
+                const float gcr = rs[R::GC + r];
+                const float4 s4 = *reinterpret_cast<const float4*>(Ss + r * 64 + cx);
+                acc[m] = make_float4(gcr * s4.x, gcr * s4.y, gcr * s4.z, gcr * s4.w);
+            }
+#pragma unroll
+            for (int t = 0; t < CD; ++t) {
+                const float4 ut = *reinterpret_cast<const float4*>(Us + t * 64 + cx);
+                const float* kd = rs + R::KD + t * DK + i;
+#pragma unroll
+                for (int m = 0; m < DK / 16; ++m) {
+                    const float w = kd[16 * m];
+                    acc[m].x = fmaf(w, ut.x, acc[m].x); acc[m].y = fmaf(w, ut.y, acc[m].y);
+                    acc[m].z = fmaf(w, ut.z, acc[m].z); acc[m].w = fmaf(w, ut.w, acc[m].w);
+                }
+            }
+#pragma unroll
+            for (int m = 0; m < DK / 16; ++m) *reinterpret_cast<float4*>(Ss + (i + 16 * m) * 64 + cx) = acc[m];
+        }
+        __syncthreads();  // the stage and Us are read: refill the stage
+        if (tid == 0 && ci + 2 < NC) request(ci + 2, st);
+    }
+    if (!ok && tid == 0) atomicOr(&g_diag_error, 1u);
+    __syncthreads();
+    if (ok && a.S_T) {
+        for (int x = tid; x < DK * 16; x += NT) {
+            const int r = x >> 4, c4 = 4 * (x & 15);
+            *reinterpret_cast<float4*>(a.S_T + sbase + (size_t)r * DV + v0 + c4) =
+                *reinterpret_cast<const float4*>(Ss + r * 64 + c4);
+        }
+    }
+}
+
+template <int DK, int DV, typename Tin, typename TOut>
+cudaError_t diag_split_launch(const FwdArgs& a, void* ws, cudaStream_t st) {
+    const size_t ps = diag_prep_smem_bytes<DK, DV>(), ss = diag_state_smem_bytes<DK, DV>();
+    cudaError_t e = cudaFuncSetAttribute(diag_prep_kernel<DK, DV, Tin>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)ps);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(diag_state_kernel<DK, DV, TOut>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ss);
+    if (e != cudaSuccess) return e;
+    const int NC = (a.T + CD - 1) / CD;
+    float* recs = static_cast<float*>(ws);
+    diag_prep_kernel<DK, DV, Tin><<<dim3(NC, a.B * a.H), NT, ps, st>>>(a, recs);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    diag_state_kernel<DK, DV, TOut><<<dim3(DV / 64, a.H, a.B), NT, ss, st>>>(a, recs);
+    return cudaGetLastError();
+}
+
+template <int DK, typename Tin, typename TOut>
+cudaError_t diag_split_dv(const FwdArgs& a, void* ws, cudaStream_t st) {
+    return a.Dv == 128 ? diag_split_launch<DK, 128, Tin, TOut>(a, ws, st) : diag_split_launch<DK, 64, Tin, TOut>(a, ws, st);
+}
+template <int DK, typename Tin>
+cudaError_t diag_split_o(const FwdArgs& a, void* ws, cudaStream_t st) {
+    return a.out_bf16 ? diag_split_dv<DK, Tin, __nv_bfloat16>(a, ws, st) : diag_split_dv<DK, Tin, float>(a, ws, st);
+}
+
 template <int DK, typename Tin, typename TOut>
 cudaError_t diag_fwd_launch(const FwdArgs& a, cudaStream_t st) {
     const size_t smem = diag_fwd_smem_bytes<DK>();
@@ -748,15 +1036,37 @@ cudaError_t diag_bwd_o(const BwdArgs& a, const FwdArgs& f, cudaStream_t st) {
 
 int diag_chunk_len() { return CD; }
 
-cudaError_t launch_chunk_fwd_diag(const FwdArgs& a, cudaStream_t st) {
+size_t diag_fwd_workspace(int B, int T, int H, int Dk, int Dv) {
+    const size_t NC = ((size_t)T + CD - 1) / CD;
+    const size_t rec = Dk == 128 ? (Dv == 128 ? DiagRec<128, 128>::kFloats : DiagRec<128, 64>::kFloats)
+                                 : (Dv == 128 ? DiagRec<64, 128>::kFloats : DiagRec<64, 64>::kFloats);
+    return (size_t)B * H * NC * rec * sizeof(float);
+}
+
+cudaError_t launch_chunk_fwd_diag(const FwdArgs& a, void* ws, size_t ws_bytes, cudaStream_t st) {
+    if (ws != nullptr && ws_bytes >= diag_fwd_workspace(a.B, a.T, a.H, a.Dk, a.Dv)) {
+        if (a.bf16) return a.Dk == 128 ? diag_split_o<128, __nv_bfloat16>(a, ws, st) : diag_split_o<64, __nv_bfloat16>(a, ws, st);
+        return a.Dk == 128 ? diag_split_o<128, float>(a, ws, st) : diag_split_o<64, float>(a, ws, st);
+    }
     if (a.bf16) return a.Dk == 128 ? diag_fwd_o<128, __nv_bfloat16>(a, st) : diag_fwd_o<64, __nv_bfloat16>(a, st);
     return a.Dk == 128 ? diag_fwd_o<128, float>(a, st) : diag_fwd_o<64, float>(a, st);
 }
 
-// The backward: the forward kernel first writes every 16-token chunk's starting state into
-// a.S_chunks (the workspace), then the reverse pass, the finishing kernel and the dg scan.
-// The accumulators in `a` must be zeroed before this is called.
-cudaError_t launch_chunk_bwd_diag(const BwdArgs& a, const float* S0, cudaStream_t st) {
+cudaError_t diag_take_error(cudaStream_t st, unsigned int* flag) {
+    cudaError_t e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return e;
+    e = cudaMemcpyFromSymbol(flag, g_diag_error, sizeof(unsigned int));
+    if (e != cudaSuccess) return e;
+    const unsigned int zero = 0;
+    return cudaMemcpyToSymbol(g_diag_error, &zero, sizeof(unsigned int));
+}
+
+// The backward: the forward first writes every 16-token chunk's starting state into
+// a.S_chunks (the workspace; the split forward's records go to rec_ws when it is large enough),
+// then the reverse pass, the finishing kernel and the dg scan.  The accumulators in `a` must be
+// zeroed before this is called.
+cudaError_t launch_chunk_bwd_diag(const BwdArgs& a, const float* S0, void* rec_ws, size_t rec_bytes,
+                                  cudaStream_t st) {
     FwdArgs f{};
     f.q = a.q;
     f.k = a.k;
@@ -775,7 +1085,7 @@ cudaError_t launch_chunk_bwd_diag(const BwdArgs& a, const float* S0, cudaStream_
     f.Dv = a.Dv;
     f.bf16 = a.bf16;
     f.out_bf16 = false;
-    cudaError_t e = launch_chunk_fwd_diag(f, st);
+    cudaError_t e = launch_chunk_fwd_diag(f, rec_ws, rec_bytes, st);
     if (e != cudaSuccess) return e;
     if (a.bf16) return a.Dk == 128 ? diag_bwd_o<128, __nv_bfloat16>(a, f, st) : diag_bwd_o<64, __nv_bfloat16>(a, f, st);
     return a.Dk == 128 ? diag_bwd_o<128, float>(a, f, st) : diag_bwd_o<64, float>(a, f, st);

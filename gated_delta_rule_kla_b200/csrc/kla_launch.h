@@ -123,9 +123,15 @@ cudaError_t gates_take_error(cudaStream_t st, unsigned int* flag);
 // chunks of diag_chunk_len() tokens; S_chunks of the forward (optional) and of the backward
 // (required: the workspace region the backward launcher fills first) are per such chunk.  The
 // backward's acc_dG is [B, T, H, Dk]; every accumulator must be zeroed before the launch.
+// With at least diag_fwd_workspace() bytes in ws the forward runs split: a chunk-parallel
+// preparation kernel writes fp32 records there, then a sequential state pass reads them;
+// otherwise one kernel per (head, 64 value columns) does everything.
 int diag_chunk_len();
-cudaError_t launch_chunk_fwd_diag(const FwdArgs& a, cudaStream_t st);
-cudaError_t launch_chunk_bwd_diag(const BwdArgs& a, const float* S0, cudaStream_t st);
+size_t diag_fwd_workspace(int B, int T, int H, int Dk, int Dv);
+cudaError_t launch_chunk_fwd_diag(const FwdArgs& a, void* ws, size_t ws_bytes, cudaStream_t st);
+cudaError_t launch_chunk_bwd_diag(const BwdArgs& a, const float* S0, void* rec_ws, size_t rec_bytes,
+                                  cudaStream_t st);
+cudaError_t diag_take_error(cudaStream_t st, unsigned int* flag);
 cudaError_t launch_chunk_fwd_simt(const FwdArgs& a, cudaStream_t st);
 cudaError_t launch_chunk_bwd_simt(const BwdArgs& a, cudaStream_t st);
 // Tensor-core (tcgen05) forward for bf16 inputs with Dk == Dv == 128.

@@ -229,20 +229,28 @@ kla_status kla_decode_step(const void *q, const void *k, const void *v, const fl
  * TMA-pipelined kernel of kla_decode_step with the per-channel decay folded in.
  *
  * kla_chunk_fwd_diag   -- prefill: o ([B,T,H,Dv] of out_dtype, or NULL) and S_T ([B,H,Dk,Dv]
- *                         fp32, or NULL; may alias S0) from S0 (NULL = zero state).  No workspace.
+ *                         fp32, or NULL; may alias S0) from S0 (NULL = zero state).  ws (device,
+ *                         16-byte aligned, caller-owned, contents need not be initialised) of at
+ *                         least kla_chunk_fwd_diag_workspace() bytes selects the split path: a
+ *                         chunk-parallel kernel stores every 16-token chunk's state-independent
+ *                         operands there (about 34 KiB per chunk and head at Dk = Dv = 128),
+ *                         then a sequential state pass reads them; with NULL or less, one kernel
+ *                         per (head, 64 value columns) does both (slower, no workspace).
  * kla_chunk_bwd_diag   -- gradients of <o, dO> + <S_T, dS_T> with respect to q, k, v, eta, g
  *                         (dg per channel, [B,T,H,Dk]) and S0; dS_T may be NULL.  ws: device,
  *                         16-byte aligned, caller-owned, at least kla_chunk_bwd_diag_workspace()
- *                         bytes (the state at every internal chunk start plus fp32
- *                         accumulators, cleared by the call), else KLA_ERR_WORKSPACE.  At a key
+ *                         bytes (the state at every internal chunk start, fp32 accumulators
+ *                         cleared by the call, and the split forward's records), else
+ *                         KLA_ERR_WORKSPACE.  At a key
  *                         of zero norm dk is exact, as for kla_chunk_bwd.
  * kla_decode_step_diag -- one token for every (b, h); S [B,H,Dk,Dv] updated in place.
  * Returns KLA_OK or an error status; on error nothing is launched.
  */
+size_t kla_chunk_fwd_diag_workspace(int B, int T, int H, int Dk, int Dv, int chunk, int dtype);
 kla_status kla_chunk_fwd_diag(const void *q, const void *k, const void *v, const float *eta,
                               const float *g, float eps, const float *S0, void *o, float *S_T,
                               int B, int T, int H, int Dk, int Dv, int chunk, int dtype,
-                              int out_dtype, void *stream);
+                              int out_dtype, void *ws, size_t ws_bytes, void *stream);
 size_t kla_chunk_bwd_diag_workspace(int B, int T, int H, int Dk, int Dv, int chunk, int dtype);
 kla_status kla_chunk_bwd_diag(const void *q, const void *k, const void *v, const float *eta,
                               const float *g, float eps, const float *S0, const void *dO,

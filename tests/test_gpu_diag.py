@@ -82,6 +82,25 @@ def test_fwd_diag_matches_oracle(kla, oracle_mod, B, T, H, Dk, Dv, dtype, gate_l
     assert rel_err(ST, rST) <= TOL[dtype]
 
 
+@pytest.mark.parametrize("B,T,H,Dk,Dv,dtype,gate_lo", [(1, 50, 2, 64, 64, "f32", -0.5),
+                                                       (2, 77, 3, 128, 64, "f32", -4.0),
+                                                       (1, 200, 2, 128, 128, "bf16", -4.0),
+                                                       (1, 40, 2, 64, 128, "bf16", -0.5)])
+def test_fwd_diag_one_kernel_path_matches_oracle(kla, oracle_mod, B, T, H, Dk, Dv, dtype, gate_lo):
+    """Without a workspace the forward runs as one kernel per (head, 64 value columns); with one
+    (the default above) as the chunk-parallel preparation plus the state pass."""
+    w, inp = diag_inputs(B, T, H, Dk, Dv, dtype, seed=T + H + 1, gate_lo=gate_lo)
+    d = {k: (v.cuda() if v is not None else None) for k, v in inp.items()}
+    o1, S1 = kla.chunk_fwd_diag(d["q"], d["k"], d["v"], d["eta"], d["g"], w.eps, d["S0"], fused=True)
+    o2, S2 = kla.chunk_fwd_diag(d["q"], d["k"], d["v"], d["eta"], d["g"], w.eps, d["S0"])
+    torch.cuda.synchronize()
+    kla.check_device_error()
+    ro, rST = oracle_mod.forward_diag(*(np64(inp[k]) for k in ("q", "k", "v", "eta", "g")), w.eps, np64(inp["S0"]))
+    for o, ST in ((o1, S1), (o2, S2)):
+        assert rel_err(o, ro) <= TOL[dtype]
+        assert rel_err(ST, rST) <= TOL[dtype]
+
+
 def test_fwd_diag_uniform_channels_equal_scalar_gating(kla):
     """When every channel decays alike the diagonal-gated forward is the scalar-gated one
     (fp32, CUDA cores on both sides)."""

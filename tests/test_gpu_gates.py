@@ -39,6 +39,15 @@ def np64(t):
     return t.detach().double().cpu().numpy()
 
 
+def assert_qhat_one_rounding(qhat, ref, dtype):
+    """qhat is stored in the input dtype: each element within one unit in the last place of the
+    exact value (bf16 carries 8 significant bits, so one ulp is at most 2^-7 of the value; the
+    fp32 normalisation before the rounding adds ~1e-7; fp32 storage: 1e-6)."""
+    got = np64(qhat)
+    bound = (2.0 ** -7 if dtype == "bf16" else 1e-6) * np.abs(ref) + 1e-30
+    assert np.all(np.abs(got - ref) <= bound)
+
+
 CASES = [
     # N, D, H, Dk, dtype   (tensor cores: bf16, D % 64 == 0, H % 8 == 0)
     (300, 1024, 8, 128, "bf16"),   # tensor cores, ragged last tile
@@ -62,7 +71,7 @@ def test_gate_prologue_matches_oracle(kla, N, D, H, Dk, dtype):
     assert rel_err(eta, re) <= 1e-4 and rel_err(g, rg) <= 1e-4
     assert torch.equal(eta, eta2) and torch.equal(g, g2)
     assert float(g.max()) <= 0.0 and float(eta.min()) >= 0.0 and float(eta.max()) <= 1.0
-    assert rel_err(qhat, og.normalize_q(np64(inp["q"]))) <= (2e-2 if dtype == "bf16" else 1e-4)
+    assert_qhat_one_rounding(qhat, og.normalize_q(np64(inp["q"])), dtype)
 
 
 def test_gate_prologue_zero_query_and_empty(kla):
@@ -101,8 +110,11 @@ def test_gate_prologue_bwd_matches_oracle(kla, N, D, H, Dk, dtype):
 
 
 def test_prologue_feeds_the_recurrence_end_to_end(kla, oracle_mod):
-    """x, W, bias and raw q -> (eta, g, qhat) -> kla_chunk_fwd (split tensor-core path) matches
-    the oracle's gates -> normalise -> token recurrence, i.e. Algorithm 1 with its readout."""
+    """x, W, bias and raw q -> (eta, g, qhat) -> kla_chunk_fwd (split tensor-core path) against
+    the oracle's gates -> token recurrence, i.e. Algorithm 1 with its normalised readout.  qhat
+    enters the recurrence in bf16 (the dtype of k and v), one rounding of the exact q/||q||: the
+    oracle is fed that same rounded qhat (the rounding itself is checked elementwise), and its
+    own eta and g from the exact inputs."""
     from oracle import gates as og
     B, T, H, D, Dk = 2, 150, 8, 1024, 128
     gi = make_gate_inputs(B * T, D, H, Dk, "bf16", seed=21)
@@ -114,8 +126,8 @@ def test_prologue_feeds_the_recurrence_end_to_end(kla, oracle_mod):
     o, ST = kla.chunk_fwd(qhat, rec["k"].cuda(), rec["v"].cuda(), eta, g, w.eps, rec["S0"].cuda())
     torch.cuda.synchronize()
     re, rg = og.gates(np64(gi["x"]), np64(gi["W"]), np64(gi["bias"]), H)
-    rq = og.normalize_q(np64(gi["q"])).reshape(B, T, H, Dk)
-    ro, rST = oracle_mod.forward(rq, np64(rec["k"]), np64(rec["v"]), re.reshape(B, T, H), rg.reshape(B, T, H),
-                                 w.eps, np64(rec["S0"]))
+    assert_qhat_one_rounding(qhat, og.normalize_q(np64(gi["q"])).reshape(B, T, H, Dk), "bf16")
+    ro, rST = oracle_mod.forward(np64(qhat), np64(rec["k"]), np64(rec["v"]), re.reshape(B, T, H),
+                                 rg.reshape(B, T, H), w.eps, np64(rec["S0"]))
     assert rel_err(o, ro) <= 2e-2
     assert rel_err(ST, rST) <= 2e-2
