@@ -531,10 +531,7 @@ static kla_status gate_checks(int N, int D, int H, int Dk, int dtype, bool with_
     if (H > 64) return fail(KLA_ERR_UNSUPPORTED, "at most 64 heads (got H=%d)", H);
     if (dtype != KLA_F32 && dtype != KLA_BF16)
         return fail(KLA_ERR_UNSUPPORTED, "dtype must be KLA_F32 or KLA_BF16 (got %d)", dtype);
-    if (dtype == KLA_BF16 && D % 8 != 0)
-        return fail(KLA_ERR_UNSUPPORTED, "bf16 rows must be 16-byte multiples: D %% 8 == 0 (got D=%d)", D);
-    if (dtype == KLA_F32 && D % 4 != 0)
-        return fail(KLA_ERR_UNSUPPORTED, "fp32 rows must be 16-byte multiples: D %% 4 == 0 (got D=%d)", D);
+    if (D % 8 != 0) return fail(KLA_ERR_UNSUPPORTED, "D must be a multiple of 8 (got D=%d)", D);
     if (with_q && Dk != 64 && Dk != 128) return fail(KLA_ERR_UNSUPPORTED, "Dk must be 64 or 128 (got %d)", Dk);
     return KLA_OK;
 }

@@ -148,6 +148,18 @@ __device__ __forceinline__ void chunk_grams(const float* Ks, const float* Qs, co
     }
 }
 
+// Per-(head, 16-token chunk) record of the split path (floats; see the split forward below).
+template <int DK, int DV>
+struct DiagRec {
+    static constexpr int kHead = 3 * CD * DK + CD * CD + DK;  // W, QG, KD, P, GC (floats)
+    static constexpr int kSlice = CD * 64;                     // one 64-column slice of UP
+    static constexpr int kExtra = 2 * CD * CD + CD * DK;       // A, T, G (backward only)
+    static constexpr int kFloats = kHead + (DV / 64) * kSlice + kExtra;  // record stride
+    static constexpr int W = 0, QG = CD * DK, KD = 2 * CD * DK, P = 3 * CD * DK, GC = 3 * CD * DK + CD * CD,
+                         UP = kHead, XA = kHead + (DV / 64) * kSlice, XT = XA + CD * CD, XG = XT + CD * CD;
+    static_assert((kHead * 4) % 16 == 0 && (kFloats * 4) % 16 == 0 && (XA * 4) % 16 == 0, "bulk copy alignment");
+};
+
 // ------------------------------------------------------------------------------------
 // Forward: grid (Dv / NV, H, B); S_chunks (optional) receives the state at the start of every
 // 16-token chunk, [B, H, ceil(T/16), Dk, Dv] (the backward's input).
@@ -327,9 +339,12 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_diag_kernel(FwdArgs a) {
 
 // ------------------------------------------------------------------------------------
 // Backward.  Per chunk (newest first) with incoming state S and lambda = dS' (gradient of the
-// outgoing state), Gam_i = exp(G_i), Del_j = exp(G_last - G_j) (vectors over channels):
-//   dU  = P^T dO + (Khat o Del) lambda,   dR = (I + L)^{-T} dU (back substitution)
-//   dS  = Diag(Gam_last) lambda + (Q o Gam)^T dO - (Diag(b) (Khat o Gam))^T dR     (carried on)
+// outgoing state), Gam_i = exp(G_i), Del_j = exp(G_last - G_j) (vectors over channels), and
+// the forward preparation's record of the chunk (W, QG = Q o Gam, KD = Khat o Del, P, GC, UP,
+// A, T, G):
+//   U   = UP - W S + Diag(u - c) V     (u = c except at a zero-norm key, where u = beta: see below)
+//   dU  = P^T dO + KD lambda,   dR = T^T dU
+//   dS  = Diag(GC) lambda + QG^T dO - W^T dU                                     (carried on)
 //   dv  = Diag(c) dR,  dc_i = dR_i . v_i
 //   Y   = dO U^T (lower),  D = -dR U^T (strictly lower)
 //   Z1 = dO S^T, Z2 = dR S^T, Z3 = U lambda^T                     (rows: tokens, columns: channels)
@@ -340,315 +355,362 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_diag_kernel(FwdArgs a) {
 //   db_i    = sum_{j<i} D_ij A_ij - (khat_i o Gam_i) . Z2_i
 //   dG_i    = Gam_i o q_i o Z1_i + q_i o F1_i - b_i Gam_i o khat_i o Z2_i - khat_i o F2_i
 //             + b_i khat_i o F3_i - khat_i o F4_i - Del_i o khat_i o Z3_i
-//   dG_last += sum_j Del_j o khat_j o Z3_j + Gam_last o rowsum(lambda o S)
+//   dG_last += sum_j Del_j o khat_j o Z3_j + GC o rowsum(lambda o S)
+// (W^T dU = (T Diag(b)(Khat o Gam))^T dU = (Diag(b)(Khat o Gam))^T dR.)  At a key of zero norm
+// U's row takes u = beta v: that row only ever meets khat = 0, except in row i of dkhat, which
+// then is the exact dk = beta Gbar_i v_i.  One CTA per (head, 64 value columns); the columns'
+// partial sums of dq, dkhat, dG, db and dc go out by vector reductions into fp32 accumulators.
 // ------------------------------------------------------------------------------------
-template <int DK>
+constexpr int BLD = 68;  // row stride of the [rows][64] fp32 tiles (16-byte rows, 2-way banks)
+
+template <int DK, int DV>
 constexpr size_t diag_bwd_smem_bytes() {
-    constexpr int NV = 32;
-    return sizeof(float) * (2 * CD * (DK + 1) + CD * DK + NP * DK + 2 * DK * (NV + 1) + 4 * CD * (NV + 1) +
-                            5 * CD * (CD + 1) + 4 * CD + 8 + DK + CD * DK);
+    using R = DiagRec<DK, DV>;
+    return 128 + sizeof(float) * ((size_t)2 * DK * BLD + NP * DK + R::kHead + R::kExtra + CD * 64 +
+                                  2 * CD * (DK + 1) + 5 * CD * BLD + 2 * CD * (CD + 1) + DK + 4 * CD) +
+           NP * 2 + 32;
 }
 
-template <int DK, typename Tin, typename TOut>
-__global__ void __launch_bounds__(NT, 1) chunk_bwd_diag_kernel(BwdArgs a, FwdArgs f) {
-    constexpr int NV = 32;
-    constexpr int LDK = DK + 1, LDV = NV + 1, LDC = CD + 1;
-    constexpr int TMK = DK / 16;
-    constexpr int EPT = CD * DK / NT;  // (token, channel) elements per thread
-    extern __shared__ float sm[];
-    float* Ks = sm;               // CD x LDK  unit keys
-    float* Qs = Ks + CD * LDK;    // CD x LDK
-    float* Gs = Qs + CD * LDK;    // CD x DK   log-decay prefix
-    float* Es = Gs + CD * DK;     // NP x DK   E_ij per channel
-    float* Ss = Es + NP * DK;     // DK x LDV  incoming state slice
-    float* dSs = Ss + DK * LDV;   // DK x LDV  gradient of the outgoing state slice
-    float* Us = dSs + DK * LDV;   // CD x LDV  cV -> R -> U
-    float* dRs = Us + CD * LDV;   // CD x LDV  dU -> dR
-    float* dOs = dRs + CD * LDV;  // CD x LDV
-    float* Xs = dOs + CD * LDV;   // CD x LDV  (Khat o Gam) S, then (Khat o Del) lambda
-    float* Am = Xs + CD * LDV;    // CD x LDC  A (strictly lower, without b)
-    float* Lm = Am + CD * LDC;    // CD x LDC  L = Diag(b) A
-    float* Pm = Lm + CD * LDC;    // CD x LDC
-    float* Ym = Pm + CD * LDC;    // CD x LDC  Y = dO U^T (lower)
-    float* Dm = Ym + CD * LDC;    // CD x LDC  D = -dR U^T (strictly lower)
-    float* bs = Dm + CD * LDC;
+__device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d) {
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d)
+                 : "memory");
+}
+
+template <int DK, int DV, typename Tin, typename TOut>
+__global__ void __launch_bounds__(NT, 1) diag_bwd_kernel(BwdArgs a, FwdArgs f, const float* __restrict__ recs) {
+    using R = DiagRec<DK, DV>;
+    constexpr int LDK = DK + 1, LDC = CD + 1;
+    constexpr int EPT = CD * DK / NT;  // (token, channel) elements per thread: tx + 16 u
+    extern __shared__ uint8_t smem_raw[];
+    float* sm = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+    float* Ss = sm;                      // DK x BLD  incoming state slice
+    float* Ls = Ss + DK * BLD;           // DK x BLD  lambda slice
+    float* Es = Ls + DK * BLD;           // NP x DK   E_ij, then the results [3][CD][DK]
+    float* Rh = Es + NP * DK;            // record head: W, QG, KD, P, GC
+    float* Rx = Rh + R::kHead;           // record extras: A, T, G
+    float* UPs = Rx + R::kExtra;         // CD x 64   UP slice
+    float* Kh = UPs + CD * 64;           // CD x LDK  unit keys
+    float* Qs = Kh + CD * LDK;           // CD x LDK
+    float* Us = Qs + CD * LDK;           // CD x BLD
+    float* dUs = Us + CD * BLD;          // CD x BLD
+    float* dRs = dUs + CD * BLD;         // CD x BLD
+    float* dOs = dRs + CD * BLD;         // CD x BLD
+    float* Vs = dOs + CD * BLD;          // CD x BLD
+    float* Ym = Vs + CD * BLD;           // CD x LDC
+    float* Dm = Ym + CD * LDC;           // CD x LDC
+    float* lsS = Dm + CD * LDC;          // DK
+    float* bs = lsS + DK;
     float* cs = bs + CD;
     float* us = cs + CD;
     float* dbs = us + CD;
-    float* red = dbs + CD;        // 8
-    float* lsS = red + 8;         // DK: row sums of lambda o S over this slice
-    float* xs = lsS + DK;         // CD x DK: per-token terms of the last token's dG
+    uint8_t* pij = reinterpret_cast<uint8_t*>(dbs + CD);  // NP x (i, j)
+    uint64_t* bars = reinterpret_cast<uint64_t*>(((reinterpret_cast<uintptr_t>(pij + 2 * NP)) + 15) & ~uintptr_t(15));
 
-    const int v0 = blockIdx.x * NV, h = blockIdx.y, b = blockIdx.z;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int tx = tid & 15, ty = tid >> 4;
-    const int T = a.T, H = a.H, Dv = a.Dv;
+    const int tid = threadIdx.x, lane = tid & 31;
+    const int sl = blockIdx.x, v0 = sl * 64, h = blockIdx.y, b = blockIdx.z;
+    const int T = a.T, H = a.H;
+    const int NC = (T + CD - 1) / CD;
+    const size_t head = (size_t)b * H + h;
+    const size_t sbase = head * DK * DV;
+    const float* hrec = recs + head * NC * R::kFloats;
     const Tin* v = static_cast<const Tin*>(a.v);
     const Tin* dO = static_cast<const Tin*>(a.dO);
     TOut* dv = static_cast<TOut*>(a.dv);
-    const size_t sbase = ((size_t)b * H + h) * DK * Dv;
-    const int NC = (T + CD - 1) / CD;
+    const uint32_t bar_r = smem_u32(&bars[0]), bar_s = smem_u32(&bars[1]);
 
-    for (int x = tid; x < DK * NV; x += NT) {
-        const int r = x / NV, c = x % NV;
-        dSs[r * LDV + c] = a.dS_T ? a.dS_T[sbase + (size_t)r * Dv + v0 + c] : 0.f;
+    // the chunk's record parts (head, its UP slice, extras) and the incoming state's slice rows
+    auto request_rec = [&](int c) {
+        const float* r = hrec + (size_t)c * R::kFloats;
+        mbar_expect_tx(bar_r, (R::kHead + CD * 64 + R::kExtra) * 4);
+        bulk_load(smem_u32(Rh), r, R::kHead * 4, bar_r);
+        bulk_load(smem_u32(UPs), r + R::UP + sl * R::kSlice, CD * 64 * 4, bar_r);
+        bulk_load(smem_u32(Rx), r + R::XA, R::kExtra * 4, bar_r);
+    };
+    auto request_state = [&](int c) {
+        const float* src = a.S_chunks + (head * NC + c) * DK * DV + v0;
+        mbar_expect_tx(bar_s, DK * 64 * 4);
+        for (int r = 0; r < DK; ++r) bulk_load(smem_u32(Ss + r * BLD), src + (size_t)r * DV, 256, bar_s);
+    };
+    if (tid == 0) {
+        mbar_init(bar_r, 1);
+        mbar_init(bar_s, 1);
+        fence_mbar_init();
+        if (NC > 0) {
+            request_rec(NC - 1);
+            request_state(NC - 1);
+        }
+    }
+    if (tid < NP) {
+        int i = 0;
+        while ((i + 1) * (i + 2) / 2 <= tid) ++i;
+        pij[2 * tid] = (uint8_t)i;
+        pij[2 * tid + 1] = (uint8_t)(tid - i * (i + 1) / 2);
+    }
+    for (int x = tid; x < DK * 64; x += NT) {
+        const int r = x >> 6, c = x & 63;
+        Ls[r * BLD + c] = a.dS_T ? a.dS_T[sbase + (size_t)r * DV + v0 + c] : 0.f;
     }
 
+    const int i = tid >> 4, tx = tid & 15, cx = 4 * tx;  // token row and this thread's columns
+    bool ok = true;
     for (int ci = NC - 1; ci >= 0; --ci) {
-        const int t0 = ci * CD;
-        const int n = min(CD, T - t0);
+        const int t0 = ci * CD, n = min(CD, T - t0);
+        const int ph = (NC - 1 - ci) & 1;
         __syncthreads();
-        load_rows<DK, Tin>(f, b, h, t0, n, Ks, Qs, Gs, bs, cs, us);
+        // rows of the chunk: unit keys, queries and coefficients (u: the U coefficient); v, dO slices
         {
-            const float* src = a.S_chunks + (((size_t)b * H + h) * NC + ci) * DK * Dv;
-            for (int x = tid; x < DK * NV; x += NT) {
-                const int r = x / NV, c = x % NV;
-                Ss[r * LDV + c] = src[(size_t)r * Dv + v0 + c];
-            }
+            float* gdummy = Es;  // load_rows also stages the raw decays: the E area is free here
+            load_rows<DK, Tin>(f, b, h, t0, n, Kh, Qs, gdummy, bs, cs, us);
         }
-        for (int x = tid; x < CD * NV; x += NT) {  // one column per lane
-            const int i = x / NV, j = x % NV;
-            float uv = 0.f, dov = 0.f;
-            if (i < n) {
-                const size_t ti = tok_index(b, t0 + i, h, T, H);
-                uv = to_f32(v[ti * Dv + v0 + j]);
-                dov = to_f32(dO[ti * Dv + v0 + j]);
+        for (int x = tid; x < CD * 16; x += NT) {
+            const int r = x >> 4, c4 = 4 * (x & 15);
+            float vv[4] = {0.f, 0.f, 0.f, 0.f}, oo[4] = {0.f, 0.f, 0.f, 0.f};
+            if (r < n) {
+                const size_t ti = tok_index(b, t0 + r, h, T, H) * DV + v0 + c4;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    vv[e] = to_f32(v[ti + e]);
+                    oo[e] = to_f32(dO[ti + e]);
+                }
             }
-            Us[i * LDV + j] = uv;  // scaled by its coefficient below
-            dOs[i * LDV + j] = dov;
+            *reinterpret_cast<float4*>(Vs + r * BLD + c4) = make_float4(vv[0], vv[1], vv[2], vv[3]);
+            *reinterpret_cast<float4*>(dOs + r * BLD + c4) = make_float4(oo[0], oo[1], oo[2], oo[3]);
         }
         if (tid < CD) dbs[tid] = 0.f;
-        __syncthreads();
-        cumsum_rows<DK>(Gs);
-        for (int x = tid; x < CD * NV; x += NT) {
-            const int i = x / NV, j = x % NV;
-            Us[i * LDV + j] *= us[i];
+        const bool got = mbar_wait_bounded(bar_r, ph, 2000000000ull) && mbar_wait_bounded(bar_s, ph, 2000000000ull);
+        if (__syncthreads_or(!got)) { ok = false; break; }
+        const float* Gs = Rx + (R::XG - R::XA);
+        const float* Am = Rx;
+        const float* Tm = Rx + CD * CD;
+        // ---- E_ij = exp(G_i - G_j) per channel, j <= i
+        for (int x = tid; x < NP * DK; x += NT) {
+            const int p = x / DK, c = x % DK;
+            Es[x] = __expf(Gs[pij[2 * p] * DK + c] - Gs[pij[2 * p + 1] * DK + c]);
         }
-        __syncthreads();
-        chunk_grams<DK>(Ks, Qs, Gs, Am, Pm, Es);
-        // X = (Khat o Gam) S and the lambda o S row sums
+        // ---- U = UP - W S + (u - c) v  and  dU = P^T dO + KD lambda (row i, columns cx .. cx + 3)
         {
-            float ax[2] = {0.f, 0.f};
+            float4 u = *reinterpret_cast<const float4*>(UPs + i * 64 + cx);
+            float4 du = make_float4(0.f, 0.f, 0.f, 0.f);
+            const float* wr = Rh + R::W + i * DK;
+            const float* kr = Rh + R::KD + i * DK;
 #pragma unroll 4
             for (int d = 0; d < DK; ++d) {
-                const float w = Ks[ty * LDK + d] * __expf(Gs[ty * DK + d]);
-#pragma unroll
-                for (int nn = 0; nn < 2; ++nn) ax[nn] = fmaf(w, Ss[d * LDV + tx + 16 * nn], ax[nn]);
+                const float w = wr[d], kd = kr[d];
+                const float4 s4 = *reinterpret_cast<const float4*>(Ss + d * BLD + cx);
+                const float4 l4 = *reinterpret_cast<const float4*>(Ls + d * BLD + cx);
+                u.x = fmaf(-w, s4.x, u.x); u.y = fmaf(-w, s4.y, u.y); u.z = fmaf(-w, s4.z, u.z); u.w = fmaf(-w, s4.w, u.w);
+                du.x = fmaf(kd, l4.x, du.x); du.y = fmaf(kd, l4.y, du.y); du.z = fmaf(kd, l4.z, du.z); du.w = fmaf(kd, l4.w, du.w);
             }
+            const float* pc = Rh + R::P + i;  // column i of P
 #pragma unroll
-            for (int nn = 0; nn < 2; ++nn) Xs[ty * LDV + tx + 16 * nn] = ax[nn];
+            for (int t = 0; t < CD; ++t) {
+                const float pt = pc[t * CD];
+                const float4 o4 = *reinterpret_cast<const float4*>(dOs + t * BLD + cx);
+                du.x = fmaf(pt, o4.x, du.x); du.y = fmaf(pt, o4.y, du.y); du.z = fmaf(pt, o4.z, du.z); du.w = fmaf(pt, o4.w, du.w);
+            }
+            const float zc = us[i] - cs[i];
+            if (zc != 0.f) {
+                const float4 v4 = *reinterpret_cast<const float4*>(Vs + i * BLD + cx);
+                u.x = fmaf(zc, v4.x, u.x); u.y = fmaf(zc, v4.y, u.y); u.z = fmaf(zc, v4.z, u.z); u.w = fmaf(zc, v4.w, u.w);
+            }
+            *reinterpret_cast<float4*>(Us + i * BLD + cx) = u;
+            *reinterpret_cast<float4*>(dUs + i * BLD + cx) = du;
+        }
+        __syncthreads();
+        // ---- dR = T^T dU (row j = i here); lambda o S row sums
+        {
+            float4 r4 = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int t = i; t < CD; ++t) {
+                const float tt = Tm[t * CD + i];
+                const float4 d4 = *reinterpret_cast<const float4*>(dUs + t * BLD + cx);
+                r4.x = fmaf(tt, d4.x, r4.x); r4.y = fmaf(tt, d4.y, r4.y); r4.z = fmaf(tt, d4.z, r4.z); r4.w = fmaf(tt, d4.w, r4.w);
+            }
+            *reinterpret_cast<float4*>(dRs + i * BLD + cx) = r4;
         }
         if (tid < DK) {
             float p = 0.f;
 #pragma unroll 8
-            for (int c = 0; c < NV; ++c) p = fmaf(dSs[tid * LDV + c], Ss[tid * LDV + c], p);
+            for (int c = 0; c < 64; ++c) p = fmaf(Ls[tid * BLD + c], Ss[tid * BLD + c], p);
             lsS[tid] = p;
         }
         __syncthreads();
-        for (int x = tid; x < CD * NV; x += NT) {
-            const int i = x / NV, j = x % NV;
-            Us[i * LDV + j] -= bs[i] * Xs[i * LDV + j];
-        }
-        if (tid < CD * CD) {
-            const int i = tid / CD, j = tid % CD;
-            Lm[i * LDC + j] = bs[i] * Am[i * LDC + j];
-        }
-        __syncthreads();
-        // U = (I + L)^{-1} R, row by row
+        // ---- dv, dc; Y, D; the D o A part of db
         {
-            const int col = tid >> 3, part = tid & 7;
-            for (int i = 1; i < n; ++i) {
-                float s = 0.f;
-                for (int j = part; j < i; j += 8) s = fmaf(Lm[i * LDC + j], Us[j * LDV + col], s);
-                s += __shfl_xor_sync(0xffffffffu, s, 1);
-                s += __shfl_xor_sync(0xffffffffu, s, 2);
-                s += __shfl_xor_sync(0xffffffffu, s, 4);
-                if (part == 0) Us[i * LDV + col] -= s;
-                __syncthreads();
-            }
-        }
-        // dU = P^T dO + (Khat o Del) lambda
-        {
-            float ad[2] = {0.f, 0.f};
-            const int i = ty;
-#pragma unroll 4
-            for (int d = 0; d < DK; ++d) {
-                const float w = Ks[i * LDK + d] * __expf(Gs[(n - 1) * DK + d] - Gs[i * DK + d]);
+            const float4 r4 = *reinterpret_cast<const float4*>(dRs + i * BLD + cx);
+            const float4 v4 = *reinterpret_cast<const float4*>(Vs + i * BLD + cx);
+            float dcp = r4.x * v4.x + r4.y * v4.y + r4.z * v4.z + r4.w * v4.w;
 #pragma unroll
-                for (int nn = 0; nn < 2; ++nn) ad[nn] = fmaf(w, dSs[d * LDV + tx + 16 * nn], ad[nn]);
+            for (int o = 1; o < 16; o <<= 1) dcp += __shfl_xor_sync(0xffffffffu, dcp, o);
+            if (i < n) {
+                const size_t ti = tok_index(b, t0 + i, h, T, H);
+                const float ci_ = cs[i];
+                TOut* dvr = dv + ti * DV + v0 + cx;
+                dvr[0] = from_f32<TOut>(ci_ * r4.x);
+                dvr[1] = from_f32<TOut>(ci_ * r4.y);
+                dvr[2] = from_f32<TOut>(ci_ * r4.z);
+                dvr[3] = from_f32<TOut>(ci_ * r4.w);
+                if (tx == 0) atomicAdd(&a.acc_dc[ti], dcp);
             }
-#pragma unroll
-            for (int t = 0; t < CD; ++t) {
-                const float p = Pm[t * LDC + i];
-#pragma unroll
-                for (int nn = 0; nn < 2; ++nn) ad[nn] = fmaf(p, dOs[t * LDV + tx + 16 * nn], ad[nn]);
-            }
-#pragma unroll
-            for (int nn = 0; nn < 2; ++nn) dRs[i * LDV + tx + 16 * nn] = ad[nn];
-        }
-        __syncthreads();
-        // dR = (I + L)^{-T} dU, newest row first
-        {
-            const int col = tid >> 3, part = tid & 7;
-            for (int j = n - 2; j >= 0; --j) {
-                float s = 0.f;
-                for (int i = j + 1 + part; i < n; i += 8) s = fmaf(Lm[i * LDC + j], dRs[i * LDV + col], s);
-                s += __shfl_xor_sync(0xffffffffu, s, 1);
-                s += __shfl_xor_sync(0xffffffffu, s, 2);
-                s += __shfl_xor_sync(0xffffffffu, s, 4);
-                if (part == 0) dRs[j * LDV + col] -= s;
-                __syncthreads();
-            }
-        }
-        // dv, dc; Y = dO U^T, D = -dR U^T; then db's D o A part
-        for (int i = warp; i < n; i += NT / 32) {
-            const size_t ti = tok_index(b, t0 + i, h, T, H);
-            const float dr = dRs[i * LDV + lane];
-            dv[ti * Dv + v0 + lane] = from_f32<TOut>(cs[i] * dr);
-            const float s_rv = warp_sum(dr * to_f32(v[ti * Dv + v0 + lane]));
-            if (lane == 0) atomicAdd(&a.acc_dc[ti], s_rv);
-        }
-        {
-            const int i = ty, j = tx;  // 16 x 16 = 256 threads
+            const int j = tx;
             float y = 0.f, dd = 0.f;
-#pragma unroll 8
-            for (int c = 0; c < NV; ++c) {
-                const float uj = Us[j * LDV + c];
-                y = fmaf(dOs[i * LDV + c], uj, y);
-                dd = fmaf(dRs[i * LDV + c], uj, dd);
-            }
-            Ym[i * LDC + j] = (j <= i) ? y : 0.f;
-            Dm[i * LDC + j] = (j < i) ? -dd : 0.f;
-        }
-        __syncthreads();
-        if (tid < CD) {
-            float s = 0.f;
-            for (int j = 0; j < tid; ++j) s = fmaf(Dm[tid * LDC + j], Am[tid * LDC + j], s);
-            atomicAdd(&dbs[tid], s);
-        }
-        // per (token, channel): dq, dkhat and dG partials (this thread: token ty, channels
-        // tx + 16 u)
-        {
-            const int i = ty;
-            float zq[EPT], zr[EPT], zl[EPT];
-#pragma unroll
-            for (int u = 0; u < EPT; ++u) zq[u] = zr[u] = zl[u] = 0.f;
-            // Z1 = dO S^T, Z2 = dR S^T, Z3 = U lambda^T (contraction over this CTA's columns)
 #pragma unroll 4
-            for (int c = 0; c < NV; ++c) {
-                const float o_ = dOs[i * LDV + c], r_ = dRs[i * LDV + c], u_ = Us[i * LDV + c];
-#pragma unroll
-                for (int u = 0; u < EPT; ++u) {
-                    const int d = tx + 16 * u;
-                    zq[u] = fmaf(o_, Ss[d * LDV + c], zq[u]);
-                    zr[u] = fmaf(r_, Ss[d * LDV + c], zr[u]);
-                    zl[u] = fmaf(u_, dSs[d * LDV + c], zl[u]);
-                }
+            for (int c = 0; c < 64; c += 4) {
+                const float4 uj = *reinterpret_cast<const float4*>(Us + j * BLD + c);
+                const float4 oi = *reinterpret_cast<const float4*>(dOs + i * BLD + c);
+                const float4 ri = *reinterpret_cast<const float4*>(dRs + i * BLD + c);
+                y += oi.x * uj.x + oi.y * uj.y + oi.z * uj.z + oi.w * uj.w;
+                dd += ri.x * uj.x + ri.y * uj.y + ri.z * uj.z + ri.w * uj.w;
             }
+            const float Y = (j <= i) ? y : 0.f, D = (j < i) ? -dd : 0.f;
+            Ym[i * LDC + j] = Y;
+            Dm[i * LDC + j] = D;
+            float da = D * Am[i * CD + j];
+#pragma unroll
+            for (int o = 1; o < 16; o <<= 1) da += __shfl_xor_sync(0xffffffffu, da, o);
+            if (tx == 0) dbs[i] = da;
+        }
+        // ---- Z1 = dO S^T, Z2 = dR S^T, Z3 = U lambda^T for (row i, channels tx + 16 u)
+        float zq[EPT], zr[EPT], zl[EPT];
+#pragma unroll
+        for (int u = 0; u < EPT; ++u) zq[u] = zr[u] = zl[u] = 0.f;
+#pragma unroll 2
+        for (int c = 0; c < 64; c += 4) {
+            const float4 o4 = *reinterpret_cast<const float4*>(dOs + i * BLD + c);
+            const float4 r4 = *reinterpret_cast<const float4*>(dRs + i * BLD + c);
+            const float4 u4 = *reinterpret_cast<const float4*>(Us + i * BLD + c);
+#pragma unroll
+            for (int u = 0; u < EPT; ++u) {
+                const int d = tx + 16 * u;
+                const float4 s4 = *reinterpret_cast<const float4*>(Ss + d * BLD + c);
+                const float4 l4 = *reinterpret_cast<const float4*>(Ls + d * BLD + c);
+                zq[u] += o4.x * s4.x + o4.y * s4.y + o4.z * s4.z + o4.w * s4.w;
+                zr[u] += r4.x * s4.x + r4.y * s4.y + r4.z * s4.z + r4.w * s4.w;
+                zl[u] += u4.x * l4.x + u4.y * l4.y + u4.z * l4.z + u4.w * l4.w;
+            }
+        }
+        __syncthreads();  // Ym, Dm written; S read: the previous chunk's state may come in
+        if (tid == 0 && ci > 0) request_state(ci - 1);
+        // ---- F terms and the per-(token, channel) gradients
+        float rq[EPT], rk[EPT], rg[EPT], rx[EPT];
+        {
             float f1[EPT], f2[EPT], f3[EPT], f4[EPT];
 #pragma unroll
             for (int u = 0; u < EPT; ++u) f1[u] = f2[u] = f3[u] = f4[u] = 0.f;
-            for (int j = 0; j <= i; ++j) {  // F1, F3: row i against earlier tokens j
+            for (int j = 0; j <= i; ++j) {
                 const float y = Ym[i * LDC + j], dd = Dm[i * LDC + j];
                 const float* E = Es + pair_index(i, j) * DK;
 #pragma unroll
                 for (int u = 0; u < EPT; ++u) {
                     const int d = tx + 16 * u;
-                    const float ke = Ks[j * LDK + d] * E[d];
+                    const float ke = Kh[j * LDK + d] * E[d];
                     f1[u] = fmaf(y, ke, f1[u]);
                     f3[u] = fmaf(dd, ke, f3[u]);
                 }
             }
-            for (int r = i; r < n; ++r) {  // F2, F4: column i against later tokens r
+            for (int r = i; r < n; ++r) {
                 const float y = Ym[r * LDC + i], dd = Dm[r * LDC + i] * bs[r];
                 const float* E = Es + pair_index(r, i) * DK;
 #pragma unroll
                 for (int u = 0; u < EPT; ++u) {
                     const int d = tx + 16 * u;
                     f2[u] = fmaf(y, Qs[r * LDK + d] * E[d], f2[u]);
-                    f4[u] = fmaf(dd, Ks[r * LDK + d] * E[d], f4[u]);
+                    f4[u] = fmaf(dd, Kh[r * LDK + d] * E[d], f4[u]);
                 }
             }
+            const float bi = bs[i];
             float kgz = 0.f;
-            if (i < n) {
-                const size_t ti = tok_index(b, t0 + i, h, T, H);
-                const float bi = bs[i];
 #pragma unroll
-                for (int u = 0; u < EPT; ++u) {
-                    const int d = tx + 16 * u;
-                    const float G = Gs[i * DK + d], Gl = Gs[(n - 1) * DK + d];
-                    const float gam = __expf(G), del = __expf(Gl - G);
-                    const float qd = Qs[i * LDK + d], kd = Ks[i * LDK + d];
-                    const float dq = fmaf(gam, zq[u], f1[u]);
-                    const float dk = -bi * gam * zr[u] + del * zl[u] + f2[u] + bi * f3[u] + f4[u];
-                    float dG = gam * qd * zq[u] + qd * f1[u] - bi * gam * kd * zr[u] - kd * f2[u] + bi * kd * f3[u] -
-                               kd * f4[u] - del * kd * zl[u];
-                    kgz = fmaf(kd * gam, zr[u], kgz);
-                    atomicAdd(&a.acc_dq[ti * DK + d], dq);
-                    atomicAdd(&a.acc_dkh[ti * DK + d], dk);
-                    atomicAdd(&a.acc_dG[ti * DK + d], dG);
-                    // the outgoing decays Del_j feed dG of the chunk's last token: summed over
-                    // the chunk's tokens below, one atomic per channel
-                    xs[i * DK + d] = del * kd * zl[u];
-                }
-            } else {
-#pragma unroll
-                for (int u = 0; u < EPT; ++u) xs[i * DK + tx + 16 * u] = 0.f;
+            for (int u = 0; u < EPT; ++u) {
+                const int d = tx + 16 * u;
+                const float G = Gs[i * DK + d], Gl = Gs[(n - 1) * DK + d];
+                const float gam = __expf(G), del = __expf(Gl - G);
+                const float qd = Qs[i * LDK + d], kd = Kh[i * LDK + d];
+                rq[u] = fmaf(gam, zq[u], f1[u]);
+                rk[u] = -bi * gam * zr[u] + del * zl[u] + f2[u] + bi * f3[u] + f4[u];
+                rg[u] = gam * qd * zq[u] + qd * f1[u] - bi * gam * kd * zr[u] - kd * f2[u] + bi * kd * f3[u] -
+                        kd * f4[u] - del * kd * zl[u];
+                rx[u] = del * kd * zl[u];
+                kgz = fmaf(kd * gam, zr[u], kgz);
             }
-            // db: - (khat_i o Gam_i) . Z2_i (this thread's channels, then the row's 16 threads)
-            kgz += __shfl_xor_sync(0xffffffffu, kgz, 1);
-            kgz += __shfl_xor_sync(0xffffffffu, kgz, 2);
-            kgz += __shfl_xor_sync(0xffffffffu, kgz, 4);
-            kgz += __shfl_xor_sync(0xffffffffu, kgz, 8);
-            if (tx == 0 && i < n) atomicAdd(&dbs[i], -kgz);
-        }
-        __syncthreads();
-        if (tid < DK) {  // dG of the last token: sum_j Del_j o khat_j o Z3_j + Gam_last o rowsum(lambda o S)
-            float e = __expf(Gs[(n - 1) * DK + tid]) * lsS[tid];
-            for (int r = 0; r < n; ++r) e += xs[r * DK + tid];
-            atomicAdd(&a.acc_dG[tok_index(b, t0 + n - 1, h, T, H) * DK + tid], e);
-        }
-        // new lambda = Diag(Gam_last) lambda + (Q o Gam)^T dO - (Diag(b) (Khat o Gam))^T dR
-        {
-            float as[TMK][2];
 #pragma unroll
-            for (int m = 0; m < TMK; ++m) as[m][0] = as[m][1] = 0.f;
+            for (int o = 1; o < 16; o <<= 1) kgz += __shfl_xor_sync(0xffffffffu, kgz, o);
+            if (tx == 0) dbs[i] -= kgz;
+        }
+        __syncthreads();  // Es read: it takes the results
+        float* Rq = Es;
+        float* Rk = Es + CD * DK;
+        float* Rg = Es + 2 * CD * DK;
+        float* Rxs = Es + 3 * CD * DK;  // NP >= 4 CD rows of DK: room for the last token's terms
+#pragma unroll
+        for (int u = 0; u < EPT; ++u) {
+            const int d = tx + 16 * u;
+            Rq[i * DK + d] = rq[u];
+            Rk[i * DK + d] = rk[u];
+            Rg[i * DK + d] = rg[u];
+            Rxs[i * DK + d] = (i < n) ? rx[u] : 0.f;
+        }
+        // ---- new lambda = Diag(GC) lambda + QG^T dO - W^T dU (rows i + 16 m, columns cx .. cx + 3)
+        {
+            float4 acc[DK / 16];
+#pragma unroll
+            for (int m = 0; m < DK / 16; ++m) {
+                const int r = i + 16 * m;
+                const float gc = Rh[R::GC + r];
+                const float4 l4 = *reinterpret_cast<const float4*>(Ls + r * BLD + cx);
+                acc[m] = make_float4(gc * l4.x, gc * l4.y, gc * l4.z, gc * l4.w);
+            }
 #pragma unroll
             for (int t = 0; t < CD; ++t) {
-                float o2[2], r2[2];
+                const float4 o4 = *reinterpret_cast<const float4*>(dOs + t * BLD + cx);
+                const float4 d4 = *reinterpret_cast<const float4*>(dUs + t * BLD + cx);
+                const float* qg = Rh + R::QG + t * DK + i;
+                const float* wr = Rh + R::W + t * DK + i;
 #pragma unroll
-                for (int nn = 0; nn < 2; ++nn) {
-                    o2[nn] = dOs[t * LDV + tx + 16 * nn];
-                    r2[nn] = -bs[t] * dRs[t * LDV + tx + 16 * nn];
-                }
-#pragma unroll
-                for (int m = 0; m < TMK; ++m) {
-                    const int r = ty + 16 * m;
-                    const float gm = __expf(Gs[t * DK + r]);
-                    const float wq = Qs[t * LDK + r] * gm, wk = Ks[t * LDK + r] * gm;
-#pragma unroll
-                    for (int nn = 0; nn < 2; ++nn) as[m][nn] = fmaf(wq, o2[nn], fmaf(wk, r2[nn], as[m][nn]));
+                for (int m = 0; m < DK / 16; ++m) {
+                    const float wq = qg[16 * m], ww = wr[16 * m];
+                    acc[m].x = fmaf(wq, o4.x, fmaf(-ww, d4.x, acc[m].x));
+                    acc[m].y = fmaf(wq, o4.y, fmaf(-ww, d4.y, acc[m].y));
+                    acc[m].z = fmaf(wq, o4.z, fmaf(-ww, d4.z, acc[m].z));
+                    acc[m].w = fmaf(wq, o4.w, fmaf(-ww, d4.w, acc[m].w));
                 }
             }
-            __syncthreads();
 #pragma unroll
-            for (int m = 0; m < TMK; ++m) {
-                const int r = ty + 16 * m;
-                const float gl_r = __expf(Gs[(n - 1) * DK + r]);
-#pragma unroll
-                for (int nn = 0; nn < 2; ++nn) {
-                    float* sp = &dSs[r * LDV + tx + 16 * nn];
-                    *sp = fmaf(gl_r, *sp, as[m][nn]);
-                }
-            }
+            for (int m = 0; m < DK / 16; ++m) *reinterpret_cast<float4*>(Ls + (i + 16 * m) * BLD + cx) = acc[m];
         }
         __syncthreads();
+        if (tid < DK) {  // dG of the last token: sum_j Del_j o khat_j o Z3_j + GC o rowsum(lambda o S)
+            float e = Rh[R::GC + tid] * lsS[tid];
+            for (int r = 0; r < n; ++r) e += Rxs[r * DK + tid];
+            Rg[(n - 1) * DK + tid] += e;
+        }
+        __syncthreads();
+        // ---- out: dq, dkhat, dG of this chunk's tokens (eight consecutive channels a thread)
+        for (int x = tid; x < CD * DK / 8; x += NT) {
+            const int r = x / (DK / 8), c8 = 8 * (x % (DK / 8));
+            if (r < n) {
+                const size_t o = tok_index(b, t0 + r, h, T, H) * DK + c8;
+                const float* pq = Rq + r * DK + c8;
+                const float* pk = Rk + r * DK + c8;
+                const float* pg = Rg + r * DK + c8;
+                red_add_v4(a.acc_dq + o, pq[0], pq[1], pq[2], pq[3]);
+                red_add_v4(a.acc_dq + o + 4, pq[4], pq[5], pq[6], pq[7]);
+                red_add_v4(a.acc_dkh + o, pk[0], pk[1], pk[2], pk[3]);
+                red_add_v4(a.acc_dkh + o + 4, pk[4], pk[5], pk[6], pk[7]);
+                red_add_v4(a.acc_dG + o, pg[0], pg[1], pg[2], pg[3]);
+                red_add_v4(a.acc_dG + o + 4, pg[4], pg[5], pg[6], pg[7]);
+            }
+        }
         if (tid < n) atomicAdd(&a.acc_db[tok_index(b, t0 + tid, h, T, H)], dbs[tid]);
+        if (tid == 0 && ci > 0) request_rec(ci - 1);  // every read of the record is done
+        (void)lane;
     }
+    if (!ok && tid == 0) atomicOr(&g_diag_error, 2u);
     __syncthreads();
-    for (int x = tid; x < DK * NV; x += NT) {
-        const int r = x / NV, c = x % NV;
-        a.dS0[sbase + (size_t)r * Dv + v0 + c] = dSs[r * LDV + c];
+    if (ok) {
+        for (int x = tid; x < DK * 64; x += NT) {
+            const int r = x >> 6, c = x & 63;
+            a.dS0[sbase + (size_t)r * DV + v0 + c] = Ls[r * BLD + c];
+        }
     }
 }
 
@@ -732,18 +794,11 @@ __global__ void diag_dg_kernel(BwdArgs a) {
 //   P                             [16][16]
 //   GC = Gam_last                 [DK]
 //   UP = T Diag(c) V              [DV/64][16][64]   (in 64-column slices)
+// and, for the backward, A [16][16] (Gram without b), T [16][16] and G [16][DK].
 // `diag_state_kernel` then walks each head's chunks in order on a 64-column slice of the state:
 //   U = UP - W S,   O = QG S + P U,   S' = Diag(GC) S + KD^T U,
 // with the records double-buffered in shared memory by bulk copies.
 // ------------------------------------------------------------------------------------
-template <int DK, int DV>
-struct DiagRec {
-    static constexpr int kHead = 3 * CD * DK + CD * CD + DK;  // W, QG, KD, P, GC (floats)
-    static constexpr int kSlice = CD * 64;                     // one 64-column slice of UP
-    static constexpr int kFloats = kHead + (DV / 64) * kSlice;
-    static constexpr int W = 0, QG = CD * DK, KD = 2 * CD * DK, P = 3 * CD * DK, GC = 3 * CD * DK + CD * CD,
-                         UP = kHead;
-};
 
 template <int DK, int DV, typename Tin>
 __global__ void __launch_bounds__(NT) diag_prep_kernel(FwdArgs a, float* __restrict__ recs) {
@@ -827,6 +882,13 @@ __global__ void __launch_bounds__(NT) diag_prep_kernel(FwdArgs a, float* __restr
             for (int j = 0; j <= i; ++j) s = fmaf(Tm[i * LDC + j], Vs[j * LDV + c], s);
             rec[R::UP + (c >> 6) * R::kSlice + i * 64 + (c & 63)] = s;
         }
+    }
+    if (a.rec_extras) {
+        for (int x = tid; x < CD * CD; x += NT) {
+            rec[R::XA + x] = Am[(x / CD) * LDC + x % CD];
+            rec[R::XT + x] = Tm[(x / CD) * LDC + x % CD];
+        }
+        for (int x = tid; x < CD * DK; x += NT) rec[R::XG + x] = Gs[x];
     }
 }
 
@@ -1007,13 +1069,13 @@ cudaError_t diag_fwd_launch(const FwdArgs& a, cudaStream_t st) {
     return cudaGetLastError();
 }
 
-template <int DK, typename Tin, typename TOut>
-cudaError_t diag_bwd_launch(const BwdArgs& a, const FwdArgs& f, cudaStream_t st) {
-    const size_t smem = diag_bwd_smem_bytes<DK>();
-    cudaError_t e = cudaFuncSetAttribute(chunk_bwd_diag_kernel<DK, Tin, TOut>,
+template <int DK, int DV, typename Tin, typename TOut>
+cudaError_t diag_bwd_launch(const BwdArgs& a, const FwdArgs& f, const float* recs, cudaStream_t st) {
+    const size_t smem = diag_bwd_smem_bytes<DK, DV>();
+    cudaError_t e = cudaFuncSetAttribute(diag_bwd_kernel<DK, DV, Tin, TOut>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    chunk_bwd_diag_kernel<DK, Tin, TOut><<<dim3(a.Dv / 32, a.H, a.B), NT, smem, st>>>(a, f);
+    diag_bwd_kernel<DK, DV, Tin, TOut><<<dim3(DV / 64, a.H, a.B), NT, smem, st>>>(a, f, recs);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     const size_t ntok = (size_t)a.B * a.T * a.H;
     diag_finalize_kernel<DK, Tin, TOut><<<(unsigned)((ntok + 7) / 8), 256, 0, st>>>(a, ntok);
@@ -1027,9 +1089,14 @@ template <int DK, typename Tin>
 cudaError_t diag_fwd_o(const FwdArgs& a, cudaStream_t st) {
     return a.out_bf16 ? diag_fwd_launch<DK, Tin, __nv_bfloat16>(a, st) : diag_fwd_launch<DK, Tin, float>(a, st);
 }
+template <int DK, typename Tin, typename TOut>
+cudaError_t diag_bwd_dv(const BwdArgs& a, const FwdArgs& f, const float* recs, cudaStream_t st) {
+    return a.Dv == 128 ? diag_bwd_launch<DK, 128, Tin, TOut>(a, f, recs, st)
+                       : diag_bwd_launch<DK, 64, Tin, TOut>(a, f, recs, st);
+}
 template <int DK, typename Tin>
-cudaError_t diag_bwd_o(const BwdArgs& a, const FwdArgs& f, cudaStream_t st) {
-    return a.out_bf16 ? diag_bwd_launch<DK, Tin, __nv_bfloat16>(a, f, st) : diag_bwd_launch<DK, Tin, float>(a, f, st);
+cudaError_t diag_bwd_o(const BwdArgs& a, const FwdArgs& f, const float* recs, cudaStream_t st) {
+    return a.out_bf16 ? diag_bwd_dv<DK, Tin, __nv_bfloat16>(a, f, recs, st) : diag_bwd_dv<DK, Tin, float>(a, f, recs, st);
 }
 
 }  // namespace
@@ -1085,10 +1152,14 @@ cudaError_t launch_chunk_bwd_diag(const BwdArgs& a, const float* S0, void* rec_w
     f.Dv = a.Dv;
     f.bf16 = a.bf16;
     f.out_bf16 = false;
+    f.rec_extras = true;
+    if (rec_ws == nullptr || rec_bytes < diag_fwd_workspace(a.B, a.T, a.H, a.Dk, a.Dv)) return cudaErrorInvalidValue;
     cudaError_t e = launch_chunk_fwd_diag(f, rec_ws, rec_bytes, st);
     if (e != cudaSuccess) return e;
-    if (a.bf16) return a.Dk == 128 ? diag_bwd_o<128, __nv_bfloat16>(a, f, st) : diag_bwd_o<64, __nv_bfloat16>(a, f, st);
-    return a.Dk == 128 ? diag_bwd_o<128, float>(a, f, st) : diag_bwd_o<64, float>(a, f, st);
+    const float* recs = static_cast<const float*>(rec_ws);
+    if (a.bf16)
+        return a.Dk == 128 ? diag_bwd_o<128, __nv_bfloat16>(a, f, recs, st) : diag_bwd_o<64, __nv_bfloat16>(a, f, recs, st);
+    return a.Dk == 128 ? diag_bwd_o<128, float>(a, f, recs, st) : diag_bwd_o<64, float>(a, f, recs, st);
 }
 
 }  // namespace kla

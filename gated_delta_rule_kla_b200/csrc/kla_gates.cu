@@ -10,10 +10,11 @@
 // x is read once for all heads, which is why this is its own kernel rather than part of the
 // per-(chunk, head) preparation kernel (that would read each token's x once per head).
 //
-// bf16 with D % 64 == 0 and 2H in {16, 32, ..., 256}: one CTA per 128 tokens runs the
+// bf16 with D % 64 == 0 and 2H in {16, 32, ..., 128}: one CTA per 128 tokens runs the
 // projection on the tensor cores (tcgen05, M = 128 tokens, N = 2H, K = D in 64-wide steps
-// through a 4-stage TMA ring), the activations in the TMEM epilogue, and the query
-// normalisation on the warps that neither load nor issue.  Other shapes and fp32: CUDA cores.
+// through a 6-stage TMA ring) and the activations in the TMEM epilogue.  Other shapes and fp32:
+// CUDA cores.  The query normalisation is a streaming kernel of its own (a group of Dk/8 lanes
+// per row, 16-byte accesses), launched first on the same stream.
 //
 // Backward (CUDA cores): with dz = [deta * eta (1 - eta), dg * expm1(g)] (d(-softplus z)/dz =
 // -sigmoid(z) = expm1(g)),  dx = dz W,  dW = dz^T x,  dbias = sum_t dz,
@@ -37,30 +38,102 @@ using namespace sm100;
 constexpr uint64_t kWaitNs = 2000000000ull;
 constexpr int GM = 128;    // tokens per CTA
 constexpr int GKT = 64;    // K elements per stage (128 bytes of bf16)
-constexpr int GST = 4;     // stages
-constexpr int GTH = 256;   // threads: warps 0-3 epilogue, 4 loader, 5 MMA issuer; q rows on 0-3, 6, 7
+constexpr int GST = 6;     // stages
+constexpr int GTH = 192;   // threads: warps 0-3 epilogue, 4 loader, 5 MMA issuer
 
 __device__ __forceinline__ float sigmoidf_(float z) { return 1.f / (1.f + __expf(-z)); }
 __device__ __forceinline__ float softplusf_(float z) { return fmaxf(z, 0.f) + log1pf(__expf(-fabsf(z))); }
 
-// q rows (token, head) of tokens [tok0, tok0 + ntok), warp-strided: qhat = q / ||q||.
-template <typename Tin>
-__device__ __forceinline__ void normalize_rows(const Tin* q, Tin* qhat, size_t tok0, int ntok, int H, int Dk,
-                                               int wid, int nwarps) {
-    const int lane = threadIdx.x & 31;
-    const int per = Dk / 32;
-    for (int r = wid; r < ntok * H; r += nwarps) {
-        const size_t base = (tok0 * H + r) * (size_t)Dk;
-        float x[4];
-        float s = 0.f;
-        for (int u = 0; u < per; ++u) {
-            x[u] = to_f32(q[base + lane + 32 * u]);
-            s = fmaf(x[u], x[u], s);
-        }
-        s = warp_sum(s);
-        const float inv = s > 0.f ? rsqrtf(s) : 0.f;
-        for (int u = 0; u < per; ++u) qhat[base + lane + 32 * u] = from_f32<Tin>(x[u] * inv);
+// Eight consecutive elements as fp32 and back (16 bytes of bf16, 32 of fp32).
+__device__ __forceinline__ void ld8(const __nv_bfloat16* p, float* f) {
+    unpack_bf16x8(*reinterpret_cast<const uint4*>(p), f);
+}
+__device__ __forceinline__ void ld8(const float* p, float* f) {
+    const float4 a = reinterpret_cast<const float4*>(p)[0], b = reinterpret_cast<const float4*>(p)[1];
+    f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w; f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+}
+__device__ __forceinline__ void st8(__nv_bfloat16* p, const float* f) {
+    uint4 w;
+    w.x = pack_bf16x2(f[0], f[1]); w.y = pack_bf16x2(f[2], f[3]);
+    w.z = pack_bf16x2(f[4], f[5]); w.w = pack_bf16x2(f[6], f[7]);
+    *reinterpret_cast<uint4*>(p) = w;
+}
+__device__ __forceinline__ void st8(float* p, const float* f) {
+    reinterpret_cast<float4*>(p)[0] = make_float4(f[0], f[1], f[2], f[3]);
+    reinterpret_cast<float4*>(p)[1] = make_float4(f[4], f[5], f[6], f[7]);
+}
+
+// qhat = q / ||q|| for every (token, head) row of Dk elements: a group of Dk / 8 lanes per row,
+// eight elements per lane, the sum of squares reduced inside the group.  Streams q once.
+template <typename Tin, int DK>
+__global__ void __launch_bounds__(256) qnorm_kernel(const Tin* __restrict__ q, Tin* __restrict__ qhat, size_t rows) {
+    constexpr int G = DK / 8;
+    const size_t gid = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const size_t row = gid / G;
+    const bool live = row < rows;
+    const size_t off = (live ? row : 0) * DK + (gid % G) * 8;
+    float x[8];
+    ld8(q + off, x);
+    float s = 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) s = fmaf(x[e], x[e], s);
+#pragma unroll
+    for (int o = G / 2; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    const float inv = s > 0.f ? rsqrtf(s) : 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) x[e] *= inv;
+    if (live) st8(qhat + off, x);
+}
+
+// dq = (dqhat - qhat (qhat . dqhat)) / ||q|| per row (zero where q is zero), same layout.
+template <typename Tin, int DK>
+__global__ void __launch_bounds__(256) qnorm_bwd_kernel(const Tin* __restrict__ q, const float* __restrict__ dqhat,
+                                                        float* __restrict__ dq, size_t rows) {
+    constexpr int G = DK / 8;
+    const size_t gid = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const size_t row = gid / G;
+    const bool live = row < rows;
+    const size_t off = (live ? row : 0) * DK + (gid % G) * 8;
+    float x[8], d[8];
+    ld8(q + off, x);
+    ld8(dqhat + off, d);
+    float s = 0.f, p = 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        s = fmaf(x[e], x[e], s);
+        p = fmaf(x[e], d[e], p);
     }
+#pragma unroll
+    for (int o = G / 2; o > 0; o >>= 1) {
+        s += __shfl_xor_sync(0xffffffffu, s, o);
+        p += __shfl_xor_sync(0xffffffffu, p, o);
+    }
+    const float inv = s > 0.f ? rsqrtf(s) : 0.f;  // 1 / ||q||;  qhat . dqhat = p / ||q||
+    const float c = inv * inv * p;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) d[e] = inv * (d[e] - x[e] * c);
+    if (live) st8(dq + off, d);
+}
+
+template <typename Tin>
+cudaError_t launch_qnorm(const Tin* q, Tin* qhat, size_t rows, int Dk, cudaStream_t st) {
+    const size_t threads = rows * (size_t)(Dk / 8);
+    const unsigned grid = (unsigned)((threads + 255) / 256);
+    if (Dk == 128)
+        qnorm_kernel<Tin, 128><<<grid, 256, 0, st>>>(q, qhat, rows);
+    else
+        qnorm_kernel<Tin, 64><<<grid, 256, 0, st>>>(q, qhat, rows);
+    return cudaGetLastError();
+}
+template <typename Tin>
+cudaError_t launch_qnorm_bwd(const Tin* q, const float* dqhat, float* dq, size_t rows, int Dk, cudaStream_t st) {
+    const size_t threads = rows * (size_t)(Dk / 8);
+    const unsigned grid = (unsigned)((threads + 255) / 256);
+    if (Dk == 128)
+        qnorm_bwd_kernel<Tin, 128><<<grid, 256, 0, st>>>(q, dqhat, dq, rows);
+    else
+        qnorm_bwd_kernel<Tin, 64><<<grid, 256, 0, st>>>(q, dqhat, dq, rows);
+    return cudaGetLastError();
 }
 
 // ------------------------------------------------------------------------------------
@@ -74,9 +147,8 @@ struct GateBars {
 
 __global__ void __launch_bounds__(GTH, 1)
     gate_prologue_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
-                            const float* __restrict__ bias, float* __restrict__ eta, float* __restrict__ g,
-                            const __nv_bfloat16* __restrict__ q, __nv_bfloat16* __restrict__ qhat, int N, int D,
-                            int H, int Dk, uint32_t w_bytes, uint32_t tmem_cols) {
+                            const float* __restrict__ bias, float* __restrict__ eta, float* __restrict__ g, int N,
+                            int D, int H, uint32_t w_bytes, uint32_t tmem_cols) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t stage_bytes = 16384 + w_bytes;
@@ -137,9 +209,6 @@ __global__ void __launch_bounds__(GTH, 1)
             mma_commit(smem_u32(&bars->done));
         }
     }
-    // query normalisation on the other warps while the projection runs
-    if (q != nullptr && warp != 4 && warp != 5)
-        normalize_rows<__nv_bfloat16>(q, qhat, (size_t)tok0, ntok, H, Dk, warp < 4 ? warp : warp - 2, 6);
     if (warp < 4) {  // epilogue: lane = token
         const bool got = mbar_wait_bounded(smem_u32(&bars->done), 0, kWaitNs);
         if (__any_sync(0xffffffffu, !got)) {
@@ -183,8 +252,7 @@ __global__ void __launch_bounds__(GTH, 1)
 template <typename Tin>
 __global__ void __launch_bounds__(256) gate_prologue_simt_kernel(const Tin* __restrict__ x, const Tin* __restrict__ W,
                                                                  const float* __restrict__ bias, float* __restrict__ eta,
-                                                                 float* __restrict__ g, const Tin* __restrict__ q,
-                                                                 Tin* __restrict__ qhat, int N, int D, int H, int Dk) {
+                                                                 float* __restrict__ g, int N, int D, int H) {
     const int lane = threadIdx.x & 31;
     const size_t t = (size_t)blockIdx.x * 8 + (threadIdx.x >> 5);
     if (t >= (size_t)N) return;
@@ -213,7 +281,6 @@ __global__ void __launch_bounds__(256) gate_prologue_simt_kernel(const Tin* __re
                 g[t * H + (j - H)] = -softplusf_(zz);
         }
     }
-    if (q != nullptr) normalize_rows<Tin>(q, qhat, t, 1, H, Dk, 0, 1);
 }
 
 // ------------------------------------------------------------------------------------
@@ -227,10 +294,8 @@ template <typename Tin>
 __global__ void __launch_bounds__(256) gate_bwd_tile_kernel(const Tin* __restrict__ x, const Tin* __restrict__ W,
                                                             const float* __restrict__ eta, const float* __restrict__ g,
                                                             const float* __restrict__ deta, const float* __restrict__ dg,
-                                                            const Tin* __restrict__ q, const float* __restrict__ dqhat,
-                                                            float* __restrict__ dx, float* __restrict__ dq,
-                                                            float* __restrict__ part_w, float* __restrict__ part_b,
-                                                            int N, int D, int H, int Dk) {
+                                                            float* __restrict__ dx, float* __restrict__ part_w,
+                                                            float* __restrict__ part_b, int N, int D, int H) {
     extern __shared__ float smf[];
     const int NW = 2 * H;
     float* dz = smf;                   // [BT][NW]
@@ -263,13 +328,20 @@ __global__ void __launch_bounds__(256) gate_bwd_tile_kernel(const Tin* __restric
     for (int d0 = 0; d0 < D; d0 += BD) {
         const int nd = min(BD, D - d0);
         __syncthreads();
-        for (int i = tid; i < BT * BD; i += 256) {
-            const int t = i / BD, c = i % BD;
-            xs[t * (BD + 1) + c] = (t < nt && c < nd) ? to_f32(x[(size_t)(t0 + t) * D + d0 + c]) : 0.f;
+        // eight elements per access (D % 8 == 0, so a group of eight is either in range or not)
+        for (int i = tid; i < BT * (BD / 8); i += 256) {
+            const int t = i / (BD / 8), c8 = 8 * (i % (BD / 8));
+            float f[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            if (t < nt && c8 < nd) ld8(x + (size_t)(t0 + t) * D + d0 + c8, f);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) xs[t * (BD + 1) + c8 + e] = f[e];
         }
-        for (int i = tid; i < NW * BD; i += 256) {
-            const int j = i / BD, c = i % BD;
-            wsh[j * (BD + 1) + c] = c < nd ? to_f32(W[(size_t)j * D + d0 + c]) : 0.f;
+        for (int i = tid; i < NW * (BD / 8); i += 256) {
+            const int j = i / (BD / 8), c8 = 8 * (i % (BD / 8));
+            float f[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            if (c8 < nd) ld8(W + (size_t)j * D + d0 + c8, f);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) wsh[j * (BD + 1) + c8 + e] = f[e];
         }
         __syncthreads();
         // dx[t][c] = sum_j dz[t][j] W[j][c]: thread = column c (128) x token half
@@ -291,27 +363,6 @@ __global__ void __launch_bounds__(256) gate_bwd_tile_kernel(const Tin* __restric
                 for (int t = 0; t < BT; ++t) s = fmaf(dz[t * NW + j], xs[t * (BD + 1) + c], s);
                 part_w[((size_t)tile * NW + j) * D + d0 + c] = s;
             }
-        }
-    }
-    // dq = (dqhat - qhat (qhat . dqhat)) / ||q||, one warp per (token, head)
-    if (q != nullptr) {
-        const int lane = tid & 31, wid = tid >> 5;
-        const int per = Dk / 32;
-        for (int r = wid; r < nt * H; r += 8) {
-            const size_t base = ((size_t)t0 * H + r) * Dk;
-            float qv[4], dv[4];
-            float s = 0.f, p = 0.f;
-            for (int u = 0; u < per; ++u) {
-                qv[u] = to_f32(q[base + lane + 32 * u]);
-                dv[u] = dqhat[base + lane + 32 * u];
-                s = fmaf(qv[u], qv[u], s);
-                p = fmaf(qv[u], dv[u], p);
-            }
-            s = warp_sum(s);
-            p = warp_sum(p);
-            const float inv = s > 0.f ? rsqrtf(s) : 0.f;  // 1 / ||q||
-            // qhat . dqhat = p / ||q||
-            for (int u = 0; u < per; ++u) dq[base + lane + 32 * u] = inv * (dv[u] - qv[u] * inv * (p * inv));
         }
     }
 }
@@ -346,6 +397,14 @@ size_t gate_bwd_workspace(int N, int D, int H) {
 
 cudaError_t launch_gate_prologue(const GateArgs& a, cudaStream_t st) {
     if (a.N == 0) return cudaSuccess;
+    if (a.q != nullptr) {
+        const size_t rows = (size_t)a.N * a.H;
+        const cudaError_t e = a.bf16 ? launch_qnorm(static_cast<const __nv_bfloat16*>(a.q),
+                                                    static_cast<__nv_bfloat16*>(a.qhat), rows, a.Dk, st)
+                                     : launch_qnorm(static_cast<const float*>(a.q), static_cast<float*>(a.qhat), rows,
+                                                    a.Dk, st);
+        if (e != cudaSuccess) return e;
+    }
     if (gate_tc_shape(a)) {
         EncodeTiledFn enc = get_encode_fn();
         if (enc != nullptr) {
@@ -371,21 +430,20 @@ cudaError_t launch_gate_prologue(const GateArgs& a, cudaStream_t st) {
             cudaError_t e = cudaFuncSetAttribute(gate_prologue_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                  (int)smem);
             if (e != cudaSuccess) return e;
-            gate_prologue_tc_kernel<<<(a.N + GM - 1) / GM, GTH, smem, st>>>(
-                mx, mw, a.bias, a.eta, a.g, static_cast<const __nv_bfloat16*>(a.q),
-                static_cast<__nv_bfloat16*>(a.qhat), a.N, a.D, a.H, a.Dk, w_bytes, cols);
+            gate_prologue_tc_kernel<<<(a.N + GM - 1) / GM, GTH, smem, st>>>(mx, mw, a.bias, a.eta, a.g, a.N, a.D,
+                                                                            a.H, w_bytes, cols);
             return cudaGetLastError();
         }
     }
     const unsigned grid = (unsigned)(((size_t)a.N + 7) / 8);
     if (a.bf16)
         gate_prologue_simt_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
-            static_cast<const __nv_bfloat16*>(a.x), static_cast<const __nv_bfloat16*>(a.W), a.bias, a.eta, a.g,
-            static_cast<const __nv_bfloat16*>(a.q), static_cast<__nv_bfloat16*>(a.qhat), a.N, a.D, a.H, a.Dk);
+            static_cast<const __nv_bfloat16*>(a.x), static_cast<const __nv_bfloat16*>(a.W), a.bias, a.eta, a.g, a.N,
+            a.D, a.H);
     else
-        gate_prologue_simt_kernel<float><<<grid, 256, 0, st>>>(
-            static_cast<const float*>(a.x), static_cast<const float*>(a.W), a.bias, a.eta, a.g,
-            static_cast<const float*>(a.q), static_cast<float*>(a.qhat), a.N, a.D, a.H, a.Dk);
+        gate_prologue_simt_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float*>(a.x),
+                                                                static_cast<const float*>(a.W), a.bias, a.eta, a.g,
+                                                                a.N, a.D, a.H);
     return cudaGetLastError();
 }
 
@@ -407,15 +465,21 @@ cudaError_t launch_gate_prologue_bwd(const GateBwdArgs& a, void* ws, cudaStream_
         if (e != cudaSuccess) return e;
         gate_bwd_tile_kernel<__nv_bfloat16><<<ntile, 256, smem, st>>>(
             static_cast<const __nv_bfloat16*>(a.x), static_cast<const __nv_bfloat16*>(a.W), a.eta, a.g, a.deta, a.dg,
-            static_cast<const __nv_bfloat16*>(a.q), a.dqhat, a.dx, a.dq, part_w, part_b, a.N, a.D, a.H, a.Dk);
+            a.dx, part_w, part_b, a.N, a.D, a.H);
     } else {
         e = cudaFuncSetAttribute(gate_bwd_tile_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        gate_bwd_tile_kernel<float><<<ntile, 256, smem, st>>>(
-            static_cast<const float*>(a.x), static_cast<const float*>(a.W), a.eta, a.g, a.deta, a.dg,
-            static_cast<const float*>(a.q), a.dqhat, a.dx, a.dq, part_w, part_b, a.N, a.D, a.H, a.Dk);
+        gate_bwd_tile_kernel<float><<<ntile, 256, smem, st>>>(static_cast<const float*>(a.x),
+                                                               static_cast<const float*>(a.W), a.eta, a.g, a.deta,
+                                                               a.dg, a.dx, part_w, part_b, a.N, a.D, a.H);
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (a.q != nullptr) {
+        const size_t rows = (size_t)a.N * a.H;
+        e = a.bf16 ? launch_qnorm_bwd(static_cast<const __nv_bfloat16*>(a.q), a.dqhat, a.dq, rows, a.Dk, st)
+                   : launch_qnorm_bwd(static_cast<const float*>(a.q), a.dqhat, a.dq, rows, a.Dk, st);
+        if (e != cudaSuccess) return e;
+    }
     const size_t total = (size_t)NW * a.D;
     gate_bwd_reduce_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(part_w, part_b, a.dW, a.db, ntile, NW,
                                                                             a.D);

@@ -48,6 +48,9 @@ struct FwdArgs {
     // First chunk of a non-segmented state-pass run of seg_chunks chunks (0 for a whole
     // sequence): the host splits a sequence into slabs handled by consecutive runs.
     int chunk0;
+    // Diagonal-gated split forward: also store what the backward needs in each record (the Gram
+    // A, the inverse T and the per-channel log-decay prefix G of every 16-token chunk).
+    bool rec_extras = false;
 };
 
 struct BwdArgs {

@@ -271,7 +271,7 @@ kla_status kla_decode_step_diag(const void *q, const void *k, const void *v, con
  * ||q_t||; o is linear in q, so the recurrence run on qhat gives that readout; a zero query
  * gives qhat = 0).  The pages print no projection for g: the one here is a reading (a linear
  * projection through -softplus, so that g <= 0).
- *   x      in   [N, D] of `dtype` (N = B*T tokens; D % 8 == 0 for bf16, % 4 for fp32)
+ *   x      in   [N, D] of `dtype` (N = B*T tokens; D % 8 == 0)
  *   W      in   [2H, D] of `dtype`: rows 0..H-1 project eta, rows H..2H-1 project g
  *   bias   in   [2H] fp32
  *   q      in   [N, H, Dk] of `dtype`, or NULL (no normalisation); Dk in {64, 128}
