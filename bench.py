@@ -510,6 +510,36 @@ def bench_long(kla, WORKLOADS, make_inputs, dev, stream, rank, world, hbm_peak, 
     # timed on their own
     stages = time_fwd_stages(kla, d, w, ws, o, ST, lambda: None, stream, nsteps)
     stages["chunk_state_kernel"]["includes"] = "transition pass + seg_scan_kernel + output pass"
+    del ws
+    # the long-context training step: kla_chunk_fwd_train + kla_chunk_bwd_after_train sharing
+    # one workspace (records and tile images: about 5 GB here)
+    dO = torch.randn(w.B, w.T, w.H, w.Dv, device=dev).to(d["q"].dtype)
+    wst = kla.train_workspace(d["k"], d["v"])
+
+    def fwd_t():
+        kla.chunk_fwd_train(d["q"], d["k"], d["v"], d["eta"], d["g"], w.eps, d["S0"], workspace=wst, o=o, S_T=ST)
+
+    def bwd_t():
+        kla.chunk_bwd_after_train(d["q"], d["k"], d["v"], d["eta"], d["g"], dO, wst, w.eps)
+
+    fwd_t()
+    bwd_t()
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(2)]
+    for e in ev:
+        e[0].record(stream)
+        fwd_t()
+        e[1].record(stream)
+        bwd_t()
+        e[2].record(stream)
+    torch.cuda.synchronize()
+    f_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+    b_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
+    del wst
+    train = {"ms_per_step": f_ms + b_ms, "forward_ms": f_ms, "backward_ms": b_ms,
+             "value": w.B * w.T / ((f_ms + b_ms) / 1e3), "unit": "tokens/s",
+             "what": "kla_chunk_fwd_train + kla_chunk_bwd_after_train (reverse state pass over 1024 chunks per head, "
+                     "then the chunk-parallel gradient kernel)"}
     barrier(world)
     total_ms = max_over_ranks(sum(ms), world)
     tokens = sum_over_ranks(float(w.B * w.T), world) * nsteps
@@ -519,7 +549,7 @@ def bench_long(kla, WORKLOADS, make_inputs, dev, stream, rank, world, hbm_peak, 
     return {"workload": w.name, "value": tokens / (total_ms / 1e3), "unit": "tokens/s",
             "steps": nsteps, "ms_per_step": total_ms / nsteps, "l2": "inputs larger than L2",
             # preparation, transition pass, segment scan, output pass
-            "gpu_launches_per_step": 4, "stages": stages,
+            "gpu_launches_per_step": 4, "stages": stages, "train": train,
             "roofline": {"bound": "hbm", "achieved": alg / mean_s / 1e9, "peak": hbm_peak, "unit": "GB/s",
                          "frac": alg / mean_s / 1e9 / hbm_peak,
                          "tensor_frac": flops / mean_s / 1e12 / tc_peak}}

@@ -69,6 +69,8 @@ def lib():
         L.kla_chunk_bwd_workspace.restype = sz
         L.kla_chunk_bwd_workspace_min.argtypes = [i, i, i, i, i, i, i, i]
         L.kla_chunk_bwd_workspace_min.restype = sz
+        L.kla_chunk_bwd_reverse_segments.argtypes = [i, i, i, i, i, i, i]
+        L.kla_chunk_bwd_reverse_segments.restype = i
         L.kla_chunk_fwd_train.argtypes = [vp, vp, vp, fp, fp, f, fp, vp, fp, i, i, i, i, i, i, i, i, vp, sz, vp]
         L.kla_chunk_fwd_train.restype = i
         L.kla_chunk_bwd_after_train.argtypes = [vp, vp, vp, fp, fp, f, vp, fp, vp, vp, vp, fp, fp, fp,

@@ -272,6 +272,16 @@ size_t kla_chunk_bwd_workspace_min(int B, int T, int H, int Dk, int Dv, int chun
     return bwd_ws_layout(B, T, H, Dk, Dv, have_S_chunks != 0, off);
 }
 
+int kla_chunk_bwd_reverse_segments(int B, int T, int H, int Dk, int Dv, int chunk, int dtype) {
+    take_beta_flag(dtype);
+    if (B < 1 || H < 1 || T < 1 || chunk != kla::kChunkLen || !tc_bwd_shape(T, Dk, Dv, dtype)) return 0;
+    const int NC = (T + kla::kChunkLen - 1) / kla::kChunkLen;
+    const int ns = kla::reverse_nseg(B * H, NC);
+    if (ns <= 1) return 1;
+    const int segc = (NC + ns - 1) / ns;
+    return (NC + segc - 1) / segc;
+}
+
 size_t kla_chunk_bwd_workspace(int B, int T, int H, int Dk, int Dv, int chunk, int dtype,
                                int have_S_chunks) {
     take_beta_flag(dtype);

@@ -115,6 +115,15 @@ struct BwdDev {
     void *dq, *dk, *dv;
     float *deta, *dg, *dS0;
     int B, T, H;
+    // Reverse state pass over segments (long sequences over few heads).  mode 0: one run per
+    // head from dS_T.  mode 1 (transition pass, grid y = kind): per segment, kind 0 runs from
+    // lambda = 0 with dO, kind 1 from lambda = I without dO; the final lambda goes to
+    // MN[kind][head][nseg - 1 - seg] (reversed, so that the forward's segment scan chains them
+    // newest first).  mode 2 (output pass): per segment from Lstart[head][nseg - 1 - seg] (the
+    // scan's output), with the tile and dR stores; dS0 comes from the scan.
+    int mode, nseg, segc;
+    float* MN;
+    const float* Lstart;
 };
 
 // =====================================================================================
@@ -166,13 +175,21 @@ __global__ void __launch_bounds__(RT, 1)
     const int ch = (tid >> 7) & 1;  // half of every epilogue's columns
     const int H = a.H, T = a.T;
     const int NC = (T + CH - 1) / CH;
-    const int head = blockIdx.x, b = head / H, h = head % H;
+    const int nseg = a.mode == 0 ? 1 : a.nseg;
+    const int head = blockIdx.x / nseg, seg = blockIdx.x % nseg, b = head / H, h = head % H;
+    const int c_lo = a.mode == 0 ? 0 : seg * a.segc, c_hi = a.mode == 0 ? NC : min(NC, c_lo + a.segc);
+    const int nch = c_hi > c_lo ? c_hi - c_lo : 0;  // chunks of this run, processed newest first
+    const bool ident = a.mode == 1 && blockIdx.y == 1;  // transition from lambda = I, no dO
+    const bool need_do = !ident;
+    const bool outputs = a.mode != 1;                   // lambda tiles and dR for the gradient kernel
     const uint32_t sbase = smem_u32(sm);
     const uint32_t full0 = smem_u32(&ms->full[0]), freed0 = smem_u32(&ms->freed[0]);
     const uint32_t bar_u = smem_u32(&ms->bar_u), bar_s = smem_u32(&ms->bar_s), bar_r = smem_u32(&ms->bar_r);
     const uint32_t l_ready0 = smem_u32(&ms->l_ready[0]), u_ready0 = smem_u32(&ms->u_ready[0]),
                    gd_ready = smem_u32(&ms->gd_ready);
-    const float* dST = a.dS_T ? a.dS_T + (size_t)head * DK * DV : nullptr;
+    const float* dST = a.mode == 0 ? (a.dS_T ? a.dS_T + (size_t)head * DK * DV : nullptr)
+                                   : (a.mode == 2 ? a.Lstart + ((size_t)head * nseg + (nseg - 1 - seg)) * DK * DV
+                                                  : nullptr);
     uint8_t* Ltl = a.Ltl + (size_t)head * NC * 65536;
     float* dRh = a.dR + (size_t)head * NC * CH * DV;
 
@@ -196,9 +213,9 @@ __global__ void __launch_bounds__(RT, 1)
         tmem_alloc(smem_u32(&ms->tmem_base), 512);
         tmem_relinquish();
     }
-    if (warp < 2) {  // gamma_last of the newest chunk
-        const int t = (NC - 1) * CH + tid;
-        const float gv = t < T ? a.g[tok_index(b, t, h, T, H)] : 0.f;
+    if (warp < 2) {  // gamma_last of the run's newest chunk
+        const int t = (c_hi - 1) * CH + tid;
+        const float gv = (nch > 0 && t < T) ? a.g[tok_index(b, t, h, T, H)] : 0.f;
         const float sg = warp_sum(gv);
         if (lane == 0) ms->gsum[warp] = sg;
     }
@@ -214,30 +231,33 @@ __global__ void __launch_bounds__(RT, 1)
         if (lane == 0) {
             prefetch_tmap(&tm_q);
             prefetch_tmap(&tm_do);
-            constexpr uint32_t kBytes = 65536 + 16384 + REC_SCB + 4 * 8192;
+            // without dO (the identity transition) neither dO, Q nor T is needed
+            const uint32_t kBytes = 65536 + REC_SCB + (need_do ? 16384 + 4 * 8192 : 0);
             auto load = [&](int c, int st) {
                 const uint32_t bar = full0 + 8 * st;
                 const uint32_t base = sbase + st * R_STAGE;
                 const uint8_t* rec = a.recs + ((size_t)head * NC + c) * REC_BYTES;
                 mbar_expect_tx(bar, kBytes);
                 bulk_load(base + SR_W, rec + REC_W, 65536, bar);
-                bulk_load(base + SR_T, a.Ttl + ((size_t)head * NC + c) * 16384, 16384, bar);
                 bulk_load(sbase + R_SC + st * REC_SCB, rec + REC_SC, REC_SCB, bar);
-                tma_load_4d(base + SR_DO, &tm_do, bar, 0, h, c * CH, b);
-                tma_load_4d(base + SR_DO + 8192, &tm_do, bar, 64, h, c * CH, b);
-                tma_load_4d(base + SR_Q, &tm_q, bar, 0, h, c * CH, b);
-                tma_load_4d(base + SR_Q + 8192, &tm_q, bar, 64, h, c * CH, b);
+                if (need_do) {
+                    bulk_load(base + SR_T, a.Ttl + ((size_t)head * NC + c) * 16384, 16384, bar);
+                    tma_load_4d(base + SR_DO, &tm_do, bar, 0, h, c * CH, b);
+                    tma_load_4d(base + SR_DO + 8192, &tm_do, bar, 64, h, c * CH, b);
+                    tma_load_4d(base + SR_Q, &tm_q, bar, 0, h, c * CH, b);
+                    tma_load_4d(base + SR_Q + 8192, &tm_q, bar, 64, h, c * CH, b);
+                }
             };
             int requested = 0;  // chunks (in processing order) whose loads were issued
-            for (int i = 0; i < min(NC, 2); ++i) {
-                load(NC - 1 - i, i);
+            for (int i = 0; i < min(nch, 2); ++i) {
+                load(c_hi - 1 - i, i);
                 requested = i + 1;
             }
-            for (int lc = 0; lc + 2 < NC; ++lc) {
+            for (int lc = 0; lc + 2 < nch; ++lc) {
                 const int st = lc & 1;
                 // every MMA of chunk lc done (the epilogue's reads of the stage precede them)
                 if (!mbar_wait_bounded(freed0 + 8 * st, (lc >> 1) & 1, kWaitNs)) { aborted = true; break; }
-                load(NC - 1 - (lc + 2), st);
+                load(c_hi - 1 - (lc + 2), st);
                 requested = lc + 3;
             }
             if (aborted) {
@@ -256,20 +276,22 @@ __global__ void __launch_bounds__(RT, 1)
             const uint32_t i_q = idesc_bf16(128, 128, false, true);   // (gamma dO)^T x Q (MN-major)
             const uint32_t i_w = idesc_bf16(128, 128, false, true);   // dU^T x (-W) ([token][dk] tiles: MN-major)
             const uint32_t i_t = idesc_bf16(128, 64, false, true);    // dU^T x T (MN-major)
-            for (int lc = 0; lc < NC && !aborted; ++lc) {
+            for (int lc = 0; lc < nch && !aborted; ++lc) {
                 const int st = lc & 1;
                 const uint32_t stg = sbase + st * R_STAGE;
                 if (!mbar_wait_bounded(full0 + 8 * st, (lc >> 1) & 1, kWaitNs)) { aborted = true; break; }
                 tc_fence_after();
                 // dU^T = dO^T P (independent of lambda), then + lambda^T Ktil^T by halves of lambda
                 // (products hi x hi, hi x lo, lo x hi): K steps {0,1,4,5} read the first half of
-                // each thread's lambda columns
+                // each thread's lambda columns.  Without dO the first lambda product starts dU.
+                if (need_do) {
 #pragma unroll
-                for (int p = 0; p < 2; ++p)
+                    for (int p = 0; p < 2; ++p)
 #pragma unroll
-                    for (int s = 0; s < 4; ++s)
-                        mma_bf16(tmem + TR_U, smem_desc(stg + SR_DO + s * 2048, 8192, 1024),
-                                 smem_desc(stg + SR_P + p * 8192 + s * 2048, 8192, 1024), i_dop, (p | s) > 0);
+                        for (int s = 0; s < 4; ++s)
+                            mma_bf16(tmem + TR_U, smem_desc(stg + SR_DO + s * 2048, 8192, 1024),
+                                     smem_desc(stg + SR_P + p * 8192 + s * 2048, 8192, 1024), i_dop, (p | s) > 0);
+                }
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
                     if (!mbar_wait_bounded(l_ready0 + 8 * half, lc & 1, kWaitNs)) { aborted = true; break; }
@@ -282,20 +304,22 @@ __global__ void __launch_bounds__(RT, 1)
                             mma_bf16_ts(tmem + TR_U, tmem + (p == 2 ? TR_LL : TR_LH) + 8 * s,
                                         smem_desc(stg + (p == 1 ? SR_KTLO : SR_KT) + (s >> 2) * 8192 + (s & 3) * 32,
                                                   16, 1024),
-                                        i_lk, 1);
+                                        i_lk, (need_do || half > 0 || p > 0 || j > 0) ? 1u : 0u);
                         }
                 }
                 if (aborted) break;
                 mma_commit(bar_u);
                 // lambda^T += (gamma dO)^T Q, once gamma dO is in TMEM and the master rescaled
-                if (!mbar_wait_bounded(gd_ready, lc & 1, kWaitNs)) { aborted = true; break; }
-                tc_fence_after();
+                if (need_do) {
+                    if (!mbar_wait_bounded(gd_ready, lc & 1, kWaitNs)) { aborted = true; break; }
+                    tc_fence_after();
 #pragma unroll
-                for (int p = 0; p < 2; ++p)
+                    for (int p = 0; p < 2; ++p)
 #pragma unroll
-                    for (int s = 0; s < 4; ++s)
-                        mma_bf16_ts(tmem + TR_L, tmem + (p ? TR_GL : TR_GH) + 8 * s,
-                                    smem_desc(stg + SR_Q + s * 2048, 8192, 1024), i_q, 1);
+                        for (int s = 0; s < 4; ++s)
+                            mma_bf16_ts(tmem + TR_L, tmem + (p ? TR_GL : TR_GH) + 8 * s,
+                                        smem_desc(stg + SR_Q + s * 2048, 8192, 1024), i_q, 1);
+                }
                 // lambda^T += dU^T (-W): token steps {0,2} (first half of each thread's tokens),
                 // then {1,3}; dU hi and lo against the one-bf16 W
 #pragma unroll
@@ -313,16 +337,18 @@ __global__ void __launch_bounds__(RT, 1)
                 }
                 if (aborted) break;
                 mma_commit(bar_s);
-                // dR^T = dU^T T: products hi x hi, hi x lo, lo x hi
-                const uint32_t ua[3] = {TR_UH, TR_UH, TR_UL};
-                const uint32_t tb[3] = {stg + SR_T, stg + SR_T + 8192, stg + SR_T};
+                // dR^T = dU^T T: products hi x hi, hi x lo, lo x hi (only for the gradient kernel)
+                if (outputs) {
+                    const uint32_t ua[3] = {TR_UH, TR_UH, TR_UL};
+                    const uint32_t tb[3] = {stg + SR_T, stg + SR_T + 8192, stg + SR_T};
 #pragma unroll
-                for (int p = 0; p < 3; ++p)
+                    for (int p = 0; p < 3; ++p)
 #pragma unroll
-                    for (int s = 0; s < 4; ++s)
-                        mma_bf16_ts(tmem + TR_R, tmem + ua[p] + 8 * s, smem_desc(tb[p] + s * 2048, 8192, 1024), i_t,
-                                    (p | s) > 0);
-                mma_commit(bar_r);
+                        for (int s = 0; s < 4; ++s)
+                            mma_bf16_ts(tmem + TR_R, tmem + ua[p] + 8 * s, smem_desc(tb[p] + s * 2048, 8192, 1024),
+                                        i_t, (p | s) > 0);
+                    mma_commit(bar_r);
+                }
                 mma_commit(freed0 + 8 * st);
             }
             if (aborted) atomicOr(&ms->abort, 1u);
@@ -339,7 +365,8 @@ __global__ void __launch_bounds__(RT, 1)
                 const int dk0 = 64 * ch + 32 * q2;
                 float x[32];
 #pragma unroll
-                for (int e = 0; e < 32; ++e) x[e] = dST ? dST[(size_t)(dk0 + e) * DV + row] : 0.f;
+                for (int e = 0; e < 32; ++e)
+                    x[e] = ident ? (dk0 + e == row ? 1.f : 0.f) : (dST ? dST[(size_t)(dk0 + e) * DV + row] : 0.f);
                 uint32_t hp[16], lp[16];
                 split_pack<32>(x, hp, lp);
                 tmem_st16u(tmem + lane_base + TR_LH + 32 * ch + 16 * q2, hp);
@@ -360,6 +387,7 @@ __global__ void __launch_bounds__(RT, 1)
             if (__any_sync(0xffffffffu, !ok)) return false;
             const float* sc = reinterpret_cast<const float*>(sm + R_SC + st2 * REC_SCB);
             gprev = sc[CH + 1];
+            if (!need_do) return true;
             const uint8_t* dob = sm + st2 * R_STAGE + SR_DO + (row >> 6) * 8192;
             float x[32];
 #pragma unroll
@@ -374,10 +402,10 @@ __global__ void __launch_bounds__(RT, 1)
             epi_signal(gd_ready, tid);
             return true;
         };
-        if (!gamma_do(0)) aborted = true;
-        for (int lc = 0; lc < NC && !aborted; ++lc) {
-            const int c = NC - 1 - lc;
-            const bool has_next = c > 0;
+        if (nch > 0 && !gamma_do(0)) aborted = true;
+        for (int lc = 0; lc < nch && !aborted; ++lc) {
+            const int c = c_hi - 1 - lc;
+            const bool has_next = lc + 1 < nch;
             // ---- dU epilogue: hi/lo A operands, released in two halves of 16 tokens
             {
                 const bool ok = mbar_wait_bounded(bar_u, lc & 1, kWaitNs);
@@ -395,8 +423,9 @@ __global__ void __launch_bounds__(RT, 1)
                     epi_signal(u_ready0 + 8 * half, tid);
                 }
                 // lambda_c (still the dU product's operand) to its tiles while the W product runs
-                st_tmem_row_global(tmem + lane_base + TR_LH + 32 * ch, tmem + lane_base + TR_LL + 32 * ch,
-                                   Ltl + (size_t)c * 65536 + ch * 16384, 32768, row);
+                if (outputs)
+                    st_tmem_row_global(tmem + lane_base + TR_LH + 32 * ch, tmem + lane_base + TR_LL + 32 * ch,
+                                       Ltl + (size_t)c * 65536 + ch * 16384, 32768, row);
             }
             // ---- lambda epilogue: hi/lo of the next chunk's lambda in two halves, the master
             //      pre-scaled by gamma_last of chunk c - 1, the next chunk's gamma dO
@@ -434,7 +463,7 @@ __global__ void __launch_bounds__(RT, 1)
                 }
             }
             // ---- dR epilogue: dR as [token][dv] rows to the workspace
-            {
+            if (outputs) {
                 const bool ok = mbar_wait_bounded(bar_r, lc & 1, kWaitNs);
                 if (__any_sync(0xffffffffu, !ok)) { aborted = true; break; }
                 tc_fence_after();
@@ -453,9 +482,12 @@ __global__ void __launch_bounds__(RT, 1)
     __syncthreads();
     if (ms->abort) {
         if (tid == 0) atomicOr(&g_bwd_error, 1u);
-    } else if (warp < kRIssuer) {
+    } else if (warp < kRIssuer && a.mode != 2) {
         tc_fence_after();
-        float* dS0 = a.dS0 + (size_t)head * DK * DV;
+        // the gradient of the run's oldest state: dS0, or the segment's map in the transition pass
+        float* dS0 = a.mode == 0 ? a.dS0 + (size_t)head * DK * DV
+                                 : a.MN + (((size_t)blockIdx.y * (gridDim.x / nseg) + head) * nseg + (nseg - 1 - seg)) *
+                                              DK * DV;
 #pragma unroll 1
         for (int q2 = 0; q2 < 2; ++q2) {
             const int dk0 = 64 * ch + 32 * q2;
@@ -1014,10 +1046,13 @@ done:
 size_t align1k(size_t x) { return (x + 1023) & ~size_t(1023); }
 
 struct BwdLayout {
-    size_t fwd, T, S, U, L, dR, total;
+    size_t fwd, T, S, U, L, dR, seg, total;
+    int nseg, segc;
 };
 
-// [forward records | T tiles | S tiles | U tiles | lambda tiles | dR], each 1 KB aligned
+// [forward records | T tiles | S tiles | U tiles | lambda tiles | dR | segment maps], each 1 KB
+// aligned; the segment maps ([2, BH, nseg] + [BH, nseg] states) only when the reverse state pass
+// runs in segments (long sequences over few heads: the forward's cost model)
 BwdLayout bwd_layout(int B, int T, int H) {
     FwdArgs fa{};
     fa.B = B;
@@ -1039,6 +1074,16 @@ BwdLayout bwd_layout(int B, int T, int H) {
     o += align1k(nch * 65536);
     L.dR = o;
     o += align1k(nch * CH * DV * sizeof(float));
+    L.seg = o;
+    const int NC = (T + CH - 1) / CH;
+    const int ns = reverse_nseg(B * H, NC);
+    L.nseg = 1;
+    L.segc = NC;
+    if (ns > 1) {
+        L.segc = (NC + ns - 1) / ns;
+        L.nseg = (NC + L.segc - 1) / L.segc;
+        o += align1k((size_t)3 * B * H * L.nseg * DK * DV * sizeof(float));
+    }
     L.total = o;
     return L;
 }
@@ -1107,8 +1152,29 @@ cudaError_t launch_chunk_bwd_tc_reverse(const BwdTcArgs& a, void* ws, size_t ws_
     cudaError_t e =
         cudaFuncSetAttribute(chunk_bwd_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)R_SMEM);
     if (e != cudaSuccess) return e;
-    chunk_bwd_state_kernel<<<BH, RT, R_SMEM, st>>>(mq, mdo, d);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (L.nseg <= 1) {
+        d.mode = 0;
+        chunk_bwd_state_kernel<<<BH, RT, R_SMEM, st>>>(mq, mdo, d);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    } else {
+        // transition pass (each segment's map from lambda = I and its offset from lambda = 0),
+        // the scan newest segment first (dS_T in, every segment's lambda_end and dS0 out), then
+        // each segment's pass from its lambda_end with the tile stores
+        const size_t SZ = (size_t)DK * DV;
+        float* MN = reinterpret_cast<float*>(w + L.seg);  // [2, BH, nseg, DK, DV]
+        float* Lst = MN + 2 * (size_t)BH * L.nseg * SZ;    // [BH, nseg, DK, DV]
+        d.nseg = L.nseg;
+        d.segc = L.segc;
+        d.MN = MN;
+        d.Lstart = Lst;
+        d.mode = 1;
+        chunk_bwd_state_kernel<<<dim3(BH * L.nseg, 2), RT, R_SMEM, st>>>(mq, mdo, d);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        if ((e = launch_seg_scan(a.dS_T, MN, Lst, a.dS0, BH, L.nseg, st)) != cudaSuccess) return e;
+        d.mode = 2;
+        chunk_bwd_state_kernel<<<dim3(BH * L.nseg, 1), RT, R_SMEM, st>>>(mq, mdo, d);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
     return a.out_bf16 ? launch_grad<__nv_bfloat16>(mq, mk, mdo, d, NC, BH, st)
                       : launch_grad<float>(mq, mk, mdo, d, NC, BH, st);
 }

@@ -1101,6 +1101,8 @@ int chunk_fwd_split_launches(const FwdArgs& a) {
     return L.nseg > 1 ? 4 : (L.nc1 > 0 ? 4 : 2);
 }
 
+int reverse_nseg(int BH, int NC) { return choose_nseg_split(BH, NC); }
+
 cudaError_t split_take_error(cudaStream_t st, unsigned int* flag) {
     cudaError_t e = cudaStreamSynchronize(st);
     if (e != cudaSuccess) return e;

@@ -157,6 +157,9 @@ int chunk_fwd_split_launches(const FwdArgs& a);
 cudaError_t launch_chunk_fwd_split_prep(const FwdArgs& a, void* ws, cudaStream_t st);
 cudaError_t launch_chunk_fwd_split_state(const FwdArgs& a, void* ws, cudaStream_t st);
 cudaError_t split_take_error(cudaStream_t st, unsigned int* flag);
+// Segments of the backward's reverse state pass for BH heads of NC chunks (1: one run per head);
+// the forward state pass's cost model, which the reverse pass shares.
+int reverse_nseg(int BH, int NC);
 // Synchronise `st`, then read and clear the device error word of the tensor-core kernels
 // (non-zero when a bounded wait expired).
 cudaError_t tc_take_error(cudaStream_t st, unsigned int* flag);

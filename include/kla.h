@@ -157,13 +157,20 @@ kla_status kla_chunk_fwd_state(const void *q, const float *g, const float *S0, v
  * KLA_ERR_WORKSPACE).  With at least kla_chunk_bwd_workspace() bytes, bf16 inputs with
  * Dk == Dv == 128 run on the tensor cores: the split forward's preparation and state pass are
  * recomputed into ws (about 305 KiB per chunk and head; S_chunks is then not read), a reverse
- * state pass carries the state gradient chunk by chunk, and a chunk-parallel kernel forms every
- * gradient.  With less, and for every other shape, the CUDA-core backward runs.
+ * state pass carries the state gradient chunk by chunk (in parallel segments chained by a scan
+ * for long sequences over few heads: kla_chunk_bwd_reverse_segments), and a chunk-parallel
+ * kernel forms every gradient.  With less, and for every other shape, the CUDA-core backward runs.
  * The workspace must not be shared with a concurrent call.
  * Every output is fully overwritten.
  */
 size_t kla_chunk_bwd_workspace(int B, int T, int H, int Dk, int Dv, int chunk, int dtype,
                                int have_S_chunks);
+/* Segments of the tensor-core backward's reverse state pass for these shapes: 1 for one run per
+ * head; more when the sequences are long and the heads few (each segment's map of the state
+ * gradient in parallel, a scan over segments newest first, then every segment's pass from its
+ * true end gradient, as for the forward's segmented state pass); 0 for shapes without the
+ * tensor-core backward. */
+int kla_chunk_bwd_reverse_segments(int B, int T, int H, int Dk, int Dv, int chunk, int dtype);
 size_t kla_chunk_bwd_workspace_min(int B, int T, int H, int Dk, int Dv, int chunk, int dtype,
                                    int have_S_chunks);
 kla_status kla_chunk_bwd(const void *q, const void *k, const void *v, const float *eta,

@@ -182,3 +182,14 @@ def test_forward_launch_plan(L):
         assert L.kla_chunk_fwd_kernel_launches(B, T, H, 128, 128, 64, 1) == n, (B, T, H)
     assert L.kla_chunk_fwd_kernel_launches(1, 300, 2, 64, 64, 64, 0) == 1  # fp32 d = 64: one kernel
     assert L.kla_chunk_fwd_kernel_launches(0, 300, 2, 128, 128, 64, 1) == 0  # invalid shape
+
+
+def test_backward_reverse_segments(L):
+    """The reverse state pass is segmented exactly where the forward's cost model segments the
+    forward state pass: long sequences over few heads; one run for the workloads' other shapes."""
+    assert L.kla_chunk_bwd_reverse_segments(8, 2048, 8, 128, 128, 64, 1) == 1
+    assert L.kla_chunk_bwd_reverse_segments(4, 4096, 16, 128, 128, 64, 1) == 1
+    assert L.kla_chunk_bwd_reverse_segments(1, 65536, 16, 128, 128, 64, 1) > 1
+    assert L.kla_chunk_bwd_reverse_segments(1, 4100, 2, 128, 128, 64, 1) > 1
+    assert L.kla_chunk_bwd_reverse_segments(1, 4100, 2, 64, 64, 64, 1) == 0  # no tensor-core backward
+    assert L.kla_chunk_bwd_reverse_segments(1, 4100, 2, 128, 128, 64, 0) == 0

@@ -468,6 +468,29 @@ def test_bwd_zero_norm_keys_exact(kla, oracle_mod, Dk, Dv, dtype, beta, eps, cud
             assert rel_err(got[zmask], want[zmask]) <= tol, "dk, zero-norm keys"
 
 
+@pytest.mark.parametrize("T,H,s0,with_dST", [(4100, 2, True, True), (3000, 3, False, False)])
+def test_bwd_segmented_reverse_pass(kla, oracle_mod, T, H, s0, with_dST):
+    """Long sequences over few heads run the reverse state pass in segments: each segment's map
+    of the state gradient (from lambda = I without dO) and offset (from lambda = 0 with dO) in
+    parallel, a scan newest segment first, then each segment from its true end gradient.  Every
+    gradient against the oracle (a ragged tail chunk in the first shape)."""
+    nseg = kla.lib().kla_chunk_bwd_reverse_segments(1, T, H, 128, 128, 64, 1)
+    assert nseg > 1
+    inp = small_inputs(1, T, H, 128, 128, "bf16", seed=T + H, s0=s0, g_lo=-0.05)
+    gen = torch.Generator().manual_seed(T)
+    dO = torch.randn(1, T, H, 128, generator=gen).to(torch.bfloat16)
+    dST = torch.randn(1, H, 128, 128, generator=gen) if with_dST else None
+    d = {k: (v.cuda() if v is not None else None) for k, v in inp.items()}
+    gr = kla.chunk_bwd(d["q"], d["k"], d["v"], d["eta"], d["g"], dO.cuda(), 1e-6, d["S0"],
+                       dST.cuda() if dST is not None else None)
+    torch.cuda.synchronize()
+    kla.check_device_error()
+    ref = oracle_mod.backward(*(np64(inp[k]) for k in ("q", "k", "v", "eta", "g")), 1e-6, np64(inp["S0"]),
+                              np64(dO), np64(dST))
+    for name in GRADS:
+        assert rel_err(gr[name], ref[name]) <= 2e-2, name
+
+
 def test_bwd_tensor_cores_more_heads_than_sms(kla, oracle_mod):
     B, T, H = 10, 70, 16  # 160 reverse-pass CTAs: more than one wave
     inp = small_inputs(B, T, H, 128, 128, "bf16", seed=77)
