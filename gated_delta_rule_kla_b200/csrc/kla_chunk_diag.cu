@@ -803,20 +803,22 @@ __global__ void diag_dg_kernel(BwdArgs a) {
 template <int DK, int DV, typename Tin>
 __global__ void __launch_bounds__(NT) diag_prep_kernel(FwdArgs a, float* __restrict__ recs) {
     using R = DiagRec<DK, DV>;
-    constexpr int LDK = DK + 1, LDC = CD + 1, LDV = DV + 1;
+    constexpr int LDK = DK + 1, LDC = CD + 1;
+    constexpr int NR = DK + DV + CD;  // right-hand sides: Diag(b)(Khat o Gam) | Diag(c) V | I
+    constexpr int LDR = NR + 1;
+    constexpr int NQ = 4;             // channel quarters of the Gram sums
     extern __shared__ float sm[];
     float* Ks = sm;               // CD x LDK  unit keys
     float* Qs = Ks + CD * LDK;    // CD x LDK  queries
-    float* Bk = Qs + CD * LDK;    // CD x LDK  b_j khat_j o Gam_j
-    float* Gs = Bk + CD * LDK;    // CD x DK   log-decay prefix
-    float* Vs = Gs + CD * DK;     // CD x LDV  c_j v_j
-    float* Am = Vs + CD * LDV;    // CD x LDC
-    float* Pm = Am + CD * LDC;    // CD x LDC
-    float* Tm = Pm + CD * LDC;    // CD x LDC  T = (I + L)^{-1}
-    float* bs = Tm + CD * LDC;
+    float* Gs = Qs + CD * LDK;    // CD x DK   log-decay prefix
+    float* Rs = Gs + CD * DK;     // CD x LDR  right-hand sides, solved in place: W | UP | T
+    float* Ap = Rs + CD * LDR;    // NQ x NP   partial Gram sums (A), then
+    float* Pp = Ap + NQ * NP;     // NQ x NP   (P)
+    float* Am = Pp + NQ * NP;     // CD x LDC  A (strictly lower)
+    float* bs = Am + CD * LDC;
     float* cs = bs + CD;
 
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int tid = threadIdx.x;
     const int ci = blockIdx.x, head = blockIdx.y;
     const int b = head / a.H, h = head % a.H;
     const int NC = (a.T + CD - 1) / CD;
@@ -827,66 +829,78 @@ __global__ void __launch_bounds__(NT) diag_prep_kernel(FwdArgs a, float* __restr
     load_rows<DK, Tin>(a, b, h, t0, n, Ks, Qs, Gs, bs, cs, nullptr);
     __syncthreads();
     cumsum_rows<DK>(Gs);
-    for (int x = tid; x < CD * DV; x += NT) {
+    for (int x = tid; x < CD * DV; x += NT) {  // Diag(c) V
         const int i = x / DV, j = x % DV;
-        Vs[i * LDV + j] = i < n ? cs[i] * to_f32(v[tok_index(b, t0 + i, h, a.T, a.H) * DV + j]) : 0.f;
+        Rs[i * LDR + DK + j] = i < n ? cs[i] * to_f32(v[tok_index(b, t0 + i, h, a.T, a.H) * DV + j]) : 0.f;
     }
+    for (int x = tid; x < CD * CD; x += NT) Rs[(x / CD) * LDR + DK + DV + x % CD] = (x / CD == x % CD) ? 1.f : 0.f;
     __syncthreads();
-    chunk_grams<DK>(Ks, Qs, Gs, Am, Pm, nullptr);
-    // elementwise operands: Bk (for W), and the QG, KD, GC records
+    // Gram sums over one channel quarter per item: A_ij = sum_c khat_i khat_j E_ij (j < i),
+    // P_ij = sum_c q_i khat_j E_ij (j <= i); elementwise operands and the QG, KD, GC records
+    for (int it = tid; it < NQ * NP; it += NT) {
+        const int p = it % NP, qd = it / NP;
+        int i = 0;
+        while ((i + 1) * (i + 2) / 2 <= p) ++i;
+        const int j = p - i * (i + 1) / 2;
+        float sa0 = 0.f, sa1 = 0.f, sp0 = 0.f, sp1 = 0.f;
+        const int c0 = qd * (DK / NQ);
+#pragma unroll 4
+        for (int c = c0; c < c0 + DK / NQ; c += 2) {
+            const float e0 = __expf(Gs[i * DK + c] - Gs[j * DK + c]);
+            const float e1 = __expf(Gs[i * DK + c + 1] - Gs[j * DK + c + 1]);
+            const float k0 = Ks[j * LDK + c] * e0, k1 = Ks[j * LDK + c + 1] * e1;
+            sa0 = fmaf(Ks[i * LDK + c], k0, sa0);
+            sa1 = fmaf(Ks[i * LDK + c + 1], k1, sa1);
+            sp0 = fmaf(Qs[i * LDK + c], k0, sp0);
+            sp1 = fmaf(Qs[i * LDK + c + 1], k1, sp1);
+        }
+        Ap[qd * NP + p] = sa0 + sa1;
+        Pp[qd * NP + p] = sp0 + sp1;
+    }
     for (int x = tid; x < CD * DK; x += NT) {
         const int i = x / DK, c = x % DK;
         const float G = Gs[i * DK + c], Gl = Gs[(CD - 1) * DK + c];  // G is flat past the last token
         const float gam = __expf(G);
         const float kh = Ks[i * LDK + c];
-        Bk[i * LDK + c] = bs[i] * kh * gam;
+        Rs[i * LDR + c] = bs[i] * kh * gam;
         rec[R::QG + x] = Qs[i * LDK + c] * gam;
         rec[R::KD + x] = kh * __expf(Gl - G);
         if (i == 0) rec[R::GC + c] = __expf(Gl);
     }
     __syncthreads();
-    // T = (I + Diag(b) A)^{-1}: lane j of warp 0 builds column j by forward substitution;
-    // the other warps store P
-    if (warp == 0) {
-        if (lane < CD) {
-            const int j = lane;
-            float col[CD];
-#pragma unroll
-            for (int i = 0; i < CD; ++i) {
-                float s = 0.f;
-#pragma unroll
-                for (int m = 0; m < i; ++m) s = fmaf(Am[i * LDC + m], col[m], s);
-                col[i] = (i < j) ? 0.f : ((i == j) ? 1.f : -bs[i] * s);
-            }
-#pragma unroll
-            for (int i = 0; i < CD; ++i) Tm[i * LDC + j] = col[i];
+    // the quarters added in a fixed order: A to shared memory, P to the record
+    for (int x = tid; x < CD * CD; x += NT) {
+        const int i = x / CD, j = x % CD;
+        float av = 0.f, pv = 0.f;
+        if (j <= i) {
+            const int p = i * (i + 1) / 2 + j;
+            pv = (Pp[p] + Pp[NP + p]) + (Pp[2 * NP + p] + Pp[3 * NP + p]);
+            if (j < i) av = (Ap[p] + Ap[NP + p]) + (Ap[2 * NP + p] + Ap[3 * NP + p]);
         }
-    } else {
-        for (int x = tid - 32; x < CD * CD; x += NT - 32) rec[R::P + x] = Pm[(x / CD) * LDC + x % CD];
+        Am[i * LDC + j] = av;
+        rec[R::P + x] = pv;
     }
     __syncthreads();
-    // W = T Bk and UP = T Vs (T is unit lower triangular)
-    {
-        const int i = tid >> 4, cx = tid & 15;
-#pragma unroll 4
-        for (int u = 0; u < DK / 16; ++u) {
-            const int c = cx + 16 * u;
-            float s = 0.f;
-            for (int j = 0; j <= i; ++j) s = fmaf(Tm[i * LDC + j], Bk[j * LDK + c], s);
-            rec[R::W + i * DK + c] = s;
+    // (I + Diag(b) A) [W | UP | T] = [Diag(b)(Khat o Gam) | Diag(c) V | I], row by row
+    // (Appendix B.2), every column of the right-hand sides at once
+    for (int i = 1; i < n; ++i) {
+        const float bi = bs[i];
+        for (int col = tid; col < NR; col += NT) {
+            float sacc = 0.f;
+            for (int j = 0; j < i; ++j) sacc = fmaf(Am[i * LDC + j], Rs[j * LDR + col], sacc);
+            Rs[i * LDR + col] -= bi * sacc;
         }
-#pragma unroll 4
-        for (int u = 0; u < DV / 16; ++u) {
-            const int c = cx + 16 * u;
-            float s = 0.f;
-            for (int j = 0; j <= i; ++j) s = fmaf(Tm[i * LDC + j], Vs[j * LDV + c], s);
-            rec[R::UP + (c >> 6) * R::kSlice + i * 64 + (c & 63)] = s;
-        }
+        __syncthreads();
+    }
+    for (int x = tid; x < CD * DK; x += NT) rec[R::W + x] = Rs[(x / DK) * LDR + x % DK];
+    for (int x = tid; x < CD * DV; x += NT) {
+        const int i = x / DV, c = x % DV;
+        rec[R::UP + (c >> 6) * R::kSlice + i * 64 + (c & 63)] = Rs[i * LDR + DK + c];
     }
     if (a.rec_extras) {
         for (int x = tid; x < CD * CD; x += NT) {
             rec[R::XA + x] = Am[(x / CD) * LDC + x % CD];
-            rec[R::XT + x] = Tm[(x / CD) * LDC + x % CD];
+            rec[R::XT + x] = Rs[(x / CD) * LDR + DK + DV + x % CD];
         }
         for (int x = tid; x < CD * DK; x += NT) rec[R::XG + x] = Gs[x];
     }
@@ -894,29 +908,35 @@ __global__ void __launch_bounds__(NT) diag_prep_kernel(FwdArgs a, float* __restr
 
 template <int DK, int DV>
 constexpr size_t diag_prep_smem_bytes() {
-    return sizeof(float) * (3 * CD * (DK + 1) + CD * DK + CD * (DV + 1) + 3 * CD * (CD + 1) + 2 * CD);
+    return sizeof(float) * (2 * CD * (DK + 1) + CD * DK + CD * (DK + DV + CD + 1) + 8 * NP + CD * (CD + 1) + 2 * CD);
 }
 
 template <int DK, int DV>
 constexpr size_t diag_state_smem_bytes() {
     using R = DiagRec<DK, DV>;
-    return 128 + sizeof(float) * ((size_t)DK * 64 + 2 * (R::kHead + R::kSlice) + CD * 64) + 64;
+    return 128 + sizeof(float) * ((size_t)DK * 64 + 2 * (R::kHead + R::kSlice) + 3 * CD * 64) + 64;
 }
 
+constexpr int NTS = 512;  // state pass threads: two halves split every contraction
+
 template <int DK, int DV, typename TOut>
-__global__ void __launch_bounds__(NT, 1) diag_state_kernel(FwdArgs a, const float* __restrict__ recs) {
+__global__ void __launch_bounds__(NTS, 1) diag_state_kernel(FwdArgs a, const float* __restrict__ recs) {
     using R = DiagRec<DK, DV>;
     constexpr uint32_t kHeadBytes = R::kHead * 4, kSliceBytes = R::kSlice * 4;
     constexpr int kStage = R::kHead + R::kSlice;
+    constexpr int MH = DK / 32;  // state rows per thread in S' (each half takes every other 16-row block)
     static_assert(kHeadBytes % 16 == 0 && kSliceBytes % 16 == 0, "bulk copy sizes");
     extern __shared__ uint8_t smem_raw[];
     float* sm = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
     float* Ss = sm;                     // DK x 64 state slice
     float* stg = Ss + DK * 64;          // 2 stages: [record head | UP slice]
     float* Us = stg + 2 * kStage;       // CD x 64
-    uint64_t* full = reinterpret_cast<uint64_t*>(Us + CD * 64);
+    float* Pu = Us + CD * 64;           // CD x 64  second half's partial of -W S
+    float* Po = Pu + CD * 64;           // CD x 64  second half's partial of QG S
+    uint64_t* full = reinterpret_cast<uint64_t*>(Po + CD * 64);
 
     const int tid = threadIdx.x;
+    const int half = tid >> 8, t8 = tid & 255;
     const int sl = blockIdx.x, v0 = sl * 64, h = blockIdx.y, b = blockIdx.z;
     const int T = a.T, H = a.H;
     const int NC = (T + CD - 1) / CD;
@@ -938,13 +958,13 @@ __global__ void __launch_bounds__(NT, 1) diag_state_kernel(FwdArgs a, const floa
         fence_mbar_init();
         for (int c = 0; c < min(NC, 2); ++c) request(c, c);
     }
-    for (int x = tid; x < DK * 64; x += NT) {
+    for (int x = tid; x < DK * 64; x += NTS) {
         const int r = x >> 6, c = x & 63;
         Ss[x] = a.S0 ? a.S0[sbase + (size_t)r * DV + v0 + c] : 0.f;
     }
     __syncthreads();
 
-    const int i = tid >> 4, cx = 4 * (tid & 15);  // row (token) and the four columns of this thread
+    const int i = t8 >> 4, cx = 4 * (t8 & 15);  // row (token) and the four columns of this thread
     bool ok = true;
     for (int ci = 0; ci < NC; ++ci) {
         const int st = ci & 1;
@@ -954,20 +974,20 @@ __global__ void __launch_bounds__(NT, 1) diag_state_kernel(FwdArgs a, const floa
         const float* rs = stg + st * kStage;
         if (a.S_chunks) {
             float* dst = a.S_chunks + (head * NC + ci) * DK * DV;
-            for (int x = tid; x < DK * 16; x += NT) {
+            for (int x = tid; x < DK * 16; x += NTS) {
                 const int r = x >> 4, c4 = 4 * (x & 15);
                 *reinterpret_cast<float4*>(dst + (size_t)r * DV + v0 + c4) =
                     *reinterpret_cast<const float4*>(Ss + r * 64 + c4);
             }
         }
-        // U = UP - W S and O1 = QG S (row i, columns cx .. cx + 3)
-        float4 u = *reinterpret_cast<const float4*>(rs + R::kHead + i * 64 + cx);
-        float4 oo = make_float4(0.f, 0.f, 0.f, 0.f);
+        // -W S and QG S over this half's state rows d in [half DK/2, half DK/2 + DK/2)
+        float4 u = make_float4(0.f, 0.f, 0.f, 0.f), oo = u;
         {
             const float* wr = rs + R::W + i * DK;
             const float* qr = rs + R::QG + i * DK;
+            const int d0 = half * (DK / 2);
 #pragma unroll 8
-            for (int d = 0; d < DK; ++d) {
+            for (int d = d0; d < d0 + DK / 2; ++d) {
                 const float w = wr[d], q = qr[d];
                 const float4 s4 = *reinterpret_cast<const float4*>(Ss + d * 64 + cx);
                 u.x = fmaf(-w, s4.x, u.x); u.y = fmaf(-w, s4.y, u.y);
@@ -976,10 +996,22 @@ __global__ void __launch_bounds__(NT, 1) diag_state_kernel(FwdArgs a, const floa
                 oo.z = fmaf(q, s4.z, oo.z); oo.w = fmaf(q, s4.w, oo.w);
             }
         }
-        *reinterpret_cast<float4*>(Us + i * 64 + cx) = u;
+        if (half) {
+            *reinterpret_cast<float4*>(Pu + i * 64 + cx) = u;
+            *reinterpret_cast<float4*>(Po + i * 64 + cx) = oo;
+        }
         __syncthreads();
-        // O = O1 + P U (row i)
-        if (o != nullptr) {
+        if (!half) {  // U = UP + both halves of -W S
+            const float4 up = *reinterpret_cast<const float4*>(rs + R::kHead + i * 64 + cx);
+            const float4 pu = *reinterpret_cast<const float4*>(Pu + i * 64 + cx);
+            u = make_float4(up.x + u.x + pu.x, up.y + u.y + pu.y, up.z + u.z + pu.z, up.w + u.w + pu.w);
+            *reinterpret_cast<float4*>(Us + i * 64 + cx) = u;
+        }
+        __syncthreads();
+        // O = O1 + P U (row i; the first half adds the second half's O1 partial and stores)
+        if (!half && o != nullptr) {
+            const float4 po = *reinterpret_cast<const float4*>(Po + i * 64 + cx);
+            oo.x += po.x; oo.y += po.y; oo.z += po.z; oo.w += po.w;
             const float* pr = rs + R::P + i * CD;
 #pragma unroll
             for (int t = 0; t < CD; ++t) {
@@ -996,12 +1028,12 @@ __global__ void __launch_bounds__(NT, 1) diag_state_kernel(FwdArgs a, const floa
                 orow[3] = from_f32<TOut>(oo.w);
             }
         }
-        // S' = Diag(GC) S + KD^T U: rows i + 16 m of the state, columns cx .. cx + 3
+        // S' = Diag(GC) S + KD^T U: rows i + 16 (2 m + half) of the state, columns cx .. cx + 3
         {
-            float4 acc[DK / 16];
+            float4 acc[MH];
 #pragma unroll
-            for (int m = 0; m < DK / 16; ++m) {
-                const int r = i + 16 * m;
+            for (int m = 0; m < MH; ++m) {
+                const int r = i + 16 * (2 * m + half);
                 const float gcr = rs[R::GC + r];
                 const float4 s4 = *reinterpret_cast<const float4*>(Ss + r * 64 + cx);
                 acc[m] = make_float4(gcr * s4.x, gcr * s4.y, gcr * s4.z, gcr * s4.w);
@@ -1009,16 +1041,17 @@ __global__ void __launch_bounds__(NT, 1) diag_state_kernel(FwdArgs a, const floa
 #pragma unroll
             for (int t = 0; t < CD; ++t) {
                 const float4 ut = *reinterpret_cast<const float4*>(Us + t * 64 + cx);
-                const float* kd = rs + R::KD + t * DK + i;
+                const float* kd = rs + R::KD + t * DK + i + 16 * half;
 #pragma unroll
-                for (int m = 0; m < DK / 16; ++m) {
-                    const float w = kd[16 * m];
+                for (int m = 0; m < MH; ++m) {
+                    const float w = kd[32 * m];
                     acc[m].x = fmaf(w, ut.x, acc[m].x); acc[m].y = fmaf(w, ut.y, acc[m].y);
                     acc[m].z = fmaf(w, ut.z, acc[m].z); acc[m].w = fmaf(w, ut.w, acc[m].w);
                 }
             }
 #pragma unroll
-            for (int m = 0; m < DK / 16; ++m) *reinterpret_cast<float4*>(Ss + (i + 16 * m) * 64 + cx) = acc[m];
+            for (int m = 0; m < MH; ++m)
+                *reinterpret_cast<float4*>(Ss + (i + 16 * (2 * m + half)) * 64 + cx) = acc[m];
         }
         __syncthreads();  // the stage and Us are read: refill the stage
         if (tid == 0 && ci + 2 < NC) request(ci + 2, st);
@@ -1026,7 +1059,7 @@ __global__ void __launch_bounds__(NT, 1) diag_state_kernel(FwdArgs a, const floa
     if (!ok && tid == 0) atomicOr(&g_diag_error, 1u);
     __syncthreads();
     if (ok && a.S_T) {
-        for (int x = tid; x < DK * 16; x += NT) {
+        for (int x = tid; x < DK * 16; x += NTS) {
             const int r = x >> 4, c4 = 4 * (x & 15);
             *reinterpret_cast<float4*>(a.S_T + sbase + (size_t)r * DV + v0 + c4) =
                 *reinterpret_cast<const float4*>(Ss + r * 64 + c4);
@@ -1046,7 +1079,7 @@ cudaError_t diag_split_launch(const FwdArgs& a, void* ws, cudaStream_t st) {
     float* recs = static_cast<float*>(ws);
     diag_prep_kernel<DK, DV, Tin><<<dim3(NC, a.B * a.H), NT, ps, st>>>(a, recs);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    diag_state_kernel<DK, DV, TOut><<<dim3(DV / 64, a.H, a.B), NT, ss, st>>>(a, recs);
+    diag_state_kernel<DK, DV, TOut><<<dim3(DV / 64, a.H, a.B), NTS, ss, st>>>(a, recs);
     return cudaGetLastError();
 }
 

@@ -296,15 +296,17 @@ __global__ void __launch_bounds__(256) gate_bwd_tile_kernel(const Tin* __restric
                                                             const float* __restrict__ deta, const float* __restrict__ dg,
                                                             float* __restrict__ dx, float* __restrict__ part_w,
                                                             float* __restrict__ part_b, int N, int D, int H) {
+    // one CTA per (64-token tile, 128-column block of D)
     extern __shared__ float smf[];
     const int NW = 2 * H;
     float* dz = smf;                   // [BT][NW]
     float* xs = dz + BT * NW;          // [BT][BD + 1]
     float* wsh = xs + BT * (BD + 1);   // [NW][BD + 1]
     const int tid = threadIdx.x;
-    const int tile = blockIdx.x;
+    const int tile = blockIdx.x, d0 = blockIdx.y * BD;
     const int t0 = tile * BT;
     const int nt = min(BT, N - t0);
+    const int nd = min(BD, D - d0);
     for (int i = tid; i < BT * NW; i += 256) {
         const int t = i / NW, j = i % NW;
         float v = 0.f;
@@ -319,50 +321,48 @@ __global__ void __launch_bounds__(256) gate_bwd_tile_kernel(const Tin* __restric
         }
         dz[i] = v;
     }
+    // eight elements per access (D % 8 == 0, so a group of eight is either in range or not)
+    for (int i = tid; i < BT * (BD / 8); i += 256) {
+        const int t = i / (BD / 8), c8 = 8 * (i % (BD / 8));
+        float f[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        if (t < nt && c8 < nd) ld8(x + (size_t)(t0 + t) * D + d0 + c8, f);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) xs[t * (BD + 1) + c8 + e] = f[e];
+    }
+    for (int i = tid; i < NW * (BD / 8); i += 256) {
+        const int j = i / (BD / 8), c8 = 8 * (i % (BD / 8));
+        float f[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        if (c8 < nd) ld8(W + (size_t)j * D + d0 + c8, f);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) wsh[j * (BD + 1) + c8 + e] = f[e];
+    }
     __syncthreads();
-    if (tid < NW) {  // dbias partial, fixed order over the tile's tokens
+    if (blockIdx.y == 0 && tid < NW) {  // dbias partial, fixed order over the tile's tokens
         float s = 0.f;
         for (int t = 0; t < BT; ++t) s += dz[t * NW + tid];
         part_b[(size_t)tile * NW + tid] = s;
     }
-    for (int d0 = 0; d0 < D; d0 += BD) {
-        const int nd = min(BD, D - d0);
-        __syncthreads();
-        // eight elements per access (D % 8 == 0, so a group of eight is either in range or not)
-        for (int i = tid; i < BT * (BD / 8); i += 256) {
-            const int t = i / (BD / 8), c8 = 8 * (i % (BD / 8));
-            float f[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-            if (t < nt && c8 < nd) ld8(x + (size_t)(t0 + t) * D + d0 + c8, f);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) xs[t * (BD + 1) + c8 + e] = f[e];
-        }
-        for (int i = tid; i < NW * (BD / 8); i += 256) {
-            const int j = i / (BD / 8), c8 = 8 * (i % (BD / 8));
-            float f[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-            if (c8 < nd) ld8(W + (size_t)j * D + d0 + c8, f);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) wsh[j * (BD + 1) + c8 + e] = f[e];
-        }
-        __syncthreads();
-        // dx[t][c] = sum_j dz[t][j] W[j][c]: thread = column c (128) x token half
-        {
-            const int c = tid & (BD - 1), th = tid >> 7;
-            if (c < nd) {
-                for (int t = th; t < nt; t += 2) {
-                    float s = 0.f;
-                    for (int j = 0; j < NW; ++j) s = fmaf(dz[t * NW + j], wsh[j * (BD + 1) + c], s);
-                    dx[(size_t)(t0 + t) * D + d0 + c] = s;
-                }
-            }
-        }
-        // dW partial [j][c] = sum_t dz[t][j] x[t][c]
-        for (int i = tid; i < NW * BD; i += 256) {
-            const int j = i / BD, c = i % BD;
-            if (c < nd) {
+    // dx[t][c] = sum_j dz[t][j] W[j][c]: thread = column c (128) x token half
+    {
+        const int c = tid & (BD - 1), th = tid >> 7;
+        if (c < nd) {
+            for (int t = th; t < nt; t += 2) {
                 float s = 0.f;
-                for (int t = 0; t < BT; ++t) s = fmaf(dz[t * NW + j], xs[t * (BD + 1) + c], s);
-                part_w[((size_t)tile * NW + j) * D + d0 + c] = s;
+                for (int j = 0; j < NW; ++j) s = fmaf(dz[t * NW + j], wsh[j * (BD + 1) + c], s);
+                dx[(size_t)(t0 + t) * D + d0 + c] = s;
             }
+        }
+    }
+    // dW partial [j][c] = sum_t dz[t][j] x[t][c]
+    for (int i = tid; i < NW * BD; i += 256) {
+        const int j = i / BD, c = i % BD;
+        if (c < nd) {
+            float s0 = 0.f, s1 = 0.f;
+            for (int t = 0; t < BT; t += 2) {
+                s0 = fmaf(dz[t * NW + j], xs[t * (BD + 1) + c], s0);
+                s1 = fmaf(dz[(t + 1) * NW + j], xs[(t + 1) * (BD + 1) + c], s1);
+            }
+            part_w[((size_t)tile * NW + j) * D + d0 + c] = s0 + s1;
         }
     }
 }
@@ -463,13 +463,13 @@ cudaError_t launch_gate_prologue_bwd(const GateBwdArgs& a, void* ws, cudaStream_
         e = cudaFuncSetAttribute(gate_bwd_tile_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)smem);
         if (e != cudaSuccess) return e;
-        gate_bwd_tile_kernel<__nv_bfloat16><<<ntile, 256, smem, st>>>(
+        gate_bwd_tile_kernel<__nv_bfloat16><<<dim3(ntile, (a.D + BD - 1) / BD), 256, smem, st>>>(
             static_cast<const __nv_bfloat16*>(a.x), static_cast<const __nv_bfloat16*>(a.W), a.eta, a.g, a.deta, a.dg,
             a.dx, part_w, part_b, a.N, a.D, a.H);
     } else {
         e = cudaFuncSetAttribute(gate_bwd_tile_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        gate_bwd_tile_kernel<float><<<ntile, 256, smem, st>>>(static_cast<const float*>(a.x),
+        gate_bwd_tile_kernel<float><<<dim3(ntile, (a.D + BD - 1) / BD), 256, smem, st>>>(static_cast<const float*>(a.x),
                                                                static_cast<const float*>(a.W), a.eta, a.g, a.deta,
                                                                a.dg, a.dx, part_w, part_b, a.N, a.D, a.H);
     }
