@@ -24,7 +24,7 @@ def _rand(rng, N=7, D=5, H=3):
     return x, W, b
 
 
-def test_closed_forms():
+def check_closed_forms(og):
     x = np.zeros((2, 4))
     W = np.zeros((4, 4))
     eta, g = og.gates(x, W, np.zeros(4), 2)
@@ -35,8 +35,7 @@ def test_closed_forms():
     assert abs(eta[0, 0] - 0.75) < 1e-15 and abs(g[0, 0] + 1.0) < 1e-15
 
 
-@pytest.mark.parametrize("z", [40.0, 700.0])
-def test_asymptotics(z):
+def check_asymptotics(og, z):
     x = np.ones((1, 1))
     W = np.array([[z], [-z], [z], [-z]])
     eta, g = og.gates(x, W, np.zeros(4), 2)
@@ -48,7 +47,7 @@ def test_asymptotics(z):
     assert np.all(g <= 0) and np.all(eta >= 0) and np.all(eta <= 1)
 
 
-def test_logits_affine_in_the_token_and_per_head():
+def check_logits_affine_in_the_token_and_per_head(og):
     rng = np.random.default_rng(1)
     x, W, b = _rand(rng)
     H = 3
@@ -69,7 +68,7 @@ def test_logits_affine_in_the_token_and_per_head():
     assert np.array_equal(g3[:, [0, 1]], g4[:, [0, 1]]) and not np.allclose(g3[:, 2], g4[:, 2])
 
 
-def test_normalized_readout_is_algorithm1_line6(oracle_mod):
+def check_normalized_readout_is_algorithm1_line6(og, oracle_mod):
     """o computed from qhat equals o computed from q divided by ||q_t|| (per token and head),
     and qhat is invariant to positive rescaling of q; a zero query reads out zero."""
     rng = np.random.default_rng(2)
@@ -92,7 +91,7 @@ def test_normalized_readout_is_algorithm1_line6(oracle_mod):
     assert np.all(o_hat[0, 3, 1] == 0.0)
 
 
-def test_gates_backward_finite_differences():
+def check_gates_backward_finite_differences(og):
     rng = np.random.default_rng(3)
     H = 3
     x, W, b = _rand(rng, H=H)
@@ -117,7 +116,7 @@ def test_gates_backward_finite_differences():
         assert np.abs(gr[name] - fd).max() <= 1e-7 * max(1.0, np.abs(fd).max()), name
 
 
-def test_normalize_q_backward_finite_differences():
+def check_normalize_q_backward_finite_differences(og):
     rng = np.random.default_rng(4)
     q = rng.standard_normal((3, 2, 5))
     q[1, 0] = 0.0
@@ -134,3 +133,77 @@ def test_normalize_q_backward_finite_differences():
         fd[idx] = (np.sum(og.normalize_q(p) * dqh) - np.sum(og.normalize_q(m) * dqh)) / (2 * h)
     assert np.abs(dq - fd).max() <= 1e-7
     assert np.all(dq[1, 0] == 0.0)
+
+
+def test_closed_forms():
+    check_closed_forms(og)
+
+
+@pytest.mark.parametrize("z", [40.0, 700.0])
+def test_asymptotics(z):
+    check_asymptotics(og, z)
+
+
+def test_logits_affine_in_the_token_and_per_head():
+    check_logits_affine_in_the_token_and_per_head(og)
+
+
+def test_normalized_readout_is_algorithm1_line6(oracle_mod):
+    check_normalized_readout_is_algorithm1_line6(og, oracle_mod)
+
+
+def test_gates_backward_finite_differences():
+    check_gates_backward_finite_differences(og)
+
+
+def test_normalize_q_backward_finite_differences():
+    check_normalize_q_backward_finite_differences(og)
+
+
+# ---------------------------------------------------------------------------------------
+# Planted mistakes: each copy of oracle/gates.py below carries one plausible error; at least
+# one of the checks above must fail on it (so the pins above do pin the oracle).
+# ---------------------------------------------------------------------------------------
+MUTATIONS = [
+    ("sigmoid sign", "return np.where(z >= 0, 1.0 / (1.0 + e), e / (1.0 + e))",
+     "return np.where(z >= 0, e / (1.0 + e), 1.0 / (1.0 + e))"),
+    ("softplus drops max(z, 0)", "return np.maximum(z, 0.0) + np.log1p(np.exp(-np.abs(z)))",
+     "return np.log1p(np.exp(-np.abs(z)))"),
+    ("g without the minus", "return _sigmoid(z[:, :H]), -_softplus(z[:, H:])",
+     "return _sigmoid(z[:, :H]), _softplus(z[:, H:])"),
+    ("eta and g rows swapped", "return _sigmoid(z[:, :H]), -_softplus(z[:, H:])",
+     "return _sigmoid(z[:, H:]), -_softplus(z[:, :H])"),
+    ("bias dropped", "z = x @ W.T + bias\n    return _sigmoid", "z = x @ W.T\n    return _sigmoid"),
+    ("norm without sqrt", "n = np.sqrt(np.sum(q * q, axis=-1, keepdims=True))\n    return np.where",
+     "n = np.sum(q * q, axis=-1, keepdims=True)\n    return np.where"),
+    ("sigmoid' without (1 - s)", "deta * s_eta * (1.0 - s_eta)", "deta * s_eta"),
+    ("softplus' sign", "-dg * _sigmoid(z[:, H:])", "dg * _sigmoid(z[:, H:])"),
+    ("dW transposed product", "dW=dz.T @ x", "dW=(x.T @ dz).T * 0.5"),
+    ("dq without the projection", "dq = (dqhat - qh * np.sum(qh * dqhat, axis=-1, keepdims=True)) / safe",
+     "dq = dqhat / safe"),
+]
+
+
+@pytest.mark.parametrize("name,old,new", MUTATIONS, ids=[m[0] for m in MUTATIONS])
+def test_planted_mistake_is_caught(oracle_mod, name, old, new):
+    import importlib.util
+    import os
+    src = open(os.path.join(os.path.dirname(og.__file__), "gates.py")).read()
+    old, new = old.replace("\\n", "\n"), new.replace("\\n", "\n")
+    assert old in src, name
+    spec = importlib.util.spec_from_loader("gates_mutant", loader=None)
+    mut = importlib.util.module_from_spec(spec)
+    exec(compile(src.replace(old, new), "gates_mutant", "exec"), mut.__dict__)
+    checks = [lambda: check_closed_forms(mut), lambda: check_asymptotics(mut, 40.0),
+              lambda: check_asymptotics(mut, 700.0), lambda: check_logits_affine_in_the_token_and_per_head(mut),
+              lambda: check_normalized_readout_is_algorithm1_line6(mut, oracle_mod),
+              lambda: check_gates_backward_finite_differences(mut),
+              lambda: check_normalize_q_backward_finite_differences(mut)]
+    caught = 0
+    for c in checks:
+        try:
+            with np.errstate(all="ignore"):
+                c()
+        except (AssertionError, FloatingPointError, ValueError):
+            caught += 1
+    assert caught > 0, f"planted mistake not caught: {name}"
