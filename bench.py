@@ -72,25 +72,27 @@ def load_peaks():
     return dict(PEAKS_FALLBACK), "fallback"
 
 
-def kernel_source_hash():
-    """Hash of the CUDA sources; recorded ncu traffic is only valid for the same sources."""
+def kernel_source_hash(files=None):
+    """Hash of the CUDA sources a kernel is built from (all of csrc/ when `files` is None);
+    recorded ncu traffic is only valid for the same sources."""
     h = hashlib.sha256()
     cdir = os.path.join(ROOT, "gated_delta_rule_kla_b200", "csrc")
-    for f in sorted(os.listdir(cdir)):
+    for f in sorted(files if files is not None else os.listdir(cdir)):
         with open(os.path.join(cdir, f), "rb") as fh:
             h.update(f.encode() + fh.read())
     return h.hexdigest()[:16]
 
 
 def recorded_traffic(kernel_key):
-    """DRAM bytes per launch from the committed ncu summary, or None if stale/absent."""
+    """DRAM bytes per launch from the committed ncu summary, or None if stale/absent.  An entry
+    names the source files of its kernels (`sources`) and their hash at capture time."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         d = json.load(f)
     e = d.get(kernel_key)
-    if not e or e.get("source_hash") != kernel_source_hash():
+    if not e or e.get("source_hash") != kernel_source_hash(e.get("sources")):
         return None
     return e.get("dram_bytes_per_launch")
 
@@ -630,7 +632,8 @@ def bench_diag(kla, WORKLOADS, make_inputs, dev, stream, flush, rank, world, hbm
     alu = fp32_alu_peak_tflops(peaks)
     mean_f = statistics.mean(ms_f) / 1e3
     out = {"workload": w.name, "value": tokens / (tf_f / 1e3), "unit": "tokens/s", "steps": nf,
-           "ms_per_step": tf_f, "l2": "flushed between timed steps", "gpu_launches_per_step": 1,
+           "ms_per_step": tf_f, "l2": "flushed between timed steps",
+           "gpu_launches_per_step": 2 if L.kla_chunk_fwd_diag_workspace(w.B, w.T, w.H, w.Dk, w.Dv, 64, 1) > 0 else 1,
            "roofline": {"bound": "alu", "achieved": flops / mean_f / 1e12, "peak": alu, "unit": "TFLOP/s",
                         "frac": flops / mean_f / 1e12 / alu,
                         "peak_kind": "derived: 148 SMs x 128 fp32 FMA lanes x 2 x max SM clock",
