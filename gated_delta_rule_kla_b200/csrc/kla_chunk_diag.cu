@@ -43,7 +43,6 @@ constexpr int NT = 256;
 __device__ __forceinline__ size_t tok_index(int b, int t, int h, int T, int H) {
     return ((size_t)b * T + t) * H + h;
 }
-__device__ __forceinline__ int pair_index(int i, int j) { return i * (i + 1) / 2 + j; }
 
 // Rows of one 16-token chunk: unit keys, queries, raw log-decays (into Gs, summed afterwards)
 // and the per-token coefficients.  One warp per row; rows past the sequence are zero (they then
@@ -362,13 +361,15 @@ __global__ void __launch_bounds__(NT, 1) chunk_fwd_diag_kernel(FwdArgs a) {
 // partial sums of dq, dkhat, dG, db and dc go out by vector reductions into fp32 accumulators.
 // ------------------------------------------------------------------------------------
 constexpr int BLD = 68;  // row stride of the [rows][64] fp32 tiles (16-byte rows, 2-way banks)
+constexpr float kFactorLimit = 80.f;  // |G| below this: exp(+-G) and their products stay finite in fp32
 
-template <int DK, int DV>
+// Shared memory of the backward (floats, then the raw rows of the next chunk, then barriers).
+template <int DK, int DV, typename Tin>
 constexpr size_t diag_bwd_smem_bytes() {
     using R = DiagRec<DK, DV>;
-    return 128 + sizeof(float) * ((size_t)2 * DK * BLD + NP * DK + R::kHead + R::kExtra + CD * 64 +
-                                  2 * CD * (DK + 1) + 5 * CD * BLD + 2 * CD * (CD + 1) + DK + 4 * CD) +
-           NP * 2 + 32;
+    return 128 + sizeof(float) * ((size_t)2 * DK * BLD + 6 * CD * DK + R::kHead + R::kExtra + CD * 64 +
+                                  2 * CD * (DK + 1) + 5 * CD * BLD + 2 * CD * (CD + 1) + DK + 5 * CD) +
+           sizeof(Tin) * (size_t)CD * (2 * DK + 128) + 16 + 3 * 8;
 }
 
 __device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d) {
@@ -376,6 +377,14 @@ __device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, 
                  : "memory");
 }
 
+// Per chunk the pairwise factors E_ij = exp(G_i - G_j) enter the F terms only through products
+// with per-token rows, so while every |G| of the chunk is below kFactorLimit they are taken as
+// exp(G_i) exp(-G_j):
+//   F1_i = Gam_i o sum_{j<=i} Y_ij (khat_j o Gam_j^-1)      F3_i likewise with D
+//   F2_j = Gam_j^-1 o sum_{i>=j} Y_ij (q_i o Gam_i)         F4_j = Gam_j^-1 o sum_{i>j} D_ij b_i (khat_i o Gam_i)
+// (q o Gam is the record's QG).  A chunk with a wider range forms each E_ij on the fly instead.
+// The rows of the next chunk (k, q, and this CTA's v and dO columns) come in by bulk copies
+// while the current one is worked on.
 template <int DK, int DV, typename Tin, typename TOut>
 __global__ void __launch_bounds__(NT, 1) diag_bwd_kernel(BwdArgs a, FwdArgs f, const float* __restrict__ recs) {
     using R = DiagRec<DK, DV>;
@@ -385,8 +394,13 @@ __global__ void __launch_bounds__(NT, 1) diag_bwd_kernel(BwdArgs a, FwdArgs f, c
     float* sm = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
     float* Ss = sm;                      // DK x BLD  incoming state slice
     float* Ls = Ss + DK * BLD;           // DK x BLD  lambda slice
-    float* Es = Ls + DK * BLD;           // NP x DK   E_ij, then the results [3][CD][DK]
-    float* Rh = Es + NP * DK;            // record head: W, QG, KD, P, GC
+    float* Rq = Ls + DK * BLD;           // CD x DK   results: dq, dkhat, dG, last-token terms
+    float* Rk = Rq + CD * DK;
+    float* Rg = Rk + CD * DK;
+    float* Rxs = Rg + CD * DK;
+    float* KiG = Rxs + CD * DK;          // CD x DK   khat o Gam^-1
+    float* KG = KiG + CD * DK;           // CD x DK   khat o Gam
+    float* Rh = KG + CD * DK;            // record head: W, QG, KD, P, GC
     float* Rx = Rh + R::kHead;           // record extras: A, T, G
     float* UPs = Rx + R::kExtra;         // CD x 64   UP slice
     float* Kh = UPs + CD * 64;           // CD x LDK  unit keys
@@ -403,22 +417,28 @@ __global__ void __launch_bounds__(NT, 1) diag_bwd_kernel(BwdArgs a, FwdArgs f, c
     float* cs = bs + CD;
     float* us = cs + CD;
     float* dbs = us + CD;
-    uint8_t* pij = reinterpret_cast<uint8_t*>(dbs + CD);  // NP x (i, j)
-    uint64_t* bars = reinterpret_cast<uint64_t*>(((reinterpret_cast<uintptr_t>(pij + 2 * NP)) + 15) & ~uintptr_t(15));
+    float* etaS = dbs + CD;
+    Tin* Kraw = reinterpret_cast<Tin*>((reinterpret_cast<uintptr_t>(etaS + CD) + 15) & ~uintptr_t(15));
+    Tin* Qraw = Kraw + CD * DK;          // raw rows of the next chunk: k, q [CD][DK]
+    Tin* Vraw = Qraw + CD * DK;          // v, dO columns v0 .. v0 + 63 [CD][64]
+    Tin* Oraw = Vraw + CD * 64;
+    uint64_t* bars = reinterpret_cast<uint64_t*>((reinterpret_cast<uintptr_t>(Oraw + CD * 64) + 15) & ~uintptr_t(15));
 
-    const int tid = threadIdx.x, lane = tid & 31;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int sl = blockIdx.x, v0 = sl * 64, h = blockIdx.y, b = blockIdx.z;
     const int T = a.T, H = a.H;
     const int NC = (T + CD - 1) / CD;
     const size_t head = (size_t)b * H + h;
     const size_t sbase = head * DK * DV;
     const float* hrec = recs + head * NC * R::kFloats;
+    const Tin* kin = static_cast<const Tin*>(f.k);
+    const Tin* qin = static_cast<const Tin*>(f.q);
     const Tin* v = static_cast<const Tin*>(a.v);
     const Tin* dO = static_cast<const Tin*>(a.dO);
     TOut* dv = static_cast<TOut*>(a.dv);
-    const uint32_t bar_r = smem_u32(&bars[0]), bar_s = smem_u32(&bars[1]);
+    const uint32_t bar_r = smem_u32(&bars[0]), bar_s = smem_u32(&bars[1]), bar_x = smem_u32(&bars[2]);
 
-    // the chunk's record parts (head, its UP slice, extras) and the incoming state's slice rows
+    // the chunk's record parts (head, its UP slice, extras): one thread
     auto request_rec = [&](int c) {
         const float* r = hrec + (size_t)c * R::kFloats;
         mbar_expect_tx(bar_r, (R::kHead + CD * 64 + R::kExtra) * 4);
@@ -426,66 +446,136 @@ __global__ void __launch_bounds__(NT, 1) diag_bwd_kernel(BwdArgs a, FwdArgs f, c
         bulk_load(smem_u32(UPs), r + R::UP + sl * R::kSlice, CD * 64 * 4, bar_r);
         bulk_load(smem_u32(Rx), r + R::XA, R::kExtra * 4, bar_r);
     };
+    // the incoming state's slice rows of chunk c: warp 0, rows split over the lanes
     auto request_state = [&](int c) {
         const float* src = a.S_chunks + (head * NC + c) * DK * DV + v0;
-        mbar_expect_tx(bar_s, DK * 64 * 4);
-        for (int r = 0; r < DK; ++r) bulk_load(smem_u32(Ss + r * BLD), src + (size_t)r * DV, 256, bar_s);
+        if (lane == 0) mbar_expect_tx(bar_s, DK * 64 * 4);
+        __syncwarp();
+        for (int r = lane; r < DK; r += 32) bulk_load(smem_u32(Ss + r * BLD), src + (size_t)r * DV, 256, bar_s);
+    };
+    // raw rows of chunk c (k, q, v and dO columns of this CTA): warp 0, one token per lane
+    auto request_raw = [&](int c) {
+        const int tc = c * CD, nc = min(CD, T - tc);
+        if (lane == 0) mbar_expect_tx(bar_x, (uint32_t)(nc * (2 * DK + 128) * sizeof(Tin)));
+        __syncwarp();
+        if (lane < nc) {
+            const size_t ti = tok_index(b, tc + lane, h, T, H);
+            bulk_load(smem_u32(Kraw + lane * DK), kin + ti * DK, DK * sizeof(Tin), bar_x);
+            bulk_load(smem_u32(Qraw + lane * DK), qin + ti * DK, DK * sizeof(Tin), bar_x);
+            bulk_load(smem_u32(Vraw + lane * 64), v + ti * DV + v0, 64 * sizeof(Tin), bar_x);
+            bulk_load(smem_u32(Oraw + lane * 64), dO + ti * DV + v0, 64 * sizeof(Tin), bar_x);
+        }
     };
     if (tid == 0) {
         mbar_init(bar_r, 1);
         mbar_init(bar_s, 1);
+        mbar_init(bar_x, 1);
         fence_mbar_init();
-        if (NC > 0) {
-            request_rec(NC - 1);
-            request_state(NC - 1);
-        }
+        if (NC > 0) request_rec(NC - 1);
     }
-    if (tid < NP) {
-        int i = 0;
-        while ((i + 1) * (i + 2) / 2 <= tid) ++i;
-        pij[2 * tid] = (uint8_t)i;
-        pij[2 * tid + 1] = (uint8_t)(tid - i * (i + 1) / 2);
+    if (tid < CD) {  // the newest chunk's eta (later chunks' come a chunk ahead)
+        const int t = (NC - 1) * CD + tid;
+        etaS[tid] = t < T ? f.eta[tok_index(b, t, h, T, H)] : 0.f;
     }
     for (int x = tid; x < DK * 64; x += NT) {
         const int r = x >> 6, c = x & 63;
         Ls[r * BLD + c] = a.dS_T ? a.dS_T[sbase + (size_t)r * DV + v0 + c] : 0.f;
     }
+    __syncthreads();  // barriers initialised
+    if (warp == 0 && NC > 0) {
+        request_state(NC - 1);
+        request_raw(NC - 1);
+    }
 
     const int i = tid >> 4, tx = tid & 15, cx = 4 * tx;  // token row and this thread's columns
     bool ok = true;
+    int ci_stop = 0, stop_kind = 0;  // where a bounded wait gave up (for the drain below)
     for (int ci = NC - 1; ci >= 0; --ci) {
         const int t0 = ci * CD, n = min(CD, T - t0);
         const int ph = (NC - 1 - ci) & 1;
+        float eta_next = 0.f;  // the next (older, always full) chunk's eta, stored once etaS is read
+        if (tid < CD && ci > 0) eta_next = f.eta[tok_index(b, t0 - CD + tid, h, T, H)];
         __syncthreads();
-        // rows of the chunk: unit keys, queries and coefficients (u: the U coefficient); v, dO slices
-        {
-            float* gdummy = Es;  // load_rows also stages the raw decays: the E area is free here
-            load_rows<DK, Tin>(f, b, h, t0, n, Kh, Qs, gdummy, bs, cs, us);
+        const bool gotx = mbar_wait_bounded(bar_x, ph, 2000000000ull);
+        if (__syncthreads_or(!gotx)) {
+            ok = false;
+            ci_stop = ci;
+            stop_kind = 0;
+            break;
+        }
+        // ---- rows of the chunk: unit keys, queries, coefficients (u: the U coefficient); v, dO
+        for (int r = warp; r < CD; r += NT / 32) {
+            constexpr int PER = DK / 32;
+            if (r < n) {
+                float kv[PER];
+                float r2 = 0.f;
+#pragma unroll
+                for (int u = 0; u < PER; ++u) {
+                    kv[u] = to_f32(Kraw[r * DK + lane + 32 * u]);
+                    r2 = fmaf(kv[u], kv[u], r2);
+                }
+                r2 = warp_sum(r2);
+                const float et = etaS[r];
+                const KaczCoef cf = kacz_coef(et, r2, f.eps);
+#pragma unroll
+                for (int u = 0; u < PER; ++u) {
+                    Kh[r * LDK + lane + 32 * u] = kv[u] * cf.inv_r;
+                    Qs[r * LDK + lane + 32 * u] = to_f32(Qraw[r * DK + lane + 32 * u]);
+                }
+                if (lane == 0) {
+                    bs[r] = cf.b;
+                    cs[r] = cf.c;
+                    // U's value coefficient in the backward: c, except at a key of zero norm, where
+                    // U's row takes beta v (that row meets only khat = 0, except in row r of dkhat,
+                    // which then equals the exact dk = beta Gbar_r v_r)
+                    us[r] = r2 == 0.f ? (f.eps < 0.f ? et : (f.eps > 0.f ? et / f.eps : 0.f)) : cf.c;
+                }
+            } else {
+#pragma unroll
+                for (int u = 0; u < PER; ++u) {
+                    Kh[r * LDK + lane + 32 * u] = 0.f;
+                    Qs[r * LDK + lane + 32 * u] = 0.f;
+                }
+                if (lane == 0) bs[r] = cs[r] = us[r] = 0.f;
+            }
         }
         for (int x = tid; x < CD * 16; x += NT) {
             const int r = x >> 4, c4 = 4 * (x & 15);
             float vv[4] = {0.f, 0.f, 0.f, 0.f}, oo[4] = {0.f, 0.f, 0.f, 0.f};
             if (r < n) {
-                const size_t ti = tok_index(b, t0 + r, h, T, H) * DV + v0 + c4;
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    vv[e] = to_f32(v[ti + e]);
-                    oo[e] = to_f32(dO[ti + e]);
+                    vv[e] = to_f32(Vraw[r * 64 + c4 + e]);
+                    oo[e] = to_f32(Oraw[r * 64 + c4 + e]);
                 }
             }
             *reinterpret_cast<float4*>(Vs + r * BLD + c4) = make_float4(vv[0], vv[1], vv[2], vv[3]);
             *reinterpret_cast<float4*>(dOs + r * BLD + c4) = make_float4(oo[0], oo[1], oo[2], oo[3]);
         }
         if (tid < CD) dbs[tid] = 0.f;
+        __syncthreads();  // the raw rows and etaS are read: the next chunk's may come in
+        if (warp == 0 && ci > 0) request_raw(ci - 1);
+        if (tid < CD) etaS[tid] = eta_next;
         const bool got = mbar_wait_bounded(bar_r, ph, 2000000000ull) && mbar_wait_bounded(bar_s, ph, 2000000000ull);
-        if (__syncthreads_or(!got)) { ok = false; break; }
+        if (__syncthreads_or(!got)) {
+            ok = false;
+            ci_stop = ci;
+            stop_kind = 1;
+            break;
+        }
         const float* Gs = Rx + (R::XG - R::XA);
         const float* Am = Rx;
         const float* Tm = Rx + CD * CD;
-        // ---- E_ij = exp(G_i - G_j) per channel, j <= i
-        for (int x = tid; x < NP * DK; x += NT) {
-            const int p = x / DK, c = x % DK;
-            Es[x] = __expf(Gs[pij[2 * p] * DK + c] - Gs[pij[2 * p + 1] * DK + c]);
+        const float* QGr = Rh + R::QG;
+        // ---- per-token decay factors of the keys, and whether the chunk's range allows them
+        bool wide = false;
+        for (int x = tid; x < CD * DK; x += NT) {
+            const int t = x / DK, d = x % DK;
+            const float G = Gs[x];
+            wide |= !(fabsf(G) < kFactorLimit);
+            const float kh = Kh[t * LDK + d];
+            KiG[x] = kh * __expf(-G);
+            KG[x] = kh * __expf(G);
         }
         // ---- U = UP - W S + (u - c) v  and  dU = P^T dO + KD lambda (row i, columns cx .. cx + 3)
         {
@@ -516,7 +606,7 @@ __global__ void __launch_bounds__(NT, 1) diag_bwd_kernel(BwdArgs a, FwdArgs f, c
             *reinterpret_cast<float4*>(Us + i * BLD + cx) = u;
             *reinterpret_cast<float4*>(dUs + i * BLD + cx) = du;
         }
-        __syncthreads();
+        wide = __syncthreads_or(wide);
         // ---- dR = T^T dU (row j = i here); lambda o S row sums
         {
             float4 r4 = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -589,32 +679,60 @@ __global__ void __launch_bounds__(NT, 1) diag_bwd_kernel(BwdArgs a, FwdArgs f, c
             }
         }
         __syncthreads();  // Ym, Dm written; S read: the previous chunk's state may come in
-        if (tid == 0 && ci > 0) request_state(ci - 1);
+        if (warp == 0 && ci > 0) request_state(ci - 1);
         // ---- F terms and the per-(token, channel) gradients
-        float rq[EPT], rk[EPT], rg[EPT], rx[EPT];
         {
             float f1[EPT], f2[EPT], f3[EPT], f4[EPT];
 #pragma unroll
             for (int u = 0; u < EPT; ++u) f1[u] = f2[u] = f3[u] = f4[u] = 0.f;
-            for (int j = 0; j <= i; ++j) {
-                const float y = Ym[i * LDC + j], dd = Dm[i * LDC + j];
-                const float* E = Es + pair_index(i, j) * DK;
+            if (!wide) {
+                for (int j = 0; j <= i; ++j) {
+                    const float y = Ym[i * LDC + j], dd = Dm[i * LDC + j];
 #pragma unroll
-                for (int u = 0; u < EPT; ++u) {
-                    const int d = tx + 16 * u;
-                    const float ke = Kh[j * LDK + d] * E[d];
-                    f1[u] = fmaf(y, ke, f1[u]);
-                    f3[u] = fmaf(dd, ke, f3[u]);
+                    for (int u = 0; u < EPT; ++u) {
+                        const float kig = KiG[j * DK + tx + 16 * u];
+                        f1[u] = fmaf(y, kig, f1[u]);
+                        f3[u] = fmaf(dd, kig, f3[u]);
+                    }
                 }
-            }
-            for (int r = i; r < n; ++r) {
-                const float y = Ym[r * LDC + i], dd = Dm[r * LDC + i] * bs[r];
-                const float* E = Es + pair_index(r, i) * DK;
+                for (int r = i; r < n; ++r) {
+                    const float y = Ym[r * LDC + i], dd = Dm[r * LDC + i] * bs[r];
+#pragma unroll
+                    for (int u = 0; u < EPT; ++u) {
+                        const int d = tx + 16 * u;
+                        f2[u] = fmaf(y, QGr[r * DK + d], f2[u]);
+                        f4[u] = fmaf(dd, KG[r * DK + d], f4[u]);
+                    }
+                }
 #pragma unroll
                 for (int u = 0; u < EPT; ++u) {
-                    const int d = tx + 16 * u;
-                    f2[u] = fmaf(y, Qs[r * LDK + d] * E[d], f2[u]);
-                    f4[u] = fmaf(dd, Kh[r * LDK + d] * E[d], f4[u]);
+                    const float G = Gs[i * DK + tx + 16 * u];
+                    const float gp = __expf(G), gm = __expf(-G);
+                    f1[u] *= gp;
+                    f3[u] *= gp;
+                    f2[u] *= gm;
+                    f4[u] *= gm;
+                }
+            } else {
+                for (int j = 0; j <= i; ++j) {
+                    const float y = Ym[i * LDC + j], dd = Dm[i * LDC + j];
+#pragma unroll
+                    for (int u = 0; u < EPT; ++u) {
+                        const int d = tx + 16 * u;
+                        const float ke = Kh[j * LDK + d] * __expf(Gs[i * DK + d] - Gs[j * DK + d]);
+                        f1[u] = fmaf(y, ke, f1[u]);
+                        f3[u] = fmaf(dd, ke, f3[u]);
+                    }
+                }
+                for (int r = i; r < n; ++r) {
+                    const float y = Ym[r * LDC + i], dd = Dm[r * LDC + i] * bs[r];
+#pragma unroll
+                    for (int u = 0; u < EPT; ++u) {
+                        const int d = tx + 16 * u;
+                        const float e = __expf(Gs[r * DK + d] - Gs[i * DK + d]);
+                        f2[u] = fmaf(y, Qs[r * LDK + d] * e, f2[u]);
+                        f4[u] = fmaf(dd, Kh[r * LDK + d] * e, f4[u]);
+                    }
                 }
             }
             const float bi = bs[i];
@@ -625,31 +743,19 @@ __global__ void __launch_bounds__(NT, 1) diag_bwd_kernel(BwdArgs a, FwdArgs f, c
                 const float G = Gs[i * DK + d], Gl = Gs[(n - 1) * DK + d];
                 const float gam = __expf(G), del = __expf(Gl - G);
                 const float qd = Qs[i * LDK + d], kd = Kh[i * LDK + d];
-                rq[u] = fmaf(gam, zq[u], f1[u]);
-                rk[u] = -bi * gam * zr[u] + del * zl[u] + f2[u] + bi * f3[u] + f4[u];
-                rg[u] = gam * qd * zq[u] + qd * f1[u] - bi * gam * kd * zr[u] - kd * f2[u] + bi * kd * f3[u] -
-                        kd * f4[u] - del * kd * zl[u];
-                rx[u] = del * kd * zl[u];
+                Rq[i * DK + d] = fmaf(gam, zq[u], f1[u]);
+                Rk[i * DK + d] = -bi * gam * zr[u] + del * zl[u] + f2[u] + bi * f3[u] + f4[u];
+                Rg[i * DK + d] = gam * qd * zq[u] + qd * f1[u] - bi * gam * kd * zr[u] - kd * f2[u] +
+                                 bi * kd * f3[u] - kd * f4[u] - del * kd * zl[u];
+                Rxs[i * DK + d] = (i < n) ? del * kd * zl[u] : 0.f;
                 kgz = fmaf(kd * gam, zr[u], kgz);
             }
 #pragma unroll
             for (int o = 1; o < 16; o <<= 1) kgz += __shfl_xor_sync(0xffffffffu, kgz, o);
             if (tx == 0) dbs[i] -= kgz;
         }
-        __syncthreads();  // Es read: it takes the results
-        float* Rq = Es;
-        float* Rk = Es + CD * DK;
-        float* Rg = Es + 2 * CD * DK;
-        float* Rxs = Es + 3 * CD * DK;  // NP >= 4 CD rows of DK: room for the last token's terms
-#pragma unroll
-        for (int u = 0; u < EPT; ++u) {
-            const int d = tx + 16 * u;
-            Rq[i * DK + d] = rq[u];
-            Rk[i * DK + d] = rk[u];
-            Rg[i * DK + d] = rg[u];
-            Rxs[i * DK + d] = (i < n) ? rx[u] : 0.f;
-        }
-        // ---- new lambda = Diag(GC) lambda + QG^T dO - W^T dU (rows i + 16 m, columns cx .. cx + 3)
+        // ---- new lambda = Diag(GC) lambda + QG^T dO - W^T dU (rows i + 16 m, columns cx .. cx + 3);
+        //      every other read of lambda was before the last barrier
         {
             float4 acc[DK / 16];
 #pragma unroll
@@ -702,9 +808,18 @@ __global__ void __launch_bounds__(NT, 1) diag_bwd_kernel(BwdArgs a, FwdArgs f, c
         }
         if (tid < n) atomicAdd(&a.acc_db[tok_index(b, t0 + tid, h, T, H)], dbs[tid]);
         if (tid == 0 && ci > 0) request_rec(ci - 1);  // every read of the record is done
-        (void)lane;
     }
-    if (!ok && tid == 0) atomicOr(&g_diag_error, 2u);
+    if (!ok && tid == 0) {
+        atomicOr(&g_diag_error, 2u);
+        // let copies still in flight land before the block exits: the stopped chunk's record,
+        // state and rows, and the older chunk's rows when they were already requested (a wait
+        // on a phase that has completed returns at once)
+        const int ph = (NC - 1 - ci_stop) & 1;
+        (void)mbar_wait_bounded(bar_x, ph, 2000000000ull);
+        (void)mbar_wait_bounded(bar_r, ph, 2000000000ull);
+        (void)mbar_wait_bounded(bar_s, ph, 2000000000ull);
+        if (stop_kind == 1 && ci_stop > 0) (void)mbar_wait_bounded(bar_x, ph ^ 1, 2000000000ull);
+    }
     __syncthreads();
     if (ok) {
         for (int x = tid; x < DK * 64; x += NT) {
@@ -1104,7 +1219,7 @@ cudaError_t diag_fwd_launch(const FwdArgs& a, cudaStream_t st) {
 
 template <int DK, int DV, typename Tin, typename TOut>
 cudaError_t diag_bwd_launch(const BwdArgs& a, const FwdArgs& f, const float* recs, cudaStream_t st) {
-    const size_t smem = diag_bwd_smem_bytes<DK, DV>();
+    const size_t smem = diag_bwd_smem_bytes<DK, DV, Tin>();
     cudaError_t e = cudaFuncSetAttribute(diag_bwd_kernel<DK, DV, Tin, TOut>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;

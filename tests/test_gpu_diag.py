@@ -159,6 +159,10 @@ BWD_CASES = [
     (1, 70, 2, 128, 128, "bf16", -0.5, True, "kaczmarz"),
     (2, 100, 2, 128, 128, "bf16", -4.0, True, "kaczmarz"),
     (1, 64, 2, 128, 128, "bf16", -0.05, False, "direct"),
+    # log-decays down to -12 a token: in-chunk |G| passes 80, so the backward forms every pairwise
+    # factor exactly instead of as exp(G_i) exp(-G_j)
+    (1, 50, 2, 128, 128, "bf16", -12.0, True, "kaczmarz"),
+    (1, 37, 1, 64, 64, "f32", -12.0, False, "kaczmarz"),
 ]
 
 
