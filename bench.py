@@ -629,18 +629,26 @@ def bench_diag(kla, WORKLOADS, make_inputs, dev, stream, flush, rank, world, hbm
     # bytes as for scalar gating, plus the per-channel log-decays (Dk fp32 per token-head)
     alg = fwd_bytes(w.B, w.T, w.H, w.Dk, w.Dv, elt, False) + w.B * w.T * w.H * (w.Dk - 1) * 4
     flops = fwd_flops_per_token_head(w.Dk) * w.B * w.T * w.H
-    alu = fp32_alu_peak_tflops(peaks)
     mean_f = statistics.mean(ms_f) / 1e3
+    nl = L.kla_chunk_fwd_diag_kernel_launches(w.B, w.T, w.H, w.Dk, w.Dv, 64, 1)
+    # bf16 at Dk = Dv = 128: preparation and state pass on the tensor cores (the bound as for the
+    # headline forward: HBM on the algorithmic bytes, with the tensor-core fraction beside it)
     out = {"workload": w.name, "value": tokens / (tf_f / 1e3), "unit": "tokens/s", "steps": nf,
-           "ms_per_step": tf_f, "l2": "flushed between timed steps",
-           "gpu_launches_per_step": 2 if L.kla_chunk_fwd_diag_workspace(w.B, w.T, w.H, w.Dk, w.Dv, 64, 1) > 0 else 1,
-           "roofline": {"bound": "alu", "achieved": flops / mean_f / 1e12, "peak": alu, "unit": "TFLOP/s",
-                        "frac": flops / mean_f / 1e12 / alu,
-                        "peak_kind": "derived: 148 SMs x 128 fp32 FMA lanes x 2 x max SM clock",
-                        "hbm_frac": alg / mean_f / 1e9 / hbm_peak, "alg_bytes_per_launch": alg,
-                        "alg_flops_per_launch": flops},
+           "ms_per_step": tf_f, "l2": "flushed between timed steps", "gpu_launches_per_step": nl,
+           "path": "tensor cores: chunk_prep_diag_kernel + chunk_state_kernel (64-token chunks)",
+           "roofline": {"bound": "hbm", "achieved": alg / mean_f / 1e9, "peak": hbm_peak, "unit": "GB/s",
+                        "frac": alg / mean_f / 1e9 / hbm_peak, "alg_bytes_per_launch": alg,
+                        "tensor": {"achieved": flops / mean_f / 1e12, "peak": peaks["bf16_tflops"],
+                                   "unit": "TFLOP/s", "frac": flops / mean_f / 1e12 / peaks["bf16_tflops"],
+                                   "alg_flops_per_launch": flops}},
            "backward": {"value": tokens / (tf_b / 1e3), "unit": "tokens/s", "ms_per_step": tf_b,
                         "gpu_launches_per_step": 4,
+                        # CUDA cores, fp32: twice the forward's FLOPs (the training step's 3x
+                        # convention) against the fp32 FMA peak
+                        "roofline": {"bound": "alu", "achieved": 2 * flops / (tf_b / 1e3) / 1e12,
+                                     "peak": fp32_alu_peak_tflops(peaks), "unit": "TFLOP/s",
+                                     "frac": 2 * flops / (tf_b / 1e3) / 1e12 / fp32_alu_peak_tflops(peaks),
+                                     "peak_kind": "derived: 148 SMs x 128 fp32 FMA lanes x 2 x max SM clock"},
                         "what": "kla_chunk_bwd_diag: forward state recompute, reverse pass, finish, dg scan"}}
     out["decode"] = bench_decode(kla, WORKLOADS, make_inputs, dev, stream, flush, rank, world, hbm_peak, args,
                                  wname="decode_diag_b64_h16_d128_x1024", step_fn=kla.decode_step_diag,

@@ -87,6 +87,8 @@ def lib():
         L.kla_debug_inject_wait_timeout.restype = None
         L.kla_chunk_fwd_diag_workspace.argtypes = [i, i, i, i, i, i, i]
         L.kla_chunk_fwd_diag_workspace.restype = sz
+        L.kla_chunk_fwd_diag_kernel_launches.argtypes = [i, i, i, i, i, i, i]
+        L.kla_chunk_fwd_diag_kernel_launches.restype = i
         L.kla_chunk_fwd_diag.argtypes = [vp, vp, vp, fp, fp, f, fp, vp, fp, i, i, i, i, i, i, i, i, vp, sz, vp]
         L.kla_chunk_fwd_diag.restype = i
         L.kla_chunk_bwd_diag_workspace.argtypes = [i, i, i, i, i, i, i]

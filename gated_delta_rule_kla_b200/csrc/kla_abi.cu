@@ -35,6 +35,8 @@ kla_status cuda_fail(cudaError_t e, const char* where) {
 }
 
 bool aligned16(const void* p) { return p == nullptr || (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+// Workspaces take 32-byte stores (whole sectors of the swizzled tile images).
+bool aligned32(const void* p) { return p == nullptr || (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
 
 // KLA_BETA_DIRECT rides in a dtype argument: take it off (leaving the element type) and say
 // whether it was set.  The kernels learn it as eps = kla::kBetaDirect, a value the checks
@@ -202,7 +204,7 @@ kla_status kla_chunk_fwd(const void* q, const void* k, const void* v, const floa
         // (segmented for long sequences over few heads).  Without it: the fused one-kernel path.
         const size_t need = kla::chunk_fwd_split_workspace(a);
         if (need > 0 && ws != nullptr && ws_bytes >= need) {
-            if (!aligned16(ws)) return fail(KLA_ERR_INVALID_ARG, "ws must be 16-byte aligned");
+            if (!aligned32(ws)) return fail(KLA_ERR_INVALID_ARG, "ws must be 32-byte aligned");
             e = kla::launch_chunk_fwd_split(a, ws, s);
         } else {
             e = kla::launch_chunk_fwd_tc(a, s);
@@ -227,7 +229,7 @@ static kla_status split_stage_checks(int B, int T, int H, int Dk, int Dv, int ch
     if (ws == nullptr || ws_bytes < need)
         return fail(KLA_ERR_WORKSPACE, "%s needs %zu workspace bytes (got %zu)", name, need,
                     ws == nullptr ? (size_t)0 : ws_bytes);
-    if (!aligned16(ws)) return fail(KLA_ERR_INVALID_ARG, "ws must be 16-byte aligned");
+    if (!aligned32(ws)) return fail(KLA_ERR_INVALID_ARG, "ws must be 32-byte aligned");
     return KLA_OK;
 }
 
@@ -325,7 +327,7 @@ kla_status bwd_impl(const void* q, const void* k, const void* v, const float* et
     if (ws == nullptr || ws_bytes < need)
         return fail(KLA_ERR_WORKSPACE, "%s needs %zu workspace bytes (got %zu)", name, need,
                     ws == nullptr ? (size_t)0 : ws_bytes);
-    if (!aligned16(ws)) return fail(KLA_ERR_INVALID_ARG, "ws must be 16-byte aligned");
+    if (!aligned32(ws)) return fail(KLA_ERR_INVALID_ARG, "ws must be 32-byte aligned");
     cudaError_t e;
     if (tc_bwd_path(B, T, H, Dk, Dv, dtype, ws_bytes)) {
         kla::BwdTcArgs ta{q, k, v, eta, g, keps, S0, dO, dS_T, S_chunks, dq, dk, dv, deta, dg, dS0,
@@ -393,7 +395,7 @@ kla_status kla_chunk_fwd_train(const void* q, const void* k, const void* v, cons
     if (ws == nullptr || ws_bytes < need)
         return fail(KLA_ERR_WORKSPACE, "kla_chunk_fwd_train needs %zu workspace bytes (got %zu)", need,
                     ws == nullptr ? (size_t)0 : ws_bytes);
-    if (!aligned16(ws)) return fail(KLA_ERR_INVALID_ARG, "ws must be 16-byte aligned");
+    if (!aligned32(ws)) return fail(KLA_ERR_INVALID_ARG, "ws must be 32-byte aligned");
     kla::FwdArgs a{q, k, v, eta, g, kernel_eps(eps, direct), S0, o, S_T, nullptr, B, T, H, Dk, Dv,
                    dtype == KLA_BF16, out_dtype == KLA_BF16};
     cudaError_t e;
@@ -449,11 +451,36 @@ kla_status kla_decode_step_diag(const void* q, const void* k, const void* v, con
     return KLA_OK;
 }
 
+namespace {
+// FwdArgs of a diagonal-gated forward with only the sizes and types set (workspace queries).
+kla::FwdArgs diag_shape(int B, int T, int H, int Dk, int Dv, int dtype) {
+    kla::FwdArgs a{};
+    a.B = B;
+    a.T = T;
+    a.H = H;
+    a.Dk = Dk;
+    a.Dv = Dv;
+    a.bf16 = dtype == KLA_BF16;
+    a.diag = true;
+    return a;
+}
+}  // namespace
+
 size_t kla_chunk_fwd_diag_workspace(int B, int T, int H, int Dk, int Dv, int chunk, int dtype) {
     take_beta_flag(dtype);
     if (B < 1 || H < 1 || T < 1 || chunk != kla::kChunkLen || (Dk != 64 && Dk != 128) || (Dv != 64 && Dv != 128))
         return 0;
+    const kla::FwdArgs a = diag_shape(B, T, H, Dk, Dv, dtype);
+    if (kla::chunk_fwd_diag_tc_supported(a)) return kla::chunk_fwd_split_workspace(a);
     return kla::diag_fwd_workspace(B, T, H, Dk, Dv);
+}
+
+int kla_chunk_fwd_diag_kernel_launches(int B, int T, int H, int Dk, int Dv, int chunk, int dtype) {
+    take_beta_flag(dtype);
+    if (B < 1 || H < 1 || T < 1 || chunk != kla::kChunkLen || (Dk != 64 && Dk != 128) || (Dv != 64 && Dv != 128))
+        return 0;
+    const kla::FwdArgs a = diag_shape(B, T, H, Dk, Dv, dtype);
+    return kla::chunk_fwd_diag_tc_supported(a) ? kla::chunk_fwd_split_launches(a) : 2;
 }
 
 kla_status kla_chunk_fwd_diag(const void* q, const void* k, const void* v, const float* eta,
@@ -477,10 +504,19 @@ kla_status kla_chunk_fwd_diag(const void* q, const void* k, const void* v, const
         }
         return KLA_OK;
     }
-    if (!aligned16(ws)) return fail(KLA_ERR_INVALID_ARG, "ws must be 16-byte aligned");
+    if (!aligned32(ws)) return fail(KLA_ERR_INVALID_ARG, "ws must be 32-byte aligned");
     kla::FwdArgs a{q, k, v, eta, g, kernel_eps(eps, direct), S0, o, S_T, nullptr, B, T, H, Dk, Dv,
                    dtype == KLA_BF16, out_dtype == KLA_BF16};
-    cudaError_t e = kla::launch_chunk_fwd_diag(a, ws, ws == nullptr ? 0 : ws_bytes, s);
+    a.diag = true;
+    cudaError_t e;
+    if (kla::chunk_fwd_diag_tc_supported(a) && ws != nullptr && ws_bytes >= kla::chunk_fwd_split_workspace(a)) {
+        // bf16, Dk = Dv = 128: preparation and state pass on the tensor cores (64-token chunks)
+        e = kla::launch_chunk_fwd_split(a, ws, s);
+    } else {
+        // CUDA cores, 16-token chunks: split with a large enough workspace, else one kernel
+        a.diag = false;
+        e = kla::launch_chunk_fwd_diag(a, ws, ws == nullptr ? 0 : ws_bytes, s);
+    }
     if (e != cudaSuccess) return cuda_fail(e, "kla_chunk_fwd_diag launch");
     return KLA_OK;
 }
@@ -519,7 +555,7 @@ kla_status kla_chunk_bwd_diag(const void* q, const void* k, const void* v, const
     if (ws == nullptr || ws_bytes < need)
         return fail(KLA_ERR_WORKSPACE, "kla_chunk_bwd_diag needs %zu workspace bytes (got %zu)", need,
                     ws == nullptr ? (size_t)0 : ws_bytes);
-    if (!aligned16(ws)) return fail(KLA_ERR_INVALID_ARG, "ws must be 16-byte aligned");
+    if (!aligned32(ws)) return fail(KLA_ERR_INVALID_ARG, "ws must be 32-byte aligned");
     char* w = static_cast<char*>(ws);
     cudaError_t e = cudaMemsetAsync(w + off[1], 0, off[5] - off[1], s);
     if (e != cudaSuccess) return cuda_fail(e, "kla_chunk_bwd_diag workspace clear");
@@ -584,7 +620,7 @@ kla_status kla_gate_prologue_bwd(const void* x, const void* W, const float* eta,
     if (N > 0 && (ws == nullptr || ws_bytes < need))
         return fail(KLA_ERR_WORKSPACE, "kla_gate_prologue_bwd needs %zu workspace bytes (got %zu)", need,
                     ws == nullptr ? (size_t)0 : ws_bytes);
-    if (!aligned16(ws)) return fail(KLA_ERR_INVALID_ARG, "ws must be 16-byte aligned");
+    if (!aligned32(ws)) return fail(KLA_ERR_INVALID_ARG, "ws must be 32-byte aligned");
     kla::GateBwdArgs a{x, W, eta, g, deta, dg, q, dq_hat, dx, dW, dbias, dq, N, D, H, Dk, dtype == KLA_BF16};
     cudaError_t e = kla::launch_gate_prologue_bwd(a, ws, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "kla_gate_prologue_bwd launch");

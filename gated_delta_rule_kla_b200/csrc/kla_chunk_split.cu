@@ -379,6 +379,423 @@ done:
 }
 
 // =====================================================================================
+// Preparation kernel with diagonal gating (per-key-channel decays, "Kaczmarz Linear
+// Attention", Appendix B.5), on the tensor cores: one 64-token chunk per CTA, two CTAs per SM.
+// With G_t the in-chunk prefix of the log-decays (a vector over channels) the pairwise factor
+// exp(G_i - G_j) sits inside the channel sums of the Gram and score tiles, so it is split per
+// channel around a reference R = (max_t G_t + min_t G_t) / 2:
+//   [Q; Khat] o exp(G - R)  times  (Khat o exp(R - G))^T   (hi/lo bf16, three products)
+// gives every entry j <= i exactly; each factor is at most exp(range / 2), so a channel whose
+// in-chunk range reaches 160 takes the exact product on the CUDA cores instead (the entries
+// above the diagonal, which can overflow, are masked away).  W = T Diag(b) (Khat o Gam) and
+// U' = T Diag(c) V (Gam_t = exp(G_t) <= 1) are tensor-core products as for scalar gating; the
+// record adds Q o Gam for the state pass's O1 product and the next chunk's Gam_last per
+// channel for its rescale.
+// =====================================================================================
+constexpr uint32_t PD_K = 0;         // raw K tile (16 KB, TMA: two 64-dk blocks)
+constexpr uint32_t PD_C = 16384;     // G fp32 [64][128] (32 KB); then L/T + scratch; then T', T'' hi/lo
+constexpr uint32_t PD_D = 49152;     // next chunk's g (32 KB); then one dk half of the Gram operands
+                                     // (X hi/lo 32 KB, Y hi/lo 16 KB); then K o Gam hi/lo + V (48 KB)
+constexpr uint32_t PD_MISC = PD_D + 49152;
+constexpr uint32_t PD_SMEM = PD_MISC + 5120 + 1024;
+constexpr uint32_t PDM_G = 0, PDM_W = 64, PDM_U = 128;  // TMEM columns (256 allocated)
+constexpr float kDiagRange = 160.f;  // in-chunk range of G above which the Gram is formed exactly
+
+struct PrepDiagMisc {
+    uint64_t full, nextg, vbar, mma;
+    uint32_t tmem_base, wide;
+    float bco[CH], cco[CH], invr[CH], eta[CH];
+    float R[DK], Gl[DK], gh[DK];
+    float mx[2][DK], mn[2][DK];
+};
+static_assert(sizeof(PrepDiagMisc) <= 5120, "prep scalars");
+
+// Eight consecutive channels [d0, d0 + 8) of token row t of the raw K tile, times s.
+__device__ __forceinline__ void k_chunk8(const uint8_t* ktile, int t, int d0, float s, float* f) {
+    unpack_bf16x8(*reinterpret_cast<const uint4*>(ktile + (d0 >> 6) * 8192 + sw128_off(t, (d0 & 63) >> 3)), f);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) f[e] *= s;
+}
+// Eight consecutive channels of q at token t of (b, h) (zeros past the sequence).
+__device__ __forceinline__ void q_chunk8(const FwdArgs& a, int b, int t, int h, int d0, float* f) {
+    if (t < a.T) {
+        const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(a.q);
+        unpack_bf16x8(*reinterpret_cast<const uint4*>(q + tok_index(b, t, h, a.T, a.H) * DK + d0), f);
+    } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) f[e] = 0.f;
+    }
+}
+
+__global__ void __launch_bounds__(PT, 2)
+    chunk_prep_diag_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                           const __grid_constant__ CUtensorMap tm_g, FwdArgs a, uint8_t* __restrict__ recs,
+                           int cfirst) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    PrepDiagMisc* ms = reinterpret_cast<PrepDiagMisc*>(sm + PD_MISC);
+    float* Gs = reinterpret_cast<float*>(sm + PD_C);  // [64][DK]
+    float* Lf = Gs;                                     // later: L, then T in place
+    float* Xs = Lf + 64 * LDL;                          // 1024 floats of scratch for the inverse
+
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int row = tid & 127, ch = tid >> 7;
+    const int H = a.H, T = a.T;
+    const int NC = (T + CH - 1) / CH;
+    const int c = cfirst + blockIdx.x, head = blockIdx.y;
+    const int b = head / H, h = head % H;
+    const int t0 = c * CH, n = min(CH, T - t0);
+    const bool has_next = c + 1 < NC;
+    uint8_t* rec = recs + ((size_t)head * NC + c) * REC_BYTES_D;
+    const uint32_t sbase = smem_u32(sm);
+    const uint32_t bar_full = smem_u32(&ms->full), bar_next = smem_u32(&ms->nextg), bar_v = smem_u32(&ms->vbar),
+                   bar_mma = smem_u32(&ms->mma);
+
+    const float eta_own = (tid < n) ? a.eta[tok_index(b, t0 + tid, h, T, H)] : 0.f;
+    if (tid == 0) {
+        mbar_init(bar_full, 1);
+        mbar_init(bar_next, 1);
+        mbar_init(bar_v, 1);
+        mbar_init(bar_mma, 1);
+        fence_mbar_init();
+        mbar_expect_tx(bar_full, 16384 + 32768);
+        tma_load_4d(sbase + PD_K, &tm_k, bar_full, 0, h, t0, b);
+        tma_load_4d(sbase + PD_K + 8192, &tm_k, bar_full, 64, h, t0, b);
+        tma_load_4d(sbase + PD_C, &tm_g, bar_full, 0, h, t0, b);
+        if (has_next) {
+            mbar_expect_tx(bar_next, 32768);
+            tma_load_4d(sbase + PD_D, &tm_g, bar_next, 0, h, t0 + CH, b);
+        }
+        ms->wide = 0u;
+    }
+    if (warp == 0) {
+        tmem_alloc(smem_u32(&ms->tmem_base), 256);
+        tmem_relinquish();
+    }
+    if (tid < CH) ms->eta[tid] = eta_own;
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = ms->tmem_base;
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    bool aborted = false, next_pending = has_next, v_pending = false;
+    int mma_phase = 0;
+
+    do {
+        if (__syncthreads_or(!mbar_wait_bounded(bar_full, 0, kWaitNs))) { aborted = true; break; }
+        // ---- key norms and coefficients: four threads per key row (as for scalar gating)
+        {
+            const int j = tid >> 2, q = tid & 3;
+            const uint8_t* krow = sm + PD_K + (q >> 1) * 8192 + j * 128;
+            float ra = 0.f, rb = 0.f;
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const int cc = 4 * (q & 1) + ((m + 2 * (q >> 1)) & 3);
+                float f[8];
+                unpack_bf16x8(*reinterpret_cast<const uint4*>(krow + ((cc ^ (j & 7)) << 4)), f);
+#pragma unroll
+                for (int e = 0; e < 8; e += 2) {
+                    ra = fmaf(f[e], f[e], ra);
+                    rb = fmaf(f[e + 1], f[e + 1], rb);
+                }
+            }
+            float r2 = ra + rb;
+            r2 += __shfl_xor_sync(0xffffffffu, r2, 1);
+            r2 += __shfl_xor_sync(0xffffffffu, r2, 2);
+            if (q == 0) {
+                const KaczCoef cf = kacz_coef(ms->eta[j], r2, a.eps);
+                ms->bco[j] = cf.b;
+                ms->cco[j] = cf.c;
+                ms->invr[j] = cf.inv_r;
+            }
+        }
+        // ---- per-channel prefix sums of g over the chunk: thread (channel d, half hf) scans 32
+        //      tokens in registers; the second half then adds the first half's total
+        {
+            const int d = tid & 127, hf = tid >> 7;
+            float gv[32];
+#pragma unroll
+            for (int t = 0; t < 32; ++t) gv[t] = Gs[(32 * hf + t) * DK + d];
+#pragma unroll
+            for (int t = 1; t < 32; ++t) gv[t] += gv[t - 1];
+            if (hf == 0) ms->gh[d] = gv[31];
+            __syncthreads();
+            const float off = hf ? ms->gh[d] : 0.f;
+            float mx = -INFINITY, mn = INFINITY;
+#pragma unroll
+            for (int t = 0; t < 32; ++t) {
+                gv[t] += off;
+                Gs[(32 * hf + t) * DK + d] = gv[t];
+                mx = fmaxf(mx, gv[t]);
+                mn = fminf(mn, gv[t]);
+            }
+            ms->mx[hf][d] = mx;
+            ms->mn[hf][d] = mn;
+            __syncthreads();
+            if (hf == 0) {
+                const float hi = fmaxf(ms->mx[0][d], ms->mx[1][d]), lo = fminf(ms->mn[0][d], ms->mn[1][d]);
+                ms->R[d] = 0.5f * (hi + lo);
+                if (!(hi - lo < kDiagRange)) atomicOr(&ms->wide, 1u);
+            } else {
+                ms->Gl[d] = gv[31];  // G is flat past the last token
+            }
+        }
+        // ---- the next chunk's Gam_last per channel (the state pass's rescale)
+        if (has_next) {
+            if (__syncthreads_or(!mbar_wait_bounded(bar_next, 0, kWaitNs))) { aborted = true; break; }
+            next_pending = false;
+            const int d = tid & 127, hf = tid >> 7;
+            const float* gn = reinterpret_cast<const float*>(sm + PD_D);
+            float s = 0.f;
+#pragma unroll 8
+            for (int t = 0; t < 32; ++t) s += gn[(32 * hf + t) * DK + d];
+            if (hf == 1) ms->gh[d] = s;
+            __syncthreads();
+            if (hf == 0) reinterpret_cast<float*>(rec + REC_SC)[d] = __expf(s + ms->gh[d]);
+        } else if (tid < DK) {
+            reinterpret_cast<float*>(rec + REC_SC)[tid] = 1.f;
+        }
+        __syncthreads();
+        const bool wide = ms->wide != 0u;
+        const float* Rr = ms->R;
+
+        // ---- Gram and scores, one dk half at a time; the record's Q o Gam and Ktil hi/lo for the
+        //      same half while its products run
+        for (int hf = 0; hf < 2; ++hf) {
+            uint8_t* Xh = sm + PD_D;
+            uint8_t* Xl = Xh + 16384;
+            uint8_t* Yh = Xh + 32768;
+            uint8_t* Yl = Xh + 40960;
+            if (!wide) {
+                for (int u = tid; u < 128 * 8; u += PT) {
+                    const int r = u >> 3, cc = u & 7, i = r & 63, d0 = 64 * hf + 8 * cc;
+                    float f[8];
+                    if (r < 64) q_chunk8(a, b, t0 + i, h, d0, f);
+                    else k_chunk8(sm + PD_K, i, d0, ms->invr[i], f);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) f[e] *= __expf(Gs[i * DK + d0 + e] - Rr[d0 + e]);
+                    uint4 uh, ul;
+                    split_chunk8(f, uh, ul);
+                    *reinterpret_cast<uint4*>(Xh + sw128_off(r, cc)) = uh;
+                    *reinterpret_cast<uint4*>(Xl + sw128_off(r, cc)) = ul;
+                }
+                for (int u = tid; u < 64 * 8; u += PT) {
+                    const int j = u >> 3, cc = u & 7, d0 = 64 * hf + 8 * cc;
+                    float f[8];
+                    k_chunk8(sm + PD_K, j, d0, ms->invr[j], f);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) f[e] *= __expf(Rr[d0 + e] - Gs[j * DK + d0 + e]);
+                    uint4 uh, ul;
+                    split_chunk8(f, uh, ul);
+                    *reinterpret_cast<uint4*>(Yh + sw128_off(j, cc)) = uh;
+                    *reinterpret_cast<uint4*>(Yl + sw128_off(j, cc)) = ul;
+                }
+                fence_proxy_async();
+                tc_fence_before();
+                __syncthreads();
+                if (tid == kPrepIssuer) {
+                    tc_fence_after();
+                    const uint32_t ig = idesc_bf16(128, 64, false, false);
+                    const uint32_t xa[3] = {sbase + PD_D, sbase + PD_D, sbase + PD_D + 16384};
+                    const uint32_t yb[3] = {sbase + PD_D + 32768, sbase + PD_D + 40960, sbase + PD_D + 32768};
+#pragma unroll
+                    for (int p = 0; p < 3; ++p)
+#pragma unroll
+                        for (int s = 0; s < 4; ++s)
+                            mma_bf16(tmem + PDM_G, smem_desc(xa[p] + s * 32, 16, 1024), smem_desc(yb[p] + s * 32, 16, 1024),
+                                     ig, (hf | p | s) > 0);
+                    mma_commit(bar_mma);
+                }
+            }
+            for (int u = tid; u < 64 * 8; u += PT) {
+                const int t = u >> 3, cc = u & 7, d0 = 64 * hf + 8 * cc;
+                float f[8], kq[8];
+                q_chunk8(a, b, t0 + t, h, d0, f);
+                k_chunk8(sm + PD_K, t, d0, ms->invr[t], kq);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const float G = Gs[t * DK + d0 + e];
+                    f[e] *= __expf(G);
+                    kq[e] *= __expf(ms->Gl[d0 + e] - G);
+                }
+                uint4 uq;
+                uq.x = pack_bf16x2(f[0], f[1]); uq.y = pack_bf16x2(f[2], f[3]);
+                uq.z = pack_bf16x2(f[4], f[5]); uq.w = pack_bf16x2(f[6], f[7]);
+                *reinterpret_cast<uint4*>(rec + REC_QG + hf * 8192 + sw128_off(t, cc)) = uq;
+                uint4 uh, ul;
+                split_chunk8(kq, uh, ul);
+                *reinterpret_cast<uint4*>(rec + REC_KT + hf * 8192 + sw128_off(t, cc)) = uh;
+                *reinterpret_cast<uint4*>(rec + REC_KTLO + hf * 8192 + sw128_off(t, cc)) = ul;
+            }
+            if (!wide) {
+                const bool okm = mbar_wait_bounded(bar_mma, mma_phase & 1, kWaitNs);
+                ++mma_phase;
+                if (__syncthreads_or(!okm)) { aborted = true; break; }
+                tc_fence_after();
+            }
+        }
+        if (aborted) break;
+        // ---- V for U' over the consumed Y operands
+        if (tid == 0) {
+            mbar_expect_tx(bar_v, 16384);
+            tma_load_4d(sbase + PD_D + 32768, &tm_v, bar_v, 0, h, t0, b);
+            tma_load_4d(sbase + PD_D + 40960, &tm_v, bar_v, 64, h, t0, b);
+        }
+        v_pending = true;
+        // ---- a chunk too wide for the factored products: the Gram and scores exactly (row of
+        //      [Q; Khat] = TMEM lane, 32 key columns a thread)
+        if (wide) {
+            const int i = row & 63;
+            float acc[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) acc[e] = 0.f;
+            for (int d0 = 0; d0 < DK; d0 += 8) {
+                float x[8], gi[8];
+                if (row < 64) q_chunk8(a, b, t0 + i, h, d0, x);
+                else k_chunk8(sm + PD_K, i, d0, ms->invr[i], x);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) gi[e] = Gs[i * DK + d0 + e];
+                for (int e2 = 0; e2 < 32; ++e2) {
+                    const int j = 32 * ch + e2;
+                    float kj[8];
+                    k_chunk8(sm + PD_K, j, d0, ms->invr[j], kj);
+                    float s = acc[e2];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) s = fmaf(x[e] * kj[e], __expf(gi[e] - Gs[j * DK + d0 + e]), s);
+                    acc[e2] = s;
+                }
+            }
+            tmem_st32(tmem + lane_base + PDM_G + 32 * ch, acc);
+            tmem_st_wait();
+        }
+        // ---- K o Gam hi/lo (the A operand of W^T), [token][dk] blocks like the raw K tile
+        for (int u = tid; u < 64 * 16; u += PT) {
+            const int t = u >> 4, c16 = u & 15, d0 = 8 * c16;
+            float f[8];
+            k_chunk8(sm + PD_K, t, d0, ms->invr[t], f);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) f[e] *= __expf(Gs[t * DK + d0 + e]);
+            uint4 uh, ul;
+            split_chunk8(f, uh, ul);
+            const uint32_t o = (c16 >> 3) * 8192 + sw128_off(t, c16 & 7);
+            *reinterpret_cast<uint4*>(sm + PD_D + o) = uh;
+            *reinterpret_cast<uint4*>(sm + PD_D + 16384 + o) = ul;
+        }
+        tc_fence_before();
+        __syncthreads();  // G is no longer read: L takes its place
+        tc_fence_after();
+        // ---- Gram epilogue: P (rows 0-63, hi/lo to the record) and L (rows 64-127, fp32)
+        {
+            float x[32];
+            tmem_ld32(tmem + lane_base + PDM_G + 32 * ch, x);
+            tmem_ld_wait();
+            if (row < CH) {
+                const int i = row;
+#pragma unroll
+                for (int e = 0; e < 32; ++e) x[e] = (32 * ch + e <= i) ? x[e] : 0.f;
+                st_chunks_split_global(rec + REC_P, rec + REC_P + 8192, i, 4 * ch, 4, x);
+            } else {
+                const int i = row - CH;
+                const float bi = ms->bco[i];
+#pragma unroll
+                for (int e = 0; e < 32; ++e) x[e] = (32 * ch + e < i) ? bi * x[e] : 0.f;
+                float4* lrow = reinterpret_cast<float4*>(Lf + i * LDL + 32 * ch);
+#pragma unroll
+                for (int q = 0; q < 8; ++q) lrow[q] = make_float4(x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]);
+            }
+        }
+        tc_fence_before();
+        __syncthreads();
+        invert_unit_lower64_doubling<PT>(Lf, Xs, tid);
+        // ---- T' = T Diag(b) and T'' = T Diag(c) as bf16 hi/lo over the L/T area
+        {
+            const int i = tid >> 2, qq = tid & 3;
+            float tv[16];
+            {
+                const float* src = Lf + i * LDL + 16 * qq;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const float4 t4 = *reinterpret_cast<const float4*>(src + 4 * q);
+                    tv[4 * q] = t4.x; tv[4 * q + 1] = t4.y; tv[4 * q + 2] = t4.z; tv[4 * q + 3] = t4.w;
+                }
+            }
+            __syncthreads();  // T is read; T' and T'' overwrite it
+            float v[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) v[e] = tv[e] * ms->bco[16 * qq + e];
+            st_chunks_split(sm + PD_C, sm + PD_C + 8192, i, 2 * qq, 2, v);
+#pragma unroll
+            for (int e = 0; e < 16; ++e) v[e] = tv[e] * ms->cco[16 * qq + e];
+            st_chunks_split(sm + PD_C + 16384, sm + PD_C + 24576, i, 2 * qq, 2, v);
+        }
+        fence_proxy_async();
+        tc_fence_before();
+        if (__syncthreads_or(!mbar_wait_bounded(bar_v, 0, kWaitNs))) { aborted = true; break; }
+        v_pending = false;
+        // ---- MMA: W^T = (K o Gam)^T T'^T (lane = dk; products hi.hi, hi.lo, lo.hi) and
+        //      U'^T = V^T T''^T (lane = dv)
+        if (tid == kPrepIssuer) {
+            tc_fence_after();
+            const uint32_t iw = idesc_bf16(128, 64, true, false);
+#pragma unroll
+            for (int p = 0; p < 3; ++p)
+#pragma unroll
+                for (int s = 0; s < 4; ++s)
+                    mma_bf16(tmem + PDM_W, smem_desc(sbase + PD_D + (p == 2 ? 16384 : 0) + s * 2048, 8192, 1024),
+                             smem_desc(sbase + PD_C + (p == 1 ? 8192 : 0) + s * 32, 16, 1024), iw, (p | s) > 0);
+#pragma unroll
+            for (int part = 0; part < 2; ++part)
+#pragma unroll
+                for (int s = 0; s < 4; ++s)
+                    mma_bf16(tmem + PDM_U, smem_desc(sbase + PD_D + 32768 + s * 2048, 8192, 1024),
+                             smem_desc(sbase + PD_C + 16384 + part * 8192 + s * 32, 16, 1024), iw, (part | s) > 0);
+            mma_commit(bar_mma);
+        }
+        {
+            const bool okm = mbar_wait_bounded(bar_mma, mma_phase & 1, kWaitNs);
+            ++mma_phase;
+            if (__syncthreads_or(!okm)) { aborted = true; break; }
+        }
+        tc_fence_after();
+        // ---- -W transposed to [token][dk] over the consumed K o Gam tiles (one bulk copy to the
+        //      record); U' as [token][dv] rows straight to the record
+        {
+            float x[32];
+            tmem_ld32(tmem + lane_base + PDM_W + 32 * ch, x);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) x[e] = -x[e];
+            st_w_tokens_smem(sm + PD_D, row, 32 * ch, x, tid & 31);
+            tmem_ld32(tmem + lane_base + PDM_U + 32 * ch, x);
+            tmem_ld_wait();
+            float* up = reinterpret_cast<float*>(rec + REC_UP);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) up[(32 * ch + e) * DV + row] = x[e];
+            fence_proxy_async();
+            __syncthreads();
+            if (tid == 0) {
+                bulk_store(rec + REC_W, sbase + PD_D, 16384);
+                bulk_commit();
+                bulk_wait_read();
+            }
+        }
+    } while (false);
+    if (aborted && tid == 0) {
+        atomicOr(&g_split_error, 1u);
+        // copies still in flight land before the block exits
+        if (next_pending) (void)mbar_wait_bounded(bar_next, 0, kWaitNs);
+        if (v_pending) (void)mbar_wait_bounded(bar_v, 0, kWaitNs);
+        (void)mbar_wait_bounded(bar_full, 0, kWaitNs);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 256);
+    }
+}
+
+// =====================================================================================
 // State pass: one CTA per (b, h) [segment, kind], chunks in order.  Warp-specialised:
 // warps 0-7 run the epilogues (thread pair = one TMEM lane = one dv column, the two threads
 // splitting the columns), warp 8 issues the MMAs, warp 9 moves the stages in and the outputs
@@ -412,7 +829,8 @@ static_assert(SO_KT == REC_KT + 16384 && SO_KTLO == REC_KTLO + 16384 && SO_P == 
 static_assert(S_STAGE - SO_KT == 32768 + 16384 + 32768, "Ktil, P, U' fill the rest of the stage");
 constexpr uint32_t S_SC = 2 * S_STAGE;  // 2 x 512 B record scalars
 constexpr uint32_t S_MISC = S_SC + 2 * REC_SCB;
-constexpr uint32_t S_SMEM = S_MISC + 128 + 1024;
+constexpr uint32_t S_GL0 = S_MISC + 256;  // diagonal gating: the first chunk's Gam_last[128]
+constexpr uint32_t S_SMEM = S_GL0 + 512 + 1024;
 constexpr uint32_t TM_S = 0, TM_SH = 128, TM_SL = 192, TM_U = 256, TM_O1 = 320, TM_UH = 384, TM_UL = 416,
                    TM_O2 = 448;
 static_assert(TM_O1 == TM_U + 64, "U and O1 are one N = 128 accumulator");
@@ -425,6 +843,7 @@ struct StateMisc {
     uint32_t tmem_base, abort;
     float gsum[2];
 };
+static_assert(sizeof(StateMisc) <= 256, "state scalars");
 
 __device__ __forceinline__ void tma_store_4d(const void* tmap, uint32_t src, int c0, int c1, int c2, int c3) {
     asm volatile(
@@ -433,7 +852,7 @@ __device__ __forceinline__ void tma_store_4d(const void* tmap, uint32_t src, int
         "r"(src), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
         : "memory");
 }
-template <typename TOut>
+template <typename TOut, bool DIAG>
 __global__ void __launch_bounds__(ST, 1)
     chunk_state_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_o, FwdArgs a,
                        const uint8_t* __restrict__ recs) {
@@ -473,6 +892,11 @@ __global__ void __launch_bounds__(ST, 1)
     // Without outputs (the transition pass of the segmented mode) Q, P and the O products are not
     // needed; with zero values (its identity kind) neither is U'.
     const bool need_vals = !ident;
+    // Diagonal gating: Q o Gam comes with the record (the output needs no per-token gamma), the
+    // master state's rescale is per key channel, and records are longer.
+    constexpr bool diag = DIAG;
+    const size_t rstride = diag ? REC_BYTES_D : REC_BYTES;
+    const float* gl0 = reinterpret_cast<const float*>(sm + S_GL0);
 
     if (tid == 0) {
         mbar_init(full_a0, 1);
@@ -497,7 +921,15 @@ __global__ void __launch_bounds__(ST, 1)
         tmem_alloc(smem_u32(&ms->tmem_base), 512);
         tmem_relinquish();
     }
-    if (warp < 2) {  // gamma_last of the first chunk
+    if (diag) {  // Gam_last of the first chunk, per key channel
+        if (tid < DK) {
+            float sg = 0.f;
+            const int tb = c0 * CH, nn = NC > 0 ? min(CH, T - tb) : 0;
+#pragma unroll 8
+            for (int t = 0; t < nn; ++t) sg += a.g[tok_index(b, tb + t, h, T, H) * DK + tid];
+            reinterpret_cast<float*>(sm + S_GL0)[tid] = __expf(sg);
+        }
+    } else if (warp < 2) {  // gamma_last of the first chunk
         const bool live = NC > 0 && c0 * CH + tid < T;
         const float gv = live ? a.g[tok_index(b, c0 * CH + tid, h, T, H)] : 0.f;
         const float sg = warp_sum(gv);
@@ -524,13 +956,18 @@ __global__ void __launch_bounds__(ST, 1)
             auto load_a = [&](int c, int st) {
                 const uint32_t bar = full_a0 + 8 * st;
                 const uint32_t base = sbase + st * S_STAGE;
-                const uint8_t* rec = recs + ((size_t)head_idx * NCtot + c) * REC_BYTES;
+                const uint8_t* rec = recs + ((size_t)head_idx * NCtot + c) * rstride;
                 mbar_expect_tx(bar, a_bytes);
                 bulk_load(base + SO_WQ, rec + REC_W, 8192, bar);
                 bulk_load(base + SO_WQ + 16384, rec + REC_W + 8192, 8192, bar);
                 if (write_o) {
-                    tma_load_4d(base + SO_WQ + 8192, &tm_q, bar, 0, h, c * CH, b);
-                    tma_load_4d(base + SO_WQ + 24576, &tm_q, bar, 64, h, c * CH, b);
+                    if (diag) {
+                        bulk_load(base + SO_WQ + 8192, rec + REC_QG, 8192, bar);
+                        bulk_load(base + SO_WQ + 24576, rec + REC_QG + 8192, 8192, bar);
+                    } else {
+                        tma_load_4d(base + SO_WQ + 8192, &tm_q, bar, 0, h, c * CH, b);
+                        tma_load_4d(base + SO_WQ + 24576, &tm_q, bar, 64, h, c * CH, b);
+                    }
                     bulk_load(base + SO_P, rec + REC_P, 16384, bar);
                 }
                 if (need_vals) {
@@ -541,7 +978,7 @@ __global__ void __launch_bounds__(ST, 1)
             auto load_b = [&](int c, int st) {
                 const uint32_t bar = full_b0 + 8 * st;
                 const uint32_t base = sbase + st * S_STAGE;
-                const uint8_t* rec = recs + ((size_t)head_idx * NCtot + c) * REC_BYTES;
+                const uint8_t* rec = recs + ((size_t)head_idx * NCtot + c) * rstride;
                 mbar_expect_tx(bar, b_bytes);
                 bulk_load(base + SO_KT, rec + REC_KT, 16384, bar);
                 bulk_load(base + SO_KTLO, rec + REC_KTLO, 16384, bar);
@@ -683,7 +1120,7 @@ __global__ void __launch_bounds__(ST, 1)
                 tmem_st16u(tmem + lane_base + TM_SH + 32 * ch + 16 * q2, hp);
                 tmem_st16u(tmem + lane_base + TM_SL + 32 * ch + 16 * q2, lp);
 #pragma unroll
-                for (int e = 0; e < 32; ++e) x[e] *= g0;
+                for (int e = 0; e < 32; ++e) x[e] *= diag ? gl0[dk0 + e] : g0;
                 tmem_st32(tmem + lane_base + TM_S + 64 * ch + 32 * q2, x);
             }
             epi_signal(s_ready0, tid);
@@ -760,11 +1197,20 @@ __global__ void __launch_bounds__(ST, 1)
                         }
                     }
 
-                    const float gN = reinterpret_cast<const float*>(sm + S_SC + st * REC_SCB)[CH];
+                    const float* scs = reinterpret_cast<const float*>(sm + S_SC + st * REC_SCB);
+                    if (diag) {  // per key channel: this thread holds dk 64 ch .. 64 ch + 63
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        x0[e] *= gN;
-                        x1[e] *= gN;
+                        for (int e = 0; e < 32; ++e) {
+                            x0[e] *= scs[64 * ch + e];
+                            x1[e] *= scs[64 * ch + 32 + e];
+                        }
+                    } else {
+                        const float gN = scs[CH];
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) {
+                            x0[e] *= gN;
+                            x1[e] *= gN;
+                        }
                     }
                     tmem_st32(tmem + lane_base + TM_S + 64 * ch, x0);
                     tmem_st32(tmem + lane_base + TM_S + 64 * ch + 32, x1);
@@ -787,7 +1233,7 @@ __global__ void __launch_bounds__(ST, 1)
 #pragma unroll
                     for (int e = 0; e < 32; ++e) {
                         const int t = 32 * ch + e;
-                        stage_o[t * DV + row] = from_f32<TOut>(fmaf(gm[t], o1[e], o2[e]));
+                        stage_o[t * DV + row] = from_f32<TOut>(fmaf(diag ? 1.f : gm[t], o1[e], o2[e]));
                     }
                     fence_proxy_async();
                 }
@@ -901,7 +1347,7 @@ SplitLayout split_layout(const FwdArgs& a) {
     SplitLayout L{};
     const int NC = (a.T + CH - 1) / CH;
     const int BH = a.B * a.H;
-    L.rec_bytes = align1k((size_t)BH * NC * REC_BYTES);
+    L.rec_bytes = align1k((size_t)BH * NC * (a.diag ? REC_BYTES_D : REC_BYTES));
     L.seg_off = L.rec_bytes;
     const int ns = choose_nseg_split(BH, NC);
     if (ns > 1) {
@@ -960,10 +1406,10 @@ cudaError_t launch_state(const CUtensorMap& mq, const FwdArgs& a, const uint8_t*
     CUtensorMap mo;
     memset(&mo, 0, sizeof(mo));
     if (a.o != nullptr && !make_out_map(&mo, a.o, a.B, a.T, a.H, a.out_bf16)) return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(chunk_state_kernel<TOut>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)S_SMEM);
+    auto kern = a.diag ? chunk_state_kernel<TOut, true> : chunk_state_kernel<TOut, false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)S_SMEM);
     if (e != cudaSuccess) return e;
-    chunk_state_kernel<TOut><<<grid, ST, S_SMEM, st>>>(mq, mo, a, recs);
+    kern<<<grid, ST, S_SMEM, st>>>(mq, mo, a, recs);
     return cudaGetLastError();
 }
 
@@ -974,9 +1420,26 @@ size_t chunk_fwd_split_workspace(const FwdArgs& a) {
     return split_layout(a).total;
 }
 
+bool chunk_fwd_diag_tc_supported(const FwdArgs& a) {
+    return a.diag && a.bf16 && a.Dk == 128 && a.Dv == 128 && a.T > 0 && a.S_chunks == nullptr &&
+           a.T_tiles == nullptr && a.S_tiles == nullptr && a.U_tiles == nullptr && !a.rec_extras;
+}
+
 namespace {
 // Preparation of chunks [cfirst, cfirst + count) of every head.
 cudaError_t launch_prep_range(const FwdArgs& a, void* ws, int cfirst, int count, cudaStream_t st) {
+    if (a.diag) {
+        CUtensorMap mk, mv, mg;
+        if (!make_map(&mk, a.k, a.B, a.T, a.H) || !make_map(&mv, a.v, a.B, a.T, a.H) ||
+            !make_out_map(&mg, const_cast<float*>(a.g), a.B, a.T, a.H, false))
+            return cudaErrorInvalidValue;
+        cudaError_t e =
+            cudaFuncSetAttribute(chunk_prep_diag_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PD_SMEM);
+        if (e != cudaSuccess) return e;
+        chunk_prep_diag_kernel<<<dim3(count, a.B * a.H), PT, PD_SMEM, st>>>(mk, mv, mg, a, static_cast<uint8_t*>(ws),
+                                                                           cfirst);
+        return cudaGetLastError();
+    }
     CUtensorMap mq, mk, mv;
     if (!make_map(&mq, a.q, a.B, a.T, a.H) || !make_map(&mk, a.k, a.B, a.T, a.H) ||
         !make_map(&mv, a.v, a.B, a.T, a.H))

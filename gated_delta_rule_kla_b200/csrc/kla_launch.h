@@ -51,6 +51,10 @@ struct FwdArgs {
     // Diagonal-gated split forward: also store what the backward needs in each record (the Gram
     // A, the inverse T and the per-channel log-decay prefix G of every 16-token chunk).
     bool rec_extras = false;
+    // Tensor-core split forward with diagonal gating: g is [B, T, H, Dk] (one log-decay per key
+    // channel) and each chunk's record also holds Q o Gam and the next chunk's per-channel
+    // decay (the split path's entry points choose it; the CUDA-core kernels do not read it).
+    bool diag = false;
 };
 
 struct BwdArgs {
@@ -149,6 +153,8 @@ cudaError_t launch_seg_scan(const float* S0, const float* MN, float* Sstart, flo
 // state-independent operands to the workspace, then a sequential state pass (segmented for
 // long sequences over few heads).  Workspace bytes for these sizes (0: shapes not supported).
 size_t chunk_fwd_split_workspace(const FwdArgs& a);
+// Diagonal gating on the split tensor-core path (bf16, Dk = Dv = 128): a.diag must be set.
+bool chunk_fwd_diag_tc_supported(const FwdArgs& a);
 cudaError_t launch_chunk_fwd_split(const FwdArgs& a, void* ws, cudaStream_t st);
 // Kernels one launch_chunk_fwd_split call launches (preparation and state passes).
 int chunk_fwd_split_launches(const FwdArgs& a);

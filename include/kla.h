@@ -92,7 +92,7 @@ int kla_version(void);
  *   S_T          out  [B,H,Dk,Dv] fp32 final state, or NULL.  May alias S0.
  *   S_chunks     out  [B,H,ceil(T/chunk),Dk,Dv] fp32 state at the start of every chunk, or
  *                     NULL.  Passing it to kla_chunk_bwd saves the backward's recompute.
- *   ws, ws_bytes      caller workspace (device memory, 16-byte aligned, owned by the caller,
+ *   ws, ws_bytes      caller workspace (device memory, 32-byte aligned, owned by the caller,
  *                     contents need not be initialised), or NULL.  With at least
  *                     kla_chunk_fwd_workspace() bytes, bf16 inputs with Dk == Dv == 128 run the
  *                     split path: a chunk-parallel kernel stores every chunk's state-independent
@@ -127,7 +127,7 @@ kla_status kla_chunk_fwd(const void *q, const void *k, const void *v, const floa
  * runs the sequential state pass from ws.  Together they equal one kla_chunk_fwd call with that
  * workspace, bit for bit.
  *   Arguments as for kla_chunk_fwd.  Only dtype == KLA_BF16 with Dk == Dv == 128 and T >= 1 is
- *   supported (KLA_ERR_UNSUPPORTED / KLA_ERR_INVALID_ARG otherwise).  ws (device, 16-byte
+ *   supported (KLA_ERR_UNSUPPORTED / KLA_ERR_INVALID_ARG otherwise).  ws (device, 32-byte
  *   aligned, at least kla_chunk_fwd_workspace() bytes, owned by the caller) is required
  *   (KLA_ERR_WORKSPACE otherwise); _state must get the same ws, q, g and sizes as the _prep
  *   call it follows, ordered after it (same stream, or an event), with ws untouched between.
@@ -152,7 +152,7 @@ kla_status kla_chunk_fwd_state(const void *q, const float *g, const float *S0, v
  * At a key of exactly zero norm the write vanishes but dk does not: it is returned exactly,
  * dk_t = beta_t Gbar_t v_t with beta_t = eta_t / eps (eta_t in the direct mode; 0 when
  * eps == 0) and Gbar_t the gradient of the state after token t.
- * ws, ws_bytes: caller workspace (device, 16-byte aligned, owned by the caller, contents need
+ * ws, ws_bytes: caller workspace (device, 32-byte aligned, owned by the caller, contents need
  * not be initialised) of at least kla_chunk_bwd_workspace_min() bytes (required; smaller is
  * KLA_ERR_WORKSPACE).  With at least kla_chunk_bwd_workspace() bytes, bf16 inputs with
  * Dk == Dv == 128 run on the tensor cores: the split forward's preparation and state pass are
@@ -193,7 +193,7 @@ kla_status kla_chunk_bwd(const void *q, const void *k, const void *v, const floa
  *   kla_chunk_bwd_after_train: arguments as kla_chunk_bwd without S0 and S_chunks; must get the
  *     same q, k, v, eta, g, eps, sizes, dtype, ws and ws_bytes as the kla_chunk_fwd_train call it
  *     follows (ordered after it: same stream, or an event), with ws untouched in between.
- * ws: device memory, 16-byte aligned, owned by the caller, contents need not be initialised;
+ * ws: device memory, 32-byte aligned, owned by the caller, contents need not be initialised;
  * too small is KLA_ERR_WORKSPACE.  Returns KLA_OK or an error status; on error nothing is
  * launched.
  */
@@ -237,15 +237,23 @@ kla_status kla_decode_step(const void *q, const void *k, const void *v, const fl
  *
  * kla_chunk_fwd_diag   -- prefill: o ([B,T,H,Dv] of out_dtype, or NULL) and S_T ([B,H,Dk,Dv]
  *                         fp32, or NULL; may alias S0) from S0 (NULL = zero state).  ws (device,
- *                         16-byte aligned, caller-owned, contents need not be initialised) of at
+ *                         32-byte aligned, caller-owned, contents need not be initialised) of at
  *                         least kla_chunk_fwd_diag_workspace() bytes selects the split path: a
- *                         chunk-parallel kernel stores every 16-token chunk's state-independent
- *                         operands there (about 34 KiB per chunk and head at Dk = Dv = 128),
- *                         then a sequential state pass reads them; with NULL or less, one kernel
- *                         per (head, 64 value columns) does both (slower, no workspace).
+ *                         chunk-parallel kernel stores every chunk's state-independent operands
+ *                         there, then a sequential state pass reads them.  bf16 with Dk = Dv =
+ *                         128 runs both on the tensor cores over 64-token chunks (a 112.5 KiB
+ *                         record per chunk and head, as two slabs or parallel segments like
+ *                         kla_chunk_fwd); other shapes run on the CUDA cores over 16-token
+ *                         chunks (about 34 KiB per chunk and head at Dk = Dv = 128).  With NULL
+ *                         or less, one kernel per (head, 64 value columns) does both on the
+ *                         CUDA cores (slower, no workspace).
+ *                         The tensor-core preparation forms the chunk's pairwise decay factors
+ *                         exp(G_i - G_j) per channel as exp(G_i - R) exp(R - G_j) around the
+ *                         channel's mid-range R; a chunk where some channel's prefix G spans
+ *                         160 or more takes them exactly, on the CUDA cores (slower).
  * kla_chunk_bwd_diag   -- gradients of <o, dO> + <S_T, dS_T> with respect to q, k, v, eta, g
  *                         (dg per channel, [B,T,H,Dk]) and S0; dS_T may be NULL.  ws: device,
- *                         16-byte aligned, caller-owned, at least kla_chunk_bwd_diag_workspace()
+ *                         32-byte aligned, caller-owned, at least kla_chunk_bwd_diag_workspace()
  *                         bytes (the state at every internal chunk start, fp32 accumulators
  *                         cleared by the call, and the split forward's records), else
  *                         KLA_ERR_WORKSPACE.  At a key
@@ -254,6 +262,9 @@ kla_status kla_decode_step(const void *q, const void *k, const void *v, const fl
  * Returns KLA_OK or an error status; on error nothing is launched.
  */
 size_t kla_chunk_fwd_diag_workspace(int B, int T, int H, int Dk, int Dv, int chunk, int dtype);
+/* Kernels one kla_chunk_fwd_diag call launches for these shapes when given at least
+ * kla_chunk_fwd_diag_workspace() bytes; 0 for invalid shapes. */
+int kla_chunk_fwd_diag_kernel_launches(int B, int T, int H, int Dk, int Dv, int chunk, int dtype);
 kla_status kla_chunk_fwd_diag(const void *q, const void *k, const void *v, const float *eta,
                               const float *g, float eps, const float *S0, void *o, float *S_T,
                               int B, int T, int H, int Dk, int Dv, int chunk, int dtype,
@@ -293,7 +304,7 @@ kla_status kla_decode_step_diag(const void *q, const void *k, const void *v, con
  *     dz = [deta * eta (1 - eta), dg * expm1(g)],  dx = dz W,  dW = dz^T x,  dbias = sum_t dz,
  *     dq = (dq_hat - q_hat (q_hat . dq_hat)) / ||q||   (zero where q is zero)
  * deta, dg [N, H], dq_hat [N, H, Dk] fp32 in; dx [N, D], dW [2H, D], dbias [2H], dq [N, H, Dk]
- * fp32 out (q, dq_hat and dq all given or all NULL).  ws: device, 16-byte aligned,
+ * fp32 out (q, dq_hat and dq all given or all NULL).  ws: device, 32-byte aligned,
  * caller-owned, at least kla_gate_prologue_bwd_workspace() bytes (per-tile partial sums of dW
  * and dbias, added in a fixed order: the result is deterministic).
  */

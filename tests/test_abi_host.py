@@ -193,3 +193,15 @@ def test_backward_reverse_segments(L):
     assert L.kla_chunk_bwd_reverse_segments(1, 4100, 2, 128, 128, 64, 1) > 1
     assert L.kla_chunk_bwd_reverse_segments(1, 4100, 2, 64, 64, 64, 1) == 0  # no tensor-core backward
     assert L.kla_chunk_bwd_reverse_segments(1, 4100, 2, 128, 128, 64, 0) == 0
+
+
+def test_diag_forward_workspace_by_path(L):
+    """bf16 at Dk = Dv = 128 takes the tensor-core split path: one record of 112.5 KiB per 64-token
+    chunk and head; other shapes the CUDA-core split path over 16-token chunks."""
+    tc = L.kla_chunk_fwd_diag_workspace(2, 300, 3, 128, 128, 64, 1)
+    assert tc >= 2 * 3 * 5 * 115200
+    assert L.kla_chunk_fwd_diag_kernel_launches(2, 300, 3, 128, 128, 64, 1) >= 2
+    simt = L.kla_chunk_fwd_diag_workspace(2, 300, 3, 128, 128, 64, 0)
+    assert simt >= 2 * 3 * 19 * 4 * (3 * 16 * 128 + 16 * 16 + 128)
+    assert L.kla_chunk_fwd_diag_kernel_launches(2, 300, 3, 128, 128, 64, 0) == 2
+    assert L.kla_chunk_fwd_diag_kernel_launches(2, 300, 3, 96, 128, 64, 1) == 0
