@@ -617,11 +617,15 @@ __global__ void __launch_bounds__(NT, 1) diag_bwd_kernel(BwdArgs a, FwdArgs f, c
             }
             *reinterpret_cast<float4*>(dRs + i * BLD + cx) = r4;
         }
-        if (tid < DK) {
-            float p = 0.f;
-#pragma unroll 8
-            for (int c = 0; c < 64; ++c) p = fmaf(Ls[tid * BLD + c], Ss[tid * BLD + c], p);
-            lsS[tid] = p;
+        // rows of lambda o S summed: sixteen lanes per row, each a 4-column group (whole 256-byte
+        // rows per half-warp, no bank conflicts), then a 16-lane shuffle sum
+        for (int d = tid >> 4; d < DK; d += NT / 16) {
+            const float4 l4 = *reinterpret_cast<const float4*>(Ls + d * BLD + cx);
+            const float4 s4 = *reinterpret_cast<const float4*>(Ss + d * BLD + cx);
+            float p = l4.x * s4.x + l4.y * s4.y + l4.z * s4.z + l4.w * s4.w;
+#pragma unroll
+            for (int o = 1; o < 16; o <<= 1) p += __shfl_xor_sync(0xffffffffu, p, o);
+            if (tx == 0) lsS[d] = p;
         }
         __syncthreads();
         // ---- dv, dc; Y, D; the D o A part of db

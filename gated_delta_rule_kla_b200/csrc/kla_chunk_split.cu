@@ -452,6 +452,20 @@ __global__ void __launch_bounds__(PT, 2)
                    bar_mma = smem_u32(&ms->mma);
 
     const float eta_own = (tid < n) ? a.eta[tok_index(b, t0 + tid, h, T, H)] : 0.f;
+    // this thread's q chunks, loaded first so that their latency overlaps the set-up: rows tq and
+    // tq + 32, 16-byte chunk cq of each 64-channel half (the X operands' Q rows and the record's
+    // Q o Gam take the same ones)
+    const int tq = tid >> 3, cq = tid & 7;
+    uint4 qv[2][2];
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+            const int t = t0 + tq + 32 * k;
+            qv[hf][k] = t < T ? *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(a.q) +
+                                                                 tok_index(b, t, h, T, H) * DK + 64 * hf + 8 * cq)
+                              : make_uint4(0u, 0u, 0u, 0u);
+        }
     if (tid == 0) {
         mbar_init(bar_full, 1);
         mbar_init(bar_next, 1);
@@ -538,6 +552,7 @@ __global__ void __launch_bounds__(PT, 2)
                 if (!(hi - lo < kDiagRange)) atomicOr(&ms->wide, 1u);
             } else {
                 ms->Gl[d] = gv[31];  // G is flat past the last token
+                reinterpret_cast<float*>(rec + REC_GL)[d] = __expf(gv[31]);
             }
         }
         // ---- the next chunk's Gam_last per channel (the state pass's rescale)
@@ -561,23 +576,25 @@ __global__ void __launch_bounds__(PT, 2)
 
         // ---- Gram and scores, one dk half at a time; the record's Q o Gam and Ktil hi/lo for the
         //      same half while its products run
+#pragma unroll
         for (int hf = 0; hf < 2; ++hf) {
             uint8_t* Xh = sm + PD_D;
             uint8_t* Xl = Xh + 16384;
             uint8_t* Yh = Xh + 32768;
             uint8_t* Yl = Xh + 40960;
             if (!wide) {
-                for (int u = tid; u < 128 * 8; u += PT) {
-                    const int r = u >> 3, cc = u & 7, i = r & 63, d0 = 64 * hf + 8 * cc;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int r = tq + 32 * k, i = r & 63, d0 = 64 * hf + 8 * cq;
                     float f[8];
-                    if (r < 64) q_chunk8(a, b, t0 + i, h, d0, f);
+                    if (k < 2) unpack_bf16x8(qv[hf][k & 1], f);
                     else k_chunk8(sm + PD_K, i, d0, ms->invr[i], f);
 #pragma unroll
                     for (int e = 0; e < 8; ++e) f[e] *= __expf(Gs[i * DK + d0 + e] - Rr[d0 + e]);
                     uint4 uh, ul;
                     split_chunk8(f, uh, ul);
-                    *reinterpret_cast<uint4*>(Xh + sw128_off(r, cc)) = uh;
-                    *reinterpret_cast<uint4*>(Xl + sw128_off(r, cc)) = ul;
+                    *reinterpret_cast<uint4*>(Xh + sw128_off(r, cq)) = uh;
+                    *reinterpret_cast<uint4*>(Xl + sw128_off(r, cq)) = ul;
                 }
                 for (int u = tid; u < 64 * 8; u += PT) {
                     const int j = u >> 3, cc = u & 7, d0 = 64 * hf + 8 * cc;
@@ -607,10 +624,11 @@ __global__ void __launch_bounds__(PT, 2)
                     mma_commit(bar_mma);
                 }
             }
-            for (int u = tid; u < 64 * 8; u += PT) {
-                const int t = u >> 3, cc = u & 7, d0 = 64 * hf + 8 * cc;
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                const int t = tq + 32 * k, cc = cq, d0 = 64 * hf + 8 * cc;
                 float f[8], kq[8];
-                q_chunk8(a, b, t0 + t, h, d0, f);
+                unpack_bf16x8(qv[hf][k], f);
                 k_chunk8(sm + PD_K, t, d0, ms->invr[t], kq);
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
@@ -921,14 +939,11 @@ __global__ void __launch_bounds__(ST, 1)
         tmem_alloc(smem_u32(&ms->tmem_base), 512);
         tmem_relinquish();
     }
-    if (diag) {  // Gam_last of the first chunk, per key channel
-        if (tid < DK) {
-            float sg = 0.f;
-            const int tb = c0 * CH, nn = NC > 0 ? min(CH, T - tb) : 0;
-#pragma unroll 8
-            for (int t = 0; t < nn; ++t) sg += a.g[tok_index(b, tb + t, h, T, H) * DK + tid];
-            reinterpret_cast<float*>(sm + S_GL0)[tid] = __expf(sg);
-        }
+    if (diag) {  // Gam_last of the first chunk, per key channel, from its record
+        if (tid < DK)
+            reinterpret_cast<float*>(sm + S_GL0)[tid] =
+                NC > 0 ? reinterpret_cast<const float*>(recs + ((size_t)head_idx * NCtot + c0) * rstride + REC_GL)[tid]
+                       : 1.f;
     } else if (warp < 2) {  // gamma_last of the first chunk
         const bool live = NC > 0 && c0 * CH + tid < T;
         const float gv = live ? a.g[tok_index(b, c0 * CH + tid, h, T, H)] : 0.f;
@@ -1199,10 +1214,12 @@ __global__ void __launch_bounds__(ST, 1)
 
                     const float* scs = reinterpret_cast<const float*>(sm + S_SC + st * REC_SCB);
                     if (diag) {  // per key channel: this thread holds dk 64 ch .. 64 ch + 63
+                        const float4* sc4 = reinterpret_cast<const float4*>(scs + 64 * ch);
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) {
-                            x0[e] *= scs[64 * ch + e];
-                            x1[e] *= scs[64 * ch + 32 + e];
+                        for (int e = 0; e < 8; ++e) {
+                            const float4 a4 = sc4[e], b4 = sc4[8 + e];
+                            x0[4 * e] *= a4.x; x0[4 * e + 1] *= a4.y; x0[4 * e + 2] *= a4.z; x0[4 * e + 3] *= a4.w;
+                            x1[4 * e] *= b4.x; x1[4 * e + 1] *= b4.y; x1[4 * e + 2] *= b4.z; x1[4 * e + 3] *= b4.w;
                         }
                     } else {
                         const float gN = scs[CH];

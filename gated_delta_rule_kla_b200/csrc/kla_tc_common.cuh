@@ -421,10 +421,12 @@ constexpr uint32_t REC_TILES = 98304;
 constexpr uint32_t REC_SC = REC_TILES;  // gamma[64], gamma_last of the next chunk, of the previous chunk  512 B
 constexpr uint32_t REC_SCB = 512;
 constexpr size_t REC_BYTES = REC_TILES + REC_SCB;
-// Diagonal gating: the scalars are the next chunk's per-channel decay Gam_last[128], and
-// Q o Gam (one bf16 rounding, [64 tokens x 64 dk] x 2 blocks, swizzled) follows.
+// Diagonal gating: the scalars are the next chunk's per-channel decay Gam_last[128]; Q o Gam
+// (one bf16 rounding, [64 tokens x 64 dk] x 2 blocks, swizzled) and the chunk's own
+// Gam_last[128] follow.
 constexpr uint32_t REC_QG = (uint32_t)REC_BYTES;                                //  16 KB
-constexpr size_t REC_BYTES_D = REC_BYTES + 16384;
+constexpr uint32_t REC_GL = REC_QG + 16384;                                     //  512 B
+constexpr size_t REC_BYTES_D = REC_GL + 512;
 
 // Split fp32 values into bf16 hi + lo words, two consecutive K indices per 32-bit word (the
 // lower index in the low half): hi = rn(x), lo = rn(x - hi).

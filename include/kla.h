@@ -241,7 +241,7 @@ kla_status kla_decode_step(const void *q, const void *k, const void *v, const fl
  *                         least kla_chunk_fwd_diag_workspace() bytes selects the split path: a
  *                         chunk-parallel kernel stores every chunk's state-independent operands
  *                         there, then a sequential state pass reads them.  bf16 with Dk = Dv =
- *                         128 runs both on the tensor cores over 64-token chunks (a 112.5 KiB
+ *                         128 runs both on the tensor cores over 64-token chunks (a 113 KiB
  *                         record per chunk and head, as two slabs or parallel segments like
  *                         kla_chunk_fwd); other shapes run on the CUDA cores over 16-token
  *                         chunks (about 34 KiB per chunk and head at Dk = Dv = 128).  With NULL

@@ -196,7 +196,7 @@ def test_backward_reverse_segments(L):
 
 
 def test_diag_forward_workspace_by_path(L):
-    """bf16 at Dk = Dv = 128 takes the tensor-core split path: one record of 112.5 KiB per 64-token
+    """bf16 at Dk = Dv = 128 takes the tensor-core split path: one record of 113 KiB per 64-token
     chunk and head; other shapes the CUDA-core split path over 16-token chunks."""
     tc = L.kla_chunk_fwd_diag_workspace(2, 300, 3, 128, 128, 64, 1)
     assert tc >= 2 * 3 * 5 * 115200
