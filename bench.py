@@ -541,7 +541,9 @@ def bench_long(kla, WORKLOADS, make_inputs, dev, stream, rank, world, hbm_peak, 
     train = {"ms_per_step": f_ms + b_ms, "forward_ms": f_ms, "backward_ms": b_ms,
              "value": w.B * w.T / ((f_ms + b_ms) / 1e3), "unit": "tokens/s",
              "what": "kla_chunk_fwd_train + kla_chunk_bwd_after_train (reverse state pass over 1024 chunks per head, "
-                     "then the chunk-parallel gradient kernel)"}
+                     "as parallel segments when kla_chunk_bwd_reverse_segments > 1; then the chunk-parallel "
+                     "gradient kernel)",
+             "reverse_segments": kla.lib().kla_chunk_bwd_reverse_segments(w.B, w.T, w.H, w.Dk, w.Dv, 64, 1)}
     barrier(world)
     total_ms = max_over_ranks(sum(ms), world)
     tokens = sum_over_ranks(float(w.B * w.T), world) * nsteps

@@ -191,6 +191,31 @@ def test_bwd_diag_matches_oracle(kla, oracle_mod, B, T, H, Dk, Dv, dtype, gate_l
         assert rel_err(gr[name], ref[name]) <= TOL[dtype], name
 
 
+def test_fwd_diag_tensor_cores_zero_keys_zero_eta_and_T1(kla, oracle_mod):
+    """The tensor-core forward (bf16, Dk = Dv = 128) with keys of zero norm (they write nothing),
+    eta = 0 tokens, a ragged last chunk, S_T aliasing S0, and a one-token sequence."""
+    w, inp = diag_inputs(2, 75, 2, 128, 128, "bf16", seed=31, gate_lo=-1.0)
+    for b, t, h in ((0, 0, 0), (0, 63, 1), (1, 64, 0), (1, 74, 1), (0, 30, 0)):
+        inp["k"][b, t, h] = 0
+    inp["eta"][:, 5::9] = 0
+    d = {k: v.cuda() for k, v in inp.items()}
+    S = d["S0"].clone()
+    o, _ = kla.chunk_fwd_diag(d["q"], d["k"], d["v"], d["eta"], d["g"], w.eps, S, S_T=S)
+    torch.cuda.synchronize()
+    kla.check_device_error()
+    ro, rST = oracle_mod.forward_diag(*(np64(inp[k]) for k in ("q", "k", "v", "eta", "g")), w.eps, np64(inp["S0"]))
+    assert rel_err(o, ro) <= 2e-2
+    assert rel_err(S, rST) <= 2e-2
+    w1, inp1 = diag_inputs(1, 1, 3, 128, 128, "bf16", seed=32)
+    d1 = {k: v.cuda() for k, v in inp1.items()}
+    o1, S1 = kla.chunk_fwd_diag(d1["q"], d1["k"], d1["v"], d1["eta"], d1["g"], w1.eps, d1["S0"])
+    torch.cuda.synchronize()
+    ro1, rS1 = oracle_mod.forward_diag(*(np64(inp1[k]) for k in ("q", "k", "v", "eta", "g")), w1.eps,
+                                       np64(inp1["S0"]))
+    assert rel_err(o1, ro1) <= 2e-2
+    assert rel_err(S1, rS1) <= 2e-2
+
+
 def test_bwd_diag_zero_norm_keys_exact(kla, oracle_mod):
     """dk at keys of zero norm is beta_t Gbar_t v_t (compared on its own scale)."""
     w, inp = diag_inputs(1, 60, 2, 128, 128, "f32", seed=23, gate_lo=-1.0)
