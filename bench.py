@@ -357,7 +357,7 @@ def time_fwd_stages(kla, d, w, ws, o, ST, flush, stream, nsteps):
         ev[i][0].record(stream)
         kla.chunk_fwd_prep(d["q"], d["k"], d["v"], d["eta"], d["g"], w.eps, ws)
         ev[i][1].record(stream)
-        kla.chunk_fwd_state(d["q"], d["g"], d["S0"], ws, o=o, S_T=ST)
+        kla.chunk_fwd_state(d["q"], d["v"], d["g"], d["S0"], ws, o=o, S_T=ST)
         ev[i][2].record(stream)
     torch.cuda.synchronize()
     prep = statistics.median(e[0].elapsed_time(e[1]) for e in ev) * 1e3

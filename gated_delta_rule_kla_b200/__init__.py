@@ -63,7 +63,7 @@ def lib():
         L.kla_chunk_fwd.restype = i
         L.kla_chunk_fwd_prep.argtypes = [vp, vp, vp, fp, fp, f, i, i, i, i, i, i, i, vp, sz, vp]
         L.kla_chunk_fwd_prep.restype = i
-        L.kla_chunk_fwd_state.argtypes = [vp, fp, fp, vp, fp, fp, i, i, i, i, i, i, i, i, vp, sz, vp]
+        L.kla_chunk_fwd_state.argtypes = [vp, vp, fp, fp, vp, fp, fp, i, i, i, i, i, i, i, i, vp, sz, vp]
         L.kla_chunk_fwd_state.restype = i
         L.kla_chunk_bwd_workspace.argtypes = [i, i, i, i, i, i, i, i]
         L.kla_chunk_bwd_workspace.restype = sz
@@ -232,13 +232,15 @@ def chunk_fwd_prep(q, k, v, eta, g, eps, workspace, *, stream=None, beta="kaczma
     _check(st, "kla_chunk_fwd_prep")
 
 
-def chunk_fwd_state(q, g, S0, workspace, *, Dv=None, o=None, S_T=None, S_chunks=None,
+def chunk_fwd_state(q, v, g, S0, workspace, *, o=None, S_T=None, S_chunks=None,
                     out_dtype=torch.float32, stream=None):
     """Second stage of the split forward: the state pass over the records that chunk_fwd_prep
-    left in `workspace`.  Writes o, S_T, S_chunks when given (allocates o and S_T when None)."""
+    left in `workspace` (it also reads q and v).  Writes o, S_T, S_chunks when given (allocates o
+    and S_T when None)."""
     dev = q.device
     B, T, H, Dk = q.shape
-    Dv = Dk if Dv is None else Dv
+    Dv = v.shape[-1]
+    _need(v, "v", dev, q.dtype, (B, T, H, Dv))
     _need(g, "g", dev, torch.float32, (B, T, H)); _need(S0, "S0", dev, torch.float32, (B, H, Dk, Dv))
     if o is None:
         o = torch.empty(B, T, H, Dv, device=dev, dtype=out_dtype)
@@ -248,7 +250,7 @@ def chunk_fwd_state(q, g, S0, workspace, *, Dv=None, o=None, S_T=None, S_chunks=
     _need(S_chunks, "S_chunks", dev, torch.float32, (B, H, (T + CHUNK - 1) // CHUNK, Dk, Dv))
     _need(workspace, "workspace", dev, torch.uint8)
     L = lib()
-    st = L.kla_chunk_fwd_state(_ptr(q), _ptr(g), _ptr(S0), _ptr(o), _ptr(S_T), _ptr(S_chunks), B, T, H, Dk, Dv,
+    st = L.kla_chunk_fwd_state(_ptr(q), _ptr(v), _ptr(g), _ptr(S0), _ptr(o), _ptr(S_T), _ptr(S_chunks), B, T, H, Dk, Dv,
                                CHUNK, _dtype_code(q), _dtype_code(o), _ptr(workspace), workspace.numel(),
                                _stream(dev, stream))
     _check(st, "kla_chunk_fwd_state")

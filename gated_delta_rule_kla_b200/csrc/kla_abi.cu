@@ -249,17 +249,17 @@ kla_status kla_chunk_fwd_prep(const void* q, const void* k, const void* v, const
     return KLA_OK;
 }
 
-kla_status kla_chunk_fwd_state(const void* q, const float* g, const float* S0, void* o, float* S_T,
-                               float* S_chunks, int B, int T, int H, int Dk, int Dv, int chunk,
+kla_status kla_chunk_fwd_state(const void* q, const void* v, const float* g, const float* S0, void* o,
+                               float* S_T, float* S_chunks, int B, int T, int H, int Dk, int Dv, int chunk,
                                int dtype, int out_dtype, void* ws, size_t ws_bytes, void* stream) {
     take_beta_flag(dtype);  // the state pass reads the preparation's coefficients
     kla::FwdArgs a{};
     kla_status st = split_stage_checks(B, T, H, Dk, Dv, chunk, dtype, out_dtype, 0.f, ws, ws_bytes,
                                        "kla_chunk_fwd_state", &a);
     if (st != KLA_OK) return st;
-    REQUIRE_PTR(q); REQUIRE_PTR(g);
+    REQUIRE_PTR(q); REQUIRE_PTR(v); REQUIRE_PTR(g);
     OPTIONAL_PTR(S0); OPTIONAL_PTR(o); OPTIONAL_PTR(S_T); OPTIONAL_PTR(S_chunks);
-    a.q = q; a.g = g; a.S0 = S0; a.o = o; a.S_T = S_T; a.S_chunks = S_chunks;
+    a.q = q; a.v = v; a.g = g; a.S0 = S0; a.o = o; a.S_T = S_T; a.S_chunks = S_chunks;
     cudaError_t e = kla::launch_chunk_fwd_split_state(a, ws, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "kla_chunk_fwd_state launch");
     return KLA_OK;

@@ -7,19 +7,20 @@
 //   W   = T Diag(b gamma) Khat,   U' = T Diag(c) V                      (independent of S)
 //   U   = U' - W S,   O = Diag(gamma) Q S + P U,   S' = gamma_last S + Ktil^T U,
 //   Ktil = Diag(delta) Khat,  delta_j = e^{G_last - G_j}.
-// Everything that does not depend on the incoming state -- P, W, U', Ktil and the decays --
-// is computed for all chunks at once by `chunk_prep_kernel` (one CTA per chunk, two CTAs per
-// SM) and written to a per-chunk record in the workspace, already in the shared-memory image
-// the MMAs read.  `chunk_state_kernel` then walks the chunks of each head in order and does
-// only what the state feeds: U = U' - W S, S' and O, with every A operand (S and U as bf16
-// hi/lo pairs) held in TMEM, so a step is two dependent MMA groups and two short epilogues.
+// Everything that does not depend on the incoming state -- P, W, T'' = T Diag(c), Ktil and the
+// decays -- is computed for all chunks at once by `chunk_prep_kernel` (one CTA per chunk, four
+// CTAs per SM) and written to a per-chunk record in the workspace, already in the
+// shared-memory image the MMAs read.  `chunk_state_kernel` then walks the chunks of each head in
+// order: U' = T'' V (its own V tile; independent of S, so it runs off the chain), U = U' - W S,
+// S' and O, with every A operand (S and U as bf16 hi/lo pairs) held in TMEM, so a step is two
+// dependent MMA groups and two short epilogues.
 //
 // State-pass TMEM (lane = dv throughout, 512 columns):
 //   [0,128)   S^T master, fp32, pre-scaled by the coming chunk's gamma_last
 //   [128,192) S^T hi bf16, [192,256) S^T lo     -- A operand, K = dk
-//   [256,320) U^T accumulator fp32 (col = token)
-//   [320,352) U^T hi bf16, [352,384) U^T lo     -- A operand, K = token
-//   [384,448) O1 = S^T Q^T,  [448,512) O2 = U^T P^T;   o = gamma o O1 + O2
+//   [256,320) U^T accumulator fp32 (col = token), [320,384) O1 = S^T Q^T: one N = 128 accumulator
+//   [384,416) U^T hi bf16, [416,448) U^T lo     -- A operand, K = token
+//   [448,512) O2 = U^T P^T;   o = gamma o O1 + O2
 #include <cuda.h>
 #include <string.h>
 
@@ -46,18 +47,20 @@ constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s
 // The per-chunk record layout (REC_*) is defined in kla_tc_common.cuh.
 
 // =====================================================================================
-// Preparation kernel: one chunk per CTA, three CTAs per SM.  Shared memory holds only the
-// inputs and the MMA operands; every output goes from registers straight to its record.
+// Preparation kernel: one chunk per CTA, four CTAs per SM.  Shared memory holds only the
+// [Q; K] tile and the MMA operands; every output goes from registers straight to its record.
+// U' = T'' V is left to the state pass (the record carries T''), so V is not read here.
 // =====================================================================================
 constexpr int PT = 256;
 constexpr int kPrepIssuer = 128;
-constexpr uint32_t P_QK = 0;       // [Q; K] tile (32 KB); after the Gram MMA, T' hi/lo over Q
-constexpr uint32_t P_V = 32768;    // V tile (16 KB)
-constexpr uint32_t P_Z = 49152;    // L/T fp32 (64 x LDL) + 1024 floats scratch; then T'' hi/lo
-constexpr uint32_t P_MISC = P_Z + 64 * LDL * 4 + 4096;
+constexpr uint32_t P_QK = 0;       // [Q; K] tile (32 KB); after the Gram MMA the inverse's scratch
+                                   // (4 KB) over Q block 0, then T' hi/lo over Q
+constexpr uint32_t P_Z = 32768;    // L/T fp32 (64 x LDL); then -W staged as [token][dk] tiles
+constexpr uint32_t P_MISC = P_Z + 64 * LDL * 4;
 constexpr uint32_t P_SMEM = P_MISC + 3072 + 1024;
 static_assert(P_MISC % 1024 == 0, "prep scalars alignment");
-constexpr uint32_t PM_G = 0, PM_W = 0, PM_U = 64;  // TMEM columns (128 allocated); W reuses G's
+static_assert(64 * LDL * 4 >= 16384, "-W staging fits over L/T");
+constexpr uint32_t PM_G = 0, PM_W = 0;  // TMEM columns (64 allocated); W reuses G's
 
 struct PrepMisc {
     uint64_t full, mma;
@@ -68,14 +71,14 @@ struct PrepMisc {
 };
 static_assert(sizeof(PrepMisc) <= 3072, "prep scalars");
 
-__global__ void __launch_bounds__(PT, 3)
+__global__ void __launch_bounds__(PT, 4)
     chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                      const __grid_constant__ CUtensorMap tm_v, FwdArgs a, uint8_t* __restrict__ recs, int cfirst) {
+                      FwdArgs a, uint8_t* __restrict__ recs, int cfirst) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     PrepMisc* ms = reinterpret_cast<PrepMisc*>(sm + P_MISC);
     float* Lf = reinterpret_cast<float*>(sm + P_Z);  // 64 x LDL fp32: L, then T in place
-    float* Xs = Lf + 64 * LDL;                         // 1024 floats of scratch for the inverse
+    float* Xs = reinterpret_cast<float*>(sm + P_QK);   // 1024 floats of scratch for the inverse (over Q)
 
     const int tid = threadIdx.x, warp = tid >> 5;
     const int row = tid & 127, ch = tid >> 7;
@@ -106,16 +109,14 @@ __global__ void __launch_bounds__(PT, 3)
         mbar_init(bar_full, 1);
         mbar_init(bar_mma, 1);
         fence_mbar_init();
-        mbar_expect_tx(bar_full, 6 * 8192);
+        mbar_expect_tx(bar_full, 4 * 8192);
         tma_load_4d(sbase + P_QK, &tm_q, bar_full, 0, h, t0, b);
         tma_load_4d(sbase + P_QK + 16384, &tm_q, bar_full, 64, h, t0, b);
         tma_load_4d(sbase + P_QK + 8192, &tm_k, bar_full, 0, h, t0, b);
         tma_load_4d(sbase + P_QK + 24576, &tm_k, bar_full, 64, h, t0, b);
-        tma_load_4d(sbase + P_V, &tm_v, bar_full, 0, h, t0, b);
-        tma_load_4d(sbase + P_V + 8192, &tm_v, bar_full, 64, h, t0, b);
     }
     if (warp == 0) {
-        tmem_alloc(smem_u32(&ms->tmem_base), 128);
+        tmem_alloc(smem_u32(&ms->tmem_base), 64);
         tmem_relinquish();
     }
     if (tid < CH) {
@@ -134,7 +135,7 @@ __global__ void __launch_bounds__(PT, 3)
     const uint32_t tmem = ms->tmem_base;
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const uint8_t* qk = sm + P_QK;
-    const uint32_t qk_a = sbase + P_QK, v_a = sbase + P_V;
+    const uint32_t qk_a = sbase + P_QK;
 
     bool ok = mbar_wait_bounded(bar_full, 0, kWaitNs);
     if (__syncthreads_or(!ok)) {
@@ -273,8 +274,8 @@ __global__ void __launch_bounds__(PT, 3)
     tc_fence_before();
     __syncthreads();
     invert_unit_lower64_doubling<PT>(Lf, Xs, tid);
-    // ---- T' = T Diag(b gamma / r) over the Q slots of the [Q; K] tile, T'' = T Diag(c) over
-    //      L/T: thread -> row tid/4, 16 columns (T is zero above its diagonal)
+    // ---- T' = T Diag(b gamma / r) over the Q slots of the [Q; K] tile, T'' = T Diag(c) straight
+    //      to the record: thread -> row tid/4, 16 columns (T is zero above its diagonal)
     {
         const int i = tid >> 2, qq = tid & 3;
         float tv[16];
@@ -286,7 +287,7 @@ __global__ void __launch_bounds__(PT, 3)
                 tv[4 * q] = t4.x; tv[4 * q + 1] = t4.y; tv[4 * q + 2] = t4.z; tv[4 * q + 3] = t4.w;
             }
         }
-        __syncthreads();  // T is read; T'' overwrites it
+        __syncthreads();  // T is read (and the scratch over Q): T' overwrites Q
         if (a.T_tiles) {
             uint8_t* tt = static_cast<uint8_t*>(a.T_tiles) + ((size_t)head * NC + c) * 16384;
             st_chunks_split_global(tt, tt + 8192, i, 2 * qq, 2, tv);
@@ -297,12 +298,12 @@ __global__ void __launch_bounds__(PT, 3)
         st_chunks_split(sm + P_QK, sm + P_QK + 16384, i, 2 * qq, 2, v);
 #pragma unroll
         for (int e = 0; e < 16; ++e) v[e] = tv[e] * ms->cco[16 * qq + e];
-        st_chunks_split(sm + P_Z, sm + P_Z + 8192, i, 2 * qq, 2, v);
+        st_chunks_split_global(rec + REC_TPP, rec + REC_TPP + 8192, i, 2 * qq, 2, v);
     }
     fence_proxy_async();
     tc_fence_before();
     __syncthreads();
-    // ---- MMA: W^T = K^T T'^T (lane = dk) and U'^T = V^T T''^T (lane = dv)
+    // ---- MMA: W^T = K^T T'^T (lane = dk)
     if (tid == kPrepIssuer) {
         tc_fence_after();
         const uint32_t iw = idesc_bf16(128, 64, true, false);
@@ -312,12 +313,6 @@ __global__ void __launch_bounds__(PT, 3)
             for (int s = 0; s < 4; ++s)
                 mma_bf16(tmem + PM_W, smem_desc(qk_a + 8192 + s * 2048, 16384, 1024),
                          smem_desc(qk_a + part * 16384 + s * 32, 16, 1024), iw, (part | s) > 0);
-#pragma unroll
-        for (int part = 0; part < 2; ++part)
-#pragma unroll
-            for (int s = 0; s < 4; ++s)
-                mma_bf16(tmem + PM_U, smem_desc(v_a + s * 2048, 8192, 1024),
-                         smem_desc(sbase + P_Z + part * 8192 + s * 32, 16, 1024), iw, (part | s) > 0);
         mma_commit(bar_mma);
     }
     ok = mbar_wait_bounded(bar_mma, 1, kWaitNs);
@@ -328,19 +323,13 @@ __global__ void __launch_bounds__(PT, 3)
     tc_fence_after();
     {
         // ---- -W (thread = dk column, 32 tokens) transposed to [token][dk] tiles over the consumed
-        //      V tile, then one bulk copy to the record; U' as [token][dv] rows and Ktil hi/lo
-        //      straight to the record
+        //      L/T area, then one bulk copy to the record; Ktil hi/lo straight to the record
         float x[32];
         tmem_ld32(tmem + lane_base + PM_W + 32 * ch, x);
         tmem_ld_wait();
 #pragma unroll
         for (int e = 0; e < 32; ++e) x[e] = -x[e];
-        st_w_tokens_smem(sm + P_V, row, 32 * ch, x, tid & 31);
-        tmem_ld32(tmem + lane_base + PM_U + 32 * ch, x);
-        tmem_ld_wait();
-        float* up = reinterpret_cast<float*>(rec + REC_UP);
-#pragma unroll
-        for (int e = 0; e < 32; ++e) up[(32 * ch + e) * DV + row] = x[e];
+        st_w_tokens_smem(sm + P_Z, row, 32 * ch, x, tid & 31);
         // Ktil row j, dk block blk, logical chunks cq .. cq + 3, in pairs (one 32-byte store
         // each); the pair order alternates with blk so the two blocks' reads of a row (16 KB
         // apart, same banks) do not collide
@@ -364,7 +353,7 @@ __global__ void __launch_bounds__(PT, 3)
         fence_proxy_async();
         __syncthreads();
         if (tid == 0) {
-            bulk_store(rec + REC_W, sbase + P_V, 16384);
+            bulk_store(rec + REC_W, sbase + P_Z, 16384);
             bulk_commit();
             bulk_wait_read();
         }
@@ -374,7 +363,7 @@ done:
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
-        tmem_dealloc(tmem, 128);
+        tmem_dealloc(tmem, 64);
     }
 }
 
@@ -387,22 +376,23 @@ done:
 //   [Q; Khat] o exp(G - R)  times  (Khat o exp(R - G))^T   (hi/lo bf16, three products)
 // gives every entry j <= i exactly; each factor is at most exp(range / 2), so a channel whose
 // in-chunk range reaches 160 takes the exact product on the CUDA cores instead (the entries
-// above the diagonal, which can overflow, are masked away).  W = T Diag(b) (Khat o Gam) and
-// U' = T Diag(c) V (Gam_t = exp(G_t) <= 1) are tensor-core products as for scalar gating; the
-// record adds Q o Gam for the state pass's O1 product and the next chunk's Gam_last per
-// channel for its rescale.
+// above the diagonal, which can overflow, are masked away).  W = T Diag(b) (Khat o Gam)
+// (Gam_t = exp(G_t) <= 1) is a tensor-core product as for scalar gating, and T'' = T Diag(c)
+// goes to the record for the state pass's U' = T'' V; the record adds Q o Gam for the state
+// pass's O1 product and the chunk's own and the next chunk's Gam_last per channel for its
+// rescale.
 // =====================================================================================
 constexpr uint32_t PD_K = 0;         // raw K tile (16 KB, TMA: two 64-dk blocks)
-constexpr uint32_t PD_C = 16384;     // G fp32 [64][128] (32 KB); then L/T + scratch; then T', T'' hi/lo
+constexpr uint32_t PD_C = 16384;     // G fp32 [64][128] (32 KB); then L/T + scratch; then T' hi/lo
 constexpr uint32_t PD_D = 49152;     // next chunk's g (32 KB); then one dk half of the Gram operands
-                                     // (X hi/lo 32 KB, Y hi/lo 16 KB); then K o Gam hi/lo + V (48 KB)
+                                     // (X hi/lo 32 KB, Y hi/lo 16 KB); then K o Gam hi/lo (32 KB)
 constexpr uint32_t PD_MISC = PD_D + 49152;
 constexpr uint32_t PD_SMEM = PD_MISC + 5120 + 1024;
-constexpr uint32_t PDM_G = 0, PDM_W = 64, PDM_U = 128;  // TMEM columns (256 allocated)
+constexpr uint32_t PDM_G = 0, PDM_W = 64;  // TMEM columns (128 allocated)
 constexpr float kDiagRange = 160.f;  // in-chunk range of G above which the Gram is formed exactly
 
 struct PrepDiagMisc {
-    uint64_t full, nextg, vbar, mma;
+    uint64_t full, nextg, mma;
     uint32_t tmem_base, wide;
     float bco[CH], cco[CH], invr[CH], eta[CH];
     float R[DK], Gl[DK], gh[DK];
@@ -428,9 +418,8 @@ __device__ __forceinline__ void q_chunk8(const FwdArgs& a, int b, int t, int h, 
 }
 
 __global__ void __launch_bounds__(PT, 2)
-    chunk_prep_diag_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                           const __grid_constant__ CUtensorMap tm_g, FwdArgs a, uint8_t* __restrict__ recs,
-                           int cfirst) {
+    chunk_prep_diag_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_g, FwdArgs a,
+                           uint8_t* __restrict__ recs, int cfirst) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     PrepDiagMisc* ms = reinterpret_cast<PrepDiagMisc*>(sm + PD_MISC);
@@ -448,7 +437,7 @@ __global__ void __launch_bounds__(PT, 2)
     const bool has_next = c + 1 < NC;
     uint8_t* rec = recs + ((size_t)head * NC + c) * REC_BYTES_D;
     const uint32_t sbase = smem_u32(sm);
-    const uint32_t bar_full = smem_u32(&ms->full), bar_next = smem_u32(&ms->nextg), bar_v = smem_u32(&ms->vbar),
+    const uint32_t bar_full = smem_u32(&ms->full), bar_next = smem_u32(&ms->nextg),
                    bar_mma = smem_u32(&ms->mma);
 
     const float eta_own = (tid < n) ? a.eta[tok_index(b, t0 + tid, h, T, H)] : 0.f;
@@ -469,7 +458,6 @@ __global__ void __launch_bounds__(PT, 2)
     if (tid == 0) {
         mbar_init(bar_full, 1);
         mbar_init(bar_next, 1);
-        mbar_init(bar_v, 1);
         mbar_init(bar_mma, 1);
         fence_mbar_init();
         mbar_expect_tx(bar_full, 16384 + 32768);
@@ -483,7 +471,7 @@ __global__ void __launch_bounds__(PT, 2)
         ms->wide = 0u;
     }
     if (warp == 0) {
-        tmem_alloc(smem_u32(&ms->tmem_base), 256);
+        tmem_alloc(smem_u32(&ms->tmem_base), 128);
         tmem_relinquish();
     }
     if (tid < CH) ms->eta[tid] = eta_own;
@@ -492,7 +480,7 @@ __global__ void __launch_bounds__(PT, 2)
     tc_fence_after();
     const uint32_t tmem = ms->tmem_base;
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-    bool aborted = false, next_pending = has_next, v_pending = false;
+    bool aborted = false, next_pending = has_next;
     int mma_phase = 0;
 
     do {
@@ -653,13 +641,6 @@ __global__ void __launch_bounds__(PT, 2)
             }
         }
         if (aborted) break;
-        // ---- V for U' over the consumed Y operands
-        if (tid == 0) {
-            mbar_expect_tx(bar_v, 16384);
-            tma_load_4d(sbase + PD_D + 32768, &tm_v, bar_v, 0, h, t0, b);
-            tma_load_4d(sbase + PD_D + 40960, &tm_v, bar_v, 64, h, t0, b);
-        }
-        v_pending = true;
         // ---- a chunk too wide for the factored products: the Gram and scores exactly (row of
         //      [Q; Khat] = TMEM lane, 32 key columns a thread)
         if (wide) {
@@ -725,7 +706,7 @@ __global__ void __launch_bounds__(PT, 2)
         tc_fence_before();
         __syncthreads();
         invert_unit_lower64_doubling<PT>(Lf, Xs, tid);
-        // ---- T' = T Diag(b) and T'' = T Diag(c) as bf16 hi/lo over the L/T area
+        // ---- T' = T Diag(b) as bf16 hi/lo over the L/T area, T'' = T Diag(c) straight to the record
         {
             const int i = tid >> 2, qq = tid & 3;
             float tv[16];
@@ -737,21 +718,19 @@ __global__ void __launch_bounds__(PT, 2)
                     tv[4 * q] = t4.x; tv[4 * q + 1] = t4.y; tv[4 * q + 2] = t4.z; tv[4 * q + 3] = t4.w;
                 }
             }
-            __syncthreads();  // T is read; T' and T'' overwrite it
+            __syncthreads();  // T is read; T' overwrites it
             float v[16];
 #pragma unroll
             for (int e = 0; e < 16; ++e) v[e] = tv[e] * ms->bco[16 * qq + e];
             st_chunks_split(sm + PD_C, sm + PD_C + 8192, i, 2 * qq, 2, v);
 #pragma unroll
             for (int e = 0; e < 16; ++e) v[e] = tv[e] * ms->cco[16 * qq + e];
-            st_chunks_split(sm + PD_C + 16384, sm + PD_C + 24576, i, 2 * qq, 2, v);
+            st_chunks_split_global(rec + REC_TPP, rec + REC_TPP + 8192, i, 2 * qq, 2, v);
         }
         fence_proxy_async();
         tc_fence_before();
-        if (__syncthreads_or(!mbar_wait_bounded(bar_v, 0, kWaitNs))) { aborted = true; break; }
-        v_pending = false;
-        // ---- MMA: W^T = (K o Gam)^T T'^T (lane = dk; products hi.hi, hi.lo, lo.hi) and
-        //      U'^T = V^T T''^T (lane = dv)
+        __syncthreads();
+        // ---- MMA: W^T = (K o Gam)^T T'^T (lane = dk; products hi.hi, hi.lo, lo.hi)
         if (tid == kPrepIssuer) {
             tc_fence_after();
             const uint32_t iw = idesc_bf16(128, 64, true, false);
@@ -761,12 +740,6 @@ __global__ void __launch_bounds__(PT, 2)
                 for (int s = 0; s < 4; ++s)
                     mma_bf16(tmem + PDM_W, smem_desc(sbase + PD_D + (p == 2 ? 16384 : 0) + s * 2048, 8192, 1024),
                              smem_desc(sbase + PD_C + (p == 1 ? 8192 : 0) + s * 32, 16, 1024), iw, (p | s) > 0);
-#pragma unroll
-            for (int part = 0; part < 2; ++part)
-#pragma unroll
-                for (int s = 0; s < 4; ++s)
-                    mma_bf16(tmem + PDM_U, smem_desc(sbase + PD_D + 32768 + s * 2048, 8192, 1024),
-                             smem_desc(sbase + PD_C + 16384 + part * 8192 + s * 32, 16, 1024), iw, (part | s) > 0);
             mma_commit(bar_mma);
         }
         {
@@ -776,7 +749,7 @@ __global__ void __launch_bounds__(PT, 2)
         }
         tc_fence_after();
         // ---- -W transposed to [token][dk] over the consumed K o Gam tiles (one bulk copy to the
-        //      record); U' as [token][dv] rows straight to the record
+        //      record)
         {
             float x[32];
             tmem_ld32(tmem + lane_base + PDM_W + 32 * ch, x);
@@ -784,11 +757,6 @@ __global__ void __launch_bounds__(PT, 2)
 #pragma unroll
             for (int e = 0; e < 32; ++e) x[e] = -x[e];
             st_w_tokens_smem(sm + PD_D, row, 32 * ch, x, tid & 31);
-            tmem_ld32(tmem + lane_base + PDM_U + 32 * ch, x);
-            tmem_ld_wait();
-            float* up = reinterpret_cast<float*>(rec + REC_UP);
-#pragma unroll
-            for (int e = 0; e < 32; ++e) up[(32 * ch + e) * DV + row] = x[e];
             fence_proxy_async();
             __syncthreads();
             if (tid == 0) {
@@ -802,14 +770,13 @@ __global__ void __launch_bounds__(PT, 2)
         atomicOr(&g_split_error, 1u);
         // copies still in flight land before the block exits
         if (next_pending) (void)mbar_wait_bounded(bar_next, 0, kWaitNs);
-        if (v_pending) (void)mbar_wait_bounded(bar_v, 0, kWaitNs);
         (void)mbar_wait_bounded(bar_full, 0, kWaitNs);
     }
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
-        tmem_dealloc(tmem, 256);
+        tmem_dealloc(tmem, 128);
     }
 }
 
@@ -828,23 +795,27 @@ __global__ void __launch_bounds__(PT, 2)
 // An MMA issue blocks its thread while the tensor pipe drains, so no epilogue work sits on the
 // issuing warp; and the S and U operands are released in halves, so the first K steps of the
 // MMA that consumes them run while the epilogue finishes the second half.  Per chunk c:
-//   issuer    [U | O1 hi](c) [2 halves] | O1 lo(c) | S(c) [2 halves] O2(c)
-//   epilogue  U epi(c) -> S hi/lo(c+1) -> master rescale -> O epi(c)
-//   loader    refill of chunk c's stage with chunk c + 2 (part A: -W, Q, P, U' once chunk c's
-//             MMAs are done; part B: Ktil and scalars once the o tile has left by TMA store)
+//   issuer    U'(c) = V^T T''^T | [U | O1 hi](c) [2 halves] | O1 lo(c) | S(c) [2 halves] O2(c)
+//   epilogue  U epi(c) -> S hi/lo(c+1) -> master rescale -> O epi(c) (O1 zeroed once read)
+//   loader    refill of chunk c's stage with chunk c + 2 (part A: -W, Q, P, T'', V once chunk
+//             c's MMAs are done; part B: Ktil and scalars once the o tile has left by TMA store)
+// U'(c) accumulates into U's columns ahead of the S-dependent product, so it runs while the
+// previous chunk's state epilogue does; O1, which shares that N = 128 accumulator, is zeroed by
+// the output epilogue after reading it so that the [U | O1] product can always accumulate.
 // =====================================================================================
 constexpr int ST = 320;
 constexpr int kIssuerWarp = 8, kLoaderWarp = 9;
-constexpr uint32_t S_STAGE = 114688;  // Q 16 KB + the record's tiles (96 KB)
+constexpr uint32_t S_STAGE = 114688;  // Q 16 KB + the record's tiles (80 KB) + V 16 KB
 // SO_WQ: [-W block 0 | Q block 0 | -W block 1 | Q block 1], 8 KB each ([64 tokens x 64 dk]),
 // so that one K-major descriptor over 128 rows reads -W then Q for the same 16 dk: the U and
 // O1 products share their A operand (S^T) and run as N = 128 MMAs.  The o tile is staged over
 // Ktil (32 KB) once the chunk's MMAs are done.
-constexpr uint32_t SO_WQ = 0, SO_KT = 32768, SO_KTLO = 49152, SO_P = 65536, SO_PLO = 73728, SO_UP = 81920;
+constexpr uint32_t SO_WQ = 0, SO_KT = 32768, SO_KTLO = 49152, SO_P = 65536, SO_PLO = 73728, SO_TPP = 81920,
+                   SO_V = 98304;
 static_assert(SO_KT == REC_KT + 16384 && SO_KTLO == REC_KTLO + 16384 && SO_P == REC_P + 16384 &&
-                  SO_UP == REC_UP + 16384,
+                  SO_TPP == REC_TPP + 16384,
               "stage mirrors the record");
-static_assert(S_STAGE - SO_KT == 32768 + 16384 + 32768, "Ktil, P, U' fill the rest of the stage");
+static_assert(S_STAGE - SO_KT == 32768 + 16384 + 16384 + 16384, "Ktil, P, T'', V fill the rest of the stage");
 constexpr uint32_t S_SC = 2 * S_STAGE;  // 2 x 512 B record scalars
 constexpr uint32_t S_MISC = S_SC + 2 * REC_SCB;
 constexpr uint32_t S_GL0 = S_MISC + 256;  // diagonal gating: the first chunk's Gam_last[128]
@@ -872,8 +843,8 @@ __device__ __forceinline__ void tma_store_4d(const void* tmap, uint32_t src, int
 }
 template <typename TOut, bool DIAG>
 __global__ void __launch_bounds__(ST, 1)
-    chunk_state_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_o, FwdArgs a,
-                       const uint8_t* __restrict__ recs) {
+    chunk_state_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_v,
+                       const __grid_constant__ CUtensorMap tm_o, FwdArgs a, const uint8_t* __restrict__ recs) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     StateMisc* ms = reinterpret_cast<StateMisc*>(sm + S_MISC);
@@ -961,8 +932,9 @@ __global__ void __launch_bounds__(ST, 1)
         // ================================ loader ================================
         if (lane == 0) {
             prefetch_tmap(&tm_q);
+            if (need_vals) prefetch_tmap(&tm_v);
             if (write_o) prefetch_tmap(&tm_o);
-            // Part A of chunk c (-W, Q, P, U': the operands of its first products) can land as soon
+            // Part A of chunk c (-W, Q, P, T'', V: the operands of its first products) can land as soon
             // as chunk c - 2's MMAs are done; part B (Ktil, needed from the S product on, and the
             // scalars, read by the epilogues up to chunk c - 2's o tile) only after that tile,
             // staged over Ktil, has left by TMA store.
@@ -986,8 +958,9 @@ __global__ void __launch_bounds__(ST, 1)
                     bulk_load(base + SO_P, rec + REC_P, 16384, bar);
                 }
                 if (need_vals) {
-                    bulk_load(base + SO_UP, rec + REC_UP, 16384, bar);
-                    bulk_load(base + SO_UP + 16384, rec + REC_UP + 16384, 16384, bar);
+                    bulk_load(base + SO_TPP, rec + REC_TPP, 16384, bar);
+                    tma_load_4d(base + SO_V, &tm_v, bar, 0, h, c * CH, b);
+                    tma_load_4d(base + SO_V + 8192, &tm_v, bar, 64, h, c * CH, b);
                 }
             };
             auto load_b = [&](int c, int st) {
@@ -1047,8 +1020,20 @@ __global__ void __launch_bounds__(ST, 1)
                 const int lc = c - c0, st = lc & 1;
                 const uint32_t stg = sbase + st * S_STAGE;
                 if (!mbar_wait_bounded(full_a0 + 8 * st, (lc >> 1) & 1, kWaitNs)) { aborted = true; break; }
-                // [U^T | O1] = S^T [-W^T | Q^T] (N = 128; the record holds -W, U' is added in the
-                // epilogue), once the previous chunk's O1 and O2 are read.  K steps {0,1,4,5} read
+                // U'^T = V^T T''^T into U's columns (the previous chunk's U was read before its
+                // u_ready arrivals, which this thread has waited for): products V x T'' hi, lo
+                if (need_vals) {
+                    tc_fence_after();
+                    const uint32_t iv = idesc_bf16(128, 64, true, false);
+#pragma unroll
+                    for (int part = 0; part < 2; ++part)
+#pragma unroll
+                        for (int s = 0; s < 4; ++s)
+                            mma_bf16(tmem + TM_U, smem_desc(stg + SO_V + s * 2048, 8192, 1024),
+                                     smem_desc(stg + SO_TPP + part * 8192 + s * 32, 16, 1024), iv, (part | s) > 0);
+                }
+                // [U^T | O1] = S^T [-W^T | Q^T] (N = 128; the record holds -W), accumulated onto U'
+                // and onto the zeroed O1 once the previous chunk's O1 and O2 are read.  K steps {0,1,4,5} read
                 // the first half of each thread's S columns, {2,3,6,7} the second.  U takes S as its
                 // bf16 hi part only: W is itself one bf16 rounding, and the lo part's share is
                 // below that (measured: max|err|/rms of o and S_T 3.3e-3 against 2.7e-3 with both
@@ -1067,7 +1052,7 @@ __global__ void __launch_bounds__(ST, 1)
                         const int s = 2 * half + (j & 1) + 4 * (j >> 1);
                         mma_bf16_ts(tmem + TM_U, tmem + TM_SH + 8 * s,
                                     smem_desc(stg + SO_WQ + (s >> 2) * 16384 + (s & 3) * 32, 16, 1024),
-                                    write_o ? iuo : iu, (half | j) > 0);
+                                    write_o ? iuo : iu, need_vals || (half | j) > 0);
                     }
                 }
                 if (aborted) break;
@@ -1138,15 +1123,20 @@ __global__ void __launch_bounds__(ST, 1)
                 for (int e = 0; e < 32; ++e) x[e] *= diag ? gl0[dk0 + e] : g0;
                 tmem_st32(tmem + lane_base + TM_S + 64 * ch + 32 * q2, x);
             }
+            if (write_o) {  // O1 starts at zero: the [U | O1] product always accumulates
+                float z[32];
+#pragma unroll
+                for (int e = 0; e < 32; ++e) z[e] = 0.f;
+                tmem_st32(tmem + lane_base + TM_O1 + 32 * ch, z);
+            }
             epi_signal(s_ready0, tid);
             if (lane == 0) mbar_arrive(s_ready0 + 8);
         }
         for (int c = c0; c < c1; ++c) {
             const int lc = c - c0, st = lc & 1;
-            const uint8_t* stg_p = sm + st * S_STAGE;
             const bool has_next = c + 1 < c1;
-            // ---- U epilogue: U = U' + acc to bf16 hi/lo A operands (thread = dv, tokens
-            //      32 ch .. + 32), released in two halves of 16 tokens
+            // ---- U epilogue: U (U' - W S, accumulated) to bf16 hi/lo A operands (thread = dv,
+            //      tokens 32 ch .. + 32), released in two halves of 16 tokens
             {
                 const bool ok = mbar_wait_bounded(bar_u, lc & 1, kWaitNs);
                 if (__any_sync(0xffffffffu, !ok)) { aborted = true; break; }
@@ -1154,14 +1144,9 @@ __global__ void __launch_bounds__(ST, 1)
                 float x[32];
                 tmem_ld32(tmem + lane_base + TM_U + 32 * ch, x);
                 tmem_ld_wait();
-                const float* up = reinterpret_cast<const float*>(stg_p + SO_UP);
                 uint8_t* Ut = Utl ? Utl + (size_t)c * 32768 : nullptr;
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
-                    if (!ident) {
-#pragma unroll
-                        for (int e = 16 * half; e < 16 * half + 16; ++e) x[e] += up[(32 * ch + e) * DV + row];
-                    }
                     uint32_t hp[8], lp[8];
                     split_pack<16>(x + 16 * half, hp, lp);
                     tmem_st8u(tmem + lane_base + TM_UH + 16 * ch + 8 * half, hp);
@@ -1246,6 +1231,12 @@ __global__ void __launch_bounds__(ST, 1)
                     tmem_ld32(tmem + lane_base + TM_O1 + 32 * ch, o1);
                     tmem_ld32(tmem + lane_base + TM_O2 + 32 * ch, o2);
                     tmem_ld_wait();
+                    {  // O1 back to zero for the next chunk's accumulating [U | O1] product
+                        float z[32];
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) z[e] = 0.f;
+                        tmem_st32(tmem + lane_base + TM_O1 + 32 * ch, z);
+                    }
                     epi_signal(o_read, tid);  // the next chunk's [U | O1] product may start
 #pragma unroll
                     for (int e = 0; e < 32; ++e) {
@@ -1420,13 +1411,14 @@ bool make_out_map(CUtensorMap* m, void* base, int B, int T, int H, bool bf16) {
 
 template <typename TOut>
 cudaError_t launch_state(const CUtensorMap& mq, const FwdArgs& a, const uint8_t* recs, dim3 grid, cudaStream_t st) {
-    CUtensorMap mo;
+    CUtensorMap mo, mv;
     memset(&mo, 0, sizeof(mo));
     if (a.o != nullptr && !make_out_map(&mo, a.o, a.B, a.T, a.H, a.out_bf16)) return cudaErrorInvalidValue;
+    if (!make_map(&mv, a.v, a.B, a.T, a.H)) return cudaErrorInvalidValue;  // V for U' = T'' V (required)
     auto kern = a.diag ? chunk_state_kernel<TOut, true> : chunk_state_kernel<TOut, false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)S_SMEM);
     if (e != cudaSuccess) return e;
-    kern<<<grid, ST, S_SMEM, st>>>(mq, mo, a, recs);
+    kern<<<grid, ST, S_SMEM, st>>>(mq, mv, mo, a, recs);
     return cudaGetLastError();
 }
 
@@ -1446,24 +1438,20 @@ namespace {
 // Preparation of chunks [cfirst, cfirst + count) of every head.
 cudaError_t launch_prep_range(const FwdArgs& a, void* ws, int cfirst, int count, cudaStream_t st) {
     if (a.diag) {
-        CUtensorMap mk, mv, mg;
-        if (!make_map(&mk, a.k, a.B, a.T, a.H) || !make_map(&mv, a.v, a.B, a.T, a.H) ||
-            !make_out_map(&mg, const_cast<float*>(a.g), a.B, a.T, a.H, false))
+        CUtensorMap mk, mg;
+        if (!make_map(&mk, a.k, a.B, a.T, a.H) || !make_out_map(&mg, const_cast<float*>(a.g), a.B, a.T, a.H, false))
             return cudaErrorInvalidValue;
         cudaError_t e =
             cudaFuncSetAttribute(chunk_prep_diag_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PD_SMEM);
         if (e != cudaSuccess) return e;
-        chunk_prep_diag_kernel<<<dim3(count, a.B * a.H), PT, PD_SMEM, st>>>(mk, mv, mg, a, static_cast<uint8_t*>(ws),
-                                                                           cfirst);
+        chunk_prep_diag_kernel<<<dim3(count, a.B * a.H), PT, PD_SMEM, st>>>(mk, mg, a, static_cast<uint8_t*>(ws), cfirst);
         return cudaGetLastError();
     }
-    CUtensorMap mq, mk, mv;
-    if (!make_map(&mq, a.q, a.B, a.T, a.H) || !make_map(&mk, a.k, a.B, a.T, a.H) ||
-        !make_map(&mv, a.v, a.B, a.T, a.H))
-        return cudaErrorInvalidValue;
+    CUtensorMap mq, mk;
+    if (!make_map(&mq, a.q, a.B, a.T, a.H) || !make_map(&mk, a.k, a.B, a.T, a.H)) return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(chunk_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)P_SMEM);
     if (e != cudaSuccess) return e;
-    chunk_prep_kernel<<<dim3(count, a.B * a.H), PT, P_SMEM, st>>>(mq, mk, mv, a, static_cast<uint8_t*>(ws), cfirst);
+    chunk_prep_kernel<<<dim3(count, a.B * a.H), PT, P_SMEM, st>>>(mq, mk, a, static_cast<uint8_t*>(ws), cfirst);
     return cudaGetLastError();
 }
 // One non-segmented state-pass run over chunks [f.chunk0, f.chunk0 + f.seg_chunks) of every head.

@@ -570,7 +570,7 @@ EncodeTiledFn get_encode_fn() {
 
 bool make_map(CUtensorMap* m, const void* base, int B, int T, int H) {
     EncodeTiledFn enc = get_encode_fn();
-    if (!enc) return false;
+    if (!enc || base == nullptr) return false;
     cuuint64_t dims[4] = {(cuuint64_t)128, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
     cuuint64_t strides[3] = {(cuuint64_t)128 * 2, (cuuint64_t)H * 128 * 2, (cuuint64_t)T * H * 128 * 2};
     cuuint32_t box[4] = {64, 1, 64, 1};

@@ -191,11 +191,11 @@ __global__ void __launch_bounds__(NT, CTAS_PER_SM)
         }
         // lanes c, c + CG, ... hold the same columns (several rows of the warp): fold them
 #pragma unroll
-        for (int o = CG; o < 32; o <<= 1) {
-            pk.x += __shfl_xor_sync(0xffffffffu, pk.x, o); pk.y += __shfl_xor_sync(0xffffffffu, pk.y, o);
-            pk.z += __shfl_xor_sync(0xffffffffu, pk.z, o); pk.w += __shfl_xor_sync(0xffffffffu, pk.w, o);
-            pq.x += __shfl_xor_sync(0xffffffffu, pq.x, o); pq.y += __shfl_xor_sync(0xffffffffu, pq.y, o);
-            pq.z += __shfl_xor_sync(0xffffffffu, pq.z, o); pq.w += __shfl_xor_sync(0xffffffffu, pq.w, o);
+        for (int sh = CG; sh < 32; sh <<= 1) {
+            pk.x += __shfl_xor_sync(0xffffffffu, pk.x, sh); pk.y += __shfl_xor_sync(0xffffffffu, pk.y, sh);
+            pk.z += __shfl_xor_sync(0xffffffffu, pk.z, sh); pk.w += __shfl_xor_sync(0xffffffffu, pk.w, sh);
+            pq.x += __shfl_xor_sync(0xffffffffu, pq.x, sh); pq.y += __shfl_xor_sync(0xffffffffu, pq.y, sh);
+            pq.z += __shfl_xor_sync(0xffffffffu, pq.z, sh); pq.w += __shfl_xor_sync(0xffffffffu, pq.w, sh);
         }
         kk = warp_sum(kk);
         kq = warp_sum(kq);

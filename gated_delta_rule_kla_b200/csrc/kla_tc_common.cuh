@@ -416,8 +416,9 @@ constexpr uint32_t REC_W = 0;        // -W bf16: [64 tokens x 64 dk] x 2 blocks 
 constexpr uint32_t REC_KT = 16384;   // Ktil hi: [64 tokens x 64 dk] x 2 blocks        16 KB
 constexpr uint32_t REC_KTLO = 32768; // Ktil lo                                        16 KB
 constexpr uint32_t REC_P = 49152;    // P hi [64 x 64], then P lo                       16 KB
-constexpr uint32_t REC_UP = 65536;   // U' fp32 [64 tokens][128 dv]                      32 KB
-constexpr uint32_t REC_TILES = 98304;
+constexpr uint32_t REC_TPP = 65536;  // T'' = T Diag(c) hi [64 x 64], then lo              16 KB
+                                     // (the state pass forms U' = T'' V itself)
+constexpr uint32_t REC_TILES = 81920;
 constexpr uint32_t REC_SC = REC_TILES;  // gamma[64], gamma_last of the next chunk, of the previous chunk  512 B
 constexpr uint32_t REC_SCB = 512;
 constexpr size_t REC_BYTES = REC_TILES + REC_SCB;

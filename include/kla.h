@@ -96,7 +96,7 @@ int kla_version(void);
  *                     contents need not be initialised), or NULL.  With at least
  *                     kla_chunk_fwd_workspace() bytes, bf16 inputs with Dk == Dv == 128 run the
  *                     split path: a chunk-parallel kernel stores every chunk's state-independent
- *                     operands there (about 97 KiB per chunk and head), then a sequential state
+ *                     operands there (about 80.5 KiB per chunk and head), then a sequential state
  *                     pass consumes them (segmented, for long sequences over few heads).  With
  *                     NULL or a smaller buffer the forward still runs, as one fused kernel per
  *                     head.  The workspace must not be shared with a concurrent call.
@@ -123,23 +123,23 @@ kla_status kla_chunk_fwd(const void *q, const void *k, const void *v, const floa
  * another stream, or timing each stage).  Same math as kla_chunk_fwd ("Kaczmarz Linear
  * Attention", section 4, Eqs. 7-9): _prep computes, for every chunk in parallel, everything that
  * does not depend on the incoming state (key norms and Kaczmarz coefficients, decays, the UT
- * transform inverse, W, U', the decayed keys, the masked scores) and stores it in ws; _state then
- * runs the sequential state pass from ws.  Together they equal one kla_chunk_fwd call with that
- * workspace, bit for bit.
+ * transform inverse and W, T Diag(c) for U' = T Diag(c) V, the decayed keys, the masked scores)
+ * and stores it in ws; _state then runs the sequential state pass from ws, reading q and v
+ * (for U') itself.  Together they equal one kla_chunk_fwd call with that workspace, bit for bit.
  *   Arguments as for kla_chunk_fwd.  Only dtype == KLA_BF16 with Dk == Dv == 128 and T >= 1 is
  *   supported (KLA_ERR_UNSUPPORTED / KLA_ERR_INVALID_ARG otherwise).  ws (device, 32-byte
  *   aligned, at least kla_chunk_fwd_workspace() bytes, owned by the caller) is required
- *   (KLA_ERR_WORKSPACE otherwise); _state must get the same ws, q, g and sizes as the _prep
+ *   (KLA_ERR_WORKSPACE otherwise); _state must get the same ws, q, v, g and sizes as the _prep
  *   call it follows, ordered after it (same stream, or an event), with ws untouched between.
  * Returns KLA_OK or an error status; on error nothing is launched.
  */
 kla_status kla_chunk_fwd_prep(const void *q, const void *k, const void *v, const float *eta,
                               const float *g, float eps, int B, int T, int H, int Dk, int Dv,
                               int chunk, int dtype, void *ws, size_t ws_bytes, void *stream);
-kla_status kla_chunk_fwd_state(const void *q, const float *g, const float *S0, void *o,
-                               float *S_T, float *S_chunks, int B, int T, int H, int Dk, int Dv,
-                               int chunk, int dtype, int out_dtype, void *ws, size_t ws_bytes,
-                               void *stream);
+kla_status kla_chunk_fwd_state(const void *q, const void *v, const float *g, const float *S0,
+                               void *o, float *S_T, float *S_chunks, int B, int T, int H, int Dk,
+                               int Dv, int chunk, int dtype, int out_dtype, void *ws,
+                               size_t ws_bytes, void *stream);
 
 /*
  * kla_chunk_bwd -- gradients of the chunkwise forward.
@@ -241,7 +241,7 @@ kla_status kla_decode_step(const void *q, const void *k, const void *v, const fl
  *                         least kla_chunk_fwd_diag_workspace() bytes selects the split path: a
  *                         chunk-parallel kernel stores every chunk's state-independent operands
  *                         there, then a sequential state pass reads them.  bf16 with Dk = Dv =
- *                         128 runs both on the tensor cores over 64-token chunks (a 113 KiB
+ *                         128 runs both on the tensor cores over 64-token chunks (a 97 KiB
  *                         record per chunk and head, as two slabs or parallel segments like
  *                         kla_chunk_fwd); other shapes run on the CUDA cores over 16-token
  *                         chunks (about 34 KiB per chunk and head at Dk = Dv = 128).  With NULL

@@ -62,16 +62,16 @@ def test_fwd_rejects_before_launch(L, kw, code):
 
 def test_fwd_stages_reject_before_launch(L):
     need = L.kla_chunk_fwd_workspace(2, 300, 3, 128, 128, 64, 1)
-    assert need >= 2 * 3 * 5 * 98816  # one record of ~97 KiB per chunk and head
+    assert need >= 2 * 3 * 5 * 82432  # one record of ~80.5 KiB per chunk and head
     prep = lambda dtype=1, Dk=128, T=300, ws=FAKE, n=need: L.kla_chunk_fwd_prep(
         FAKE, FAKE, FAKE, FAKE, FAKE, 1e-6, 2, T, 3, Dk, 128, 64, dtype, ws, n, None)
-    state = lambda dtype=1, ws=FAKE, n=need, q=FAKE: L.kla_chunk_fwd_state(
-        q, FAKE, None, FAKE, None, None, 2, 300, 3, 128, 128, 64, dtype, 0, ws, n, None)
+    state = lambda dtype=1, ws=FAKE, n=need, q=FAKE, v=FAKE: L.kla_chunk_fwd_state(
+        q, v, FAKE, None, FAKE, None, None, 2, 300, 3, 128, 128, 64, dtype, 0, ws, n, None)
     assert prep(dtype=0) == UNSUPPORTED and prep(Dk=64) == UNSUPPORTED
     assert prep(T=0) == INVALID
     assert prep(ws=None) == WORKSPACE and prep(n=need - 1) == WORKSPACE
     assert state(dtype=0) == UNSUPPORTED and state(ws=None) == WORKSPACE
-    assert state(q=None) == INVALID and state(ws=MISALIGNED) == INVALID
+    assert state(q=None) == INVALID and state(v=None) == INVALID and state(ws=MISALIGNED) == INVALID
     assert b"aligned" in L.kla_last_error()
     assert state(ws=None) == WORKSPACE and b"kla_chunk_fwd_state" in L.kla_last_error()
 
@@ -196,10 +196,10 @@ def test_backward_reverse_segments(L):
 
 
 def test_diag_forward_workspace_by_path(L):
-    """bf16 at Dk = Dv = 128 takes the tensor-core split path: one record of 113 KiB per 64-token
+    """bf16 at Dk = Dv = 128 takes the tensor-core split path: one record of 97 KiB per 64-token
     chunk and head; other shapes the CUDA-core split path over 16-token chunks."""
     tc = L.kla_chunk_fwd_diag_workspace(2, 300, 3, 128, 128, 64, 1)
-    assert tc >= 2 * 3 * 5 * 115200
+    assert tc >= 2 * 3 * 5 * 99328
     assert L.kla_chunk_fwd_diag_kernel_launches(2, 300, 3, 128, 128, 64, 1) >= 2
     simt = L.kla_chunk_fwd_diag_workspace(2, 300, 3, 128, 128, 64, 0)
     assert simt >= 2 * 3 * 19 * 4 * (3 * 16 * 128 + 16 * 16 + 128)

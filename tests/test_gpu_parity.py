@@ -189,7 +189,7 @@ def test_fwd_prep_and_state_stages_equal_one_call(kla, B, T, H, launches):
     ws2 = kla.fwd_workspace(d["k"], d["v"])
     Sc2 = torch.empty_like(Sc)
     kla.chunk_fwd_prep(d["q"], d["k"], d["v"], d["eta"], d["g"], 1e-6, ws2)
-    o2, ST2 = kla.chunk_fwd_state(d["q"], d["g"], d["S0"], ws2, S_chunks=Sc2)
+    o2, ST2 = kla.chunk_fwd_state(d["q"], d["v"], d["g"], d["S0"], ws2, S_chunks=Sc2)
     torch.cuda.synchronize()
     kla.check_device_error()
     assert torch.equal(o, o2) and torch.equal(ST, ST2) and torch.equal(Sc, Sc2)
