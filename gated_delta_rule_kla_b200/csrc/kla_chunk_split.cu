@@ -1311,25 +1311,25 @@ size_t align1k(size_t x) { return (x + 1023) & ~size_t(1023); }
 // Two slabs: the state pass holds one SM per head for the whole sequence, so with few heads
 // most SMs idle while it runs.  Splitting the chunks into two slabs lets the second slab's
 // preparation run on those SMs while the first slab's state pass runs, the second state pass
-// starting from the first one's final state.  Cost model in
-// state steps (one chunk of the state pass, ~2.3 us here); a wave of preparation CTAs (three
-// per SM) takes kPrepWaveSteps of them (measured: ~18.7 us per wave).  Returns the first
-// slab's chunk count, or 0 for one run.
+// starting from the first one's final state.  Cost model in state steps (one chunk of the
+// state pass, ~2.5 us here); a wave of preparation CTAs (four per SM for scalar gating, two for
+// diagonal gating) takes prep_wave of them (measured: ~21 us and ~27 us per wave).  Returns
+// the first slab's chunk count, or 0 for one run.
 // The first slab's preparation has the whole GPU: whole waves, and a last partial wave that
 // costs 0.45 + 0.55 x its fill (its CTAs share their SMs with fewer others); the second slab's
 // runs beside the state pass and spills onto its SMs when it ends, so it is counted fluidly.
-// Calibrated on the B=8 T=2048 H=8 and B=4 T=4096 H=16 forwards (sweeps of the split point:
-// optima at 20 of 32 and 41-42 of 64 chunks).
-constexpr double kPrepWaveSteps = 8.1;
-int choose_slab_split(int BH, int NC) {
+// Calibrated on the B=8 T=2048 H=8 forward (a sweep of the split point: optimum at 18 of 32
+// chunks, 151.6 us, against 155.6 us at 20 and 164.9 us as one run).
+int choose_slab_split(int BH, int NC, bool diag) {
     const int sms = sm_count();
     if (NC < 8 || 2 * BH > sms) return 0;
+    const double per_sm = diag ? 2.0 : 4.0, prep_wave = diag ? 10.4 : 8.5;
     auto prep_all = [&](long long items) {
-        const long long slots = 3LL * sms, full = items / slots;
+        const long long slots = (long long)per_sm * sms, full = items / slots;
         const double frac = (double)(items - full * slots) / slots;
-        return (full + (frac > 0 ? 0.45 + 0.55 * frac : 0.0)) * kPrepWaveSteps;
+        return (full + (frac > 0 ? 0.45 + 0.55 * frac : 0.0)) * prep_wave;
     };
-    auto prep_beside = [&](double items) { return items / (3.0 * (sms - BH)) * kPrepWaveSteps; };
+    auto prep_beside = [&](double items) { return items / (per_sm * (sms - BH)) * prep_wave; };
     const double base = prep_all((long long)NC * BH) + NC;
     double best = base;
     int nc1 = 0;
@@ -1366,7 +1366,7 @@ SplitLayout split_layout(const FwdArgs& a) {
         L.nseg = 1;
         L.segc = NC;
         L.total = L.seg_off;
-        L.nc1 = choose_slab_split(BH, NC);
+        L.nc1 = choose_slab_split(BH, NC, a.diag);
         if (L.nc1 > 0) {
             L.slab_off = L.total;
             L.total += (size_t)BH * DK * DV * sizeof(float);

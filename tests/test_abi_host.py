@@ -205,3 +205,6 @@ def test_diag_forward_workspace_by_path(L):
     assert simt >= 2 * 3 * 19 * 4 * (3 * 16 * 128 + 16 * 16 + 128)
     assert L.kla_chunk_fwd_diag_kernel_launches(2, 300, 3, 128, 128, 64, 0) == 2
     assert L.kla_chunk_fwd_diag_kernel_launches(2, 300, 3, 96, 128, 64, 1) == 0
+    # 32 heads over 10 chunks run as two slabs (148 SMs); one head over 65 chunks as segments
+    assert L.kla_chunk_fwd_diag_kernel_launches(2, 640, 16, 128, 128, 64, 1) == 4
+    assert L.kla_chunk_fwd_diag_kernel_launches(1, 4100, 1, 128, 128, 64, 1) == 4

@@ -70,7 +70,7 @@ FWD_CASES = [
     # preparation forms the pairwise decay factors exactly instead of around a reference
     (1, 130, 2, 128, 128, "bf16", -5.0, True, "kaczmarz"),
     (1, 70, 1, 128, 128, "bf16", -12.0, False, "kaczmarz"),
-    (1, 1024, 2, 128, 128, "bf16", -0.5, True, "kaczmarz"),  # two slabs
+    (2, 640, 16, 128, 128, "bf16", -0.5, True, "kaczmarz"),  # two slabs (5 and 5 chunks)
     (1, 4100, 1, 128, 128, "bf16", -0.5, True, "kaczmarz"),  # parallel segments and the scan
 ]
 
