@@ -1099,25 +1099,36 @@ __global__ void __launch_bounds__(NTS, 1) diag_state_kernel(FwdArgs a, const flo
                     *reinterpret_cast<const float4*>(Ss + r * 64 + c4);
             }
         }
-        // -W S and QG S over this half's state rows d in [half DK/2, half DK/2 + DK/2)
+        // -W S (and QG S when o is wanted; the backward's state recompute wants none) over this
+        // half's state rows d in [half DK/2, half DK/2 + DK/2)
         float4 u = make_float4(0.f, 0.f, 0.f, 0.f), oo = u;
         {
             const float* wr = rs + R::W + i * DK;
             const float* qr = rs + R::QG + i * DK;
             const int d0 = half * (DK / 2);
+            if (o != nullptr) {
 #pragma unroll 8
-            for (int d = d0; d < d0 + DK / 2; ++d) {
-                const float w = wr[d], q = qr[d];
-                const float4 s4 = *reinterpret_cast<const float4*>(Ss + d * 64 + cx);
-                u.x = fmaf(-w, s4.x, u.x); u.y = fmaf(-w, s4.y, u.y);
-                u.z = fmaf(-w, s4.z, u.z); u.w = fmaf(-w, s4.w, u.w);
-                oo.x = fmaf(q, s4.x, oo.x); oo.y = fmaf(q, s4.y, oo.y);
-                oo.z = fmaf(q, s4.z, oo.z); oo.w = fmaf(q, s4.w, oo.w);
+                for (int d = d0; d < d0 + DK / 2; ++d) {
+                    const float w = wr[d], q = qr[d];
+                    const float4 s4 = *reinterpret_cast<const float4*>(Ss + d * 64 + cx);
+                    u.x = fmaf(-w, s4.x, u.x); u.y = fmaf(-w, s4.y, u.y);
+                    u.z = fmaf(-w, s4.z, u.z); u.w = fmaf(-w, s4.w, u.w);
+                    oo.x = fmaf(q, s4.x, oo.x); oo.y = fmaf(q, s4.y, oo.y);
+                    oo.z = fmaf(q, s4.z, oo.z); oo.w = fmaf(q, s4.w, oo.w);
+                }
+            } else {
+#pragma unroll 8
+                for (int d = d0; d < d0 + DK / 2; ++d) {
+                    const float w = wr[d];
+                    const float4 s4 = *reinterpret_cast<const float4*>(Ss + d * 64 + cx);
+                    u.x = fmaf(-w, s4.x, u.x); u.y = fmaf(-w, s4.y, u.y);
+                    u.z = fmaf(-w, s4.z, u.z); u.w = fmaf(-w, s4.w, u.w);
+                }
             }
         }
         if (half) {
             *reinterpret_cast<float4*>(Pu + i * 64 + cx) = u;
-            *reinterpret_cast<float4*>(Po + i * 64 + cx) = oo;
+            if (o != nullptr) *reinterpret_cast<float4*>(Po + i * 64 + cx) = oo;
         }
         __syncthreads();
         if (!half) {  // U = UP + both halves of -W S

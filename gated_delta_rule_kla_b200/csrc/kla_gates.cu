@@ -342,45 +342,91 @@ __global__ void __launch_bounds__(256) gate_bwd_tile_kernel(const Tin* __restric
         for (int t = 0; t < BT; ++t) s += dz[t * NW + tid];
         part_b[(size_t)tile * NW + tid] = s;
     }
-    // dx[t][c] = sum_j dz[t][j] W[j][c]: thread = column c (128) x token half
+    // thread = column c (128) x half th; NW = 2H is even, so dz rows are read two gates at a time
+    const int c = tid & (BD - 1), th = tid >> 7;
+    // dx[t][c] = sum_j dz[t][j] W[j][c] for the thread's tokens t = th + 2 m: W's column held in
+    // registers 16 gates at a time, dz rows broadcast
     {
-        const int c = tid & (BD - 1), th = tid >> 7;
+        float acc[BT / 2];
+#pragma unroll
+        for (int m = 0; m < BT / 2; ++m) acc[m] = 0.f;
+        for (int jb = 0; jb < NW; jb += 16) {
+            float wr[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) wr[e] = (jb + e < NW) ? wsh[(jb + e) * (BD + 1) + c] : 0.f;
+#pragma unroll
+            for (int m = 0; m < BT / 2; ++m) {
+                const float* zr = dz + (th + 2 * m) * NW + jb;
+                float s = acc[m];
+#pragma unroll
+                for (int e = 0; e < 16; e += 2) {
+                    if (jb + e < NW) {
+                        const float2 z2 = *reinterpret_cast<const float2*>(zr + e);
+                        s = fmaf(z2.x, wr[e], s);
+                        s = fmaf(z2.y, wr[e + 1], s);
+                    }
+                }
+                acc[m] = s;
+            }
+        }
         if (c < nd) {
-            for (int t = th; t < nt; t += 2) {
-                float s = 0.f;
-                for (int j = 0; j < NW; ++j) s = fmaf(dz[t * NW + j], wsh[j * (BD + 1) + c], s);
-                dx[(size_t)(t0 + t) * D + d0 + c] = s;
+#pragma unroll
+            for (int m = 0; m < BT / 2; ++m) {
+                const int t = th + 2 * m;
+                if (t < nt) dx[(size_t)(t0 + t) * D + d0 + c] = acc[m];
             }
         }
     }
-    // dW partial [j][c] = sum_t dz[t][j] x[t][c]
-    for (int i = tid; i < NW * BD; i += 256) {
-        const int j = i / BD, c = i % BD;
-        if (c < nd) {
-            float s0 = 0.f, s1 = 0.f;
-            for (int t = 0; t < BT; t += 2) {
-                s0 = fmaf(dz[t * NW + j], xs[t * (BD + 1) + c], s0);
-                s1 = fmaf(dz[(t + 1) * NW + j], xs[(t + 1) * (BD + 1) + c], s1);
+    // dW partial [j][c] = sum_t dz[t][j] x[t][c]: the thread's gates j = th (mod 2), eight at a time
+    for (int jb = th * 8; jb < NW; jb += 16) {
+        float acc[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+        for (int t = 0; t < BT; ++t) {
+            const float xv = xs[t * (BD + 1) + c];
+            const float* zr = dz + t * NW + jb;
+#pragma unroll
+            for (int e = 0; e < 8; e += 2) {
+                if (jb + e < NW) {
+                    const float2 z2 = *reinterpret_cast<const float2*>(zr + e);
+                    acc[e] = fmaf(z2.x, xv, acc[e]);
+                    acc[e + 1] = fmaf(z2.y, xv, acc[e + 1]);
+                }
             }
-            part_w[((size_t)tile * NW + j) * D + d0 + c] = s0 + s1;
+        }
+        if (c < nd) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                if (jb + e < NW) part_w[((size_t)tile * NW + jb + e) * D + d0 + c] = acc[e];
         }
     }
 }
 
 // dW[j][d] = sum over tiles (fixed order), dbias[j] likewise.
-__global__ void gate_bwd_reduce_kernel(const float* __restrict__ part_w, const float* __restrict__ part_b,
-                                       float* __restrict__ dW, float* __restrict__ db, int ntile, int NW, int D) {
-    const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+// dW and dbias: the tiles' partial sums added in a fixed order.  A block takes 64 outputs; its
+// four thread groups each sum a quarter of the tiles in order, then the quarters are added in
+// order, so the result does not depend on scheduling.
+constexpr int RED_OUT = 64, RED_PARTS = 4;
+__global__ void __launch_bounds__(RED_OUT * RED_PARTS)
+    gate_bwd_reduce_kernel(const float* __restrict__ part_w, const float* __restrict__ part_b, float* __restrict__ dW,
+                           float* __restrict__ db, int ntile, int NW, int D) {
+    __shared__ float sums[RED_PARTS][RED_OUT];
+    const int p = threadIdx.x / RED_OUT, o = threadIdx.x % RED_OUT;
+    const size_t i = (size_t)blockIdx.x * RED_OUT + o;
     const size_t total = (size_t)NW * D;
-    if (i < total) {
-        float s = 0.f;
-        for (int t = 0; t < ntile; ++t) s += part_w[(size_t)t * total + i];
-        dW[i] = s;
-    }
-    if (i < (size_t)NW) {
-        float s = 0.f;
-        for (int t = 0; t < ntile; ++t) s += part_b[(size_t)t * NW + i];
-        db[i] = s;
+    const int per = (ntile + RED_PARTS - 1) / RED_PARTS, ta = p * per, tb = min(ntile, ta + per);
+    float s = 0.f;
+    if (i < total)
+        for (int t = ta; t < tb; ++t) s += part_w[(size_t)t * total + i];
+    sums[p][o] = s;
+    __syncthreads();
+    if (p == 0 && i < total) dW[i] = ((sums[0][o] + sums[1][o]) + sums[2][o]) + sums[3][o];
+    if (blockIdx.x == 0 && p == 0) {
+        for (int j = o; j < NW; j += RED_OUT) {
+            float sb = 0.f;
+            for (int t = 0; t < ntile; ++t) sb += part_b[(size_t)t * NW + j];
+            db[j] = sb;
+        }
     }
 }
 
@@ -481,8 +527,8 @@ cudaError_t launch_gate_prologue_bwd(const GateBwdArgs& a, void* ws, cudaStream_
         if (e != cudaSuccess) return e;
     }
     const size_t total = (size_t)NW * a.D;
-    gate_bwd_reduce_kernel<<<(unsigned)((total + 255) / 256), 256, 0, st>>>(part_w, part_b, a.dW, a.db, ntile, NW,
-                                                                            a.D);
+    gate_bwd_reduce_kernel<<<(unsigned)((total + RED_OUT - 1) / RED_OUT), RED_OUT * RED_PARTS, 0, st>>>(
+        part_w, part_b, a.dW, a.db, ntile, NW, a.D);
     return cudaGetLastError();
 }
 
