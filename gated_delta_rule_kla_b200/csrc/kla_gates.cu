@@ -22,6 +22,9 @@
 // the workspace and then over tiles in a fixed order (deterministic).
 #include <cuda.h>
 
+#include <mutex>
+#include <unordered_map>
+
 #include "kla_device.cuh"
 #include "kla_launch.h"
 #include "kla_sm100.cuh"
@@ -441,16 +444,72 @@ size_t gate_bwd_workspace(int N, int D, int H) {
     return ntile * 2 * H * ((size_t)D + 1) * sizeof(float);
 }
 
+namespace {
+// The query normalisation shares no data with the gate projection (nor, in the backward, with
+// the dx / dW kernels), so it runs on a second stream of the device beside them: the projection
+// launches fewer CTAs than there are SMs.  The caller's stream waits for both before anything
+// after the call.
+cudaError_t side_stream(cudaStream_t* out) {
+    static std::mutex mu;
+    static std::unordered_map<int, cudaStream_t> streams;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = streams.find(dev);
+    if (it == streams.end()) {
+        cudaStream_t s = nullptr;
+        if ((e = cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking)) != cudaSuccess) return e;
+        it = streams.emplace(dev, s).first;
+    }
+    *out = it->second;
+    return cudaSuccess;
+}
+
+// Runs `side_work` on the side stream after everything already queued on st, and `main_work`
+// on st; st then waits for the side stream.  Falls back to st alone if a side stream cannot be
+// had.  The side work is always joined back, whatever either part returns.
+template <typename FS, typename FM>
+cudaError_t run_beside(cudaStream_t st, FS side_work, FM main_work) {
+    cudaStream_t side = nullptr;
+    cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
+    cudaError_t e = side_stream(&side);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ev_fork, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ev_join, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventRecord(ev_fork, st);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(side, ev_fork, 0);
+    if (e != cudaSuccess) {
+        if (ev_fork) cudaEventDestroy(ev_fork);
+        if (ev_join) cudaEventDestroy(ev_join);
+        e = side_work(st);
+        return e == cudaSuccess ? main_work(st) : e;
+    }
+    e = side_work(side);
+    const cudaError_t er = cudaEventRecord(ev_join, side);
+    const cudaError_t em = e == cudaSuccess ? main_work(st) : e;
+    const cudaError_t ej = er == cudaSuccess ? cudaStreamWaitEvent(st, ev_join, 0) : er;
+    cudaEventDestroy(ev_fork);  // released once the work that uses them is done
+    cudaEventDestroy(ev_join);
+    return em != cudaSuccess ? em : ej;
+}
+
+cudaError_t launch_gates_only(const GateArgs& a, cudaStream_t st);
+}  // namespace
+
 cudaError_t launch_gate_prologue(const GateArgs& a, cudaStream_t st) {
     if (a.N == 0) return cudaSuccess;
-    if (a.q != nullptr) {
-        const size_t rows = (size_t)a.N * a.H;
-        const cudaError_t e = a.bf16 ? launch_qnorm(static_cast<const __nv_bfloat16*>(a.q),
-                                                    static_cast<__nv_bfloat16*>(a.qhat), rows, a.Dk, st)
-                                     : launch_qnorm(static_cast<const float*>(a.q), static_cast<float*>(a.qhat), rows,
-                                                    a.Dk, st);
-        if (e != cudaSuccess) return e;
-    }
+    if (a.q == nullptr) return launch_gates_only(a, st);
+    const size_t rows = (size_t)a.N * a.H;
+    auto qn = [&](cudaStream_t s) {
+        return a.bf16 ? launch_qnorm(static_cast<const __nv_bfloat16*>(a.q), static_cast<__nv_bfloat16*>(a.qhat), rows,
+                                     a.Dk, s)
+                      : launch_qnorm(static_cast<const float*>(a.q), static_cast<float*>(a.qhat), rows, a.Dk, s);
+    };
+    return run_beside(st, qn, [&](cudaStream_t s) { return launch_gates_only(a, s); });
+}
+
+namespace {
+cudaError_t launch_gates_only(const GateArgs& a, cudaStream_t st) {
     if (gate_tc_shape(a)) {
         EncodeTiledFn enc = get_encode_fn();
         if (enc != nullptr) {
@@ -492,6 +551,7 @@ cudaError_t launch_gate_prologue(const GateArgs& a, cudaStream_t st) {
                                                                 a.N, a.D, a.H);
     return cudaGetLastError();
 }
+}  // namespace
 
 cudaError_t launch_gate_prologue_bwd(const GateBwdArgs& a, void* ws, cudaStream_t st) {
     if (a.N == 0) {
@@ -504,32 +564,37 @@ cudaError_t launch_gate_prologue_bwd(const GateBwdArgs& a, void* ws, cudaStream_
     float* part_w = static_cast<float*>(ws);
     float* part_b = part_w + (size_t)ntile * NW * a.D;
     const size_t smem = sizeof(float) * ((size_t)BT * NW + (size_t)BT * (BD + 1) + (size_t)NW * (BD + 1));
-    cudaError_t e;
-    if (a.bf16) {
-        e = cudaFuncSetAttribute(gate_bwd_tile_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)smem);
-        if (e != cudaSuccess) return e;
-        gate_bwd_tile_kernel<__nv_bfloat16><<<dim3(ntile, (a.D + BD - 1) / BD), 256, smem, st>>>(
-            static_cast<const __nv_bfloat16*>(a.x), static_cast<const __nv_bfloat16*>(a.W), a.eta, a.g, a.deta, a.dg,
-            a.dx, part_w, part_b, a.N, a.D, a.H);
-    } else {
-        e = cudaFuncSetAttribute(gate_bwd_tile_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        gate_bwd_tile_kernel<float><<<dim3(ntile, (a.D + BD - 1) / BD), 256, smem, st>>>(static_cast<const float*>(a.x),
-                                                               static_cast<const float*>(a.W), a.eta, a.g, a.deta,
-                                                               a.dg, a.dx, part_w, part_b, a.N, a.D, a.H);
-    }
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    if (a.q != nullptr) {
-        const size_t rows = (size_t)a.N * a.H;
-        e = a.bf16 ? launch_qnorm_bwd(static_cast<const __nv_bfloat16*>(a.q), a.dqhat, a.dq, rows, a.Dk, st)
-                   : launch_qnorm_bwd(static_cast<const float*>(a.q), a.dqhat, a.dq, rows, a.Dk, st);
-        if (e != cudaSuccess) return e;
-    }
-    const size_t total = (size_t)NW * a.D;
-    gate_bwd_reduce_kernel<<<(unsigned)((total + RED_OUT - 1) / RED_OUT), RED_OUT * RED_PARTS, 0, st>>>(
-        part_w, part_b, a.dW, a.db, ntile, NW, a.D);
-    return cudaGetLastError();
+    // dx and the dW / dbias partials, then their fixed-order reduction
+    auto dxw = [&](cudaStream_t s) {
+        cudaError_t e;
+        if (a.bf16) {
+            e = cudaFuncSetAttribute(gate_bwd_tile_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)smem);
+            if (e != cudaSuccess) return e;
+            gate_bwd_tile_kernel<__nv_bfloat16><<<dim3(ntile, (a.D + BD - 1) / BD), 256, smem, s>>>(
+                static_cast<const __nv_bfloat16*>(a.x), static_cast<const __nv_bfloat16*>(a.W), a.eta, a.g, a.deta,
+                a.dg, a.dx, part_w, part_b, a.N, a.D, a.H);
+        } else {
+            e = cudaFuncSetAttribute(gate_bwd_tile_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)smem);
+            if (e != cudaSuccess) return e;
+            gate_bwd_tile_kernel<float><<<dim3(ntile, (a.D + BD - 1) / BD), 256, smem, s>>>(
+                static_cast<const float*>(a.x), static_cast<const float*>(a.W), a.eta, a.g, a.deta, a.dg, a.dx, part_w,
+                part_b, a.N, a.D, a.H);
+        }
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        const size_t total = (size_t)NW * a.D;
+        gate_bwd_reduce_kernel<<<(unsigned)((total + RED_OUT - 1) / RED_OUT), RED_OUT * RED_PARTS, 0, s>>>(
+            part_w, part_b, a.dW, a.db, ntile, NW, a.D);
+        return cudaGetLastError();
+    };
+    if (a.q == nullptr) return dxw(st);
+    const size_t rows = (size_t)a.N * a.H;
+    auto qn = [&](cudaStream_t s) {
+        return a.bf16 ? launch_qnorm_bwd(static_cast<const __nv_bfloat16*>(a.q), a.dqhat, a.dq, rows, a.Dk, s)
+                      : launch_qnorm_bwd(static_cast<const float*>(a.q), a.dqhat, a.dq, rows, a.Dk, s);
+    };
+    return run_beside(st, qn, dxw);
 }
 
 cudaError_t gates_take_error(cudaStream_t st, unsigned int* flag) {
