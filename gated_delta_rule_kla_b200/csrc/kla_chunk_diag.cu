@@ -663,100 +663,114 @@ __global__ void __launch_bounds__(NT, 1) diag_bwd_kernel(BwdArgs a, FwdArgs f, c
             for (int o = 1; o < 16; o <<= 1) da += __shfl_xor_sync(0xffffffffu, da, o);
             if (tx == 0) dbs[i] = da;
         }
-        // ---- Z1 = dO S^T, Z2 = dR S^T, Z3 = U lambda^T for (row i, channels tx + 16 u)
-        float zq[EPT], zr[EPT], zl[EPT];
+        // ---- Z1 = dO S^T, Z2 = dR S^T, Z3 = U lambda^T: warp w takes token rows 2w and 2w + 1,
+        //      lane l channels l + 32 v (a warp reads whole rows: no bank conflicts, and the row
+        //      operands are broadcast)
+        constexpr int NVC = DK / 32;
+        const int rw = 2 * warp;
+        float zq[2][NVC], zr[2][NVC], zl[2][NVC];
 #pragma unroll
-        for (int u = 0; u < EPT; ++u) zq[u] = zr[u] = zl[u] = 0.f;
+        for (int h2 = 0; h2 < 2; ++h2)
+#pragma unroll
+            for (int v = 0; v < NVC; ++v) zq[h2][v] = zr[h2][v] = zl[h2][v] = 0.f;
 #pragma unroll 2
         for (int c = 0; c < 64; c += 4) {
-            const float4 o4 = *reinterpret_cast<const float4*>(dOs + i * BLD + c);
-            const float4 r4 = *reinterpret_cast<const float4*>(dRs + i * BLD + c);
-            const float4 u4 = *reinterpret_cast<const float4*>(Us + i * BLD + c);
+            float4 o4[2], r4[2], u4[2];
 #pragma unroll
-            for (int u = 0; u < EPT; ++u) {
-                const int d = tx + 16 * u;
+            for (int h2 = 0; h2 < 2; ++h2) {
+                o4[h2] = *reinterpret_cast<const float4*>(dOs + (rw + h2) * BLD + c);
+                r4[h2] = *reinterpret_cast<const float4*>(dRs + (rw + h2) * BLD + c);
+                u4[h2] = *reinterpret_cast<const float4*>(Us + (rw + h2) * BLD + c);
+            }
+#pragma unroll
+            for (int v = 0; v < NVC; ++v) {
+                const int d = lane + 32 * v;
                 const float4 s4 = *reinterpret_cast<const float4*>(Ss + d * BLD + c);
                 const float4 l4 = *reinterpret_cast<const float4*>(Ls + d * BLD + c);
-                zq[u] += o4.x * s4.x + o4.y * s4.y + o4.z * s4.z + o4.w * s4.w;
-                zr[u] += r4.x * s4.x + r4.y * s4.y + r4.z * s4.z + r4.w * s4.w;
-                zl[u] += u4.x * l4.x + u4.y * l4.y + u4.z * l4.z + u4.w * l4.w;
+#pragma unroll
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    zq[h2][v] += o4[h2].x * s4.x + o4[h2].y * s4.y + o4[h2].z * s4.z + o4[h2].w * s4.w;
+                    zr[h2][v] += r4[h2].x * s4.x + r4[h2].y * s4.y + r4[h2].z * s4.z + r4[h2].w * s4.w;
+                    zl[h2][v] += u4[h2].x * l4.x + u4[h2].y * l4.y + u4[h2].z * l4.z + u4[h2].w * l4.w;
+                }
             }
         }
         __syncthreads();  // Ym, Dm written; S read: the previous chunk's state may come in
         if (warp == 0 && ci > 0) request_state(ci - 1);
-        // ---- F terms and the per-(token, channel) gradients
-        {
-            float f1[EPT], f2[EPT], f3[EPT], f4[EPT];
+        // ---- F terms and the per-(token, channel) gradients, row by row of the warp's two
 #pragma unroll
-            for (int u = 0; u < EPT; ++u) f1[u] = f2[u] = f3[u] = f4[u] = 0.f;
+        for (int h2 = 0; h2 < 2; ++h2) {
+            const int ii = rw + h2;
+            float f1[NVC], f2[NVC], f3[NVC], f4[NVC];
+#pragma unroll
+            for (int v = 0; v < NVC; ++v) f1[v] = f2[v] = f3[v] = f4[v] = 0.f;
             if (!wide) {
-                for (int j = 0; j <= i; ++j) {
-                    const float y = Ym[i * LDC + j], dd = Dm[i * LDC + j];
+                for (int j = 0; j <= ii; ++j) {
+                    const float y = Ym[ii * LDC + j], dd = Dm[ii * LDC + j];
 #pragma unroll
-                    for (int u = 0; u < EPT; ++u) {
-                        const float kig = KiG[j * DK + tx + 16 * u];
-                        f1[u] = fmaf(y, kig, f1[u]);
-                        f3[u] = fmaf(dd, kig, f3[u]);
+                    for (int v = 0; v < NVC; ++v) {
+                        const float kig = KiG[j * DK + lane + 32 * v];
+                        f1[v] = fmaf(y, kig, f1[v]);
+                        f3[v] = fmaf(dd, kig, f3[v]);
                     }
                 }
-                for (int r = i; r < n; ++r) {
-                    const float y = Ym[r * LDC + i], dd = Dm[r * LDC + i] * bs[r];
+                for (int r = ii; r < n; ++r) {
+                    const float y = Ym[r * LDC + ii], dd = Dm[r * LDC + ii] * bs[r];
 #pragma unroll
-                    for (int u = 0; u < EPT; ++u) {
-                        const int d = tx + 16 * u;
-                        f2[u] = fmaf(y, QGr[r * DK + d], f2[u]);
-                        f4[u] = fmaf(dd, KG[r * DK + d], f4[u]);
+                    for (int v = 0; v < NVC; ++v) {
+                        const int d = lane + 32 * v;
+                        f2[v] = fmaf(y, QGr[r * DK + d], f2[v]);
+                        f4[v] = fmaf(dd, KG[r * DK + d], f4[v]);
                     }
                 }
 #pragma unroll
-                for (int u = 0; u < EPT; ++u) {
-                    const float G = Gs[i * DK + tx + 16 * u];
+                for (int v = 0; v < NVC; ++v) {
+                    const float G = Gs[ii * DK + lane + 32 * v];
                     const float gp = __expf(G), gm = __expf(-G);
-                    f1[u] *= gp;
-                    f3[u] *= gp;
-                    f2[u] *= gm;
-                    f4[u] *= gm;
+                    f1[v] *= gp;
+                    f3[v] *= gp;
+                    f2[v] *= gm;
+                    f4[v] *= gm;
                 }
             } else {
-                for (int j = 0; j <= i; ++j) {
-                    const float y = Ym[i * LDC + j], dd = Dm[i * LDC + j];
+                for (int j = 0; j <= ii; ++j) {
+                    const float y = Ym[ii * LDC + j], dd = Dm[ii * LDC + j];
 #pragma unroll
-                    for (int u = 0; u < EPT; ++u) {
-                        const int d = tx + 16 * u;
-                        const float ke = Kh[j * LDK + d] * __expf(Gs[i * DK + d] - Gs[j * DK + d]);
-                        f1[u] = fmaf(y, ke, f1[u]);
-                        f3[u] = fmaf(dd, ke, f3[u]);
+                    for (int v = 0; v < NVC; ++v) {
+                        const int d = lane + 32 * v;
+                        const float ke = Kh[j * LDK + d] * __expf(Gs[ii * DK + d] - Gs[j * DK + d]);
+                        f1[v] = fmaf(y, ke, f1[v]);
+                        f3[v] = fmaf(dd, ke, f3[v]);
                     }
                 }
-                for (int r = i; r < n; ++r) {
-                    const float y = Ym[r * LDC + i], dd = Dm[r * LDC + i] * bs[r];
+                for (int r = ii; r < n; ++r) {
+                    const float y = Ym[r * LDC + ii], dd = Dm[r * LDC + ii] * bs[r];
 #pragma unroll
-                    for (int u = 0; u < EPT; ++u) {
-                        const int d = tx + 16 * u;
-                        const float e = __expf(Gs[r * DK + d] - Gs[i * DK + d]);
-                        f2[u] = fmaf(y, Qs[r * LDK + d] * e, f2[u]);
-                        f4[u] = fmaf(dd, Kh[r * LDK + d] * e, f4[u]);
+                    for (int v = 0; v < NVC; ++v) {
+                        const int d = lane + 32 * v;
+                        const float e = __expf(Gs[r * DK + d] - Gs[ii * DK + d]);
+                        f2[v] = fmaf(y, Qs[r * LDK + d] * e, f2[v]);
+                        f4[v] = fmaf(dd, Kh[r * LDK + d] * e, f4[v]);
                     }
                 }
             }
-            const float bi = bs[i];
+            const float bi = bs[ii];
             float kgz = 0.f;
 #pragma unroll
-            for (int u = 0; u < EPT; ++u) {
-                const int d = tx + 16 * u;
-                const float G = Gs[i * DK + d], Gl = Gs[(n - 1) * DK + d];
+            for (int v = 0; v < NVC; ++v) {
+                const int d = lane + 32 * v;
+                const float G = Gs[ii * DK + d], Gl = Gs[(n - 1) * DK + d];
                 const float gam = __expf(G), del = __expf(Gl - G);
-                const float qd = Qs[i * LDK + d], kd = Kh[i * LDK + d];
-                Rq[i * DK + d] = fmaf(gam, zq[u], f1[u]);
-                Rk[i * DK + d] = -bi * gam * zr[u] + del * zl[u] + f2[u] + bi * f3[u] + f4[u];
-                Rg[i * DK + d] = gam * qd * zq[u] + qd * f1[u] - bi * gam * kd * zr[u] - kd * f2[u] +
-                                 bi * kd * f3[u] - kd * f4[u] - del * kd * zl[u];
-                Rxs[i * DK + d] = (i < n) ? del * kd * zl[u] : 0.f;
-                kgz = fmaf(kd * gam, zr[u], kgz);
+                const float qd = Qs[ii * LDK + d], kd = Kh[ii * LDK + d];
+                Rq[ii * DK + d] = fmaf(gam, zq[h2][v], f1[v]);
+                Rk[ii * DK + d] = -bi * gam * zr[h2][v] + del * zl[h2][v] + f2[v] + bi * f3[v] + f4[v];
+                Rg[ii * DK + d] = gam * qd * zq[h2][v] + qd * f1[v] - bi * gam * kd * zr[h2][v] - kd * f2[v] +
+                                  bi * kd * f3[v] - kd * f4[v] - del * kd * zl[h2][v];
+                Rxs[ii * DK + d] = (ii < n) ? del * kd * zl[h2][v] : 0.f;
+                kgz = fmaf(kd * gam, zr[h2][v], kgz);
             }
-#pragma unroll
-            for (int o = 1; o < 16; o <<= 1) kgz += __shfl_xor_sync(0xffffffffu, kgz, o);
-            if (tx == 0) dbs[i] -= kgz;
+            kgz = warp_sum(kgz);
+            if (lane == 0) dbs[ii] -= kgz;
         }
         // ---- new lambda = Diag(GC) lambda + QG^T dO - W^T dU (rows i + 16 m, columns cx .. cx + 3);
         //      every other read of lambda was before the last barrier
