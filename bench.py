@@ -349,23 +349,34 @@ def gpu_arm(args, rank, world, local_rank):
 
 def time_fwd_stages(kla, d, w, ws, o, ST, flush, stream, nsteps):
     """Each stage of the split forward timed on its own with CUDA events on the launching
-    stream (L2 flushed before every step): the preparation kernel and the state pass."""
+    stream (L2 flushed before every step): the preparation kernel and the state pass -- with
+    parallel segments, the state pass's transition pass, segment scan and output pass apart."""
     import torch
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(nsteps)]
+    nseg = kla.fwd_state_segments(d["k"], d["v"])
+    parts = [("chunk_state_kernel", 0)] if nseg <= 1 else [
+        ("transition_pass", 1), ("seg_scan_kernel", 2), ("output_pass", 3)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2 + len(parts))] for _ in range(nsteps)]
     for i in range(nsteps):
         flush()
         ev[i][0].record(stream)
         kla.chunk_fwd_prep(d["q"], d["k"], d["v"], d["eta"], d["g"], w.eps, ws)
         ev[i][1].record(stream)
-        kla.chunk_fwd_state(d["q"], d["v"], d["g"], d["S0"], ws, o=o, S_T=ST)
-        ev[i][2].record(stream)
+        for j, (_, stage) in enumerate(parts):
+            kla.chunk_fwd_state(d["q"], d["v"], d["g"], d["S0"], ws, o=o, S_T=ST, stage=stage)
+            ev[i][2 + j].record(stream)
     torch.cuda.synchronize()
-    prep = statistics.median(e[0].elapsed_time(e[1]) for e in ev) * 1e3
-    state = statistics.median(e[1].elapsed_time(e[2]) for e in ev) * 1e3
-    tot = prep + state
-    return {"chunk_prep_kernel": {"us": prep, "share": prep / tot},
-            "chunk_state_kernel": {"us": state, "share": state / tot},
-            "dominant": "chunk_prep_kernel" if prep >= state else "chunk_state_kernel"}
+    us = {"chunk_prep_kernel": statistics.median(e[0].elapsed_time(e[1]) for e in ev) * 1e3}
+    for j, (name, _) in enumerate(parts):
+        us[name] = statistics.median(e[1 + j].elapsed_time(e[2 + j]) for e in ev) * 1e3
+    tot = sum(us.values())
+    out = {k: {"us": v, "share": v / tot} for k, v in us.items()}
+    if nseg > 1:
+        out["segments_per_head"] = nseg
+        out["transition_pass"]["what"] = ("chunk_state_kernel, two runs per segment (from zero and from the "
+                                          "identity), no outputs")
+        out["output_pass"]["what"] = "chunk_state_kernel, one run per segment from its start state, with o"
+    out["dominant"] = max(us, key=us.get)
+    return out
 
 
 def bench_decode(kla, WORKLOADS, make_inputs, dev, stream, flush, rank, world, hbm_peak, args,
@@ -511,7 +522,6 @@ def bench_long(kla, WORKLOADS, make_inputs, dev, stream, rank, world, hbm_peak, 
     # the preparation and the segmented state pass (transition pass, segment scan, output pass)
     # timed on their own
     stages = time_fwd_stages(kla, d, w, ws, o, ST, lambda: None, stream, nsteps)
-    stages["chunk_state_kernel"]["includes"] = "transition pass + seg_scan_kernel + output pass"
     del ws
     # the long-context training step: kla_chunk_fwd_train + kla_chunk_bwd_after_train sharing
     # one workspace (records and tile images: about 5 GB here)

@@ -18,7 +18,8 @@ import os
 
 import torch
 
-__all__ = ["lib", "chunk_fwd", "chunk_fwd_prep", "chunk_fwd_state", "fwd_workspace", "fwd_kernel_launches",
+__all__ = ["lib", "chunk_fwd", "chunk_fwd_prep", "chunk_fwd_state", "fwd_state_segments", "fwd_workspace",
+           "fwd_kernel_launches",
            "chunk_bwd", "chunk_fwd_train", "chunk_bwd_after_train", "train_workspace",
            "decode_step", "check_device_error", "debug_inject_wait_timeout",
            "chunk_fwd_diag", "chunk_bwd_diag", "decode_step_diag", "gate_prologue", "gate_prologue_bwd", "KLAError", "CHUNK", "KLA_BETA_DIRECT",
@@ -65,6 +66,10 @@ def lib():
         L.kla_chunk_fwd_prep.restype = i
         L.kla_chunk_fwd_state.argtypes = [vp, vp, fp, fp, vp, fp, fp, i, i, i, i, i, i, i, i, vp, sz, vp]
         L.kla_chunk_fwd_state.restype = i
+        L.kla_chunk_fwd_state_stage.argtypes = [i, vp, vp, fp, fp, vp, fp, fp, i, i, i, i, i, i, i, i, vp, sz, vp]
+        L.kla_chunk_fwd_state_stage.restype = i
+        L.kla_chunk_fwd_state_segments.argtypes = [i, i, i, i, i, i, i]
+        L.kla_chunk_fwd_state_segments.restype = i
         L.kla_chunk_bwd_workspace.argtypes = [i, i, i, i, i, i, i, i]
         L.kla_chunk_bwd_workspace.restype = sz
         L.kla_chunk_bwd_workspace_min.argtypes = [i, i, i, i, i, i, i, i]
@@ -233,10 +238,11 @@ def chunk_fwd_prep(q, k, v, eta, g, eps, workspace, *, stream=None, beta="kaczma
 
 
 def chunk_fwd_state(q, v, g, S0, workspace, *, o=None, S_T=None, S_chunks=None,
-                    out_dtype=torch.float32, stream=None):
+                    out_dtype=torch.float32, stream=None, stage=0):
     """Second stage of the split forward: the state pass over the records that chunk_fwd_prep
     left in `workspace` (it also reads q and v).  Writes o, S_T, S_chunks when given (allocates o
-    and S_T when None)."""
+    and S_T when None).  `stage` 1, 2, 3 run the transition pass, segment scan and output pass
+    of a segmented state pass alone (see fwd_state_segments); 0 runs all of it."""
     dev = q.device
     B, T, H, Dk = q.shape
     Dv = v.shape[-1]
@@ -250,11 +256,18 @@ def chunk_fwd_state(q, v, g, S0, workspace, *, o=None, S_T=None, S_chunks=None,
     _need(S_chunks, "S_chunks", dev, torch.float32, (B, H, (T + CHUNK - 1) // CHUNK, Dk, Dv))
     _need(workspace, "workspace", dev, torch.uint8)
     L = lib()
-    st = L.kla_chunk_fwd_state(_ptr(q), _ptr(v), _ptr(g), _ptr(S0), _ptr(o), _ptr(S_T), _ptr(S_chunks), B, T, H, Dk, Dv,
-                               CHUNK, _dtype_code(q), _dtype_code(o), _ptr(workspace), workspace.numel(),
-                               _stream(dev, stream))
+    st = L.kla_chunk_fwd_state_stage(int(stage), _ptr(q), _ptr(v), _ptr(g), _ptr(S0), _ptr(o), _ptr(S_T),
+                                     _ptr(S_chunks), B, T, H, Dk, Dv, CHUNK, _dtype_code(q), _dtype_code(o),
+                                     _ptr(workspace), workspace.numel(), _stream(dev, stream))
     _check(st, "kla_chunk_fwd_state")
     return o, S_T
+
+
+def fwd_state_segments(k, v):
+    """Parallel segments per head of the split forward's state pass for k, v (1: one run per
+    head; 0: shapes the split path does not take)."""
+    B, T, H, Dk = k.shape
+    return lib().kla_chunk_fwd_state_segments(B, T, H, Dk, v.shape[-1], CHUNK, _dtype_code(k))
 
 
 def chunk_bwd(q, k, v, eta, g, dO, eps=1e-6, S0=None, dS_T=None, S_chunks=None, *, stream=None,

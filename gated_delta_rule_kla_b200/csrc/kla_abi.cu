@@ -249,10 +249,11 @@ kla_status kla_chunk_fwd_prep(const void* q, const void* k, const void* v, const
     return KLA_OK;
 }
 
-kla_status kla_chunk_fwd_state(const void* q, const void* v, const float* g, const float* S0, void* o,
-                               float* S_T, float* S_chunks, int B, int T, int H, int Dk, int Dv, int chunk,
-                               int dtype, int out_dtype, void* ws, size_t ws_bytes, void* stream) {
+kla_status kla_chunk_fwd_state_stage(int stage, const void* q, const void* v, const float* g, const float* S0,
+                                     void* o, float* S_T, float* S_chunks, int B, int T, int H, int Dk, int Dv,
+                                     int chunk, int dtype, int out_dtype, void* ws, size_t ws_bytes, void* stream) {
     take_beta_flag(dtype);  // the state pass reads the preparation's coefficients
+    if (stage < 0 || stage > 3) return fail(KLA_ERR_INVALID_ARG, "stage must be 0, 1, 2 or 3 (got %d)", stage);
     kla::FwdArgs a{};
     kla_status st = split_stage_checks(B, T, H, Dk, Dv, chunk, dtype, out_dtype, 0.f, ws, ws_bytes,
                                        "kla_chunk_fwd_state", &a);
@@ -260,9 +261,24 @@ kla_status kla_chunk_fwd_state(const void* q, const void* v, const float* g, con
     REQUIRE_PTR(q); REQUIRE_PTR(v); REQUIRE_PTR(g);
     OPTIONAL_PTR(S0); OPTIONAL_PTR(o); OPTIONAL_PTR(S_T); OPTIONAL_PTR(S_chunks);
     a.q = q; a.v = v; a.g = g; a.S0 = S0; a.o = o; a.S_T = S_T; a.S_chunks = S_chunks;
-    cudaError_t e = kla::launch_chunk_fwd_split_state(a, ws, static_cast<cudaStream_t>(stream));
+    cudaError_t e = kla::launch_chunk_fwd_split_state(a, ws, static_cast<cudaStream_t>(stream), stage);
     if (e != cudaSuccess) return cuda_fail(e, "kla_chunk_fwd_state launch");
     return KLA_OK;
+}
+
+kla_status kla_chunk_fwd_state(const void* q, const void* v, const float* g, const float* S0, void* o,
+                               float* S_T, float* S_chunks, int B, int T, int H, int Dk, int Dv, int chunk,
+                               int dtype, int out_dtype, void* ws, size_t ws_bytes, void* stream) {
+    return kla_chunk_fwd_state_stage(0, q, v, g, S0, o, S_T, S_chunks, B, T, H, Dk, Dv, chunk, dtype, out_dtype, ws,
+                                     ws_bytes, stream);
+}
+
+int kla_chunk_fwd_state_segments(int B, int T, int H, int Dk, int Dv, int chunk, int dtype) {
+    take_beta_flag(dtype);
+    kla::FwdArgs a{};
+    if (B < 1 || H < 1 || T < 1 || chunk != kla::kChunkLen || dtype != KLA_BF16 || Dk != 128 || Dv != 128) return 0;
+    a.B = B; a.T = T; a.H = H; a.Dk = Dk; a.Dv = Dv; a.bf16 = true;
+    return kla::chunk_fwd_split_segments(a);
 }
 
 size_t kla_chunk_bwd_workspace_min(int B, int T, int H, int Dk, int Dv, int chunk, int dtype,

@@ -65,11 +65,12 @@ constexpr uint32_t PM_G = 0, PM_W = 0;  // TMEM columns (64 allocated); W reuses
 struct PrepMisc {
     uint64_t full, mma;
     uint32_t tmem_base, pad[3];
-    float G[CH], gam[CH], del[CH], bco[CH], cco[CH], invr[CH], graw[CH], eta[CH], pk[CH];
+    float G[CH], gam[CH], del[CH], bco[CH], cco[CH], invr[CH], eta[CH], pk[CH];
     float wsc[CH];  // b gamma / r: column scale of T'
-    float gsum[2], gprev[2], grange;
+    float gsum[4], grange;  // the next chunk's g sums (two halves), then the previous chunk's
 };
 static_assert(sizeof(PrepMisc) <= 3072, "prep scalars");
+static_assert(offsetof(PrepMisc, G) % 8 == 0, "float2 access to the per-token scalars");
 
 __global__ void __launch_bounds__(PT, 4)
     chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -91,19 +92,24 @@ __global__ void __launch_bounds__(PT, 4)
     const uint32_t sbase = smem_u32(sm);
     const uint32_t bar_full = smem_u32(&ms->full), bar_mma = smem_u32(&ms->mma);
 
-    // per-token gates first: their latency overlaps the barrier set-up and the tile loads
-    float g_own = 0.f, eta_own = 0.f, g_next = 0.f, g_prev = 0.f;
-    if (tid < CH) {
-        if (tid < n) {
-            const size_t ti = tok_index(b, t0 + tid, h, T, H);
-            g_own = a.g[ti];
-            eta_own = a.eta[ti];
-        }
+    // Per-token gates first: their latency, and the in-chunk scan of g and its decays (warp 0),
+    // overlap the barrier set-up and the tile loads.  Warp 0 lane l: tokens 2l, 2l + 1 (g zero
+    // past the sequence, so G stays flat there); warp 1: eta; warps 2-3 / 4-5: the next /
+    // previous chunk's g for its gamma_last.
+    float g0 = 0.f, g1 = 0.f, gx = 0.f;
+    if (warp == 0) {
+        const int l = tid;
+        if (2 * l < n) g0 = a.g[tok_index(b, t0 + 2 * l, h, T, H)];
+        if (2 * l + 1 < n) g1 = a.g[tok_index(b, t0 + 2 * l + 1, h, T, H)];
+    } else if (warp == 1) {
+        const int l = tid - 32;
+        if (2 * l < n) g0 = a.eta[tok_index(b, t0 + 2 * l, h, T, H)];
+        if (2 * l + 1 < n) g1 = a.eta[tok_index(b, t0 + 2 * l + 1, h, T, H)];
     } else if (tid < 2 * CH) {
         const int j = tid - CH;
-        if (c + 1 < NC && (c + 1) * CH + j < T) g_next = a.g[tok_index(b, (c + 1) * CH + j, h, T, H)];
+        if (c + 1 < NC && (c + 1) * CH + j < T) gx = a.g[tok_index(b, (c + 1) * CH + j, h, T, H)];
     } else if (tid < 3 * CH) {  // the previous chunk (always full) for the reverse pass
-        if (c > 0) g_prev = a.g[tok_index(b, (c - 1) * CH + tid - 2 * CH, h, T, H)];
+        if (c > 0) gx = a.g[tok_index(b, (c - 1) * CH + tid - 2 * CH, h, T, H)];
     }
     if (tid == 0) {
         mbar_init(bar_full, 1);
@@ -118,16 +124,31 @@ __global__ void __launch_bounds__(PT, 4)
     if (warp == 0) {
         tmem_alloc(smem_u32(&ms->tmem_base), 64);
         tmem_relinquish();
-    }
-    if (tid < CH) {
-        ms->graw[tid] = g_own;
-        ms->eta[tid] = eta_own;
-    } else if (tid < 2 * CH) {  // the next chunk's gamma_last
-        const float sg = warp_sum(g_next);
+        // inclusive prefix sum G of g inside the chunk, gamma = e^G, delta = e^{G_last - G}
+        const int l = tid;
+        float sc = g0 + g1;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const float y = __shfl_up_sync(0xffffffffu, sc, o);
+            if (l >= o) sc += y;
+        }
+        const float excl = sc - (g0 + g1);
+        const float G0 = excl + g0, G1 = excl + g0 + g1;
+        const float Glast = __shfl_sync(0xffffffffu, G1, 31);
+        float gr = fmaxf(fabsf(G0), fabsf(G1));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) gr = fmaxf(gr, __shfl_xor_sync(0xffffffffu, gr, o));
+        const float gm0 = __expf(G0), gm1 = __expf(G1);
+        reinterpret_cast<float2*>(ms->G)[l] = make_float2(G0, G1);
+        reinterpret_cast<float2*>(ms->gam)[l] = make_float2(gm0, gm1);
+        reinterpret_cast<float2*>(ms->del)[l] = make_float2(__expf(Glast - G0), __expf(Glast - G1));
+        reinterpret_cast<float2*>(rec + REC_SC)[l] = make_float2(gm0, gm1);
+        if (l == 0) ms->grange = gr;
+    } else if (warp == 1) {
+        reinterpret_cast<float2*>(ms->eta)[tid - 32] = make_float2(g0, g1);
+    } else if (tid < 3 * CH) {  // the next (warps 2-3) and previous (warps 4-5) chunks' gamma_last
+        const float sg = warp_sum(gx);
         if ((tid & 31) == 0) ms->gsum[warp - 2] = sg;
-    } else if (tid < 3 * CH) {  // the previous chunk's gamma_last
-        const float sg = warp_sum(g_prev);
-        if ((tid & 31) == 0) ms->gprev[warp - 4] = sg;
     }
     tc_fence_before();
     __syncthreads();
@@ -154,69 +175,42 @@ __global__ void __launch_bounds__(PT, 4)
         }
         mma_commit(bar_mma);
     }
-    // key norms and Kaczmarz coefficients: four threads per key row j = tid / 4, thread q of the
-    // four summing 32 features (dk block q / 2, logical 16-byte chunks 4 (q & 1) .. + 3 of it, in
-    // an order rotated by q / 2 so that the eight lanes of a quarter warp -- rows j and j + 1,
-    // whose swizzle phases differ in parity -- hit eight different bank groups)
-    {
-        const int j = tid >> 2, q = tid & 3;
-        const uint8_t* krow = qk + (q >> 1) * 16384 + 8192 + j * 128;
-        float ra = 0.f, rb = 0.f;
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {
-            const int cc = 4 * (q & 1) + ((m + 2 * (q >> 1)) & 3);
-            float f[8];
-            unpack_bf16x8(*reinterpret_cast<const uint4*>(krow + ((cc ^ (j & 7)) << 4)), f);
-#pragma unroll
-            for (int e = 0; e < 8; e += 2) {
-                ra = fmaf(f[e], f[e], ra);
-                rb = fmaf(f[e + 1], f[e + 1], rb);
-            }
-        }
-        float r2 = ra + rb;
-        r2 += __shfl_xor_sync(0xffffffffu, r2, 1);
-        r2 += __shfl_xor_sync(0xffffffffu, r2, 2);
-        if (q == 0) {
-            const KaczCoef cf = kacz_coef(ms->eta[j], r2, a.eps);
-            ms->bco[j] = cf.b;
-            ms->cco[j] = cf.c;
-            ms->invr[j] = cf.inv_r;
-        }
-    }
-    if (warp == 0) {  // inclusive prefix sum of g inside the chunk (2 tokens per lane)
-        const int l = tid;
-        const float x0 = ms->graw[2 * l], x1 = ms->graw[2 * l + 1];
-        float s = x0 + x1;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const float y = __shfl_up_sync(0xffffffffu, s, o);
-            if (l >= o) s += y;
-        }
-        const float excl = s - (x0 + x1);
-        const float G0 = excl + x0, G1 = excl + x0 + x1;
-        ms->G[2 * l] = G0;
-        ms->G[2 * l + 1] = G1;
-        float gr = fmaxf(fabsf(G0), fabsf(G1));
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) gr = fmaxf(gr, __shfl_xor_sync(0xffffffffu, gr, o));
-        if (l == 0) ms->grange = gr;
-    }
-    __syncthreads();
     {
         // e^{G_i - G_j} = gamma_i * e^{-G_j} while every |G_j| < 80; otherwise the exact exp of
         // the difference.  Uniform over the CTA.
         const bool factored = ms->grange < 80.f;
-        if (tid < CH) {
-            const float gm = __expf(ms->G[tid]);
-            ms->gam[tid] = gm;
-            reinterpret_cast<float*>(rec + REC_SC)[tid] = gm;
-            ms->del[tid] = __expf(ms->G[CH - 1] - ms->G[tid]);  // G is flat past the last token
-            ms->pk[tid] = factored ? __expf(-ms->G[tid]) * ms->invr[tid] : 0.f;
-            ms->wsc[tid] = ms->bco[tid] * gm * ms->invr[tid];
-        } else if (tid == CH) {
-            reinterpret_cast<float*>(rec + REC_SC)[CH] = __expf(ms->gsum[0] + ms->gsum[1]);
-        } else if (tid == CH + 1) {
-            reinterpret_cast<float*>(rec + REC_SC)[CH + 1] = __expf(ms->gprev[0] + ms->gprev[1]);
+        // key norms and Kaczmarz coefficients: four threads per key row j = tid / 4, thread q of
+        // the four summing 32 features (dk block q / 2, logical 16-byte chunks 4 (q & 1) .. + 3 of
+        // it, in an order rotated by q / 2 so that the eight lanes of a quarter warp -- rows j and
+        // j + 1, whose swizzle phases differ in parity -- hit eight different bank groups)
+        {
+            const int j = tid >> 2, q = tid & 3;
+            const uint8_t* krow = qk + (q >> 1) * 16384 + 8192 + j * 128;
+            float ra = 0.f, rb = 0.f;
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const int cc = 4 * (q & 1) + ((m + 2 * (q >> 1)) & 3);
+                float f[8];
+                unpack_bf16x8(*reinterpret_cast<const uint4*>(krow + ((cc ^ (j & 7)) << 4)), f);
+#pragma unroll
+                for (int e = 0; e < 8; e += 2) {
+                    ra = fmaf(f[e], f[e], ra);
+                    rb = fmaf(f[e + 1], f[e + 1], rb);
+                }
+            }
+            float r2 = ra + rb;
+            r2 += __shfl_xor_sync(0xffffffffu, r2, 1);
+            r2 += __shfl_xor_sync(0xffffffffu, r2, 2);
+            if (q == 0) {
+                const KaczCoef cf = kacz_coef(ms->eta[j], r2, a.eps);
+                ms->bco[j] = cf.b;
+                ms->cco[j] = cf.c;
+                ms->invr[j] = cf.inv_r;
+                ms->pk[j] = factored ? __expf(-ms->G[j]) * cf.inv_r : 0.f;
+                ms->wsc[j] = cf.b * ms->gam[j] * cf.inv_r;
+            } else if (q == 1 && j < 2) {  // the next / previous chunk's gamma_last
+                reinterpret_cast<float*>(rec + REC_SC)[CH + j] = __expf(ms->gsum[2 * j] + ms->gsum[2 * j + 1]);
+            }
         }
         ok = mbar_wait_bounded(bar_mma, 0, kWaitNs);
         if (__syncthreads_or(!ok)) {
@@ -1468,7 +1462,7 @@ cudaError_t launch_chunk_fwd_split_prep(const FwdArgs& a, void* ws, cudaStream_t
     return launch_prep_range(a, ws, 0, (a.T + CH - 1) / CH, st);
 }
 
-cudaError_t launch_chunk_fwd_split_state(const FwdArgs& a, void* ws, cudaStream_t st) {
+cudaError_t launch_chunk_fwd_split_state(const FwdArgs& a, void* ws, cudaStream_t st, int stage) {
     CUtensorMap mq;
     if (!make_map(&mq, a.q, a.B, a.T, a.H)) return cudaErrorInvalidValue;
     const SplitLayout L = split_layout(a);
@@ -1479,7 +1473,8 @@ cudaError_t launch_chunk_fwd_split_state(const FwdArgs& a, void* ws, cudaStream_
         return f.out_bf16 ? launch_state<__nv_bfloat16>(mq, f, recs, grid, st)
                           : launch_state<float>(mq, f, recs, grid, st);
     };
-    if (L.nseg <= 1) {
+    if (L.nseg <= 1) {  // one run: it is the output pass (stages 1 and 2 have nothing to do)
+        if (stage == 1 || stage == 2) return cudaSuccess;
         FwdArgs f = a;
         f.nseg = 1;
         f.seg_chunks = NC;
@@ -1501,9 +1496,11 @@ cudaError_t launch_chunk_fwd_split_state(const FwdArgs& a, void* ws, cudaStream_
     p1.seg_chunks = L.segc;
     p1.kinds = 2;
     p1.chunk0 = 0;
-    cudaError_t e = state(p1, dim3(BH * L.nseg, 2));
+    cudaError_t e = cudaSuccess;
+    if (stage == 0 || stage == 1) e = state(p1, dim3(BH * L.nseg, 2));
     if (e != cudaSuccess) return e;
-    if ((e = launch_seg_scan(a.S0, MN, Sstart, a.S_T, BH, L.nseg, st)) != cudaSuccess) return e;
+    if (stage == 0 || stage == 2) e = launch_seg_scan(a.S0, MN, Sstart, a.S_T, BH, L.nseg, st);
+    if (e != cudaSuccess || stage == 1 || stage == 2) return e;
     FwdArgs p2 = a;
     p2.S0 = Sstart;
     p2.S_T = nullptr;
@@ -1568,6 +1565,8 @@ int chunk_fwd_split_launches(const FwdArgs& a) {
     const SplitLayout L = split_layout(a);
     return L.nseg > 1 ? 4 : (L.nc1 > 0 ? 4 : 2);
 }
+
+int chunk_fwd_split_segments(const FwdArgs& a) { return split_layout(a).nseg; }
 
 int reverse_nseg(int BH, int NC) { return choose_nseg_split(BH, NC); }
 

@@ -615,50 +615,80 @@ cudaError_t launch_chunk_fwd_tc(const FwdArgs& a, cudaStream_t st) {
 // ------------------------------------------------------------------------------------
 namespace {
 
-constexpr int SCAN_LD = 129;  // padded row of M in shared memory
+constexpr int SCAN_LD = 132;  // padded row of M in shared memory (16-byte rows: vector reads)
 
 // One CTA per (head, 16-column slice of the state): the columns of S evolve independently,
-// S_{s+1}[:, cols] = M_s S_s[:, cols] + N_s[:, cols].
+// S_{s+1}[:, cols] = M_s S_s[:, cols] + N_s[:, cols].  M_{s+1} streams into the second of two
+// shared-memory buffers (per-thread async copies) and N_{s+1} into registers while step s runs,
+// so the chain pays no load latency.  Thread: column tx, rows ty + 16 i (i < 8); the sum over
+// k runs in order (k = 0 .. 127), one fma per term.
 constexpr int SCAN_W = 16;  // state columns per CTA
+constexpr size_t SCAN_SMEM = sizeof(float) * (2 * DK * SCAN_LD + DK * SCAN_W);
 
 __global__ void __launch_bounds__(256) seg_scan_kernel(const float* __restrict__ S0, const float* __restrict__ MN,
                                                        float* __restrict__ Sstart, float* __restrict__ S_T, int BH,
                                                        int nseg) {
-    extern __shared__ float scan_sm[];
-    float* Ms = scan_sm;                 // 128 x SCAN_LD transition of the segment
-    float* Ss = Ms + DK * SCAN_LD;       // 128 x SCAN_W current state columns
+    extern __shared__ __align__(16) float scan_sm[];
+    float* Mbuf = scan_sm;                   // two 128 x SCAN_LD transitions
+    float* Ss = scan_sm + 2 * DK * SCAN_LD;  // 128 x SCAN_W current state columns
     const int head = blockIdx.x, c0 = blockIdx.y * SCAN_W, tid = threadIdx.x;
     const int tx = tid & (SCAN_W - 1), ty = tid >> 4;  // column, row group (rows ty + 16 i)
     const size_t SZ = (size_t)DK * DV;
+    auto fetch_M = [&](int sgm) {  // M_sgm (kind 1) into buffer sgm & 1: 16 copies per thread
+        const float* M = MN + ((size_t)BH + head) * nseg * SZ + (size_t)sgm * SZ;
+        const uint32_t dst = smem_u32(Mbuf + (sgm & 1) * DK * SCAN_LD);
+        for (int x = tid; x < DK * DV / 4; x += 256) {
+            const int r = (4 * x) / DV, cc = (4 * x) % DV;
+            cp_async16(dst + 4 * (uint32_t)(r * SCAN_LD + cc), M + 4 * (size_t)x);
+        }
+        cp_async_commit();
+    };
+    auto N_of = [&](int sgm) { return MN + (size_t)head * nseg * SZ + (size_t)sgm * SZ; };  // kind 0
+    fetch_M(0);
     for (int x = tid; x < DK * SCAN_W; x += 256) {
         const int r = x / SCAN_W, c = x % SCAN_W;
         Ss[x] = S0 ? S0[head * SZ + (size_t)r * DV + c0 + c] : 0.f;
     }
+    float nxt[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) nxt[i] = N_of(0)[(size_t)(ty + 16 * i) * DV + c0 + tx];
     for (int sgm = 0; sgm < nseg; ++sgm) {
-        const float* M = MN + ((size_t)BH + head) * nseg * SZ + (size_t)sgm * SZ;   // kind 1
-        const float* N = MN + (size_t)head * nseg * SZ + (size_t)sgm * SZ;          // kind 0
-        float* out = Sstart + ((size_t)head * nseg + sgm) * SZ;
-        for (int x = tid; x < DK * DV / 4; x += 256) {
-            const float4 m4 = reinterpret_cast<const float4*>(M)[x];
-            float* dst = Ms + (4 * x / DV) * SCAN_LD + (4 * x) % DV;
-            dst[0] = m4.x; dst[1] = m4.y; dst[2] = m4.z; dst[3] = m4.w;
+        if (sgm + 1 < nseg) {
+            fetch_M(sgm + 1);  // its buffer's last reader was step sgm - 1, behind the barrier below
+        } else {
+            cp_async_commit();  // an empty group keeps the wait below uniform
         }
-        __syncthreads();  // M and the current columns are in place
-        for (int x = tid; x < DK * SCAN_W; x += 256) out[(size_t)(x / SCAN_W) * DV + c0 + x % SCAN_W] = Ss[x];
         float acc[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) acc[i] = N[(size_t)(ty + 16 * i) * DV + c0 + tx];
-#pragma unroll 4
-        for (int kk = 0; kk < DK; ++kk) {
-            const float b = Ss[kk * SCAN_W + tx];
+        for (int i = 0; i < 8; ++i) acc[i] = nxt[i];
+        if (sgm + 1 < nseg) {
 #pragma unroll
-            for (int i = 0; i < 8; ++i) acc[i] = fmaf(Ms[(ty + 16 * i) * SCAN_LD + kk], b, acc[i]);
+            for (int i = 0; i < 8; ++i) nxt[i] = N_of(sgm + 1)[(size_t)(ty + 16 * i) * DV + c0 + tx];
         }
-        __syncthreads();  // every read of S and M is done
+        cp_async_wait<1>();  // this thread's copies of M_sgm have landed
+        __syncthreads();     // ... and every thread's; the current columns are in place
+        float* out = Sstart + ((size_t)head * nseg + sgm) * SZ;
+        for (int x = tid; x < DK * SCAN_W; x += 256) out[(size_t)(x / SCAN_W) * DV + c0 + x % SCAN_W] = Ss[x];
+        const float* Ms = Mbuf + (sgm & 1) * DK * SCAN_LD;
+#pragma unroll 2
+        for (int kk = 0; kk < DK; kk += 4) {
+            float bk[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) bk[u] = Ss[(kk + u) * SCAN_W + tx];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float4 m = *reinterpret_cast<const float4*>(Ms + (ty + 16 * i) * SCAN_LD + kk);
+                acc[i] = fmaf(m.x, bk[0], acc[i]);
+                acc[i] = fmaf(m.y, bk[1], acc[i]);
+                acc[i] = fmaf(m.z, bk[2], acc[i]);
+                acc[i] = fmaf(m.w, bk[3], acc[i]);
+            }
+        }
+        __syncthreads();  // every read of S and of this M buffer is done
 #pragma unroll
         for (int i = 0; i < 8; ++i) Ss[(ty + 16 * i) * SCAN_W + tx] = acc[i];
-        __syncthreads();
     }
+    __syncthreads();
     if (S_T)
         for (int x = tid; x < DK * SCAN_W; x += 256)
             S_T[head * SZ + (size_t)(x / SCAN_W) * DV + c0 + x % SCAN_W] = Ss[x];
@@ -668,10 +698,10 @@ __global__ void __launch_bounds__(256) seg_scan_kernel(const float* __restrict__
 
 cudaError_t launch_seg_scan(const float* S0, const float* MN, float* Sstart, float* S_T, int BH, int nseg,
                             cudaStream_t st) {
-    const size_t scan_smem = sizeof(float) * (DK * SCAN_LD + DK * SCAN_W);
-    cudaError_t e = cudaFuncSetAttribute(seg_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)scan_smem);
+    if (nseg < 1) return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(seg_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SCAN_SMEM);
     if (e != cudaSuccess) return e;
-    seg_scan_kernel<<<dim3(BH, DV / SCAN_W), 256, scan_smem, st>>>(S0, MN, Sstart, S_T, BH, nseg);
+    seg_scan_kernel<<<dim3(BH, DV / SCAN_W), 256, SCAN_SMEM, st>>>(S0, MN, Sstart, S_T, BH, nseg);
     return cudaGetLastError();
 }
 

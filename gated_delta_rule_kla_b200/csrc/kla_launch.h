@@ -159,9 +159,13 @@ cudaError_t launch_chunk_fwd_split(const FwdArgs& a, void* ws, cudaStream_t st);
 // Kernels one launch_chunk_fwd_split call launches (preparation and state passes).
 int chunk_fwd_split_launches(const FwdArgs& a);
 // The two stages of the split path: the chunk-parallel preparation (writes the per-chunk
-// records into ws) and the state pass that reads them.
+// records into ws) and the state pass that reads them.  stage 0 runs the whole state pass;
+// with parallel segments 1, 2 and 3 run its transition pass, segment scan and output pass
+// alone (in that order they equal stage 0); with one run per head 3 runs it and 1, 2 do nothing.
 cudaError_t launch_chunk_fwd_split_prep(const FwdArgs& a, void* ws, cudaStream_t st);
-cudaError_t launch_chunk_fwd_split_state(const FwdArgs& a, void* ws, cudaStream_t st);
+cudaError_t launch_chunk_fwd_split_state(const FwdArgs& a, void* ws, cudaStream_t st, int stage = 0);
+// Parallel segments of the split path's state pass per head (1: one run per head).
+int chunk_fwd_split_segments(const FwdArgs& a);
 cudaError_t split_take_error(cudaStream_t st, unsigned int* flag);
 // Segments of the backward's reverse state pass for BH heads of NC chunks (1: one run per head);
 // the forward state pass's cost model, which the reverse pass shares.

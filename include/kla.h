@@ -140,6 +140,29 @@ kla_status kla_chunk_fwd_state(const void *q, const void *v, const float *g, con
                                void *o, float *S_T, float *S_chunks, int B, int T, int H, int Dk,
                                int Dv, int chunk, int dtype, int out_dtype, void *ws,
                                size_t ws_bytes, void *stream);
+/*
+ * kla_chunk_fwd_state_segments -- how the state pass of the split path runs for these shapes:
+ * 1 = one run per head over all its chunks (as one or two slabs inside kla_chunk_fwd), n > 1 =
+ * n parallel segments per head chained by a scan ("Kaczmarz Linear Attention", section 4: the
+ * chunk-to-chunk state map S -> gamma_last S + Ktil^T (U' - W S) is affine in S, so a segment's
+ * map is found from two runs, one from zero and one from the identity, and the segments' start
+ * states follow by composing the maps in order).  0 for shapes the split path does not take.
+ *
+ * kla_chunk_fwd_state_stage -- one part of kla_chunk_fwd_state, for timing or scheduling them
+ * apart.  stage 0 is the whole state pass (= kla_chunk_fwd_state).  With segments (above > 1):
+ * 1 the transition pass (both runs of every segment, into ws), 2 the segment scan (start
+ * states, and S_T, into ws), 3 the output pass (o and S_chunks from every segment's start
+ * state); run 1, 2, 3 in order on one stream, with the same arguments, they equal stage 0 bit
+ * for bit.  With one run per head stage 3 is the whole pass and 1, 2 launch nothing.
+ *   Other arguments, requirements and ownership as for kla_chunk_fwd_state.
+ * Returns KLA_OK, KLA_ERR_INVALID_ARG for a stage outside 0..3, or the errors of
+ * kla_chunk_fwd_state; on error nothing is launched.
+ */
+int kla_chunk_fwd_state_segments(int B, int T, int H, int Dk, int Dv, int chunk, int dtype);
+kla_status kla_chunk_fwd_state_stage(int stage, const void *q, const void *v, const float *g,
+                                     const float *S0, void *o, float *S_T, float *S_chunks,
+                                     int B, int T, int H, int Dk, int Dv, int chunk, int dtype,
+                                     int out_dtype, void *ws, size_t ws_bytes, void *stream);
 
 /*
  * kla_chunk_bwd -- gradients of the chunkwise forward.

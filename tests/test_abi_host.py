@@ -74,6 +74,20 @@ def test_fwd_stages_reject_before_launch(L):
     assert state(q=None) == INVALID and state(v=None) == INVALID and state(ws=MISALIGNED) == INVALID
     assert b"aligned" in L.kla_last_error()
     assert state(ws=None) == WORKSPACE and b"kla_chunk_fwd_state" in L.kla_last_error()
+    stage = lambda k: L.kla_chunk_fwd_state_stage(k, FAKE, FAKE, FAKE, None, FAKE, None, None, 2, 300, 3, 128, 128,
+                                                  64, 1, 0, FAKE, need, None)
+    assert stage(-1) == INVALID and stage(4) == INVALID and b"stage" in L.kla_last_error()
+
+
+def test_fwd_state_segments_query(L):
+    # many heads or short sequences: one run per head; few heads over a long sequence: parallel
+    # segments (with the 148 SMs assumed when no device answers)
+    assert L.kla_chunk_fwd_state_segments(8, 2048, 8, 128, 128, 64, 1) == 1
+    assert L.kla_chunk_fwd_state_segments(1, 65536, 16, 128, 128, 64, 1) > 1
+    assert L.kla_chunk_fwd_state_segments(1, 4100, 1, 128, 128, 64, 1) > 1
+    assert L.kla_chunk_fwd_state_segments(8, 2048, 8, 64, 128, 64, 1) == 0
+    assert L.kla_chunk_fwd_state_segments(8, 2048, 8, 128, 128, 64, 0) == 0
+    assert L.kla_chunk_fwd_state_segments(0, 2048, 8, 128, 128, 64, 1) == 0
 
 
 def test_bwd_workspace_checked(L):

@@ -193,6 +193,21 @@ def test_fwd_prep_and_state_stages_equal_one_call(kla, B, T, H, launches):
     torch.cuda.synchronize()
     kla.check_device_error()
     assert torch.equal(o, o2) and torch.equal(ST, ST2) and torch.equal(Sc, Sc2)
+    # the state pass's parts one by one (transition pass, segment scan, output pass)
+    nseg = kla.fwd_state_segments(d["k"], d["v"])
+    assert (nseg > 1) == (launches == 4 and B * H < 16)
+    ws3 = kla.fwd_workspace(d["k"], d["v"])
+    o3, ST3, Sc3 = torch.zeros_like(o), torch.zeros_like(ST), torch.zeros_like(Sc)
+    kla.chunk_fwd_prep(d["q"], d["k"], d["v"], d["eta"], d["g"], 1e-6, ws3)
+    for stage in (1, 2):
+        kla.chunk_fwd_state(d["q"], d["v"], d["g"], d["S0"], ws3, o=o3, S_T=ST3, S_chunks=Sc3, stage=stage)
+    torch.cuda.synchronize()
+    if nseg == 1:  # nothing launched yet
+        assert not o3.any() and not ST3.any() and not Sc3.any()
+    kla.chunk_fwd_state(d["q"], d["v"], d["g"], d["S0"], ws3, o=o3, S_T=ST3, S_chunks=Sc3, stage=3)
+    torch.cuda.synchronize()
+    kla.check_device_error()
+    assert torch.equal(o, o3) and torch.equal(ST, ST3) and torch.equal(Sc, Sc3)
 
 
 def test_fwd_split_more_heads_than_sms(kla, oracle_mod):
