@@ -298,15 +298,19 @@ __device__ __forceinline__ void st_pair_sw128_global(uint8_t* block, int r, int 
                  : "memory");
 }
 
-// bf16 hi/lo words of 8 fp32 values (one 16-byte chunk of each of the two blocks).
+// bf16 hi/lo words of 8 fp32 values (one 16-byte chunk of each of the two blocks): per pair,
+// the hi word is one paired rounding, the hi values are read back from its halves, and the
+// remainders are rounded as a pair (hi = rn(x), lo = rn(x - hi), as split_bf16).
+__device__ __forceinline__ uint32_t split_word2(float a, float b, uint32_t& lo) {
+    const uint32_t hw = pack_bf16x2(a, b);
+    lo = pack_bf16x2(a - __uint_as_float(hw << 16), b - __uint_as_float(hw & 0xffff0000u));
+    return hw;
+}
 __device__ __forceinline__ void split_chunk8(const float* v, uint4& uh, uint4& ul) {
-    float h[8], l[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) split_bf16(v[e], h[e], l[e]);
-    uh.x = pack_bf16x2(h[0], h[1]); uh.y = pack_bf16x2(h[2], h[3]);
-    uh.z = pack_bf16x2(h[4], h[5]); uh.w = pack_bf16x2(h[6], h[7]);
-    ul.x = pack_bf16x2(l[0], l[1]); ul.y = pack_bf16x2(l[2], l[3]);
-    ul.z = pack_bf16x2(l[4], l[5]); ul.w = pack_bf16x2(l[6], l[7]);
+    uh.x = split_word2(v[0], v[1], ul.x);
+    uh.y = split_word2(v[2], v[3], ul.y);
+    uh.z = split_word2(v[4], v[5], ul.z);
+    uh.w = split_word2(v[6], v[7], ul.w);
 }
 
 // Global versions of st_chunks_split / st_chunks_bf16 for an even count of chunks starting
@@ -396,14 +400,8 @@ __device__ __forceinline__ void st_chunks_split(uint8_t* hi_block, uint8_t* lo_b
                                                 const float* v) {
 #pragma unroll
     for (int c = 0; c < n; ++c) {
-        float h[8], l[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) split_bf16(v[8 * c + e], h[e], l[e]);
         uint4 uh, ul;
-        uh.x = pack_bf16x2(h[0], h[1]); uh.y = pack_bf16x2(h[2], h[3]);
-        uh.z = pack_bf16x2(h[4], h[5]); uh.w = pack_bf16x2(h[6], h[7]);
-        ul.x = pack_bf16x2(l[0], l[1]); ul.y = pack_bf16x2(l[2], l[3]);
-        ul.z = pack_bf16x2(l[4], l[5]); ul.w = pack_bf16x2(l[6], l[7]);
+        split_chunk8(v + 8 * c, uh, ul);
         *reinterpret_cast<uint4*>(hi_block + sw128_off(r, c0 + c)) = uh;
         *reinterpret_cast<uint4*>(lo_block + sw128_off(r, c0 + c)) = ul;
     }
