@@ -50,6 +50,15 @@ def fwd_bytes(B, T, H, Dk, Dv, elt, s0, s_out=True, out_elt=4):
     return B * T * H * per_tok + state
 
 
+def attainable(flops, nbytes, tc_peak_tflops, hbm_peak_gbs, seconds):
+    """Floors of a call's algorithmic work on the measured peaks, and the measured time's
+    fraction of the slower one (the attainable roofline)."""
+    t_tc = flops / (tc_peak_tflops * 1e12)
+    t_hbm = nbytes / (hbm_peak_gbs * 1e9)
+    return {"t_tensor_us": t_tc * 1e6, "t_hbm_us": t_hbm * 1e6, "bound": "hbm" if t_hbm >= t_tc else "tensor",
+            "frac": max(t_tc, t_hbm) / seconds}
+
+
 def decode_bytes(B, H, Dk, Dv, elt, out_elt=4):
     return B * H * (2 * Dk * Dv * 4 + (2 * Dk + Dv) * elt + Dv * out_elt + 8)
 
@@ -338,7 +347,10 @@ def gpu_arm(args, rank, world, local_rank):
                      "alg_bytes_bf16_o": alg_bytes_bf16_o,
                      "frac_bf16_o": alg_bytes_bf16_o / mean_s / 1e9 / hbm_peak,
                      "tensor": {"achieved": achieved_tf, "peak": tc_peak, "unit": "TFLOP/s",
-                                "frac": achieved_tf / tc_peak, "alg_flops_per_launch": alg_flops}},
+                                "frac": achieved_tf / tc_peak, "alg_flops_per_launch": alg_flops},
+                     # the attainable roofline: the slower of the tensor-core and HBM floors of
+                     # the call's algorithmic work (fp32 o as written), over the measured time
+                     "attainable": attainable(alg_flops, alg_bytes, tc_peak, hbm_peak, mean_s)},
         "e2e": e2e,
         "gpu_launches": launches * args.steps,
         "clocks": clocks,
@@ -496,7 +508,8 @@ def bench_train(kla, WORKLOADS, make_inputs, dev, stream, flush, rank, world, hb
             "roofline": {"bound": "tensor", "achieved": flops / mean_s / 1e12, "peak": tc_peak,
                          "unit": "TFLOP/s", "frac": flops / mean_s / 1e12 / tc_peak,
                          "hbm_frac": alg / mean_s / 1e9 / hbm_peak, "alg_flops_per_step": flops,
-                         "alg_bytes_per_step": alg}}
+                         "alg_bytes_per_step": alg,
+                         "attainable": attainable(flops, alg, tc_peak, hbm_peak, mean_s)}}
 
 
 def bench_long(kla, WORKLOADS, make_inputs, dev, stream, rank, world, hbm_peak, tc_peak, args):
@@ -566,7 +579,8 @@ def bench_long(kla, WORKLOADS, make_inputs, dev, stream, rank, world, hbm_peak, 
             "gpu_launches_per_step": 4, "stages": stages, "train": train,
             "roofline": {"bound": "hbm", "achieved": alg / mean_s / 1e9, "peak": hbm_peak, "unit": "GB/s",
                          "frac": alg / mean_s / 1e9 / hbm_peak,
-                         "tensor_frac": flops / mean_s / 1e12 / tc_peak}}
+                         "tensor_frac": flops / mean_s / 1e12 / tc_peak,
+                         "attainable": attainable(flops, alg, tc_peak, hbm_peak, mean_s)}}
 
 
 def bench_direct(kla, w, d, ws, o, ST, flush, stream, world, hbm_peak, args):
