@@ -488,7 +488,10 @@ def bench_train(kla, WORKLOADS, make_inputs, dev, stream, flush, rank, world, hb
         kla.chunk_bwd_after_train(d["q"], d["k"], d["v"], d["eta"], d["g"], dO, ws, w.eps)
 
     nsteps = 2 if args.quick else 5
-    launches = kla.fwd_kernel_launches(d["k"], d["v"]) + 2  # + reverse state pass, gradient kernel
+    # + the reverse state pass and the gradient kernel, each twice when the reverse pass runs as
+    # two slabs (the gradient kernel of the newest chunks beside the reverse pass over the rest)
+    slab = kla.lib().kla_chunk_bwd_reverse_slab_chunks(w.B, w.T, w.H, w.Dk, w.Dv, 64, 1)
+    launches = kla.fwd_kernel_launches(d["k"], d["v"]) + (4 if slab > 0 else 2)
     step()
     torch.cuda.synchronize()
     barrier(world)
@@ -503,8 +506,9 @@ def bench_train(kla, WORKLOADS, make_inputs, dev, stream, flush, rank, world, hb
     return {"workload": w.name, "value": tokens / (total_ms / 1e3), "unit": "tokens/s",
             "steps": nsteps, "ms_per_step": total_ms / nsteps,
             # forward: preparation + state pass (each twice with two slabs); backward: reverse
-            # state pass + gradient kernel
+            # state pass + gradient kernel (each twice with two slabs)
             "gpu_launches_per_step": launches,
+            "reverse_slab_newest_chunks": slab,
             "roofline": {"bound": "tensor", "achieved": flops / mean_s / 1e12, "peak": tc_peak,
                          "unit": "TFLOP/s", "frac": flops / mean_s / 1e12 / tc_peak,
                          "hbm_frac": alg / mean_s / 1e9 / hbm_peak, "alg_flops_per_step": flops,

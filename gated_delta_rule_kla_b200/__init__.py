@@ -70,6 +70,8 @@ def lib():
         L.kla_chunk_fwd_state_stage.restype = i
         L.kla_chunk_fwd_state_segments.argtypes = [i, i, i, i, i, i, i]
         L.kla_chunk_fwd_state_segments.restype = i
+        L.kla_chunk_bwd_reverse_slab_chunks.argtypes = [i, i, i, i, i, i, i]
+        L.kla_chunk_bwd_reverse_slab_chunks.restype = i
         L.kla_chunk_bwd_workspace.argtypes = [i, i, i, i, i, i, i, i]
         L.kla_chunk_bwd_workspace.restype = sz
         L.kla_chunk_bwd_workspace_min.argtypes = [i, i, i, i, i, i, i, i]

@@ -300,6 +300,14 @@ int kla_chunk_bwd_reverse_segments(int B, int T, int H, int Dk, int Dv, int chun
     return (NC + segc - 1) / segc;
 }
 
+int kla_chunk_bwd_reverse_slab_chunks(int B, int T, int H, int Dk, int Dv, int chunk, int dtype) {
+    take_beta_flag(dtype);
+    if (B < 1 || H < 1 || T < 1 || chunk != kla::kChunkLen || !tc_bwd_shape(T, Dk, Dv, dtype)) return 0;
+    const int NC = (T + kla::kChunkLen - 1) / kla::kChunkLen;
+    if (kla::reverse_nseg(B * H, NC) > 1) return 0;
+    return kla::bwd_slab_newest(B * H, NC);
+}
+
 size_t kla_chunk_bwd_workspace(int B, int T, int H, int Dk, int Dv, int chunk, int dtype,
                                int have_S_chunks) {
     take_beta_flag(dtype);

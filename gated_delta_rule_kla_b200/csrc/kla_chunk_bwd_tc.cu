@@ -124,6 +124,10 @@ struct BwdDev {
     int mode, nseg, segc;
     float* MN;
     const float* Lstart;
+    // mode 0 runs chunks [run_lo, run_hi) of every head (from dS_T, the gradient of the state
+    // after chunk run_hi - 1, to dS0, that of the state entering chunk run_lo); the gradient
+    // kernel takes chunks cfirst + blockIdx.x
+    int run_lo, run_hi, cfirst;
 };
 
 // =====================================================================================
@@ -177,7 +181,7 @@ __global__ void __launch_bounds__(RT, 1)
     const int NC = (T + CH - 1) / CH;
     const int nseg = a.mode == 0 ? 1 : a.nseg;
     const int head = blockIdx.x / nseg, seg = blockIdx.x % nseg, b = head / H, h = head % H;
-    const int c_lo = a.mode == 0 ? 0 : seg * a.segc, c_hi = a.mode == 0 ? NC : min(NC, c_lo + a.segc);
+    const int c_lo = a.mode == 0 ? a.run_lo : seg * a.segc, c_hi = a.mode == 0 ? a.run_hi : min(NC, c_lo + a.segc);
     const int nch = c_hi > c_lo ? c_hi - c_lo : 0;  // chunks of this run, processed newest first
     const bool ident = a.mode == 1 && blockIdx.y == 1;  // transition from lambda = I, no dO
     const bool need_do = !ident;
@@ -557,7 +561,7 @@ __global__ void __launch_bounds__(GT, 1)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int H = a.H, T = a.T;
     const int NC = (T + CH - 1) / CH;
-    const int c = blockIdx.x, head = blockIdx.y;
+    const int c = a.cfirst + blockIdx.x, head = blockIdx.y;
     const int b = head / H, h = head % H;
     const int t0 = c * CH, n = min(CH, T - t0);
     const size_t crow = (size_t)head * NC + c;  // chunk index in the workspace arrays
@@ -1046,7 +1050,7 @@ done:
 size_t align1k(size_t x) { return (x + 1023) & ~size_t(1023); }
 
 struct BwdLayout {
-    size_t fwd, T, S, U, L, dR, seg, total;
+    size_t fwd, T, S, U, L, dR, seg, mid, total;
     int nseg, segc;
 };
 
@@ -1084,17 +1088,22 @@ BwdLayout bwd_layout(int B, int T, int H) {
         L.nseg = (NC + L.segc - 1) / L.segc;
         o += align1k((size_t)3 * B * H * L.nseg * DK * DV * sizeof(float));
     }
+    L.mid = o;  // [B*H, DK, DV] fp32: lambda between the two slabs of the reverse pass
+    o += align1k((size_t)B * H * DK * DV * sizeof(float));
     L.total = o;
     return L;
 }
 
+// The gradient kernel over chunks [cfirst, cfirst + count) of every head.
 template <typename TOut>
-cudaError_t launch_grad(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mdo, const BwdDev& d,
-                        int NC, int BH, cudaStream_t st) {
+cudaError_t launch_grad(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mdo, BwdDev d,
+                        int cfirst, int count, int BH, cudaStream_t st) {
+    if (count <= 0) return cudaSuccess;
     cudaError_t e = cudaFuncSetAttribute(chunk_bwd_grad_kernel<TOut>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)G_SMEM);
     if (e != cudaSuccess) return e;
-    chunk_bwd_grad_kernel<TOut><<<dim3(NC, BH), GT, G_SMEM, st>>>(mq, mk, mdo, d);
+    d.cfirst = cfirst;
+    chunk_bwd_grad_kernel<TOut><<<dim3(count, BH), GT, G_SMEM, st>>>(mq, mk, mdo, d);
     return cudaGetLastError();
 }
 
@@ -1152,10 +1161,61 @@ cudaError_t launch_chunk_bwd_tc_reverse(const BwdTcArgs& a, void* ws, size_t ws_
     cudaError_t e =
         cudaFuncSetAttribute(chunk_bwd_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)R_SMEM);
     if (e != cudaSuccess) return e;
+    auto grad = [&](const BwdDev& dd, int cfirst, int count, cudaStream_t s) {
+        return a.out_bf16 ? launch_grad<__nv_bfloat16>(mq, mk, mdo, dd, cfirst, count, BH, s)
+                          : launch_grad<float>(mq, mk, mdo, dd, cfirst, count, BH, s);
+    };
     if (L.nseg <= 1) {
         d.mode = 0;
-        chunk_bwd_state_kernel<<<BH, RT, R_SMEM, st>>>(mq, mdo, d);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        const int n1 = bwd_slab_newest(BH, NC);
+        if (n1 <= 0) {
+            d.run_lo = 0;
+            d.run_hi = NC;
+            chunk_bwd_state_kernel<<<BH, RT, R_SMEM, st>>>(mq, mdo, d);
+            if ((e = cudaGetLastError()) != cudaSuccess) return e;
+            return grad(d, 0, NC, st);
+        }
+        // Two slabs: the reverse pass over the newest n1 chunks, then over the rest from the
+        // lambda it leaves, on `st` (it takes its SMs, one per head, before the gradient kernel
+        // queued beside it); the gradient kernel of the newest chunks runs on the side stream
+        // over the other SMs meanwhile, that of the older chunks on `st` once the reverse pass
+        // is done, and `st` takes the side stream's work back.  No kernel waits on another.
+        const int csplit = NC - n1;
+        float* Lmid = reinterpret_cast<float*>(w + L.mid);
+        cudaStream_t side = nullptr;
+        cudaEvent_t ev_rev = nullptr, ev_grad = nullptr;
+        e = split_side_stream(&side);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ev_rev, cudaEventDisableTiming);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ev_grad, cudaEventDisableTiming);
+        if (e == cudaSuccess) {
+            BwdDev d1 = d;
+            d1.run_lo = csplit;
+            d1.run_hi = NC;
+            d1.dS0 = Lmid;
+            chunk_bwd_state_kernel<<<BH, RT, R_SMEM, st>>>(mq, mdo, d1);
+            e = cudaGetLastError();
+        }
+        if (e == cudaSuccess) e = cudaEventRecord(ev_rev, st);
+        if (e == cudaSuccess) {
+            BwdDev d2 = d;
+            d2.run_lo = 0;
+            d2.run_hi = csplit;
+            d2.dS_T = Lmid;
+            chunk_bwd_state_kernel<<<BH, RT, R_SMEM, st>>>(mq, mdo, d2);
+            e = cudaGetLastError();
+        }
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(side, ev_rev, 0);
+        if (e == cudaSuccess) {
+            e = grad(d, csplit, n1, side);
+            // the caller's stream takes the side stream's work back whatever happens next
+            const cudaError_t er = cudaEventRecord(ev_grad, side);
+            if (e == cudaSuccess) e = grad(d, 0, csplit, st);
+            const cudaError_t ej = er == cudaSuccess ? cudaStreamWaitEvent(st, ev_grad, 0) : er;
+            if (e == cudaSuccess) e = ej;
+        }
+        if (ev_rev) cudaEventDestroy(ev_rev);  // released once the work that uses them is done
+        if (ev_grad) cudaEventDestroy(ev_grad);
+        return e;
     } else {
         // transition pass (each segment's map from lambda = I and its offset from lambda = 0),
         // the scan newest segment first (dS_T in, every segment's lambda_end and dS0 out), then
@@ -1175,8 +1235,7 @@ cudaError_t launch_chunk_bwd_tc_reverse(const BwdTcArgs& a, void* ws, size_t ws_
         chunk_bwd_state_kernel<<<dim3(BH * L.nseg, 1), RT, R_SMEM, st>>>(mq, mdo, d);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
-    return a.out_bf16 ? launch_grad<__nv_bfloat16>(mq, mk, mdo, d, NC, BH, st)
-                      : launch_grad<float>(mq, mk, mdo, d, NC, BH, st);
+    return grad(d, 0, NC, st);
 }
 
 cudaError_t launch_chunk_bwd_tc(const BwdTcArgs& a, void* ws, size_t ws_bytes, cudaStream_t st) {

@@ -1570,6 +1570,34 @@ int chunk_fwd_split_segments(const FwdArgs& a) { return split_layout(a).nseg; }
 
 int reverse_nseg(int BH, int NC) { return choose_nseg_split(BH, NC); }
 
+cudaError_t split_side_stream(cudaStream_t* out) { return slab_stream(out); }
+
+// Two slabs for the backward's reverse pass (one run per head): the reverse pass over the newest
+// n1 chunks first, then over the rest while the gradient kernel (one CTA per SM) takes the
+// newest chunks on the SMs the reverse pass leaves free; the older chunks' gradient kernel runs
+// on every SM at the end.  Cost model in microseconds, calibrated on the B=4 T=4096 H=16
+// training backward (reverse pass 228 us over 64 chunks: about 14 us per launch + 3.3 us per
+// chunk; gradient kernel 521 us over 4096 items: 18.8 us per wave of one CTA per SM).  Returns
+// n1, or 0 for one run.
+int bwd_slab_newest(int BH, int NC) {
+    const int sms = sm_count();
+    if (NC < 8 || 2 * BH > sms) return 0;
+    const double F = 14.0, r = 3.3, g = 18.8;
+    auto waves = [](long long items, long long slots) { return (double)((items + slots - 1) / slots); };
+    const double base = F + r * NC + waves((long long)NC * BH, sms) * g;
+    double best = base;
+    int n1 = 0;
+    for (int k = 2; k <= NC - 2; ++k) {
+        const double t = F + r * k + std::max(F + r * (NC - k), waves((long long)k * BH, sms - BH) * g) +
+                         waves((long long)(NC - k) * BH, sms) * g;
+        if (t < best) {
+            best = t;
+            n1 = k;
+        }
+    }
+    return best < 0.95 * base ? n1 : 0;
+}
+
 cudaError_t split_take_error(cudaStream_t st, unsigned int* flag) {
     cudaError_t e = cudaStreamSynchronize(st);
     if (e != cudaSuccess) return e;

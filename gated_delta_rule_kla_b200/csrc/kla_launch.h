@@ -167,6 +167,10 @@ cudaError_t launch_chunk_fwd_split_state(const FwdArgs& a, void* ws, cudaStream_
 // Parallel segments of the split path's state pass per head (1: one run per head).
 int chunk_fwd_split_segments(const FwdArgs& a);
 cudaError_t split_take_error(cudaStream_t st, unsigned int* flag);
+// The side stream of the split path's two-slab schedules (one per device, created once).
+cudaError_t split_side_stream(cudaStream_t* out);
+// Newest chunks in the first of the backward reverse pass's two slabs (0: one run per head).
+int bwd_slab_newest(int BH, int NC);
 // Segments of the backward's reverse state pass for BH heads of NC chunks (1: one run per head);
 // the forward state pass's cost model, which the reverse pass shares.
 int reverse_nseg(int BH, int NC);

@@ -194,6 +194,12 @@ size_t kla_chunk_bwd_workspace(int B, int T, int H, int Dk, int Dv, int chunk, i
  * true end gradient, as for the forward's segmented state pass); 0 for shapes without the
  * tensor-core backward. */
 int kla_chunk_bwd_reverse_segments(int B, int T, int H, int Dk, int Dv, int chunk, int dtype);
+/* With one reverse run per head (above == 1): how many of the newest chunks the reverse pass
+ * takes first as a slab of its own, 0 for one run.  With a slab the gradient kernel of those
+ * chunks runs on an internal stream of the device, on the SMs the reverse pass leaves free,
+ * while the reverse pass goes on over the older chunks from the gradient it left (the call stays
+ * ordered on `stream`).  0 also for shapes without the tensor-core backward. */
+int kla_chunk_bwd_reverse_slab_chunks(int B, int T, int H, int Dk, int Dv, int chunk, int dtype);
 size_t kla_chunk_bwd_workspace_min(int B, int T, int H, int Dk, int Dv, int chunk, int dtype,
                                    int have_S_chunks);
 kla_status kla_chunk_bwd(const void *q, const void *k, const void *v, const float *eta,

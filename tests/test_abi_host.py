@@ -207,6 +207,13 @@ def test_backward_reverse_segments(L):
     assert L.kla_chunk_bwd_reverse_segments(1, 4100, 2, 128, 128, 64, 1) > 1
     assert L.kla_chunk_bwd_reverse_segments(1, 4100, 2, 64, 64, 64, 1) == 0  # no tensor-core backward
     assert L.kla_chunk_bwd_reverse_segments(1, 4100, 2, 128, 128, 64, 0) == 0
+    # one reverse run per head: the newest chunks as a slab of their own when the gradient
+    # kernel has enough work to fill the other SMs meanwhile (148 SMs assumed without a device)
+    assert 0 < L.kla_chunk_bwd_reverse_slab_chunks(4, 4096, 16, 128, 128, 64, 1) < 64
+    assert 0 < L.kla_chunk_bwd_reverse_slab_chunks(4, 2048, 16, 128, 128, 64, 1) < 32
+    assert L.kla_chunk_bwd_reverse_slab_chunks(2, 150, 3, 128, 128, 64, 1) == 0
+    assert L.kla_chunk_bwd_reverse_slab_chunks(1, 65536, 16, 128, 128, 64, 1) == 0  # segmented instead
+    assert L.kla_chunk_bwd_reverse_slab_chunks(4, 4096, 16, 64, 64, 64, 1) == 0
 
 
 def test_diag_forward_workspace_by_path(L):

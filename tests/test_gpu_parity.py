@@ -582,6 +582,30 @@ def test_bwd_training_workload_sampled_heads(kla, oracle_mod):
         assert rel_err(got, ref[name]) <= 2e-2, name
 
 
+def test_bwd_two_slab_reverse_pass_sampled_heads(kla, oracle_mod):
+    """B=4 T=2048 H=16 (32 chunks per head): the reverse pass runs the newest chunks as a slab of
+    its own while the gradient kernel takes them on the other SMs, then goes on over the older
+    chunks from the state gradient it left.  Long memory (g >= -0.05), an initial state and a
+    dS_T, so that the gradient crosses the slab boundary; sampled heads against the oracle."""
+    B, T, H = 4, 2048, 16
+    assert kla.lib().kla_chunk_bwd_reverse_slab_chunks(B, T, H, 128, 128, 64, 1) > 0
+    inp = small_inputs(B, T, H, 128, 128, "bf16", seed=91, g_lo=-0.05)
+    d = {k: (v.cuda() if v is not None else None) for k, v in inp.items()}
+    gen = torch.Generator().manual_seed(92)
+    dO = torch.randn(B, T, H, 128, generator=gen).to(torch.bfloat16)
+    dST = torch.randn(B, H, 128, 128, generator=gen) * 0.1
+    gr = kla.chunk_bwd(d["q"], d["k"], d["v"], d["eta"], d["g"], dO.cuda(), 1e-6, d["S0"], dST.cuda())
+    torch.cuda.synchronize()
+    kla.check_device_error()
+    pairs = [(0, 1), (3, 14)]
+    args = [heads_slice(np64(inp[k]), pairs) for k in ("q", "k", "v", "eta", "g")]
+    ref = oracle_mod.backward(*args, 1e-6, heads_slice(np64(inp["S0"]), pairs, state=True),
+                              heads_slice(np64(dO), pairs), heads_slice(np64(dST), pairs, state=True))
+    for name in GRADS:
+        got = heads_slice(np64(gr[name]), pairs, state=(name == "dS0"))
+        assert rel_err(got, ref[name]) <= 2e-2, name
+
+
 def test_bwd_long_context_sampled_heads(kla, oracle_mod):
     """The tensor-core backward at the long-context shape (B=1, T=65536, H=16: 1024 chunks per
     head through the reverse pass, the segmented forward recomputed inside), sampled heads
