@@ -179,7 +179,7 @@ kla_status kla_chunk_fwd_state_stage(int stage, const void *q, const void *v, co
  * not be initialised) of at least kla_chunk_bwd_workspace_min() bytes (required; smaller is
  * KLA_ERR_WORKSPACE).  With at least kla_chunk_bwd_workspace() bytes, bf16 inputs with
  * Dk == Dv == 128 run on the tensor cores: the split forward's preparation and state pass are
- * recomputed into ws (about 305 KiB per chunk and head; S_chunks is then not read), a reverse
+ * recomputed into ws (about 290 KiB per chunk and head; S_chunks is then not read), a reverse
  * state pass carries the state gradient chunk by chunk (in parallel segments chained by a scan
  * for long sequences over few heads: kla_chunk_bwd_reverse_segments), and a chunk-parallel
  * kernel forms every gradient.  With less, and for every other shape, the CUDA-core backward runs.
